@@ -1,0 +1,385 @@
+#!/usr/bin/env python3
+"""Benchmark of the Kronecker delta rule mixer on B200.
+
+One step = one pass of the whole hot path over one batch: the chunked
+forward (saving what the backward needs) followed by the backward, on the
+forward+backward workload B=1, H=16, T=16384, d_k=d_v=128, bf16 q/k/v/dO,
+fp32 gates and state, beta in (0,2), nonzero S0.  The decode step
+(B=256, H=16, d=128, 1000 consecutive in-place steps) is timed in the same run
+and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched by torchrun): each rank runs its own batch of the same
+shape (independent (b,h) units, no collective on the data path; weak
+scaling); time is the max over ranks.  Inputs (~0.5 GB per step) are larger
+than L2 (126 MB), so no L2 flush is needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WL = dict(B=1, H=16, T=16384, dk=128, dv=128)
+CHUNK = 64
+METRIC = "Kron-delta fwd+bwd tokens/s (H16,d128,T16K) & % bf16 TC peak; decode GB/s"
+WORKLOAD_NAME = "fwdbwd-B1-H16-T16384-d128-beta2"
+CPU_SAMPLE_T = 4096     # tokens of the workload the oracle baseline runs (all 16 heads)
+REF_STEP_T = 512        # tokens per step of the reference (oracle) arm
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0,
+                source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per kernel, per token-head (d_k = d_v = d, C = 64, bf16 I/O)
+#   flops count dense contractions only (2 per multiply-add); bytes count
+#   what a kernel must move across HBM with its inputs and outputs.
+# ---------------------------------------------------------------------------
+def kernel_work(name, d=128, C=CHUNK):
+    io_in = 3 * d * 2 + d * 4 + 8          # q,k,v bf16 + logf fp32 + beta,c
+    works = {
+        # Grams K K^T, V V^T, Q K^T (3 C x C x d); writes y, A, P (fp32)
+        "fwd_prep_simt": dict(flops=6 * C * d, bytes=io_in + 4 + 2 * C * 4),
+        # S K+^T, S Q+^T, V^T diag(u) K^e (3 d x d x C) + P diag(u) V (C x C x d)
+        "fwd_chain_simt": dict(flops=6 * d * d + 2 * C * d,
+                               bytes=io_in + 4 + 2 * C * 4 + d * 2 + d * d * 4 // C + 8),
+        # dS K^e^T, dO^T Q+, V^T diag(db0) K+ (3 d x d x C) + P^T dO (C x C x d)
+        "bwd_chain_simt": dict(flops=6 * d * d + 2 * C * d,
+                               bytes=io_in + d * 2 + 2 * C * 4 + d * d * 4 // C + 4),
+        # K K^T, V V^T, dO V^T (3 C x C x d)
+        "bwd_cc_simt": dict(flops=6 * C * d, bytes=2 * d * 2 + d * 4 + d * 2 + 16 + 3 * C * 4),
+        # dO S0, V S0, V dS, K+ S0^T, K^e dS^T (5 d x d x C)
+        "bwd_state_simt": dict(flops=10 * d * d, bytes=4 * d * 2 + d * 4 + 2 * d * d * 4 // C + 4 * d * 4),
+        # dP K-, dP^T Q+, dG_K K-, dG_K^T K+, P^T dO, dG_V V (6 C x C x d)
+        "bwd_intra_simt": dict(flops=12 * C * d, bytes=4 * d * 2 + d * 4 + 3 * C * 4 + 4 * d * 4 + 3 * d * 2 + d * 4),
+    }
+    return works.get(name)
+
+
+def fp32_alu_peak_tflops(sm_mhz):
+    # 148 SMs x 128 FP32 lanes x 2 flops per FFMA
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
+                    reasons=reasons, samples=len(rows))
+
+
+# ---------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def oracle_baseline(T_sample, seed=1004):
+    """The fp64 oracle, as it stands, on the first T_sample tokens of the
+    workload (all heads), fwd + bwd, all host cores."""
+    from delta_rule_linear_kron_b200 import inputs as kin
+    from oracle import oracle
+    inp = kin.make_inputs(4, T=T_sample, seed=seed)
+    cores = len(os.sched_getaffinity(0))
+    t = time.perf_counter()
+    oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], nthreads=cores)
+    oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], inp["dO"],
+               nthreads=cores)
+    el = time.perf_counter() - t
+    return dict(value=WL["B"] * T_sample / el, unit="tokens/s", cores=min(cores, WL["H"]), kind="oracle",
+                sample=f"first {T_sample} tokens x {WL['H']} heads of the workload, fwd+bwd, fp64, "
+                       f"threaded over heads ({min(cores, WL['H'])} threads used of {cores} cores)",
+                seconds=el)
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from delta_rule_linear_kron_b200 import inputs as kin
+    from oracle import oracle
+    cores = len(os.sched_getaffinity(0))
+    inp = kin.make_inputs(4, T=REF_STEP_T, seed=1004)
+
+    def step():
+        oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], nthreads=cores)
+        oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], inp["dO"],
+                   nthreads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t
+    value = WL["B"] * REF_STEP_T * args.steps / el
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD_NAME, "B": WL["B"], "H": WL["H"], "T": REF_STEP_T, "dk": WL["dk"],
+                       "dv": WL["dv"], "note": "each step: the first 512 tokens of the workload, all heads"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(cores, WL["H"]), "kind": "oracle",
+                             "sample": f"{REF_STEP_T} tokens x {WL['H']} heads per step, fwd+bwd, fp64"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import delta_rule_linear_kron_b200 as kd
+    from delta_rule_linear_kron_b200 import inputs as kin
+
+    ws_n, rank, local = dist_env()
+    if ws_n > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    B, H, T, dk, dv = WL["B"], WL["H"], WL["T"], WL["dk"], WL["dv"]
+
+    def barrier():
+        if ws_n > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if ws_n == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- inputs (each rank its own batch) -------------------------------
+    inp = kin.make_inputs(4, seed=1004 + rank)
+    bf, f32 = torch.bfloat16, torch.float32
+    host = {n: torch.from_numpy(inp[n]).to(bf if n in ("q", "k", "v", "dO") else f32)
+            for n in ("q", "k", "v", "dO", "beta", "c", "logf", "S0")}
+    d = {n: t.to(dev) for n, t in host.items()}
+    del inp
+    fws = torch.empty(kd.workspace_size(kd.KD_WS_FWD_SAVE, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+    bws = torch.empty(kd.workspace_size(kd.KD_WS_BWD, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, T, H, dv), dtype=bf, device=dev)
+
+    def step(src):
+        o, ST, _ = kd.fwd(src["q"], src["k"], src["v"], src["beta"], src["c"], src["logf"], src["S0"], out=out,
+                          save=True, workspace=fws)
+        g = kd.bwd(src["q"], src["k"], src["v"], src["beta"], src["c"], src["logf"], src["S0"], src["dO"],
+                   fwd_workspace=fws, workspace=bws)
+        return o, ST, g
+
+    for _ in range(args.warmup):
+        step(d)
+    torch.cuda.synchronize()
+    kd.device_status()
+    barrier()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    kd.lib().kron_delta_profile_enable(1)
+    kd.lib().kron_delta_profile_report(None, 0, 1)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(d)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    import ctypes
+    buf = ctypes.create_string_buffer(1 << 16)
+    kd.lib().kron_delta_profile_report(buf, len(buf), 1)
+    kd.lib().kron_delta_profile_enable(0)
+    per_kernel = {}
+    for line in buf.value.decode().splitlines():
+        name, n, ms = line.split()
+        per_kernel[name] = dict(launches=int(n), ms=float(ms))
+    launches = sum(v["launches"] for v in per_kernel.values())
+
+    # ---- decode: 1000 consecutive in-place steps --------------------------
+    decode = None
+    if not args.no_decode:
+        Bd, Hd = 256, 16
+        dd = kin.decode_token_inputs_torch(args.decode_steps, B=Bd, H=Hd, seed=1005 + rank, device=dev)
+        S = dd["S"]
+        o_dec = torch.empty((Bd, Hd, dv), dtype=bf, device=dev)
+        for t in range(3):
+            kd.decode(dd["q"][t], dd["k"][t], dd["v"][t], dd["beta"][t], dd["c"][t], dd["logf"][t], S, out=o_dec)
+        torch.cuda.synchronize()
+        barrier()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for t in range(args.decode_steps):
+            kd.decode(dd["q"][t], dd["k"][t], dd["v"][t], dd["beta"][t], dd["c"][t], dd["logf"][t], S, out=o_dec)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(d0.elapsed_time(d1))
+        per_head = 2 * dv * dk * 4 + 2 * dk * 2 + dv * 2 + dk * 4 + 8 + dv * 2
+        bytes_total = ws_n * args.decode_steps * Bd * Hd * per_head
+        decode = dict(value=bytes_total / (dms / 1e3) / 1e9, unit="GB/s", steps=args.decode_steps,
+                      us_per_step=1e3 * dms / args.decode_steps, B=Bd, H=Hd, d=dk,
+                      bytes_per_head=per_head,
+                      hbm_frac=(bytes_total / ws_n / (dms / 1e3) / 1e9) / peaks["hbm_gbs"])
+        del dd, S
+    clocks = sampler.stop()
+
+    # ---- end to end through the public API with pinned host buffers -----
+    e2e = None
+    if not args.no_e2e:
+        pinned = {n: t.pin_memory() for n, t in host.items()}
+        staged = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+        out_h = torch.empty((B, T, H, dv), dtype=bf).pin_memory()
+        dS0_h = torch.empty((B, H, dv, dk), dtype=f32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        d2h = out_h.numel() * out_h.element_size() + dS0_h.numel() * dS0_h.element_size()
+        barrier()
+        torch.cuda.synchronize()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(args.e2e_steps):
+            for n in staged:
+                staged[n].copy_(pinned[n], non_blocking=True)
+            o, ST, g = step(staged)
+            out_h.copy_(o, non_blocking=True)
+            dS0_h.copy_(g["dS0"], non_blocking=True)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        xms = max_over_ranks(x0.elapsed_time(x1))
+        e2e = dict(value=ws_n * B * T * args.e2e_steps / (xms / 1e3), unit="tokens/s",
+                   h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
+
+    value = ws_n * B * T * args.steps / (ms_total / 1e3)
+
+    # ---- roofline of the dominant kernel ---------------------------------
+    roofline = None
+    if per_kernel:
+        top = max(per_kernel, key=lambda n: per_kernel[n]["ms"])
+        w = kernel_work(top)
+        avg_s = per_kernel[top]["ms"] / per_kernel[top]["launches"] / 1e3
+        units = B * H * T  # token-heads per launch
+        sm_mhz = clocks["sm_mhz"] or peaks["sm_max_mhz"]
+        if w is not None:
+            achieved = w["flops"] * units / avg_s / 1e12
+            peak = fp32_alu_peak_tflops(peaks["sm_max_mhz"])
+            roofline = dict(kernel=top, bound="alu", achieved=achieved, peak=peak, unit="TFLOP/s",
+                            frac=achieved / peak, traffic=None,
+                            algorithmic_flops_per_launch=w["flops"] * units,
+                            algorithmic_bytes_per_launch=w["bytes"] * units,
+                            hbm_achieved_gbs=w["bytes"] * units / avg_s / 1e9,
+                            peak_note="fp32 FFMA: 148 SMs x 128 lanes x 2 flops x max SM clock",
+                            avg_launch_ms=avg_s * 1e3, sm_mhz_median=sm_mhz)
+    step_flops = 524288 * B * H * T
+    tc_frac = step_flops / (ms_total / args.steps / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
+
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(CPU_SAMPLE_T)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "T": T, "dk": dk, "dv": dv, "chunk": CHUNK,
+                           "global_batch": B * ws_n, "seq_len": T, "parallelism": f"dp{ws_n}",
+                           "step": "fwd(save) + bwd", "l2": "inputs larger than L2 (no flush)"},
+                "tc_frac_of_bf16_peak": tc_frac,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+                "gpu_launches": launches, "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
+                "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                           "reasons": clocks["reasons"], "samples": clocks["samples"]},
+                "peaks": peaks}
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,228 @@
-"""Kronecker delta rule (KronLSTM token mixer) for NVIDIA B200 (sm_100a)."""
+"""Kronecker delta rule (KronLSTM token mixer) for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libkron_delta.so`` (declared in
+``include/kron_delta.h``).  It only marshals arguments: torch provides device
+memory and the current stream; every step of the computation runs in the
+library's CUDA kernels.  There is no CPU or PyTorch fallback: if the library
+is missing, every call raises.
+
+Per head, with fp32 state S (dv x dk), for each token:
+    Sbar = S diag(exp(logf)); b = v^T Sbar k; u = c - beta b
+    S = Sbar + u v k^T;       o = S q
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["fwd", "bwd", "decode", "workspace_size", "device_status", "library_path",
+           "KronDeltaError", "KronDeltaFunction", "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libkron_delta.so")
+_lib = None
+
+KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE, KD_ERR_CUDA, KD_ERR_TIMEOUT = range(6)
+KD_F32, KD_BF16 = 0, 1
+KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD = 0, 1, 2
+_CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
+          4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
+
+
+class KronDeltaError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{_CODES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m delta_rule_linear_kron_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.kron_delta_version.restype = i
+        L.kron_delta_last_error.restype = ctypes.c_char_p
+        L.kron_delta_workspace_size.restype = sz
+        L.kron_delta_workspace_size.argtypes = [i] * 7
+        L.kron_delta_fwd.restype = i
+        L.kron_delta_fwd.argtypes = [vp] * 9 + [i] * 6 + [vp, sz, i, vp]
+        L.kron_delta_bwd.restype = i
+        L.kron_delta_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp, sz, vp]
+        L.kron_delta_decode.restype = i
+        L.kron_delta_decode.argtypes = [vp] * 8 + [i] * 5 + [vp]
+        L.kron_delta_device_status.restype = i
+        L.kron_delta_device_status.argtypes = [vp]
+        L.kron_delta_profile_enable.restype = None
+        L.kron_delta_profile_enable.argtypes = [i]
+        L.kron_delta_profile_report.restype = i
+        L.kron_delta_profile_report.argtypes = [ctypes.c_char_p, sz, i]
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != KD_OK:
+        raise KronDeltaError(rc, lib().kron_delta_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return KD_F32
+    if t.dtype == torch.bfloat16:
+        return KD_BF16
+    raise KronDeltaError(KD_ERR_UNSUPPORTED, f"q/k/v dtype {t.dtype} (want float32 or bfloat16)")
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise KronDeltaError(KD_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise KronDeltaError(KD_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise KronDeltaError(KD_ERR_INVALID_ARG, f"{name} must be {dtype} (got {t.dtype})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise KronDeltaError(KD_ERR_INVALID_ARG, f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+
+
+def workspace_size(kind, B, H, T, dk, dv, dtype=KD_BF16) -> int:
+    n = lib().kron_delta_workspace_size(kind, B, H, T, dk, dv, dtype)
+    if n == 0:
+        raise KronDeltaError(KD_ERR_INVALID_ARG, lib().kron_delta_last_error().decode())
+    return n
+
+
+def _alloc_ws(nbytes, device):
+    import torch
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def fwd(q, k, v, beta, c, logf, S0=None, *, out=None, want_state=True, save=False,
+        workspace=None, stream=None):
+    """Chunk-parallel forward.  q,k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32);
+    beta, c [B,T,H] fp32; logf [B,T,H,dk] fp32; S0 [B,H,dv,dk] fp32 or None.
+    Returns (out [B,T,H,dv], ST [B,H,dv,dk] or None, workspace)."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(beta, "beta", f32, (B, T, H)); _need(c, "c", f32, (B, T, H))
+    _need(logf, "logf", f32, (B, T, H, dk)); _need(S0, "S0", f32, (B, H, dv, dk))
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, (B, T, H, dv))
+    ST = torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_state else None
+    need = workspace_size(KD_WS_FWD_SAVE if save else KD_WS_FWD, B, H, T, dk, dv, dt)
+    if workspace is None:
+        workspace = _alloc_ws(need, q.device)
+    _check(lib().kron_delta_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S0),
+                                _ptr(out), _ptr(ST), B, H, T, dk, dv, dt, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), int(bool(save)),
+                                _stream(stream)))
+    return out, ST, workspace
+
+
+def bwd(q, k, v, beta, c, logf, S0, dO, dST=None, *, fwd_workspace, workspace=None,
+        want_dS0=True, stream=None):
+    """Backward for loss <dO, out> + <dST, ST>, reading what fwd(save=True)
+    left in fwd_workspace.  Returns dict dq, dk, dv, dbeta, dc, dlogf, dS0."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(beta, "beta", f32, (B, T, H)); _need(c, "c", f32, (B, T, H))
+    _need(logf, "logf", f32, (B, T, H, dk)); _need(S0, "S0", f32, (B, H, dv, dk))
+    _need(dO, "dO", q.dtype, (B, T, H, dv)); _need(dST, "dST", f32, (B, H, dv, dk))
+    dt = _dtype_code(q)
+    g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+             dbeta=torch.empty_like(beta), dc=torch.empty_like(c), dlogf=torch.empty_like(logf),
+             dS0=torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_dS0 else None)
+    need = workspace_size(KD_WS_BWD, B, H, T, dk, dv, dt)
+    if workspace is None:
+        workspace = _alloc_ws(need, q.device)
+    _check(lib().kron_delta_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S0),
+                                _ptr(dO), _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                _ptr(g["dbeta"]), _ptr(g["dc"]), _ptr(g["dlogf"]), _ptr(g["dS0"]),
+                                B, H, T, dk, dv, dt, _ptr(fwd_workspace),
+                                fwd_workspace.numel() * fwd_workspace.element_size(),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream)))
+    return g
+
+
+def decode(q, k, v, beta, c, logf, S, *, out=None, stream=None):
+    """One decode step.  q,k [B,H,dk], v [B,H,dv], beta,c [B,H], logf [B,H,dk],
+    S [B,H,dv,dk] fp32 (updated in place).  Returns out [B,H,dv]."""
+    import torch
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, H, dv))
+    _need(beta, "beta", f32, (B, H)); _need(c, "c", f32, (B, H)); _need(logf, "logf", f32, (B, H, dk))
+    _need(S, "S", f32, (B, H, dv, dk))
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, (B, H, dv))
+    _check(lib().kron_delta_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S),
+                                   _ptr(out), B, H, dk, dv, dt, _stream(stream)))
+    return out
+
+
+def device_status(stream=None):
+    """Synchronise the stream and raise if an earlier call failed on the device."""
+    _check(lib().kron_delta_device_status(_stream(stream)))
+
+
+def _make_function():
+    import torch
+
+    class KronDeltaFunction(torch.autograd.Function):
+        """autograd wrapper: forward saves what the backward kernels read."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, beta, c, logf, S0=None):
+            out, ST, ws = fwd(q, k, v, beta, c, logf, S0, save=True)
+            ctx.save_for_backward(q, k, v, beta, c, logf, S0, ws)
+            return out, ST
+
+        @staticmethod
+        def backward(ctx, dO, dST):
+            q, k, v, beta, c, logf, S0, ws = ctx.saved_tensors
+            g = bwd(q, k, v, beta, c, logf, S0, dO.contiguous(),
+                    None if dST is None else dST.contiguous(), fwd_workspace=ws,
+                    want_dS0=S0 is not None)
+            return g["dq"], g["dk"], g["dv"], g["dbeta"], g["dc"], g["dlogf"], g["dS0"]
+
+    return KronDeltaFunction
+
+
+def __getattr__(name):
+    if name == "KronDeltaFunction":
+        fn = _make_function()
+        globals()[name] = fn
+        return fn
+    raise AttributeError(name)

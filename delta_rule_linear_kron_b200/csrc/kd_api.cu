@@ -1,0 +1,314 @@
+// kd_api.cu -- C ABI and chunk scheduler of the Kronecker delta rule library.
+//
+// The scheduler validates a call, derives the chunk count NC = ceil(T/64)
+// (Gated DeltaNet-2 article, "기술 상세": C = 64), lays out the workspace and
+// enqueues the kernels of the call on the caller's stream, in order, without
+// synchronising.  Declarations and argument contracts: include/kron_delta.h.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/kron_delta.h"
+#include "kd_kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int ok() {
+  g_err.clear();
+  return KD_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool dim_supported(int d) { return d == 32 || d == 64 || d == 128; }
+
+// Validates sizes and fills the workspace layout.  Returns KD_OK or an error.
+int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
+  if (B <= 0 || H <= 0 || T <= 0) return fail(KD_ERR_INVALID_ARG, "B, H, T must be >= 1 (got %d, %d, %d)", B, H, T);
+  if (!dim_supported(dk) || !dim_supported(dv))
+    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  if (H > 65535 || B > 65535) return fail(KD_ERR_INVALID_ARG, "B and H must be <= 65535 (got %d, %d)", B, H);
+  const int NC = (T + kd::kChunk - 1) / kd::kChunk;
+  const size_t chunks = (size_t)B * H * NC;
+  if (chunks > (size_t(1) << 31)) return fail(KD_ERR_INVALID_ARG, "problem too large (%zu chunks)", chunks);
+  L->B = B; L->H = H; L->T = T; L->dk = dk; L->dv = dv; L->dtype = dtype;
+  L->NC = NC;
+  L->chunks = chunks;
+  const size_t C = kd::kChunk;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  L->y = take(chunks * C * 4);
+  L->A = take(chunks * C * C * 4);
+  L->P = take(chunks * C * C * 4);
+  L->fwd_bytes = off;
+  L->S0 = take(chunks * (size_t)dv * dk * 4);
+  L->u = take(chunks * C * 4);
+  L->b0 = take(chunks * C * 4);
+  L->fwd_save_bytes = off;
+  off = 0;
+  L->dSC = take(chunks * (size_t)dv * dk * 4);
+  L->g = take(chunks * C * 4);
+  L->dP = take(chunks * C * C * 4);
+  L->dGK = take(chunks * C * C * 4);
+  L->dGVs = take(chunks * C * C * 4);
+  L->accq = take(chunks * C * dk * 4);
+  L->acck = take(chunks * C * dk * 4);
+  L->accL = take(chunks * C * dk * 4);
+  L->accv = take(chunks * C * dv * 4);
+  L->bwd_bytes = off;
+  return KD_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_ptr(const void* p, const char* name, bool required) {
+  if (!p) return required ? fail(KD_ERR_INVALID_ARG, "%s must not be NULL", name) : KD_OK;
+  if (!aligned(p, 16)) return fail(KD_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  return KD_OK;
+}
+
+int check_stream(void* stream) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(KD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+#if CUDART_VERSION >= 12080
+  if (stream) {
+    int sdev = -1;
+    e = cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev);
+    if (e != cudaSuccess) return fail(KD_ERR_INVALID_ARG, "invalid stream: %s", cudaGetErrorString(e));
+    if (sdev != dev)
+      return fail(KD_ERR_INVALID_ARG, "stream belongs to device %d but the current device is %d", sdev, dev);
+  }
+#endif
+  return KD_OK;
+}
+
+int launched(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(KD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+// ---- per-kernel timing (kron_delta_profile_*) ----------------------------
+struct ProfState {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  struct Pending { std::string name; cudaEvent_t a, b; };
+  std::vector<Pending> pending;
+  std::string open_name;
+  cudaEvent_t open_a = nullptr;
+  std::map<std::string, std::pair<long, double>> totals;  // launches, ms
+  cudaEvent_t get() {
+    if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+ProfState& prof() {
+  static ProfState* p = new ProfState();  // never destroyed: usable during exit
+  return *p;
+}
+
+}  // namespace
+
+namespace kd {
+void prof_begin(cudaStream_t st, const char* name) {
+  ProfState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.on) return;
+  p.open_a = p.get();
+  p.open_name = name;
+  if (p.open_a) cudaEventRecord(p.open_a, st);
+}
+void prof_end(cudaStream_t st) {
+  ProfState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.on || !p.open_a) return;
+  cudaEvent_t b = p.get();
+  if (b) {
+    cudaEventRecord(b, st);
+    p.pending.push_back({p.open_name, p.open_a, b});
+  } else {
+    p.pool.push_back(p.open_a);
+  }
+  p.open_a = nullptr;
+}
+}  // namespace kd
+
+#define KD_TRY(x)          \
+  do {                     \
+    int rc_ = (x);         \
+    if (rc_ != KD_OK) return rc_; \
+  } while (0)
+
+extern "C" {
+
+int kron_delta_version(void) { return 100; }
+
+const char* kron_delta_last_error(void) { return g_err.c_str(); }
+
+size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv, int dtype) {
+  kd::Layout L;
+  if (plan(B, H, T, dk, dv, dtype, &L) != KD_OK) return 0;
+  switch (kind) {
+    case KD_WS_FWD: ok(); return L.fwd_bytes;
+    case KD_WS_FWD_SAVE: ok(); return L.fwd_save_bytes;
+    case KD_WS_BWD: ok(); return L.bwd_bytes;
+    default: fail(KD_ERR_INVALID_ARG, "unknown workspace kind %d", kind); return 0;
+  }
+}
+
+int kron_delta_fwd(const void* q, const void* k, const void* v, const float* beta,
+                   const float* c, const float* logf, const float* S0, void* out, float* ST,
+                   int B, int H, int T, int dk, int dv, int dtype, void* workspace,
+                   size_t ws_bytes, int save, void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk, dv, dtype, &L));
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(beta, "beta", true));
+  KD_TRY(check_ptr(c, "c", true));
+  KD_TRY(check_ptr(logf, "logf", true));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(out, "out", true));
+  KD_TRY(check_ptr(ST, "ST", false));
+  if (save != 0 && save != 1) return fail(KD_ERR_INVALID_ARG, "save must be 0 or 1");
+  const size_t need = save ? L.fwd_save_bytes : L.fwd_bytes;
+  if (!workspace || ws_bytes < need)
+    return fail(KD_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  kd::FwdArgs a{q, k, v, beta, c, logf, S0, out, ST, save, static_cast<char*>(workspace), L};
+  return launched(kd::launch_fwd_simt(a, static_cast<cudaStream_t>(stream)), "forward launch");
+}
+
+int kron_delta_bwd(const void* q, const void* k, const void* v, const float* beta,
+                   const float* c, const float* logf, const float* S0, const void* dO,
+                   const float* dST, void* dq, void* dk, void* dv, float* dbeta, float* dc,
+                   float* dlogf, float* dS0, int B, int H, int T, int dk_, int dv_, int dtype,
+                   const void* fwd_ws, size_t fwd_ws_bytes, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk_, dv_, dtype, &L));
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(beta, "beta", true));
+  KD_TRY(check_ptr(c, "c", true));
+  KD_TRY(check_ptr(logf, "logf", true));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(dO, "dO", true));
+  KD_TRY(check_ptr(dST, "dST", false));
+  KD_TRY(check_ptr(dq, "dq", true));
+  KD_TRY(check_ptr(dk, "dk", true));
+  KD_TRY(check_ptr(dv, "dv", true));
+  KD_TRY(check_ptr(dbeta, "dbeta", true));
+  KD_TRY(check_ptr(dc, "dc", true));
+  KD_TRY(check_ptr(dlogf, "dlogf", true));
+  KD_TRY(check_ptr(dS0, "dS0", false));
+  if (!fwd_ws || fwd_ws_bytes < L.fwd_save_bytes)
+    return fail(KD_ERR_WORKSPACE, "forward workspace saved with save=1 of %zu bytes needed (got %zu)",
+                L.fwd_save_bytes, fwd_ws ? fwd_ws_bytes : 0);
+  if (!workspace || ws_bytes < L.bwd_bytes)
+    return fail(KD_ERR_WORKSPACE, "backward workspace of %zu bytes needed (got %zu)", L.bwd_bytes,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256) || !aligned(fwd_ws, 256))
+    return fail(KD_ERR_WORKSPACE, "workspaces must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  (void)S0;  // the forward state at every chunk start is read from fwd_ws
+  kd::BwdArgs a{q, k, v, beta, c, logf, S0, dO, dST, dq, dk, dv, dbeta, dc, dlogf, dS0,
+                static_cast<const char*>(fwd_ws), static_cast<char*>(workspace), L};
+  return launched(kd::launch_bwd_simt(a, static_cast<cudaStream_t>(stream)), "backward launch");
+}
+
+int kron_delta_decode(const void* q, const void* k, const void* v, const float* beta,
+                      const float* c, const float* logf, float* S, void* out, int B, int H,
+                      int dk, int dv, int dtype, void* stream) {
+  if (B <= 0 || H <= 0) return fail(KD_ERR_INVALID_ARG, "B, H must be >= 1 (got %d, %d)", B, H);
+  if ((size_t)B * H > 0x7fffffffu) return fail(KD_ERR_INVALID_ARG, "B*H too large");
+  if (!dim_supported(dk) || !dim_supported(dv))
+    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(beta, "beta", true));
+  KD_TRY(check_ptr(c, "c", true));
+  KD_TRY(check_ptr(logf, "logf", true));
+  KD_TRY(check_ptr(S, "S", true));
+  KD_TRY(check_ptr(out, "out", true));
+  KD_TRY(check_stream(stream));
+  kd::DecodeArgs a{q, k, v, beta, c, logf, S, out, B, H, dk, dv, dtype};
+  return launched(kd::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+void kron_delta_profile_enable(int on) {
+  ProfState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  p.on = on != 0;
+}
+
+int kron_delta_profile_report(char* buf, size_t len, int reset) {
+  ProfState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    fail(KD_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+    return -KD_ERR_CUDA;
+  }
+  for (auto& r : p.pending) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      auto& t = p.totals[r.name];
+      t.first += 1;
+      t.second += ms;
+    }
+    p.pool.push_back(r.a);
+    p.pool.push_back(r.b);
+  }
+  p.pending.clear();
+  std::string out;
+  char line[256];
+  for (auto& kv : p.totals) {
+    snprintf(line, sizeof(line), "%s %ld %.6f\n", kv.first.c_str(), kv.second.first, kv.second.second);
+    out += line;
+  }
+  if (buf && len > 0) {
+    size_t n = out.size() < len - 1 ? out.size() : len - 1;
+    memcpy(buf, out.data(), n);
+    buf[n] = 0;
+  }
+  const int count = (int)p.totals.size();
+  if (reset) p.totals.clear();
+  return count;
+}
+
+int kron_delta_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(KD_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // extern "C"

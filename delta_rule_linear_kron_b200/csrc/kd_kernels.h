@@ -1,0 +1,78 @@
+// kd_kernels.h -- internal launch interface between the chunk scheduler / C ABI
+// and the CUDA kernels.  Not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kd {
+
+// Chunk length of the chunk-parallel form (Gated DeltaNet-2 article, section
+// "기술 상세": the chunk size is fixed at 64 and the chunk's triangular
+// inverse is built by forward substitution).
+constexpr int kChunk = 64;
+
+// Workspace layout of one problem (B, H, T, dk, dv), decided by the chunk
+// scheduler.  Offsets are in bytes from the workspace base, 256-byte aligned.
+// "chunk" index ch = ((b * H) + h) * NC + n.
+struct Layout {
+  int B = 0, H = 0, T = 0, dk = 0, dv = 0, dtype = 0;
+  int NC = 0;             // ceil(T / 64)
+  size_t chunks = 0;      // B * H * NC
+  // forward scratch (always): y [ch][64], A [ch][64][64], P [ch][64][64]
+  size_t y = 0, A = 0, P = 0;
+  size_t fwd_bytes = 0;
+  // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
+  size_t S0 = 0, u = 0, b0 = 0;
+  size_t fwd_save_bytes = 0;
+  // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],
+  // accq/acck/accL [ch][64][dk], accv [ch][64][dv]
+  size_t dSC = 0, g = 0, dP = 0, dGK = 0, dGVs = 0, accq = 0, acck = 0, accL = 0, accv = 0;
+  size_t bwd_bytes = 0;
+};
+
+struct DecodeArgs {
+  const void *q, *k, *v;
+  const float *beta, *c, *logf;
+  float* S;
+  void* out;
+  int B, H, dk, dv, dtype;
+};
+
+struct FwdArgs {
+  const void *q, *k, *v;
+  const float *beta, *c, *logf, *S0;
+  void* out;
+  float* ST;
+  int save;
+  char* ws;  // workspace base
+  Layout L;
+};
+
+struct BwdArgs {
+  const void *q, *k, *v;
+  const float *beta, *c, *logf, *S0;
+  const void* dO;
+  const float* dST;
+  void *dq, *dk, *dv;
+  float *dbeta, *dc, *dlogf, *dS0;
+  const char* fws;  // forward workspace (saved)
+  char* ws;         // backward workspace
+  Layout L;
+};
+
+// Profiling brackets around each kernel launch (no-ops unless enabled).
+void prof_begin(cudaStream_t st, const char* name);
+void prof_end(cudaStream_t st);
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st);
+
+template <typename T>
+inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }
+template <typename T>
+inline const T* ws_ptr(const char* base, size_t off) { return reinterpret_cast<const T*>(base + off); }
+
+}  // namespace kd

@@ -1,0 +1,181 @@
+/*
+ * kron_delta.h -- C ABI of the B200 (sm_100a) Kronecker delta rule library.
+ *
+ * The operation is the KronLSTM token mixer.  Per (batch b, head h) there is
+ * one fp32 state S in R^{dv x dk} (row r = value channel, column j = key
+ * channel).  For each token t:
+ *
+ *     Sbar_t = S_{t-1} diag(f_t),  f_t = exp(logf_t)         (forget gate)
+ *     b_t    = v_t^T Sbar_t k_t                              (association)
+ *     u_t    = c_t - beta_t b_t                              (erase, write)
+ *     S_t    = Sbar_t + u_t v_t k_t^T
+ *     o_t    = S_t q_t
+ *
+ * Sources (web pages on the method, cited by title and section):
+ *   KronLSTM digest, "KronLSTM이 스칼라 보정으로 긴 문맥 선형 어텐션의 기억
+ *     간섭을 줄인다": section "어떻게 동작하나" (the Kronecker delta rule:
+ *     one scalar association v^T S k corrected along v k^T, erase amount beta,
+ *     write amount c), section "어떻게 쓰나" (diagonal forget gate on the key
+ *     dimension applied from the right; per-head scalar beta, c; L2-normalised
+ *     q, k, v), section "무엇과 다른가" (DeltaNet-style chunk-parallel form).
+ *   Gated DeltaNet-2 article (aitrends.kr), section "기술 상세": chunk size
+ *     C = 64 and forward substitution for the chunk's triangular inverse.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers on the current CUDA device unless
+ *     stated otherwise.  The caller owns every buffer; the library allocates
+ *     no device memory, keeps no state between calls except a thread-local
+ *     error string and a cached device-property query, and never
+ *     synchronises the stream (except kron_delta_device_status).
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work of a call is enqueued on it, in order.
+ *   - Layouts (all contiguous, row-major):
+ *       q, k            [B, T, H, dk]      dtype
+ *       v, out, dO      [B, T, H, dv]      dtype
+ *       beta, c         [B, T, H]          fp32
+ *       logf            [B, T, H, dk]      fp32 (log of the forget gate, <= 0)
+ *       S0, ST, dST,dS0 [B, H, dv, dk]     fp32
+ *     dtype = KD_F32 (fp32) or KD_BF16 (bfloat16) for q, k, v, out, dO, dq,
+ *     dk, dv; gates and states are fp32 in both cases.
+ *   - Supported sizes: dk, dv in {32, 64, 128}; B, H >= 1; T >= 1 (a final
+ *     partial chunk of fewer than 64 tokens is handled).  Pointers to fp32
+ *     data must be 4-byte aligned, to bf16 data 2-byte aligned; 16-byte
+ *     alignment of q, k, v, dO is required (checked).
+ *   - Preconditions not checked on the device: q, k, v are L2-normalised by
+ *     the caller (the library never renormalises); logf <= 0; beta in [0, 2);
+ *     outputs do not alias inputs.
+ *   - Return value: KD_OK, or an error code; on error nothing was enqueued
+ *     and kron_delta_last_error() describes the first problem found.
+ */
+#ifndef KRON_DELTA_H
+#define KRON_DELTA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define KD_API __attribute__((visibility("default")))
+#else
+#define KD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define KD_OK 0
+#define KD_ERR_INVALID_ARG 1   /* null pointer, bad size, misalignment */
+#define KD_ERR_UNSUPPORTED 2   /* dk/dv/dtype outside the supported set */
+#define KD_ERR_WORKSPACE 3     /* workspace missing or too small */
+#define KD_ERR_CUDA 4          /* a CUDA runtime call or launch failed */
+#define KD_ERR_TIMEOUT 5       /* a bounded device-side wait gave up */
+
+/* element types of q, k, v, out, dO, dq, dk, dv */
+#define KD_F32 0
+#define KD_BF16 1
+
+/* workspace kinds for kron_delta_workspace_size */
+#define KD_WS_FWD 0        /* forward only (prefill / inference) */
+#define KD_WS_FWD_SAVE 1   /* forward that keeps what the backward needs */
+#define KD_WS_BWD 2        /* backward scratch (besides the saved forward) */
+
+/* Library version, as 10000*major + 100*minor + patch. */
+KD_API int kron_delta_version(void);
+
+/* Description of the last error on the calling thread ("" if none).  The
+ * string is owned by the library and valid until the next call on the same
+ * thread. */
+KD_API const char *kron_delta_last_error(void);
+
+/* Bytes of device workspace the given call needs (0 for invalid sizes; the
+ * reason is then in kron_delta_last_error).  The workspace must be 256-byte
+ * aligned.  KD_WS_FWD_SAVE holds, per 64-token chunk and head, the chunk's
+ * triangular inverse A = (I + diag(beta) M)^{-1}, the query-key decay matrix
+ * P, the chunk-start state and the per-token b_t and u_t; kron_delta_bwd reads
+ * them back. */
+KD_API size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv,
+                                 int dtype);
+
+/*
+ * Chunk-parallel forward (C = 64).
+ *   q, k, v, beta, c, logf : inputs (layouts above).
+ *   S0  : initial state [B,H,dv,dk] fp32, or NULL for zero.
+ *   out : o_t for every token [B,T,H,dv] (dtype).
+ *   ST  : final state [B,H,dv,dk] fp32, or NULL to skip.
+ *   workspace, ws_bytes : device scratch of at least
+ *         kron_delta_workspace_size(save ? KD_WS_FWD_SAVE : KD_WS_FWD, ...).
+ *   save : 1 = keep the forward quantities the backward reads in the
+ *         workspace (pass the same workspace to kron_delta_bwd); 0 = not.
+ * Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE,
+ * KD_ERR_CUDA.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_fwd(const void *q, const void *k, const void *v,
+                   const float *beta, const float *c, const float *logf,
+                   const float *S0, void *out, float *ST, int B, int H, int T,
+                   int dk, int dv, int dtype, void *workspace, size_t ws_bytes,
+                   int save, void *stream);
+
+/*
+ * Backward of kron_delta_fwd for the loss l = <dO, out> + <dST, ST>.
+ *   fwd_ws, fwd_ws_bytes : the workspace of a kron_delta_fwd call with save=1
+ *         on exactly these inputs (read only).
+ *   dO  : upstream gradient of out [B,T,H,dv] (dtype).
+ *   dST : upstream gradient of ST [B,H,dv,dk] fp32, or NULL for zero.
+ *   dq, dk, dv : [B,T,H,dk|dv] (dtype).  dbeta, dc : [B,T,H] fp32.
+ *   dlogf : [B,T,H,dk] fp32.  dS0 : [B,H,dv,dk] fp32, or NULL to skip.
+ *   workspace, ws_bytes : scratch of at least
+ *         kron_delta_workspace_size(KD_WS_BWD, ...).
+ * S0 is the same initial state given to the forward (NULL = zero).
+ * Errors as for kron_delta_fwd.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_bwd(const void *q, const void *k, const void *v,
+                   const float *beta, const float *c, const float *logf,
+                   const float *S0, const void *dO, const float *dST,
+                   void *dq, void *dk, void *dv, float *dbeta, float *dc,
+                   float *dlogf, float *dS0, int B, int H, int T, int dk_,
+                   int dv_, int dtype, const void *fwd_ws, size_t fwd_ws_bytes,
+                   void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * One recurrent decode step: one new token per (b, h).
+ *   q, k : [B,H,dk] (dtype); v : [B,H,dv] (dtype).
+ *   beta, c : [B,H] fp32; logf : [B,H,dk] fp32.
+ *   S   : [B,H,dv,dk] fp32, read and overwritten in place with S_t.
+ *   out : o_t = S_t q_t, [B,H,dv] (dtype).
+ * No workspace.  Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_CUDA.
+ * Asynchronous on `stream`.
+ */
+KD_API int kron_delta_decode(const void *q, const void *k, const void *v,
+                      const float *beta, const float *c, const float *logf,
+                      float *S, void *out, int B, int H, int dk, int dv,
+                      int dtype, void *stream);
+
+/*
+ * Synchronises `stream` and reports device-side failures of earlier calls:
+ * KD_OK, KD_ERR_TIMEOUT (a bounded inter-CTA wait gave up; the outputs of that
+ * call are invalid) or KD_ERR_CUDA.  Clears the device error word.
+ */
+KD_API int kron_delta_device_status(void *stream);
+
+/*
+ * Per-kernel device timing (tracing aid for tests and benchmarks; off by
+ * default).  While enabled, every kernel the library launches is bracketed by
+ * two CUDA events recorded on its stream; the events are pooled and reused.
+ * Not thread-safe against concurrent calls from several host threads.
+ */
+KD_API void kron_delta_profile_enable(int on);
+
+/*
+ * Synchronises the current device, folds every finished bracket into
+ * per-kernel totals and writes one line per kernel, "name launches total_ms\n",
+ * into buf (host memory, at most len bytes including the terminating NUL;
+ * buf may be NULL when len is 0).  reset = 1 clears the totals afterwards.
+ * Returns the number of kernels listed, or -KD_ERR_CUDA on a CUDA failure.
+ */
+KD_API int kron_delta_profile_report(char *buf, size_t len, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRON_DELTA_H */

@@ -1,0 +1,107 @@
+"""The C ABI library loads, exports every function include/*.h declares, and
+rejects bad arguments with the documented error codes before touching the
+GPU (no compute calls here; runs without a GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import delta_rule_linear_kron_b200 as kd
+from delta_rule_linear_kron_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kd.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(kron_delta_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert "kron_delta_fwd" in names and "kron_delta_bwd" in names and "kron_delta_decode" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_empty_error(L):
+    assert L.kron_delta_version() >= 100
+    assert isinstance(L.kron_delta_last_error(), bytes)
+
+
+def test_workspace_sizes(L):
+    B, H, T, d = 1, 16, 16384, 128
+    f = kd.workspace_size(kd.KD_WS_FWD, B, H, T, d, d)
+    fs = kd.workspace_size(kd.KD_WS_FWD_SAVE, B, H, T, d, d)
+    bw = kd.workspace_size(kd.KD_WS_BWD, B, H, T, d, d)
+    chunks = B * H * (T // 64)
+    assert f >= chunks * (64 + 2 * 64 * 64) * 4
+    assert fs >= f + chunks * d * d * 4
+    assert bw >= chunks * d * d * 4
+    # ragged T rounds the chunk count up
+    assert kd.workspace_size(kd.KD_WS_FWD, 1, 1, 65, 32, 32) > kd.workspace_size(kd.KD_WS_FWD, 1, 1, 64, 32, 32)
+    assert L.kron_delta_workspace_size(0, 1, 1, 64, 48, 32, 1) == 0
+    assert b"32, 64 or 128" in L.kron_delta_last_error()
+    assert L.kron_delta_workspace_size(9, 1, 1, 64, 32, 32, 1) == 0
+
+
+def _fwd_call(L, **over):
+    p = ctypes.c_void_p(256)  # aligned non-null dummy: never dereferenced when validation fails
+    args = dict(q=p, k=p, v=p, beta=p, c=p, logf=p, S0=None, out=p, ST=None, B=1, H=1, T=64, dk=32, dv=32,
+                dtype=1, ws=p, ws_bytes=0, save=0, stream=None)
+    args.update(over)
+    return L.kron_delta_fwd(args["q"], args["k"], args["v"], args["beta"], args["c"], args["logf"],
+                            args["S0"], args["out"], args["ST"], args["B"], args["H"], args["T"],
+                            args["dk"], args["dv"], args["dtype"], args["ws"], args["ws_bytes"],
+                            args["save"], args["stream"])
+
+
+def test_fwd_argument_errors(L):
+    assert _fwd_call(L, dk=48) == kd.KD_ERR_UNSUPPORTED
+    assert _fwd_call(L, dtype=7) == kd.KD_ERR_UNSUPPORTED
+    assert _fwd_call(L, T=0) == kd.KD_ERR_INVALID_ARG
+    assert _fwd_call(L, B=-1) == kd.KD_ERR_INVALID_ARG
+    assert _fwd_call(L, q=None) == kd.KD_ERR_INVALID_ARG
+    assert b"q must not be NULL" in L.kron_delta_last_error()
+    assert _fwd_call(L, k=ctypes.c_void_p(258)) == kd.KD_ERR_INVALID_ARG
+    assert b"aligned" in L.kron_delta_last_error()
+    assert _fwd_call(L, save=2) == kd.KD_ERR_INVALID_ARG
+    assert _fwd_call(L, ws_bytes=10) == kd.KD_ERR_WORKSPACE
+    need = kd.workspace_size(kd.KD_WS_FWD, 1, 1, 64, 32, 32)
+    assert _fwd_call(L, ws_bytes=need, ws=ctypes.c_void_p(256 + 16)) == kd.KD_ERR_WORKSPACE
+    assert _fwd_call(L, ws_bytes=need, save=1) == kd.KD_ERR_WORKSPACE
+
+
+def test_bwd_and_decode_argument_errors(L):
+    p = ctypes.c_void_p(256)
+    rc = L.kron_delta_bwd(p, p, p, p, p, p, None, p, None, p, p, p, p, p, p, None,
+                          1, 1, 64, 32, 32, 1, p, 0, p, 0, None)
+    assert rc == kd.KD_ERR_WORKSPACE
+    rc = L.kron_delta_bwd(p, p, p, p, p, p, None, None, None, p, p, p, p, p, p, None,
+                          1, 1, 64, 32, 32, 1, p, 0, p, 0, None)
+    assert rc == kd.KD_ERR_INVALID_ARG
+    rc = L.kron_delta_decode(p, p, p, p, p, p, p, p, 1, 1, 128, 96, 1, None)
+    assert rc == kd.KD_ERR_UNSUPPORTED
+    rc = L.kron_delta_decode(p, p, p, p, p, p, None, p, 1, 1, 128, 128, 1, None)
+    assert rc == kd.KD_ERR_INVALID_ARG
+    rc = L.kron_delta_decode(p, p, p, p, p, p, p, p, 0, 1, 128, 128, 1, None)
+    assert rc == kd.KD_ERR_INVALID_ARG
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    q = torch.zeros(1, 64, 1, 32)
+    with pytest.raises(kd.KronDeltaError):
+        kd.fwd(q, q, q, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1), q)
