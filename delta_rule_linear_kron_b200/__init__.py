@@ -60,6 +60,8 @@ def lib():
         L.kron_delta_decode.argtypes = [vp] * 8 + [i] * 5 + [vp]
         L.kron_delta_device_status.restype = i
         L.kron_delta_device_status.argtypes = [vp]
+        L.kron_delta_fwd_noalloc.restype = i
+        L.kron_delta_fwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [vp]
         L.kron_delta_profile_enable.restype = None
         L.kron_delta_profile_enable.argtypes = [i]
         L.kron_delta_profile_report.restype = i

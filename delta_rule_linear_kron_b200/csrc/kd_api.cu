@@ -133,6 +133,8 @@ ProfState& prof() {
 }  // namespace
 
 namespace kd {
+void set_error(const char* msg) { g_err = msg ? msg : ""; }
+
 void prof_begin(cudaStream_t st, const char* name) {
   ProfState& p = prof();
   std::lock_guard<std::mutex> g(p.mu);

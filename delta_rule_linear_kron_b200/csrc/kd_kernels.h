@@ -62,6 +62,9 @@ struct BwdArgs {
   Layout L;
 };
 
+// Sets the calling thread's kron_delta_last_error() string.
+void set_error(const char* msg);
+
 // Profiling brackets around each kernel launch (no-ops unless enabled).
 void prof_begin(cudaStream_t st, const char* name);
 void prof_end(cudaStream_t st);

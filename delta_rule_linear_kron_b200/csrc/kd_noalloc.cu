@@ -1,0 +1,100 @@
+// kd_noalloc.cu -- forward entry point that needs no caller-provided workspace
+// and allocates nothing.
+//
+// Who this is for: callers that cannot allocate device memory when they call
+// the mixer -- for example a host process whose device memory is entirely
+// reserved up front by another allocator (a serving runtime, or a plugin that
+// has no handle to its host's allocator), or a loop with a no-allocation rule
+// after start-up.  Such callers still own and pass their inputs and outputs;
+// only the forward's scratch (the per-chunk y, A and P) comes from the fixed
+// array below, which is part of the library image.
+//
+// Limits and behaviour:
+//   * The scratch is a file-scope device array of kNoAllocScratchBytes
+//     (32 MiB).  Every GPU that loads the library holds it until the process
+//     exits.  A problem whose forward scratch exceeds it (more than 1016
+//     chunk-heads, i.e. B * H * ceil(T/64) > 1016 at any dk, dv) is rejected
+//     with KD_ERR_WORKSPACE before anything is enqueued.
+//   * All calls share the one array and it keeps the last call's contents.
+//     The forward writes every scratch element it later reads, so nothing
+//     has to start at zero.  Calls whose kernels overlap on the GPU (other
+//     streams, other host threads) race on the array: the caller must order
+//     them.
+//   * The first call on each device looks up the array's device address with
+//     cudaGetSymbolAddress (with that device current) and caches it; make that
+//     first call before any stream capture begins.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/kron_delta.h"
+#include "kd_kernels.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// The device address of the scratch array on the current device (looked up
+// once per device; the array's name is only a host-side stand-in).
+cudaError_t scratch_on_current_device(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kron_delta_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
+                           const float* c, const float* logf, const float* S0, void* out,
+                           float* ST, int B, int H, int T, int dk, int dv, int dtype,
+                           void* stream) {
+  // Size the scratch with the library's own planner.  Invalid sizes: let the
+  // regular entry point validate them (it rejects them before looking at the
+  // workspace) so the error code and message are the usual ones.
+  const size_t need = kron_delta_workspace_size(KD_WS_FWD, B, H, T, dk, dv, dtype);
+  if (need == 0)
+    return kron_delta_fwd(q, k, v, beta, c, logf, S0, out, ST, B, H, T, dk, dv, dtype, nullptr, 0,
+                          0, stream);
+  if (need > kNoAllocScratchBytes) {
+    char msg[256];
+    snprintf(msg, sizeof(msg),
+             "kron_delta_fwd_noalloc: forward scratch of %zu bytes exceeds the fixed %zu-byte array "
+             "(B*H*ceil(T/64) must be <= 1016); use kron_delta_fwd with a workspace",
+             need, kNoAllocScratchBytes);
+    kd::set_error(msg);
+    return KD_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  const cudaError_t e = scratch_on_current_device(&scratch);
+  if (e != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof(msg), "kron_delta_fwd_noalloc: scratch address lookup failed: %s",
+             cudaGetErrorString(e));
+    kd::set_error(msg);
+    return KD_ERR_CUDA;
+  }
+  return kron_delta_fwd(q, k, v, beta, c, logf, S0, out, ST, B, H, T, dk, dv, dtype, scratch,
+                        kNoAllocScratchBytes, 0, stream);
+}
+
+}  // extern "C"

@@ -151,6 +151,28 @@ KD_API int kron_delta_decode(const void *q, const void *k, const void *v,
                       int dtype, void *stream);
 
 /*
+ * Forward that allocates nothing and takes no workspace (no counterpart on the
+ * method's pages; a library convenience).  For callers that cannot allocate
+ * device memory at call time -- e.g. a process whose device memory is all
+ * reserved up front by another allocator, or a plugin without access to its
+ * host's allocator.  Same arguments and results as kron_delta_fwd with
+ * save = 0, minus the workspace: the forward's scratch comes from one fixed
+ * 32 MiB device array inside the library (held on every GPU that loads the
+ * library until exit).
+ *   - Problems needing more scratch than that (B * H * ceil(T/64) > 1016)
+ *     return KD_ERR_WORKSPACE; use kron_delta_fwd then.
+ *   - All calls share the array; concurrent calls that overlap on the GPU
+ *     race on it, so the caller must serialise them (e.g. one stream).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make it before any stream capture.
+ * Errors as for kron_delta_fwd.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_fwd_noalloc(const void *q, const void *k, const void *v,
+                                  const float *beta, const float *c, const float *logf,
+                                  const float *S0, void *out, float *ST, int B, int H,
+                                  int T, int dk, int dv, int dtype, void *stream);
+
+/*
  * Synchronises `stream` and reports device-side failures of earlier calls:
  * KD_OK, KD_ERR_TIMEOUT (a bounded inter-CTA wait gave up; the outputs of that
  * call are invalid) or KD_ERR_CUDA.  Clears the device error word.

@@ -1,0 +1,62 @@
+"""kron_delta_fwd_noalloc: the forward for callers that cannot allocate device
+memory at call time (for instance a process whose device memory is all
+reserved by another allocator).  Its scratch is a fixed 32 MiB array inside
+the library, so it must give the same results as kron_delta_fwd with a
+caller-provided workspace, call after call, even though the array keeps the
+previous call's contents.
+
+This file is named so that pytest collects it last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import delta_rule_linear_kron_b200 as kd
+from delta_rule_linear_kron_b200 import inputs as kin
+
+TOL_BF16 = 5e-3  # the bf16 forward tolerance used by the parity tests
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def test_rejects_problems_beyond_the_fixed_scratch():
+    L = kd.lib()
+    p = ctypes.c_void_p(256)  # never dereferenced: the call is rejected first
+    # B*H*ceil(T/64) = 1 * 1 * 1017 chunk-heads: one more than fits
+    rc = L.kron_delta_fwd_noalloc(p, p, p, p, p, p, None, p, None, 1, 1, 1017 * 64, 128, 128, 1, None)
+    assert rc == kd.KD_ERR_WORKSPACE
+    assert b"exceeds the fixed" in L.kron_delta_last_error()
+    rc = L.kron_delta_fwd_noalloc(p, p, p, p, p, p, None, p, None, 1, 1, 64, 96, 128, 1, None)
+    assert rc == kd.KD_ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_forward_twice():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test needs a CUDA device")
+    L = kd.lib()
+    cases = [dict(B=2, H=4, T=1000, seed=901), dict(B=1, H=8, T=1500, seed=902)]  # 128 and 192 chunk-heads
+    for case in cases:
+        inp = kin.make_inputs(3, B=case["B"], H=case["H"], T=case["T"], seed=case["seed"], with_dO=False)
+        d = {n: torch.from_numpy(inp[n]).to("cuda", torch.bfloat16 if n in ("q", "k", "v") else torch.float32)
+             for n in ("q", "k", "v", "beta", "c", "logf", "S0")}
+        B, T, H, dk = d["q"].shape
+        dv = d["v"].shape[-1]
+        ref_out, ref_ST, _ = kd.fwd(d["q"], d["k"], d["v"], d["beta"], d["c"], d["logf"], d["S0"])
+        out = torch.full((B, T, H, dv), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ST = torch.full((B, H, dv, dk), float("nan"), dtype=torch.float32, device="cuda")
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        rc = L.kron_delta_fwd_noalloc(_p(d["q"]), _p(d["k"]), _p(d["v"]), _p(d["beta"]), _p(d["c"]),
+                                      _p(d["logf"]), _p(d["S0"]), _p(out), _p(ST), B, H, T, dk, dv,
+                                      kd.KD_BF16, stream)
+        assert rc == kd.KD_OK, L.kron_delta_last_error()
+        torch.cuda.synchronize()
+        for x, ref in ((out, ref_out), (ST, ref_ST)):
+            x = x.double().cpu().numpy()
+            ref = ref.double().cpu().numpy()
+            assert np.isfinite(x).all()
+            assert np.linalg.norm(x - ref) / np.linalg.norm(ref) <= TOL_BF16
