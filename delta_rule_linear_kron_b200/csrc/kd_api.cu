@@ -57,14 +57,17 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   const size_t C = kd::kChunk;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  L->tc = dtype == KD_BF16 && dk == 128 && dv == 128;
   L->y = take(chunks * C * 4);
   L->A = take(chunks * C * C * 4);
-  L->P = take(chunks * C * C * 4);
+  L->P = take(chunks * C * C * 4);  // tensor-core path: written only when saving for the backward
   L->fwd_bytes = off;
   L->S0 = take(chunks * (size_t)dv * dk * 4);
   L->u = take(chunks * C * 4);
   L->b0 = take(chunks * C * 4);
+  L->flags = take(chunks * 4);
   L->fwd_save_bytes = off;
+  if (L->tc) L->fwd_bytes = off;  // its output kernel reads the chunk-start states
   off = 0;
   L->dSC = take(chunks * (size_t)dv * dk * 4);
   L->g = take(chunks * C * 4);
@@ -106,6 +109,38 @@ int check_stream(void* stream) {
 int launched(cudaError_t e, const char* what) {
   if (e != cudaSuccess) return fail(KD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return ok();
+}
+
+// ---- device error word (bounded device-side waits report here) ------------
+__device__ int g_kd_dev_err;
+
+struct DeviceInfo {
+  int* err = nullptr;
+  int sms = 0;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+// Error-word address and SM count of the current device (queried once).
+int device_info(DeviceInfo* out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(KD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(KD_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> g(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.err) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_kd_dev_err);
+    if (e != cudaSuccess) return fail(KD_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(KD_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    d.sms = sms;
+    d.err = static_cast<int*>(p);
+  }
+  *out = d;
+  return KD_OK;
 }
 
 // ---- per-kernel timing (kron_delta_profile_*) ----------------------------
@@ -203,6 +238,12 @@ int kron_delta_fwd(const void* q, const void* k, const void* v, const float* bet
   if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   KD_TRY(check_stream(stream));
   kd::FwdArgs a{q, k, v, beta, c, logf, S0, out, ST, save, static_cast<char*>(workspace), L};
+  if (L.tc) {
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    return launched(kd::launch_fwd_tc(a, di.err, di.sms, static_cast<cudaStream_t>(stream)),
+                    "forward launch");
+  }
   return launched(kd::launch_fwd_simt(a, static_cast<cudaStream_t>(stream)), "forward launch");
 }
 
@@ -308,8 +349,22 @@ int kron_delta_profile_report(char* buf, size_t len, int reset) {
 }
 
 int kron_delta_device_status(void* stream) {
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return fail(KD_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  DeviceInfo di;
+  KD_TRY(device_info(&di));
+  int word = 0;
+  e = cudaMemcpyAsync(&word, di.err, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(KD_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+  if (word != 0) {
+    const int zero = 0;
+    cudaMemcpyAsync(di.err, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
+    cudaStreamSynchronize(st);
+    return fail(KD_ERR_TIMEOUT, "a bounded device-side wait gave up (code %d); outputs of that call are invalid",
+                word);
+  }
   return ok();
 }
 

@@ -277,6 +277,15 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
 // ---------------------------------------------------------------------------
 constexpr int SLAB = 16;
 
+// float index of (r, j) in a 128x128 tf32 tile stored K-major with 128-byte
+// swizzle: 4 blocks of 32 columns, 1024-byte atoms of 8 rows, 16-byte chunks
+// permuted by XOR with (row % 8)
+__device__ __forceinline__ size_t sw128_index(int r, int j) {
+  const int kb = j >> 5, chunk = (j & 31) >> 2;
+  return (size_t)kb * 128 * 32 + (size_t)(r >> 3) * 256 + (size_t)(r & 7) * 32 +
+         (size_t)(((chunk ^ (r & 7)) & 7) * 4) + (j & 3);
+}
+
 template <int DK, int DV>
 constexpr size_t bstate_smem_floats() {
   return 3 * (size_t)C * (DK + 1) + 2 * (size_t)C * (DV + 1) + 2 * (size_t)SLAB * (DK + 1) + 2 * C +
@@ -289,7 +298,7 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
     const float* __restrict__ beta, const float* __restrict__ logf, const Tin* __restrict__ dO,
     int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wg,
     const float* __restrict__ wS0, const float* __restrict__ wdSC, float* __restrict__ waccq,
-    float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv) {
+    float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv, int s0_swizzled) {
   constexpr int SK = DK + 1, SV = DV + 1;
   constexpr int TPJ = 256 / DK;   // thread groups over j
   constexpr int TPG = C / TPJ;    // rows per group
@@ -357,7 +366,9 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
   for (int r0 = 0; r0 < DV; r0 += SLAB) {
     for (int e = tid; e < SLAB * DK; e += blockDim.x) {
       const int rr = e / DK, jj = e % DK;
-      S0s[rr * SK + jj] = S0c[(size_t)(r0 + rr) * DK + jj];
+      // the tensor-core forward stores each chunk-start state as a 128x128
+      // tf32 tile in the 128-byte-swizzled K-major layout of its MMAs
+      S0s[rr * SK + jj] = s0_swizzled ? S0c[sw128_index(r0 + rr, jj)] : S0c[(size_t)(r0 + rr) * DK + jj];
       dSs[rr * SK + jj] = dSc[(size_t)(r0 + rr) * DK + jj];
     }
     __syncthreads();
@@ -632,7 +643,7 @@ static cudaError_t run_bwd(const BwdArgs& a, cudaStream_t st) {
   prof_begin(st, "bwd_state_simt");
   bwd_state_simt<DK, DV, Tin><<<gridc, 256, s3, st>>>(q, k, v, a.beta, a.logf, dO, L.H, L.T,
                                                       L.NC, wu, wg, wS0, wdSC, waccq, wacck,
-                                                      waccL, waccv);
+                                                      waccL, waccv, L.tc ? 1 : 0);
   prof_end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prof_begin(st, "bwd_intra_simt");

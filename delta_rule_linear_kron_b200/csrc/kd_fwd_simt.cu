@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(256) fwd_prep_simt(
   for (int e = tid; e < C * C; e += blockDim.x) {
     const int t = e / C, i = e % C;
     wA[ch * C * C + e] = As[t * SC + i];
-    wP[ch * C * C + e] = Ps[t * SC + i];
+    if (wP) wP[ch * C * C + e] = Ps[t * SC + i];
   }
 }
 
@@ -361,6 +361,34 @@ static cudaError_t run_fwd(const FwdArgs& a, cudaStream_t st) {
       a.save ? ws_ptr<float>(a.ws, L.u) : nullptr, a.save ? ws_ptr<float>(a.ws, L.b0) : nullptr);
   prof_end(st);
   return cudaGetLastError();
+}
+
+template <int DK, int DV, typename Tin>
+static cudaError_t run_prep(const FwdArgs& a, bool with_P, cudaStream_t st) {
+  const Layout& L = a.L;
+  const size_t sp = prep_smem_floats<DK, DV>() * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(fwd_prep_simt<DK, DV, Tin>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp);
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "fwd_prep_simt");
+  fwd_prep_simt<DK, DV, Tin><<<dim3(L.NC, L.H, L.B), 256, sp, st>>>(
+      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.beta,
+      a.c, a.logf, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
+      with_P ? ws_ptr<float>(a.ws, L.P) : nullptr);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_prep(const FwdArgs& a, bool with_P, cudaStream_t st) {
+#define KD_P(DK_, DV_)                                                            \
+  if (a.L.dk == DK_ && a.L.dv == DV_)                                             \
+    return a.L.dtype == 0 ? run_prep<DK_, DV_, float>(a, with_P, st)              \
+                          : run_prep<DK_, DV_, __nv_bfloat16>(a, with_P, st);
+  KD_P(32, 32) KD_P(32, 64) KD_P(32, 128)
+  KD_P(64, 32) KD_P(64, 64) KD_P(64, 128)
+  KD_P(128, 32) KD_P(128, 64) KD_P(128, 128)
+#undef KD_P
+  return cudaErrorInvalidValue;
 }
 
 template <typename Tin>

@@ -1,0 +1,681 @@
+// kd_fwd_tc.cu -- tensor-core (tcgen05/TMEM) forward for bf16 q,k,v and
+// d_k = d_v = 128.
+//
+// Chunk form as in kd_fwd_simt.cu (KronLSTM digest, "무엇과 다른가": the
+// DeltaNet chunk-parallel scheme applies; Gated DeltaNet-2 article, "방법론" /
+// "기술 상세": WY form, C = 64, forward substitution):
+//   b0 = rowdot(V, S0 K+^T), u = y - A (beta o b0),
+//   S  <- S diag(gamma_C) + V^T diag(u) K^e,
+//   O  = Q+ S0^T + P diag(u) V.
+//
+// Kernels:
+//  1. prep (kd_fwd_simt.cu, fwd_prep_simt): A = (I + diag(beta) M)^{-1}, y.
+//  2. fwd_chain_tc: the sequential chain.  One thread-block cluster of R CTAs
+//     per (b,h); CTA c owns the key-channel slice J_c (dk/R columns) of the
+//     state, kept in tensor memory as the A operand of the MMAs:
+//       X_c = S[:,J_c] K+[:,J_c]^T            (tcgen05, A from TMEM)
+//       b0_c[t] = sum_r V[t,r] X_c[r,t]       (column sum over TMEM lanes)
+//       b0 = sum_c b0_c                       (distributed shared memory:
+//                                              st.async + mbarrier tx count)
+//       u = y - A (beta o b0)                 (every CTA, identical order)
+//       dS_c = V^T (diag(u) K^e[:,J_c])       (tcgen05)
+//       S[:,J_c] <- S[:,J_c] diag(gamma_C) + dS_c
+//     The next chunk's rows are fetched with bulk async copies while the
+//     current chunk runs.  Each chunk-start state slice is written to global
+//     memory in the 128-byte-swizzled K-major tile layout the output kernel's
+//     MMA reads directly.
+//  3. fwd_out_tc: one CTA per chunk, all chunks in parallel:
+//       O^T = S0 Q+^T + V^T (diag(u) P^T)  with P = tril(Q+ K-^T) (tcgen05).
+//     Chunks whose log-decay range makes k/gamma leave the fp32 range are
+//     flagged and recomputed exactly by fwd_out_fixup.
+#include "kd_common.cuh"
+#include "kd_kernels.h"
+#include "kd_tc.cuh"
+
+namespace kd {
+namespace {
+
+constexpr int C = kChunk;
+constexpr int D = 128;
+
+template <int R>
+struct ChainCfg {
+  static constexpr int NJ = D / R;                    // key channels per CTA
+  static constexpr int KB1 = (NJ * 4 + 127) / 128;    // 128-byte K blocks of K+ slice
+  static constexpr int TPC = 128 / NJ;                // scan threads per channel
+  static constexpr int SEG = C / TPC;                 // positions per scan thread
+  static constexpr int D1_COL = 0, S_COL = 64, D2_COL = 64 + NJ;
+  static constexpr uint32_t TMEM_COLS = (64 + 2 * NJ) <= 128 ? 128u : 256u;
+  static constexpr int KES = NJ + 1;                  // padded row of K^e (fp32)
+  // shared memory map (bytes from a 1024-aligned base)
+  static constexpr uint32_t B1 = 0;                                   // K+ slice, tf32 SW128, 64 rows
+  static constexpr uint32_t A2 = B1 + KB1 * 64 * 128;                  // V^T, tf32 SW128, 128 rows, K=64
+  static constexpr uint32_t B2 = A2 + 2 * 128 * 128;                   // diag(u) K^e slice, NJ rows, K=64
+  static constexpr uint32_t KE = B2 + 2 * NJ * 128;                    // K^e fp32 [64][KES]
+  static constexpr uint32_t STG = ((KE + 64 * KES * 4) + 127) / 128 * 128;
+  // staging buffer (one per chunk parity), offsets inside it
+  static constexpr uint32_t VROW = 272;                                // 256 B of bf16 v + 16 B pad
+  static constexpr uint32_t ST_V = 0, ST_A = ST_V + 64 * VROW, ST_Y = ST_A + 64 * 64 * 4,
+                            ST_K = ST_Y + 256, ST_L = ST_K + 64 * NJ * 2;
+  static constexpr uint32_t ST_SZ = ((ST_L + 64 * NJ * 4) + 127) / 128 * 128;
+  static constexpr uint32_t SM = STG + 2 * ST_SZ;                      // small arrays (floats)
+  static constexpr uint32_t SM_BS = SM;                                // beta [2][64]
+  static constexpr uint32_t SM_W = SM_BS + 2 * 64 * 4;                 // beta o b0 [64]
+  static constexpr uint32_t SM_U = SM_W + 64 * 4;                      // u [64]
+  static constexpr uint32_t SM_MINE = SM_U + 64 * 4;                   // own b0 partial [64]
+  static constexpr uint32_t SM_XRED = SM_MINE + 64 * 4;                // per-warp partials [4][64]
+  static constexpr uint32_t SM_RECV = SM_XRED + 4 * 64 * 4;            // [2][R][64]
+  static constexpr uint32_t SM_GC = SM_RECV + 2 * R * 64 * 4;          // gamma_C [NJ]
+  static constexpr uint32_t SM_SEG = SM_GC + NJ * 4;                   // scan segment sums [TPC][NJ]
+  static constexpr uint32_t SM_END = SM_SEG + TPC * NJ * 4;
+  static constexpr uint32_t BYTES = SM_END + 1024;                     // + alignment slack
+};
+
+__device__ __forceinline__ float bf2f(const unsigned char* p) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+
+template <int R>
+__global__ void __launch_bounds__(128, 1) fwd_chain_tc(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const float* __restrict__ beta, const float* __restrict__ logf, const float* __restrict__ S0,
+    float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy,
+    const float* __restrict__ wA, float* __restrict__ wS0blob, float* __restrict__ wu,
+    float* __restrict__ wb0, int* __restrict__ err) {
+  using Cf = ChainCfg<R>;
+  constexpr int NJ = Cf::NJ;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar[2], x_bar[2], mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = tc::cluster_rank();
+  const int unit = blockIdx.x / R;        // (b, h)
+  const int b = unit / H, h = unit % H;
+  const int j0 = static_cast<int>(rank) * NJ;  // first key channel of this CTA
+
+  float* bs = reinterpret_cast<float*>(sm + Cf::SM_BS);
+  float* ws = reinterpret_cast<float*>(sm + Cf::SM_W);
+  float* us = reinterpret_cast<float*>(sm + Cf::SM_U);
+  float* mine = reinterpret_cast<float*>(sm + Cf::SM_MINE);
+  float* xred = reinterpret_cast<float*>(sm + Cf::SM_XRED);
+  float* recv = reinterpret_cast<float*>(sm + Cf::SM_RECV);
+  float* gC = reinterpret_cast<float*>(sm + Cf::SM_GC);
+  float* segs = reinterpret_cast<float*>(sm + Cf::SM_SEG);
+  float* KE = reinterpret_cast<float*>(sm + Cf::KE);
+
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar[0], 1);
+    tc::mbar_init(&ld_bar[1], 1);
+    tc::mbar_init(&x_bar[0], 1);
+    tc::mbar_init(&x_bar[1], 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, Cf::TMEM_COLS);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);  // this warp's 32 TMEM lanes
+
+  // initial state slice -> TMEM (thread = state row r)
+  {
+    const int r = tid;
+#pragma unroll
+    for (int jj = 0; jj < NJ; jj += 16) {
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        x[i] = S0 ? S0[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] : 0.f;
+      tc::tmem_st16(my_lanes + Cf::S_COL + jj, x);
+    }
+    tc::tmem_st_wait();
+  }
+
+  // issue the bulk copies of chunk n into staging buffer n & 1
+  auto issue_loads = [&](int n) {
+    unsigned char* st = sm + Cf::STG + (n & 1) * Cf::ST_SZ;
+    uint64_t* bar = &ld_bar[n & 1];
+    const int t0 = n * C, nv = min(C, T - t0);
+    const size_t ch = (size_t)unit * NC + n;
+    tc::fence_proxy_async();
+    if (tid == 64) {
+      tc::mbar_expect_tx(bar, (uint32_t)nv * (256u + NJ * 6u) + 64u * 64u * 4u + 256u);
+      tc::bulk_g2s(st + Cf::ST_A, wA + ch * C * C, 64u * 64u * 4u, bar);
+      tc::bulk_g2s(st + Cf::ST_Y, wy + ch * C, 256u, bar);
+    }
+    if (tid < C) {
+      const int t = tid;
+      if (t < nv) {
+        const size_t row = ((size_t)b * T + t0 + t) * H + h;
+        tc::bulk_g2s(st + Cf::ST_V + t * Cf::VROW, v + row * D, 256u, bar);
+        tc::bulk_g2s(st + Cf::ST_K + t * NJ * 2, k + row * D + j0, NJ * 2u, bar);
+        tc::bulk_g2s(st + Cf::ST_L + t * NJ * 4, logf + row * D + j0, NJ * 4u, bar);
+      } else {  // rows past T are zero
+        uint4 z = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 16; ++i) reinterpret_cast<uint4*>(st + Cf::ST_V + t * Cf::VROW)[i] = z;
+        for (int i = 0; i < NJ * 2 / 16; ++i) reinterpret_cast<uint4*>(st + Cf::ST_K + t * NJ * 2)[i] = z;
+        for (int i = 0; i < NJ * 4 / 16; ++i) reinterpret_cast<uint4*>(st + Cf::ST_L + t * NJ * 4)[i] = z;
+      }
+    }
+  };
+  auto load_beta = [&](int n) -> float {
+    const int t0 = n * C;
+    return (tid < C && t0 + tid < T) ? beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
+  };
+
+  issue_loads(0);
+  float beta_next = load_beta(0);
+  int mma_par = 0;
+  const uint32_t ID1 = tc::idesc(128, 64, 2);
+  const uint32_t ID2 = tc::idesc(128, NJ, 2);
+
+  for (int n = 0; n < NC; ++n) {
+    const int buf = n & 1;
+    unsigned char* st = sm + Cf::STG + buf * Cf::ST_SZ;
+    const size_t ch = (size_t)unit * NC + n;
+    if (tid < C) bs[buf * 64 + tid] = beta_next;
+    tc::mbar_wait<false>(&ld_bar[buf], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+    __syncthreads();  // staging of chunk n visible to all; buffer n+1 free
+    if (n + 1 < NC) {
+      issue_loads(n + 1);
+      beta_next = load_beta(n + 1);
+    }
+
+    // ---- chunk set-up: V^T (tf32, swizzled); decay prefix; K+ and K^e
+    {
+      const int t = tid & 63, rh = tid >> 6;  // rows r in [64 rh, 64 rh + 64)
+      const unsigned char* vrow = st + Cf::ST_V + t * Cf::VROW;
+#pragma unroll 2
+      for (int r8 = 0; r8 < 64; r8 += 8) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(vrow + (64 * rh + r8) * 2);
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 64 * rh + r8 + i;
+          *reinterpret_cast<float*>(sm + Cf::A2 + tc::sw128_off(r, t, 128, 4)) = __bfloat162float(e[i]);
+        }
+      }
+    }
+    {
+      const int j = tid % NJ, seg = tid / NJ;
+      const float* lrow = reinterpret_cast<const float*>(st + Cf::ST_L);
+      float lp[Cf::SEG];
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < Cf::SEG; ++i) {
+        acc += lrow[(seg * Cf::SEG + i) * NJ + j];
+        lp[i] = acc;
+      }
+      segs[seg * NJ + j] = acc;
+      __syncthreads();
+      float pre = 0.f, tot = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < Cf::TPC; ++s2) {
+        const float x = segs[s2 * NJ + j];
+        if (s2 < seg) pre += x;
+        tot += x;
+      }
+      if (seg == 0) gC[j] = expf(tot);
+#pragma unroll
+      for (int i = 0; i < Cf::SEG; ++i) {
+        const int t = seg * Cf::SEG + i;
+        const float L = pre + lp[i];
+        const float kk = bf2f(st + Cf::ST_K + (t * NJ + j) * 2);
+        *reinterpret_cast<float*>(sm + Cf::B1 + tc::sw128_off(t, j, 64, 4)) = kk * expf(L);
+        KE[t * Cf::KES + j] = kk * expf(tot - L);
+      }
+    }
+    tc::fence_proxy_async();
+    tc::tc_before_sync();
+    __syncthreads();
+    tc::tc_after_sync();
+
+    // ---- MMA 1: X_c = S[:,J_c] K+[:,J_c]^T   (M=128 rows r, N=64 positions, K=NJ)
+    if (tid == 0) {
+#pragma unroll
+      for (int ks = 0; ks < NJ / 8; ++ks) {
+        const uint64_t bd = tc::desc_sw128(tc::smem_u32(sm + Cf::B1 + (ks / 4) * 64 * 128 + (ks % 4) * 32));
+        tc::mma_tf32_ts(tmem + Cf::D1_COL, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&mma_bar);
+    }
+    tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
+    mma_par ^= 1;
+    tc::tc_after_sync();
+
+    // chunk-start state slice -> global, in the output kernel's A-operand layout
+    if (wS0blob) {
+      float* blob = wS0blob + ch * D * D;
+      const int r = tid;
+#pragma unroll
+      for (int jj = 0; jj < NJ; jj += 16) {
+        float x[16];
+        tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int jg = j0 + jj + 4 * q4;
+          *reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(blob) + tc::sw128_off(r, jg, 128, 4)) =
+              make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+        }
+      }
+    }
+    // b0_c[t] = sum_r V[t,r] X_c[r,t]: per-lane products, then column sums
+    {
+      const int r = tid;
+      float lo[32], hi[32];
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float x[16];
+        tc::tmem_ld16(my_lanes + Cf::D1_COL + 16 * c16, x);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int t = 16 * c16 + i;
+          const float pv = x[i] * bf2f(st + Cf::ST_V + t * Cf::VROW + r * 2);
+          if (t < 32) lo[t] = pv;
+          else hi[t - 32] = pv;
+        }
+      }
+      warp_transpose_reduce<32>(lo, lane);
+      warp_transpose_reduce<32>(hi, lane);
+      xred[warp * 64 + lane] = lo[0];
+      xred[warp * 64 + 32 + lane] = hi[0];
+    }
+    __syncthreads();
+    if (tid < C) mine[tid] = xred[tid] + xred[64 + tid] + xred[128 + tid] + xred[192 + tid];
+    __syncthreads();
+
+    // ---- b0 = sum over the cluster of b0_c
+    if (R > 1) {
+      float* rv = recv + buf * R * 64;
+      if (tid == 0) tc::mbar_expect_tx(&x_bar[buf], R * 64u * 4u);
+      if (tid < 16 * R) {
+        const int peer = tid / 16, q4 = tid % 16;
+        const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
+        const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
+        const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[buf]), (uint32_t)peer);
+        tc::st_async_v4(raddr, val, rbar);
+      }
+      tc::mbar_wait<true>(&x_bar[buf], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
+      if (tid < C) {
+        float s = 0.f;
+#pragma unroll
+        for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + tid];  // same order in every CTA
+        ws[tid] = bs[buf * 64 + tid] * s;
+        if (rank == 0 && wb0) wb0[ch * C + tid] = s;
+      }
+    } else {
+      if (tid < C) {
+        ws[tid] = bs[buf * 64 + tid] * mine[tid];
+        if (wb0) wb0[ch * C + tid] = mine[tid];
+      }
+    }
+    __syncthreads();
+    // ---- u = y - A (beta o b0); rotated reads keep the A rows conflict-free
+    if (tid < C) {
+      const float* Arow = reinterpret_cast<const float*>(st + Cf::ST_A) + tid * 64;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < 64; i += 2) {
+        const int i0 = (i + tid) & 63, i1 = (i + 1 + tid) & 63;
+        s0 = fmaf(Arow[i0], ws[i0], s0);
+        s1 = fmaf(Arow[i1], ws[i1], s1);
+      }
+      const float u = reinterpret_cast<const float*>(st + Cf::ST_Y)[tid] - (s0 + s1);
+      us[tid] = u;
+      if (rank == 0 && wu) wu[ch * C + tid] = u;
+    }
+    __syncthreads();
+    // ---- B2 = diag(u) K^e[:, J_c]  (N = NJ rows j, K = 64 positions)
+    {
+      const int t = tid & 63, jh = tid >> 6;
+      const float u = us[t];
+#pragma unroll
+      for (int i = 0; i < NJ / 2; ++i) {
+        const int j = jh * (NJ / 2) + i;
+        *reinterpret_cast<float*>(sm + Cf::B2 + tc::sw128_off(j, t, NJ, 4)) = u * KE[t * Cf::KES + j];
+      }
+    }
+    tc::fence_proxy_async();
+    tc::tc_before_sync();
+    __syncthreads();
+    tc::tc_after_sync();
+    // ---- MMA 2: dS_c = V^T B2  (M=128 rows r, N=NJ, K=64)
+    if (tid == 0) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = tc::desc_sw128(tc::smem_u32(sm + Cf::A2 + (ks / 4) * 128 * 128 + (ks % 4) * 32));
+        const uint64_t bd = tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + (ks / 4) * NJ * 128 + (ks % 4) * 32));
+        tc::mma_tf32_ss(tmem + Cf::D2_COL, ad, bd, ID2, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&mma_bar);
+    }
+    tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
+    mma_par ^= 1;
+    tc::tc_after_sync();
+    // ---- S <- S diag(gamma_C) + dS  (in tensor memory)
+#pragma unroll
+    for (int jj = 0; jj < NJ; jj += 16) {
+      float s[16], d[16];
+      tc::tmem_ld16(my_lanes + Cf::S_COL + jj, s);
+      tc::tmem_ld16(my_lanes + Cf::D2_COL + jj, d);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], d[i]);
+      tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
+    }
+    tc::tmem_st_wait();
+    tc::tc_before_sync();
+    __syncthreads();
+    tc::tc_after_sync();
+  }
+
+  if (ST) {
+    const int r = tid;
+#pragma unroll
+    for (int jj = 0; jj < NJ; jj += 16) {
+      float x[16];
+      tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ST[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] = x[i];
+    }
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::cluster_sync();  // no peer may still write into this CTA's shared memory
+  if (warp == 0) tc::tmem_dealloc(tmem, Cf::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// output kernel: O^T[r,t] = sum_j S0[r,j] Q+[t,j] + sum_i V[i,r] u_i P[t,i]
+// ---------------------------------------------------------------------------
+struct OutCfg {
+  static constexpr uint32_t S0 = 0;                     // S0 blob, tf32 SW128 [4 kb][128][128 B]
+  static constexpr uint32_t QK = S0 + 65536;            // [Q+ ; 0] tf32 SW128 [4 kb][128][128 B]
+  static constexpr uint32_t KM = QK + 65536;            // K- tf32 SW128 [4 kb][64][128 B]
+  static constexpr uint32_t VT = KM + 32768;            // V^T tf32 SW128 [2 kb][128][128 B]
+  static constexpr uint32_t B3 = VT + 32768;            // diag(u) P^T: tf32 SW128 [2 kb][64][128 B]
+  static constexpr uint32_t U = B3 + 16384;             // u [64]
+  static constexpr uint32_t END = U + 256;
+  static constexpr uint32_t BYTES = END + 1024;
+};
+
+__global__ void __launch_bounds__(128, 1) fwd_out_tc(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, const float* __restrict__ logf, int H, int T, int NC,
+    const float* __restrict__ wS0blob, const float* __restrict__ wu, __nv_bfloat16* __restrict__ out,
+    int* __restrict__ unsafe_flags, int* __restrict__ err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar, mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int unsafe, abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = (size_t)unit * NC + n;
+
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    unsafe = 0;
+    abort_flag = 0;
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 0) {
+    tc::mbar_expect_tx(&ld_bar, 65536u);
+#pragma unroll
+    for (int part = 0; part < 4; ++part)
+      tc::bulk_g2s(sm + OutCfg::S0 + part * 16384, wS0blob + ch * D * D + part * 4096, 16384u, &ld_bar);
+  }
+  float* us = reinterpret_cast<float*>(sm + OutCfg::U);
+  if (tid < C) us[tid] = wu[ch * C + tid];
+
+  // Q+ = q o gamma and K- = k / gamma (thread = key channel j); rows 64..127 of QK are zero
+  {
+    const int j = tid;
+    float L = 0.f, mx = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < C; ++t) {
+      const bool ok = t < nv;
+      const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
+      L += ok ? logf[g] : 0.f;
+      mx = fmaxf(mx, fabsf(L));
+      const float qq = ok ? __bfloat162float(q[g]) : 0.f, kk = ok ? __bfloat162float(k[g]) : 0.f;
+      *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = qq * expf(L);
+      *reinterpret_cast<float*>(sm + OutCfg::KM + tc::sw128_off(t, j, 64, 4)) = kk * expf(-L);
+    }
+    if (!(mx < kSafeLogRange)) atomicOr(&unsafe, 1);
+#pragma unroll 4
+    for (int t = 64; t < 128; ++t) *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = 0.f;
+  }
+  // V^T (tf32): thread = position t (two halves of r)
+  {
+    const int t = tid & 63, rh = tid >> 6;
+    const bool ok = t < nv;
+    const __nv_bfloat16* vrow = v + (((size_t)b * T + t0 + t) * H + h) * D;
+#pragma unroll 2
+    for (int r8 = 0; r8 < 64; r8 += 8) {
+      uint4 raw = make_uint4(0, 0, 0, 0);
+      if (ok) raw = *reinterpret_cast<const uint4*>(vrow + 64 * rh + r8);
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float*>(sm + OutCfg::VT + tc::sw128_off(64 * rh + r8 + i, t, 128, 4)) =
+            __bfloat162float(e[i]);
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const bool is_unsafe = unsafe != 0;
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  // MMA: D_P[t,i] (cols 0..63) = [Q+;0] K-^T ; D_O[r,t] (cols 64..127) = S0 Q+^T
+  if (tid == 0) {
+    const uint32_t IDP = tc::idesc(128, 64, 2);
+#pragma unroll
+    for (int ks = 0; ks < 16; ++ks) {
+      const uint32_t kb = ks / 4, within = (ks % 4) * 32;
+      const uint64_t qa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::QK + kb * 128 * 128 + within));
+      const uint64_t kmb = tc::desc_sw128(tc::smem_u32(sm + OutCfg::KM + kb * 64 * 128 + within));
+      const uint64_t sa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::S0 + kb * 128 * 128 + within));
+      tc::mma_tf32_ss(tmem + 0, qa, kmb, IDP, ks > 0 ? 1u : 0u);
+      tc::mma_tf32_ss(tmem + 64, sa, qa, IDP, ks > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  // B3[t][i] = u_i P[t,i] for i <= t (rows t: warps 0-1 own TMEM lanes 0..63)
+  if (warp < 2) {
+    const int t = tid;
+#pragma unroll
+    for (int c16 = 0; c16 < 4; ++c16) {
+      float x[16];
+      tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, 16 * c16), x);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) {
+        const int i = 16 * c16 + i2;
+        const float pv = (i <= t && !is_unsafe) ? x[i2] * us[i] : 0.f;
+        *reinterpret_cast<float*>(sm + OutCfg::B3 + tc::sw128_off(t, i, 64, 4)) = pv;
+      }
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    const uint32_t IDO = tc::idesc(128, 64, 2);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t kb = ks / 4, within = (ks % 4) * 32;
+      const uint64_t va = tc::desc_sw128(tc::smem_u32(sm + OutCfg::VT + kb * 128 * 128 + within));
+      const uint64_t pb = tc::desc_sw128(tc::smem_u32(sm + OutCfg::B3 + kb * 64 * 128 + within));
+      tc::mma_tf32_ss(tmem + 64, va, pb, IDO, 1u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  tc::mbar_wait<false>(&mma_bar, 1, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  // O[t, r] from D_O lane r
+  {
+    const int r = tid;
+#pragma unroll
+    for (int c16 = 0; c16 < 4; ++c16) {
+      float x[16];
+      tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, 64 + 16 * c16), x);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * c16 + i;
+        if (t < nv) out[(((size_t)b * T + t0 + t) * H + h) * D + r] = __float2bfloat16_rn(x[i]);
+      }
+    }
+  }
+  if (tid == 0 && unsafe_flags) unsafe_flags[ch] = is_unsafe ? 1 : 0;
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
+// Exact recomputation of O for chunks whose decay range is outside the
+// factorised form's fp32 range (flagged by fwd_out_tc): per-element decays.
+__global__ void __launch_bounds__(128) fwd_out_fixup(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, const float* __restrict__ logf, int H, int T, int NC,
+    const float* __restrict__ wS0blob, const float* __restrict__ wu, const int* __restrict__ unsafe_flags,
+    __nv_bfloat16* __restrict__ out) {
+  const size_t ch = blockIdx.x;
+  if (unsafe_flags[ch] == 0) return;
+  extern __shared__ float fx[];
+  float (*Ls)[D + 1] = reinterpret_cast<float (*)[D + 1]>(fx);
+  float (*qs)[D + 1] = reinterpret_cast<float (*)[D + 1]>(fx + C * (D + 1));
+  float (*ks)[D + 1] = reinterpret_cast<float (*)[D + 1]>(fx + 2 * C * (D + 1));
+  float* us = fx + 3 * C * (D + 1);
+  const int tid = threadIdx.x;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  for (int e = tid; e < C * D; e += 128) {
+    const int t = e / D, j = e % D;
+    const bool ok = t < nv;
+    const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
+    Ls[t][j] = ok ? logf[g] : 0.f;
+    qs[t][j] = ok ? __bfloat162float(q[g]) : 0.f;
+    ks[t][j] = ok ? __bfloat162float(k[g]) : 0.f;
+  }
+  if (tid < C) us[tid] = wu[ch * C + tid];
+  __syncthreads();
+  {
+    float acc = 0.f;
+    for (int t = 0; t < C; ++t) {
+      acc += Ls[t][tid];
+      Ls[t][tid] = acc;
+    }
+  }
+  __syncthreads();
+  const unsigned char* blob = reinterpret_cast<const unsigned char*>(wS0blob + ch * D * D);
+  const int r = tid;
+  for (int t = 0; t < nv; ++t) {
+    float o = 0.f;
+    for (int j = 0; j < D; ++j)
+      o = fmaf(*reinterpret_cast<const float*>(blob + tc::sw128_off(r, j, 128, 4)), qs[t][j] * expf(Ls[t][j]), o);
+    for (int i = 0; i <= t; ++i) {
+      float p = 0.f;
+      for (int j = 0; j < D; ++j) p = fmaf(qs[t][j] * ks[i][j], expf(Ls[t][j] - Ls[i][j]), p);
+      o = fmaf(p * us[i], __bfloat162float(v[(((size_t)b * T + t0 + i) * H + h) * D + r]), o);
+    }
+    out[(((size_t)b * T + t0 + t) * H + h) * D + r] = __float2bfloat16_rn(o);
+  }
+}
+
+template <int R>
+cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, float* blob, float* wu,
+                         float* wb0, int* err, cudaStream_t st) {
+  const Layout& L = a.L;
+  cudaError_t e = cudaFuncSetAttribute(fwd_chain_tc<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ChainCfg<R>::BYTES);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(L.B * L.H * R);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = R;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  prof_begin(st, "fwd_chain_tc");
+  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, static_cast<const __nv_bfloat16*>(a.k),
+                         static_cast<const __nv_bfloat16*>(a.v), a.beta, a.logf, a.S0, a.ST, L.H, L.T,
+                         L.NC, wy, wA, blob, wu, wb0, err);
+  prof_end(st);
+  return e;
+}
+
+}  // namespace
+
+int choose_cluster(int units, int sms) {
+  if (units * 8 <= sms) return 8;
+  if (units * 4 <= sms) return 4;
+  return 2;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) {
+  const Layout& L = a.L;
+  cudaError_t e = launch_fwd_prep(a, /*with_P=*/a.save != 0, st);
+  if (e != cudaSuccess) return e;
+  const float* wy = ws_ptr<float>(a.ws, L.y);
+  const float* wA = ws_ptr<float>(a.ws, L.A);
+  float* blob = ws_ptr<float>(a.ws, L.S0);
+  float* wu = ws_ptr<float>(a.ws, L.u);
+  float* wb0 = ws_ptr<float>(a.ws, L.b0);
+  int* flags = ws_ptr<int>(a.ws, L.flags);
+  const int R = choose_cluster(L.B * L.H, sms);
+  if (R == 8) e = launch_chain<8>(a, wy, wA, blob, wu, wb0, err, st);
+  else if (R == 4) e = launch_chain<4>(a, wy, wA, blob, wu, wb0, err, st);
+  else e = launch_chain<2>(a, wy, wA, blob, wu, wb0, err, st);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(fwd_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)OutCfg::BYTES)) != cudaSuccess)
+    return e;
+  prof_begin(st, "fwd_out_tc");
+  fwd_out_tc<<<(unsigned)L.chunks, 128, OutCfg::BYTES, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), a.logf, L.H, L.T, L.NC, blob, wu,
+      static_cast<__nv_bfloat16*>(a.out), flags, err);
+  prof_end(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  constexpr int kFixSmem = (3 * C * (D + 1) + C) * 4;
+  if ((e = cudaFuncSetAttribute(fwd_out_fixup, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem)) !=
+      cudaSuccess)
+    return e;
+  prof_begin(st, "fwd_out_fixup");
+  fwd_out_fixup<<<(unsigned)L.chunks, 128, kFixSmem, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), a.logf, L.H, L.T, L.NC, blob, wu, flags,
+      static_cast<__nv_bfloat16*>(a.out));
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+}  // namespace kd

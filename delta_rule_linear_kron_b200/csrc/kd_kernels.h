@@ -18,13 +18,17 @@ constexpr int kChunk = 64;
 // "chunk" index ch = ((b * H) + h) * NC + n.
 struct Layout {
   int B = 0, H = 0, T = 0, dk = 0, dv = 0, dtype = 0;
+  // true: the tensor-core path (bf16, dk = dv = 128).  Its saved chunk-start
+  // states are 128-byte-swizzled K-major tf32 tiles (see kd_fwd_tc.cu), and
+  // its forward scratch always holds them.
+  bool tc = false;
   int NC = 0;             // ceil(T / 64)
   size_t chunks = 0;      // B * H * NC
   // forward scratch (always): y [ch][64], A [ch][64][64], P [ch][64][64]
   size_t y = 0, A = 0, P = 0;
   size_t fwd_bytes = 0;
   // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
-  size_t S0 = 0, u = 0, b0 = 0;
+  size_t S0 = 0, u = 0, b0 = 0, flags = 0;  // flags: one int per chunk (tensor-core path)
   size_t fwd_save_bytes = 0;
   // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],
   // accq/acck/accL [ch][64][dk], accv [ch][64][dv]
@@ -71,6 +75,10 @@ void prof_end(cudaStream_t st);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_fwd_prep(const FwdArgs& a, bool with_P, cudaStream_t st);
+// err: the library's device error word; sms: multiprocessors of the device.
+cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st);
+int choose_cluster(int units, int sms);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st);
 
 template <typename T>

@@ -47,9 +47,13 @@ def test_workspace_sizes(L):
     fs = kd.workspace_size(kd.KD_WS_FWD_SAVE, B, H, T, d, d)
     bw = kd.workspace_size(kd.KD_WS_BWD, B, H, T, d, d)
     chunks = B * H * (T // 64)
-    assert f >= chunks * (64 + 2 * 64 * 64) * 4
-    assert fs >= f + chunks * d * d * 4
+    assert f >= chunks * (64 + 64 * 64) * 4                      # y, A
+    assert fs >= chunks * (64 + 2 * 64 * 64 + d * d + 2 * 64) * 4  # + P, chunk-start states, u, b0
+    assert fs >= f
     assert bw >= chunks * d * d * 4
+    # the fp32 path keeps the chunk-start states only when saving for the backward
+    f32 = kd.workspace_size(kd.KD_WS_FWD, B, H, T, d, d, kd.KD_F32)
+    assert kd.workspace_size(kd.KD_WS_FWD_SAVE, B, H, T, d, d, kd.KD_F32) >= f32 + chunks * d * d * 4
     # ragged T rounds the chunk count up
     assert kd.workspace_size(kd.KD_WS_FWD, 1, 1, 65, 32, 32) > kd.workspace_size(kd.KD_WS_FWD, 1, 1, 64, 32, 32)
     assert L.kron_delta_workspace_size(0, 1, 1, 64, 48, 32, 1) == 0
