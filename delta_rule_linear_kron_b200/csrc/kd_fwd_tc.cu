@@ -31,6 +31,7 @@
 #include "kd_common.cuh"
 #include "kd_kernels.h"
 #include "kd_tc.cuh"
+#include "kd_tmap.h"
 
 namespace kd {
 namespace {
@@ -41,44 +42,65 @@ constexpr int D = 128;
 template <int R>
 struct ChainCfg {
   static constexpr int NJ = D / R;                    // key channels per CTA
-  static constexpr int KB1 = (NJ * 4 + 127) / 128;    // 128-byte K blocks of K+ slice
-  static constexpr int TPC = 128 / NJ;                // scan threads per channel
+  static constexpr int KB1 = (NJ * 4 + 127) / 128;    // 128-byte K blocks of the K+ slice
+  static constexpr int TPC = 128 / NJ;                // producer scan threads per channel
   static constexpr int SEG = C / TPC;                 // positions per scan thread
-  static constexpr int D1_COL = 0, S_COL = 64, D2_COL = 64 + NJ;
-  static constexpr uint32_t TMEM_COLS = (64 + 2 * NJ) <= 128 ? 128u : 256u;
   static constexpr int KES = NJ + 1;                  // padded row of K^e (fp32)
-  // shared memory map (bytes from a 1024-aligned base)
-  static constexpr uint32_t B1 = 0;                                   // K+ slice, tf32 SW128, 64 rows
-  static constexpr uint32_t A2 = B1 + KB1 * 64 * 128;                  // V^T, tf32 SW128, 128 rows, K=64
-  static constexpr uint32_t B2 = A2 + 2 * 128 * 128;                   // diag(u) K^e slice, NJ rows, K=64
-  static constexpr uint32_t KE = B2 + 2 * NJ * 128;                    // K^e fp32 [64][KES]
-  static constexpr uint32_t STG = ((KE + 64 * KES * 4) + 127) / 128 * 128;
-  // staging buffer (one per chunk parity), offsets inside it
-  static constexpr uint32_t VROW = 272;                                // 256 B of bf16 v + 16 B pad
-  static constexpr uint32_t ST_V = 0, ST_A = ST_V + 64 * VROW, ST_Y = ST_A + 64 * 64 * 4,
-                            ST_K = ST_Y + 256, ST_L = ST_K + 64 * NJ * 2;
-  static constexpr uint32_t ST_SZ = ((ST_L + 64 * NJ * 4) + 127) / 128 * 128;
-  static constexpr uint32_t SM = STG + 2 * ST_SZ;                      // small arrays (floats)
-  static constexpr uint32_t SM_BS = SM;                                // beta [2][64]
-  static constexpr uint32_t SM_W = SM_BS + 2 * 64 * 4;                 // beta o b0 [64]
-  static constexpr uint32_t SM_U = SM_W + 64 * 4;                      // u [64]
-  static constexpr uint32_t SM_MINE = SM_U + 64 * 4;                   // own b0 partial [64]
-  static constexpr uint32_t SM_XRED = SM_MINE + 64 * 4;                // per-warp partials [4][64]
-  static constexpr uint32_t SM_RECV = SM_XRED + 4 * 64 * 4;            // [2][R][64]
-  static constexpr uint32_t SM_GC = SM_RECV + 2 * R * 64 * 4;          // gamma_C [NJ]
-  static constexpr uint32_t SM_SEG = SM_GC + NJ * 4;                   // scan segment sums [TPC][NJ]
+  // tensor memory columns: X (64), state slice, two halves of the update
+  static constexpr int D1_COL = 0, S_COL = 64, D2A_COL = 64 + NJ, D2B_COL = 64 + 2 * NJ;
+  static constexpr uint32_t TMEM_COLS = (64 + 3 * NJ) <= 128 ? 128u : 256u;
+  static constexpr uint32_t up1k(uint32_t x) { return (x + 1023u) / 1024u * 1024u; }
+  // operand buffer (two, by chunk parity), built by the producer warps
+  static constexpr uint32_t OP_B1 = 0;                         // K+ slice: tf32 SW128, 64 rows
+  static constexpr uint32_t OP_A2 = OP_B1 + KB1 * 8192;        // V^T: tf32 SW128, 128 rows, K = 64
+  static constexpr uint32_t OP_KE = OP_A2 + 32768;             // K^e slice fp32 [64][KES]
+  static constexpr uint32_t OP_GC = OP_KE + 64 * KES * 4;      // gamma_C slice [NJ]
+  static constexpr uint32_t OP_SZ = up1k(OP_GC + NJ * 4);
+  // raw staging (two, by chunk parity), written by TMA / bulk copies
+  static constexpr uint32_t ST_V = 0;                          // v bf16 [64][128]
+  static constexpr uint32_t ST_A = 16384;                      // A fp32 [64][64]
+  static constexpr uint32_t ST_Y = 32768;                      // y [64]
+  static constexpr uint32_t ST_K = ST_Y + 256;                 // k slice bf16 [64][NJ]
+  static constexpr uint32_t ST_L = ST_K + 64 * NJ * 2;         // logf slice fp32 [64][NJ]
+  static constexpr uint32_t ST_SZ = up1k(ST_L + 64 * NJ * 4);
+  static constexpr uint32_t LOAD_BYTES = 16384 + 16384 + 256 + 64 * NJ * 6;
+  static constexpr uint32_t OPS = 0, STG = OPS + 2 * OP_SZ;
+  static constexpr uint32_t B2 = STG + 2 * ST_SZ;              // diag(u) K^e: tf32 SW128, NJ rows, K = 64
+  static constexpr uint32_t SM = B2 + 2 * NJ * 128;            // small arrays (floats)
+  static constexpr uint32_t SM_BS = SM;                        // beta [2][64]
+  static constexpr uint32_t SM_W = SM_BS + 2 * 64 * 4;         // beta o b0 [64]
+  static constexpr uint32_t SM_U = SM_W + 64 * 4;              // u [64]
+  static constexpr uint32_t SM_UP = SM_U + 64 * 4;             // u partial sums [2][64]
+  static constexpr uint32_t SM_MINE = SM_UP + 2 * 64 * 4;      // own b0 partial [64]
+  static constexpr uint32_t SM_XRED = SM_MINE + 64 * 4;        // per-warp partials [4][64]
+  static constexpr uint32_t SM_RECV = SM_XRED + 4 * 64 * 4;    // [2][R][64]
+  static constexpr uint32_t SM_SEG = SM_RECV + 2 * R * 64 * 4; // scan segment sums [TPC][NJ]
   static constexpr uint32_t SM_END = SM_SEG + TPC * NJ * 4;
-  static constexpr uint32_t BYTES = SM_END + 1024;                     // + alignment slack
+  static constexpr uint32_t BYTES = SM_END + 1024;             // + alignment slack
 };
 
-__device__ __forceinline__ float bf2f(const unsigned char* p) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+// named barriers: 1 = the 4 chain warps, 2 = the 4 producer warps
+__device__ __forceinline__ void bar_chain() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_prod() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(b)) : "memory");
 }
 
+// Warp roles (256 threads):
+//   warps 0-3  chain: MMAs, the b0 column sums, the cluster all-reduce, u,
+//              the state update; thread r owns tensor-memory lane r.
+//   warps 4-7  producer: issues the TMA / bulk loads, builds the next chunk's
+//              MMA operands (decay prefix, K+, K^e, V^T), saves each
+//              chunk-start state slice to global memory.
+// Hand-offs (mbarriers, one arrival each): raw_full (loads landed),
+// op_full (operands of a chunk built), free (chain done with a chunk's
+// buffers), s_ready (state of chunk n in tensor memory), s_saved (producer
+// has read it).
 template <int R>
-__global__ void __launch_bounds__(128, 1) fwd_chain_tc(
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-    const float* __restrict__ beta, const float* __restrict__ logf, const float* __restrict__ S0,
+__global__ void __launch_bounds__(256, 1) fwd_chain_tc(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const __grid_constant__ CUtensorMap tm_logf,
+    const float* __restrict__ beta, const float* __restrict__ S0,
     float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy,
     const float* __restrict__ wA, float* __restrict__ wS0blob, float* __restrict__ wu,
     float* __restrict__ wb0, int* __restrict__ err) {
@@ -86,31 +108,34 @@ __global__ void __launch_bounds__(128, 1) fwd_chain_tc(
   constexpr int NJ = Cf::NJ;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ uint64_t ld_bar[2], x_bar[2], mma_bar;
+  __shared__ uint64_t raw_full[2], op_full[2], freeb[2], s_ready, s_saved, x_bar[2], mma_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = tc::cluster_rank();
-  const int unit = blockIdx.x / R;        // (b, h)
+  const int unit = blockIdx.x / R;  // (b, h)
   const int b = unit / H, h = unit % H;
-  const int j0 = static_cast<int>(rank) * NJ;  // first key channel of this CTA
+  const int j0 = static_cast<int>(rank) * NJ;
 
   float* bs = reinterpret_cast<float*>(sm + Cf::SM_BS);
   float* ws = reinterpret_cast<float*>(sm + Cf::SM_W);
   float* us = reinterpret_cast<float*>(sm + Cf::SM_U);
+  float* up = reinterpret_cast<float*>(sm + Cf::SM_UP);
   float* mine = reinterpret_cast<float*>(sm + Cf::SM_MINE);
   float* xred = reinterpret_cast<float*>(sm + Cf::SM_XRED);
   float* recv = reinterpret_cast<float*>(sm + Cf::SM_RECV);
-  float* gC = reinterpret_cast<float*>(sm + Cf::SM_GC);
   float* segs = reinterpret_cast<float*>(sm + Cf::SM_SEG);
-  float* KE = reinterpret_cast<float*>(sm + Cf::KE);
 
   if (tid == 0) {
-    tc::mbar_init(&ld_bar[0], 1);
-    tc::mbar_init(&ld_bar[1], 1);
-    tc::mbar_init(&x_bar[0], 1);
-    tc::mbar_init(&x_bar[1], 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&raw_full[i], 1);
+      tc::mbar_init(&op_full[i], 1);
+      tc::mbar_init(&freeb[i], 1);
+      tc::mbar_init(&x_bar[i], 1);
+    }
+    tc::mbar_init(&s_ready, 1);
+    tc::mbar_init(&s_saved, 1);
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
@@ -118,273 +143,286 @@ __global__ void __launch_bounds__(128, 1) fwd_chain_tc(
   if (warp == 0) tc::tmem_alloc(&tmem_slot, Cf::TMEM_COLS);
   tc::tc_before_sync();
   __syncthreads();
+  tc::cluster_sync();  // peers' barriers are initialised before any remote arrive
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
-  const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);  // this warp's 32 TMEM lanes
+  const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);  // lanes 32*(warp%4) ..
 
-  // initial state slice -> TMEM (thread = state row r)
-  {
-    const int r = tid;
-#pragma unroll
-    for (int jj = 0; jj < NJ; jj += 16) {
-      float x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        x[i] = S0 ? S0[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] : 0.f;
-      tc::tmem_st16(my_lanes + Cf::S_COL + jj, x);
-    }
-    tc::tmem_st_wait();
-  }
-
-  // issue the bulk copies of chunk n into staging buffer n & 1
-  auto issue_loads = [&](int n) {
-    unsigned char* st = sm + Cf::STG + (n & 1) * Cf::ST_SZ;
-    uint64_t* bar = &ld_bar[n & 1];
-    const int t0 = n * C, nv = min(C, T - t0);
-    const size_t ch = (size_t)unit * NC + n;
-    tc::fence_proxy_async();
-    if (tid == 64) {
-      tc::mbar_expect_tx(bar, (uint32_t)nv * (256u + NJ * 6u) + 64u * 64u * 4u + 256u);
+  if (warp >= 4) {
+    // =========================== producer warps ===========================
+    const int p = tid - 128;
+    auto issue = [&](int n) {
+      unsigned char* st = sm + Cf::STG + (n & 1) * Cf::ST_SZ;
+      uint64_t* bar = &raw_full[n & 1];
+      const size_t ch = (size_t)unit * NC + n;
+      tc::fence_proxy_async();
+      tc::mbar_expect_tx(bar, Cf::LOAD_BYTES);
+      tc::tma_load_4d(st + Cf::ST_V, &tm_v, 0, h, n * C, b, bar);
+      tc::tma_load_4d(st + Cf::ST_K, &tm_k, j0, h, n * C, b, bar);
+      tc::tma_load_4d(st + Cf::ST_L, &tm_logf, j0, h, n * C, b, bar);
       tc::bulk_g2s(st + Cf::ST_A, wA + ch * C * C, 64u * 64u * 4u, bar);
       tc::bulk_g2s(st + Cf::ST_Y, wy + ch * C, 256u, bar);
+    };
+    if (p == 0) {
+      issue(0);
+      if (NC > 1) issue(1);
     }
-    if (tid < C) {
-      const int t = tid;
-      if (t < nv) {
-        const size_t row = ((size_t)b * T + t0 + t) * H + h;
-        tc::bulk_g2s(st + Cf::ST_V + t * Cf::VROW, v + row * D, 256u, bar);
-        tc::bulk_g2s(st + Cf::ST_K + t * NJ * 2, k + row * D + j0, NJ * 2u, bar);
-        tc::bulk_g2s(st + Cf::ST_L + t * NJ * 4, logf + row * D + j0, NJ * 4u, bar);
-      } else {  // rows past T are zero
-        uint4 z = make_uint4(0, 0, 0, 0);
-        for (int i = 0; i < 16; ++i) reinterpret_cast<uint4*>(st + Cf::ST_V + t * Cf::VROW)[i] = z;
-        for (int i = 0; i < NJ * 2 / 16; ++i) reinterpret_cast<uint4*>(st + Cf::ST_K + t * NJ * 2)[i] = z;
-        for (int i = 0; i < NJ * 4 / 16; ++i) reinterpret_cast<uint4*>(st + Cf::ST_L + t * NJ * 4)[i] = z;
+    for (int n = 0; n < NC; ++n) {
+      const int pb = n & 1;
+      unsigned char* st = sm + Cf::STG + pb * Cf::ST_SZ;
+      unsigned char* op = sm + Cf::OPS + pb * Cf::OP_SZ;
+      if (n >= 2) {
+        // the chain has finished chunk n-2: both buffers of this parity are free
+        tc::mbar_wait<false>(&freeb[pb], (uint32_t)(((n - 2) >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
+        if (p == 0) issue(n);
       }
-    }
-  };
-  auto load_beta = [&](int n) -> float {
-    const int t0 = n * C;
-    return (tid < C && t0 + tid < T) ? beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
-  };
-
-  issue_loads(0);
-  float beta_next = load_beta(0);
-  int mma_par = 0;
-  const uint32_t ID1 = tc::idesc(128, 64, 2);
-  const uint32_t ID2 = tc::idesc(128, NJ, 2);
-
-  for (int n = 0; n < NC; ++n) {
-    const int buf = n & 1;
-    unsigned char* st = sm + Cf::STG + buf * Cf::ST_SZ;
-    const size_t ch = (size_t)unit * NC + n;
-    if (tid < C) bs[buf * 64 + tid] = beta_next;
-    tc::mbar_wait<false>(&ld_bar[buf], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
-    __syncthreads();  // staging of chunk n visible to all; buffer n+1 free
-    if (n + 1 < NC) {
-      issue_loads(n + 1);
-      beta_next = load_beta(n + 1);
-    }
-
-    // ---- chunk set-up: V^T (tf32, swizzled); decay prefix; K+ and K^e
-    {
-      const int t = tid & 63, rh = tid >> 6;  // rows r in [64 rh, 64 rh + 64)
-      const unsigned char* vrow = st + Cf::ST_V + t * Cf::VROW;
+      const float bt = (p < C && n * C + p < T) ? beta[((size_t)b * T + n * C + p) * H + h] : 0.f;
+      tc::mbar_wait<false>(&raw_full[pb], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      if (p < C) bs[pb * 64 + p] = bt;
+      // V^T as tf32 (thread = position t, half of the value channels)
+      {
+        const int t = p & 63, rh = p >> 6;
 #pragma unroll 2
-      for (int r8 = 0; r8 < 64; r8 += 8) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(vrow + (64 * rh + r8) * 2);
-        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+        for (int r8 = 0; r8 < 64; r8 += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(st + Cf::ST_V + t * 256 + (64 * rh + r8) * 2);
+          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = 64 * rh + r8 + i;
-          *reinterpret_cast<float*>(sm + Cf::A2 + tc::sw128_off(r, t, 128, 4)) = __bfloat162float(e[i]);
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<float*>(op + Cf::OP_A2 + tc::sw128_off(64 * rh + r8 + i, t, 128, 4)) =
+                __bfloat162float(e[i]);
         }
       }
+      // decay prefix of the slice, K+ (B operand of MMA 1), K^e, gamma_C
+      {
+        const int j = p % NJ, seg = p / NJ;
+        const float* lrow = reinterpret_cast<const float*>(st + Cf::ST_L);
+        float lp[Cf::SEG];
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < Cf::SEG; ++i) {
+          acc += lrow[(seg * Cf::SEG + i) * NJ + j];
+          lp[i] = acc;
+        }
+        segs[seg * NJ + j] = acc;
+        bar_prod();
+        float pre = 0.f, tot = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < Cf::TPC; ++s2) {
+          const float x = segs[s2 * NJ + j];
+          if (s2 < seg) pre += x;
+          tot += x;
+        }
+        float* KE = reinterpret_cast<float*>(op + Cf::OP_KE);
+        if (seg == 0) reinterpret_cast<float*>(op + Cf::OP_GC)[j] = expf(tot);
+#pragma unroll
+        for (int i = 0; i < Cf::SEG; ++i) {
+          const int t = seg * Cf::SEG + i;
+          const float L = pre + lp[i];
+          const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(st + Cf::ST_K + (t * NJ + j) * 2));
+          *reinterpret_cast<float*>(op + Cf::OP_B1 + tc::sw128_off(t, j, 64, 4)) = kk * expf(L);
+          KE[t * Cf::KES + j] = kk * expf(tot - L);
+        }
+      }
+      tc::fence_proxy_async();
+      bar_prod();
+      if (p == 0) mbar_arrive(&op_full[pb]);
+      // save the chunk-start state slice once the chain has it in tensor memory
+      tc::mbar_wait<false>(&s_ready, (uint32_t)(n & 1), err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      {
+        float* blob = wS0blob + ((size_t)unit * NC + n) * D * D;
+        const int r = p;
+#pragma unroll
+        for (int jj = 0; jj < NJ; jj += 16) {
+          float x[16];
+          tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int jg = j0 + jj + 4 * q4;
+            *reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(blob) + tc::sw128_off(r, jg, 128, 4)) =
+                make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+          }
+        }
+      }
+      tc::tc_before_sync();
+      bar_prod();
+      if (p == 0) mbar_arrive(&s_saved);
     }
+  } else {
+    // ============================= chain warps ============================
+    const int r = tid;  // tensor-memory lane = state row
     {
-      const int j = tid % NJ, seg = tid / NJ;
-      const float* lrow = reinterpret_cast<const float*>(st + Cf::ST_L);
-      float lp[Cf::SEG];
-      float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < Cf::SEG; ++i) {
-        acc += lrow[(seg * Cf::SEG + i) * NJ + j];
-        lp[i] = acc;
+      for (int jj = 0; jj < NJ; jj += 16) {
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = S0 ? S0[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] : 0.f;
+        tc::tmem_st16(my_lanes + Cf::S_COL + jj, x);
       }
-      segs[seg * NJ + j] = acc;
-      __syncthreads();
-      float pre = 0.f, tot = 0.f;
+      tc::tmem_st_wait();
+      tc::tc_before_sync();
+      bar_chain();
+      if (tid == 0) mbar_arrive(&s_ready);
+    }
+    int mma_par = 0;
+    const uint32_t ID1 = tc::idesc(128, 64, 2);
+    const uint32_t ID2 = tc::idesc(128, NJ, 2);
+    for (int n = 0; n < NC; ++n) {
+      const int pb = n & 1;
+      const unsigned char* st = sm + Cf::STG + pb * Cf::ST_SZ;
+      const unsigned char* op = sm + Cf::OPS + pb * Cf::OP_SZ;
+      const size_t ch = (size_t)unit * NC + n;
+      tc::mbar_wait<false>(&op_full[pb], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      tc::tc_after_sync();
+      // ---- MMA 1: X_c = S[:,J_c] K+[:,J_c]^T  (M=128 rows r, N=64 positions, K=NJ)
+      if (tid == 0) {
 #pragma unroll
-      for (int s2 = 0; s2 < Cf::TPC; ++s2) {
-        const float x = segs[s2 * NJ + j];
-        if (s2 < seg) pre += x;
-        tot += x;
+        for (int ks = 0; ks < NJ / 8; ++ks) {
+          const uint64_t bd = tc::desc_sw128(tc::smem_u32(op + Cf::OP_B1 + (ks / 4) * 8192 + (ks % 4) * 32));
+          tc::mma_tf32_ts(tmem + Cf::D1_COL, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&mma_bar);
       }
-      if (seg == 0) gC[j] = expf(tot);
+      tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
+      mma_par ^= 1;
+      tc::tc_after_sync();
+      // ---- b0_c[t] = sum_r V[t,r] X_c[r,t]
+      {
+        float x[64];
 #pragma unroll
-      for (int i = 0; i < Cf::SEG; ++i) {
-        const int t = seg * Cf::SEG + i;
-        const float L = pre + lp[i];
-        const float kk = bf2f(st + Cf::ST_K + (t * NJ + j) * 2);
-        *reinterpret_cast<float*>(sm + Cf::B1 + tc::sw128_off(t, j, 64, 4)) = kk * expf(L);
-        KE[t * Cf::KES + j] = kk * expf(tot - L);
+        for (int c16 = 0; c16 < 4; ++c16) {
+          float y16[16];
+          tc::tmem_ld16(my_lanes + Cf::D1_COL + 16 * c16, y16);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[16 * c16 + i] = y16[i];
+        }
+        tc::tmem_ld_wait();
+        const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(st + Cf::ST_V) + r;
+        float lo[32], hi[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          lo[t] = x[t] * __bfloat162float(vcol[t * 128]);
+          hi[t] = x[32 + t] * __bfloat162float(vcol[(32 + t) * 128]);
+        }
+        warp_transpose_reduce<32>(lo, lane);
+        warp_transpose_reduce<32>(hi, lane);
+        xred[warp * 64 + lane] = lo[0];
+        xred[warp * 64 + 32 + lane] = hi[0];
+      }
+      bar_chain();
+      if (tid < C) mine[tid] = xred[tid] + xred[64 + tid] + xred[128 + tid] + xred[192 + tid];
+      bar_chain();
+      // ---- b0 = sum over the cluster of b0_c (fixed order in every CTA)
+      {
+        float* rv = recv + pb * R * 64;
+        if (tid == 0) tc::mbar_expect_tx(&x_bar[pb], R * 64u * 4u);
+        if (tid < 16 * R) {
+          const int peer = tid / 16, q4 = tid % 16;
+          const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
+          const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
+          const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[pb]), (uint32_t)peer);
+          tc::st_async_v4(raddr, val, rbar);
+        }
+        tc::mbar_wait<true>(&x_bar[pb], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
+        if (tid < C) {
+          float s = 0.f;
+#pragma unroll
+          for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + tid];
+          ws[tid] = bs[pb * 64 + tid] * s;
+          if (rank == 0 && wb0) wb0[ch * C + tid] = s;
+        }
+      }
+      bar_chain();
+      // ---- u = y - A (beta o b0): two threads per position, rotated reads
+      {
+        const int t = tid & 63, half = tid >> 6;
+        const float* Arow = reinterpret_cast<const float*>(st + Cf::ST_A) + t * 64 + 32 * half;
+        const float* wh = ws + 32 * half;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const int i0 = (i + t) & 31, i1 = (i + 1 + t) & 31, i2 = (i + 2 + t) & 31, i3 = (i + 3 + t) & 31;
+          a0 = fmaf(Arow[i0], wh[i0], a0);
+          a1 = fmaf(Arow[i1], wh[i1], a1);
+          a2 = fmaf(Arow[i2], wh[i2], a2);
+          a3 = fmaf(Arow[i3], wh[i3], a3);
+        }
+        up[half * 64 + t] = (a0 + a1) + (a2 + a3);
+      }
+      bar_chain();
+      if (tid < C) {
+        const float u = reinterpret_cast<const float*>(st + Cf::ST_Y)[tid] - (up[tid] + up[64 + tid]);
+        us[tid] = u;
+        if (rank == 0 && wu) wu[ch * C + tid] = u;
+      }
+      bar_chain();
+      // ---- B2 = diag(u) K^e[:, J_c]  (N = NJ rows j, K = 64 positions)
+      {
+        const int t = tid & 63, jh = tid >> 6;
+        const float u = us[t];
+        const float* KE = reinterpret_cast<const float*>(op + Cf::OP_KE);
+#pragma unroll
+        for (int i = 0; i < NJ / 2; ++i) {
+          const int j = jh * (NJ / 2) + i;
+          *reinterpret_cast<float*>(sm + Cf::B2 + tc::sw128_off(j, t, NJ, 4)) = u * KE[t * Cf::KES + j];
+        }
+      }
+      tc::fence_proxy_async();
+      tc::tc_before_sync();
+      bar_chain();
+      tc::tc_after_sync();
+      // ---- MMA 2: dS_c = V^T B2 as two independent K halves (M=128, N=NJ)
+      if (tid == 0) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t a0 = tc::desc_sw128(tc::smem_u32(op + Cf::OP_A2 + ks * 32));
+          const uint64_t b0d = tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + ks * 32));
+          const uint64_t a1 = tc::desc_sw128(tc::smem_u32(op + Cf::OP_A2 + 128 * 128 + ks * 32));
+          const uint64_t b1d = tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + NJ * 128 + ks * 32));
+          tc::mma_tf32_ss(tmem + Cf::D2A_COL, a0, b0d, ID2, ks > 0 ? 1u : 0u);
+          tc::mma_tf32_ss(tmem + Cf::D2B_COL, a1, b1d, ID2, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&mma_bar);
+      }
+      tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
+      mma_par ^= 1;
+      // the producer must have saved this chunk's start state before it changes
+      tc::mbar_wait<false>(&s_saved, (uint32_t)(n & 1), err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      // ---- S <- S diag(gamma_C) + dS
+      {
+        const float* gC = reinterpret_cast<const float*>(op + Cf::OP_GC);
+#pragma unroll
+        for (int jj = 0; jj < NJ; jj += 16) {
+          float s[16], da[16], db[16];
+          tc::tmem_ld16(my_lanes + Cf::S_COL + jj, s);
+          tc::tmem_ld16(my_lanes + Cf::D2A_COL + jj, da);
+          tc::tmem_ld16(my_lanes + Cf::D2B_COL + jj, db);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], da[i] + db[i]);
+          tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
+        }
+        tc::tmem_st_wait();
+      }
+      tc::tc_before_sync();
+      bar_chain();
+      if (tid == 0) {
+        mbar_arrive(&freeb[pb]);
+        mbar_arrive(&s_ready);
       }
     }
-    tc::fence_proxy_async();
-    tc::tc_before_sync();
-    __syncthreads();
-    tc::tc_after_sync();
-
-    // ---- MMA 1: X_c = S[:,J_c] K+[:,J_c]^T   (M=128 rows r, N=64 positions, K=NJ)
-    if (tid == 0) {
-#pragma unroll
-      for (int ks = 0; ks < NJ / 8; ++ks) {
-        const uint64_t bd = tc::desc_sw128(tc::smem_u32(sm + Cf::B1 + (ks / 4) * 64 * 128 + (ks % 4) * 32));
-        tc::mma_tf32_ts(tmem + Cf::D1_COL, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
-      }
-      tc::mma_commit(&mma_bar);
-    }
-    tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
-    mma_par ^= 1;
-    tc::tc_after_sync();
-
-    // chunk-start state slice -> global, in the output kernel's A-operand layout
-    if (wS0blob) {
-      float* blob = wS0blob + ch * D * D;
-      const int r = tid;
+    if (ST) {
+      tc::tc_after_sync();
 #pragma unroll
       for (int jj = 0; jj < NJ; jj += 16) {
         float x[16];
         tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int jg = j0 + jj + 4 * q4;
-          *reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(blob) + tc::sw128_off(r, jg, 128, 4)) =
-              make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
-        }
+        for (int i = 0; i < 16; ++i) ST[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] = x[i];
       }
-    }
-    // b0_c[t] = sum_r V[t,r] X_c[r,t]: per-lane products, then column sums
-    {
-      const int r = tid;
-      float lo[32], hi[32];
-#pragma unroll
-      for (int c16 = 0; c16 < 4; ++c16) {
-        float x[16];
-        tc::tmem_ld16(my_lanes + Cf::D1_COL + 16 * c16, x);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = 16 * c16 + i;
-          const float pv = x[i] * bf2f(st + Cf::ST_V + t * Cf::VROW + r * 2);
-          if (t < 32) lo[t] = pv;
-          else hi[t - 32] = pv;
-        }
-      }
-      warp_transpose_reduce<32>(lo, lane);
-      warp_transpose_reduce<32>(hi, lane);
-      xred[warp * 64 + lane] = lo[0];
-      xred[warp * 64 + 32 + lane] = hi[0];
-    }
-    __syncthreads();
-    if (tid < C) mine[tid] = xred[tid] + xred[64 + tid] + xred[128 + tid] + xred[192 + tid];
-    __syncthreads();
-
-    // ---- b0 = sum over the cluster of b0_c
-    if (R > 1) {
-      float* rv = recv + buf * R * 64;
-      if (tid == 0) tc::mbar_expect_tx(&x_bar[buf], R * 64u * 4u);
-      if (tid < 16 * R) {
-        const int peer = tid / 16, q4 = tid % 16;
-        const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
-        const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
-        const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[buf]), (uint32_t)peer);
-        tc::st_async_v4(raddr, val, rbar);
-      }
-      tc::mbar_wait<true>(&x_bar[buf], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
-      if (tid < C) {
-        float s = 0.f;
-#pragma unroll
-        for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + tid];  // same order in every CTA
-        ws[tid] = bs[buf * 64 + tid] * s;
-        if (rank == 0 && wb0) wb0[ch * C + tid] = s;
-      }
-    } else {
-      if (tid < C) {
-        ws[tid] = bs[buf * 64 + tid] * mine[tid];
-        if (wb0) wb0[ch * C + tid] = mine[tid];
-      }
-    }
-    __syncthreads();
-    // ---- u = y - A (beta o b0); rotated reads keep the A rows conflict-free
-    if (tid < C) {
-      const float* Arow = reinterpret_cast<const float*>(st + Cf::ST_A) + tid * 64;
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < 64; i += 2) {
-        const int i0 = (i + tid) & 63, i1 = (i + 1 + tid) & 63;
-        s0 = fmaf(Arow[i0], ws[i0], s0);
-        s1 = fmaf(Arow[i1], ws[i1], s1);
-      }
-      const float u = reinterpret_cast<const float*>(st + Cf::ST_Y)[tid] - (s0 + s1);
-      us[tid] = u;
-      if (rank == 0 && wu) wu[ch * C + tid] = u;
-    }
-    __syncthreads();
-    // ---- B2 = diag(u) K^e[:, J_c]  (N = NJ rows j, K = 64 positions)
-    {
-      const int t = tid & 63, jh = tid >> 6;
-      const float u = us[t];
-#pragma unroll
-      for (int i = 0; i < NJ / 2; ++i) {
-        const int j = jh * (NJ / 2) + i;
-        *reinterpret_cast<float*>(sm + Cf::B2 + tc::sw128_off(j, t, NJ, 4)) = u * KE[t * Cf::KES + j];
-      }
-    }
-    tc::fence_proxy_async();
-    tc::tc_before_sync();
-    __syncthreads();
-    tc::tc_after_sync();
-    // ---- MMA 2: dS_c = V^T B2  (M=128 rows r, N=NJ, K=64)
-    if (tid == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = tc::desc_sw128(tc::smem_u32(sm + Cf::A2 + (ks / 4) * 128 * 128 + (ks % 4) * 32));
-        const uint64_t bd = tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + (ks / 4) * NJ * 128 + (ks % 4) * 32));
-        tc::mma_tf32_ss(tmem + Cf::D2_COL, ad, bd, ID2, ks > 0 ? 1u : 0u);
-      }
-      tc::mma_commit(&mma_bar);
-    }
-    tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
-    mma_par ^= 1;
-    tc::tc_after_sync();
-    // ---- S <- S diag(gamma_C) + dS  (in tensor memory)
-#pragma unroll
-    for (int jj = 0; jj < NJ; jj += 16) {
-      float s[16], d[16];
-      tc::tmem_ld16(my_lanes + Cf::S_COL + jj, s);
-      tc::tmem_ld16(my_lanes + Cf::D2_COL + jj, d);
-      tc::tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], d[i]);
-      tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
-    }
-    tc::tmem_st_wait();
-    tc::tc_before_sync();
-    __syncthreads();
-    tc::tc_after_sync();
-  }
-
-  if (ST) {
-    const int r = tid;
-#pragma unroll
-    for (int jj = 0; jj < NJ; jj += 16) {
-      float x[16];
-      tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
-      tc::tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) ST[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] = x[i];
     }
   }
   tc::tc_before_sync();
@@ -609,12 +647,18 @@ template <int R>
 cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, float* blob, float* wu,
                          float* wb0, int* err, cudaStream_t st) {
   const Layout& L = a.L;
+  constexpr int NJ = ChainCfg<R>::NJ;
+  CUtensorMap tm_k, tm_v, tm_logf;
+  if (!make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, NJ, false) ||
+      !make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, NJ, false))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_chain_tc<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)ChainCfg<R>::BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L.B * L.H * R);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -625,19 +669,44 @@ cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, flo
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(st, "fwd_chain_tc");
-  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, static_cast<const __nv_bfloat16*>(a.k),
-                         static_cast<const __nv_bfloat16*>(a.v), a.beta, a.logf, a.S0, a.ST, L.H, L.T,
-                         L.NC, wy, wA, blob, wu, wb0, err);
+  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_k, tm_v, tm_logf, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy,
+                         wA, blob, wu, wb0, err);
   prof_end(st);
   return e;
 }
 
 }  // namespace
 
+template <int R>
+static int max_active_clusters() {
+  if (cudaFuncSetAttribute(fwd_chain_tc<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)ChainCfg<R>::BYTES) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(R * 1024);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = R;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fwd_chain_tc<R>, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+// Largest cluster (8 or 4 CTAs per head) for which every head's cluster is
+// resident at once; 4 when none is.
 int choose_cluster(int units, int sms) {
-  if (units * 8 <= sms) return 8;
-  if (units * 4 <= sms) return 4;
-  return 2;
+  (void)sms;
+  static int cap8 = -1, cap4 = -1;  // per process; the library targets one GPU model
+  if (cap8 < 0) cap8 = max_active_clusters<8>();
+  if (cap4 < 0) cap4 = max_active_clusters<4>();
+  if (units <= cap8) return 8;
+  return 4;
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) {
@@ -652,8 +721,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
   int* flags = ws_ptr<int>(a.ws, L.flags);
   const int R = choose_cluster(L.B * L.H, sms);
   if (R == 8) e = launch_chain<8>(a, wy, wA, blob, wu, wb0, err, st);
-  else if (R == 4) e = launch_chain<4>(a, wy, wA, blob, wu, wb0, err, st);
-  else e = launch_chain<2>(a, wy, wA, blob, wu, wb0, err, st);
+  else e = launch_chain<4>(a, wy, wA, blob, wu, wb0, err, st);
   if (e != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(fwd_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)OutCfg::BYTES)) != cudaSuccess)
