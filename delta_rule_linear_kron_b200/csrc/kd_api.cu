@@ -78,6 +78,7 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->acck = take(chunks * C * dk * 4);
   L->accL = take(chunks * C * dk * 4);
   L->accv = take(chunks * C * dv * 4);
+  L->du = take(chunks * C * 4);
   L->bwd_bytes = off;
   return KD_OK;
 }
@@ -283,6 +284,12 @@ int kron_delta_bwd(const void* q, const void* k, const void* v, const float* bet
   (void)S0;  // the forward state at every chunk start is read from fwd_ws
   kd::BwdArgs a{q, k, v, beta, c, logf, S0, dO, dST, dq, dk, dv, dbeta, dc, dlogf, dS0,
                 static_cast<const char*>(fwd_ws), static_cast<char*>(workspace), L};
+  if (L.tc) {
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    return launched(kd::launch_bwd_tc(a, di.err, di.sms, static_cast<cudaStream_t>(stream)),
+                    "backward launch");
+  }
   return launched(kd::launch_bwd_simt(a, static_cast<cudaStream_t>(stream)), "backward launch");
 }
 

@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
 }
 
 template <int DK, int DV, typename Tin>
-static cudaError_t run_bwd(const BwdArgs& a, cudaStream_t st) {
+static cudaError_t run_bwd(const BwdArgs& a, bool chain, cudaStream_t st) {
   const Layout& L = a.L;
   const size_t s1 = bchain_smem_floats<DK, DV>() * 4, s2 = bcc_smem_floats<DK, DV>() * 4;
   const size_t s3 = bstate_smem_floats<DK, DV>() * 4, s4 = bintra_smem_floats<DK, DV>() * 4;
@@ -630,11 +630,13 @@ static cudaError_t run_bwd(const BwdArgs& a, cudaStream_t st) {
   float* waccL = ws_ptr<float>(a.ws, L.accL);
   float* waccv = ws_ptr<float>(a.ws, L.accv);
   const dim3 gridc(L.NC, L.H, L.B);
-  prof_begin(st, "bwd_chain_simt");
-  bwd_chain_simt<DK, DV, Tin><<<dim3(L.H, L.B), 2 * DV, s1, st>>>(
-      q, k, v, a.beta, a.logf, dO, a.dST, L.H, L.T, L.NC, wA, wP, a.dS0, wdSC, wg);
-  prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (chain) {  // the tensor-core path runs its own reverse chain first
+    prof_begin(st, "bwd_chain_simt");
+    bwd_chain_simt<DK, DV, Tin><<<dim3(L.H, L.B), 2 * DV, s1, st>>>(
+        q, k, v, a.beta, a.logf, dO, a.dST, L.H, L.T, L.NC, wA, wP, a.dS0, wdSC, wg);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   prof_begin(st, "bwd_cc_simt");
   bwd_cc_simt<DK, DV, Tin><<<gridc, 256, s2, st>>>(k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, wu,
                                                    wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs);
@@ -655,9 +657,9 @@ static cudaError_t run_bwd(const BwdArgs& a, cudaStream_t st) {
 }
 
 template <typename Tin>
-static cudaError_t run_bwd_t(const BwdArgs& a, cudaStream_t st) {
+static cudaError_t run_bwd_t(const BwdArgs& a, bool chain, cudaStream_t st) {
 #define KD_B(DK_, DV_) \
-  if (a.L.dk == DK_ && a.L.dv == DV_) return run_bwd<DK_, DV_, Tin>(a, st);
+  if (a.L.dk == DK_ && a.L.dv == DV_) return run_bwd<DK_, DV_, Tin>(a, chain, st);
   KD_B(32, 32) KD_B(32, 64) KD_B(32, 128)
   KD_B(64, 32) KD_B(64, 64) KD_B(64, 128)
   KD_B(128, 32) KD_B(128, 64) KD_B(128, 128)
@@ -666,7 +668,11 @@ static cudaError_t run_bwd_t(const BwdArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st) {
-  return a.L.dtype == 0 ? run_bwd_t<float>(a, st) : run_bwd_t<__nv_bfloat16>(a, st);
+  return a.L.dtype == 0 ? run_bwd_t<float>(a, true, st) : run_bwd_t<__nv_bfloat16>(a, true, st);
+}
+
+cudaError_t launch_bwd_simt_rest(const BwdArgs& a, cudaStream_t st) {
+  return a.L.dtype == 0 ? run_bwd_t<float>(a, false, st) : run_bwd_t<__nv_bfloat16>(a, false, st);
 }
 
 }  // namespace kd

@@ -33,6 +33,7 @@ struct Layout {
   // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],
   // accq/acck/accL [ch][64][dk], accv [ch][64][dv]
   size_t dSC = 0, g = 0, dP = 0, dGK = 0, dGVs = 0, accq = 0, acck = 0, accL = 0, accv = 0;
+  size_t du = 0;  // per-chunk intra-chunk part of du (tensor-core path) [ch][64]
   size_t bwd_bytes = 0;
 };
 
@@ -80,6 +81,9 @@ cudaError_t launch_fwd_prep(const FwdArgs& a, bool with_P, cudaStream_t st);
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st);
 int choose_cluster(int units, int sms);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st);
+// the per-chunk parallel part of the backward (after the reverse chain)
+cudaError_t launch_bwd_simt_rest(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
 
 template <typename T>
 inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }

@@ -46,6 +46,19 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Same for an MN-major operand in the 128-byte-swizzle layout (the layout a
+// TMA tile of [K rows][64 bf16 along MN] lands in): leading byte offset =
+// distance between 64-element MN blocks, stride byte offset = 1024 between
+// 8-row K groups.  One bf16 MMA step (K = 16) advances the start by 2048 B.
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
 // Instruction descriptor: dense, fp32 accumulator, A and B K-major.
 // fmt: 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32).
 __host__ __device__ constexpr uint32_t idesc(int M, int N, int fmt) {
