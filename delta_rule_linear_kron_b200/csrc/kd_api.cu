@@ -66,10 +66,15 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->u = take(chunks * C * 4);
   L->b0 = take(chunks * C * 4);
   L->flags = take(chunks * 4);
+  if (L->tc) {
+    L->fwd_bytes = off;  // the output kernel reads the chunk-start states
+    L->S0b = take(chunks * (size_t)dv * dk * 2);
+    L->S0bt = take(chunks * (size_t)dv * dk * 2);
+  }
   L->fwd_save_bytes = off;
-  if (L->tc) L->fwd_bytes = off;  // its output kernel reads the chunk-start states
+
   off = 0;
-  L->dSC = take(chunks * (size_t)dv * dk * 4);
+  L->dSC = L->tc ? 0 : take(chunks * (size_t)dv * dk * 4);  // the tensor-core path keeps bf16 tiles
   L->g = take(chunks * C * 4);
   L->dP = take(chunks * C * C * 4);
   L->dGK = take(chunks * C * C * 4);
@@ -79,6 +84,11 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->accL = take(chunks * C * dk * 4);
   L->accv = take(chunks * C * dv * 4);
   L->du = take(chunks * C * 4);
+  if (L->tc) {
+    L->dSCb = take(chunks * (size_t)dv * dk * 2);
+    L->dSCbt = take(chunks * (size_t)dv * dk * 2);
+    L->bflags = take(chunks * 4);
+  }
   L->bwd_bytes = off;
   return KD_OK;
 }

@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
     const float* __restrict__ wdGK, const float* __restrict__ wdGVs,
     const float* __restrict__ waccq, const float* __restrict__ wacck,
     const float* __restrict__ waccL, const float* __restrict__ waccv, Tin* __restrict__ dq,
-    Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf) {
+    Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf, const int* __restrict__ only) {
   constexpr int SK = DK + 1, SV = DV + 1, SC = C + 1;
   extern __shared__ float smem[];
   float* us = smem;            // [C]
@@ -453,6 +453,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)b * H + h) * NC + n;
+  if (only && only[ch] == 0) return;  // only the chunks flagged by the tensor-core kernel
 
   // ---- phase A: dv = accv + u o (P^T dO) + (dG_V + dG_V^T) V
   {
@@ -597,7 +598,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
 }
 
 template <int DK, int DV, typename Tin>
-static cudaError_t run_bwd(const BwdArgs& a, bool chain, cudaStream_t st) {
+static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaStream_t st) {
   const Layout& L = a.L;
   const size_t s1 = bchain_smem_floats<DK, DV>() * 4, s2 = bcc_smem_floats<DK, DV>() * 4;
   const size_t s3 = bstate_smem_floats<DK, DV>() * 4, s4 = bintra_smem_floats<DK, DV>() * 4;
@@ -630,36 +631,41 @@ static cudaError_t run_bwd(const BwdArgs& a, bool chain, cudaStream_t st) {
   float* waccL = ws_ptr<float>(a.ws, L.accL);
   float* waccv = ws_ptr<float>(a.ws, L.accv);
   const dim3 gridc(L.NC, L.H, L.B);
-  if (chain) {  // the tensor-core path runs its own reverse chain first
+  if (stages & kStageChain) {
     prof_begin(st, "bwd_chain_simt");
     bwd_chain_simt<DK, DV, Tin><<<dim3(L.H, L.B), 2 * DV, s1, st>>>(
         q, k, v, a.beta, a.logf, dO, a.dST, L.H, L.T, L.NC, wA, wP, a.dS0, wdSC, wg);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  prof_begin(st, "bwd_cc_simt");
-  bwd_cc_simt<DK, DV, Tin><<<gridc, 256, s2, st>>>(k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, wu,
-                                                   wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs);
-  prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (stages & kStageCC) {
+    prof_begin(st, "bwd_cc_simt");
+    bwd_cc_simt<DK, DV, Tin><<<gridc, 256, s2, st>>>(k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, wu,
+                                                     wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (stages & kStageState) {
   prof_begin(st, "bwd_state_simt");
   bwd_state_simt<DK, DV, Tin><<<gridc, 256, s3, st>>>(q, k, v, a.beta, a.logf, dO, L.H, L.T,
                                                       L.NC, wu, wg, wS0, wdSC, waccq, wacck,
                                                       waccL, waccv, L.tc ? 1 : 0);
   prof_end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (!(stages & kStageIntra)) return cudaSuccess;
   prof_begin(st, "bwd_intra_simt");
   bwd_intra_simt<DK, DV, Tin><<<gridc, 256, s4, st>>>(
       q, k, v, a.logf, dO, L.H, L.T, L.NC, wP, wu, wdP, wdGK, wdGVs, waccq, wacck, waccL, waccv,
-      static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf);
+      static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf, only);
   prof_end(st);
   return cudaGetLastError();
 }
 
 template <typename Tin>
-static cudaError_t run_bwd_t(const BwdArgs& a, bool chain, cudaStream_t st) {
+static cudaError_t run_bwd_t(const BwdArgs& a, int stages, const int* only, cudaStream_t st) {
 #define KD_B(DK_, DV_) \
-  if (a.L.dk == DK_ && a.L.dv == DV_) return run_bwd<DK_, DV_, Tin>(a, chain, st);
+  if (a.L.dk == DK_ && a.L.dv == DV_) return run_bwd<DK_, DV_, Tin>(a, stages, only, st);
   KD_B(32, 32) KD_B(32, 64) KD_B(32, 128)
   KD_B(64, 32) KD_B(64, 64) KD_B(64, 128)
   KD_B(128, 32) KD_B(128, 64) KD_B(128, 128)
@@ -667,12 +673,10 @@ static cudaError_t run_bwd_t(const BwdArgs& a, bool chain, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st) {
-  return a.L.dtype == 0 ? run_bwd_t<float>(a, true, st) : run_bwd_t<__nv_bfloat16>(a, true, st);
-}
+cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st) { return launch_bwd_simt_stages(a, kStageAll, nullptr, st); }
 
-cudaError_t launch_bwd_simt_rest(const BwdArgs& a, cudaStream_t st) {
-  return a.L.dtype == 0 ? run_bwd_t<float>(a, false, st) : run_bwd_t<__nv_bfloat16>(a, false, st);
+cudaError_t launch_bwd_simt_stages(const BwdArgs& a, int stages, const int* only, cudaStream_t st) {
+  return a.L.dtype == 0 ? run_bwd_t<float>(a, stages, only, st) : run_bwd_t<__nv_bfloat16>(a, stages, only, st);
 }
 
 }  // namespace kd

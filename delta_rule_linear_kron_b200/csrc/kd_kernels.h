@@ -29,11 +29,16 @@ struct Layout {
   size_t fwd_bytes = 0;
   // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
   size_t S0 = 0, u = 0, b0 = 0, flags = 0;  // flags: one int per chunk (tensor-core path)
+  // tensor-core path, saved for the backward: chunk-start states as bf16
+  // 128-byte-swizzled tiles, "[r][j]" (rows r, K = j) and "[j][r]"
+  size_t S0b = 0, S0bt = 0;
   size_t fwd_save_bytes = 0;
   // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],
   // accq/acck/accL [ch][64][dk], accv [ch][64][dv]
   size_t dSC = 0, g = 0, dP = 0, dGK = 0, dGVs = 0, accq = 0, acck = 0, accL = 0, accv = 0;
   size_t du = 0;  // per-chunk intra-chunk part of du (tensor-core path) [ch][64]
+  size_t dSCb = 0, dSCbt = 0;  // tensor-core path: dS per chunk as bf16 tiles (as S0b, S0bt)
+  size_t bflags = 0;           // tensor-core path: one int per chunk (exact-path fallback)
   size_t bwd_bytes = 0;
 };
 
@@ -81,8 +86,10 @@ cudaError_t launch_fwd_prep(const FwdArgs& a, bool with_P, cudaStream_t st);
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st);
 int choose_cluster(int units, int sms);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st);
-// the per-chunk parallel part of the backward (after the reverse chain)
-cudaError_t launch_bwd_simt_rest(const BwdArgs& a, cudaStream_t st);
+// CUDA-core backward kernels by stage; `only` (nullable) restricts the intra
+// stage to chunks whose flag is set.
+constexpr int kStageChain = 1, kStageCC = 2, kStageState = 4, kStageIntra = 8, kStageAll = 15;
+cudaError_t launch_bwd_simt_stages(const BwdArgs& a, int stages, const int* only, cudaStream_t st);
 cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
 
 template <typename T>
