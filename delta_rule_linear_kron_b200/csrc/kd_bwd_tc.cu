@@ -922,6 +922,191 @@ __global__ void __launch_bounds__(256, 1) bwd_intra_tc(
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------------------
+// C x C adjoints of the backward, one CTA per chunk, all chunks in parallel:
+//   K+ K-^T (tf32) -> decayed key Gram G_K;  [V; dO] V^T (bf16) -> G_V, dO V^T
+//   dP = (dO V^T) o u (i <= t);  dM = -(beta o g) u^T (i < t)
+//   dG_K = dM o G_V;  dG_V' = dM o G_K + (dM o G_K)^T
+//   dbeta = -g o (b0 + M u),  dc = g
+// Chunks outside the factorised decay range take exact per-element Grams.
+// ---------------------------------------------------------------------------
+struct CcCfg {
+  static constexpr uint32_t AK = 0;         // [K+; unused] tf32, 4 K blocks x 128 rows x 128 B
+  static constexpr uint32_t BKM = 65536;    // K- tf32, 4 K blocks x 64 rows x 128 B
+  static constexpr uint32_t AVD = 98304;    // [V; dO] bf16, 2 K blocks x 128 rows x 128 B
+  static constexpr uint32_t LS = 131072;    // L fp32 [64][129]
+  static constexpr uint32_t GV = LS + 64 * 129 * 4;   // dG_V fp32 [64][65]
+  static constexpr uint32_t SMALL = GV + 64 * 65 * 4; // u, g, beta, b0 [64] each
+  static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
+};
+
+__global__ void __launch_bounds__(256, 1) bwd_cc_tc(
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    const __nv_bfloat16* __restrict__ k, const float* __restrict__ beta, const float* __restrict__ logf, int H,
+    int T, int NC, const float* __restrict__ wu, const float* __restrict__ wb0, const float* __restrict__ wg,
+    float* __restrict__ dbeta, float* __restrict__ dc, float* __restrict__ wdP, float* __restrict__ wdGK,
+    float* __restrict__ wdGVs, int* __restrict__ err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar, mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag, unsafe;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = blockIdx.x;
+  float* Ls = reinterpret_cast<float*>(sm + CcCfg::LS);
+  float* GVs = reinterpret_cast<float*>(sm + CcCfg::GV);
+  float* us = reinterpret_cast<float*>(sm + CcCfg::SMALL);
+  float* gs = us + 64;
+  float* bs = gs + 64;
+  float* b0s = bs + 64;
+
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+    unsafe = 0;
+    tc::mbar_expect_tx(&ld_bar, 32768u);
+    tc::tma_load_4d(sm + CcCfg::AVD, &tm_v, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CcCfg::AVD + 16384, &tm_v, 64, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CcCfg::AVD + 8192, &tm_do, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CcCfg::AVD + 16384 + 8192, &tm_do, 64, h, t0, b, &ld_bar);
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  if (tid < 128) {
+    const int j = tid;
+    float L = 0.f, mx = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < C; ++t) {
+      const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
+      const bool ok = t < nv;
+      L += ok ? logf[g] : 0.f;
+      mx = fmaxf(mx, fabsf(L));
+      Ls[t * 129 + j] = L;
+      const float kk = ok ? __bfloat162float(k[g]) : 0.f;
+      *reinterpret_cast<float*>(sm + CcCfg::AK + tc::sw128_off(t, j, 128, 4)) = kk * expf(L);
+      *reinterpret_cast<float*>(sm + CcCfg::BKM + tc::sw128_off(t, j, 64, 4)) = kk * expf(-L);
+    }
+    if (!(mx < kSafeLogRange)) atomicOr(&unsafe, 1);
+  } else {
+    const int i = tid - 128;
+    if (i < C) {
+      us[i] = wu[ch * C + i];
+      gs[i] = wg[ch * C + i];
+      b0s[i] = wb0[ch * C + i];
+      bs[i] = i < nv ? beta[((size_t)b * T + t0 + i) * H + h] : 0.f;
+    }
+  }
+  tc::fence_proxy_async();
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    const uint32_t IDT = tc::idesc(128, 64, 2), IDB = tc::idesc(128, 64, 1);
+#pragma unroll
+    for (int ks = 0; ks < 16; ++ks) {
+      const uint32_t kb = ks / 4, w = (ks % 4) * 32;
+      tc::mma_tf32_ss(tmem + 0, tc::desc_sw128(tc::smem_u32(sm + CcCfg::AK + kb * 16384 + w)),
+                      tc::desc_sw128(tc::smem_u32(sm + CcCfg::BKM + kb * 8192 + w)), IDT, ks > 0 ? 1u : 0u);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
+      const uint64_t vd = tc::desc_sw128(tc::smem_u32(sm + CcCfg::AVD + o));
+      tc::mma_bf16_ss(tmem + 64, vd, vd, IDB, ks > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  const bool is_unsafe = unsafe != 0;
+  if (warp < 4) {
+    const int row = warp * 32 + lane;
+    const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, 0);
+    if (row < 64) {
+      const int t = row;
+      const float bg = -bs[t] * gs[t];
+      float* dgk = wdGK + ch * C * C + t * C;
+      float brow = 0.f;
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float gk[16], gv[16];
+        tc::tmem_ld16(lanes + 16 * c16, gk);
+        tc::tmem_ld16(lanes + 64 + 16 * c16, gv);
+        tc::tmem_ld_wait();
+        if (is_unsafe) {  // exact decay weights for this row
+#pragma unroll 1
+          for (int ii = 0; ii < 16; ++ii) {
+            const int i = 16 * c16 + ii;
+            float x = 0.f;
+            if (i < t) {
+              const size_t gt = (((size_t)b * T + t0 + t) * H + h) * D, gi = (((size_t)b * T + t0 + i) * H + h) * D;
+              for (int j = 0; j < D; ++j)
+                x = fmaf(__bfloat162float(k[gt + j]) * __bfloat162float(k[gi + j]),
+                         expf(Ls[t * 129 + j] - Ls[i * 129 + j]), x);
+            }
+            gk[ii] = x;
+          }
+        }
+        float o[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+          const int i = 16 * c16 + ii;
+          const bool low = i < t;
+          const float mm = low ? gk[ii] * gv[ii] : 0.f;
+          brow = fmaf(mm, us[i], brow);
+          const float dM = low ? bg * us[i] : 0.f;
+          o[ii] = dM * gv[ii];
+          GVs[t * 65 + i] = dM * gk[ii];
+        }
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4)
+          *reinterpret_cast<float4*>(dgk + 16 * c16 + 4 * i4) = make_float4(o[4 * i4], o[4 * i4 + 1], o[4 * i4 + 2], o[4 * i4 + 3]);
+      }
+      if (t < nv) {
+        const size_t g = ((size_t)b * T + t0 + t) * H + h;
+        dc[g] = gs[t];
+        dbeta[g] = -gs[t] * (b0s[t] + brow);
+      }
+    } else {
+      const int t = row - 64;
+      float* dp = wdP + ch * C * C + t * C;
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float dov[16];
+        tc::tmem_ld16(lanes + 64 + 16 * c16, dov);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          float4 v4;
+          const int i = 16 * c16 + 4 * i4;
+          v4.x = i <= t ? us[i] * dov[4 * i4] : 0.f;
+          v4.y = i + 1 <= t ? us[i + 1] * dov[4 * i4 + 1] : 0.f;
+          v4.z = i + 2 <= t ? us[i + 2] * dov[4 * i4 + 2] : 0.f;
+          v4.w = i + 3 <= t ? us[i + 3] * dov[4 * i4 + 3] : 0.f;
+          *reinterpret_cast<float4*>(dp + i) = v4;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < C * C; e += 256) {
+    const int t = e / C, i = e % C;
+    wdGVs[ch * C * C + e] = GVs[t * 65 + i] + GVs[i * 65 + t];
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
 template <int R>
 cudaError_t launch_bchain(const BwdArgs& a, int* err, cudaStream_t st) {
   const Layout& L = a.L;
@@ -989,8 +1174,17 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st) 
       ws_ptr<float>(a.ws, L.acck), ws_ptr<float>(a.ws, L.accL), ws_ptr<float>(a.ws, L.accv), err);
   prof_end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // C x C adjoints (CUDA cores), then the intra-chunk products (tensor cores)
-  if ((e = launch_bwd_simt_stages(a, kStageCC, nullptr, st)) != cudaSuccess) return e;
+  // C x C adjoints, then the intra-chunk products
+  if ((e = cudaFuncSetAttribute(bwd_cc_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CcCfg::BYTES)) !=
+      cudaSuccess)
+    return e;
+  prof_begin(st, "bwd_cc_tc");
+  bwd_cc_tc<<<(unsigned)L.chunks, 256, CcCfg::BYTES, st>>>(
+      tm_v, tm_do, static_cast<const __nv_bfloat16*>(a.k), a.beta, a.logf, L.H, L.T, L.NC,
+      ws_ptr<float>(a.fws, L.u), ws_ptr<float>(a.fws, L.b0), ws_ptr<float>(a.ws, L.g), a.dbeta, a.dc,
+      ws_ptr<float>(a.ws, L.dP), ws_ptr<float>(a.ws, L.dGK), ws_ptr<float>(a.ws, L.dGVs), err);
+  prof_end(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   int* flags = ws_ptr<int>(a.ws, L.bflags);
   if ((e = cudaFuncSetAttribute(bwd_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)InCfg::BYTES)) != cudaSuccess)

@@ -664,6 +664,234 @@ __global__ void __launch_bounds__(128) fwd_out_fixup(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Chunk preparation on tensor cores, one CTA per chunk, all chunks in parallel:
+//   [K+; Q+] K-^T (tf32)  -> rows 0-63: decayed key Gram, rows 64-127: P
+//   V V^T (bf16, exact)   -> value Gram
+//   M = tril(G_K o G_V, -1); A = (I + diag(beta) M)^{-1}; y = A c
+// The inverse is blocked by 16: the four diagonal blocks by forward
+// substitution in parallel, then the off-diagonal blocks block-row by
+// block-row, X_ab = -X_aa sum_{c=b}^{a-1} N_ac X_cb, all in fp32.
+// Chunks outside the factorised decay range take exact per-element Grams.
+// ---------------------------------------------------------------------------
+struct PrepCfg {
+  static constexpr uint32_t AKQ = 0;        // [K+; Q+] tf32, 4 K blocks x 128 rows x 128 B
+  static constexpr uint32_t BKM = 65536;    // K- tf32, 4 K blocks x 64 rows x 128 B
+  static constexpr uint32_t VT = 98304;     // V bf16, 2 K blocks x 128 rows x 128 B (rows 64..127 unused)
+  static constexpr uint32_t LS = 131072;    // L fp32 [64][129]
+  static constexpr uint32_t NS = LS + 64 * 129 * 4;   // N = diag(beta) M, fp32 [64][65]
+  static constexpr uint32_t XS = NS + 64 * 65 * 4;    // A, fp32 [64][65]
+  static constexpr uint32_t TS = XS + 64 * 65 * 4;    // block temporaries [3][16][17]
+  static constexpr uint32_t SMALL = TS + 3 * 16 * 17 * 4;  // beta, c [64] each
+  static constexpr uint32_t BYTES = SMALL + 512 + 1024;
+};
+
+__global__ void __launch_bounds__(256, 1) fwd_prep_tc(
+    const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const float* __restrict__ beta, const float* __restrict__ c,
+    const float* __restrict__ logf, int H, int T, int NC, float* __restrict__ wy, float* __restrict__ wA,
+    float* __restrict__ wP, int* __restrict__ err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar, mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag, unsafe;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = blockIdx.x;
+  float* Ls = reinterpret_cast<float*>(sm + PrepCfg::LS);
+  float* Ns = reinterpret_cast<float*>(sm + PrepCfg::NS);
+  float* Xs = reinterpret_cast<float*>(sm + PrepCfg::XS);
+  float* Ts = reinterpret_cast<float*>(sm + PrepCfg::TS);
+  float* bs = reinterpret_cast<float*>(sm + PrepCfg::SMALL);
+  float* cs = bs + 64;
+
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+    unsafe = 0;
+    tc::mbar_expect_tx(&ld_bar, 16384u);
+    tc::tma_load_4d(sm + PrepCfg::VT, &tm_v, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PrepCfg::VT + 16384, &tm_v, 64, h, t0, b, &ld_bar);
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  if (tid < 128) {
+    const int j = tid;
+    float L = 0.f, mx = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < C; ++t) {
+      const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
+      const bool ok = t < nv;
+      L += ok ? logf[g] : 0.f;
+      mx = fmaxf(mx, fabsf(L));
+      Ls[t * 129 + j] = L;
+      const float qq = ok ? __bfloat162float(q[g]) : 0.f, kk = ok ? __bfloat162float(k[g]) : 0.f;
+      const float gm = expf(L), ig = expf(-L);
+      *reinterpret_cast<float*>(sm + PrepCfg::AKQ + tc::sw128_off(t, j, 128, 4)) = kk * gm;
+      *reinterpret_cast<float*>(sm + PrepCfg::AKQ + tc::sw128_off(64 + t, j, 128, 4)) = qq * gm;
+      *reinterpret_cast<float*>(sm + PrepCfg::BKM + tc::sw128_off(t, j, 64, 4)) = kk * ig;
+    }
+    if (!(mx < kSafeLogRange)) atomicOr(&unsafe, 1);
+  } else {
+    const int i = tid - 128;
+    if (i < C) {
+      const bool ok = i < nv;
+      const size_t g = ((size_t)b * T + t0 + i) * H + h;
+      bs[i] = ok ? beta[g] : 0.f;
+      cs[i] = ok ? c[g] : 0.f;
+    }
+  }
+  tc::fence_proxy_async();
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    const uint32_t IDT = tc::idesc(128, 64, 2), IDB = tc::idesc(128, 64, 1);
+#pragma unroll
+    for (int ks = 0; ks < 16; ++ks) {
+      const uint32_t kb = ks / 4, w = (ks % 4) * 32;
+      tc::mma_tf32_ss(tmem + 0, tc::desc_sw128(tc::smem_u32(sm + PrepCfg::AKQ + kb * 16384 + w)),
+                      tc::desc_sw128(tc::smem_u32(sm + PrepCfg::BKM + kb * 8192 + w)), IDT, ks > 0 ? 1u : 0u);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
+      const uint64_t vd = tc::desc_sw128(tc::smem_u32(sm + PrepCfg::VT + o));
+      tc::mma_bf16_ss(tmem + 64, vd, vd, IDB, ks > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  const bool is_unsafe = unsafe != 0;
+  // rows t (TMEM lanes 0..63): N[t][i] = beta_t G_K G_V (i < t); lanes 64+t: P row t
+  if (warp < 4) {
+    const int row = warp * 32 + lane;
+    const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, 0);
+    if (row < 64) {
+      const int t = row;
+      const float bt = bs[t];
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float gk[16], gv[16];
+        tc::tmem_ld16(lanes + 16 * c16, gk);
+        tc::tmem_ld16(lanes + 64 + 16 * c16, gv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+          const int i = 16 * c16 + ii;
+          Ns[t * 65 + i] = i < t ? bt * gk[ii] * gv[ii] : 0.f;
+        }
+      }
+    } else if (wP && !is_unsafe) {
+      const int t = row - 64;
+      float* prow = wP + ch * C * C + t * C;
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float pv[16];
+        tc::tmem_ld16(lanes + 16 * c16, pv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          float4 o;
+          const int i = 16 * c16 + 4 * i4;
+          o.x = i <= t ? pv[4 * i4] : 0.f;
+          o.y = i + 1 <= t ? pv[4 * i4 + 1] : 0.f;
+          o.z = i + 2 <= t ? pv[4 * i4 + 2] : 0.f;
+          o.w = i + 3 <= t ? pv[4 * i4 + 3] : 0.f;
+          *reinterpret_cast<float4*>(prow + i) = o;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (is_unsafe) {
+    // exact decay weights e^{L_t - L_i} <= 1 per element (rare: extreme decays)
+    for (int e = tid; e < C * C; e += 256) {
+      const int t = e / C, i = e % C;
+      float gk = 0.f, gv = 0.f, pq = 0.f;
+      if (i <= t) {
+        const size_t gt = (((size_t)b * T + t0 + t) * H + h) * D, gi = (((size_t)b * T + t0 + i) * H + h) * D;
+        const bool okt = t < nv, oki = i < nv;
+        for (int j = 0; j < D; ++j) {
+          const float w = expf(Ls[t * 129 + j] - Ls[i * 129 + j]);
+          const float kt = okt ? __bfloat162float(k[gt + j]) : 0.f, ki = oki ? __bfloat162float(k[gi + j]) : 0.f;
+          const float qt = okt ? __bfloat162float(q[gt + j]) : 0.f;
+          gk = fmaf(kt * ki, w, gk);
+          pq = fmaf(qt * ki, w, pq);
+        }
+        for (int r = 0; r < D; ++r)
+          gv = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::VT + tc::sw128_off(t, r, 128, 2) + 0 * 0)),
+                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::VT + tc::sw128_off(i, r, 128, 2))), gv);
+      }
+      Ns[t * 65 + i] = i < t ? bs[t] * gk * gv : 0.f;
+      if (wP) wP[ch * C * C + e] = i <= t ? pq : 0.f;
+    }
+    __syncthreads();
+  }
+  // ---- X = (I + N)^{-1}, blocked by 16
+  {
+    // diagonal blocks: thread (blk, m) solves column m of block blk
+    if (tid < 64) {
+      const int blk = tid >> 4, m = tid & 15, o = 16 * blk;
+      float col[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        float s = t == m ? 1.f : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2)
+          if (s2 >= m && s2 < t) s = fmaf(-Ns[(o + t) * 65 + o + s2], col[s2], s);
+        col[t] = t < m ? 0.f : s;
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) Xs[(o + t) * 65 + o + m] = col[t];
+    }
+    // zero the strictly upper blocks
+    for (int e = tid; e < C * C; e += 256) {
+      const int t = e / C, i = e % C;
+      if ((i >> 4) > (t >> 4)) Xs[t * 65 + i] = 0.f;
+    }
+    __syncthreads();
+    for (int a = 1; a < 4; ++a) {
+      // T_ab = sum_{cb=b}^{a-1} N_{a,cb} X_{cb,b} for b < a (16 x 16 each)
+      for (int e = tid; e < a * 256; e += 256) {
+        const int bb = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        float s = 0.f;
+        for (int kk = 16 * bb; kk < 16 * a; ++kk) s = fmaf(Ns[(16 * a + rr) * 65 + kk], Xs[kk * 65 + 16 * bb + cc], s);
+        Ts[bb * 272 + rr * 17 + cc] = s;
+      }
+      __syncthreads();
+      // X_ab = -X_aa T_ab
+      for (int e = tid; e < a * 256; e += 256) {
+        const int bb = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        float s = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) s = fmaf(Xs[(16 * a + rr) * 65 + 16 * a + kk], Ts[bb * 272 + kk * 17 + cc], s);
+        Xs[(16 * a + rr) * 65 + 16 * bb + cc] = -s;
+      }
+      __syncthreads();
+    }
+  }
+  if (tid < C) {
+    float s = 0.f;
+    for (int m = 0; m <= tid; ++m) s = fmaf(Xs[tid * 65 + m], cs[m], s);
+    wy[ch * C + tid] = s;
+  }
+  for (int e = tid; e < C * C; e += 256) wA[ch * C * C + e] = Xs[(e / C) * 65 + (e % C)];
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
 template <int R>
 cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, float* blob, float* wu,
                          float* wb0, int* err, cudaStream_t st) {
@@ -734,8 +962,21 @@ int choose_cluster(int units, int sms) {
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) {
   const Layout& L = a.L;
-  cudaError_t e = launch_fwd_prep(a, /*with_P=*/a.save != 0, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  {
+    CUtensorMap tm_v;
+    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true)) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(fwd_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PrepCfg::BYTES)) != cudaSuccess)
+      return e;
+    prof_begin(st, "fwd_prep_tc");
+    fwd_prep_tc<<<(unsigned)L.chunks, 256, PrepCfg::BYTES, st>>>(
+        tm_v, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.beta, a.c,
+        a.logf, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
+        a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, err);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const float* wy = ws_ptr<float>(a.ws, L.y);
   const float* wA = ws_ptr<float>(a.ws, L.A);
   float* blob = ws_ptr<float>(a.ws, L.S0);
