@@ -52,33 +52,93 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# algorithmic work per kernel, per token-head (d_k = d_v = d, C = 64, bf16 I/O)
-#   flops count dense contractions only (2 per multiply-add); bytes count
-#   what a kernel must move across HBM with its inputs and outputs.
+# Algorithmic work per kernel, per token-head (d_k = d_v = d = 128, C = 64,
+# bf16 activations).  flops: the dense contractions the kernel performs (2
+# per multiply-add).  They add up to 180,224 forward and 425,984 backward
+# flops per token-head, above the method's 163,840 / 360,448 because the
+# output kernel recomputes the masked Gram Q+ K-^T and the backward
+# recomputes two products with S0; the step-level tensor fraction uses the
+# method's 524,288.  bytes: the kernel's own inputs and outputs in HBM.
+# kind: the unit that executes the contractions.
 # ---------------------------------------------------------------------------
 def kernel_work(name, d=128, C=CHUNK):
-    io_in = 3 * d * 2 + d * 4 + 8          # q,k,v bf16 + logf fp32 + beta,c
-    works = {
-        # Grams K K^T, V V^T, Q K^T (3 C x C x d); writes y, A, P (fp32)
-        "fwd_prep_simt": dict(flops=6 * C * d, bytes=io_in + 4 + 2 * C * 4),
-        # S K+^T, S Q+^T, V^T diag(u) K^e (3 d x d x C) + P diag(u) V (C x C x d)
-        "fwd_chain_simt": dict(flops=6 * d * d + 2 * C * d,
-                               bytes=io_in + 4 + 2 * C * 4 + d * 2 + d * d * 4 // C + 8),
-        # dS K^e^T, dO^T Q+, V^T diag(db0) K+ (3 d x d x C) + P^T dO (C x C x d)
-        "bwd_chain_simt": dict(flops=6 * d * d + 2 * C * d,
-                               bytes=io_in + d * 2 + 2 * C * 4 + d * d * 4 // C + 4),
-        # K K^T, V V^T, dO V^T (3 C x C x d)
-        "bwd_cc_simt": dict(flops=6 * C * d, bytes=2 * d * 2 + d * 4 + d * 2 + 16 + 3 * C * 4),
-        # dO S0, V S0, V dS, K+ S0^T, K^e dS^T (5 d x d x C)
-        "bwd_state_simt": dict(flops=10 * d * d, bytes=4 * d * 2 + d * 4 + 2 * d * d * 4 // C + 4 * d * 4),
-        # dP K-, dP^T Q+, dG_K K-, dG_K^T K+, P^T dO, dG_V V (6 C x C x d)
-        "bwd_intra_simt": dict(flops=12 * C * d, bytes=4 * d * 2 + d * 4 + 3 * C * 4 + 4 * d * 4 + 3 * d * 2 + d * 4),
+    act = d * 2                      # one bf16 activation row
+    lf = d * 4                       # one fp32 logf row
+    tile_f32 = d * d * 4 // C        # one fp32 d x d tile per chunk, per token
+    tile_bf16 = d * d * 2 // C
+    cc = C * 4                       # one fp32 C x C matrix per chunk, per token
+    table = {
+        # Grams [K+;Q+] K-^T (tf32) and V V^T (bf16); writes A, y (+ P when saving)
+        "fwd_prep_tc": ("tf32", 6 * C * d, 3 * act + lf + 8 + cc + 4 + cc),
+        # X = S K+^T and dS = V^T diag(u) K^e over the cluster; writes u, b0 and the chunk-start state tiles
+        "fwd_chain_tc": ("tf32", 4 * d * d, 2 * act + lf + 4 + cc + 4 + 8 + tile_f32 + 2 * tile_bf16),
+        # S0 Q+^T, [Q+;0] K-^T, V^T (u o P^T); writes O
+        "fwd_out_tc": ("tf32", 2 * d * d + 4 * C * d, 3 * act + lf + 4 + tile_f32 + act),
+        "fwd_out_fixup": ("alu", 0, 4),
+        # dO V^T masked by P
+        "bwd_du_intra": ("alu", 2 * C * d, 2 * act + cc + 4),
+        # dS K^e^T (tf32), dO^T Q+ and V^T (db0 o K+) (bf16); writes dS tiles, g
+        "bwd_chain_tc": ("bf16", 6 * d * d, 4 * act + lf + 4 + cc + 4 + 2 * tile_bf16 + 4),
+        # K+ K-^T (tf32) and [V;dO] V^T (bf16); writes dP, dG_K, dG_V', dbeta, dc
+        "bwd_cc_tc": ("bf16", 6 * C * d, 3 * act + lf + 16 + 3 * cc + 8),
+        # dO S0, V S0, V dS, K+ S0^T, K^e dS^T; writes the four accumulators
+        "bwd_state_tc": ("bf16", 10 * d * d, 4 * act + lf + 12 + 4 * tile_bf16 + 4 * d * 4),
+        # [dP;dG_K] K-, [dP^T|dG_K^T][Q+;K+], [uP^T|dG_V'][dO;V]; writes dq, dk, dv, dlogf
+        "bwd_intra_tc": ("bf16", 12 * C * d, 4 * act + lf + 4 * cc + 4 + 4 * d * 4 + 3 * act + lf),
+        # CUDA-core kernels of the general (fp32 / small-d) path
+        "fwd_prep_simt": ("alu", 6 * C * d, 3 * act + lf + 8 + 2 * cc + 4),
+        "fwd_chain_simt": ("alu", 6 * d * d + 2 * C * d, 3 * act + lf + 4 + 2 * cc + act + tile_f32 + 8),
+        "bwd_chain_simt": ("alu", 6 * d * d + 2 * C * d, 4 * act + lf + 2 * cc + tile_f32 + 4),
+        "bwd_cc_simt": ("alu", 6 * C * d, 3 * act + lf + 16 + 3 * cc + 8),
+        "bwd_state_simt": ("alu", 10 * d * d, 4 * act + lf + 2 * tile_f32 + 4 * d * 4),
+        "decode_kernel": ("alu", 0, 0),
     }
-    return works.get(name)
+    w = table.get(name)
+    return None if w is None else dict(kind=w[0], flops=w[1], bytes=w[2])
+
+
+# DRAM bytes (read + write) per launch from one ncu capture of this workload
+# (dram__bytes_read.sum + dram__bytes_write.sum), with the source file the
+# kernel lives in and the first 16 hex digits of its sha256 at capture time;
+# a kernel whose source has changed since reports no traffic.
+NCU_TRAFFIC = {
+    "fwd_prep_tc": (449772288, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
+    "fwd_chain_tc": (823336192, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
+    "fwd_out_tc": (662604544, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
+    "bwd_du_intra": (202038784, "kd_bwd_tc.cu", "c73c3f747a52806b"),
+    "bwd_chain_tc": (707717632, "kd_bwd_tc.cu", "c73c3f747a52806b"),
+    "bwd_cc_tc": (507570688, "kd_bwd_tc.cu", "c73c3f747a52806b"),
+    "bwd_state_tc": (1496024320, "kd_bwd_tc.cu", "c73c3f747a52806b"),
+    "bwd_intra_tc": (1521490176, "kd_bwd_tc.cu", "c73c3f747a52806b"),
+}
+
+
+def ncu_traffic(name):
+    t = NCU_TRAFFIC.get(name)
+    if t is None:
+        return None
+    import hashlib
+    path = os.path.join(ROOT, "delta_rule_linear_kron_b200", "csrc", t[1])
+    try:
+        with open(path, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return t[0] if digest == t[2] else None
+
+
+def compute_peak_tflops(kind, peaks):
+    """Peak for a kernel timed inside a long step: sustained bf16 (measured);
+    tf32 = that x the nominal tf32/bf16 ratio (1.1 / 2.25 PF dense); alu =
+    148 SMs x 128 FP32 lanes x 2 flops x the max SM clock."""
+    if kind == "bf16":
+        return peaks["bf16_tflops_sustained"]
+    if kind == "tf32":
+        return peaks["bf16_tflops_sustained"] * 1.1 / 2.25
+    return fp32_alu_peak_tflops(peaks["sm_max_mhz"])
 
 
 def fp32_alu_peak_tflops(sm_mhz):
-    # 148 SMs x 128 FP32 lanes x 2 flops per FFMA
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
@@ -339,22 +399,38 @@ def main(argv=None):
 
     # ---- roofline of the dominant kernel ---------------------------------
     roofline = None
-    if per_kernel:
-        top = max(per_kernel, key=lambda n: per_kernel[n]["ms"])
-        w = kernel_work(top)
-        avg_s = per_kernel[top]["ms"] / per_kernel[top]["launches"] / 1e3
-        units = B * H * T  # token-heads per launch
-        sm_mhz = clocks["sm_mhz"] or peaks["sm_max_mhz"]
-        if w is not None:
-            achieved = w["flops"] * units / avg_s / 1e12
-            peak = fp32_alu_peak_tflops(peaks["sm_max_mhz"])
-            roofline = dict(kernel=top, bound="alu", achieved=achieved, peak=peak, unit="TFLOP/s",
-                            frac=achieved / peak, traffic=None,
-                            algorithmic_flops_per_launch=w["flops"] * units,
-                            algorithmic_bytes_per_launch=w["bytes"] * units,
-                            hbm_achieved_gbs=w["bytes"] * units / avg_s / 1e9,
-                            peak_note="fp32 FFMA: 148 SMs x 128 lanes x 2 flops x max SM clock",
-                            avg_launch_ms=avg_s * 1e3, sm_mhz_median=sm_mhz)
+    kernels = {}
+    units = B * H * T  # token-heads per launch of every per-step kernel
+    for name, v in per_kernel.items():
+        w = kernel_work(name)
+        if w is None or v["launches"] == 0:
+            continue
+        avg_s = v["ms"] / v["launches"] / 1e3
+        pk = compute_peak_tflops(w["kind"], peaks)
+        t_c = w["flops"] * units / (pk * 1e12)
+        t_m = w["bytes"] * units / (peaks["hbm_gbs"] * 1e9)
+        if t_c >= t_m:
+            ach = w["flops"] * units / avg_s / 1e12
+            kernels[name] = dict(bound="alu" if w["kind"] == "alu" else "tensor", kind=w["kind"], achieved=ach,
+                                 peak=pk, unit="TFLOP/s", frac=ach / pk)
+        else:
+            ach = w["bytes"] * units / avg_s / 1e9
+            kernels[name] = dict(bound="hbm", kind=w["kind"], achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
+                                 frac=ach / peaks["hbm_gbs"])
+        kernels[name].update(avg_launch_ms=avg_s * 1e3, algorithmic_flops_per_launch=w["flops"] * units,
+                             algorithmic_bytes_per_launch=w["bytes"] * units, traffic=ncu_traffic(name))
+    if kernels:
+        top = max(kernels, key=lambda n: per_kernel[n]["ms"])
+        k = kernels[top]
+        roofline = dict(kernel=top, bound=k["bound"], achieved=k["achieved"], peak=k["peak"], unit=k["unit"],
+                        frac=k["frac"], traffic=k["traffic"], avg_launch_ms=k["avg_launch_ms"],
+                        algorithmic_flops_per_launch=k["algorithmic_flops_per_launch"],
+                        algorithmic_bytes_per_launch=k["algorithmic_bytes_per_launch"],
+                        peak_note=("measured HBM copy bandwidth" if k["bound"] == "hbm" else
+                                   "measured sustained bf16 GEMM" + (" x 1.1/2.25 (tf32)" if k["kind"] == "tf32" else "")
+                                   if k["bound"] == "tensor" else "148 SMs x 128 FP32 lanes x 2 x max SM clock")
+                        + " (" + peaks["source"] + ")",
+                        sm_mhz_median=clocks["sm_mhz"])
     step_flops = 524288 * B * H * T
     tc_frac = step_flops / (ms_total / args.steps / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
 
@@ -372,6 +448,7 @@ def main(argv=None):
                 "tc_frac_of_bf16_peak": tc_frac,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
                 "gpu_launches": launches, "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
+                "kernel_rooflines": kernels,
                 "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                            "reasons": clocks["reasons"], "samples": clocks["samples"]},
                 "peaks": peaks}
