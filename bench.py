@@ -54,12 +54,14 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 # Algorithmic work per kernel, per token-head (d_k = d_v = d = 128, C = 64,
 # bf16 activations).  flops: the dense contractions the kernel performs (2
-# per multiply-add).  They add up to 180,224 forward and 425,984 backward
+# per multiply-add).  They add up to 180,224 forward and 409,600 backward
 # flops per token-head, above the method's 163,840 / 360,448 because the
-# output kernel recomputes the masked Gram Q+ K-^T and the backward
-# recomputes two products with S0; the step-level tensor fraction uses the
-# method's 524,288.  bytes: the kernel's own inputs and outputs in HBM.
-# kind: the unit that executes the contractions.
+# output kernel recomputes the masked Gram Q+ K-^T and the post-chain kernel
+# forms the chunk-end term from separate accumulators; the step-level tensor
+# fraction uses the method's 524,288.  bytes: the kernel's own inputs and
+# outputs in HBM.  kind: the unit that executes the contractions.  The exact
+# CUDA-core kernels that recompute flagged chunks (extreme decays) only touch
+# those chunks and have no per-token figure.
 # ---------------------------------------------------------------------------
 def kernel_work(name, d=128, C=CHUNK):
     act = d * 2                      # one bf16 activation row
@@ -67,31 +69,21 @@ def kernel_work(name, d=128, C=CHUNK):
     tile_f32 = d * d * 4 // C        # one fp32 d x d tile per chunk, per token
     tile_bf16 = d * d * 2 // C
     cc = C * 4                       # one fp32 C x C matrix per chunk, per token
+    ccb = C * 2                      # one bf16 C x C tile per chunk, per token
     table = {
-        # Grams [K+;Q+] K-^T (tf32) and V V^T (bf16); writes A, y (+ P when saving)
+        # Grams [K+; Q+] K-^T (tf32) and V V^T (bf16); writes A, y and P
         "fwd_prep_tc": ("tf32", 6 * C * d, 3 * act + lf + 8 + cc + 4 + cc),
         # X = S K+^T and dS = V^T diag(u) K^e over the cluster; writes u, b0 and the chunk-start state tiles
-        "fwd_chain_tc": ("tf32", 4 * d * d, 2 * act + lf + 4 + cc + 4 + 8 + tile_f32 + 2 * tile_bf16),
-        # S0 Q+^T, [Q+;0] K-^T, V^T (u o P^T); writes O
+        "fwd_chain_tc": ("tf32", 4 * d * d, 2 * act + lf + 4 + cc + 4 + 8 + tile_f32 + tile_bf16),
+        # S0 Q+^T, [Q+; K-] K-^T (tf32), V^T (u o P^T) (bf16); writes O
         "fwd_out_tc": ("tf32", 2 * d * d + 4 * C * d, 3 * act + lf + 4 + tile_f32 + act),
-        "fwd_out_fixup": ("alu", 0, 4),
-        # dO V^T masked by P
-        "bwd_du_intra": ("alu", 2 * C * d, 2 * act + cc + 4),
-        # dS K^e^T (tf32), dO^T Q+ and V^T (db0 o K+) (bf16); writes dS tiles, g
-        "bwd_chain_tc": ("bf16", 6 * d * d, 4 * act + lf + 4 + cc + 4 + 2 * tile_bf16 + 4),
-        # K+ K-^T (tf32) and [V;dO] V^T (bf16); writes dP, dG_K, dG_V', dbeta, dc
-        "bwd_cc_tc": ("bf16", 6 * C * d, 3 * act + lf + 16 + 3 * cc + 8),
-        # dO S0, V S0, V dS, K+ S0^T, K^e dS^T; writes the four accumulators
-        "bwd_state_tc": ("bf16", 10 * d * d, 4 * act + lf + 12 + 4 * tile_bf16 + 4 * d * 4),
-        # [dP;dG_K] K-, [dP^T|dG_K^T][Q+;K+], [uP^T|dG_V'][dO;V]; writes dq, dk, dv, dlogf
-        "bwd_intra_tc": ("bf16", 12 * C * d, 4 * act + lf + 4 * cc + 4 + 4 * d * 4 + 3 * act + lf),
-        # CUDA-core kernels of the general (fp32 / small-d) path
-        "fwd_prep_simt": ("alu", 6 * C * d, 3 * act + lf + 8 + 2 * cc + 4),
-        "fwd_chain_simt": ("alu", 6 * d * d + 2 * C * d, 3 * act + lf + 4 + 2 * cc + act + tile_f32 + 8),
-        "bwd_chain_simt": ("alu", 6 * d * d + 2 * C * d, 4 * act + lf + 2 * cc + tile_f32 + 4),
-        "bwd_cc_simt": ("alu", 6 * C * d, 3 * act + lf + 16 + 3 * cc + 8),
-        "bwd_state_simt": ("alu", 10 * d * d, 4 * act + lf + 2 * tile_f32 + 4 * d * 4),
-        "decode_kernel": ("alu", 0, 0),
+        # K+ K-^T (tf32), [V; dO] V^T and [V; dO] dO^T (bf16); writes du_intra, M u and three bf16 tiles
+        "bwd_pre_tc": ("bf16", 6 * C * d, 3 * act + lf + cc + 4 + 2 * ccb + ccb + ccb + 8),
+        # dS K^e^T (tf32), dO^T Q+ and V^T (db0 o K+) (bf16); writes the dS tile and g
+        "bwd_chain_tc": ("bf16", 6 * d * d, 4 * act + lf + 4 + cc + 4 + tile_bf16 + 4),
+        # the five state / intra-chunk accumulators; writes dq, dk, dv, dlogf, dbeta, dc
+        "bwd_post_tc": ("bf16", 16 * d * d, 4 * act + lf + 2 * tile_bf16 + 2 * ccb + ccb + ccb + 20
+                        + 3 * act + lf + 8),
     }
     w = table.get(name)
     return None if w is None else dict(kind=w[0], flops=w[1], bytes=w[2])
@@ -105,11 +97,6 @@ NCU_TRAFFIC = {
     "fwd_prep_tc": (449772288, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
     "fwd_chain_tc": (823336192, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
     "fwd_out_tc": (662604544, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
-    "bwd_du_intra": (202038784, "kd_bwd_tc.cu", "c73c3f747a52806b"),
-    "bwd_chain_tc": (707717632, "kd_bwd_tc.cu", "c73c3f747a52806b"),
-    "bwd_cc_tc": (507570688, "kd_bwd_tc.cu", "c73c3f747a52806b"),
-    "bwd_state_tc": (1496024320, "kd_bwd_tc.cu", "c73c3f747a52806b"),
-    "bwd_intra_tc": (1521490176, "kd_bwd_tc.cu", "c73c3f747a52806b"),
 }
 
 

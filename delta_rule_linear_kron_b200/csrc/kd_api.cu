@@ -69,7 +69,6 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   if (L->tc) {
     L->fwd_bytes = off;  // the output kernel reads the chunk-start states
     L->S0b = take(chunks * (size_t)dv * dk * 2);
-    L->S0bt = take(chunks * (size_t)dv * dk * 2);
   }
   L->fwd_save_bytes = off;
 
@@ -86,8 +85,11 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->du = take(chunks * C * 4);
   if (L->tc) {
     L->dSCb = take(chunks * (size_t)dv * dk * 2);
-    L->dSCbt = take(chunks * (size_t)dv * dk * 2);
     L->bflags = take(chunks * 4);
+    L->T1 = take(chunks * 2 * C * C * 2);
+    L->PU = take(chunks * C * C * 2);
+    L->EK = take(chunks * C * C * 2);
+    L->Mu = take(chunks * C * 4);
   }
   L->bwd_bytes = off;
   return KD_OK;

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
     const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T, int NC,
     const float* __restrict__ wu, const float* __restrict__ wb0, const float* __restrict__ wg,
     float* __restrict__ dbeta, float* __restrict__ dc, float* __restrict__ wdP,
-    float* __restrict__ wdGK, float* __restrict__ wdGVs) {
+    float* __restrict__ wdGK, float* __restrict__ wdGVs, const int* __restrict__ only) {
   constexpr int SK = DK + 1, SV = DV + 1, SC = C + 1;
   extern __shared__ float smem[];
   float* Kp = smem;            // [C][SK]
@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)b * H + h) * NC + n;
+  if (only && only[ch] == 0) return;  // only the chunks flagged by the tensor-core kernel
 
   for (int e = tid; e < C * DK; e += blockDim.x) {
     const int t = e / DK, j = e % DK;
@@ -286,6 +287,14 @@ __device__ __forceinline__ size_t sw128_index(int r, int j) {
          (size_t)(((chunk ^ (r & 7)) & 7) * 4) + (j & 3);
 }
 
+// byte offset of (r, j) in a 128x128 bf16 tile stored K-major with 128-byte
+// swizzle: 2 blocks of 64 columns, 1024-byte atoms of 8 rows
+__device__ __forceinline__ size_t sw128_bf16_off(int r, int j) {
+  const int kb = j >> 6, chunk = (j & 63) >> 3;
+  return (size_t)kb * 128 * 128 + (size_t)(r >> 3) * 1024 + (size_t)(r & 7) * 128 +
+         (size_t)(((chunk ^ (r & 7)) & 7) * 16) + (size_t)(j & 7) * 2;
+}
+
 template <int DK, int DV>
 constexpr size_t bstate_smem_floats() {
   return 3 * (size_t)C * (DK + 1) + 2 * (size_t)C * (DV + 1) + 2 * (size_t)SLAB * (DK + 1) + 2 * C +
@@ -298,7 +307,8 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
     const float* __restrict__ beta, const float* __restrict__ logf, const Tin* __restrict__ dO,
     int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wg,
     const float* __restrict__ wS0, const float* __restrict__ wdSC, float* __restrict__ waccq,
-    float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv, int s0_swizzled) {
+    float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv, int s0_swizzled,
+    const __nv_bfloat16* __restrict__ wdSb, const int* __restrict__ only) {
   constexpr int SK = DK + 1, SV = DV + 1;
   constexpr int TPJ = 256 / DK;   // thread groups over j
   constexpr int TPG = C / TPJ;    // rows per group
@@ -319,6 +329,7 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)b * H + h) * NC + n;
+  if (only && only[ch] == 0) return;  // only the chunks flagged by the tensor-core kernel
 
   for (int e = tid; e < C * DK; e += blockDim.x) {
     const int t = e / DK, j = e % DK;
@@ -362,14 +373,18 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
   for (int i = 0; i < TPG; ++i) aQ[i] = aVS[i] = aVD[i] = 0.f;
   float cs_local = 0.f;
   const float* S0c = wS0 + ch * DV * DK;
-  const float* dSc = wdSC + ch * DV * DK;
+  const float* dSc = wdSb ? nullptr : wdSC + ch * DV * DK;
+  // the tensor-core path keeps dS as a bf16 tile [r][j], 128-byte-swizzled K-major
+  const unsigned char* dSt = wdSb ? reinterpret_cast<const unsigned char*>(wdSb + ch * DV * DK) : nullptr;
   for (int r0 = 0; r0 < DV; r0 += SLAB) {
     for (int e = tid; e < SLAB * DK; e += blockDim.x) {
       const int rr = e / DK, jj = e % DK;
       // the tensor-core forward stores each chunk-start state as a 128x128
       // tf32 tile in the 128-byte-swizzled K-major layout of its MMAs
       S0s[rr * SK + jj] = s0_swizzled ? S0c[sw128_index(r0 + rr, jj)] : S0c[(size_t)(r0 + rr) * DK + jj];
-      dSs[rr * SK + jj] = dSc[(size_t)(r0 + rr) * DK + jj];
+      dSs[rr * SK + jj] = dSt ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                     dSt + sw128_bf16_off(r0 + rr, jj)))
+                              : dSc[(size_t)(r0 + rr) * DK + jj];
     }
     __syncthreads();
     // C x dk products, accumulated over all slabs
@@ -621,7 +636,7 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
   const float* wu = ws_ptr<float>(a.fws, L.u);
   const float* wb0 = ws_ptr<float>(a.fws, L.b0);
   const float* wS0 = ws_ptr<float>(a.fws, L.S0);
-  float* wdSC = ws_ptr<float>(a.ws, L.dSC);
+  float* wdSC = L.tc ? nullptr : ws_ptr<float>(a.ws, L.dSC);
   float* wg = ws_ptr<float>(a.ws, L.g);
   float* wdP = ws_ptr<float>(a.ws, L.dP);
   float* wdGK = ws_ptr<float>(a.ws, L.dGK);
@@ -641,7 +656,7 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
   if (stages & kStageCC) {
     prof_begin(st, "bwd_cc_simt");
     bwd_cc_simt<DK, DV, Tin><<<gridc, 256, s2, st>>>(k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, wu,
-                                                     wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs);
+                                                     wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs, only);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -649,7 +664,8 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
   prof_begin(st, "bwd_state_simt");
   bwd_state_simt<DK, DV, Tin><<<gridc, 256, s3, st>>>(q, k, v, a.beta, a.logf, dO, L.H, L.T,
                                                       L.NC, wu, wg, wS0, wdSC, waccq, wacck,
-                                                      waccL, waccv, L.tc ? 1 : 0);
+                                                      waccL, waccv, L.tc ? 1 : 0,
+                                                      L.tc ? ws_ptr<__nv_bfloat16>(a.ws, L.dSCb) : nullptr, only);
   prof_end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -79,13 +79,11 @@ struct ChainCfg {
   static constexpr uint32_t BYTES = SM_END + 1024;             // + alignment slack
 };
 
-// Writes 16 state values (row r, columns j..j+15) of one chunk into the two
-// bf16 tiles the backward's state-product MMAs read: "[r][j]" (rows r, K = j)
-// and "[j][r]" (rows j, K = r), both 128-byte-swizzled K-major, 32 KB each.
-__device__ __forceinline__ void save_bf16_tiles(__nv_bfloat16* rj, __nv_bfloat16* jr, size_t ch, int r, int j,
-                                                const float (&x)[16]) {
+// Writes 16 state values (row r, columns j..j+15) of one chunk into the bf16
+// tile the backward's MMAs read: [r][j] (rows r, K = j), 128-byte-swizzled
+// K-major, 32 KB.  The backward also reads it transposed, as an MN-major operand.
+__device__ __forceinline__ void save_bf16_tile(__nv_bfloat16* rj, size_t ch, int r, int j, const float (&x)[16]) {
   unsigned char* a = reinterpret_cast<unsigned char*>(rj + ch * D * D);
-  unsigned char* t = reinterpret_cast<unsigned char*>(jr + ch * D * D);
 #pragma unroll
   for (int h8 = 0; h8 < 2; ++h8) {
     __align__(16) __nv_bfloat16 v8[8];
@@ -93,9 +91,6 @@ __device__ __forceinline__ void save_bf16_tiles(__nv_bfloat16* rj, __nv_bfloat16
     for (int i = 0; i < 8; ++i) v8[i] = __float2bfloat16_rn(x[8 * h8 + i]);
     *reinterpret_cast<uint4*>(a + tc::sw128_off(r, j + 8 * h8, 128, 2)) = *reinterpret_cast<const uint4*>(v8);
   }
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    *reinterpret_cast<__nv_bfloat16*>(t + tc::sw128_off(j + i, r, 128, 2)) = __float2bfloat16_rn(x[i]);
 }
 
 // named barriers: 1 = the 4 chain warps, 2 = the 4 producer warps
@@ -122,7 +117,7 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
     const float* __restrict__ beta, const float* __restrict__ S0,
     float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy,
     const float* __restrict__ wA, float* __restrict__ wS0blob, float* __restrict__ wu,
-    float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, __nv_bfloat16* __restrict__ wS0bt,
+    float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b,
     int* __restrict__ err) {
   using Cf = ChainCfg<R>;
   constexpr int NJ = Cf::NJ;
@@ -263,7 +258,7 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
             *reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(blob) + tc::sw128_off(r, jg, 128, 4)) =
                 make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
           }
-          if (wS0b) save_bf16_tiles(wS0b, wS0bt, (size_t)unit * NC + n, r, j0 + jj, x);
+          if (wS0b) save_bf16_tile(wS0b, (size_t)unit * NC + n, r, j0 + jj, x);
         }
       }
       tc::tc_before_sync();
@@ -919,9 +914,8 @@ cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, flo
   cfg.numAttrs = 1;
   prof_begin(st, "fwd_chain_tc");
   __nv_bfloat16* s0b = a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0b) : nullptr;
-  __nv_bfloat16* s0bt = a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0bt) : nullptr;
   e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_k, tm_v, tm_logf, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy,
-                         wA, blob, wu, wb0, s0b, s0bt, err);
+                         wA, blob, wu, wb0, s0b, err);
   prof_end(st);
   return e;
 }

@@ -30,15 +30,19 @@ struct Layout {
   // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
   size_t S0 = 0, u = 0, b0 = 0, flags = 0;  // flags: one int per chunk (tensor-core path)
   // tensor-core path, saved for the backward: chunk-start states as bf16
-  // 128-byte-swizzled tiles, "[r][j]" (rows r, K = j) and "[j][r]"
-  size_t S0b = 0, S0bt = 0;
+  // 128-byte-swizzled K-major tiles [r][j] (rows r, K = j)
+  size_t S0b = 0;
   size_t fwd_save_bytes = 0;
   // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],
   // accq/acck/accL [ch][64][dk], accv [ch][64][dv]
   size_t dSC = 0, g = 0, dP = 0, dGK = 0, dGVs = 0, accq = 0, acck = 0, accL = 0, accv = 0;
   size_t du = 0;  // per-chunk intra-chunk part of du (tensor-core path) [ch][64]
-  size_t dSCb = 0, dSCbt = 0;  // tensor-core path: dS per chunk as bf16 tiles (as S0b, S0bt)
-  size_t bflags = 0;           // tensor-core path: one int per chunk (exact-path fallback)
+  size_t dSCb = 0;    // tensor-core path: dS per chunk as a bf16 tile (as S0b)
+  size_t bflags = 0;  // tensor-core path: one int per chunk (exact-path fallback)
+  // tensor-core path, chunk adjoints known before the reverse chain (bf16
+  // 128-byte-swizzled tiles): [dP; E_V] (128 x 64), P diag(u) and E_K
+  // (64 x 64 each); M u [ch][64]
+  size_t T1 = 0, PU = 0, EK = 0, Mu = 0;
   size_t bwd_bytes = 0;
 };
 
@@ -86,11 +90,14 @@ cudaError_t launch_fwd_prep(const FwdArgs& a, bool with_P, cudaStream_t st);
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st);
 int choose_cluster(int units, int sms);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st);
-// CUDA-core backward kernels by stage; `only` (nullable) restricts the intra
-// stage to chunks whose flag is set.
+// CUDA-core backward kernels by stage; `only` (nullable) restricts the
+// per-chunk stages (cc, state, intra) to chunks whose flag is set.
 constexpr int kStageChain = 1, kStageCC = 2, kStageState = 4, kStageIntra = 8, kStageAll = 15;
 cudaError_t launch_bwd_simt_stages(const BwdArgs& a, int stages, const int* only, cudaStream_t st);
 cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
+// per-chunk tensor-core kernels before / after the reverse chain (kd_bwd_chunk_tc.cu)
+cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st);
+cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st);
 
 template <typename T>
 inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }

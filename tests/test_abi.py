@@ -50,7 +50,7 @@ def test_workspace_sizes(L):
     assert f >= chunks * (64 + 64 * 64) * 4                      # y, A
     assert fs >= chunks * (64 + 2 * 64 * 64 + d * d + 2 * 64) * 4  # + P, chunk-start states, u, b0
     assert fs >= f
-    assert bw >= chunks * d * d * 2 * 2  # dS per chunk as two bf16 tiles
+    assert bw >= chunks * (d * d * 2 + 4 * 64 * 64 * 2)  # dS tile and the chunk adjoint tiles (bf16)
     # the fp32 path keeps the chunk-start states only when saving for the backward
     f32 = kd.workspace_size(kd.KD_WS_FWD, B, H, T, d, d, kd.KD_F32)
     assert kd.workspace_size(kd.KD_WS_FWD_SAVE, B, H, T, d, d, kd.KD_F32) >= f32 + chunks * d * d * 4

@@ -234,6 +234,25 @@ def test_bwd_extreme_decay(oracle, dtype, d):
               TOL_GRAD_F32 if dtype == "f32" else TOL_GRAD_BF16, oracle)
 
 
+def test_bwd_bf16_ragged_with_dST(oracle):
+    """Tensor-core backward with a nonzero final-state gradient and a ragged tail."""
+    inp = kin.make_inputs(4, B=1, H=3, T=130, seed=91)
+    dST = np.random.default_rng(5).standard_normal((1, 3, 128, 128)) / 128.0
+    check_bwd(inp, "bf16", TOL_BF16, TOL_GRAD_BF16, oracle, dST)
+
+
+def test_bwd_bf16_decay_bands(oracle):
+    """Heads whose in-chunk cumulative decay stays mild, reaches the 40..80
+    band (tensor-core pre-chain products, exact post-chain path) and goes
+    beyond it (exact path throughout)."""
+    inp = kin.make_inputs(4, B=1, H=3, T=200, seed=92)
+    lf = inp["logf"].copy()
+    lf[:, :, 1, :] = -0.9                     # |L| up to ~57 inside a chunk
+    lf[:, :, 2, :] = np.minimum(lf[:, :, 2, :] * 30.0, -1.5)  # |L| far beyond 80
+    inp["logf"] = kin.round_to_dtype(lf, "f32")
+    check_bwd(inp, "bf16", TOL_BF16, TOL_GRAD_BF16, oracle)
+
+
 def test_fwdbwd_workload_T16384_state_tracking(oracle):
     """Forward+backward workload: B=1, H=16, T=16384, d=128, beta in (0,2)."""
     check_bwd(kin.make_inputs(4), "bf16", TOL_BF16, TOL_GRAD_BF16, oracle)
