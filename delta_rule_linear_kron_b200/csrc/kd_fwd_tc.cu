@@ -448,115 +448,117 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
 }
 
 // ---------------------------------------------------------------------------
-// output kernel: O^T[r,t] = sum_j S0[r,j] Q+[t,j] + sum_i V[i,r] u_i P[t,i]
+// output kernel, one CTA per chunk:
+//   O^T[r,t] = sum_j S0[r,j] Q+[t,j] + sum_i V[i,r] u_i P[t,i],  P = tril(Q+ K-^T)
+// The state product and P run in tf32 (the state and the decays are fp32);
+// the intra-chunk product V^T (diag(u) P^T) in bf16 (V is bf16 already).
 // ---------------------------------------------------------------------------
 struct OutCfg {
-  static constexpr uint32_t S0 = 0;                     // S0 blob, tf32 SW128 [4 kb][128][128 B]
-  static constexpr uint32_t QK = S0 + 65536;            // [Q+ ; 0] tf32 SW128 [4 kb][128][128 B]
-  static constexpr uint32_t KM = QK + 65536;            // K- tf32 SW128 [4 kb][64][128 B]
-  static constexpr uint32_t VT = KM + 32768;            // V^T tf32 SW128 [2 kb][128][128 B]
-  static constexpr uint32_t B3 = VT + 32768;            // diag(u) P^T: tf32 SW128 [2 kb][64][128 B]
-  static constexpr uint32_t U = B3 + 16384;             // u [64]
-  static constexpr uint32_t END = U + 256;
-  static constexpr uint32_t BYTES = END + 1024;
+  static constexpr uint32_t S0 = 0;           // S0 blob, tf32 SW128 [4 kb][128][128 B]
+  static constexpr uint32_t QK = 65536;       // tf32 [Q+; K-]: per 32-channel K block rows 0-63 Q+, 64-127 K-
+  static constexpr uint32_t VB = 131072;      // V bf16 [i][r], 2 K blocks x 64 rows (TMA, 128-byte swizzle)
+  static constexpr uint32_t B3 = 147456;      // diag(u) P^T as bf16 [t][i], 64 rows x 64
+  static constexpr uint32_t QR = 155648;      // q bf16 [64][128] (TMA)
+  static constexpr uint32_t KR = 172032;      // k bf16 [64][128] (TMA)
+  static constexpr uint32_t LG = 188416;      // logf fp32 [64][128] (TMA)
+  static constexpr uint32_t U = 221184;       // u [64]
+  static constexpr uint32_t XCH = U + 256;    // prefix exchange [128]
+  static constexpr uint32_t BYTES = XCH + 512 + 1024;
+  static constexpr uint32_t LOAD_BYTES = 65536 + 16384 + 2 * 16384 + 32768 + 256;
+  static constexpr uint32_t OO = QK;          // output staging O bf16 [t][r] (after the MMAs)
 };
 
-__global__ void __launch_bounds__(128, 1) fwd_out_tc(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const float* __restrict__ logf, int H, int T, int NC,
-    const float* __restrict__ wS0blob, const float* __restrict__ wu, __nv_bfloat16* __restrict__ out,
-    int* __restrict__ unsafe_flags, int* __restrict__ err) {
+__global__ void __launch_bounds__(256, 1) fwd_out_tc(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_logf,
+    const __grid_constant__ CUtensorMap tm_out, int H, int NC, const float* __restrict__ wS0blob,
+    const float* __restrict__ wu, int* __restrict__ unsafe_flags, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
   __shared__ uint32_t tmem_slot;
-  __shared__ int unsafe, abort_flag;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
   const int b = unit / H, h = unit % H;
-  const int t0 = n * C, nv = min(C, T - t0);
+  const int t0 = n * C;
   const size_t ch = (size_t)unit * NC + n;
 
   if (tid == 0) {
     tc::mbar_init(&ld_bar, 1);
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
-    unsafe = 0;
     abort_flag = 0;
+    tc::mbar_expect_tx(&ld_bar, OutCfg::LOAD_BYTES);
+#pragma unroll
+    for (int part = 0; part < 4; ++part)
+      tc::bulk_g2s(sm + OutCfg::S0 + part * 16384, wS0blob + ch * D * D + part * 4096, 16384u, &ld_bar);
+    tc::tma_load_4d(sm + OutCfg::VB, &tm_v, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + OutCfg::VB + 8192, &tm_v, 64, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + OutCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + OutCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + OutCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
+    tc::bulk_g2s(sm + OutCfg::U, wu + ch * C, 256u, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
-  if (tid == 0) {
-    tc::mbar_expect_tx(&ld_bar, 65536u);
-#pragma unroll
-    for (int part = 0; part < 4; ++part)
-      tc::bulk_g2s(sm + OutCfg::S0 + part * 16384, wS0blob + ch * D * D + part * 4096, 16384u, &ld_bar);
-  }
-  float* us = reinterpret_cast<float*>(sm + OutCfg::U);
-  if (tid < C) us[tid] = wu[ch * C + tid];
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
 
-  // Q+ = q o gamma and K- = k / gamma (thread = key channel j); rows 64..127 of QK are zero
+  // Q+ = q o gamma, K- = k / gamma (tf32); thread (j, half) covers 32 positions
+  const int j = tid & 127, half = tid >> 7;
+  float mx = 0.f;
   {
-    const int j = tid;
-    float L = 0.f, mx = 0.f;
-#pragma unroll 4
-    for (int t = 0; t < C; ++t) {
-      const bool ok = t < nv;
-      const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
-      L += ok ? logf[g] : 0.f;
-      mx = fmaxf(mx, fabsf(L));
-      const float qq = ok ? __bfloat162float(q[g]) : 0.f, kk = ok ? __bfloat162float(k[g]) : 0.f;
-      *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = qq * expf(L);
-      *reinterpret_cast<float*>(sm + OutCfg::KM + tc::sw128_off(t, j, 64, 4)) = kk * expf(-L);
-    }
-    if (!(mx < kSafeLogRange)) atomicOr(&unsafe, 1);
-#pragma unroll 4
-    for (int t = 64; t < 128; ++t) *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = 0.f;
-  }
-  // V^T (tf32): thread = position t (two halves of r)
-  {
-    const int t = tid & 63, rh = tid >> 6;
-    const bool ok = t < nv;
-    const __nv_bfloat16* vrow = v + (((size_t)b * T + t0 + t) * H + h) * D;
-#pragma unroll 2
-    for (int r8 = 0; r8 < 64; r8 += 8) {
-      uint4 raw = make_uint4(0, 0, 0, 0);
-      if (ok) raw = *reinterpret_cast<const uint4*>(vrow + 64 * rh + r8);
-      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    float Lr[32];
+    const float* lg = reinterpret_cast<const float*>(sm + OutCfg::LG);
+    float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<float*>(sm + OutCfg::VT + tc::sw128_off(64 * rh + r8 + i, t, 128, 4)) =
-            __bfloat162float(e[i]);
+    for (int i = 0; i < 32; ++i) {
+      acc += lg[(32 * half + i) * D + j];
+      Lr[i] = acc;
+    }
+    float* xch = reinterpret_cast<float*>(sm + OutCfg::XCH);
+    if (half == 0) xch[j] = acc;
+    __syncthreads();
+    const float off = half ? xch[j] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = 32 * half + i;
+      const float L = Lr[i] + off;
+      mx = fmaxf(mx, fabsf(L));
+      const float qq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OutCfg::QR + (t * D + j) * 2));
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OutCfg::KR + (t * D + j) * 2));
+      *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = qq * expf(L);
+      *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(-L);
     }
   }
+  const bool is_unsafe = __syncthreads_or(!(mx < kSafeLogRange)) != 0;
   tc::fence_proxy_async();
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
-  const bool is_unsafe = unsafe != 0;
-  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
-  // MMA: D_P[t,i] (cols 0..63) = [Q+;0] K-^T ; D_O[r,t] (cols 64..127) = S0 Q+^T
+  // MMA: D_P[t,i] (cols 0..63, lanes 0..63) = [Q+; K-] K-^T ; D_O[r,t] (cols 64..127) = S0 Q+^T
   if (tid == 0) {
-    const uint32_t IDP = tc::idesc(128, 64, 2);
+    const uint32_t IDT = tc::idesc(128, 64, 2);
 #pragma unroll
     for (int ks = 0; ks < 16; ++ks) {
-      const uint32_t kb = ks / 4, within = (ks % 4) * 32;
-      const uint64_t qa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::QK + kb * 128 * 128 + within));
-      const uint64_t kmb = tc::desc_sw128(tc::smem_u32(sm + OutCfg::KM + kb * 64 * 128 + within));
-      const uint64_t sa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::S0 + kb * 128 * 128 + within));
-      tc::mma_tf32_ss(tmem + 0, qa, kmb, IDP, ks > 0 ? 1u : 0u);
-      tc::mma_tf32_ss(tmem + 64, sa, qa, IDP, ks > 0 ? 1u : 0u);
+      const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
+      const uint64_t qa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::QK + o));
+      const uint64_t kmb = tc::desc_sw128(tc::smem_u32(sm + OutCfg::QK + o + 8192));
+      const uint64_t sa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::S0 + o));
+      tc::mma_tf32_ss(tmem + 0, qa, kmb, IDT, ks > 0 ? 1u : 0u);
+      tc::mma_tf32_ss(tmem + 64, sa, qa, IDT, ks > 0 ? 1u : 0u);
     }
     tc::mma_commit(&mma_bar);
   }
   tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
-  // B3[t][i] = u_i P[t,i] for i <= t (rows t: warps 0-1 own TMEM lanes 0..63)
+  // B3[t][i] = u_i P[t,i] for i <= t (bf16; rows t: warps 0-1 own TMEM lanes 0..63)
   if (warp < 2) {
     const int t = tid;
+    const float* us = reinterpret_cast<const float*>(sm + OutCfg::U);
 #pragma unroll
     for (int c16 = 0; c16 < 4; ++c16) {
       float x[16];
@@ -565,8 +567,15 @@ __global__ void __launch_bounds__(128, 1) fwd_out_tc(
 #pragma unroll
       for (int i2 = 0; i2 < 16; ++i2) {
         const int i = 16 * c16 + i2;
-        const float pv = (i <= t && !is_unsafe) ? x[i2] * us[i] : 0.f;
-        *reinterpret_cast<float*>(sm + OutCfg::B3 + tc::sw128_off(t, i, 64, 4)) = pv;
+        x[i2] = (i <= t && !is_unsafe) ? x[i2] * us[i] : 0.f;
+      }
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        __align__(16) __nv_bfloat16 v8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v8[i] = __float2bfloat16_rn(x[8 * h8 + i]);
+        *reinterpret_cast<uint4*>(sm + OutCfg::B3 + tc::sw128_off(t, 16 * c16 + 8 * h8, 64, 2)) =
+            *reinterpret_cast<const uint4*>(v8);
       }
     }
   }
@@ -575,37 +584,45 @@ __global__ void __launch_bounds__(128, 1) fwd_out_tc(
   __syncthreads();
   tc::tc_after_sync();
   if (tid == 0) {
-    const uint32_t IDO = tc::idesc(128, 64, 2);
+    // D_O += V^T (diag(u) P^T): A = V as an MN-major operand (M = r, K = i)
+    const uint32_t IDO = tc::idesc(128, 64, 1) | (1u << 15);
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t kb = ks / 4, within = (ks % 4) * 32;
-      const uint64_t va = tc::desc_sw128(tc::smem_u32(sm + OutCfg::VT + kb * 128 * 128 + within));
-      const uint64_t pb = tc::desc_sw128(tc::smem_u32(sm + OutCfg::B3 + kb * 64 * 128 + within));
-      tc::mma_tf32_ss(tmem + 64, va, pb, IDO, 1u);
-    }
+    for (int ks = 0; ks < 4; ++ks)
+      tc::mma_bf16_ss(tmem + 64, tc::desc_sw128_mn(tc::smem_u32(sm + OutCfg::VB + ks * 2048), 8192u),
+                      tc::desc_sw128(tc::smem_u32(sm + OutCfg::B3 + ks * 32)), IDO, 1u);
     tc::mma_commit(&mma_bar);
   }
   tc::mbar_wait<false>(&mma_bar, 1, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
-  // O[t, r] from D_O lane r
-  {
-    const int r = tid;
+  if (!is_unsafe) {
+    // O[t, r] from D_O lane r (positions 32*half .. +31), staged as the bf16 tile of the TMA store
+    unsigned char* oo = sm + OutCfg::OO;
 #pragma unroll
-    for (int c16 = 0; c16 < 4; ++c16) {
+    for (int c16 = 0; c16 < 2; ++c16) {
       float x[16];
-      tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, 64 + 16 * c16), x);
+      const int tb = 32 * half + 16 * c16;
+      tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, 64 + tb), x);
       tc::tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = 16 * c16 + i;
-        if (t < nv) out[(((size_t)b * T + t0 + t) * H + h) * D + r] = __float2bfloat16_rn(x[i]);
-      }
+      for (int i = 0; i < 16; ++i)
+        *reinterpret_cast<__nv_bfloat16*>(oo + tc::sw128_off(tb + i, j, 64, 2)) = __float2bfloat16_rn(x[i]);
     }
+    tc::fence_proxy_async();
   }
-  if (tid == 0 && unsafe_flags) unsafe_flags[ch] = is_unsafe ? 1 : 0;
+  __syncthreads();
+  if (tid == 0) {
+    if (!is_unsafe) {
+      tc::tma_store_4d(&tm_out, sm + OutCfg::OO, 0, h, t0, b);
+      tc::tma_store_4d(&tm_out, sm + OutCfg::OO + 8192, 64, h, t0, b);
+      tc::bulk_commit();
+      tc::bulk_wait_read();
+    }
+    if (unsafe_flags) unsafe_flags[ch] = is_unsafe ? 1 : 0;
+  }
   tc::tc_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
+  (void)lane;
 }
 
 // Exact recomputation of O for chunks whose decay range is outside the
@@ -672,25 +689,29 @@ __global__ void __launch_bounds__(128) fwd_out_fixup(
 struct PrepCfg {
   static constexpr uint32_t AKQ = 0;        // [K+; Q+] tf32, 4 K blocks x 128 rows x 128 B
   static constexpr uint32_t BKM = 65536;    // K- tf32, 4 K blocks x 64 rows x 128 B
-  static constexpr uint32_t VT = 98304;     // V bf16, 2 K blocks x 128 rows x 128 B (rows 64..127 unused)
-  static constexpr uint32_t LS = 131072;    // L fp32 [64][129]
-  static constexpr uint32_t NS = LS + 64 * 129 * 4;   // N = diag(beta) M, fp32 [64][65]
+  static constexpr uint32_t VT = 98304;     // V bf16 [t][r], 2 K blocks x 64 rows (TMA, 128-byte swizzle);
+                                            // the Gram's M = 128 rows read 8 KB past a block (unused lanes)
+  static constexpr uint32_t QR = 114688;    // q bf16 [64][128] (TMA)
+  static constexpr uint32_t KR = 131072;    // k bf16 [64][128] (TMA)
+  static constexpr uint32_t LS = 147456;    // logf fp32 [64][128] (TMA), then L in place
+  static constexpr uint32_t NS = 180224;    // N = diag(beta) M, fp32 [64][65]
   static constexpr uint32_t XS = NS + 64 * 65 * 4;    // A, fp32 [64][65]
   static constexpr uint32_t TS = XS + 64 * 65 * 4;    // block temporaries [3][16][17]
-  static constexpr uint32_t SMALL = TS + 3 * 16 * 17 * 4;  // beta, c [64] each
-  static constexpr uint32_t BYTES = SMALL + 512 + 1024;
+  static constexpr uint32_t SMALL = TS + 3 * 16 * 17 * 4;  // beta, c [64] each; prefix exchange [128]
+  static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
+  static constexpr uint32_t LOAD_BYTES = 16384 + 2 * 16384 + 32768;
 };
 
 __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
-    const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ q,
-    const __nv_bfloat16* __restrict__ k, const float* __restrict__ beta, const float* __restrict__ c,
-    const float* __restrict__ logf, int H, int T, int NC, float* __restrict__ wy, float* __restrict__ wA,
-    float* __restrict__ wP, int* __restrict__ err) {
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf,
+    const float* __restrict__ beta, const float* __restrict__ c, int H, int T, int NC, float* __restrict__ wy,
+    float* __restrict__ wA, float* __restrict__ wP, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
   __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag, unsafe;
+  __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
   const int b = unit / H, h = unit % H;
@@ -702,50 +723,63 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
   float* Ts = reinterpret_cast<float*>(sm + PrepCfg::TS);
   float* bs = reinterpret_cast<float*>(sm + PrepCfg::SMALL);
   float* cs = bs + 64;
+  float* xch = cs + 64;
 
   if (tid == 0) {
     tc::mbar_init(&ld_bar, 1);
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    unsafe = 0;
-    tc::mbar_expect_tx(&ld_bar, 16384u);
+    tc::mbar_expect_tx(&ld_bar, PrepCfg::LOAD_BYTES);
     tc::tma_load_4d(sm + PrepCfg::VT, &tm_v, 0, h, t0, b, &ld_bar);
-    tc::tma_load_4d(sm + PrepCfg::VT + 16384, &tm_v, 64, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PrepCfg::VT + 8192, &tm_v, 64, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PrepCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PrepCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PrepCfg::LS, &tm_logf, 0, h, t0, b, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  if (tid < C) {
+    const bool ok = tid < nv;
+    const size_t g = ((size_t)b * T + t0 + tid) * H + h;
+    bs[tid] = ok ? beta[g] : 0.f;
+    cs[tid] = ok ? c[g] : 0.f;
+  }
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
-  if (tid < 128) {
-    const int j = tid;
-    float L = 0.f, mx = 0.f;
-#pragma unroll 4
-    for (int t = 0; t < C; ++t) {
-      const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
-      const bool ok = t < nv;
-      L += ok ? logf[g] : 0.f;
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  // decay prefix (thread (j, half) covers 32 positions; L is written back for
+  // the exact path) and the tf32 operands K+, Q+, K-
+  float mx = 0.f;
+  {
+    const int j = tid & 127, half = tid >> 7;
+    float Lr[32];
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      acc += Ls[(32 * half + i) * D + j];
+      Lr[i] = acc;
+    }
+    if (half == 0) xch[j] = acc;
+    __syncthreads();
+    const float off = half ? xch[j] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = 32 * half + i;
+      const float L = Lr[i] + off;
       mx = fmaxf(mx, fabsf(L));
-      Ls[t * 129 + j] = L;
-      const float qq = ok ? __bfloat162float(q[g]) : 0.f, kk = ok ? __bfloat162float(k[g]) : 0.f;
+      Ls[t * D + j] = L;
+      const float qq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::QR + (t * D + j) * 2));
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::KR + (t * D + j) * 2));
       const float gm = expf(L), ig = expf(-L);
       *reinterpret_cast<float*>(sm + PrepCfg::AKQ + tc::sw128_off(t, j, 128, 4)) = kk * gm;
       *reinterpret_cast<float*>(sm + PrepCfg::AKQ + tc::sw128_off(64 + t, j, 128, 4)) = qq * gm;
       *reinterpret_cast<float*>(sm + PrepCfg::BKM + tc::sw128_off(t, j, 64, 4)) = kk * ig;
     }
-    if (!(mx < kSafeLogRange)) atomicOr(&unsafe, 1);
-  } else {
-    const int i = tid - 128;
-    if (i < C) {
-      const bool ok = i < nv;
-      const size_t g = ((size_t)b * T + t0 + i) * H + h;
-      bs[i] = ok ? beta[g] : 0.f;
-      cs[i] = ok ? c[g] : 0.f;
-    }
   }
+  const bool is_unsafe = __syncthreads_or(!(mx < kSafeLogRange)) != 0;
   tc::fence_proxy_async();
-  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
@@ -759,15 +793,13 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     }
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
-      const uint64_t vd = tc::desc_sw128(tc::smem_u32(sm + PrepCfg::VT + o));
+      const uint64_t vd = tc::desc_sw128(tc::smem_u32(sm + PrepCfg::VT + (ks / 4) * 8192 + (ks % 4) * 32));
       tc::mma_bf16_ss(tmem + 64, vd, vd, IDB, ks > 0 ? 1u : 0u);
     }
     tc::mma_commit(&mma_bar);
   }
   tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
-  const bool is_unsafe = unsafe != 0;
   // rows t (TMEM lanes 0..63): N[t][i] = beta_t G_K G_V (i < t); lanes 64+t: P row t
   if (warp < 4) {
     const int row = warp * 32 + lane;
@@ -811,22 +843,21 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
   __syncthreads();
   if (is_unsafe) {
     // exact decay weights e^{L_t - L_i} <= 1 per element (rare: extreme decays)
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::QR);
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::KR);
     for (int e = tid; e < C * C; e += 256) {
       const int t = e / C, i = e % C;
       float gk = 0.f, gv = 0.f, pq = 0.f;
       if (i <= t) {
-        const size_t gt = (((size_t)b * T + t0 + t) * H + h) * D, gi = (((size_t)b * T + t0 + i) * H + h) * D;
-        const bool okt = t < nv, oki = i < nv;
         for (int j = 0; j < D; ++j) {
-          const float w = expf(Ls[t * 129 + j] - Ls[i * 129 + j]);
-          const float kt = okt ? __bfloat162float(k[gt + j]) : 0.f, ki = oki ? __bfloat162float(k[gi + j]) : 0.f;
-          const float qt = okt ? __bfloat162float(q[gt + j]) : 0.f;
-          gk = fmaf(kt * ki, w, gk);
-          pq = fmaf(qt * ki, w, pq);
+          const float w = expf(Ls[t * D + j] - Ls[i * D + j]);
+          const float ki = __bfloat162float(ks[i * D + j]);
+          gk = fmaf(__bfloat162float(ks[t * D + j]) * ki, w, gk);
+          pq = fmaf(__bfloat162float(qs[t * D + j]) * ki, w, pq);
         }
         for (int r = 0; r < D; ++r)
-          gv = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::VT + tc::sw128_off(t, r, 128, 2) + 0 * 0)),
-                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::VT + tc::sw128_off(i, r, 128, 2))), gv);
+          gv = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::VT + tc::sw128_off(t, r, 64, 2))),
+                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + PrepCfg::VT + tc::sw128_off(i, r, 64, 2))), gv);
       }
       Ns[t * 65 + i] = i < t ? bs[t] * gk * gv : 0.f;
       if (wP) wP[ch * C * C + e] = i <= t ? pq : 0.f;
@@ -958,15 +989,18 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
   const Layout& L = a.L;
   cudaError_t e;
   {
-    CUtensorMap tm_v;
-    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true)) return cudaErrorInvalidValue;
+    CUtensorMap tm_v, tm_q, tm_k, tm_logf;
+    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
+        !make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false))
+      return cudaErrorInvalidValue;
     if ((e = cudaFuncSetAttribute(fwd_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)PrepCfg::BYTES)) != cudaSuccess)
       return e;
     prof_begin(st, "fwd_prep_tc");
     fwd_prep_tc<<<(unsigned)L.chunks, 256, PrepCfg::BYTES, st>>>(
-        tm_v, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.beta, a.c,
-        a.logf, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
+        tm_v, tm_q, tm_k, tm_logf, a.beta, a.c, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
         a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -984,13 +1018,20 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
   if ((e = cudaFuncSetAttribute(fwd_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)OutCfg::BYTES)) != cudaSuccess)
     return e;
-  prof_begin(st, "fwd_out_tc");
-  fwd_out_tc<<<(unsigned)L.chunks, 128, OutCfg::BYTES, st>>>(
-      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-      static_cast<const __nv_bfloat16*>(a.v), a.logf, L.H, L.T, L.NC, blob, wu,
-      static_cast<__nv_bfloat16*>(a.out), flags, err);
-  prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    CUtensorMap tm_q, tm_k, tm_v, tm_logf, tm_out;
+    if (!make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
+        !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_out, a.out, 2, L.B, L.T, L.H, D, 64, true))
+      return cudaErrorInvalidValue;
+    prof_begin(st, "fwd_out_tc");
+    fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, blob,
+                                                               wu, flags, err);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   constexpr int kFixSmem = (3 * C * (D + 1) + C) * 4;
   if ((e = cudaFuncSetAttribute(fwd_out_fixup, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem)) !=
       cudaSuccess)
