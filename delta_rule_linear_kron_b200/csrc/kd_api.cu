@@ -61,6 +61,12 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->y = take(chunks * C * 4);
   L->A = take(chunks * C * C * 4);
   L->P = take(chunks * C * C * 4);  // tensor-core path: written only when saving for the backward
+  if (L->tc) {
+    L->Hx = take(chunks * C * C * 4);
+    L->Kt = take((size_t)B * T * H * dk * 4);
+    L->Ke = take((size_t)B * T * H * dk * 4);
+    L->GC = take(chunks * (size_t)dk * 4);
+  }
   L->fwd_bytes = off;
   L->S0 = take(chunks * (size_t)dv * dk * 4);
   L->u = take(chunks * C * 4);

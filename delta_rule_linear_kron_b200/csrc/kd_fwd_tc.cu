@@ -42,40 +42,33 @@ constexpr int D = 128;
 template <int R>
 struct ChainCfg {
   static constexpr int NJ = D / R;                    // key channels per CTA
-  static constexpr int KB1 = (NJ * 4 + 127) / 128;    // 128-byte K blocks of the K+ slice
-  static constexpr int TPC = 128 / NJ;                // producer scan threads per channel
-  static constexpr int SEG = C / TPC;                 // positions per scan thread
-  static constexpr int KES = NJ + 1;                  // padded row of K^e (fp32)
-  // tensor memory columns: X (64), state slice, two halves of the update
-  static constexpr int D1_COL = 0, S_COL = 64, D2A_COL = 64 + NJ, D2B_COL = 64 + 2 * NJ;
-  static constexpr uint32_t TMEM_COLS = (64 + 3 * NJ) <= 128 ? 128u : 256u;
+  static constexpr int KBJ = (R == 8) ? 2 : 0;        // K steps of the K~ block that precede this CTA's channels (odd R=8 ranks)
+  // tensor memory columns: X' (64), state slice, update
+  static constexpr int D1_COL = 0, S_COL = 64, D2_COL = 64 + NJ;
+  static constexpr uint32_t TMEM_COLS = (64 + 2 * NJ) <= 128 ? 128u : 256u;
   static constexpr uint32_t up1k(uint32_t x) { return (x + 1023u) / 1024u * 1024u; }
-  // operand buffer (two, by chunk parity), built by the producer warps
-  static constexpr uint32_t OP_B1 = 0;                         // K+ slice: tf32 SW128, 64 rows
-  static constexpr uint32_t OP_A2 = OP_B1 + KB1 * 8192;        // V^T: tf32 SW128, 128 rows, K = 64
-  static constexpr uint32_t OP_KE = OP_A2 + 32768;             // K^e slice fp32 [64][KES]
-  static constexpr uint32_t OP_GC = OP_KE + 64 * KES * 4;      // gamma_C slice [NJ]
-  static constexpr uint32_t OP_SZ = up1k(OP_GC + NJ * 4);
-  // raw staging (two, by chunk parity), written by TMA / bulk copies
-  static constexpr uint32_t ST_V = 0;                          // v bf16 [64][128]
-  static constexpr uint32_t ST_A = 16384;                      // A fp32 [64][64]
-  static constexpr uint32_t ST_Y = 32768;                      // y [64]
-  static constexpr uint32_t ST_K = ST_Y + 256;                 // k slice bf16 [64][NJ]
-  static constexpr uint32_t ST_L = ST_K + 64 * NJ * 2;         // logf slice fp32 [64][NJ]
-  static constexpr uint32_t ST_SZ = up1k(ST_L + 64 * NJ * 4);
-  static constexpr uint32_t LOAD_BYTES = 16384 + 16384 + 256 + 64 * NJ * 6;
-  static constexpr uint32_t OPS = 0, STG = OPS + 2 * OP_SZ;
-  static constexpr uint32_t B2 = STG + 2 * ST_SZ;              // diag(u) K^e: tf32 SW128, NJ rows, K = 64
+  // chunk slot (ring of three), all written by TMA / bulk copies
+  static constexpr uint32_t SL_V = 0;                          // V bf16 [t][r], 128-byte swizzle, 2 x 8 KB
+  static constexpr uint32_t SL_B1 = 16384;                     // K~, the 32-channel block holding this CTA's channels:
+                                                               //   tf32 [t][32], 128-byte swizzle (8 KB)
+  static constexpr uint32_t SL_KE = SL_B1 + 8192;              // K^e slice fp32 [64][NJ]
+  static constexpr uint32_t SL_GC = SL_KE + 64 * NJ * 4;       // gamma_C slice [NJ]
+  static constexpr uint32_t SL_Y = SL_GC + 128;                // y [64]
+  static constexpr uint32_t SL_SZ = up1k(SL_Y + 256);
+  static constexpr uint32_t LOAD_BYTES = 16384 + 8192 + 64 * NJ * 4 + NJ * 4 + 256;
+  // per-chunk matrices of the u recursion (ring of two): A, H
+  static constexpr uint32_t AUX = 3 * SL_SZ;
+  static constexpr uint32_t AUX_SZ = 32768;
+  static constexpr uint32_t B2 = AUX + 2 * AUX_SZ;             // diag(u) K^e slice, bf16 hi / lo, NJ rows x 128 B each
   static constexpr uint32_t SM = B2 + 2 * NJ * 128;            // small arrays (floats)
-  static constexpr uint32_t SM_BS = SM;                        // beta [2][64]
-  static constexpr uint32_t SM_W = SM_BS + 2 * 64 * 4;         // beta o b0 [64]
-  static constexpr uint32_t SM_U = SM_W + 64 * 4;              // u [64]
-  static constexpr uint32_t SM_UP = SM_U + 64 * 4;             // u partial sums [2][64]
-  static constexpr uint32_t SM_MINE = SM_UP + 2 * 64 * 4;      // own b0 partial [64]
+  static constexpr uint32_t SM_BS = SM;                        // beta [3][64]
+  static constexpr uint32_t SM_W = SM_BS + 3 * 64 * 4;         // beta o b0 [64]
+  static constexpr uint32_t SM_U = SM_W + 64 * 4;              // u [64] (previous chunk's until replaced)
+  static constexpr uint32_t SM_UP = SM_U + 64 * 4;             // partial sums [2][64]
+  static constexpr uint32_t SM_MINE = SM_UP + 2 * 64 * 4;      // own c partial [64]
   static constexpr uint32_t SM_XRED = SM_MINE + 64 * 4;        // per-warp partials [4][64]
   static constexpr uint32_t SM_RECV = SM_XRED + 4 * 64 * 4;    // [2][R][64]
-  static constexpr uint32_t SM_SEG = SM_RECV + 2 * R * 64 * 4; // scan segment sums [TPC][NJ]
-  static constexpr uint32_t SM_END = SM_SEG + TPC * NJ * 4;
+  static constexpr uint32_t SM_END = SM_RECV + 2 * R * 64 * 4;
   static constexpr uint32_t BYTES = SM_END + 1024;             // + alignment slack
 };
 
@@ -93,37 +86,49 @@ __device__ __forceinline__ void save_bf16_tile(__nv_bfloat16* rj, size_t ch, int
   }
 }
 
-// named barriers: 1 = the 4 chain warps, 2 = the 4 producer warps
+// named barriers: 1 = the 4 chain warps, 2 = the 4 producer warps;
+// 3 = chain -> issuer "update operand ready", 4 = chain -> issuer "state updated"
+// (the chain warps arrive, the issuer warp waits: 160 threads)
 __device__ __forceinline__ void bar_chain() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void bar_prod() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_arrive_issuer(int id) { asm volatile("bar.arrive %0, 160;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void bar_wait_chain(int id) { asm volatile("bar.sync %0, 160;" ::"r"(id) : "memory"); }
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(b)) : "memory");
 }
 
-// Warp roles (256 threads):
-//   warps 0-3  chain: MMAs, the b0 column sums, the cluster all-reduce, u,
-//              the state update; thread r owns tensor-memory lane r.
-//   warps 4-7  producer: issues the TMA / bulk loads, builds the next chunk's
-//              MMA operands (decay prefix, K+, K^e, V^T), saves each
-//              chunk-start state slice to global memory.
-// Hand-offs (mbarriers, one arrival each): raw_full (loads landed),
-// op_full (operands of a chunk built), free (chain done with a chunk's
-// buffers), s_ready (state of chunk n in tensor memory), s_saved (producer
-// has read it).
+// The chain with a one-chunk lookahead.  With c_{n+1} = rowdot(V_{n+1}, S_n K~_{n+1}^T),
+// K~_{n+1} = K+_{n+1} diag(gamma_C of chunk n), and the cross-chunk matrix
+// H_{n+1} = (V_{n+1} V_n^T) o (K+_{n+1} K^e_n^T) (fwd_cross_tc):
+//   b0_{n+1} = rowdot(V_{n+1}, S_{n+1} K+_{n+1}^T) = c_{n+1} + H_{n+1} u_n,
+// so c_{n+1} (an MMA on the state, a column dot and the cluster all-reduce)
+// is formed while u_n and the update of chunk n proceed; only two 64 x 64
+// matrix-vector products separate u_n from u_{n+1}.
+//
+// Warp roles (288 threads):
+//   warps 0-3  chain: u, the update operand, the column dots, the cluster
+//              all-reduce, the state update; thread r owns tensor-memory lane r.
+//   warps 4-7  producer: TMA / bulk loads of each chunk's operands (built by
+//              fwd_cross_tc) into a ring of three slots, A and H into a ring
+//              of two, and the save of each chunk-start state slice.
+//   warp 8     issuer: one thread issues every tcgen05 MMA.
+// Hand-offs: mbarriers raw_full (a slot's loads landed), slot_free (chain done
+// with a slot), aux_full / aux_free (A, H), s_ready (state of chunk n in
+// tensor memory), s_saved (producer has read it), mma1 / mma2 (MMA done);
+// named barriers 3 and 4 (chain -> issuer).
 template <int R>
-__global__ void __launch_bounds__(256, 1) fwd_chain_tc(
-    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-    const __grid_constant__ CUtensorMap tm_logf,
-    const float* __restrict__ beta, const float* __restrict__ S0,
-    float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy,
-    const float* __restrict__ wA, float* __restrict__ wS0blob, float* __restrict__ wu,
-    float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b,
-    int* __restrict__ err) {
+__global__ void __launch_bounds__(288, 1) fwd_chain_tc(
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+    const __grid_constant__ CUtensorMap tm_ke, const float* __restrict__ beta, const float* __restrict__ S0,
+    float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy, const float* __restrict__ wA,
+    const float* __restrict__ wHx, const float* __restrict__ wGC, float* __restrict__ wS0blob,
+    float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, int* __restrict__ err) {
   using Cf = ChainCfg<R>;
   constexpr int NJ = Cf::NJ;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ uint64_t raw_full[2], op_full[2], freeb[2], s_ready, s_saved, x_bar[2], mma_bar;
+  __shared__ uint64_t raw_full[3], slot_free[3], aux_full[2], aux_free[2], s_ready, s_saved, x_bar[2], mma1_bar,
+      mma2_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -132,6 +137,7 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
   const int unit = blockIdx.x / R;  // (b, h)
   const int b = unit / H, h = unit % H;
   const int j0 = static_cast<int>(rank) * NJ;
+  const int jb = j0 & ~31;  // first channel of the 32-channel K~ block
 
   float* bs = reinterpret_cast<float*>(sm + Cf::SM_BS);
   float* ws = reinterpret_cast<float*>(sm + Cf::SM_W);
@@ -140,18 +146,22 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
   float* mine = reinterpret_cast<float*>(sm + Cf::SM_MINE);
   float* xred = reinterpret_cast<float*>(sm + Cf::SM_XRED);
   float* recv = reinterpret_cast<float*>(sm + Cf::SM_RECV);
-  float* segs = reinterpret_cast<float*>(sm + Cf::SM_SEG);
+  auto slot = [&](int m) { return sm + (m % 3) * Cf::SL_SZ; };
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       tc::mbar_init(&raw_full[i], 1);
-      tc::mbar_init(&op_full[i], 1);
-      tc::mbar_init(&freeb[i], 1);
+      tc::mbar_init(&slot_free[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&aux_full[i], 1);
+      tc::mbar_init(&aux_free[i], 1);
       tc::mbar_init(&x_bar[i], 1);
     }
     tc::mbar_init(&s_ready, 1);
     tc::mbar_init(&s_saved, 1);
-    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init(&mma1_bar, 1);
+    tc::mbar_init(&mma2_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
   }
@@ -163,89 +173,100 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
   const uint32_t tmem = tmem_slot;
   const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);  // lanes 32*(warp%4) ..
 
-  if (warp >= 4) {
+  if (warp == 8) {
+    // ============================== issuer warp ==============================
+    const uint32_t ID1 = tc::idesc(128, 64, 2);
+    const uint32_t ID2 = tc::idesc(128, NJ, 1) | (1u << 15);  // bf16, A (V^T) MN-major
+    // X' = S K~_m^T  (M = 128 rows r, N = 64 positions, K = NJ; A = the state in tensor memory)
+    auto issue_x = [&](int m) {
+      tc::mbar_wait<false>(&raw_full[m % 3], (uint32_t)((m / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      tc::tc_after_sync();
+      if (lane == 0) {
+        const unsigned char* st = slot(m);
+#pragma unroll
+        for (int ks = 0; ks < NJ / 8; ++ks) {
+          const uint64_t bd = tc::desc_sw128(tc::smem_u32(st + Cf::SL_B1 + (Cf::KBJ * (rank & 1) + ks) * 32));
+          tc::mma_tf32_ts(tmem + Cf::D1_COL, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&mma1_bar);
+      }
+      __syncwarp();
+    };
+    bar_wait_chain(4);  // S_0 in tensor memory
+    tc::tc_after_sync();
+    issue_x(0);
+    for (int n = 0; n < NC; ++n) {
+      if (n + 1 < NC) {
+        if (n >= 1) {
+          bar_wait_chain(4);  // S_n in tensor memory (update of chunk n-1 done)
+          tc::tc_after_sync();
+        }
+        issue_x(n + 1);
+      }
+      bar_wait_chain(3);  // update operand of chunk n built
+      tc::tc_after_sync();
+      if (lane == 0) {
+        const unsigned char* st = slot(n);
+        // dS = V_n^T (B2hi + B2lo)^T  (M = 128 rows r, N = NJ, K = 64 positions)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = tc::desc_sw128_mn(tc::smem_u32(st + Cf::SL_V + ks * 2048), 8192u);
+          tc::mma_bf16_ss(tmem + Cf::D2_COL, ad, tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + ks * 32)), ID2,
+                          ks > 0 ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + Cf::D2_COL, ad, tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + NJ * 128 + ks * 32)),
+                          ID2, 1u);
+        }
+        tc::mma_commit(&mma2_bar);
+      }
+      __syncwarp();
+    }
+  } else if (warp >= 4) {
     // =========================== producer warps ===========================
     const int p = tid - 128;
-    auto issue = [&](int n) {
-      unsigned char* st = sm + Cf::STG + (n & 1) * Cf::ST_SZ;
-      uint64_t* bar = &raw_full[n & 1];
-      const size_t ch = (size_t)unit * NC + n;
-      tc::fence_proxy_async();
-      tc::mbar_expect_tx(bar, Cf::LOAD_BYTES);
-      tc::tma_load_4d(st + Cf::ST_V, &tm_v, 0, h, n * C, b, bar);
-      tc::tma_load_4d(st + Cf::ST_K, &tm_k, j0, h, n * C, b, bar);
-      tc::tma_load_4d(st + Cf::ST_L, &tm_logf, j0, h, n * C, b, bar);
-      tc::bulk_g2s(st + Cf::ST_A, wA + ch * C * C, 64u * 64u * 4u, bar);
-      tc::bulk_g2s(st + Cf::ST_Y, wy + ch * C, 256u, bar);
+    // the operands of chunk m into its slot (chunk m - 3 must be done)
+    auto prepare = [&](int m) {
+      unsigned char* st = slot(m);
+      const int si = m % 3;
+      if (m >= 3)
+        tc::mbar_wait<false>(&slot_free[si], (uint32_t)((m / 3 - 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
+      if (p == 0) {
+        uint64_t* bar = &raw_full[si];
+        const size_t ch = (size_t)unit * NC + m;
+        tc::fence_proxy_async();
+        tc::mbar_expect_tx(bar, Cf::LOAD_BYTES);
+        tc::tma_load_4d(st + Cf::SL_V, &tm_v, 0, h, m * C, b, bar);
+        tc::tma_load_4d(st + Cf::SL_V + 8192, &tm_v, 64, h, m * C, b, bar);
+        tc::tma_load_4d(st + Cf::SL_B1, &tm_kt, jb, h, m * C, b, bar);
+        tc::tma_load_4d(st + Cf::SL_KE, &tm_ke, j0, h, m * C, b, bar);
+        tc::bulk_g2s(st + Cf::SL_GC, wGC + ch * D + j0, NJ * 4u, bar);
+        tc::bulk_g2s(st + Cf::SL_Y, wy + ch * C, 256u, bar);
+      }
+      if (p < C) bs[si * 64 + p] = (m * C + p < T) ? beta[((size_t)b * T + m * C + p) * H + h] : 0.f;
     };
-    if (p == 0) {
-      issue(0);
-      if (NC > 1) issue(1);
-    }
-    for (int n = 0; n < NC; ++n) {
-      const int pb = n & 1;
-      unsigned char* st = sm + Cf::STG + pb * Cf::ST_SZ;
-      unsigned char* op = sm + Cf::OPS + pb * Cf::OP_SZ;
-      if (n >= 2) {
-        // the chain has finished chunk n-2: both buffers of this parity are free
-        tc::mbar_wait<false>(&freeb[pb], (uint32_t)(((n - 2) >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
-        if (p == 0) issue(n);
-      }
-      const float bt = (p < C && n * C + p < T) ? beta[((size_t)b * T + n * C + p) * H + h] : 0.f;
-      tc::mbar_wait<false>(&raw_full[pb], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
-      if (p < C) bs[pb * 64 + p] = bt;
-      // V^T as tf32 (thread = position t, half of the value channels)
-      {
-        const int t = p & 63, rh = p >> 6;
-#pragma unroll 2
-        for (int r8 = 0; r8 < 64; r8 += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(st + Cf::ST_V + t * 256 + (64 * rh + r8) * 2);
-          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            *reinterpret_cast<float*>(op + Cf::OP_A2 + tc::sw128_off(64 * rh + r8 + i, t, 128, 4)) =
-                __bfloat162float(e[i]);
-        }
-      }
-      // decay prefix of the slice, K+ (B operand of MMA 1), K^e, gamma_C
-      {
-        const int j = p % NJ, seg = p / NJ;
-        const float* lrow = reinterpret_cast<const float*>(st + Cf::ST_L);
-        float lp[Cf::SEG];
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < Cf::SEG; ++i) {
-          acc += lrow[(seg * Cf::SEG + i) * NJ + j];
-          lp[i] = acc;
-        }
-        segs[seg * NJ + j] = acc;
-        bar_prod();
-        float pre = 0.f, tot = 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < Cf::TPC; ++s2) {
-          const float x = segs[s2 * NJ + j];
-          if (s2 < seg) pre += x;
-          tot += x;
-        }
-        float* KE = reinterpret_cast<float*>(op + Cf::OP_KE);
-        if (seg == 0) reinterpret_cast<float*>(op + Cf::OP_GC)[j] = expf(tot);
-#pragma unroll
-        for (int i = 0; i < Cf::SEG; ++i) {
-          const int t = seg * Cf::SEG + i;
-          const float L = pre + lp[i];
-          const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(st + Cf::ST_K + (t * NJ + j) * 2));
-          *reinterpret_cast<float*>(op + Cf::OP_B1 + tc::sw128_off(t, j, 64, 4)) = kk * expf(L);
-          KE[t * Cf::KES + j] = kk * expf(tot - L);
-        }
-      }
+    // A and H of chunk m (chunk m - 2 must have consumed its buffer)
+    auto aux = [&](int m) {
+      if (p != 0) return;
+      const int ai = m & 1;
+      if (m >= 2)
+        tc::mbar_wait<false>(&aux_free[ai], (uint32_t)(((m - 2) >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
+      unsigned char* ax = sm + Cf::AUX + ai * Cf::AUX_SZ;
+      const size_t ch = (size_t)unit * NC + m;
       tc::fence_proxy_async();
-      bar_prod();
-      if (p == 0) mbar_arrive(&op_full[pb]);
-      // save the chunk-start state slice once the chain has it in tensor memory
-      tc::mbar_wait<false>(&s_ready, (uint32_t)(n & 1), err, tc::kErrTimeoutMma, &abort_flag);
+      tc::mbar_expect_tx(&aux_full[ai], m >= 1 ? 32768u : 16384u);
+      tc::bulk_g2s(ax, wA + ch * C * C, 16384u, &aux_full[ai]);
+      if (m >= 1) tc::bulk_g2s(ax + 16384, wHx + ch * C * C, 16384u, &aux_full[ai]);
+    };
+    prepare(0);
+    aux(0);
+    if (NC > 1) prepare(1);
+    for (int m = 0; m < NC; ++m) {
+      if (m + 2 < NC) prepare(m + 2);
+      if (m + 1 < NC) aux(m + 1);
+      // save the chunk-start state slice of chunk m once the chain has it in tensor memory
+      tc::mbar_wait<false>(&s_ready, (uint32_t)(m & 1), err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
       {
-        float* blob = wS0blob + ((size_t)unit * NC + n) * D * D;
+        float* blob = wS0blob + ((size_t)unit * NC + m) * D * D;
         const int r = p;
 #pragma unroll
         for (int jj = 0; jj < NJ; jj += 16) {
@@ -258,7 +279,7 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
             *reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(blob) + tc::sw128_off(r, jg, 128, 4)) =
                 make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
           }
-          if (wS0b) save_bf16_tile(wS0b, (size_t)unit * NC + n, r, j0 + jj, x);
+          if (wS0b) save_bf16_tile(wS0b, (size_t)unit * NC + m, r, j0 + jj, x);
         }
       }
       tc::tc_before_sync();
@@ -280,30 +301,14 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
       tc::tc_before_sync();
       bar_chain();
       if (tid == 0) mbar_arrive(&s_ready);
+      bar_arrive_issuer(4);
     }
-    int mma_par = 0;
-    const uint32_t ID1 = tc::idesc(128, 64, 2);
-    const uint32_t ID2 = tc::idesc(128, NJ, 2);
-    for (int n = 0; n < NC; ++n) {
-      const int pb = n & 1;
-      const unsigned char* st = sm + Cf::STG + pb * Cf::ST_SZ;
-      const unsigned char* op = sm + Cf::OPS + pb * Cf::OP_SZ;
-      const size_t ch = (size_t)unit * NC + n;
-      tc::mbar_wait<false>(&op_full[pb], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+    int mma1_par = 0, mma2_par = 0;
+    // c_m partial: sum_r V_m[t,r] X'[r,t] over this CTA's rows, then all-reduce over the cluster
+    auto column_dot_send = [&](int m) {
+      tc::mbar_wait<false>(&mma1_bar, (uint32_t)mma1_par, err, tc::kErrTimeoutMma, &abort_flag);
+      mma1_par ^= 1;
       tc::tc_after_sync();
-      // ---- MMA 1: X_c = S[:,J_c] K+[:,J_c]^T  (M=128 rows r, N=64 positions, K=NJ)
-      if (tid == 0) {
-#pragma unroll
-        for (int ks = 0; ks < NJ / 8; ++ks) {
-          const uint64_t bd = tc::desc_sw128(tc::smem_u32(op + Cf::OP_B1 + (ks / 4) * 8192 + (ks % 4) * 32));
-          tc::mma_tf32_ts(tmem + Cf::D1_COL, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&mma_bar);
-      }
-      tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
-      mma_par ^= 1;
-      tc::tc_after_sync();
-      // ---- b0_c[t] = sum_r V[t,r] X_c[r,t]
       {
         float x[64];
 #pragma unroll
@@ -314,46 +319,71 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
           for (int i = 0; i < 16; ++i) x[16 * c16 + i] = y16[i];
         }
         tc::tmem_ld_wait();
-        const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(st + Cf::ST_V) + r;
+        const unsigned char* vt = slot(m) + Cf::SL_V;
         float lo[32], hi[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          lo[t] = x[t] * __bfloat162float(vcol[t * 128]);
-          hi[t] = x[32 + t] * __bfloat162float(vcol[(32 + t) * 128]);
+          lo[t] = x[t] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + tc::sw128_off(t, r, 64, 2)));
+          hi[t] = x[32 + t] *
+                  __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + tc::sw128_off(32 + t, r, 64, 2)));
         }
         warp_transpose_reduce<32>(lo, lane);
         warp_transpose_reduce<32>(hi, lane);
         xred[warp * 64 + lane] = lo[0];
         xred[warp * 64 + 32 + lane] = hi[0];
       }
+      tc::tc_before_sync();
       bar_chain();
       if (tid < C) mine[tid] = xred[tid] + xred[64 + tid] + xred[128 + tid] + xred[192 + tid];
       bar_chain();
-      // ---- b0 = sum over the cluster of b0_c (fixed order in every CTA)
-      {
-        float* rv = recv + pb * R * 64;
-        if (tid == 0) tc::mbar_expect_tx(&x_bar[pb], R * 64u * 4u);
-        if (tid < 16 * R) {
-          const int peer = tid / 16, q4 = tid % 16;
-          const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
-          const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
-          const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[pb]), (uint32_t)peer);
-          tc::st_async_v4(raddr, val, rbar);
-        }
-        tc::mbar_wait<true>(&x_bar[pb], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
-        if (tid < C) {
-          float s = 0.f;
+      const int xb = m & 1;
+      float* rv = recv + xb * R * 64;
+      if (tid == 0) tc::mbar_expect_tx(&x_bar[xb], R * 64u * 4u);
+      if (tid < 16 * R) {
+        const int peer = tid / 16, q4 = tid % 16;
+        const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
+        const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
+        const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[xb]), (uint32_t)peer);
+        tc::st_async_v4(raddr, val, rbar);
+      }
+    };
+    column_dot_send(0);
+    for (int n = 0; n < NC; ++n) {
+      const unsigned char* st = slot(n);
+      const size_t ch = (size_t)unit * NC + n;
+      // ---- b0_n = c_n + H_n u_{n-1};  u_n = y_n - A_n (beta o b0_n)
+      tc::mbar_wait<true>(&x_bar[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
+      tc::mbar_wait<false>(&aux_full[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      const float* Am = reinterpret_cast<const float*>(sm + Cf::AUX + (n & 1) * Cf::AUX_SZ);
+      const float* Hm = Am + C * C;
+      const int t = tid & 63, half = tid >> 6;
+      if (n > 0) {
+        const float* Hrow = Hm + t * 64 + 32 * half;
+        const float* uh = us + 32 * half;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-          for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + tid];
-          ws[tid] = bs[pb * 64 + tid] * s;
-          if (rank == 0 && wb0) wb0[ch * C + tid] = s;
+        for (int i = 0; i < 32; i += 4) {
+          const int i0 = (i + t) & 31, i1 = (i + 1 + t) & 31, i2 = (i + 2 + t) & 31, i3 = (i + 3 + t) & 31;
+          a0 = fmaf(Hrow[i0], uh[i0], a0);
+          a1 = fmaf(Hrow[i1], uh[i1], a1);
+          a2 = fmaf(Hrow[i2], uh[i2], a2);
+          a3 = fmaf(Hrow[i3], uh[i3], a3);
         }
+        up[half * 64 + t] = (a0 + a1) + (a2 + a3);
       }
       bar_chain();
-      // ---- u = y - A (beta o b0): two threads per position, rotated reads
+      if (tid < C) {
+        const float* rv = recv + (n & 1) * R * 64;
+        float s = 0.f;
+#pragma unroll
+        for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + tid];
+        if (n > 0) s += up[tid] + up[64 + tid];
+        ws[tid] = bs[(n % 3) * 64 + tid] * s;
+        if (rank == 0 && wb0) wb0[ch * C + tid] = s;
+      }
+      bar_chain();
       {
-        const int t = tid & 63, half = tid >> 6;
-        const float* Arow = reinterpret_cast<const float*>(st + Cf::ST_A) + t * 64 + 32 * half;
+        const float* Arow = Am + t * 64 + 32 * half;
         const float* wh = ws + 32 * half;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
@@ -368,56 +398,54 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
       }
       bar_chain();
       if (tid < C) {
-        const float u = reinterpret_cast<const float*>(st + Cf::ST_Y)[tid] - (up[tid] + up[64 + tid]);
+        const float u = reinterpret_cast<const float*>(st + Cf::SL_Y)[tid] - (up[tid] + up[64 + tid]);
         us[tid] = u;
         if (rank == 0 && wu) wu[ch * C + tid] = u;
       }
       bar_chain();
-      // ---- B2 = diag(u) K^e[:, J_c]  (N = NJ rows j, K = 64 positions)
+      if (tid == 0) mbar_arrive(&aux_free[n & 1]);
+      // ---- B2 = diag(u_n) K^e_n slice as bf16 hi + lo (N = NJ rows j, K = 64 positions):
+      //      thread (channel jl, 64/TQ consecutive positions) writes 16-byte pieces of row jl
       {
-        const int t = tid & 63, jh = tid >> 6;
-        const float u = us[t];
-        const float* KE = reinterpret_cast<const float*>(op + Cf::OP_KE);
+        constexpr int TQ = 128 / NJ, TPT = C / TQ;  // position groups, positions per thread
+        const int jl = tid % NJ, tq = tid / NJ;
+        const float* KE = reinterpret_cast<const float*>(st + Cf::SL_KE);
 #pragma unroll
-        for (int i = 0; i < NJ / 2; ++i) {
-          const int j = jh * (NJ / 2) + i;
-          *reinterpret_cast<float*>(sm + Cf::B2 + tc::sw128_off(j, t, NJ, 4)) = u * KE[t * Cf::KES + j];
+        for (int g8 = 0; g8 < TPT; g8 += 8) {
+          __align__(16) __nv_bfloat16 hi8[8], lo8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int tt = tq * TPT + g8 + i;
+            const float x = us[tt] * KE[tt * NJ + jl];
+            hi8[i] = __float2bfloat16_rn(x);
+            lo8[i] = __float2bfloat16_rn(x - __bfloat162float(hi8[i]));
+          }
+          const uint32_t off = tc::sw128_off(jl, tq * TPT + g8, NJ, 2);
+          *reinterpret_cast<uint4*>(sm + Cf::B2 + off) = *reinterpret_cast<const uint4*>(hi8);
+          *reinterpret_cast<uint4*>(sm + Cf::B2 + NJ * 128 + off) = *reinterpret_cast<const uint4*>(lo8);
         }
       }
       tc::fence_proxy_async();
       tc::tc_before_sync();
-      bar_chain();
-      tc::tc_after_sync();
-      // ---- MMA 2: dS_c = V^T B2 as two independent K halves (M=128, N=NJ)
-      if (tid == 0) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t a0 = tc::desc_sw128(tc::smem_u32(op + Cf::OP_A2 + ks * 32));
-          const uint64_t b0d = tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + ks * 32));
-          const uint64_t a1 = tc::desc_sw128(tc::smem_u32(op + Cf::OP_A2 + 128 * 128 + ks * 32));
-          const uint64_t b1d = tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + NJ * 128 + ks * 32));
-          tc::mma_tf32_ss(tmem + Cf::D2A_COL, a0, b0d, ID2, ks > 0 ? 1u : 0u);
-          tc::mma_tf32_ss(tmem + Cf::D2B_COL, a1, b1d, ID2, ks > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&mma_bar);
-      }
-      tc::mbar_wait<false>(&mma_bar, (uint32_t)mma_par, err, tc::kErrTimeoutMma, &abort_flag);
-      mma_par ^= 1;
+      bar_arrive_issuer(3);
+      // ---- c_{n+1} from X' (its all-reduce overlaps the update)
+      if (n + 1 < NC) column_dot_send(n + 1);
+      tc::mbar_wait<false>(&mma2_bar, (uint32_t)mma2_par, err, tc::kErrTimeoutMma, &abort_flag);
+      mma2_par ^= 1;
       // the producer must have saved this chunk's start state before it changes
       tc::mbar_wait<false>(&s_saved, (uint32_t)(n & 1), err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
       // ---- S <- S diag(gamma_C) + dS
       {
-        const float* gC = reinterpret_cast<const float*>(op + Cf::OP_GC);
+        const float* gC = reinterpret_cast<const float*>(st + Cf::SL_GC);
 #pragma unroll
         for (int jj = 0; jj < NJ; jj += 16) {
-          float s[16], da[16], db[16];
+          float s[16], d2[16];
           tc::tmem_ld16(my_lanes + Cf::S_COL + jj, s);
-          tc::tmem_ld16(my_lanes + Cf::D2A_COL + jj, da);
-          tc::tmem_ld16(my_lanes + Cf::D2B_COL + jj, db);
+          tc::tmem_ld16(my_lanes + Cf::D2_COL + jj, d2);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], da[i] + db[i]);
+          for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], d2[i]);
           tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
         }
         tc::tmem_st_wait();
@@ -425,9 +453,10 @@ __global__ void __launch_bounds__(256, 1) fwd_chain_tc(
       tc::tc_before_sync();
       bar_chain();
       if (tid == 0) {
-        mbar_arrive(&freeb[pb]);
+        mbar_arrive(&slot_free[n % 3]);
         mbar_arrive(&s_ready);
       }
+      if (n + 2 < NC) bar_arrive_issuer(4);
     }
     if (ST) {
       tc::tc_after_sync();
@@ -918,22 +947,181 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
 }
 
+// ---------------------------------------------------------------------------
+// Per-chunk operands of the chain, one CTA per chunk n, all chunks in parallel:
+//   K~_n  = k_n o e^{L_n + Lambda_{n-1}}   (B of the chain's lookahead MMA)
+//   K^e_n = k_n o e^{Lambda_n - L_n}       (update operand),  gamma_C,n = e^{Lambda_n}
+// and, for n >= 1, the cross-chunk matrix of the lookahead
+//   H_n = (V_n V_{n-1}^T) o (K+_n K^e_{n-1}^T),   K+_n = k_n o e^{L_n}.
+// Every factor is bounded by |k| (the exponents are <= 0), so all chunks take
+// this path.  The key Gram runs in tf32, the value Gram in bf16 (exact
+// products, fp32 sums).
+// ---------------------------------------------------------------------------
+struct CrossCfg {
+  static constexpr uint32_t KK = 0;        // tf32 per 32-channel K block (16 KB): rows 0-63 K+_n, 64-127 K^e_{n-1}
+  static constexpr uint32_t VV = 65536;    // bf16, 2 K blocks x 128 rows: rows 0-63 V_n, 64-127 V_{n-1} (TMA)
+  static constexpr uint32_t KR = 98304;    // k_n, k_{n-1} bf16 [64][128] each (TMA)
+  static constexpr uint32_t LG = 131072;   // logf_n, then K~_n staged in place; logf_{n-1}, then K^e_n (fp32 [64][128])
+  static constexpr uint32_t XCH = 196608;  // Lambda_{n-1} [128]
+  static constexpr uint32_t BYTES = XCH + 512 + 1024;
+  static constexpr uint32_t LOAD_CUR = 16384 + 16384 + 32768, LOAD_PREV = LOAD_CUR;
+};
+
+__global__ void __launch_bounds__(256, 1) fwd_cross_tc(
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_logf, const __grid_constant__ CUtensorMap tm_kt,
+    const __grid_constant__ CUtensorMap tm_ke, int H, int NC, float* __restrict__ wGC, float* __restrict__ wHx,
+    int* __restrict__ err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar, mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, tp = t0 - C;
+  const bool has_prev = n > 0;
+  const size_t ch = blockIdx.x;
+  float* xch = reinterpret_cast<float*>(sm + CrossCfg::XCH);
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+    tc::mbar_expect_tx(&ld_bar, CrossCfg::LOAD_CUR + (has_prev ? CrossCfg::LOAD_PREV : 0u));
+    tc::tma_load_4d(sm + CrossCfg::VV, &tm_v, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CrossCfg::VV + 16384, &tm_v, 64, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CrossCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CrossCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
+    if (has_prev) {
+      tc::tma_load_4d(sm + CrossCfg::VV + 8192, &tm_v, 0, h, tp, b, &ld_bar);
+      tc::tma_load_4d(sm + CrossCfg::VV + 24576, &tm_v, 64, h, tp, b, &ld_bar);
+      tc::tma_load_4d(sm + CrossCfg::KR + 16384, &tm_k, 0, h, tp, b, &ld_bar);
+      tc::tma_load_4d(sm + CrossCfg::LG + 32768, &tm_logf, 0, h, tp, b, &ld_bar);
+    }
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  // half 0: chunk n (channel j); half 1: chunk n-1 (channel j)
+  const int j = tid & 127, half = tid >> 7;
+  float* lg = reinterpret_cast<float*>(sm + CrossCfg::LG + half * 32768);
+  const unsigned char* kr = sm + CrossCfg::KR + half * 16384;
+  float tot = 0.f;
+  if (half == 0 || has_prev) {
+#pragma unroll 8
+    for (int t = 0; t < C; ++t) tot += lg[t * D + j];
+  }
+  if (half) xch[j] = has_prev ? tot : 0.f;
+  __syncthreads();
+  float Lr[C];
+  if (half == 0) {
+    // K+_n (Gram operand, tf32) and K~_n (staged in place of logf_n)
+    const float lam_prev = xch[j];
+    float L = 0.f;
+#pragma unroll
+    for (int t = 0; t < C; ++t) {
+      L += lg[t * D + j];
+      Lr[t] = L;
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kr + (t * D + j) * 2));
+      const float kp = kk * expf(L);
+      *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(t, j, 128, 4)) = kp;
+      lg[t * D + j] = kk * expf(L + lam_prev);
+    }
+    wGC[ch * D + j] = expf(tot);
+  } else if (has_prev) {
+    // K^e_{n-1} (Gram operand, tf32)
+    float L = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < C; ++t) {
+      L += lg[t * D + j];
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kr + (t * D + j) * 2));
+      *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(tot - L);
+    }
+  }
+  __syncthreads();  // logf_{n-1} is dead: K^e_n goes there
+  if (half == 0) {
+    float* ke = reinterpret_cast<float*>(sm + CrossCfg::LG + 32768);
+#pragma unroll
+    for (int t = 0; t < C; ++t) {
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kr + (t * D + j) * 2));
+      ke[t * D + j] = kk * expf(tot - Lr[t]);
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    tc::tma_store_4d(&tm_kt, sm + CrossCfg::LG, 0, h, t0, b);
+    tc::tma_store_4d(&tm_ke, sm + CrossCfg::LG + 32768, 0, h, t0, b);
+    tc::bulk_commit();
+    if (has_prev) {
+      const uint32_t IDT = tc::idesc(128, 64, 2), IDB = tc::idesc(128, 64, 1);
+      // cols 0-63, lanes 0-63: K+_n K^e_{n-1}^T
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
+        tc::mma_tf32_ss(tmem + 0, tc::desc_sw128(tc::smem_u32(sm + CrossCfg::KK + o)),
+                        tc::desc_sw128(tc::smem_u32(sm + CrossCfg::KK + o + 8192)), IDT, ks > 0 ? 1u : 0u);
+      }
+      // cols 64-127, lanes 0-63: V_n V_{n-1}^T
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
+        tc::mma_bf16_ss(tmem + 64, tc::desc_sw128(tc::smem_u32(sm + CrossCfg::VV + o)),
+                        tc::desc_sw128(tc::smem_u32(sm + CrossCfg::VV + o + 8192)), IDB, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&mma_bar);
+    }
+  }
+  if (has_prev) {
+    tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+    tc::tc_after_sync();
+    if (warp < 2) {
+      const int t = warp * 32 + lane;
+      const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, 0);
+      float* hrow = wHx + ch * C * C + t * C;
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float gk[16], gv[16];
+        tc::tmem_ld16(lanes + 16 * c16, gk);
+        tc::tmem_ld16(lanes + 64 + 16 * c16, gv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4)
+          *reinterpret_cast<float4*>(hrow + 16 * c16 + 4 * i4) =
+              make_float4(gk[4 * i4] * gv[4 * i4], gk[4 * i4 + 1] * gv[4 * i4 + 1], gk[4 * i4 + 2] * gv[4 * i4 + 2],
+                          gk[4 * i4 + 3] * gv[4 * i4 + 3]);
+      }
+    }
+  }
+  if (tid == 0) tc::bulk_wait_read();
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
 template <int R>
 cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, float* blob, float* wu,
                          float* wb0, int* err, cudaStream_t st) {
   const Layout& L = a.L;
   constexpr int NJ = ChainCfg<R>::NJ;
-  CUtensorMap tm_k, tm_v, tm_logf;
-  if (!make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, NJ, false) ||
-      !make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 128, false) ||
-      !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, NJ, false))
+  CUtensorMap tm_v, tm_kt, tm_ke;
+  if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
+      !make_tmap_bthd(&tm_kt, ws_ptr<float>(a.ws, L.Kt), 4, L.B, L.T, L.H, D, 32, true) ||
+      !make_tmap_bthd(&tm_ke, ws_ptr<float>(a.ws, L.Ke), 4, L.B, L.T, L.H, D, NJ, false))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_chain_tc<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)ChainCfg<R>::BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L.B * L.H * R);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(288);
   cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -945,8 +1133,9 @@ cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, flo
   cfg.numAttrs = 1;
   prof_begin(st, "fwd_chain_tc");
   __nv_bfloat16* s0b = a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0b) : nullptr;
-  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_k, tm_v, tm_logf, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy,
-                         wA, blob, wu, wb0, s0b, err);
+  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_v, tm_kt, tm_ke, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy, wA,
+                         (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC), blob, wu,
+                         wb0, s0b, err);
   prof_end(st);
   return e;
 }
@@ -960,7 +1149,7 @@ static int max_active_clusters() {
     return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(R * 1024);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(288);
   cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1002,6 +1191,23 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     fwd_prep_tc<<<(unsigned)L.chunks, 256, PrepCfg::BYTES, st>>>(
         tm_v, tm_q, tm_k, tm_logf, a.beta, a.c, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
         a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, err);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    CUtensorMap tm_v, tm_k, tm_logf, tm_kt, tm_ke;
+    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
+        !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_kt, ws_ptr<float>(a.ws, L.Kt), 4, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_ke, ws_ptr<float>(a.ws, L.Ke), 4, L.B, L.T, L.H, D, 128, false))
+      return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(fwd_cross_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)CrossCfg::BYTES)) != cudaSuccess)
+      return e;
+    prof_begin(st, "fwd_cross_tc");
+    fwd_cross_tc<<<(unsigned)L.chunks, 256, CrossCfg::BYTES, st>>>(
+        tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx), err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
