@@ -66,6 +66,7 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
     L->Kt = take((size_t)B * T * H * dk * 4);
     L->Ke = take((size_t)B * T * H * dk * 4);
     L->GC = take(chunks * (size_t)dk * 4);
+    L->Vt = take(chunks * (size_t)dv * C * 2);
   }
   L->fwd_bytes = off;
   L->S0 = take(chunks * (size_t)dv * dk * 4);

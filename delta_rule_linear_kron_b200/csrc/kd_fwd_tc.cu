@@ -48,7 +48,7 @@ struct ChainCfg {
   static constexpr uint32_t TMEM_COLS = (64 + 2 * NJ) <= 128 ? 128u : 256u;
   static constexpr uint32_t up1k(uint32_t x) { return (x + 1023u) / 1024u * 1024u; }
   // chunk slot (ring of three), all written by TMA / bulk copies
-  static constexpr uint32_t SL_V = 0;                          // V bf16 [t][r], 128-byte swizzle, 2 x 8 KB
+  static constexpr uint32_t SL_V = 0;                          // V^T bf16 [r][t], K-major, 128-byte swizzle (16 KB)
   static constexpr uint32_t SL_B1 = 16384;                     // K~, the 32-channel block holding this CTA's channels:
                                                                //   tf32 [t][32], 128-byte swizzle (8 KB)
   static constexpr uint32_t SL_KE = SL_B1 + 8192;              // K^e slice fp32 [64][NJ]
@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
     const __grid_constant__ CUtensorMap tm_ke, const float* __restrict__ beta, const float* __restrict__ S0,
     float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy, const float* __restrict__ wA,
-    const float* __restrict__ wHx, const float* __restrict__ wGC, float* __restrict__ wS0blob,
+    const float* __restrict__ wHx, const float* __restrict__ wGC, const __nv_bfloat16* __restrict__ wVt,
+    float* __restrict__ wS0blob,
     float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, int* __restrict__ err) {
   using Cf = ChainCfg<R>;
   constexpr int NJ = Cf::NJ;
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
   if (warp == 8) {
     // ============================== issuer warp ==============================
     const uint32_t ID1 = tc::idesc(128, 64, 2);
-    const uint32_t ID2 = tc::idesc(128, NJ, 1) | (1u << 15);  // bf16, A (V^T) MN-major
+    const uint32_t ID2 = tc::idesc(128, NJ, 1);  // bf16, both K-major
     // X' = S K~_m^T  (M = 128 rows r, N = 64 positions, K = NJ; A = the state in tensor memory)
     auto issue_x = [&](int m) {
       tc::mbar_wait<false>(&raw_full[m % 3], (uint32_t)((m / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
         // dS = V_n^T (B2hi + B2lo)^T  (M = 128 rows r, N = NJ, K = 64 positions)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = tc::desc_sw128_mn(tc::smem_u32(st + Cf::SL_V + ks * 2048), 8192u);
+          const uint64_t ad = tc::desc_sw128(tc::smem_u32(st + Cf::SL_V + ks * 32));
           tc::mma_bf16_ss(tmem + Cf::D2_COL, ad, tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + ks * 32)), ID2,
                           ks > 0 ? 1u : 0u);
           tc::mma_bf16_ss(tmem + Cf::D2_COL, ad, tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + NJ * 128 + ks * 32)),
@@ -234,8 +235,7 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
         const size_t ch = (size_t)unit * NC + m;
         tc::fence_proxy_async();
         tc::mbar_expect_tx(bar, Cf::LOAD_BYTES);
-        tc::tma_load_4d(st + Cf::SL_V, &tm_v, 0, h, m * C, b, bar);
-        tc::tma_load_4d(st + Cf::SL_V + 8192, &tm_v, 64, h, m * C, b, bar);
+        tc::bulk_g2s(st + Cf::SL_V, wVt + ch * (D * C), 16384u, bar);
         tc::tma_load_4d(st + Cf::SL_B1, &tm_kt, jb, h, m * C, b, bar);
         tc::tma_load_4d(st + Cf::SL_KE, &tm_ke, j0, h, m * C, b, bar);
         tc::bulk_g2s(st + Cf::SL_GC, wGC + ch * D + j0, NJ * 4u, bar);
@@ -319,13 +319,18 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
           for (int i = 0; i < 16; ++i) x[16 * c16 + i] = y16[i];
         }
         tc::tmem_ld_wait();
-        const unsigned char* vt = slot(m) + Cf::SL_V;
+        const unsigned char* vt = slot(m) + Cf::SL_V;  // row r of V^T: V[t, r] for t = 0..63
         float lo[32], hi[32];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          lo[t] = x[t] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + tc::sw128_off(t, r, 64, 2)));
-          hi[t] = x[32 + t] *
-                  __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + tc::sw128_off(32 + t, r, 64, 2)));
+        for (int g8 = 0; g8 < 8; ++g8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(vt + tc::sw128_off(r, 8 * g8, 128, 2));
+          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int t = 8 * g8 + i;
+            if (t < 32) lo[t] = x[t] * __bfloat162float(e[i]);
+            else hi[t - 32] = x[t] * __bfloat162float(e[i]);
+          }
         }
         warp_transpose_reduce<32>(lo, lane);
         warp_transpose_reduce<32>(hi, lane);
@@ -356,51 +361,58 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
       tc::mbar_wait<false>(&aux_full[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
       const float* Am = reinterpret_cast<const float*>(sm + Cf::AUX + (n & 1) * Cf::AUX_SZ);
       const float* Hm = Am + C * C;
-      const int t = tid & 63, half = tid >> 6;
+      // two threads per position t (lanes 2t', 2t'+1 of a warp), halves of i, rotated reads
+      const int t = tid >> 1, half = tid & 1;
+      const int rot = t + 16 * half;
+      float s = 0.f;
+      {
+        const float* rv = recv + (n & 1) * R * 64;
+#pragma unroll
+        for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + t];
+      }
       if (n > 0) {
         const float* Hrow = Hm + t * 64 + 32 * half;
         const float* uh = us + 32 * half;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          const int i0 = (i + t) & 31, i1 = (i + 1 + t) & 31, i2 = (i + 2 + t) & 31, i3 = (i + 3 + t) & 31;
+          const int i0 = (i + rot) & 31, i1 = (i + 1 + rot) & 31, i2 = (i + 2 + rot) & 31, i3 = (i + 3 + rot) & 31;
           a0 = fmaf(Hrow[i0], uh[i0], a0);
           a1 = fmaf(Hrow[i1], uh[i1], a1);
           a2 = fmaf(Hrow[i2], uh[i2], a2);
           a3 = fmaf(Hrow[i3], uh[i3], a3);
         }
-        up[half * 64 + t] = (a0 + a1) + (a2 + a3);
+        float hu = (a0 + a1) + (a2 + a3);
+        hu += __shfl_xor_sync(0xffffffffu, hu, 1);
+        s += hu;
+      }
+      // s = b0_n[t] in both threads of the pair
+      if (half == 0) {
+        ws[t] = bs[(n % 3) * 64 + t] * s;
+        if (rank == 0 && wb0) wb0[ch * C + t] = s;
       }
       bar_chain();
-      if (tid < C) {
-        const float* rv = recv + (n & 1) * R * 64;
-        float s = 0.f;
-#pragma unroll
-        for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + tid];
-        if (n > 0) s += up[tid] + up[64 + tid];
-        ws[tid] = bs[(n % 3) * 64 + tid] * s;
-        if (rank == 0 && wb0) wb0[ch * C + tid] = s;
-      }
-      bar_chain();
+      float uval;
       {
         const float* Arow = Am + t * 64 + 32 * half;
         const float* wh = ws + 32 * half;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          const int i0 = (i + t) & 31, i1 = (i + 1 + t) & 31, i2 = (i + 2 + t) & 31, i3 = (i + 3 + t) & 31;
+          const int i0 = (i + rot) & 31, i1 = (i + 1 + rot) & 31, i2 = (i + 2 + rot) & 31, i3 = (i + 3 + rot) & 31;
           a0 = fmaf(Arow[i0], wh[i0], a0);
           a1 = fmaf(Arow[i1], wh[i1], a1);
           a2 = fmaf(Arow[i2], wh[i2], a2);
           a3 = fmaf(Arow[i3], wh[i3], a3);
         }
-        up[half * 64 + t] = (a0 + a1) + (a2 + a3);
+        float aw = (a0 + a1) + (a2 + a3);
+        aw += __shfl_xor_sync(0xffffffffu, aw, 1);
+        uval = reinterpret_cast<const float*>(st + Cf::SL_Y)[t] - aw;
       }
-      bar_chain();
-      if (tid < C) {
-        const float u = reinterpret_cast<const float*>(st + Cf::SL_Y)[tid] - (up[tid] + up[64 + tid]);
-        us[tid] = u;
-        if (rank == 0 && wu) wu[ch * C + tid] = u;
+      bar_chain();  // every thread has read u_{n-1} (us) and w
+      if (half == 0) {
+        us[t] = uval;
+        if (rank == 0 && wu) wu[ch * C + t] = uval;
       }
       bar_chain();
       if (tid == 0) mbar_arrive(&aux_free[n & 1]);
@@ -963,7 +975,8 @@ struct CrossCfg {
   static constexpr uint32_t KR = 98304;    // k_n, k_{n-1} bf16 [64][128] each (TMA)
   static constexpr uint32_t LG = 131072;   // logf_n, then K~_n staged in place; logf_{n-1}, then K^e_n (fp32 [64][128])
   static constexpr uint32_t XCH = 196608;  // Lambda_{n-1} [128]
-  static constexpr uint32_t BYTES = XCH + 512 + 1024;
+  static constexpr uint32_t VT = 197632;   // V_n^T bf16 [r][t], 128 rows x 128 B, 128-byte swizzle (staging)
+  static constexpr uint32_t BYTES = VT + 16384 + 1024;
   static constexpr uint32_t LOAD_CUR = 16384 + 16384 + 32768, LOAD_PREV = LOAD_CUR;
 };
 
@@ -971,7 +984,7 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_logf, const __grid_constant__ CUtensorMap tm_kt,
     const __grid_constant__ CUtensorMap tm_ke, int H, int NC, float* __restrict__ wGC, float* __restrict__ wHx,
-    int* __restrict__ err) {
+    __nv_bfloat16* __restrict__ wVt, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -1043,6 +1056,19 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
       *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(tot - L);
     }
   }
+  // V_n^T as the K-major tile [r][t] the chain's column dot and update MMA read
+  {
+    const int r = tid & 127, tb = 32 * (tid >> 7);
+#pragma unroll
+    for (int g8 = 0; g8 < 32; g8 += 8) {
+      __align__(16) __nv_bfloat16 v8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        v8[i] = *reinterpret_cast<const __nv_bfloat16*>(sm + CrossCfg::VV + tc::sw128_off(tb + g8 + i, r, 128, 2));
+      *reinterpret_cast<uint4*>(sm + CrossCfg::VT + tc::sw128_off(r, tb + g8, 128, 2)) =
+          *reinterpret_cast<const uint4*>(v8);
+    }
+  }
   __syncthreads();  // logf_{n-1} is dead: K^e_n goes there
   if (half == 0) {
     float* ke = reinterpret_cast<float*>(sm + CrossCfg::LG + 32768);
@@ -1059,6 +1085,7 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
   if (tid == 0) {
     tc::tma_store_4d(&tm_kt, sm + CrossCfg::LG, 0, h, t0, b);
     tc::tma_store_4d(&tm_ke, sm + CrossCfg::LG + 32768, 0, h, t0, b);
+    tc::bulk_s2g(wVt + ch * (D * C), sm + CrossCfg::VT, 16384u);
     tc::bulk_commit();
     if (has_prev) {
       const uint32_t IDT = tc::idesc(128, 64, 2), IDB = tc::idesc(128, 64, 1);
@@ -1134,8 +1161,8 @@ cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, flo
   prof_begin(st, "fwd_chain_tc");
   __nv_bfloat16* s0b = a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0b) : nullptr;
   e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_v, tm_kt, tm_ke, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy, wA,
-                         (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC), blob, wu,
-                         wb0, s0b, err);
+                         (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC),
+                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt), blob, wu, wb0, s0b, err);
   prof_end(st);
   return e;
 }
@@ -1207,7 +1234,8 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
       return e;
     prof_begin(st, "fwd_cross_tc");
     fwd_cross_tc<<<(unsigned)L.chunks, 256, CrossCfg::BYTES, st>>>(
-        tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx), err);
+        tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx),
+        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -26,8 +26,8 @@ struct Layout {
   size_t chunks = 0;      // B * H * NC
   // forward scratch (always): y [ch][64], A [ch][64][64], P [ch][64][64];
   // tensor-core path, operands of the chain: cross-chunk matrix Hx [ch][64][64],
-  // K~ and K^e [B][T][H][dk] (fp32), gamma_C [ch][dk]
-  size_t y = 0, A = 0, P = 0, Hx = 0, Kt = 0, Ke = 0, GC = 0;
+  // K~ and K^e [B][T][H][dk] (fp32), gamma_C [ch][dk], V^T [ch][dv][64] (bf16 tile)
+  size_t y = 0, A = 0, P = 0, Hx = 0, Kt = 0, Ke = 0, GC = 0, Vt = 0;
   size_t fwd_bytes = 0;
   // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
   size_t S0 = 0, u = 0, b0 = 0, flags = 0;  // flags: one int per chunk (tensor-core path)

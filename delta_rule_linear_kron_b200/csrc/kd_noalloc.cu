@@ -12,10 +12,11 @@
 // Limits and behaviour:
 //   * The scratch is a file-scope device array of kNoAllocScratchBytes
 //     (32 MiB).  Every GPU that loads the library holds it until the process
-//     exits.  A problem whose forward scratch exceeds it is rejected with
-//     KD_ERR_WORKSPACE before anything is enqueued: more than 184 chunk-heads
-//     (B * H * ceil(T/64)) on the tensor-core path (bf16, dk = dv = 128, whose
-//     chain also keeps per-token operands), more than 1016 on the others.
+//     exits.  A problem whose forward scratch (kron_delta_workspace_size with
+//     KD_WS_FWD) exceeds it is rejected with KD_ERR_WORKSPACE before anything
+//     is enqueued: beyond 169 chunk-heads (B * H * ceil(T/64)) on the
+//     tensor-core path (bf16, dk = dv = 128, whose chain also keeps per-token
+//     operands there), beyond 1016 on the others.
 //   * All calls share the one array and it keeps the last call's contents.
 //     The forward writes every scratch element it later reads, so nothing
 //     has to start at zero.  Calls whose kernels overlap on the GPU (other
@@ -79,9 +80,8 @@ int kron_delta_fwd_noalloc(const void* q, const void* k, const void* v, const fl
   if (need > kNoAllocScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof(msg),
-             "kron_delta_fwd_noalloc: forward scratch of %zu bytes exceeds the fixed %zu-byte array "
-             "(B*H*ceil(T/64) must be <= 184 for bf16 with dk = dv = 128, <= 1016 otherwise); use "
-             "kron_delta_fwd with a workspace",
+             "kron_delta_fwd_noalloc: forward scratch of %zu bytes exceeds the fixed %zu-byte array; "
+             "use kron_delta_fwd with a workspace",
              need, kNoAllocScratchBytes);
     kd::set_error(msg);
     return KD_ERR_WORKSPACE;

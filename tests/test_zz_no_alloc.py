@@ -25,14 +25,18 @@ def _p(t):
 def test_rejects_problems_beyond_the_fixed_scratch():
     L = kd.lib()
     p = ctypes.c_void_p(256)  # never dereferenced: the call is rejected first
-    # B*H*ceil(T/64) = 185 chunk-heads (bf16, d = 128) and 1017 (fp32): one more than fits
-    rc = L.kron_delta_fwd_noalloc(p, p, p, p, p, p, None, p, None, 1, 1, 185 * 64, 128, 128, 1, None)
+    # the largest bf16 d = 128 problem (in chunk-heads B*H*ceil(T/64)) per the library's own planner
+    n = 1
+    while kd.workspace_size(kd.KD_WS_FWD, 1, 1, (n + 1) * 64, 128, 128) <= 32 << 20:
+        n += 1
+    assert n >= 160  # the GPU case below uses 160
+    rc = L.kron_delta_fwd_noalloc(p, p, p, p, p, p, None, p, None, 1, 1, (n + 1) * 64, 128, 128, 1, None)
     assert rc == kd.KD_ERR_WORKSPACE
     assert b"exceeds the fixed" in L.kron_delta_last_error()
+    # fp32 (CUDA-core path): 1016 chunk-heads fit, 1017 do not
+    assert kd.workspace_size(kd.KD_WS_FWD, 1, 1, 1016 * 64, 128, 128, kd.KD_F32) <= 32 << 20
     rc = L.kron_delta_fwd_noalloc(p, p, p, p, p, p, None, p, None, 1, 1, 1017 * 64, 128, 128, 0, None)
     assert rc == kd.KD_ERR_WORKSPACE
-    # the largest bf16 d = 128 problem still fits
-    assert kd.workspace_size(kd.KD_WS_FWD, 1, 1, 184 * 64, 128, 128) <= 32 << 20
     rc = L.kron_delta_fwd_noalloc(p, p, p, p, p, p, None, p, None, 1, 1, 64, 96, 128, 1, None)
     assert rc == kd.KD_ERR_UNSUPPORTED
 
@@ -43,7 +47,7 @@ def test_noalloc_matches_workspace_forward_twice():
     if not torch.cuda.is_available():
         pytest.fail("GPU test needs a CUDA device")
     L = kd.lib()
-    cases = [dict(B=2, H=4, T=1000, seed=901), dict(B=1, H=8, T=1400, seed=902)]  # 128 and 176 chunk-heads
+    cases = [dict(B=2, H=4, T=1000, seed=901), dict(B=1, H=8, T=1280, seed=902)]  # 128 and 160 chunk-heads
     for case in cases:
         inp = kin.make_inputs(3, B=case["B"], H=case["H"], T=case["T"], seed=case["seed"], with_dO=False)
         d = {n: torch.from_numpy(inp[n]).to("cuda", torch.bfloat16 if n in ("q", "k", "v") else torch.float32)
