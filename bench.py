@@ -73,8 +73,13 @@ def kernel_work(name, d=128, C=CHUNK):
     table = {
         # Grams [K+; Q+] K-^T (tf32) and V V^T (bf16); writes A, y and P
         "fwd_prep_tc": ("tf32", 6 * C * d, 3 * act + lf + 8 + cc + 4 + cc),
-        # X = S K+^T and dS = V^T diag(u) K^e over the cluster; writes u, b0 and the chunk-start state tiles
-        "fwd_chain_tc": ("tf32", 4 * d * d, 2 * act + lf + 4 + cc + 4 + 8 + tile_f32 + tile_bf16),
+        # K~, K^e, gamma_C, V^T and the cross-chunk matrix H for every chunk (reads chunks n and n-1)
+        # (chunk n-1's k, v, logf were read by the neighbouring CTA and come from L2)
+        "fwd_cross_tc": ("tf32", 4 * C * d, 2 * act + lf + 2 * lf + 8 + cc + act),
+        # X' = S K~^T (tf32) and dS = V^T diag(u) K^e (bf16 hi+lo) over an R=4 cluster: reads K~, K^e,
+        # gamma_C, V^T, A, H, y, beta (the cluster's repeated reads of A, H, V^T are served by L2);
+        # writes u, b0 and the chunk-start states (fp32 and bf16 tiles)
+        "fwd_chain_tc": ("tf32", 4 * d * d, 2 * lf + 8 + act + 2 * cc + 8 + tile_f32 + tile_bf16 + 8),
         # S0 Q+^T, [Q+; K-] K-^T (tf32), V^T (u o P^T) (bf16); writes O
         "fwd_out_tc": ("tf32", 2 * d * d + 4 * C * d, 3 * act + lf + 4 + tile_f32 + act),
         # K+ K-^T (tf32), [V; dO] V^T and [V; dO] dO^T (bf16); writes du_intra, M u and three bf16 tiles
@@ -94,9 +99,13 @@ def kernel_work(name, d=128, C=CHUNK):
 # kernel lives in and the first 16 hex digits of its sha256 at capture time;
 # a kernel whose source has changed since reports no traffic.
 NCU_TRAFFIC = {
-    "fwd_prep_tc": (449772288, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
-    "fwd_chain_tc": (823336192, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
-    "fwd_out_tc": (662604544, "kd_fwd_tc.cu", "f6edfec7c050e06b"),
+    "fwd_prep_tc": (449185024, "kd_fwd_tc.cu", "3423dbfb894ff939"),
+    "fwd_cross_tc": (619071744, "kd_fwd_tc.cu", "3423dbfb894ff939"),
+    "fwd_chain_tc": (833273088, "kd_fwd_tc.cu", "3423dbfb894ff939"),
+    "fwd_out_tc": (662141440, "kd_fwd_tc.cu", "3423dbfb894ff939"),
+    "bwd_pre_tc": (514533888, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
+    "bwd_post_tc": (1126970880, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
+    "bwd_chain_tc": (586813952, "kd_bwd_tc.cu", "e5fe06fa04c57d84"),
 }
 
 
