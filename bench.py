@@ -314,8 +314,6 @@ def main(argv=None):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    kd.lib().kron_delta_profile_enable(1)
-    kd.lib().kron_delta_profile_report(None, 0, 1)
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -327,7 +325,15 @@ def main(argv=None):
     torch.cuda.synchronize()
     barrier()
     ms_total = max_over_ranks(e0.elapsed_time(e1))
+    # per-kernel times: the same steps again with the library's CUDA-event
+    # profiler, whose events between launches also serialise the kernels that
+    # otherwise overlap (each output kernel runs beside its chain)
     import ctypes
+    kd.lib().kron_delta_profile_enable(1)
+    kd.lib().kron_delta_profile_report(None, 0, 1)
+    for _ in range(args.steps):
+        step(d)
+    torch.cuda.synchronize()
     buf = ctypes.create_string_buffer(1 << 16)
     kd.lib().kron_delta_profile_report(buf, len(buf), 1)
     kd.lib().kron_delta_profile_enable(0)
