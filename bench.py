@@ -326,8 +326,7 @@ def main(argv=None):
     barrier()
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     # per-kernel times: the same steps again with the library's CUDA-event
-    # profiler, whose events between launches also serialise the kernels that
-    # otherwise overlap (each output kernel runs beside its chain)
+    # profiler (its events between launches are kept out of the headline timing)
     import ctypes
     kd.lib().kron_delta_profile_enable(1)
     kd.lib().kron_delta_profile_report(None, 0, 1)

@@ -67,7 +67,6 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
     L->Ke = take((size_t)B * T * H * dk * 4);
     L->GC = take(chunks * (size_t)dk * 4);
     L->Vt = take(chunks * (size_t)dv * C * 2);
-    L->fready = take((chunks + 1) * 4);  // + the output kernel's count of finished blocks
   }
   L->fwd_bytes = off;
   L->S0 = take(chunks * (size_t)dv * dk * 4);
@@ -98,7 +97,6 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
     L->PU = take(chunks * C * C * 2);
     L->EK = take(chunks * C * C * 2);
     L->Mu = take(chunks * C * 4);
-    L->ready = take((chunks + 1) * 4);  // + the post-chain kernel's count of finished blocks
   }
   L->bwd_bytes = off;
   return KD_OK;

@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
     const float* __restrict__ wMu, const __nv_bfloat16* __restrict__ wS0b, const __nv_bfloat16* __restrict__ wdSb,
     const __nv_bfloat16* __restrict__ wT1, const __nv_bfloat16* __restrict__ wPU,
     const __nv_bfloat16* __restrict__ wEK, float* __restrict__ dbeta, float* __restrict__ dc,
-    int* __restrict__ flags, const int* __restrict__ ready, int ready_target, int* __restrict__ err) {
+    int* __restrict__ flags, int* __restrict__ err) {
   using Cf = PostCfg;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -307,12 +307,10 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5;
-  // blocks visit the chunks in the order the reverse chain finishes them
-  const int units = gridDim.x / NC;
-  const int n = NC - 1 - static_cast<int>(blockIdx.x) / units, unit = static_cast<int>(blockIdx.x) % units;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
   const int b = unit / H, h = unit % H;
   const int t0 = n * C, nv = min(C, T - t0);
-  const size_t ch = (size_t)unit * NC + n;
+  const size_t ch = blockIdx.x;
   float* us = reinterpret_cast<float*>(sm + Cf::SMALL);
   float* db0s = us + 64;
   float* xch = db0s + 64;    // [128]
@@ -336,19 +334,15 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
     tc::bulk_g2s(sm + Cf::EK, wEK + ch * (C * C), 8192u, &bar_a);
     tc::mbar_expect_tx(&bar_b, Cf::LOAD_B);
     tc::bulk_g2s(sm + Cf::S0T, wS0b + ch * (D * D), 32768u, &bar_b);
+    tc::bulk_g2s(sm + Cf::DST, wdSb + ch * (D * D), 32768u, &bar_b);
     tc::tma_load_4d(sm + Cf::DOV, &tm_do, 0, h, t0, b, &bar_b);
     tc::tma_load_4d(sm + Cf::DOV + 16384, &tm_do, 64, h, t0, b, &bar_b);
     tc::tma_load_4d(sm + Cf::DOV + 8192, &tm_v, 0, h, t0, b, &bar_b);
     tc::tma_load_4d(sm + Cf::DOV + 24576, &tm_v, 64, h, t0, b, &bar_b);
     tc::bulk_g2s(sm + Cf::T1, wT1 + ch * (2 * C * C), 16384u, &bar_b);
     tc::bulk_g2s(sm + Cf::B7, wPU + ch * (C * C), 8192u, &bar_b);
-    // the chain's outputs for this chunk (dS tile, g): wait until it has published them
-    tc::wait_published(ready + ch, ready_target, err, tc::kErrTimeoutFlag);
-    tc::fence_proxy_async_global();
-    tc::bulk_g2s(sm + Cf::DST, wdSb + ch * (D * D), 32768u, &bar_b);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
-  __syncthreads();  // the chain's g is visible from here on
   if (tid < C) {
     const int t = tid;
     const float gt = wg[ch * C + t];
@@ -545,7 +539,6 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
   tc::tc_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
-  tc::finish_after_producer(const_cast<int*>(ready) + gridDim.x);
 }
 
 }  // namespace
@@ -569,7 +562,7 @@ cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_post_tc(const BwdArgs& a, int ready_target, int* err, cudaStream_t st) {
+cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st) {
   const Layout& L = a.L;
   CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_logf, tm_dq, tm_dk, tm_dv, tm_dlogf;
   if (!make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 64, true) ||
@@ -585,30 +578,14 @@ cudaError_t launch_bwd_post_tc(const BwdArgs& a, int ready_target, int* err, cud
   cudaError_t e =
       cudaFuncSetAttribute(bwd_post_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PostCfg::BYTES);
   if (e != cudaSuccess) return e;
-  // launched beside the reverse chain (programmatic dependent launch): each
-  // block waits for its chunk's published counter instead of the whole chain
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)L.chunks);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = PostCfg::BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   prof_begin(st, "bwd_post_tc");
-  e = cudaLaunchKernelEx(&cfg, bwd_post_tc, tm_q, tm_k, tm_v, tm_do, tm_logf, tm_dq, tm_dk, tm_dv, tm_dlogf,
-                         a.beta, L.H, L.T, L.NC, (const float*)ws_ptr<float>(a.fws, L.u),
-                         (const float*)ws_ptr<float>(a.fws, L.b0), (const float*)ws_ptr<float>(a.ws, L.g),
-                         (const float*)ws_ptr<float>(a.ws, L.Mu), (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.fws, L.S0b),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.dSCb),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.T1),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.PU),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.EK), a.dbeta, a.dc,
-                         ws_ptr<int>(a.ws, L.bflags), (const int*)ws_ptr<int>(a.ws, L.ready), ready_target, err);
+  bwd_post_tc<<<(unsigned)L.chunks, 256, PostCfg::BYTES, st>>>(
+      tm_q, tm_k, tm_v, tm_do, tm_logf, tm_dq, tm_dk, tm_dv, tm_dlogf, a.beta, L.H, L.T, L.NC,
+      ws_ptr<float>(a.fws, L.u), ws_ptr<float>(a.fws, L.b0), ws_ptr<float>(a.ws, L.g), ws_ptr<float>(a.ws, L.Mu),
+      ws_ptr<__nv_bfloat16>(a.fws, L.S0b), ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), ws_ptr<__nv_bfloat16>(a.ws, L.T1),
+      ws_ptr<__nv_bfloat16>(a.ws, L.PU), ws_ptr<__nv_bfloat16>(a.ws, L.EK), a.dbeta, a.dc,
+      ws_ptr<int>(a.ws, L.bflags), err);
   prof_end(st);
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(256, 1) bwd_chain_tc(
     const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ beta,
     const float* __restrict__ dST, float* __restrict__ dS0, int H, int T, int NC,
     const float* __restrict__ wA, const float* __restrict__ wdu, __nv_bfloat16* __restrict__ wdSCb,
-    float* __restrict__ wg, int* __restrict__ ready, int* __restrict__ err) {
+    float* __restrict__ wg, int* __restrict__ err) {
   using Cf = BChainCfg<R>;
   constexpr int NJ = Cf::NJ;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -124,7 +124,6 @@ __global__ void __launch_bounds__(256, 1) bwd_chain_tc(
   __syncthreads();
   tc::cluster_sync();
   tc::tc_after_sync();
-  tc::launch_dependents();  // the post-chain kernel may start beside the chain
   const uint32_t tmem = tmem_slot;
   const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);
 
@@ -220,13 +219,9 @@ __global__ void __launch_bounds__(256, 1) bwd_chain_tc(
           }
         }
       }
-      tc::publish_fence();
       tc::tc_before_sync();
       bar_prod();
-      if (p == 0) {
-        mbar_arrive(&s_saved);
-        tc::publish_add(ready + (size_t)unit * NC + n, 1);  // this CTA's slice of the dS tile
-      }
+      if (p == 0) mbar_arrive(&s_saved);
     }
   } else {
     // ============================= chain warps ============================
@@ -336,13 +331,9 @@ __global__ void __launch_bounds__(256, 1) bwd_chain_tc(
       if (tid < C) {
         const float g = gp[tid] + gp[64 + tid];
         db0[tid] = -bs[pb * 64 + tid] * g;
-        if (rank == 0) {
-          wg[ch * C + tid] = g;
-          tc::publish_fence();
-        }
+        if (rank == 0) wg[ch * C + tid] = g;
       }
       bar_chain();
-      if (rank == 0 && tid == 0) tc::publish_add(ready + ch, 1);  // g of this chunk
       // B2[j][t] = db0_t K+[t, j]  (bf16, N = NJ rows, K = 64)
       {
         const int t = tid & 63, jh = tid >> 6;
@@ -444,8 +435,7 @@ cudaError_t launch_bchain(const BwdArgs& a, int* err, cudaStream_t st) {
   prof_begin(st, "bwd_chain_tc");
   e = cudaLaunchKernelEx(&cfg, bwd_chain_tc<R>, tm_k, tm_q, tm_logf, tm_v, tm_do, a.beta, a.dST, a.dS0,
                          L.H, L.T, L.NC, ws_ptr<float>(a.fws, L.A), ws_ptr<float>(a.ws, L.du),
-                         ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), ws_ptr<float>(a.ws, L.g),
-                         ws_ptr<int>(a.ws, L.ready), err);
+                         ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), ws_ptr<float>(a.ws, L.g), err);
   prof_end(st);
   return e;
 }
@@ -456,13 +446,10 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st) 
   const Layout& L = a.L;
   cudaError_t e = launch_bwd_pre_tc(a, err, st);
   if (e != cudaSuccess) return e;
-  // per-chunk counters the chain publishes into (R dS slices + g)
-  if ((e = cudaMemsetAsync(ws_ptr<int>(a.ws, L.ready), 0, (L.chunks + 1) * sizeof(int), st)) != cudaSuccess)
-    return e;
   const int R = choose_cluster(L.B * L.H, sms);
   e = (R == 8) ? launch_bchain<8>(a, err, st) : launch_bchain<4>(a, err, st);
   if (e != cudaSuccess) return e;
-  if ((e = launch_bwd_post_tc(a, R + 1, err, st)) != cudaSuccess) return e;
+  if ((e = launch_bwd_post_tc(a, err, st)) != cudaSuccess) return e;
   // chunks outside the factorised decay range: exact CUDA-core recomputation
   return launch_bwd_simt_stages(a, kStageCC | kStageState | kStageIntra, ws_ptr<int>(a.ws, L.bflags), st);
 }

@@ -123,8 +123,7 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
     float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy, const float* __restrict__ wA,
     const float* __restrict__ wHx, const float* __restrict__ wGC, const __nv_bfloat16* __restrict__ wVt,
     float* __restrict__ wS0blob,
-    float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, int* __restrict__ ready,
-    int* __restrict__ err) {
+    float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, int* __restrict__ err) {
   using Cf = ChainCfg<R>;
   constexpr int NJ = Cf::NJ;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -172,7 +171,6 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
   __syncthreads();
   tc::cluster_sync();  // peers' barriers are initialised before any remote arrive
   tc::tc_after_sync();
-  tc::launch_dependents();  // the output kernel may start beside the chain
   const uint32_t tmem = tmem_slot;
   const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);  // lanes 32*(warp%4) ..
 
@@ -284,13 +282,9 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
           if (wS0b) save_bf16_tile(wS0b, (size_t)unit * NC + m, r, j0 + jj, x);
         }
       }
-      tc::publish_fence();
       tc::tc_before_sync();
       bar_prod();
-      if (p == 0) {
-        mbar_arrive(&s_saved);
-        tc::publish_add(ready + (size_t)unit * NC + m, 1);  // this CTA's slice of the chunk-start state
-      }
+      if (p == 0) mbar_arrive(&s_saved);
     }
   } else {
     // ============================= chain warps ============================
@@ -418,16 +412,10 @@ __global__ void __launch_bounds__(288, 1) fwd_chain_tc(
       bar_chain();  // every thread has read u_{n-1} (us) and w
       if (half == 0) {
         us[t] = uval;
-        if (rank == 0) {
-          wu[ch * C + t] = uval;
-          tc::publish_fence();
-        }
+        if (rank == 0 && wu) wu[ch * C + t] = uval;
       }
       bar_chain();
-      if (tid == 0) {
-        mbar_arrive(&aux_free[n & 1]);
-        if (rank == 0) tc::publish_add(ready + ch, 1);  // u of this chunk
-      }
+      if (tid == 0) mbar_arrive(&aux_free[n & 1]);
       // ---- B2 = diag(u_n) K^e_n slice as bf16 hi + lo (N = NJ rows j, K = 64 positions):
       //      thread (channel jl, 64/TQ consecutive positions) writes 16-byte pieces of row jl
       {
@@ -525,17 +513,14 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_logf,
     const __grid_constant__ CUtensorMap tm_out, int H, int NC, const float* __restrict__ wS0blob,
-    const float* __restrict__ wu, int* __restrict__ unsafe_flags, const int* __restrict__ ready, int ready_target,
-    int* __restrict__ err) {
+    const float* __restrict__ wu, int* __restrict__ unsafe_flags, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // blocks visit the chunks in the order the chain finishes them
-  const int units = gridDim.x / NC;
-  const int n = static_cast<int>(blockIdx.x) / units, unit = static_cast<int>(blockIdx.x) % units;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
   const int b = unit / H, h = unit % H;
   const int t0 = n * C;
   const size_t ch = (size_t)unit * NC + n;
@@ -546,17 +531,14 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     tc::mbar_init_fence();
     abort_flag = 0;
     tc::mbar_expect_tx(&ld_bar, OutCfg::LOAD_BYTES);
+#pragma unroll
+    for (int part = 0; part < 4; ++part)
+      tc::bulk_g2s(sm + OutCfg::S0 + part * 16384, wS0blob + ch * D * D + part * 4096, 16384u, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::VB, &tm_v, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::VB + 8192, &tm_v, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
-    // the chain's outputs for this chunk (start state, u): wait until it has published them
-    tc::wait_published(ready + ch, ready_target, err, tc::kErrTimeoutFlag);
-    tc::fence_proxy_async_global();
-#pragma unroll
-    for (int part = 0; part < 4; ++part)
-      tc::bulk_g2s(sm + OutCfg::S0 + part * 16384, wS0blob + ch * D * D + part * 4096, 16384u, &ld_bar);
     tc::bulk_g2s(sm + OutCfg::U, wu + ch * C, 256u, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
@@ -681,7 +663,6 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
   tc::tc_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
-  tc::finish_after_producer(const_cast<int*>(ready) + (gridDim.x));
   (void)lane;
 }
 
@@ -1181,8 +1162,7 @@ cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, flo
   __nv_bfloat16* s0b = a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0b) : nullptr;
   e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_v, tm_kt, tm_ke, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy, wA,
                          (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt), blob, wu, wb0, s0b,
-                         ws_ptr<int>(a.ws, L.fready), err);
+                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt), blob, wu, wb0, s0b, err);
   prof_end(st);
   return e;
 }
@@ -1266,9 +1246,6 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
   float* wb0 = ws_ptr<float>(a.ws, L.b0);
   int* flags = ws_ptr<int>(a.ws, L.flags);
   const int R = choose_cluster(L.B * L.H, sms);
-  // per-chunk counters the chain publishes into (R state slices + u)
-  if ((e = cudaMemsetAsync(ws_ptr<int>(a.ws, L.fready), 0, (L.chunks + 1) * sizeof(int), st)) != cudaSuccess)
-    return e;
   if (R == 8) e = launch_chain<8>(a, wy, wA, blob, wu, wb0, err, st);
   else e = launch_chain<4>(a, wy, wA, blob, wu, wb0, err, st);
   if (e != cudaSuccess) return e;
@@ -1283,23 +1260,10 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
         !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
         !make_tmap_bthd(&tm_out, a.out, 2, L.B, L.T, L.H, D, 64, true))
       return cudaErrorInvalidValue;
-    // launched beside the chain (programmatic dependent launch): each block
-    // waits for its chunk's published counter instead of the whole chain
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)L.chunks);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = OutCfg::BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     prof_begin(st, "fwd_out_tc");
-    e = cudaLaunchKernelEx(&cfg, fwd_out_tc, tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, (const float*)blob,
-                           (const float*)wu, flags, (const int*)ws_ptr<int>(a.ws, L.fready), R + 1, err);
+    fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, blob,
+                                                               wu, flags, err);
     prof_end(st);
-    if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   constexpr int kFixSmem = (3 * C * (D + 1) + C) * 4;

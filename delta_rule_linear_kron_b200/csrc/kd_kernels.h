@@ -28,7 +28,6 @@ struct Layout {
   // tensor-core path, operands of the chain: cross-chunk matrix Hx [ch][64][64],
   // K~ and K^e [B][T][H][dk] (fp32), gamma_C [ch][dk], V^T [ch][dv][64] (bf16 tile)
   size_t y = 0, A = 0, P = 0, Hx = 0, Kt = 0, Ke = 0, GC = 0, Vt = 0;
-  size_t fready = 0;  // tensor-core path: per-chunk counters the forward chain publishes into
   size_t fwd_bytes = 0;
   // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
   size_t S0 = 0, u = 0, b0 = 0, flags = 0;  // flags: one int per chunk (tensor-core path)
@@ -46,7 +45,6 @@ struct Layout {
   // 128-byte-swizzled tiles): [dP; E_V] (128 x 64), P diag(u) and E_K
   // (64 x 64 each); M u [ch][64]
   size_t T1 = 0, PU = 0, EK = 0, Mu = 0;
-  size_t ready = 0;  // tensor-core path: per-chunk counters the reverse chain publishes into
   size_t bwd_bytes = 0;
 };
 
@@ -101,8 +99,7 @@ cudaError_t launch_bwd_simt_stages(const BwdArgs& a, int stages, const int* only
 cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
 // per-chunk tensor-core kernels before / after the reverse chain (kd_bwd_chunk_tc.cu)
 cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st);
-// ready_target: the count the reverse chain publishes per finished chunk
-cudaError_t launch_bwd_post_tc(const BwdArgs& a, int ready_target, int* err, cudaStream_t st);
+cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st);
 
 template <typename T>
 inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }

@@ -14,7 +14,6 @@ namespace tc {
 constexpr int kErrTimeoutMma = 1;
 constexpr int kErrTimeoutLoad = 2;
 constexpr int kErrTimeoutCluster = 4;
-constexpr int kErrTimeoutFlag = 8;
 
 // bounded spin: ~4M polls of mbarrier.try_wait (each poll may suspend briefly)
 constexpr long kMaxPolls = 1L << 22;
@@ -116,50 +115,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, int* err
   if (err) atomicOr(err, code);
   *abort = 1;
   return false;
-}
-
-// ---- hand-off between a producing kernel and a consumer running beside it ----
-// The producer publishes a chunk by adding to its counter after every thread
-// that wrote the chunk's data has fenced (publish_fence) and the block has
-// synchronised; the consumer waits, bounded, until the counter reaches the
-// number of contributions, then reads the data.
-__device__ __forceinline__ void publish_fence() { __threadfence(); }
-__device__ __forceinline__ void publish_add(int* counter, int v) {
-  __threadfence();
-  atomicAdd(counter, v);
-}
-// Bounded wait (acquire, GPU scope) for *counter >= target; records `code` and
-// gives up after kMaxPolls polls.
-__device__ __forceinline__ bool wait_published(const int* counter, int target, int* err, int code) {
-  for (long i = 0; i < kMaxPolls; ++i) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
-    if (v >= target) return true;
-    __nanosleep(64);
-  }
-  if (err) atomicOr(err, code);
-  return false;
-}
-// Orders this thread's earlier (generic) view of global memory before its
-// later async-proxy reads of it (bulk copies, TMA loads).
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-// Programmatic dependent launch: the next kernel on the stream, launched with
-// the programmatic-serialisation attribute, may start once every block of this
-// kernel has executed this (or exited).
-__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-// Called by every block of a kernel launched beside its producer, at its end:
-// the last block to finish waits for the producer grid to complete, so this
-// grid completes after it and later work on the stream (including reuse of
-// freed memory) stays ordered after both.
-__device__ __forceinline__ void finish_after_producer(int* done_counter) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(done_counter, 1) == static_cast<int>(gridDim.x) - 1)
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-  }
 }
 
 // ---- bulk async copy global -> own shared memory (complete_tx on mbarrier) --
