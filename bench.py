@@ -191,6 +191,29 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x, world_size, device):
+    """The job's time is the slowest rank's: all-reduce MAX of a float (any
+    backend; the tensor lives on `device`)."""
+    if world_size == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world_size, units_per_rank, steps, ms_total):
+    """Whole-job rate under weak scaling: every rank processes units_per_rank
+    per step (its own batch), and the job takes the slowest rank's time."""
+    return world_size * units_per_rank * steps / (ms_total / 1e3)
+
+
+def rank_seed(base, rank):
+    """Each rank draws its own batch of the same shape."""
+    return base + rank
+
+
 def oracle_baseline(T_sample, seed=1004):
     """The fp64 oracle, as it stands, on the first T_sample tokens of the
     workload (all heads), fwd + bwd, all host cores."""
@@ -279,15 +302,8 @@ def main(argv=None):
         if ws_n > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if ws_n == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---- inputs (each rank its own batch) -------------------------------
-    inp = kin.make_inputs(4, seed=1004 + rank)
+    inp = kin.make_inputs(4, seed=rank_seed(1004, rank))
     bf, f32 = torch.bfloat16, torch.float32
     host = {n: torch.from_numpy(inp[n]).to(bf if n in ("q", "k", "v", "dO") else f32)
             for n in ("q", "k", "v", "dO", "beta", "c", "logf", "S0")}
@@ -324,7 +340,7 @@ def main(argv=None):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(e0.elapsed_time(e1), ws_n, dev)
     # per-kernel times: the same steps again with the library's CUDA-event
     # profiler (its events between launches are kept out of the headline timing)
     import ctypes
@@ -346,7 +362,7 @@ def main(argv=None):
     decode = None
     if not args.no_decode:
         Bd, Hd = 256, 16
-        dd = kin.decode_token_inputs_torch(args.decode_steps, B=Bd, H=Hd, seed=1005 + rank, device=dev)
+        dd = kin.decode_token_inputs_torch(args.decode_steps, B=Bd, H=Hd, seed=rank_seed(1005, rank), device=dev)
         S = dd["S"]
         o_dec = torch.empty((Bd, Hd, dv), dtype=bf, device=dev)
         for t in range(3):
@@ -360,7 +376,7 @@ def main(argv=None):
         d1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        dms = max_over_ranks(d0.elapsed_time(d1))
+        dms = max_over_ranks(d0.elapsed_time(d1), ws_n, dev)
         per_head = 2 * dv * dk * 4 + 2 * dk * 2 + dv * 2 + dk * 4 + 8 + dv * 2
         bytes_total = ws_n * args.decode_steps * Bd * Hd * per_head
         decode = dict(value=bytes_total / (dms / 1e3) / 1e9, unit="GB/s", steps=args.decode_steps,
@@ -392,11 +408,11 @@ def main(argv=None):
         x1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        xms = max_over_ranks(x0.elapsed_time(x1))
-        e2e = dict(value=ws_n * B * T * args.e2e_steps / (xms / 1e3), unit="tokens/s",
+        xms = max_over_ranks(x0.elapsed_time(x1), ws_n, dev)
+        e2e = dict(value=job_throughput(ws_n, B * T, args.e2e_steps, xms), unit="tokens/s",
                    h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
 
-    value = ws_n * B * T * args.steps / (ms_total / 1e3)
+    value = job_throughput(ws_n, B * T, args.steps, ms_total)
 
     # ---- roofline of the dominant kernel ---------------------------------
     roofline = None
