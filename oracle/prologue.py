@@ -85,14 +85,13 @@ def prologue_bwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, dq, dk, dv,
         y, r = l2_normalise(raw, eps)
         g = _f64(g)
         out[name] = r * (g - y * np.sum(y * g, axis=-1, keepdims=True))
-    sb = sigmoid(beta_pre)
-    out["dbeta_pre"] = _f64(dbeta) * beta_scale * sb * (1.0 - sb)
-    sc = sigmoid(c_pre)
-    out["dc_pre"] = _f64(dc) * sc * (1.0 - sc)
+    # 1 - sigmoid(x) is written sigmoid(-x) (the same number, without the
+    # cancellation of 1 - sigmoid(x) for large x)
+    out["dbeta_pre"] = _f64(dbeta) * beta_scale * sigmoid(beta_pre) * sigmoid(-_f64(beta_pre))
+    out["dc_pre"] = _f64(dc) * sigmoid(c_pre) * sigmoid(-_f64(c_pre))
     a = np.exp(_f64(a_log))
-    sf = sigmoid(f_pre)
     dlogf = _f64(dlogf)
-    out["df_pre"] = dlogf * a[None, None, :, None] * (1.0 - sf)
+    out["df_pre"] = dlogf * a[None, None, :, None] * sigmoid(-_f64(f_pre))
     logf = a[None, None, :, None] * log_sigmoid(f_pre)
     out["da_log"] = np.sum(dlogf * logf, axis=(0, 1, 3))
     return out

@@ -137,9 +137,11 @@ MUTANTS = [
     ("dx-sign", "r * (g - y * np.sum", "r * (g + y * np.sum"),
     ("dx-no-projection", "out[name] = r * (g - y * np.sum(y * g, axis=-1, keepdims=True))",
      "out[name] = r * g"),
-    ("dbeta-unscaled", "_f64(dbeta) * beta_scale * sb", "_f64(dbeta) * sb"),
-    ("df-missing-exponent", "dlogf * a[None, None, :, None] * (1.0 - sf)", "dlogf * (1.0 - sf)"),
-    ("df-sigma-not-complement", "* (1.0 - sf)", "* sf"),
+    ("dbeta-unscaled", "_f64(dbeta) * beta_scale * sigmoid", "_f64(dbeta) * sigmoid"),
+    ("df-missing-exponent", "dlogf * a[None, None, :, None] * sigmoid(-_f64(f_pre))",
+     "dlogf * sigmoid(-_f64(f_pre))"),
+    ("df-sigma-not-complement", "* sigmoid(-_f64(f_pre))", "* sigmoid(f_pre)"),
+    ("dc-one-factor", "_f64(dc) * sigmoid(c_pre) * sigmoid(-_f64(c_pre))", "_f64(dc) * sigmoid(c_pre)"),
     ("dalog-missing-logf", "np.sum(dlogf * logf, axis=(0, 1, 3))", "np.sum(dlogf, axis=(0, 1, 3))"),
 ]
 
@@ -169,3 +171,17 @@ def test_pins_reject_mutant(tmp_path, name, old, new):
         except AssertionError:
             caught += 1
     assert caught > 0, f"no pin rejects mutant {name}"
+
+
+def test_backward_tails_are_accurate(P=_P):
+    """In the saturated tails the gate derivatives keep their relative accuracy:
+    d/dx log sigmoid(x) = sigmoid(-x) ~ e^-x and sigmoid'(x) ~ e^-|x| (closed forms)."""
+    x = np.array([30.0, -30.0, 60.0])
+    z = np.zeros((1, 1, 1, 3))
+    g = P.prologue_bwd(z + 1, z + 1, z[..., :1] + 1, x.reshape(1, 1, 3)[..., :1].reshape(1, 1, 1),
+                       np.array([[[40.0]]]), x.reshape(1, 1, 1, 3), np.zeros(1),
+                       z, z, z[..., :1], np.ones((1, 1, 1)), np.ones((1, 1, 1)), np.ones((1, 1, 1, 3)))
+    assert np.allclose(g["df_pre"].reshape(-1), [np.exp(-30.0) / (1 + np.exp(-30.0)),
+                                                  1.0 / (1.0 + np.exp(-30.0)), np.exp(-60.0)], rtol=1e-12)
+    assert np.isclose(g["dc_pre"].item(), np.exp(-40.0), rtol=1e-12)
+    assert np.isclose(g["dbeta_pre"].item(), np.exp(-30.0), rtol=1e-12)
