@@ -15,7 +15,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["fwd", "bwd", "decode", "workspace_size", "device_status", "library_path",
+__all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "workspace_size", "device_status", "library_path",
            "KronDeltaError", "KronDeltaFunction", "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -24,7 +24,7 @@ _lib = None
 
 KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE, KD_ERR_CUDA, KD_ERR_TIMEOUT = range(6)
 KD_F32, KD_BF16 = 0, 1
-KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD = 0, 1, 2
+KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD = 0, 1, 2, 3
 _CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
           4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
 
@@ -62,6 +62,11 @@ def lib():
         L.kron_delta_device_status.argtypes = [vp]
         L.kron_delta_fwd_noalloc.restype = i
         L.kron_delta_fwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [vp]
+        L.kron_delta_prologue_fwd.restype = i
+        L.kron_delta_prologue_fwd.argtypes = [vp] * 7 + [ctypes.c_float] + [vp] * 6 + [i] * 6 + [vp]
+        L.kron_delta_prologue_bwd.restype = i
+        L.kron_delta_prologue_bwd.argtypes = ([vp] * 7 + [ctypes.c_float] + [vp] * 13 + [i] * 6 +
+                                              [vp, sz, vp])
         L.kron_delta_profile_enable.restype = None
         L.kron_delta_profile_enable.argtypes = [i]
         L.kron_delta_profile_report.restype = i
@@ -192,6 +197,64 @@ def decode(q, k, v, beta, c, logf, S, *, out=None, stream=None):
     _check(lib().kron_delta_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S),
                                    _ptr(out), B, H, dk, dv, dt, _stream(stream)))
     return out
+
+
+def _prologue_inputs(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log):
+    import torch
+    B, T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    f32 = torch.float32
+    _need(q_raw, "q_raw"); _need(k_raw, "k_raw", q_raw.dtype, q_raw.shape)
+    _need(v_raw, "v_raw", q_raw.dtype, (B, T, H, dv)); _need(f_pre, "f_pre", q_raw.dtype, q_raw.shape)
+    _need(beta_pre, "beta_pre", f32, (B, T, H)); _need(c_pre, "c_pre", f32, (B, T, H))
+    _need(a_log, "a_log", f32, (H,))
+    return B, T, H, dk, dv, _dtype_code(q_raw)
+
+
+def prologue_fwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale=1.0, *, stream=None):
+    """Input prologue: L2-normalised q, k, v; beta = beta_scale*sigmoid(beta_pre);
+    c = sigmoid(c_pre); logf = exp(a_log[h]) * log sigmoid(f_pre).
+    q_raw, k_raw, f_pre [B,T,H,dk], v_raw [B,T,H,dv] (bf16 or fp32, one dtype);
+    beta_pre, c_pre [B,T,H] fp32; a_log [H] fp32.  Returns dict q, k, v, beta, c, logf
+    in the layouts fwd() takes."""
+    import torch
+    B, T, H, dk, dv, dt = _prologue_inputs(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log)
+    f32 = torch.float32
+    o = dict(q=torch.empty_like(q_raw), k=torch.empty_like(k_raw), v=torch.empty_like(v_raw),
+             beta=torch.empty_like(beta_pre), c=torch.empty_like(c_pre),
+             logf=torch.empty((B, T, H, dk), dtype=f32, device=q_raw.device))
+    _check(lib().kron_delta_prologue_fwd(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(beta_pre), _ptr(c_pre),
+                                         _ptr(f_pre), _ptr(a_log), float(beta_scale), _ptr(o["q"]),
+                                         _ptr(o["k"]), _ptr(o["v"]), _ptr(o["beta"]), _ptr(o["c"]),
+                                         _ptr(o["logf"]), B, H, T, dk, dv, dt, _stream(stream)))
+    return o
+
+
+def prologue_bwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, dq, dk, dv, dbeta, dc, dlogf,
+                 beta_scale=1.0, *, workspace=None, stream=None):
+    """Backward of prologue_fwd given the gradients of its outputs (as bwd()
+    returns them).  Returns dict dq_raw, dk_raw, dv_raw, dbeta_pre, dc_pre,
+    df_pre, da_log."""
+    import torch
+    B, T, H, dk_, dv_, dt = _prologue_inputs(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log)
+    f32 = torch.float32
+    _need(dq, "dq", q_raw.dtype, (B, T, H, dk_)); _need(dk, "dk", q_raw.dtype, (B, T, H, dk_))
+    _need(dv, "dv", q_raw.dtype, (B, T, H, dv_)); _need(dbeta, "dbeta", f32, (B, T, H))
+    _need(dc, "dc", f32, (B, T, H)); _need(dlogf, "dlogf", f32, (B, T, H, dk_))
+    g = dict(dq_raw=torch.empty_like(q_raw), dk_raw=torch.empty_like(k_raw), dv_raw=torch.empty_like(v_raw),
+             dbeta_pre=torch.empty_like(beta_pre), dc_pre=torch.empty_like(c_pre),
+             df_pre=torch.empty_like(f_pre), da_log=torch.empty_like(a_log))
+    need = workspace_size(KD_WS_PROLOGUE_BWD, B, H, T, dk_, dv_, dt)
+    if workspace is None:
+        workspace = _alloc_ws(need, q_raw.device)
+    _check(lib().kron_delta_prologue_bwd(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(beta_pre), _ptr(c_pre),
+                                         _ptr(f_pre), _ptr(a_log), float(beta_scale), _ptr(dq), _ptr(dk),
+                                         _ptr(dv), _ptr(dbeta), _ptr(dc), _ptr(dlogf), _ptr(g["dq_raw"]),
+                                         _ptr(g["dk_raw"]), _ptr(g["dv_raw"]), _ptr(g["dbeta_pre"]),
+                                         _ptr(g["dc_pre"]), _ptr(g["df_pre"]), _ptr(g["da_log"]),
+                                         B, H, T, dk_, dv_, dt, _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return g
 
 
 def device_status(stream=None):

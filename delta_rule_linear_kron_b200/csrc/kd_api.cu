@@ -232,6 +232,9 @@ size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv, 
     case KD_WS_FWD: ok(); return L.fwd_bytes;
     case KD_WS_FWD_SAVE: ok(); return L.fwd_save_bytes;
     case KD_WS_BWD: ok(); return L.bwd_bytes;
+    case KD_WS_PROLOGUE_BWD:
+      ok();
+      return align256((size_t)kd::prologue_blocks((long long)B * T) * H * sizeof(float));
     default: fail(KD_ERR_INVALID_ARG, "unknown workspace kind %d", kind); return 0;
   }
 }
@@ -331,6 +334,89 @@ int kron_delta_decode(const void* q, const void* k, const void* v, const float* 
   KD_TRY(check_stream(stream));
   kd::DecodeArgs a{q, k, v, beta, c, logf, S, out, B, H, dk, dv, dtype};
   return launched(kd::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+namespace {
+int check_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
+                   const float* c_pre, const void* f_pre, const float* a_log, float beta_scale, int B,
+                   int H, int T, int dk, int dv, int dtype) {
+  if (B <= 0 || H <= 0 || T <= 0) return fail(KD_ERR_INVALID_ARG, "B, H, T must be >= 1 (got %d, %d, %d)", B, H, T);
+  if (H > 65535) return fail(KD_ERR_INVALID_ARG, "H must be <= 65535 (got %d)", H);
+  if (!dim_supported(dk) || !dim_supported(dv))
+    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  if (!(beta_scale > 0.f && beta_scale <= 2.f))
+    return fail(KD_ERR_INVALID_ARG, "beta_scale must be in (0, 2] (got %g)", (double)beta_scale);
+  KD_TRY(check_ptr(q_raw, "q_raw", true));
+  KD_TRY(check_ptr(k_raw, "k_raw", true));
+  KD_TRY(check_ptr(v_raw, "v_raw", true));
+  KD_TRY(check_ptr(beta_pre, "beta_pre", true));
+  KD_TRY(check_ptr(c_pre, "c_pre", true));
+  KD_TRY(check_ptr(f_pre, "f_pre", true));
+  return check_ptr(a_log, "a_log", true);
+}
+}  // namespace
+
+int kron_delta_prologue_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
+                            const float* beta_pre, const float* c_pre, const void* f_pre,
+                            const float* a_log, float beta_scale, void* q, void* k, void* v,
+                            float* beta, float* c, float* logf, int B, int H, int T, int dk, int dv,
+                            int dtype, void* stream) {
+  KD_TRY(check_prologue(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, B, H, T, dk, dv,
+                        dtype));
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(beta, "beta", true));
+  KD_TRY(check_ptr(c, "c", true));
+  KD_TRY(check_ptr(logf, "logf", true));
+  KD_TRY(check_stream(stream));
+  kd::PrologueArgs a{};
+  a.q_raw = q_raw; a.k_raw = k_raw; a.v_raw = v_raw;
+  a.beta_pre = beta_pre; a.c_pre = c_pre; a.f_pre = f_pre; a.a_log = a_log; a.beta_scale = beta_scale;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.c = c; a.logf = logf;
+  a.N = (long long)B * T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
+  return launched(kd::launch_prologue_fwd(a, static_cast<cudaStream_t>(stream)), "prologue launch");
+}
+
+int kron_delta_prologue_bwd(const void* q_raw, const void* k_raw, const void* v_raw,
+                            const float* beta_pre, const float* c_pre, const void* f_pre,
+                            const float* a_log, float beta_scale, const void* dq, const void* dk,
+                            const void* dv, const float* dbeta, const float* dc, const float* dlogf,
+                            void* dq_raw, void* dk_raw, void* dv_raw, float* dbeta_pre, float* dc_pre,
+                            void* df_pre, float* da_log, int B, int H, int T, int dk_, int dv_,
+                            int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  KD_TRY(check_prologue(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, B, H, T, dk_,
+                        dv_, dtype));
+  KD_TRY(check_ptr(dq, "dq", true));
+  KD_TRY(check_ptr(dk, "dk", true));
+  KD_TRY(check_ptr(dv, "dv", true));
+  KD_TRY(check_ptr(dbeta, "dbeta", true));
+  KD_TRY(check_ptr(dc, "dc", true));
+  KD_TRY(check_ptr(dlogf, "dlogf", true));
+  KD_TRY(check_ptr(dq_raw, "dq_raw", true));
+  KD_TRY(check_ptr(dk_raw, "dk_raw", true));
+  KD_TRY(check_ptr(dv_raw, "dv_raw", true));
+  KD_TRY(check_ptr(dbeta_pre, "dbeta_pre", true));
+  KD_TRY(check_ptr(dc_pre, "dc_pre", true));
+  KD_TRY(check_ptr(df_pre, "df_pre", true));
+  KD_TRY(check_ptr(da_log, "da_log", true));
+  const long long N = (long long)B * T;
+  const size_t need = (size_t)kd::prologue_blocks(N) * H * sizeof(float);
+  if (!workspace || ws_bytes < need)
+    return fail(KD_ERR_WORKSPACE, "prologue workspace of %zu bytes needed (got %zu)", need,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  kd::PrologueArgs a{};
+  a.q_raw = q_raw; a.k_raw = k_raw; a.v_raw = v_raw;
+  a.beta_pre = beta_pre; a.c_pre = c_pre; a.f_pre = f_pre; a.a_log = a_log; a.beta_scale = beta_scale;
+  a.gq = dq; a.gk = dk; a.gv = dv; a.dbeta = dbeta; a.dc = dc; a.dlogf = dlogf;
+  a.dq_raw = dq_raw; a.dk_raw = dk_raw; a.dv_raw = dv_raw;
+  a.dbeta_pre = dbeta_pre; a.dc_pre = dc_pre; a.df_pre = df_pre; a.da_log = da_log;
+  a.part = static_cast<float*>(workspace);
+  a.N = N; a.H = H; a.dk = dk_; a.dv = dv_; a.dtype = dtype;
+  return launched(kd::launch_prologue_bwd(a, static_cast<cudaStream_t>(stream)), "prologue backward launch");
 }
 
 void kron_delta_profile_enable(int on) {

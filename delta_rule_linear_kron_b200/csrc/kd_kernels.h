@@ -101,6 +101,31 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
 cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st);
 cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st);
 
+// Input prologue (kd_prologue.cu).  N = B*T tokens; rows are [N][H][d].
+struct PrologueArgs {
+  const void *q_raw, *k_raw, *v_raw;
+  const float *beta_pre, *c_pre;
+  const void* f_pre;
+  const float* a_log;
+  float beta_scale;
+  // forward outputs
+  void *q, *k, *v;
+  float *beta, *c, *logf;
+  // backward: upstream gradients in, input gradients out
+  const void *gq, *gk, *gv;  // dq, dk, dv of the normalised q, k, v
+  const float *dbeta, *dc, *dlogf;
+  void *dq_raw, *dk_raw, *dv_raw;
+  float *dbeta_pre, *dc_pre;
+  void* df_pre;
+  float* da_log;
+  float* part;  // backward scratch: prologue_blocks(N) * H floats
+  long long N;
+  int H, dk, dv, dtype;
+};
+int prologue_blocks(long long N);
+cudaError_t launch_prologue_fwd(const PrologueArgs& a, cudaStream_t st);
+cudaError_t launch_prologue_bwd(const PrologueArgs& a, cudaStream_t st);
+
 template <typename T>
 inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }
 template <typename T>

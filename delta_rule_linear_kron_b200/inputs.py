@@ -17,6 +17,12 @@ Recipe (shapes and distributions of the five workloads):
   * S0: zero, or N(0,1) scaled to Frobenius norm 1 per head.
   * decode states: N(0, 1/128) (variance 1/128).
   * dO ~ N(0,1), rounded to the storage dtype.
+  * prologue inputs (``make_prologue_inputs``), drawn in the order q~, k~, v~,
+    beta-pre, c-pre, f-pre, a_log, then the upstream gradients dq, dk, dv,
+    dbeta, dc, dlogf: raw q~, k~, v~ ~ N(0,1) (storage dtype); beta-pre,
+    c-pre ~ N(0,1) (fp32); f-pre ~ N(3,1) (storage dtype); a_log ~ U(-1,1)
+    (fp32); upstream gradients N(0,1) (dq, dk, dv in the storage dtype, the
+    gate gradients fp32).
 All arrays are returned as float64 numpy arrays holding exactly the values the
 GPU receives (bf16-representable where the dtype is bf16).
 """
@@ -26,7 +32,7 @@ from dataclasses import dataclass, replace
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs",
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs", "make_prologue_inputs",
            "round_to_dtype", "decode_token_inputs_torch"]
 
 
@@ -113,6 +119,30 @@ def make_inputs(wl: Workload | int, *, B=None, H=None, T=None, dk=None, dv=None,
     out = dict(q=q, k=k, v=v, beta=beta, c=c, logf=logf, S0=S0, wl=wl)
     if with_dO:
         out["dO"] = round_to_dtype(rng.standard_normal((B, T, H, dv)), wl.dtype)
+    return out
+
+
+def make_prologue_inputs(B, H, T, dk, dv, dtype="bf16", seed=2000, with_grads=True):
+    """Raw inputs of the prologue (and, with_grads, upstream gradients of its
+    outputs), as float64 arrays holding the values the GPU receives:
+    q_raw, k_raw, f_pre [B,T,H,dk], v_raw [B,T,H,dv], beta_pre, c_pre [B,T,H],
+    a_log [H]; dq, dk [B,T,H,dk], dv [B,T,H,dv], dbeta, dc [B,T,H],
+    dlogf [B,T,H,dk]."""
+    rng = np.random.default_rng(seed)
+    out = dict(q_raw=round_to_dtype(rng.standard_normal((B, T, H, dk)), dtype),
+               k_raw=round_to_dtype(rng.standard_normal((B, T, H, dk)), dtype),
+               v_raw=round_to_dtype(rng.standard_normal((B, T, H, dv)), dtype),
+               beta_pre=round_to_dtype(rng.standard_normal((B, T, H)), "f32"),
+               c_pre=round_to_dtype(rng.standard_normal((B, T, H)), "f32"),
+               f_pre=round_to_dtype(rng.normal(3.0, 1.0, size=(B, T, H, dk)), dtype),
+               a_log=round_to_dtype(rng.uniform(-1.0, 1.0, size=(H,)), "f32"))
+    if with_grads:
+        out.update(dq=round_to_dtype(rng.standard_normal((B, T, H, dk)), dtype),
+                   dk=round_to_dtype(rng.standard_normal((B, T, H, dk)), dtype),
+                   dv=round_to_dtype(rng.standard_normal((B, T, H, dv)), dtype),
+                   dbeta=round_to_dtype(rng.standard_normal((B, T, H)), "f32"),
+                   dc=round_to_dtype(rng.standard_normal((B, T, H)), "f32"),
+                   dlogf=round_to_dtype(rng.standard_normal((B, T, H, dk)), "f32"))
     return out
 
 

@@ -78,6 +78,8 @@ extern "C" {
 #define KD_WS_FWD 0        /* forward only (prefill / inference) */
 #define KD_WS_FWD_SAVE 1   /* forward that keeps what the backward needs */
 #define KD_WS_BWD 2        /* backward scratch (besides the saved forward) */
+#define KD_WS_PROLOGUE_BWD 3  /* scratch of kron_delta_prologue_bwd (dk, dv, dtype
+                                 must be valid but do not change the size) */
 
 /* Library version, as 10000*major + 100*minor + patch. */
 KD_API int kron_delta_version(void);
@@ -173,6 +175,54 @@ KD_API int kron_delta_fwd_noalloc(const void *q, const void *k, const void *v,
                                   const float *beta, const float *c, const float *logf,
                                   const float *S0, void *out, float *ST, int B, int H,
                                   int T, int dk, int dv, int dtype, void *stream);
+
+/*
+ * Input prologue: from the raw projections to the recurrence's inputs, one
+ * fused pass.  KronLSTM digest, section "어떻게 쓰나": q, k, v are
+ * L2-normalised; the erase and write gates are sigmoids of per-head scalar
+ * projections (the erase gate scaled by 2 for state tracking, experiments
+ * paragraph of the same page); the forget gate is sigmoid(x) raised to the
+ * head's learned exponent exp(a_log).  Per token t and head h:
+ *     q = q_raw / sqrt(|q_raw|^2 + 1e-6)      (likewise k, v)
+ *     beta = beta_scale * sigmoid(beta_pre)    c = sigmoid(c_pre)
+ *     logf[j] = exp(a_log[h]) * log sigmoid(f_pre[j])
+ *   q_raw, k_raw, f_pre : [B,T,H,dk] (dtype);  v_raw : [B,T,H,dv] (dtype).
+ *   beta_pre, c_pre : [B,T,H] fp32;  a_log : [H] fp32.
+ *   beta_scale : in (0, 2]; 1 gives beta in (0, 1), 2 gives beta in (0, 2).
+ *   q, k, v, beta, c, logf : outputs in the layouts of kron_delta_fwd, ready
+ *   to be passed to it.  All 16-byte aligned.  No workspace.
+ * Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_CUDA.  Asynchronous
+ * on `stream`.
+ */
+KD_API int kron_delta_prologue_fwd(const void *q_raw, const void *k_raw, const void *v_raw,
+                                   const float *beta_pre, const float *c_pre, const void *f_pre,
+                                   const float *a_log, float beta_scale, void *q, void *k, void *v,
+                                   float *beta, float *c, float *logf, int B, int H, int T, int dk,
+                                   int dv, int dtype, void *stream);
+
+/*
+ * Backward of kron_delta_prologue_fwd, for the loss
+ * l = <dq,q> + <dk,k> + <dv,v> + <dbeta,beta> + <dc,c> + <dlogf,logf>
+ * (dq, dk, dv, dbeta, dc, dlogf as kron_delta_bwd writes them).
+ *   Inputs as for the forward, plus the upstream gradients dq, dk [B,T,H,dk],
+ *   dv [B,T,H,dv] (dtype), dbeta, dc [B,T,H] fp32, dlogf [B,T,H,dk] fp32.
+ *   Outputs: dq_raw, dk_raw, df_pre [B,T,H,dk] and dv_raw [B,T,H,dv] (dtype);
+ *   dbeta_pre, dc_pre [B,T,H] fp32; da_log [H] fp32 (overwritten, not
+ *   accumulated; the sum over tokens and channels runs in a fixed order, so
+ *   the result is bitwise reproducible).
+ *   workspace, ws_bytes : scratch of at least
+ *     kron_delta_workspace_size(KD_WS_PROLOGUE_BWD, ...), 256-byte aligned.
+ * Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE,
+ * KD_ERR_CUDA.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_prologue_bwd(const void *q_raw, const void *k_raw, const void *v_raw,
+                                   const float *beta_pre, const float *c_pre, const void *f_pre,
+                                   const float *a_log, float beta_scale, const void *dq,
+                                   const void *dk, const void *dv, const float *dbeta,
+                                   const float *dc, const float *dlogf, void *dq_raw, void *dk_raw,
+                                   void *dv_raw, float *dbeta_pre, float *dc_pre, void *df_pre,
+                                   float *da_log, int B, int H, int T, int dk_, int dv_, int dtype,
+                                   void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Synchronises `stream` and reports device-side failures of earlier calls:

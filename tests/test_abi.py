@@ -109,3 +109,46 @@ def test_python_binding_rejects_host_tensors():
     q = torch.zeros(1, 64, 1, 32)
     with pytest.raises(kd.KronDeltaError):
         kd.fwd(q, q, q, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1), q)
+
+
+def _pro_fwd(L, **over):
+    p = ctypes.c_void_p(256)
+    a = dict(qr=p, kr=p, vr=p, bp=p, cp=p, fp=p, al=p, scale=1.0, q=p, k=p, v=p, beta=p, c=p, logf=p,
+             B=1, H=2, T=70, dk=64, dv=32, dtype=1, stream=None)
+    a.update(over)
+    return L.kron_delta_prologue_fwd(a["qr"], a["kr"], a["vr"], a["bp"], a["cp"], a["fp"], a["al"],
+                                     a["scale"], a["q"], a["k"], a["v"], a["beta"], a["c"], a["logf"],
+                                     a["B"], a["H"], a["T"], a["dk"], a["dv"], a["dtype"], a["stream"])
+
+
+def _pro_bwd(L, **over):
+    p = ctypes.c_void_p(256)
+    a = dict(al=p, scale=2.0, dq=p, dfp=p, da=p, B=1, H=2, T=70, dk=64, dv=32, dtype=1, ws=p, ws_bytes=0)
+    a.update(over)
+    return L.kron_delta_prologue_bwd(p, p, p, p, p, p, a["al"], a["scale"], a["dq"], p, p, p, p, p,
+                                     p, p, p, p, p, a["dfp"], a["da"], a["B"], a["H"], a["T"], a["dk"],
+                                     a["dv"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+def test_prologue_argument_errors(L):
+    assert L.kron_delta_prologue_fwd.argtypes[7] is ctypes.c_float
+    assert _pro_fwd(L, dk=48) == kd.KD_ERR_UNSUPPORTED
+    assert _pro_fwd(L, dtype=3) == kd.KD_ERR_UNSUPPORTED
+    assert _pro_fwd(L, T=0) == kd.KD_ERR_INVALID_ARG
+    assert _pro_fwd(L, scale=0.0) == kd.KD_ERR_INVALID_ARG
+    assert _pro_fwd(L, scale=2.5) == kd.KD_ERR_INVALID_ARG
+    assert b"beta_scale" in L.kron_delta_last_error()
+    assert _pro_fwd(L, scale=float("nan")) == kd.KD_ERR_INVALID_ARG
+    assert _pro_fwd(L, fp=None) == kd.KD_ERR_INVALID_ARG
+    assert b"f_pre must not be NULL" in L.kron_delta_last_error()
+    assert _pro_fwd(L, logf=ctypes.c_void_p(260)) == kd.KD_ERR_INVALID_ARG
+    assert _pro_bwd(L, da=None) == kd.KD_ERR_INVALID_ARG
+    assert b"da_log" in L.kron_delta_last_error()
+    assert _pro_bwd(L, dq=None) == kd.KD_ERR_INVALID_ARG
+    assert _pro_bwd(L) == kd.KD_ERR_WORKSPACE
+    need = kd.workspace_size(kd.KD_WS_PROLOGUE_BWD, 1, 2, 70, 64, 32)
+    assert need >= 2 * 4 and need % 256 == 0
+    assert _pro_bwd(L, ws_bytes=need, ws=ctypes.c_void_p(256 + 64)) == kd.KD_ERR_WORKSPACE
+    # one partial per (block of 64 tokens, head)
+    big = kd.workspace_size(kd.KD_WS_PROLOGUE_BWD, 2, 16, 16384, 128, 128)
+    assert big >= (2 * 16384 // 64) * 16 * 4
