@@ -6,7 +6,8 @@ forward (saving what the backward needs) followed by the backward, on the
 forward+backward workload B=1, H=16, T=16384, d_k=d_v=128, bf16 q/k/v/dO,
 fp32 gates and state, beta in (0,2), nonzero S0.  The decode step
 (B=256, H=16, d=128, 1000 consecutive in-place steps) is timed in the same run
-and reported under "decode".
+and reported under "decode"; the input prologue (raw projections -> normalised
+q, k, v and gates) and its backward, on the step's shape, under "prologue".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -89,6 +90,11 @@ def kernel_work(name, d=128, C=CHUNK):
         # the five state / intra-chunk accumulators; writes dq, dk, dv, dlogf, dbeta, dc
         "bwd_post_tc": ("bf16", 16 * d * d, 4 * act + lf + 2 * tile_bf16 + 2 * ccb + ccb + ccb + 20
                         + 3 * act + lf + 8),
+        # input prologue (not part of the step; timed on its own): reads q~, k~, v~, f~, beta~, c~;
+        # writes q, k, v, logf (fp32), beta, c.  About 20 flops per channel.
+        "prologue_fwd": ("alu", 20 * 4 * d, 4 * act + 8 + 3 * act + lf + 8),
+        # reads q~, k~, v~, f~, dq, dk, dv, dlogf and four gate scalars; writes dq~, dk~, dv~, df~ and two
+        "prologue_bwd": ("alu", 30 * 4 * d, 4 * act + 3 * act + lf + 16 + 4 * act + 8),
     }
     w = table.get(name)
     return None if w is None else dict(kind=w[0], flops=w[1], bytes=w[2])
@@ -275,6 +281,7 @@ def main(argv=None):
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -384,6 +391,49 @@ def main(argv=None):
                       bytes_per_head=per_head,
                       hbm_frac=(bytes_total / ws_n / (dms / 1e3) / 1e9) / peaks["hbm_gbs"])
         del dd, S
+    # ---- input prologue (raw projections -> q, k, v, beta, c, logf) and its
+    # backward, on this workload's shape, timed on their own --------------
+    prologue = None
+    if not args.no_prologue:
+        g_ = torch.Generator(device=dev)
+        g_.manual_seed(rank_seed(2004, rank))
+        rn = lambda *sh, m=0.0: torch.randn(sh, generator=g_, device=dev) + m  # noqa: E731
+        pr = dict(q_raw=rn(B, T, H, dk).to(bf), k_raw=rn(B, T, H, dk).to(bf), v_raw=rn(B, T, H, dv).to(bf),
+                  beta_pre=rn(B, T, H), c_pre=rn(B, T, H), f_pre=rn(B, T, H, dk, m=3.0).to(bf),
+                  a_log=torch.rand((H,), generator=g_, device=dev) * 2 - 1)
+        up = dict(dq=rn(B, T, H, dk).to(bf), dk=rn(B, T, H, dk).to(bf), dv=rn(B, T, H, dv).to(bf),
+                  dbeta=rn(B, T, H), dc=rn(B, T, H), dlogf=rn(B, T, H, dk))
+        pws = torch.empty(kd.workspace_size(kd.KD_WS_PROLOGUE_BWD, B, H, T, dk, dv), dtype=torch.uint8,
+                          device=dev)
+        order = ("q_raw", "k_raw", "v_raw", "beta_pre", "c_pre", "f_pre", "a_log")
+        times = {}
+        for name in ("prologue_fwd", "prologue_bwd"):
+            def call():
+                if name == "prologue_fwd":
+                    kd.prologue_fwd(*(pr[n] for n in order), 2.0)
+                else:
+                    kd.prologue_bwd(*(pr[n] for n in order), up["dq"], up["dk"], up["dv"], up["dbeta"], up["dc"],
+                                    up["dlogf"], 2.0, workspace=pws)
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            barrier()
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            p0.record(stream)
+            for _ in range(args.steps):
+                call()
+            p1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            ms = max_over_ranks(p0.elapsed_time(p1), ws_n, dev) / args.steps
+            w = kernel_work(name)
+            gbs = w["bytes"] * B * H * T / (ms / 1e3) / 1e9
+            times[name] = dict(ms=ms, algorithmic_bytes_per_launch=w["bytes"] * B * H * T, achieved_gbs=gbs,
+                               hbm_frac=gbs / peaks["hbm_gbs"])
+        kd.device_status()
+        prologue = dict(times, note="timed alone, not part of the step; the bwd time includes the small "
+                                    "fixed-order da_log reduction launch")
+        del pr, up
     clocks = sampler.stop()
 
     # ---- end to end through the public API with pinned host buffers -----
@@ -463,7 +513,7 @@ def main(argv=None):
                            "global_batch": B * ws_n, "seq_len": T, "parallelism": f"dp{ws_n}",
                            "step": "fwd(save) + bwd", "l2": "inputs larger than L2 (no flush)"},
                 "tc_frac_of_bf16_peak": tc_frac,
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "prologue": prologue,
                 "gpu_launches": launches, "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
                 "kernel_rooflines": kernels,
                 "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],

@@ -15,7 +15,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "workspace_size", "device_status", "library_path",
+__all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
+           "workspace_size", "device_status", "library_path",
            "KronDeltaError", "KronDeltaFunction", "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -24,7 +25,7 @@ _lib = None
 
 KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE, KD_ERR_CUDA, KD_ERR_TIMEOUT = range(6)
 KD_F32, KD_BF16 = 0, 1
-KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD = 0, 1, 2, 3
+KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD, KD_WS_EPILOGUE_BWD = 0, 1, 2, 3, 4
 _CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
           4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
 
@@ -67,6 +68,10 @@ def lib():
         L.kron_delta_prologue_bwd.restype = i
         L.kron_delta_prologue_bwd.argtypes = ([vp] * 7 + [ctypes.c_float] + [vp] * 13 + [i] * 6 +
                                               [vp, sz, vp])
+        L.kron_delta_epilogue_fwd.restype = i
+        L.kron_delta_epilogue_fwd.argtypes = [vp] * 4 + [i] * 5 + [vp]
+        L.kron_delta_epilogue_bwd.restype = i
+        L.kron_delta_epilogue_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, sz, vp]
         L.kron_delta_profile_enable.restype = None
         L.kron_delta_profile_enable.argtypes = [i]
         L.kron_delta_profile_report.restype = i
@@ -255,6 +260,40 @@ def prologue_bwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, dq, dk, dv,
                                          B, H, T, dk_, dv_, dt, _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _stream(stream)))
     return g
+
+
+def _epilogue_inputs(o, g, w):
+    import torch
+    B, T, H, dv = o.shape
+    _need(o, "o"); _need(g, "g", o.dtype, o.shape); _need(w, "w", torch.float32, (dv,))
+    return B, T, H, dv, _dtype_code(o)
+
+
+def epilogue_fwd(o, g, w, *, out=None, stream=None):
+    """Output epilogue: y = w * o / rms(o) * sigmoid(g) per token and head
+    (rms over the head's dv channels, eps 1e-6).  o, g [B,T,H,dv] (bf16 or
+    fp32, one dtype); w [dv] fp32.  Returns y [B,T,H,dv]."""
+    import torch
+    B, T, H, dv, dt = _epilogue_inputs(o, g, w)
+    y = torch.empty_like(o) if out is None else out
+    _need(y, "y", o.dtype, o.shape)
+    _check(lib().kron_delta_epilogue_fwd(_ptr(o), _ptr(g), _ptr(w), _ptr(y), B, H, T, dv, dt, _stream(stream)))
+    return y
+
+
+def epilogue_bwd(o, g, w, dy, *, workspace=None, stream=None):
+    """Backward of epilogue_fwd for the loss <dy, y>.  Returns dict dO, dg, dw."""
+    import torch
+    B, T, H, dv, dt = _epilogue_inputs(o, g, w)
+    _need(dy, "dy", o.dtype, o.shape)
+    r = dict(dO=torch.empty_like(o), dg=torch.empty_like(g), dw=torch.empty_like(w))
+    need = workspace_size(KD_WS_EPILOGUE_BWD, B, H, T, 32, dv, dt)
+    if workspace is None:
+        workspace = _alloc_ws(need, o.device)
+    _check(lib().kron_delta_epilogue_bwd(_ptr(o), _ptr(g), _ptr(w), _ptr(dy), _ptr(r["dO"]), _ptr(r["dg"]),
+                                         _ptr(r["dw"]), B, H, T, dv, dt, _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return r
 
 
 def device_status(stream=None):

@@ -235,6 +235,9 @@ size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv, 
     case KD_WS_PROLOGUE_BWD:
       ok();
       return align256((size_t)kd::prologue_blocks((long long)B * T) * H * sizeof(float));
+    case KD_WS_EPILOGUE_BWD:
+      ok();
+      return align256((size_t)kd::epilogue_blocks((long long)B * T * H) * dv * sizeof(float));
     default: fail(KD_ERR_INVALID_ARG, "unknown workspace kind %d", kind); return 0;
   }
 }
@@ -417,6 +420,50 @@ int kron_delta_prologue_bwd(const void* q_raw, const void* k_raw, const void* v_
   a.part = static_cast<float*>(workspace);
   a.N = N; a.H = H; a.dk = dk_; a.dv = dv_; a.dtype = dtype;
   return launched(kd::launch_prologue_bwd(a, static_cast<cudaStream_t>(stream)), "prologue backward launch");
+}
+
+namespace {
+int check_epilogue(const void* o, const void* g, const float* w, int B, int H, int T, int dv, int dtype) {
+  if (B <= 0 || H <= 0 || T <= 0) return fail(KD_ERR_INVALID_ARG, "B, H, T must be >= 1 (got %d, %d, %d)", B, H, T);
+  if (!dim_supported(dv)) return fail(KD_ERR_UNSUPPORTED, "dv must be 32, 64 or 128 (got %d)", dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  KD_TRY(check_ptr(o, "o", true));
+  KD_TRY(check_ptr(g, "g", true));
+  return check_ptr(w, "w", true);
+}
+}  // namespace
+
+int kron_delta_epilogue_fwd(const void* o, const void* g, const float* w, void* y, int B, int H, int T,
+                            int dv, int dtype, void* stream) {
+  KD_TRY(check_epilogue(o, g, w, B, H, T, dv, dtype));
+  KD_TRY(check_ptr(y, "y", true));
+  KD_TRY(check_stream(stream));
+  kd::EpilogueArgs a{};
+  a.o = o; a.g = g; a.w = w; a.y = y;
+  a.rows = (long long)B * T * H; a.dv = dv; a.dtype = dtype;
+  return launched(kd::launch_epilogue_fwd(a, static_cast<cudaStream_t>(stream)), "epilogue launch");
+}
+
+int kron_delta_epilogue_bwd(const void* o, const void* g, const float* w, const void* dy, void* dO,
+                            void* dg, float* dw, int B, int H, int T, int dv, int dtype, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  KD_TRY(check_epilogue(o, g, w, B, H, T, dv, dtype));
+  KD_TRY(check_ptr(dy, "dy", true));
+  KD_TRY(check_ptr(dO, "dO", true));
+  KD_TRY(check_ptr(dg, "dg", true));
+  KD_TRY(check_ptr(dw, "dw", true));
+  const long long rows = (long long)B * T * H;
+  const size_t need = (size_t)kd::epilogue_blocks(rows) * dv * sizeof(float);
+  if (!workspace || ws_bytes < need)
+    return fail(KD_ERR_WORKSPACE, "epilogue workspace of %zu bytes needed (got %zu)", need,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  kd::EpilogueArgs a{};
+  a.o = o; a.g = g; a.w = w; a.dy = dy; a.dO = dO; a.dg = dg; a.dw = dw;
+  a.part = static_cast<float*>(workspace);
+  a.rows = rows; a.dv = dv; a.dtype = dtype;
+  return launched(kd::launch_epilogue_bwd(a, static_cast<cudaStream_t>(stream)), "epilogue backward launch");
 }
 
 void kron_delta_profile_enable(int on) {

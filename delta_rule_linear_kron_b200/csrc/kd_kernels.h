@@ -126,6 +126,22 @@ int prologue_blocks(long long N);
 cudaError_t launch_prologue_fwd(const PrologueArgs& a, cudaStream_t st);
 cudaError_t launch_prologue_bwd(const PrologueArgs& a, cudaStream_t st);
 
+// Output epilogue (kd_epilogue.cu).  rows = B*T*H rows of dv channels.
+struct EpilogueArgs {
+  const void *o, *g;
+  const float* w;
+  void* y;                 // forward output
+  const void* dy;          // backward: upstream gradient in
+  void *dO, *dg;           // backward: gradients out
+  float* dw;
+  float* part;             // backward scratch: epilogue_blocks(rows) * dv floats
+  long long rows;
+  int dv, dtype;
+};
+int epilogue_blocks(long long rows);
+cudaError_t launch_epilogue_fwd(const EpilogueArgs& a, cudaStream_t st);
+cudaError_t launch_epilogue_bwd(const EpilogueArgs& a, cudaStream_t st);
+
 template <typename T>
 inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }
 template <typename T>

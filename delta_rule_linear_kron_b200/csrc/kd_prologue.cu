@@ -31,8 +31,8 @@
 // reduced deterministically: each block writes one partial per head in a fixed
 // warp order, and a second small kernel adds the nb partials of a head in a
 // fixed order.
-#include "kd_common.cuh"
 #include "kd_kernels.h"
+#include "kd_rows.cuh"
 
 namespace kd {
 
@@ -40,50 +40,7 @@ namespace {
 
 constexpr float kNormEps = 1e-6f;
 
-template <typename T, int E>
-struct alignas(sizeof(T) * E) Pack {
-  T x[E];
-};
-
-template <typename T, int E>
-__device__ __forceinline__ void store_row(T* p, const float (&in)[E]) {
-  Pack<T, E> t;
-#pragma unroll
-  for (int i = 0; i < E; ++i) t.x[i] = from_f<T>(in[i]);
-  *reinterpret_cast<Pack<T, E>*>(p) = t;
-}
-
-// __ldcs has no overload for the packed structs; go through their raw bits.
-template <int BYTES> struct RawOf;
-template <> struct RawOf<2> { using type = unsigned short; };
-template <> struct RawOf<4> { using type = unsigned int; };
-template <> struct RawOf<8> { using type = uint2; };
-template <> struct RawOf<16> { using type = uint4; };
-
 }  // namespace
-
-template <typename T, int E>
-__device__ __forceinline__ Pack<T, E> ldcs_pack(const Pack<T, E>* p) {
-  using R = typename RawOf<sizeof(Pack<T, E>)>::type;
-  R r = __ldcs(reinterpret_cast<const R*>(p));
-  Pack<T, E> t;
-  memcpy(&t, &r, sizeof(t));
-  return t;
-}
-
-template <typename T, int E>
-__device__ __forceinline__ void load_stream(const T* p, float (&out)[E]) {
-  const Pack<T, E> t = ldcs_pack(reinterpret_cast<const Pack<T, E>*>(p));
-#pragma unroll
-  for (int i = 0; i < E; ++i) out[i] = to_f(t.x[i]);
-}
-
-__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
-
-// log sigmoid(x) = -(max(-x, 0) + log1p(exp(-|x|))), finite for every finite x.
-__device__ __forceinline__ float log_sigmoidf_(float x) {
-  return -(fmaxf(-x, 0.f) + log1pf(expf(-fabsf(x))));
-}
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(256) prologue_fwd_kernel(

@@ -23,6 +23,9 @@ Recipe (shapes and distributions of the five workloads):
     c-pre ~ N(0,1) (fp32); f-pre ~ N(3,1) (storage dtype); a_log ~ U(-1,1)
     (fp32); upstream gradients N(0,1) (dq, dk, dv in the storage dtype, the
     gate gradients fp32).
+  * epilogue inputs (``make_epilogue_inputs``), in the order o, g, w, dy:
+    o ~ N(0, 0.1^2) (a read-out's scale), g ~ N(0,1), dy ~ N(0,1) (storage
+    dtype); w ~ 1 + N(0, 0.1^2) (fp32).
 All arrays are returned as float64 numpy arrays holding exactly the values the
 GPU receives (bf16-representable where the dtype is bf16).
 """
@@ -33,6 +36,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs", "make_prologue_inputs",
+           "make_epilogue_inputs",
            "round_to_dtype", "decode_token_inputs_torch"]
 
 
@@ -144,6 +148,16 @@ def make_prologue_inputs(B, H, T, dk, dv, dtype="bf16", seed=2000, with_grads=Tr
                    dc=round_to_dtype(rng.standard_normal((B, T, H)), "f32"),
                    dlogf=round_to_dtype(rng.standard_normal((B, T, H, dk)), "f32"))
     return out
+
+
+def make_epilogue_inputs(B, H, T, dv, dtype="bf16", seed=3000):
+    """Inputs of the output epilogue as float64 arrays holding the values the GPU
+    receives: o, g, dy [B,T,H,dv] and w [dv]."""
+    rng = np.random.default_rng(seed)
+    return dict(o=round_to_dtype(0.1 * rng.standard_normal((B, T, H, dv)), dtype),
+                g=round_to_dtype(rng.standard_normal((B, T, H, dv)), dtype),
+                w=round_to_dtype(1.0 + 0.1 * rng.standard_normal(dv), "f32"),
+                dy=round_to_dtype(rng.standard_normal((B, T, H, dv)), dtype))
 
 
 def make_decode_inputs(steps: int, *, B=256, H=16, dk=128, dv=128, dtype="bf16",

@@ -80,6 +80,8 @@ extern "C" {
 #define KD_WS_BWD 2        /* backward scratch (besides the saved forward) */
 #define KD_WS_PROLOGUE_BWD 3  /* scratch of kron_delta_prologue_bwd (dk, dv, dtype
                                  must be valid but do not change the size) */
+#define KD_WS_EPILOGUE_BWD 4  /* scratch of kron_delta_epilogue_bwd (dk and dtype
+                                 must be valid but do not change the size) */
 
 /* Library version, as 10000*major + 100*minor + patch. */
 KD_API int kron_delta_version(void);
@@ -223,6 +225,39 @@ KD_API int kron_delta_prologue_bwd(const void *q_raw, const void *k_raw, const v
                                    void *dv_raw, float *dbeta_pre, float *dc_pre, void *df_pre,
                                    float *da_log, int B, int H, int T, int dk_, int dv_, int dtype,
                                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Output epilogue: per-head RMSNorm of the read-out followed by the sigmoid
+ * output gate, one fused pass.  KronLSTM digest, section "어떻게 쓰나": the
+ * read-out passes through a sigmoid output gate and a per-head RMSNorm
+ * before the output projection (the projection is not part of this call).
+ * Reading of the order and the constant: norm first, eps = 1e-6, a weight w
+ * per channel shared by the heads.  Per token t, head h, channel j:
+ *     y[j] = w[j] * o[j] / sqrt(mean_i o[i]^2 + 1e-6) * sigmoid(g[j])
+ *   o : the read-out [B,T,H,dv] (dtype), e.g. kron_delta_fwd's out.
+ *   g : the gate's pre-activation [B,T,H,dv] (dtype).   w : [dv] fp32.
+ *   y : [B,T,H,dv] (dtype).  All 16-byte aligned.  No workspace.
+ * Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_CUDA.  Asynchronous
+ * on `stream`.
+ */
+KD_API int kron_delta_epilogue_fwd(const void *o, const void *g, const float *w, void *y, int B,
+                                   int H, int T, int dv, int dtype, void *stream);
+
+/*
+ * Backward of kron_delta_epilogue_fwd for the loss l = <dy, y>.
+ *   dy : [B,T,H,dv] (dtype).
+ *   dO, dg : gradients of o and g, [B,T,H,dv] (dtype).  dO can be passed on
+ *   to kron_delta_bwd as its dO.
+ *   dw : [dv] fp32, overwritten (not accumulated); summed over tokens and
+ *   heads in a fixed order, so bitwise reproducible.
+ *   workspace, ws_bytes : scratch of at least
+ *     kron_delta_workspace_size(KD_WS_EPILOGUE_BWD, ...), 256-byte aligned.
+ * Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE,
+ * KD_ERR_CUDA.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_epilogue_bwd(const void *o, const void *g, const float *w, const void *dy,
+                                   void *dO, void *dg, float *dw, int B, int H, int T, int dv,
+                                   int dtype, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Synchronises `stream` and reports device-side failures of earlier calls:

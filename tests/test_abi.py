@@ -152,3 +152,21 @@ def test_prologue_argument_errors(L):
     # one partial per (block of 64 tokens, head)
     big = kd.workspace_size(kd.KD_WS_PROLOGUE_BWD, 2, 16, 16384, 128, 128)
     assert big >= (2 * 16384 // 64) * 16 * 4
+
+
+def test_epilogue_argument_errors(L):
+    p = ctypes.c_void_p(256)
+    assert L.kron_delta_epilogue_fwd(p, p, p, p, 1, 2, 10, 96, 1, None) == kd.KD_ERR_UNSUPPORTED
+    assert L.kron_delta_epilogue_fwd(p, p, p, p, 1, 2, 10, 64, 5, None) == kd.KD_ERR_UNSUPPORTED
+    assert L.kron_delta_epilogue_fwd(p, p, None, p, 1, 2, 10, 64, 1, None) == kd.KD_ERR_INVALID_ARG
+    assert b"w must not be NULL" in L.kron_delta_last_error()
+    assert L.kron_delta_epilogue_fwd(p, p, p, p, 1, 0, 10, 64, 1, None) == kd.KD_ERR_INVALID_ARG
+    assert L.kron_delta_epilogue_bwd(p, p, p, p, p, p, None, 1, 2, 10, 64, 1, p, 1 << 20, None) == \
+        kd.KD_ERR_INVALID_ARG
+    assert L.kron_delta_epilogue_bwd(p, p, p, p, p, p, p, 1, 2, 10, 64, 1, p, 0, None) == kd.KD_ERR_WORKSPACE
+    need = kd.workspace_size(kd.KD_WS_EPILOGUE_BWD, 1, 2, 10, 64, 64)
+    assert need >= 64 * 4 and need % 256 == 0
+    assert L.kron_delta_epilogue_bwd(p, p, p, p, p, p, p, 1, 2, 10, 64, 1, ctypes.c_void_p(256 + 32), need,
+                                     None) == kd.KD_ERR_WORKSPACE
+    # partial rows are capped, so the scratch stays small at any size
+    assert kd.workspace_size(kd.KD_WS_EPILOGUE_BWD, 64, 64, 65536, 128, 128) <= 4096 * 128 * 4 + 256
