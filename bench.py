@@ -7,7 +7,8 @@ forward+backward workload B=1, H=16, T=16384, d_k=d_v=128, bf16 q/k/v/dO,
 fp32 gates and state, beta in (0,2), nonzero S0.  The decode step
 (B=256, H=16, d=128, 1000 consecutive in-place steps) is timed in the same run
 and reported under "decode"; the input prologue (raw projections -> normalised
-q, k, v and gates) and its backward, on the step's shape, under "prologue".
+q, k, v and gates), the output epilogue (RMSNorm and output gate) and their
+backward passes, on the step's shape, under "prologue_epilogue".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -95,6 +96,9 @@ def kernel_work(name, d=128, C=CHUNK):
         "prologue_fwd": ("alu", 20 * 4 * d, 4 * act + 8 + 3 * act + lf + 8),
         # reads q~, k~, v~, f~, dq, dk, dv, dlogf and four gate scalars; writes dq~, dk~, dv~, df~ and two
         "prologue_bwd": ("alu", 30 * 4 * d, 4 * act + 3 * act + lf + 16 + 4 * act + 8),
+        # output epilogue (timed on its own): reads o, g; writes y.  Backward: reads o, g, dy; writes dO, dg
+        "epilogue_fwd": ("alu", 20 * d, 2 * act + act),
+        "epilogue_bwd": ("alu", 40 * d, 3 * act + 2 * act),
     }
     w = table.get(name)
     return None if w is None else dict(kind=w[0], flops=w[1], bytes=w[2])
@@ -403,17 +407,26 @@ def main(argv=None):
                   a_log=torch.rand((H,), generator=g_, device=dev) * 2 - 1)
         up = dict(dq=rn(B, T, H, dk).to(bf), dk=rn(B, T, H, dk).to(bf), dv=rn(B, T, H, dv).to(bf),
                   dbeta=rn(B, T, H), dc=rn(B, T, H), dlogf=rn(B, T, H, dk))
+        ep = dict(o=(0.1 * rn(B, T, H, dv)).to(bf), g=rn(B, T, H, dv).to(bf), w=1 + 0.1 * rn(dv),
+                  dy=rn(B, T, H, dv).to(bf))
+        ews = torch.empty(kd.workspace_size(kd.KD_WS_EPILOGUE_BWD, B, H, T, dk, dv), dtype=torch.uint8,
+                          device=dev)
+        y_ep = torch.empty_like(ep["o"])
         pws = torch.empty(kd.workspace_size(kd.KD_WS_PROLOGUE_BWD, B, H, T, dk, dv), dtype=torch.uint8,
                           device=dev)
         order = ("q_raw", "k_raw", "v_raw", "beta_pre", "c_pre", "f_pre", "a_log")
         times = {}
-        for name in ("prologue_fwd", "prologue_bwd"):
+        for name in ("prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd"):
             def call():
                 if name == "prologue_fwd":
                     kd.prologue_fwd(*(pr[n] for n in order), 2.0)
-                else:
+                elif name == "prologue_bwd":
                     kd.prologue_bwd(*(pr[n] for n in order), up["dq"], up["dk"], up["dv"], up["dbeta"], up["dc"],
                                     up["dlogf"], 2.0, workspace=pws)
+                elif name == "epilogue_fwd":
+                    kd.epilogue_fwd(ep["o"], ep["g"], ep["w"], out=y_ep)
+                else:
+                    kd.epilogue_bwd(ep["o"], ep["g"], ep["w"], ep["dy"], workspace=ews)
             for _ in range(3):
                 call()
             torch.cuda.synchronize()
@@ -431,9 +444,9 @@ def main(argv=None):
             times[name] = dict(ms=ms, algorithmic_bytes_per_launch=w["bytes"] * B * H * T, achieved_gbs=gbs,
                                hbm_frac=gbs / peaks["hbm_gbs"])
         kd.device_status()
-        prologue = dict(times, note="timed alone, not part of the step; the bwd time includes the small "
-                                    "fixed-order da_log reduction launch")
-        del pr, up
+        prologue = dict(times, note="timed alone, not part of the step; each bwd time includes its small "
+                                    "fixed-order reduction launch (da_log, dw)")
+        del pr, up, ep
     clocks = sampler.stop()
 
     # ---- end to end through the public API with pinned host buffers -----
@@ -513,7 +526,7 @@ def main(argv=None):
                            "global_batch": B * ws_n, "seq_len": T, "parallelism": f"dp{ws_n}",
                            "step": "fwd(save) + bwd", "l2": "inputs larger than L2 (no flush)"},
                 "tc_frac_of_bf16_peak": tc_frac,
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "prologue": prologue,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "prologue_epilogue": prologue,
                 "gpu_launches": launches, "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
                 "kernel_rooflines": kernels,
                 "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
