@@ -26,6 +26,7 @@ _lib = None
 KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE, KD_ERR_CUDA, KD_ERR_TIMEOUT = range(6)
 KD_F32, KD_BF16 = 0, 1
 KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD, KD_WS_EPILOGUE_BWD = 0, 1, 2, 3, 4
+KD_PHASE_LOCAL, KD_PHASE_CARRY, KD_PHASE_ALL = 1, 2, 3
 _CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
           4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
 
@@ -61,6 +62,10 @@ def lib():
         L.kron_delta_decode.argtypes = [vp] * 8 + [i] * 5 + [vp]
         L.kron_delta_device_status.restype = i
         L.kron_delta_device_status.argtypes = [vp]
+        L.kron_delta_fwd_phase.restype = i
+        L.kron_delta_fwd_phase.argtypes = [vp] * 9 + [i] * 6 + [vp, sz, i, i, vp]
+        L.kron_delta_bwd_phase.restype = i
+        L.kron_delta_bwd_phase.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp, sz, i, vp]
         L.kron_delta_fwd_noalloc.restype = i
         L.kron_delta_fwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [vp]
         L.kron_delta_prologue_fwd.restype = i
@@ -130,10 +135,12 @@ def _alloc_ws(nbytes, device):
 
 
 def fwd(q, k, v, beta, c, logf, S0=None, *, out=None, want_state=True, save=False,
-        workspace=None, stream=None):
+        workspace=None, phase=KD_PHASE_ALL, state_out=None, stream=None):
     """Chunk-parallel forward.  q,k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32);
     beta, c [B,T,H] fp32; logf [B,T,H,dk] fp32; S0 [B,H,dv,dk] fp32 or None.
-    Returns (out [B,T,H,dv], ST [B,H,dv,dk] or None, workspace)."""
+    Returns (out [B,T,H,dv], ST [B,H,dv,dk] or None, workspace).
+    phase: KD_PHASE_LOCAL enqueues only the S0-independent work, KD_PHASE_CARRY
+    the rest (pass the LOCAL call's workspace, out and state_out back in)."""
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -145,21 +152,27 @@ def fwd(q, k, v, beta, c, logf, S0=None, *, out=None, want_state=True, save=Fals
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     _need(out, "out", q.dtype, (B, T, H, dv))
-    ST = torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_state else None
+    ST = state_out
+    if ST is None and want_state:
+        ST = torch.empty((B, H, dv, dk), dtype=f32, device=q.device)
+    _need(ST, "state_out", f32, (B, H, dv, dk))
     need = workspace_size(KD_WS_FWD_SAVE if save else KD_WS_FWD, B, H, T, dk, dv, dt)
     if workspace is None:
         workspace = _alloc_ws(need, q.device)
-    _check(lib().kron_delta_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S0),
-                                _ptr(out), _ptr(ST), B, H, T, dk, dv, dt, _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), int(bool(save)),
-                                _stream(stream)))
+    _check(lib().kron_delta_fwd_phase(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S0),
+                                      _ptr(out), _ptr(ST), B, H, T, dk, dv, dt, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), int(bool(save)), int(phase),
+                                      _stream(stream)))
     return out, ST, workspace
 
 
 def bwd(q, k, v, beta, c, logf, S0, dO, dST=None, *, fwd_workspace, workspace=None,
-        want_dS0=True, stream=None):
+        want_dS0=True, phase=KD_PHASE_ALL, grads=None, stream=None):
     """Backward for loss <dO, out> + <dST, ST>, reading what fwd(save=True)
-    left in fwd_workspace.  Returns dict dq, dk, dv, dbeta, dc, dlogf, dS0."""
+    left in fwd_workspace.  Returns dict dq, dk, dv, dbeta, dc, dlogf, dS0.
+    phase: KD_PHASE_LOCAL enqueues only the dST-independent work, KD_PHASE_CARRY
+    the rest (allocate the workspace with workspace_size(KD_WS_BWD, ...) and pass
+    it, and the LOCAL call's returned grads, to both calls)."""
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -169,19 +182,25 @@ def bwd(q, k, v, beta, c, logf, S0, dO, dST=None, *, fwd_workspace, workspace=No
     _need(logf, "logf", f32, (B, T, H, dk)); _need(S0, "S0", f32, (B, H, dv, dk))
     _need(dO, "dO", q.dtype, (B, T, H, dv)); _need(dST, "dST", f32, (B, H, dv, dk))
     dt = _dtype_code(q)
-    g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
-             dbeta=torch.empty_like(beta), dc=torch.empty_like(c), dlogf=torch.empty_like(logf),
-             dS0=torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_dS0 else None)
+    if grads is None:
+        g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                 dbeta=torch.empty_like(beta), dc=torch.empty_like(c), dlogf=torch.empty_like(logf),
+                 dS0=torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_dS0 else None)
+    else:
+        g = grads
+        for n, ref in (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta), ("dc", c), ("dlogf", logf)):
+            _need(g[n], n, ref.dtype, ref.shape)
+        _need(g.get("dS0"), "dS0", f32, (B, H, dv, dk))
     need = workspace_size(KD_WS_BWD, B, H, T, dk, dv, dt)
     if workspace is None:
         workspace = _alloc_ws(need, q.device)
-    _check(lib().kron_delta_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S0),
-                                _ptr(dO), _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
-                                _ptr(g["dbeta"]), _ptr(g["dc"]), _ptr(g["dlogf"]), _ptr(g["dS0"]),
-                                B, H, T, dk, dv, dt, _ptr(fwd_workspace),
-                                fwd_workspace.numel() * fwd_workspace.element_size(),
-                                _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                _stream(stream)))
+    _check(lib().kron_delta_bwd_phase(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf), _ptr(S0),
+                                      _ptr(dO), _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                      _ptr(g["dbeta"]), _ptr(g["dc"]), _ptr(g["dlogf"]), _ptr(g.get("dS0")),
+                                      B, H, T, dk, dv, dt, _ptr(fwd_workspace),
+                                      fwd_workspace.numel() * fwd_workspace.element_size(),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(), int(phase),
+                                      _stream(stream)))
     return g
 
 

@@ -246,6 +246,16 @@ int kron_delta_fwd(const void* q, const void* k, const void* v, const float* bet
                    const float* c, const float* logf, const float* S0, void* out, float* ST,
                    int B, int H, int T, int dk, int dv, int dtype, void* workspace,
                    size_t ws_bytes, int save, void* stream) {
+  return kron_delta_fwd_phase(q, k, v, beta, c, logf, S0, out, ST, B, H, T, dk, dv, dtype, workspace,
+                              ws_bytes, save, KD_PHASE_ALL, stream);
+}
+
+int kron_delta_fwd_phase(const void* q, const void* k, const void* v, const float* beta,
+                         const float* c, const float* logf, const float* S0, void* out, float* ST,
+                         int B, int H, int T, int dk, int dv, int dtype, void* workspace,
+                         size_t ws_bytes, int save, int phase, void* stream) {
+  if (phase != KD_PHASE_LOCAL && phase != KD_PHASE_CARRY && phase != KD_PHASE_ALL)
+    return fail(KD_ERR_INVALID_ARG, "phase must be KD_PHASE_LOCAL, KD_PHASE_CARRY or KD_PHASE_ALL (got %d)", phase);
   kd::Layout L;
   KD_TRY(plan(B, H, T, dk, dv, dtype, &L));
   KD_TRY(check_ptr(q, "q", true));
@@ -263,7 +273,7 @@ int kron_delta_fwd(const void* q, const void* k, const void* v, const float* bet
     return fail(KD_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace ? ws_bytes : 0);
   if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   KD_TRY(check_stream(stream));
-  kd::FwdArgs a{q, k, v, beta, c, logf, S0, out, ST, save, static_cast<char*>(workspace), L};
+  kd::FwdArgs a{q, k, v, beta, c, logf, S0, out, ST, save, static_cast<char*>(workspace), L, phase};
   if (L.tc) {
     DeviceInfo di;
     KD_TRY(device_info(&di));
@@ -279,6 +289,19 @@ int kron_delta_bwd(const void* q, const void* k, const void* v, const float* bet
                    float* dlogf, float* dS0, int B, int H, int T, int dk_, int dv_, int dtype,
                    const void* fwd_ws, size_t fwd_ws_bytes, void* workspace, size_t ws_bytes,
                    void* stream) {
+  return kron_delta_bwd_phase(q, k, v, beta, c, logf, S0, dO, dST, dq, dk, dv, dbeta, dc, dlogf, dS0, B, H,
+                              T, dk_, dv_, dtype, fwd_ws, fwd_ws_bytes, workspace, ws_bytes, KD_PHASE_ALL,
+                              stream);
+}
+
+int kron_delta_bwd_phase(const void* q, const void* k, const void* v, const float* beta,
+                         const float* c, const float* logf, const float* S0, const void* dO,
+                         const float* dST, void* dq, void* dk, void* dv, float* dbeta, float* dc,
+                         float* dlogf, float* dS0, int B, int H, int T, int dk_, int dv_, int dtype,
+                         const void* fwd_ws, size_t fwd_ws_bytes, void* workspace, size_t ws_bytes,
+                         int phase, void* stream) {
+  if (phase != KD_PHASE_LOCAL && phase != KD_PHASE_CARRY && phase != KD_PHASE_ALL)
+    return fail(KD_ERR_INVALID_ARG, "phase must be KD_PHASE_LOCAL, KD_PHASE_CARRY or KD_PHASE_ALL (got %d)", phase);
   kd::Layout L;
   KD_TRY(plan(B, H, T, dk_, dv_, dtype, &L));
   KD_TRY(check_ptr(q, "q", true));
@@ -308,7 +331,7 @@ int kron_delta_bwd(const void* q, const void* k, const void* v, const float* bet
   KD_TRY(check_stream(stream));
   (void)S0;  // the forward state at every chunk start is read from fwd_ws
   kd::BwdArgs a{q, k, v, beta, c, logf, S0, dO, dST, dq, dk, dv, dbeta, dc, dlogf, dS0,
-                static_cast<const char*>(fwd_ws), static_cast<char*>(workspace), L};
+                static_cast<const char*>(fwd_ws), static_cast<char*>(workspace), L, phase};
   if (L.tc) {
     DeviceInfo di;
     KD_TRY(device_info(&di));

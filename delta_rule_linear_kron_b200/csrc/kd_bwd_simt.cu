@@ -689,7 +689,11 @@ static cudaError_t run_bwd_t(const BwdArgs& a, int stages, const int* only, cuda
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st) { return launch_bwd_simt_stages(a, kStageAll, nullptr, st); }
+cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st) {
+  // the reverse chain comes first and needs dST: no state-independent phase
+  if (!(a.phases & kPhaseCarry)) return cudaSuccess;
+  return launch_bwd_simt_stages(a, kStageAll, nullptr, st);
+}
 
 cudaError_t launch_bwd_simt_stages(const BwdArgs& a, int stages, const int* only, cudaStream_t st) {
   return a.L.dtype == 0 ? run_bwd_t<float>(a, stages, only, st) : run_bwd_t<__nv_bfloat16>(a, stages, only, st);

@@ -444,8 +444,11 @@ cudaError_t launch_bchain(const BwdArgs& a, int* err, cudaStream_t st) {
 
 cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st) {
   const Layout& L = a.L;
-  cudaError_t e = launch_bwd_pre_tc(a, err, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if (a.phases & kPhaseLocal) {
+    if ((e = launch_bwd_pre_tc(a, err, st)) != cudaSuccess) return e;
+  }
+  if (!(a.phases & kPhaseCarry)) return cudaSuccess;
   const int R = choose_cluster(L.B * L.H, sms);
   e = (R == 8) ? launch_bchain<8>(a, err, st) : launch_bchain<4>(a, err, st);
   if (e != cudaSuccess) return e;

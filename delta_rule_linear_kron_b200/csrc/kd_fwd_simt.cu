@@ -349,11 +349,14 @@ static cudaError_t run_fwd(const FwdArgs& a, cudaStream_t st) {
   const Tin* q = static_cast<const Tin*>(a.q);
   const Tin* k = static_cast<const Tin*>(a.k);
   const Tin* v = static_cast<const Tin*>(a.v);
-  prof_begin(st, "fwd_prep_simt");
-  fwd_prep_simt<DK, DV, Tin><<<dim3(L.NC, L.H, L.B), 256, sp, st>>>(
-      q, k, v, a.beta, a.c, a.logf, L.H, L.T, L.NC, wy, wA, wP);
-  prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.phases & kPhaseLocal) {
+    prof_begin(st, "fwd_prep_simt");
+    fwd_prep_simt<DK, DV, Tin><<<dim3(L.NC, L.H, L.B), 256, sp, st>>>(
+        q, k, v, a.beta, a.c, a.logf, L.H, L.T, L.NC, wy, wA, wP);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (!(a.phases & kPhaseCarry)) return cudaSuccess;
   prof_begin(st, "fwd_chain_simt");
   fwd_chain_simt<DK, DV, Tin><<<dim3(L.H, L.B), 2 * DV, sc, st>>>(
       q, k, v, a.beta, a.logf, a.S0, static_cast<Tin*>(a.out), a.ST, L.H, L.T, L.NC, wy, wA, wP,

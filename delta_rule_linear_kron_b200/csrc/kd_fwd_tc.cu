@@ -1204,7 +1204,7 @@ int choose_cluster(int units, int sms) {
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) {
   const Layout& L = a.L;
   cudaError_t e;
-  {
+  if (a.phases & kPhaseLocal) {
     CUtensorMap tm_v, tm_q, tm_k, tm_logf;
     if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
         !make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
@@ -1220,13 +1220,8 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
         a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  {
-    CUtensorMap tm_v, tm_k, tm_logf, tm_kt, tm_ke;
-    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
-        !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
-        !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
-        !make_tmap_bthd(&tm_kt, ws_ptr<float>(a.ws, L.Kt), 4, L.B, L.T, L.H, D, 128, false) ||
+    CUtensorMap tm_kt, tm_ke;
+    if (!make_tmap_bthd(&tm_kt, ws_ptr<float>(a.ws, L.Kt), 4, L.B, L.T, L.H, D, 128, false) ||
         !make_tmap_bthd(&tm_ke, ws_ptr<float>(a.ws, L.Ke), 4, L.B, L.T, L.H, D, 128, false))
       return cudaErrorInvalidValue;
     if ((e = cudaFuncSetAttribute(fwd_cross_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1239,6 +1234,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (!(a.phases & kPhaseCarry)) return cudaSuccess;
   const float* wy = ws_ptr<float>(a.ws, L.y);
   const float* wA = ws_ptr<float>(a.ws, L.A);
   float* blob = ws_ptr<float>(a.ws, L.S0);

@@ -48,6 +48,13 @@ struct Layout {
   size_t bwd_bytes = 0;
 };
 
+// Phases of a forward or backward call.  kPhaseLocal: the work that does not
+// depend on the carried state (the initial state S0 in the forward, the
+// final-state gradient dST in the backward); kPhaseCarry: the chain over
+// chunks and everything after it.  A carry phase needs the local phase of the
+// same call to have run before it on the same workspaces and inputs.
+constexpr int kPhaseLocal = 1, kPhaseCarry = 2, kPhaseAll = 3;
+
 struct DecodeArgs {
   const void *q, *k, *v;
   const float *beta, *c, *logf;
@@ -64,6 +71,7 @@ struct FwdArgs {
   int save;
   char* ws;  // workspace base
   Layout L;
+  int phases = kPhaseAll;
 };
 
 struct BwdArgs {
@@ -76,6 +84,7 @@ struct BwdArgs {
   const char* fws;  // forward workspace (saved)
   char* ws;         // backward workspace
   Layout L;
+  int phases = kPhaseAll;
 };
 
 // Sets the calling thread's kron_delta_last_error() string.

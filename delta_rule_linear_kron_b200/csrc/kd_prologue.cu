@@ -111,7 +111,7 @@ __device__ __forceinline__ void l2norm_bwd(float (&x)[E], const float (&g)[E]) {
 }
 
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(256) prologue_bwd_kernel(
+__global__ void __launch_bounds__(256, 4) prologue_bwd_kernel(
     const Tin* __restrict__ qr, const Tin* __restrict__ kr, const Tin* __restrict__ vr,
     const float* __restrict__ beta_pre, const float* __restrict__ c_pre, const Tin* __restrict__ fr,
     const float* __restrict__ a_log, float beta_scale, const Tin* __restrict__ dq,

@@ -83,6 +83,11 @@ extern "C" {
 #define KD_WS_EPILOGUE_BWD 4  /* scratch of kron_delta_epilogue_bwd (dk and dtype
                                  must be valid but do not change the size) */
 
+/* phases of kron_delta_fwd_phase / kron_delta_bwd_phase */
+#define KD_PHASE_LOCAL 1   /* the work that does not depend on the carried state */
+#define KD_PHASE_CARRY 2   /* the chunk chain and everything after it */
+#define KD_PHASE_ALL 3     /* both, in order (what kron_delta_fwd / _bwd do) */
+
 /* Library version, as 10000*major + 100*minor + patch. */
 KD_API int kron_delta_version(void);
 
@@ -139,6 +144,41 @@ KD_API int kron_delta_bwd(const void *q, const void *k, const void *v,
                    float *dlogf, float *dS0, int B, int H, int T, int dk_,
                    int dv_, int dtype, const void *fwd_ws, size_t fwd_ws_bytes,
                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * The forward and backward split at the carried state, for a caller that
+ * holds one time segment of every sequence and receives the state at the
+ * segment's start from elsewhere (e.g. a context-parallel relay, where the
+ * previous segment lives on another GPU).  The chunk-local work (the
+ * triangular inverses, the Grams and the cross-chunk operands in the forward;
+ * the per-chunk adjoints in the backward) does not depend on S0 (forward) or
+ * dST (backward), so it can run while that state is still on its way.
+ *   phase = KD_PHASE_LOCAL : enqueue only the state-independent work.  S0,
+ *           out, ST (forward) and dST, the gradients, dS0 (backward) are
+ *           neither read nor written, but the argument checks are the same
+ *           as for the carry call: pass the buffers it will use.
+ *   phase = KD_PHASE_CARRY : enqueue the rest.  Must follow a LOCAL call with
+ *           the same inputs, sizes, save flag and workspaces, on the same
+ *           stream or after it completed; the workspace must not be reused in
+ *           between.
+ *   phase = KD_PHASE_ALL   : both; identical to kron_delta_fwd / _bwd.
+ * The KronLSTM digest's chunk-parallel form ("무엇과 다른가") is what makes the
+ * split possible: inside a chunk everything but the state terms is local.
+ * Arguments and errors otherwise as kron_delta_fwd / kron_delta_bwd.
+ */
+KD_API int kron_delta_fwd_phase(const void *q, const void *k, const void *v,
+                                const float *beta, const float *c, const float *logf,
+                                const float *S0, void *out, float *ST, int B, int H, int T,
+                                int dk, int dv, int dtype, void *workspace, size_t ws_bytes,
+                                int save, int phase, void *stream);
+
+KD_API int kron_delta_bwd_phase(const void *q, const void *k, const void *v,
+                                const float *beta, const float *c, const float *logf,
+                                const float *S0, const void *dO, const float *dST,
+                                void *dq, void *dk, void *dv, float *dbeta, float *dc,
+                                float *dlogf, float *dS0, int B, int H, int T, int dk_,
+                                int dv_, int dtype, const void *fwd_ws, size_t fwd_ws_bytes,
+                                void *workspace, size_t ws_bytes, int phase, void *stream);
 
 /*
  * One recurrent decode step: one new token per (b, h).

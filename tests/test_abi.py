@@ -170,3 +170,18 @@ def test_epilogue_argument_errors(L):
                                      None) == kd.KD_ERR_WORKSPACE
     # partial rows are capped, so the scratch stays small at any size
     assert kd.workspace_size(kd.KD_WS_EPILOGUE_BWD, 64, 64, 65536, 128, 128) <= 4096 * 128 * 4 + 256
+
+
+def test_phase_argument_errors(L):
+    p = ctypes.c_void_p(256)
+    for bad in (0, 4, -1):
+        rc = L.kron_delta_fwd_phase(p, p, p, p, p, p, None, p, None, 1, 1, 64, 32, 32, 1, p, 1 << 20, 0, bad, None)
+        assert rc == kd.KD_ERR_INVALID_ARG
+        assert b"phase" in L.kron_delta_last_error()
+        rc = L.kron_delta_bwd_phase(p, p, p, p, p, p, None, p, None, p, p, p, p, p, p, None, 1, 1, 64, 32, 32, 1,
+                                    p, 1 << 20, p, 1 << 20, bad, None)
+        assert rc == kd.KD_ERR_INVALID_ARG
+    # a valid phase still validates the rest before touching the GPU
+    rc = L.kron_delta_fwd_phase(p, p, p, p, p, p, None, p, None, 1, 1, 64, 48, 32, 1, p, 1 << 20, 0,
+                                kd.KD_PHASE_LOCAL, None)
+    assert rc == kd.KD_ERR_UNSUPPORTED
