@@ -16,6 +16,7 @@ import ctypes
 import os
 
 __all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
+           "gdn2_fwd", "gdn2_bwd",
            "workspace_size", "device_status", "library_path",
            "KronDeltaError", "KronDeltaFunction", "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
 
@@ -26,6 +27,7 @@ _lib = None
 KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE, KD_ERR_CUDA, KD_ERR_TIMEOUT = range(6)
 KD_F32, KD_BF16 = 0, 1
 KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD, KD_WS_EPILOGUE_BWD = 0, 1, 2, 3, 4
+KD_WS_GDN2_FWD, KD_WS_GDN2_BWD = 5, 6
 KD_PHASE_LOCAL, KD_PHASE_CARRY, KD_PHASE_ALL = 1, 2, 3
 _CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
           4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
@@ -77,6 +79,10 @@ def lib():
         L.kron_delta_epilogue_fwd.argtypes = [vp] * 4 + [i] * 5 + [vp]
         L.kron_delta_epilogue_bwd.restype = i
         L.kron_delta_epilogue_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, sz, vp]
+        L.kron_delta_gdn2_fwd.restype = i
+        L.kron_delta_gdn2_fwd.argtypes = [vp] * 9 + [i] * 6 + [vp, sz, vp]
+        L.kron_delta_gdn2_bwd.restype = i
+        L.kron_delta_gdn2_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp, sz, vp]
         L.kron_delta_profile_enable.restype = None
         L.kron_delta_profile_enable.argtypes = [i]
         L.kron_delta_profile_report.restype = i
@@ -313,6 +319,58 @@ def epilogue_bwd(o, g, w, dy, *, workspace=None, stream=None):
                                          _ptr(r["dw"]), B, H, T, dv, dt, _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _stream(stream)))
     return r
+
+
+def _gdn2_inputs(q, k, v, b, w, loga, S0):
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(b, "b", f32, (B, T, H, dk)); _need(w, "w", f32, (B, T, H, dv)); _need(loga, "loga", f32, (B, T, H, dk))
+    _need(S0, "S0", f32, (B, H, dv, dk))
+    return B, T, H, dk, dv, _dtype_code(q)
+
+
+def gdn2_fwd(q, k, v, b, w, loga, S0=None, *, out=None, want_state=True, workspace=None, stream=None):
+    """Gated DeltaNet-2 forward: per token Sbar = S diag(exp(loga)),
+    u = w*v - Sbar (b*k), S = Sbar + u k^T, o = S q.  q,k [B,T,H,dk], v [B,T,H,dv]
+    (bf16 or fp32); b, loga [B,T,H,dk] and w [B,T,H,dv] fp32; S0 [B,H,dv,dk] or
+    None.  Returns (out, ST or None, workspace); pass the workspace to gdn2_bwd."""
+    import torch
+    B, T, H, dk, dv, dt = _gdn2_inputs(q, k, v, b, w, loga, S0)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, (B, T, H, dv))
+    ST = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device) if want_state else None
+    if workspace is None:
+        workspace = _alloc_ws(workspace_size(KD_WS_GDN2_FWD, B, H, T, dk, dv, dt), q.device)
+    _check(lib().kron_delta_gdn2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(loga), _ptr(S0), _ptr(out),
+                                     _ptr(ST), B, H, T, dk, dv, dt, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, ST, workspace
+
+
+def gdn2_bwd(q, k, v, b, w, loga, S0, dO, dST=None, *, fwd_workspace, workspace=None, want_dS0=True,
+             stream=None):
+    """Backward of gdn2_fwd for the loss <dO, out> + <dST, ST>.  Returns dict
+    dq, dk, dv, db, dw, dloga, dS0."""
+    import torch
+    B, T, H, dk, dv, dt = _gdn2_inputs(q, k, v, b, w, loga, S0)
+    f32 = torch.float32
+    _need(dO, "dO", q.dtype, (B, T, H, dv)); _need(dST, "dST", f32, (B, H, dv, dk))
+    g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v), db=torch.empty_like(b),
+             dw=torch.empty_like(w), dloga=torch.empty_like(loga),
+             dS0=torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_dS0 else None)
+    if workspace is None:
+        workspace = _alloc_ws(workspace_size(KD_WS_GDN2_BWD, B, H, T, dk, dv, dt), q.device)
+    _check(lib().kron_delta_gdn2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(loga), _ptr(S0), _ptr(dO),
+                                     _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["db"]),
+                                     _ptr(g["dw"]), _ptr(g["dloga"]), _ptr(g["dS0"]), B, H, T, dk, dv, dt,
+                                     _ptr(fwd_workspace), fwd_workspace.numel() * fwd_workspace.element_size(),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)))
+    return g
 
 
 def device_status(stream=None):

@@ -102,6 +102,40 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   return KD_OK;
 }
 
+// Validates sizes and fills the Gated DeltaNet-2 workspace layout.
+int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
+  if (B <= 0 || H <= 0 || T <= 0) return fail(KD_ERR_INVALID_ARG, "B, H, T must be >= 1 (got %d, %d, %d)", B, H, T);
+  if (!dim_supported(dk) || !dim_supported(dv))
+    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  if (H > 65535 || B > 65535) return fail(KD_ERR_INVALID_ARG, "B and H must be <= 65535 (got %d, %d)", B, H);
+  const int NC = (T + kd::kChunk - 1) / kd::kChunk;
+  const size_t chunks = (size_t)B * H * NC;
+  if (chunks > (size_t(1) << 31)) return fail(KD_ERR_INVALID_ARG, "problem too large (%zu chunks)", chunks);
+  L->B = B; L->H = H; L->T = T; L->dk = dk; L->dv = dv; L->dtype = dtype; L->NC = NC; L->chunks = chunks;
+  const size_t C = kd::kChunk;
+  size_t off = 0;
+  auto take = [&](size_t floats) { size_t o = off; off = align256(off + floats * 4); return o; };
+  L->A = take(chunks * C * C);
+  L->P = take(chunks * C * C);
+  L->W = take(chunks * C * dk);
+  L->Up = take(chunks * C * dv);
+  L->Ke = take(chunks * C * dk);
+  L->Qp = take(chunks * C * dk);
+  L->gC = take(chunks * dk);
+  L->S0 = take(chunks * (size_t)dv * dk);
+  L->U = take(chunks * C * dv);
+  L->fwd_bytes = off;
+  off = 0;
+  L->dU = take(chunks * C * dv);
+  L->dS = take(chunks * (size_t)dv * dk);
+  L->dE = take(chunks * C * dk);
+  L->dT = take(chunks * C * C);
+  L->dP = take(chunks * C * C);
+  L->bwd_bytes = off;
+  return KD_OK;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int check_ptr(const void* p, const char* name, bool required) {
@@ -235,6 +269,13 @@ size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv, 
     case KD_WS_PROLOGUE_BWD:
       ok();
       return align256((size_t)kd::prologue_blocks((long long)B * T) * H * sizeof(float));
+    case KD_WS_GDN2_FWD:
+    case KD_WS_GDN2_BWD: {
+      kd::GdnLayout G;
+      if (gdn_plan(B, H, T, dk, dv, dtype, &G) != KD_OK) return 0;
+      ok();
+      return kind == KD_WS_GDN2_FWD ? G.fwd_bytes : G.bwd_bytes;
+    }
     case KD_WS_EPILOGUE_BWD:
       ok();
       return align256((size_t)kd::epilogue_blocks((long long)B * T * H) * dv * sizeof(float));
@@ -487,6 +528,73 @@ int kron_delta_epilogue_bwd(const void* o, const void* g, const float* w, const 
   a.part = static_cast<float*>(workspace);
   a.rows = rows; a.dv = dv; a.dtype = dtype;
   return launched(kd::launch_epilogue_bwd(a, static_cast<cudaStream_t>(stream)), "epilogue backward launch");
+}
+
+int kron_delta_gdn2_fwd(const void* q, const void* k, const void* v, const float* b, const float* w,
+                        const float* loga, const float* S0, void* out, float* ST, int B, int H, int T, int dk,
+                        int dv, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  kd::GdnLayout L;
+  KD_TRY(gdn_plan(B, H, T, dk, dv, dtype, &L));
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(b, "b", true));
+  KD_TRY(check_ptr(w, "w", true));
+  KD_TRY(check_ptr(loga, "loga", true));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(out, "out", true));
+  KD_TRY(check_ptr(ST, "ST", false));
+  if (!workspace || ws_bytes < L.fwd_bytes)
+    return fail(KD_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", L.fwd_bytes, workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  kd::GdnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.loga = loga; a.S0 = S0; a.out = out; a.ST = ST;
+  a.ws = static_cast<char*>(workspace);
+  a.L = L;
+  return launched(kd::launch_gdn2_fwd(a, static_cast<cudaStream_t>(stream)), "gdn2 forward launch");
+}
+
+int kron_delta_gdn2_bwd(const void* q, const void* k, const void* v, const float* b, const float* w,
+                        const float* loga, const float* S0, const void* dO, const float* dST, void* dq, void* dk,
+                        void* dv, float* db, float* dw, float* dloga, float* dS0, int B, int H, int T, int dk_,
+                        int dv_, int dtype, const void* fwd_ws, size_t fwd_ws_bytes, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  kd::GdnLayout L;
+  KD_TRY(gdn_plan(B, H, T, dk_, dv_, dtype, &L));
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(b, "b", true));
+  KD_TRY(check_ptr(w, "w", true));
+  KD_TRY(check_ptr(loga, "loga", true));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(dO, "dO", true));
+  KD_TRY(check_ptr(dST, "dST", false));
+  KD_TRY(check_ptr(dq, "dq", true));
+  KD_TRY(check_ptr(dk, "dk", true));
+  KD_TRY(check_ptr(dv, "dv", true));
+  KD_TRY(check_ptr(db, "db", true));
+  KD_TRY(check_ptr(dw, "dw", true));
+  KD_TRY(check_ptr(dloga, "dloga", true));
+  KD_TRY(check_ptr(dS0, "dS0", false));
+  if (!fwd_ws || fwd_ws_bytes < L.fwd_bytes)
+    return fail(KD_ERR_WORKSPACE, "forward workspace of %zu bytes needed (got %zu)", L.fwd_bytes,
+                fwd_ws ? fwd_ws_bytes : 0);
+  if (!workspace || ws_bytes < L.bwd_bytes)
+    return fail(KD_ERR_WORKSPACE, "backward workspace of %zu bytes needed (got %zu)", L.bwd_bytes,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256) || !aligned(fwd_ws, 256))
+    return fail(KD_ERR_WORKSPACE, "workspaces must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  (void)S0;  // the chunk-start states are read from fwd_ws
+  kd::GdnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.loga = loga; a.S0 = S0;
+  a.dO = dO; a.dST = dST; a.dq = dq; a.dk = dk; a.dv = dv; a.db = db; a.dw = dw; a.dloga = dloga; a.dS0 = dS0;
+  a.fws = static_cast<const char*>(fwd_ws);
+  a.ws = static_cast<char*>(workspace);
+  a.L = L;
+  return launched(kd::launch_gdn2_bwd(a, static_cast<cudaStream_t>(stream)), "gdn2 backward launch");
 }
 
 void kron_delta_profile_enable(int on) {

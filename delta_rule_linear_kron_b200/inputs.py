@@ -23,6 +23,12 @@ Recipe (shapes and distributions of the five workloads):
     c-pre ~ N(0,1) (fp32); f-pre ~ N(3,1) (storage dtype); a_log ~ U(-1,1)
     (fp32); upstream gradients N(0,1) (dq, dk, dv in the storage dtype, the
     gate gradients fp32).
+  * Gated DeltaNet-2 inputs (``make_gdn2_inputs``), in the order q, k, v, b,
+    w, a_h, decay pre-activation, S0, dO: q, k, v as above; erase and write
+    gates b = sigmoid(N(0,1)) per key channel, w = sigmoid(N(0,1)) per value
+    channel (fp32); loga = -a_h * softplus(x), x ~ N(-4,1), a_h = exp(U(-1,1))
+    per head (the article's g = -exp(a) * softplus(.) form, fp32); S0 zero or
+    N(0,1) scaled to Frobenius norm 1; dO ~ N(0,1).
   * epilogue inputs (``make_epilogue_inputs``), in the order o, g, w, dy:
     o ~ N(0, 0.1^2) (a read-out's scale), g ~ N(0,1), dy ~ N(0,1) (storage
     dtype); w ~ 1 + N(0, 0.1^2) (fp32).
@@ -36,7 +42,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs", "make_prologue_inputs",
-           "make_epilogue_inputs",
+           "make_epilogue_inputs", "make_gdn2_inputs",
            "round_to_dtype", "decode_token_inputs_torch"]
 
 
@@ -148,6 +154,26 @@ def make_prologue_inputs(B, H, T, dk, dv, dtype="bf16", seed=2000, with_grads=Tr
                    dc=round_to_dtype(rng.standard_normal((B, T, H)), "f32"),
                    dlogf=round_to_dtype(rng.standard_normal((B, T, H, dk)), "f32"))
     return out
+
+
+def make_gdn2_inputs(B, H, T, dk, dv, dtype="bf16", seed=4000, s0="fro"):
+    """Gated DeltaNet-2 inputs as float64 arrays holding the values the GPU
+    receives: q, k, b, loga [B,T,H,dk]; v, w, dO [B,T,H,dv]; S0 [B,H,dv,dk] or None."""
+    rng = np.random.default_rng(seed)
+    q = round_to_dtype(_l2n(rng.standard_normal((B, T, H, dk))), dtype)
+    k = round_to_dtype(_l2n(rng.standard_normal((B, T, H, dk))), dtype)
+    v = round_to_dtype(_l2n(rng.standard_normal((B, T, H, dv))), dtype)
+    b = round_to_dtype(_sigmoid(rng.standard_normal((B, T, H, dk))), "f32")
+    w = round_to_dtype(_sigmoid(rng.standard_normal((B, T, H, dv))), "f32")
+    a_h = np.exp(rng.uniform(-1.0, 1.0, size=(H,)))
+    x = rng.normal(-4.0, 1.0, size=(B, T, H, dk))
+    loga = round_to_dtype(-a_h[None, None, :, None] * (np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))), "f32")
+    S0 = None
+    if s0 == "fro":
+        S0 = rng.standard_normal((B, H, dv, dk))
+        S0 = round_to_dtype(S0 / np.sqrt(np.sum(S0 * S0, axis=(-2, -1), keepdims=True)), "f32")
+    dO = round_to_dtype(rng.standard_normal((B, T, H, dv)), dtype)
+    return dict(q=q, k=k, v=v, b=b, w=w, loga=loga, S0=S0, dO=dO)
 
 
 def make_epilogue_inputs(B, H, T, dv, dtype="bf16", seed=3000):

@@ -82,6 +82,8 @@ extern "C" {
                                  must be valid but do not change the size) */
 #define KD_WS_EPILOGUE_BWD 4  /* scratch of kron_delta_epilogue_bwd (dk and dtype
                                  must be valid but do not change the size) */
+#define KD_WS_GDN2_FWD 5      /* kron_delta_gdn2_fwd (kept for kron_delta_gdn2_bwd) */
+#define KD_WS_GDN2_BWD 6      /* backward scratch of kron_delta_gdn2_bwd */
 
 /* phases of kron_delta_fwd_phase / kron_delta_bwd_phase */
 #define KD_PHASE_LOCAL 1   /* the work that does not depend on the carried state */
@@ -298,6 +300,47 @@ KD_API int kron_delta_epilogue_fwd(const void *o, const void *g, const float *w,
 KD_API int kron_delta_epilogue_bwd(const void *o, const void *g, const float *w, const void *dy,
                                    void *dO, void *dg, float *dw, int B, int H, int T, int dv,
                                    int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Gated DeltaNet-2 rule on the same chunk machinery (C = 64).  Gated
+ * DeltaNet-2 article (aitrends.kr), sections "핵심 기여" and "방법론": the erase
+ * gate b (per key channel) and the write gate w (per value channel) are
+ * decoupled.  In this library's state convention (S in R^{dv x dk}, the
+ * transpose of the article's), per token t:
+ *     Sbar = S diag(exp(loga_t)),   u = w_t o v_t - Sbar (b_t o k_t),
+ *     S = Sbar + u k_t^T,           o_t = S q_t
+ * With b = w = beta 1 it is the gated delta rule (KDA); with a scalar decay,
+ * Gated DeltaNet (same article, "핵심 기여").
+ *   q, k : [B,T,H,dk] (dtype);  v : [B,T,H,dv] (dtype).
+ *   b : erase gate [B,T,H,dk] fp32;  w : write gate [B,T,H,dv] fp32.
+ *   loga : log of the channel decay [B,T,H,dk] fp32 (<= 0).
+ *   S0 : [B,H,dv,dk] fp32 or NULL (zero);  out : [B,T,H,dv] (dtype);
+ *   ST : [B,H,dv,dk] fp32 or NULL.
+ *   workspace : at least kron_delta_workspace_size(KD_WS_GDN2_FWD, ...) bytes,
+ *   256-byte aligned; it keeps what kron_delta_gdn2_bwd reads.
+ * Computed on CUDA cores in fp32 (no tensor-core path yet).  Errors as for
+ * kron_delta_fwd.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_gdn2_fwd(const void *q, const void *k, const void *v, const float *b,
+                               const float *w, const float *loga, const float *S0, void *out,
+                               float *ST, int B, int H, int T, int dk, int dv, int dtype,
+                               void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Backward of kron_delta_gdn2_fwd for the loss <dO, out> + <dST, ST>.
+ *   fwd_ws : the workspace of a kron_delta_gdn2_fwd call on exactly these
+ *   inputs (read only).  dO [B,T,H,dv] (dtype); dST [B,H,dv,dk] fp32 or NULL.
+ *   dq, dk [B,T,H,dk] and dv [B,T,H,dv] (dtype); db, dloga [B,T,H,dk] and
+ *   dw [B,T,H,dv] fp32; dS0 [B,H,dv,dk] fp32 or NULL.
+ *   workspace : at least kron_delta_workspace_size(KD_WS_GDN2_BWD, ...).
+ * Errors as for kron_delta_bwd.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_gdn2_bwd(const void *q, const void *k, const void *v, const float *b,
+                               const float *w, const float *loga, const float *S0, const void *dO,
+                               const float *dST, void *dq, void *dk, void *dv, float *db,
+                               float *dw, float *dloga, float *dS0, int B, int H, int T, int dk_,
+                               int dv_, int dtype, const void *fwd_ws, size_t fwd_ws_bytes,
+                               void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Synchronises `stream` and reports device-side failures of earlier calls:
