@@ -8,7 +8,8 @@ fp32 gates and state, beta in (0,2), nonzero S0.  The decode step
 (B=256, H=16, d=128, 1000 consecutive in-place steps) is timed in the same run
 and reported under "decode"; the input prologue (raw projections -> normalised
 q, k, v and gates), the output epilogue (RMSNorm and output gate) and their
-backward passes, on the step's shape, under "prologue_epilogue".
+backward passes, on the step's shape, under "prologue_epilogue"; the Gated
+DeltaNet-2 rule's forward + backward on the same shape under "gdn2".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -286,6 +287,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
+    ap.add_argument("--no-gdn2", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -447,6 +449,54 @@ def main(argv=None):
         prologue = dict(times, note="timed alone, not part of the step; each bwd time includes its small "
                                     "fixed-order reduction launch (da_log, dw)")
         del pr, up, ep
+    # ---- Gated DeltaNet-2 rule on the same shape: fwd + bwd, timed on its own
+    gdn2 = None
+    if not args.no_gdn2:
+        g_ = torch.Generator(device=dev)
+        g_.manual_seed(rank_seed(4004, rank))
+
+        def unit_(*sh):
+            x = torch.randn(sh, generator=g_, device=dev)
+            return (x / x.norm(dim=-1, keepdim=True)).to(bf)
+        gi = dict(q=unit_(B, T, H, dk), k=unit_(B, T, H, dk), v=unit_(B, T, H, dv),
+                  b=torch.sigmoid(torch.randn((B, T, H, dk), generator=g_, device=dev)),
+                  w=torch.sigmoid(torch.randn((B, T, H, dv), generator=g_, device=dev)),
+                  loga=-torch.nn.functional.softplus(torch.randn((B, T, H, dk), generator=g_, device=dev) - 4.0))
+        gdO = torch.randn((B, T, H, dv), generator=g_, device=dev).to(bf)
+        gS0 = torch.randn((B, H, dv, dk), generator=g_, device=dev)
+        gS0 = gS0 / gS0.norm(dim=(-2, -1), keepdim=True)
+        gfws = torch.empty(kd.workspace_size(kd.KD_WS_GDN2_FWD, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+        gbws = torch.empty(kd.workspace_size(kd.KD_WS_GDN2_BWD, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+        gorder = ("q", "k", "v", "b", "w", "loga")
+
+        def gstep():
+            kd.gdn2_fwd(*(gi[n] for n in gorder), gS0, workspace=gfws)
+            kd.gdn2_bwd(*(gi[n] for n in gorder), gS0, gdO, fwd_workspace=gfws, workspace=gbws)
+        gsteps = max(1, min(args.steps, 5))
+        for _ in range(3):
+            gstep()
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(gsteps):
+            gstep()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        gms = max_over_ranks(g0.elapsed_time(g1), ws_n, dev) / gsteps
+        kd.lib().kron_delta_profile_enable(1)
+        kd.lib().kron_delta_profile_report(None, 0, 1)
+        gstep()
+        torch.cuda.synchronize()
+        gbuf = ctypes.create_string_buffer(1 << 14)
+        kd.lib().kron_delta_profile_report(gbuf, len(gbuf), 1)
+        kd.lib().kron_delta_profile_enable(0)
+        gk = {ln.split()[0]: float(ln.split()[2]) for ln in gbuf.value.decode().splitlines()}
+        kd.device_status()
+        gdn2 = dict(value=job_throughput(ws_n, B * T, 1, gms), unit="tokens/s", ms_per_step=gms,
+                    step="gdn2_fwd + gdn2_bwd (bf16 q/k/v/dO, fp32 gates, CUDA cores)", per_kernel_ms=gk)
+        del gi, gdO, gfws, gbws
     clocks = sampler.stop()
 
     # ---- end to end through the public API with pinned host buffers -----
@@ -526,7 +576,7 @@ def main(argv=None):
                            "global_batch": B * ws_n, "seq_len": T, "parallelism": f"dp{ws_n}",
                            "step": "fwd(save) + bwd", "l2": "inputs larger than L2 (no flush)"},
                 "tc_frac_of_bf16_peak": tc_frac,
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "prologue_epilogue": prologue,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "prologue_epilogue": prologue, "gdn2": gdn2,
                 "gpu_launches": launches, "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
                 "kernel_rooflines": kernels,
                 "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
