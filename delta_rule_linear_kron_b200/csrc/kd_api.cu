@@ -132,6 +132,8 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
   L->dE = take(chunks * C * dk);
   L->dT = take(chunks * C * C);
   L->dP = take(chunks * C * C);
+  L->dQp = take(chunks * C * dk);
+  L->dKe = take(chunks * C * dk);
   L->bwd_bytes = off;
   return KD_OK;
 }

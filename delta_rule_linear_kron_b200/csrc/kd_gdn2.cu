@@ -29,8 +29,10 @@
 //   and through the gates and exact weights to dq, dk, db, dv, dw, dloga.
 //
 // Kernels: gdn2_prep (A, P, W, U', Q+, K^e, e^Lambda per chunk), gdn2_chain,
-// gdn2_out; gdn2_bchain, gdn2_bpost_a (dP, dZ -> dv, dw, dE, dT),
-// gdn2_bpost_b (dq, dk, db, dloga).
+// gdn2_out; gdn2_bchain, gdn2_bpost_a (dP, dQ+, dK^e, dZ -> dv, dw, dE, dT),
+// gdn2_bpost_b (dq, dk, db, dloga; chunks inside the safe decay range, by
+// factorised products) and gdn2_bpost_exact (the other chunks, per-element
+// weights).
 #include "kd_common.cuh"
 #include "kd_kernels.h"
 
@@ -39,7 +41,13 @@ namespace kd {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int kRows = 8;  // value rows of the state per chain CTA
+// Value rows of the state per chain CTA: d_v / 16 CTAs per head, so the
+// chains of 16 heads at d_v = 128 fit in one wave on 148 SMs.
+constexpr int kRows = 16;
+constexpr int kChainThreads = 512;  // threads of a chain CTA
+// In-chunk |L| below which the backward factors e^{L_t - L_i} = gamma_t / gamma_i
+// (e^{+-60} and their products stay well inside fp32's normal range).
+constexpr float kGdnSafeLog = 60.f;
 
 template <int DK, int DV>
 struct GP {
@@ -48,6 +56,54 @@ struct GP {
 
 __device__ __forceinline__ size_t row_bthd(int b, int T, int t, int H, int h, int D) {
   return (((size_t)b * T + t) * H + h) * D;
+}
+
+// A [N / D][D] fp32 tile held as float4s across the 256 threads of a CTA, so
+// that all of a thread's loads are in flight before any is used.  N is a
+// multiple of 1024 and D of 4; the source is 16-byte aligned.
+template <int N, int NT = 256>
+struct Frag {
+  static constexpr int V = N / (4 * NT);
+  static_assert(V >= 1 && V * 4 * NT == N, "tile size must be a multiple of 4 x threads");
+  float4 x[V];
+};
+
+template <int N, int NT>
+__device__ __forceinline__ void frag_load(Frag<N, NT>& f, const float* __restrict__ src) {
+#pragma unroll
+  for (int i = 0; i < Frag<N, NT>::V; ++i) f.x[i] = __ldg(reinterpret_cast<const float4*>(src) + threadIdx.x + NT * i);
+}
+
+// Stores the tile into shared memory rows of pitch P.
+template <int N, int D, int P, int NT>
+__device__ __forceinline__ void frag_store(float* dst, const Frag<N, NT>& f) {
+#pragma unroll
+  for (int i = 0; i < Frag<N, NT>::V; ++i) {
+    const int e = 4 * (threadIdx.x + NT * i), t = e / D, j = e % D;
+    float* d = dst + t * P + j;
+    d[0] = f.x[i].x;
+    d[1] = f.x[i].y;
+    d[2] = f.x[i].z;
+    d[3] = f.x[i].w;
+  }
+}
+
+// acc[u][v] += sum over k in [k0, k1) of A[u * ar + k * ak] * B[k * bk + v * bc]
+// (a 4 x 4 output tile per thread; A and B already point at the tile's first
+// row and column, in shared memory).
+__device__ __forceinline__ void mm4x4(float (&acc)[4][4], const float* A, int ar, int ak, const float* B, int bk,
+                                      int bc, int k0, int k1) {
+  for (int k = k0; k < k1; ++k) {
+    float a[4], b[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = A[u * ar + k * ak];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) b[v] = B[k * bk + v * bc];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+  }
 }
 
 }  // namespace
@@ -91,28 +147,59 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
     }
   }
   __syncthreads();
-  // T and P with per-element decay weights e^{L_t - L_i} <= 1
-  for (int e = tid; e < C * C; e += 256) {
-    const int t = e / C, i = e % C;
-    float sT = 0.f, sP = 0.f;
-    if (i <= t) {
-      for (int j = 0; j < DK; ++j) {
-        const float kw = Ks[i * G::PK + j] * expf(Ls[t * G::PK + j] - Ls[i * G::PK + j]);
-        sT = fmaf(Es[t * G::PK + j], kw, sT);
-        sP = fmaf(Qs[t * G::PZ + j], kw, sP);
-      }
-    }
-    Ts[t * G::PC + i] = i < t ? sT : 0.f;
-    p.P[ch * C * C + e] = i <= t ? sP : 0.f;
-  }
-  __syncthreads();
   const float* Llast = Ls + (C - 1) * G::PK;  // padded rows carry loga = 0: L at row C-1 is Lambda
-  for (int e = tid; e < C * DK; e += 256) {
-    const int t = e / DK, j = e % DK;
-    const float L = Ls[t * G::PK + j], gm = expf(L);
-    p.Qp[ch * C * DK + e] = Qs[t * G::PZ + j] * gm;
-    p.Ke[ch * C * DK + e] = Ks[t * G::PK + j] * expf(Llast[j] - L);
-    Es[t * G::PK + j] *= gm;
+  float mx = 0.f;
+  if (tid < DK) mx = fabsf(Llast[tid]);     // |L| is largest at the chunk end (L is monotone)
+  if (__syncthreads_or(!(mx < kGdnSafeLog))) {
+    // T and P with per-element decay weights e^{L_t - L_i} <= 1
+    for (int e = tid; e < C * C; e += 256) {
+      const int t = e / C, i = e % C;
+      float sT = 0.f, sP = 0.f;
+      if (i <= t) {
+        for (int j = 0; j < DK; ++j) {
+          const float kw = Ks[i * G::PK + j] * expf(Ls[t * G::PK + j] - Ls[i * G::PK + j]);
+          sT = fmaf(Es[t * G::PK + j], kw, sT);
+          sP = fmaf(Qs[t * G::PZ + j], kw, sP);
+        }
+      }
+      Ts[t * G::PC + i] = i < t ? sT : 0.f;
+      p.P[ch * C * C + e] = i <= t ? sP : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * DK; e += 256) {
+      const int t = e / DK, j = e % DK;
+      const float L = Ls[t * G::PK + j], gm = expf(L);
+      p.Qp[ch * C * DK + e] = Qs[t * G::PZ + j] * gm;
+      p.Ke[ch * C * DK + e] = Ks[t * G::PK + j] * expf(Llast[j] - L);
+      Es[t * G::PK + j] *= gm;
+    }
+  } else {
+    // inside the safe range the weights factor: T = tril(E+ K-^T, -1), P = tril(Q+ K-^T)
+    for (int e = tid; e < C * DK; e += 256) {
+      const int t = e / DK, j = e % DK;
+      const float L = Ls[t * G::PK + j], gm = expf(L);
+      const float qp = Qs[t * G::PZ + j] * gm, kk = Ks[t * G::PK + j];
+      p.Qp[ch * C * DK + e] = qp;
+      p.Ke[ch * C * DK + e] = kk * expf(Llast[j] - L);
+      Qs[t * G::PZ + j] = qp;
+      Ks[t * G::PK + j] = kk * expf(-L);
+      Es[t * G::PK + j] *= gm;
+    }
+    __syncthreads();
+    const int ti = (tid >> 4) * 4, ii = (tid & 15) * 4;  // a 4 x 4 tile of T and P per thread
+    float aT[4][4] = {}, aP[4][4] = {};
+    if (ii <= ti + 3) {
+      mm4x4(aT, Es + ti * G::PK, G::PK, 1, Ks + ii * G::PK, 1, G::PK, 0, DK);
+      mm4x4(aP, Qs + ti * G::PZ, G::PZ, 1, Ks + ii * G::PK, 1, G::PK, 0, DK);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int t = ti + u, i = ii + v;
+        Ts[t * G::PC + i] = i < t ? aT[u][v] : 0.f;
+        p.P[ch * C * C + t * C + i] = i <= t ? aP[u][v] : 0.f;
+      }
   }
   if (tid < DK) p.gC[ch * DK + tid] = expf(Llast[tid]);
   __syncthreads();
@@ -147,10 +234,10 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
 // ---------------------------------------------------------------------------
 // The chain: one CTA per (kRows value rows, head); chunks in order.
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) gdn2_chain(const float* __restrict__ S0, float* __restrict__ ST, int H,
+__global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restrict__ S0, float* __restrict__ ST, int H,
                                                   int NC, GdnWs p) {
   using G = GP<DK, DV>;
-  constexpr int RS = kRows, PR = RS + 1;
+  constexpr int RS = kRows, PR = RS + 1, NT = kChainThreads;
   extern __shared__ float gsm[];
   float* Ws = gsm;                  // [C][PK]
   float* Kes = Ws + C * G::PK;      // [C][PK]
@@ -160,28 +247,43 @@ __global__ void __launch_bounds__(256) gdn2_chain(const float* __restrict__ S0, 
   const int tid = threadIdx.x;
   const int r0 = blockIdx.x * RS, h = blockIdx.y, bb = blockIdx.z;
   const size_t unit = (size_t)bb * H + h;
-  for (int e = tid; e < RS * DK; e += 256) {
+  for (int e = tid; e < RS * DK; e += NT) {
     const int r = e / DK, j = e % DK;
     Ss[r * G::PK + j] = S0 ? S0[(unit * DV + r0 + r) * DK + j] : 0.f;
   }
+  // chunk n+1's W and K^e are loaded into registers while chunk n computes
+  constexpr int UPT = C * RS / NT;  // U' values per thread
+  Frag<C * DK, NT> fw, fk;
+  float up[UPT], gc = 0.f;
+  auto fetch = [&](int n) {
+    const size_t ch = unit * NC + n;
+    frag_load(fw, p.W + ch * C * DK);
+    frag_load(fk, p.Ke + ch * C * DK);
+#pragma unroll
+    for (int i = 0; i < UPT; ++i) {
+      const int e = tid + NT * i;
+      up[i] = p.Up[ch * C * DV + (e / RS) * DV + r0 + e % RS];
+    }
+    if (tid < DK) gc = p.gC[ch * DK + tid];
+  };
+  fetch(0);
   for (int n = 0; n < NC; ++n) {
     const size_t ch = unit * NC + n;
-    for (int e = tid; e < C * DK; e += 256) {
-      const int t = e / DK, j = e % DK;
-      Ws[t * G::PK + j] = p.W[ch * C * DK + e];
-      Kes[t * G::PK + j] = p.Ke[ch * C * DK + e];
+    frag_store<C * DK, DK, G::PK>(Ws, fw);
+    frag_store<C * DK, DK, G::PK>(Kes, fk);
+#pragma unroll
+    for (int i = 0; i < UPT; ++i) {
+      const int e = tid + NT * i;
+      Us[(e / RS) * PR + e % RS] = up[i];
     }
-    for (int e = tid; e < C * RS; e += 256) {
-      const int t = e / RS, r = e % RS;
-      Us[t * PR + r] = p.Up[ch * C * DV + t * DV + r0 + r];
-    }
-    if (tid < DK) gcs[tid] = p.gC[ch * DK + tid];
+    if (tid < DK) gcs[tid] = gc;
     __syncthreads();
-    for (int e = tid; e < RS * DK; e += 256) {
+    if (n + 1 < NC) fetch(n + 1);
+    for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       p.S0[ch * DV * DK + (size_t)(r0 + r) * DK + j] = Ss[r * G::PK + j];
     }
-    for (int e = tid; e < C * RS; e += 256) {
+    for (int e = tid; e < C * RS; e += NT) {
       const int t = e / RS, r = e % RS;
       float s = Us[t * PR + r];
       for (int j = 0; j < DK; ++j) s = fmaf(-Ws[t * G::PK + j], Ss[r * G::PK + j], s);
@@ -189,7 +291,7 @@ __global__ void __launch_bounds__(256) gdn2_chain(const float* __restrict__ S0, 
       p.U[ch * C * DV + t * DV + r0 + r] = s;
     }
     __syncthreads();
-    for (int e = tid; e < RS * DK; e += 256) {
+    for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       float s = Ss[r * G::PK + j] * gcs[j];
       for (int t = 0; t < C; ++t) s = fmaf(Us[t * PR + r], Kes[t * G::PK + j], s);
@@ -198,7 +300,7 @@ __global__ void __launch_bounds__(256) gdn2_chain(const float* __restrict__ S0, 
     __syncthreads();
   }
   if (ST)
-    for (int e = tid; e < RS * DK; e += 256) {
+    for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       ST[(unit * DV + r0 + r) * DK + j] = Ss[r * G::PK + j];
     }
@@ -218,10 +320,22 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
-  for (int e = tid; e < C * DK; e += 256) Qps[(e / DK) * G::PK + e % DK] = p.Qp[ch * C * DK + e];
-  for (int e = tid; e < DV * DK; e += 256) S0s[(e / DK) * G::PK + e % DK] = p.S0[ch * DV * DK + e];
-  for (int e = tid; e < C * C; e += 256) Ps[(e / C) * G::PC + e % C] = p.P[ch * C * C + e];
-  for (int e = tid; e < C * DV; e += 256) Uss[(e / DV) * G::PV + e % DV] = p.U[ch * C * DV + e];
+  {
+    Frag<DV * DK> fs;
+    frag_load(fs, p.S0 + ch * DV * DK);
+    frag_store<DV * DK, DK, G::PK>(S0s, fs);
+  }
+  {
+    Frag<C * DK> fq;
+    Frag<C * C> fp;
+    Frag<C * DV> fu;
+    frag_load(fq, p.Qp + ch * C * DK);
+    frag_load(fp, p.P + ch * C * C);
+    frag_load(fu, p.U + ch * C * DV);
+    frag_store<C * DK, DK, G::PK>(Qps, fq);
+    frag_store<C * C, C, G::PC>(Ps, fp);
+    frag_store<C * DV, DV, G::PV>(Uss, fu);
+  }
   __syncthreads();
   for (int e = tid; e < C * DV; e += 256) {
     const int t = e / DV, r = e % DV;
@@ -236,10 +350,10 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
 // ---------------------------------------------------------------------------
 // Reverse chain: one CTA per (kRows value rows, head); chunks last to first.
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) gdn2_bchain(const Tin* __restrict__ dO, const float* __restrict__ dST,
+__global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restrict__ dO, const float* __restrict__ dST,
                                                    float* __restrict__ dS0, int H, int T, int NC, GdnWs p) {
   using G = GP<DK, DV>;
-  constexpr int RS = kRows, PR = RS + 1;
+  constexpr int RS = kRows, PR = RS + 1, NT = kChainThreads;
   extern __shared__ float gsm[];
   float* Ps = gsm;                  // [C][PC]
   float* Kes = Ps + C * G::PC;      // [C][PK]
@@ -252,31 +366,36 @@ __global__ void __launch_bounds__(256) gdn2_bchain(const Tin* __restrict__ dO, c
   const int tid = threadIdx.x;
   const int r0 = blockIdx.x * RS, h = blockIdx.y, bb = blockIdx.z;
   const size_t unit = (size_t)bb * H + h;
-  for (int e = tid; e < RS * DK; e += 256) {
+  for (int e = tid; e < RS * DK; e += NT) {
     const int r = e / DK, j = e % DK;
     dSs[r * G::PK + j] = dST ? dST[(unit * DV + r0 + r) * DK + j] : 0.f;
   }
   for (int n = NC - 1; n >= 0; --n) {
     const size_t ch = unit * NC + n;
     const int t0 = n * C, nv = min(C, T - t0);
-    for (int e = tid; e < C * C; e += 256) Ps[(e / C) * G::PC + e % C] = p.P[ch * C * C + e];
-    for (int e = tid; e < C * DK; e += 256) {
-      const int t = e / DK, j = e % DK;
-      Kes[t * G::PK + j] = p.Ke[ch * C * DK + e];
-      Qps[t * G::PK + j] = p.Qp[ch * C * DK + e];
-      Ws[t * G::PK + j] = p.W[ch * C * DK + e];
+    {
+      Frag<C * C, NT> fp;
+      Frag<C * DK, NT> fk, fq, fw;
+      frag_load(fp, p.P + ch * C * C);
+      frag_load(fk, p.Ke + ch * C * DK);
+      frag_load(fq, p.Qp + ch * C * DK);
+      frag_load(fw, p.W + ch * C * DK);
+      frag_store<C * C, C, G::PC>(Ps, fp);
+      frag_store<C * DK, DK, G::PK>(Kes, fk);
+      frag_store<C * DK, DK, G::PK>(Qps, fq);
+      frag_store<C * DK, DK, G::PK>(Ws, fw);
     }
-    for (int e = tid; e < C * RS; e += 256) {
+    for (int e = tid; e < C * RS; e += NT) {
       const int t = e / RS, r = e % RS;
       dOs[t * PR + r] = t < nv ? to_f(dO[row_bthd(bb, T, t0 + t, H, h, DV) + r0 + r]) : 0.f;
     }
     if (tid < DK) gcs[tid] = p.gC[ch * DK + tid];
     __syncthreads();
-    for (int e = tid; e < RS * DK; e += 256) {
+    for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       p.dS[ch * DV * DK + (size_t)(r0 + r) * DK + j] = dSs[r * G::PK + j];
     }
-    for (int e = tid; e < C * RS; e += 256) {
+    for (int e = tid; e < C * RS; e += NT) {
       const int t = e / RS, r = e % RS;
       float s = 0.f;
       for (int tp = t; tp < C; ++tp) s = fmaf(Ps[tp * G::PC + t], dOs[tp * PR + r], s);
@@ -285,7 +404,7 @@ __global__ void __launch_bounds__(256) gdn2_bchain(const Tin* __restrict__ dO, c
       p.dU[ch * C * DV + t * DV + r0 + r] = s;
     }
     __syncthreads();
-    for (int e = tid; e < RS * DK; e += 256) {
+    for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       float s = dSs[r * G::PK + j] * gcs[j];
       for (int t = 0; t < C; ++t)
@@ -295,7 +414,7 @@ __global__ void __launch_bounds__(256) gdn2_bchain(const Tin* __restrict__ dO, c
     __syncthreads();
   }
   if (dS0)
-    for (int e = tid; e < RS * DK; e += 256) {
+    for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       dS0[(unit * DV + r0 + r) * DK + j] = dSs[r * G::PK + j];
     }
@@ -328,55 +447,97 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
   }
   for (int e = tid; e < C * C; e += 256) As[(e / C) * G::PC + e % C] = p.A[ch * C * C + e];
   __syncthreads();
-  // dP = tril(dO U^T)
-  for (int e = tid; e < C * C; e += 256) {
-    const int t = e / C, i = e % C;
-    float s = 0.f;
-    if (i <= t)
-      for (int r = 0; r < DV; ++r) s = fmaf(R1[t * G::PZ + r], R2[i * G::PZ + r], s);
-    dPs[t * G::PC + i] = s;
-  }
-  __syncthreads();
-  // dZ = A^T dU (A lower triangular) -> dv = dZ w, dw = dZ v;  dW = -dU S0
-  for (int e = tid; e < C * DV; e += 256) {
-    const int t = e / DV, r = e % DV;
-    float s = 0.f;
-    for (int i = t; i < C; ++i) s = fmaf(As[i * G::PC + t], R3[i * G::PZ + r], s);
-    R2[t * G::PZ + r] = s;
-    if (t < nv) {
-      const size_t g = row_bthd(bb, T, t0 + t, H, h, DV) + r;
-      dv[g] = from_f<Tin>(s * wg[g]);
-      dw[g] = s * to_f(v[g]);
+  // dQ+ = dO S0, dK^e = U dS (to the workspace) and dW = -dU S0: each thread an
+  // 8-position x 4-channel tile, the state rows streamed as float4
+  {
+    constexpr int NJG = DK / 4;
+    if (tid < NJG * 8) {
+      const int jg = tid % NJG, t8 = (tid / NJG) * 8;
+      float aq[8][4] = {}, ak[8][4] = {}, aw[8][4] = {};
+      const float4* s0 = reinterpret_cast<const float4*>(p.S0 + ch * DV * DK) + jg;
+      const float4* ds = reinterpret_cast<const float4*>(p.dS + ch * DV * DK) + jg;
+      for (int r = 0; r < DV; ++r) {
+        const float4 a = __ldg(s0 + r * NJG), d = __ldg(ds + r * NJG);
+        const float av[4] = {a.x, a.y, a.z, a.w}, dv4[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float o = R1[(t8 + u) * G::PZ + r], uu = R2[(t8 + u) * G::PZ + r], du = R3[(t8 + u) * G::PZ + r];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            aq[u][c] = fmaf(o, av[c], aq[u][c]);
+            ak[u][c] = fmaf(uu, dv4[c], ak[u][c]);
+            aw[u][c] = fmaf(du, av[c], aw[u][c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = t8 + u;
+        *reinterpret_cast<float4*>(p.dQp + ch * C * DK + t * DK + 4 * jg) =
+            make_float4(aq[u][0], aq[u][1], aq[u][2], aq[u][3]);
+        *reinterpret_cast<float4*>(p.dKe + ch * C * DK + t * DK + 4 * jg) =
+            make_float4(ak[u][0], ak[u][1], ak[u][2], ak[u][3]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) R4[t * G::PK + 4 * jg + c] = -aw[u][c];
+      }
     }
   }
-  for (int e = tid; e < C * DK; e += 256) {
-    const int t = e / DK, j = e % DK;
-    float s = 0.f;
-    for (int r = 0; r < DV; ++r) s = fmaf(R3[t * G::PZ + r], p.S0[ch * DV * DK + (size_t)r * DK + j], s);
-    R4[t * G::PK + j] = -s;
+  const int ti = (tid >> 4) * 4, ii = (tid & 15) * 4;  // this thread's 4 x 4 tile of a C x C result
+  // dP = tril(dO U^T)
+  {
+    float acc[4][4] = {};
+    if (ii <= ti + 3) mm4x4(acc, R1 + ti * G::PZ, G::PZ, 1, R2 + ii * G::PZ, 1, G::PZ, 0, DV);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dPs[(ti + u) * G::PC + ii + v] = ii + v <= ti + u ? acc[u][v] : 0.f;
   }
   __syncthreads();
-  // dE = A^T dW
-  for (int e = tid; e < C * DK; e += 256) {
-    const int t = e / DK, j = e % DK;
-    float s = 0.f;
-    for (int i = t; i < C; ++i) s = fmaf(As[i * G::PC + t], R4[i * G::PK + j], s);
-    R1[t * G::PZ + j] = s;
-    p.dE[ch * C * DK + e] = s;
+  // dZ = A^T dU (A lower triangular) -> dv = dZ w, dw = dZ v;  dE = A^T dW
+  for (int tile = tid; tile < 16 * (DV / 4); tile += 256) {
+    const int t4 = (tile / (DV / 4)) * 4, r4 = (tile % (DV / 4)) * 4;
+    float acc[4][4] = {};
+    mm4x4(acc, As + t4, 1, G::PC, R3 + r4, G::PZ, 1, t4, C);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int t = t4 + u, r = r4 + c;
+        R2[t * G::PZ + r] = acc[u][c];
+        if (t < nv) {
+          const size_t g = row_bthd(bb, T, t0 + t, H, h, DV) + r;
+          dv[g] = from_f<Tin>(acc[u][c] * wg[g]);
+          dw[g] = acc[u][c] * to_f(v[g]);
+        }
+      }
+  }
+  for (int tile = tid; tile < 16 * (DK / 4); tile += 256) {
+    const int t4 = (tile / (DK / 4)) * 4, j4 = (tile % (DK / 4)) * 4;
+    float acc[4][4] = {};
+    mm4x4(acc, As + t4, 1, G::PC, R4 + j4, G::PK, 1, t4, C);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        R1[(t4 + u) * G::PZ + j4 + c] = acc[u][c];
+        p.dE[ch * C * DK + (t4 + u) * DK + j4 + c] = acc[u][c];
+      }
   }
   __syncthreads();
   for (int e = tid; e < C * DV; e += 256) R3[(e / DV) * G::PZ + e % DV] = p.Up[ch * C * DV + e];
   for (int e = tid; e < C * DK; e += 256) R4[(e / DK) * G::PK + e % DK] = p.W[ch * C * DK + e];
   __syncthreads();
   // dT = -tril(dZ U'^T + dE W^T, -1)
-  for (int e = tid; e < C * C; e += 256) {
-    const int t = e / C, i = e % C;
-    float s = 0.f;
-    if (i < t) {
-      for (int r = 0; r < DV; ++r) s = fmaf(R2[t * G::PZ + r], R3[i * G::PZ + r], s);
-      for (int j = 0; j < DK; ++j) s = fmaf(R1[t * G::PZ + j], R4[i * G::PK + j], s);
+  {
+    float acc[4][4] = {};
+    if (ii <= ti + 3) {
+      mm4x4(acc, R2 + ti * G::PZ, G::PZ, 1, R3 + ii * G::PZ, 1, G::PZ, 0, DV);
+      mm4x4(acc, R1 + ti * G::PZ, G::PZ, 1, R4 + ii * G::PK, 1, G::PK, 0, DK);
     }
-    dTs[t * G::PC + i] = -s;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dTs[(ti + u) * G::PC + ii + v] = ii + v < ti + u ? -acc[u][v] : 0.f;
   }
   __syncthreads();
   for (int e = tid; e < C * C; e += 256) {
@@ -389,7 +550,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
 // Per chunk: dq, dk, db, dloga.  Thread e handles (t, j) with j = e % DK fixed
 // per thread (256 is a multiple of DK).
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(256) gdn2_bpost_exact(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                     const float* __restrict__ bg, const float* __restrict__ loga,
                                                     const Tin* __restrict__ dO, int H, int T, int NC, GdnWs p,
                                                     Tin* __restrict__ dq, Tin* __restrict__ dk,
@@ -409,6 +570,17 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
+  // the decay prefix first: chunks inside the safe range leave at once
+  float mx = 0.f;
+  if (tid < DK) {
+    float acc = 0.f;
+    for (int t = 0; t < C; ++t) {
+      acc += t < nv ? loga[row_bthd(bb, T, t0 + t, H, h, DK) + tid] : 0.f;
+      Ls[t * G::PK + tid] = acc;
+      mx = fmaxf(mx, fabsf(acc));
+    }
+  }
+  if (!__syncthreads_or(!(mx < kGdnSafeLog))) return;  // the factorised kernel took this chunk
   for (int e = tid; e < C * DK; e += 256) {
     const int t = e / DK, j = e % DK;
     const bool ok = t < nv;
@@ -417,19 +589,10 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
     Ks[t * G::PK + j] = kk;
     Qs[t * G::PK + j] = ok ? to_f(q[g]) : 0.f;
     Es[t * G::PK + j] = ok ? bg[g] * kk : 0.f;
-    Ls[t * G::PK + j] = ok ? loga[g] : 0.f;
   }
   for (int e = tid; e < C * C; e += 256) {
     dPs[(e / C) * G::PC + e % C] = p.dP[ch * C * C + e];
     dTs[(e / C) * G::PC + e % C] = p.dT[ch * C * C + e];
-  }
-  __syncthreads();
-  if (tid < DK) {
-    float acc = 0.f;
-    for (int t = 0; t < C; ++t) {
-      acc += Ls[t * G::PK + tid];
-      Ls[t * G::PK + tid] = acc;
-    }
   }
   __syncthreads();
   const int j = tid % DK;
@@ -439,13 +602,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
     const int t = e / DK;
     const float L = Ls[t * G::PK + j], gm = expf(L), ke = expf(Lam - L);
     const float kk = Ks[t * G::PK + j], qq = Qs[t * G::PK + j], ee = Es[t * G::PK + j];
-    float dQp = 0.f, dKe = 0.f;
-    const size_t orow = row_bthd(bb, T, t0 + t, H, h, DV);
-    for (int r = 0; r < DV; ++r) {
-      const float go = t < nv ? to_f(dO[orow + r]) : 0.f;
-      dQp = fmaf(go, p.S0[ch * DV * DK + (size_t)r * DK + j], dQp);
-      dKe = fmaf(p.U[ch * C * DV + t * DV + r], p.dS[ch * DV * DK + (size_t)r * DK + j], dKe);
-    }
+    const float dQp = p.dQp[ch * C * DK + e], dKe = p.dKe[ch * C * DK + e];
     const float dEv = p.dE[ch * C * DK + e];
     float dee = dEv * gm, dqq = dQp * gm, dkk = dKe * ke;
     float dL = dEv * ee * gm + dQp * qq * gm - dKe * kk * ke;
@@ -491,6 +648,155 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
 }
 
 // ---------------------------------------------------------------------------
+// Per chunk, chunks whose in-chunk |L| stays below kGdnSafeLog: the exact
+// weights factor as e^{L_t - L_i} = gamma_t / gamma_i, and the pair sums become
+// three products with K- = k / gamma, E+ = e o gamma, Q+ = q o gamma:
+//   X1 = dT K-,  X2 = dP K-,  Y = dT^T E+ + dP^T Q+                 ([C][DK])
+//   de = gamma (dE + X1),  dq = gamma (dQ+ + X2),  dk = dK^e e^{Lambda-L} + Y / gamma
+//   dL = dE E+ + dQ+ Q+ - dK^e K^e + E+ X1 + Q+ X2 - K- Y
+// Each thread owns an 8-position x 4-channel tile of all three products.
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                    const float* __restrict__ bg, const float* __restrict__ loga,
+                                                    int H, int T, int NC, GdnWs p, Tin* __restrict__ dq,
+                                                    Tin* __restrict__ dk, float* __restrict__ db,
+                                                    float* __restrict__ dloga) {
+  constexpr int P4 = DK + 4, PT = C + 4, NJG = DK / 4;
+  extern __shared__ __align__(16) float gsm[];
+  float* Ls = gsm;                  // [C][P4]  L
+  float* Km = Ls + C * P4;          // [C][P4]  K-
+  float* Ep = Km + C * P4;          // [C][P4]  E+
+  float* Qp = Ep + C * P4;          // [C][P4]  Q+
+  float* dTr = Qp + C * P4;         // [C][PT]  dT, rows t
+  float* dPr = dTr + C * PT;        // [C][PT]  dP, rows t
+  float* dTc = dPr + C * PT;        // [C][PT]  dT^T, then dL
+  float* dPc = dTc + C * PT;        // [C][PT]  dP^T
+  float* red = dPc + C * PT;        // [8][DK]
+  const int tid = threadIdx.x;
+  const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = ((size_t)bb * H + h) * NC + n;
+  for (int e = tid; e < C * DK; e += 256) {
+    const int t = e / DK, j = e % DK;
+    Ls[t * P4 + j] = t < nv ? loga[row_bthd(bb, T, t0 + t, H, h, DK) + j] : 0.f;
+  }
+  for (int e = tid; e < C * C; e += 256) {
+    const int t = e / C, i = e % C;
+    const float a = p.dT[ch * C * C + e], c = p.dP[ch * C * C + e];
+    dTr[t * PT + i] = a;
+    dPr[t * PT + i] = c;
+    dTc[i * PT + t] = a;
+    dPc[i * PT + t] = c;
+  }
+  __syncthreads();
+  float mx = 0.f;
+  if (tid < DK) {
+    float acc = 0.f;
+    for (int t = 0; t < C; ++t) {
+      acc += Ls[t * P4 + tid];
+      Ls[t * P4 + tid] = acc;
+      mx = fmaxf(mx, fabsf(acc));
+    }
+  }
+  if (__syncthreads_or(!(mx < kGdnSafeLog))) return;  // the exact kernel takes this chunk
+  for (int e = tid; e < C * DK; e += 256) {
+    const int t = e / DK, j = e % DK;
+    const bool ok = t < nv;
+    const size_t g = row_bthd(bb, T, t0 + t, H, h, DK) + j;
+    const float L = Ls[t * P4 + j], gm = expf(L), ig = expf(-L);
+    const float kk = ok ? to_f(k[g]) : 0.f;
+    Km[t * P4 + j] = kk * ig;
+    Ep[t * P4 + j] = ok ? bg[g] * kk * gm : 0.f;
+    Qp[t * P4 + j] = p.Qp[ch * C * DK + e];
+  }
+  __syncthreads();
+  const bool act = tid < NJG * 8;
+  const int jg = tid % NJG, t8 = (tid / NJG) * 8;
+  float x1[8][4] = {}, x2[8][4] = {}, y[8][4] = {};
+  if (act) {
+    for (int i = 0; i < C; ++i) {
+      const float4 km = *reinterpret_cast<const float4*>(Km + i * P4 + 4 * jg);
+      const float4 ta = *reinterpret_cast<const float4*>(dTc + i * PT + t8);
+      const float4 tb = *reinterpret_cast<const float4*>(dTc + i * PT + t8 + 4);
+      const float4 pa = *reinterpret_cast<const float4*>(dPc + i * PT + t8);
+      const float4 pb = *reinterpret_cast<const float4*>(dPc + i * PT + t8 + 4);
+      const float kv[4] = {km.x, km.y, km.z, km.w};
+      const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+      const float pv[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          x1[u][c] = fmaf(tv[u], kv[c], x1[u][c]);
+          x2[u][c] = fmaf(pv[u], kv[c], x2[u][c]);
+        }
+    }
+    for (int tp = 0; tp < C; ++tp) {
+      const float4 ea = *reinterpret_cast<const float4*>(Ep + tp * P4 + 4 * jg);
+      const float4 qa = *reinterpret_cast<const float4*>(Qp + tp * P4 + 4 * jg);
+      const float4 ta = *reinterpret_cast<const float4*>(dTr + tp * PT + t8);
+      const float4 tb = *reinterpret_cast<const float4*>(dTr + tp * PT + t8 + 4);
+      const float4 pa = *reinterpret_cast<const float4*>(dPr + tp * PT + t8);
+      const float4 pb = *reinterpret_cast<const float4*>(dPr + tp * PT + t8 + 4);
+      const float ev[4] = {ea.x, ea.y, ea.z, ea.w}, qv[4] = {qa.x, qa.y, qa.z, qa.w};
+      const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+      const float pv[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) y[u][c] = fmaf(tv[u], ev[c], fmaf(pv[u], qv[c], y[u][c]));
+    }
+  }
+  __syncthreads();  // dT^T is dead: dL goes there
+  float* dLs = dTc;   // [C][P4] fits in two [C][PT] regions
+  float lam[4] = {};
+  if (act) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t8 + u;
+      const bool ok = t < nv;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = 4 * jg + c;
+        const size_t e = (size_t)t * DK + j;
+        const float L = Ls[t * P4 + j], gm = expf(L), ke = expf(Ls[(C - 1) * P4 + j] - L);
+        const float dQv = p.dQp[ch * C * DK + e], dKv = p.dKe[ch * C * DK + e], dEv = p.dE[ch * C * DK + e];
+        const float ep = Ep[t * P4 + j], qp = Qp[t * P4 + j], km = Km[t * P4 + j];
+        const size_t g = row_bthd(bb, T, t0 + t, H, h, DK) + j;
+        const float kk = ok ? to_f(k[g]) : 0.f;
+        const float dee = gm * (dEv + x1[u][c]);
+        const float dqq = gm * (dQv + x2[u][c]);
+        const float dkk = fmaf(dKv, ke, y[u][c] * expf(-L));
+        lam[c] = fmaf(dKv, kk * ke, lam[c]);
+        dLs[t * P4 + j] = dEv * ep + dQv * qp - dKv * kk * ke + ep * x1[u][c] + qp * x2[u][c] - km * y[u][c];
+        if (ok) {
+          dq[g] = from_f<Tin>(dqq);
+          dk[g] = from_f<Tin>(fmaf(dee, bg[g], dkk));
+          db[g] = dee * kk;
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) red[(tid / NJG) * DK + 4 * jg + c] = lam[c];
+  }
+  __syncthreads();
+  if (tid < DK) {
+    float lm = 0.f;
+#pragma unroll
+    for (int s8 = 0; s8 < 8; ++s8) lm += red[s8 * DK + tid];
+    float st = 0.f;
+    for (int r = 0; r < DV; ++r)
+      st = fmaf(p.dS[ch * DV * DK + (size_t)r * DK + tid], p.S0[ch * DV * DK + (size_t)r * DK + tid], st);
+    const float Lam = Ls[(C - 1) * P4 + tid];
+    float acc = fmaf(st, expf(Lam), lm);
+    for (int t = C - 1; t >= 0; --t) {
+      acc += dLs[t * P4 + tid];
+      if (t < nv) dloga[row_bthd(bb, T, t0 + t, H, h, DK) + tid] = acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 namespace {
 
 template <int DK, int DV>
@@ -502,7 +808,8 @@ struct GSmem {
   static constexpr size_t bchain =
       (size_t)(C * G::PC + 3 * C * G::PK + 2 * C * (kRows + 1) + kRows * G::PK + DK) * 4;
   static constexpr size_t bpa = (size_t)(3 * C * G::PZ + C * G::PK + 3 * C * G::PC) * 4;
-  static constexpr size_t bpb = (size_t)(5 * C * G::PK + 2 * C * G::PC + 256) * 4;
+  static constexpr size_t bpe = (size_t)(5 * C * G::PK + 2 * C * G::PC + 256) * 4;
+  static constexpr size_t bpb = (size_t)(4 * C * (DK + 4) + 4 * C * (C + 4) + 8 * DK) * 4;
 };
 
 template <typename F>
@@ -531,7 +838,7 @@ cudaError_t gdn2_fwd_t(const GdnArgs& a, cudaStream_t st) {
   prof_end(st);
   KD_TRYC(cudaGetLastError());
   prof_begin(st, "gdn2_chain");
-  gdn2_chain<DK, DV><<<gr, 256, S::chain, st>>>(a.S0, a.ST, L.H, L.NC, p);
+  gdn2_chain<DK, DV><<<gr, kChainThreads, S::chain, st>>>(a.S0, a.ST, L.H, L.NC, p);
   prof_end(st);
   KD_TRYC(cudaGetLastError());
   prof_begin(st, "gdn2_out");
@@ -550,9 +857,10 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   KD_TRYC(set_smem(gdn2_bchain<DK, DV, Tin>, S::bchain));
   KD_TRYC(set_smem(gdn2_bpost_a<DK, DV, Tin>, S::bpa));
   KD_TRYC(set_smem(gdn2_bpost_b<DK, DV, Tin>, S::bpb));
+  KD_TRYC(set_smem(gdn2_bpost_exact<DK, DV, Tin>, S::bpe));
   const Tin* dO = static_cast<const Tin*>(a.dO);
   prof_begin(st, "gdn2_bchain");
-  gdn2_bchain<DK, DV, Tin><<<gr, 256, S::bchain, st>>>(dO, a.dST, a.dS0, L.H, L.T, L.NC, p);
+  gdn2_bchain<DK, DV, Tin><<<gr, kChainThreads, S::bchain, st>>>(dO, a.dST, a.dS0, L.H, L.T, L.NC, p);
   prof_end(st);
   KD_TRYC(cudaGetLastError());
   prof_begin(st, "gdn2_bpost_a");
@@ -562,8 +870,14 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   KD_TRYC(cudaGetLastError());
   prof_begin(st, "gdn2_bpost_b");
   gdn2_bpost_b<DK, DV, Tin><<<gc, 256, S::bpb, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
-                                                     a.b, a.loga, dO, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
+                                                     a.b, a.loga, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
                                                      static_cast<Tin*>(a.dk), a.db, a.dloga);
+  prof_end(st);
+  KD_TRYC(cudaGetLastError());
+  prof_begin(st, "gdn2_bpost_exact");
+  gdn2_bpost_exact<DK, DV, Tin><<<gc, 256, S::bpe, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
+                                                         a.b, a.loga, dO, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
+                                                         static_cast<Tin*>(a.dk), a.db, a.dloga);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -154,25 +154,27 @@ cudaError_t launch_epilogue_bwd(const EpilogueArgs& a, cudaStream_t st);
 // Gated DeltaNet-2 rule (kd_gdn2.cu).  Workspace per chunk ch (fp32):
 // forward (read again by the backward): A, P [C][C]; W, Q+, K^e [C][dk];
 // U', U [C][dv]; e^Lambda [dk]; chunk-start state S0 [dv][dk].  Backward:
-// dU [C][dv], chunk-end state gradient dS [dv][dk], dE [C][dk], dT, dP [C][C].
+// dU [C][dv], chunk-end state gradient dS [dv][dk], dE, dQ+, dK^e [C][dk],
+// dT, dP [C][C].
 struct GdnLayout {
   int B = 0, H = 0, T = 0, dk = 0, dv = 0, dtype = 0, NC = 0;
   size_t chunks = 0;
   size_t A = 0, P = 0, W = 0, Up = 0, Ke = 0, Qp = 0, gC = 0, S0 = 0, U = 0, fwd_bytes = 0;
-  size_t dU = 0, dS = 0, dE = 0, dT = 0, dP = 0, bwd_bytes = 0;
+  size_t dU = 0, dS = 0, dE = 0, dT = 0, dP = 0, dQp = 0, dKe = 0, bwd_bytes = 0;
 };
 struct GdnWs {
   float *A, *P, *W, *Up, *Ke, *Qp, *gC, *S0, *U;
-  float *dU, *dS, *dE, *dT, *dP;
+  float *dU, *dS, *dE, *dT, *dP, *dQp, *dKe;
 };
 inline GdnWs gdn_ws(char* base, const GdnLayout& L) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
   return GdnWs{f(L.A), f(L.P), f(L.W), f(L.Up), f(L.Ke), f(L.Qp), f(L.gC), f(L.S0), f(L.U),
-               nullptr, nullptr, nullptr, nullptr, nullptr};
+               nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
 }
 inline void gdn_bwd_ws(char* base, const GdnLayout& L, GdnWs* p) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
   p->dU = f(L.dU); p->dS = f(L.dS); p->dE = f(L.dE); p->dT = f(L.dT); p->dP = f(L.dP);
+  p->dQp = f(L.dQp); p->dKe = f(L.dKe);
 }
 struct GdnArgs {
   const void *q, *k, *v;
