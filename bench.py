@@ -284,7 +284,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-gdn2", action="store_true")
@@ -502,20 +502,40 @@ def main(argv=None):
     # ---- end to end through the public API with pinned host buffers -----
     e2e = None
     if not args.no_e2e:
+        # Every step copies its inputs from pinned host memory and reads its
+        # results back inside the timed region.  Step s+1's inputs travel on a
+        # copy stream into the other of two device buffers while step s
+        # computes; a buffer is refilled only after the step that read it ended.
         pinned = {n: t.pin_memory() for n, t in host.items()}
-        staged = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+        staged = [{n: torch.empty_like(t, device=dev) for n, t in host.items()} for _ in range(2)]
         out_h = torch.empty((B, T, H, dv), dtype=bf).pin_memory()
         dS0_h = torch.empty((B, H, dv, dk), dtype=f32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in pinned.values())
         d2h = out_h.numel() * out_h.element_size() + dS0_h.numel() * dS0_h.element_size()
+        copy = torch.cuda.Stream(device=dev)
+        loaded = [torch.cuda.Event(), torch.cuda.Event()]
+        consumed = [torch.cuda.Event(), torch.cuda.Event()]
         barrier()
         torch.cuda.synchronize()
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record(stream)
-        for _ in range(args.e2e_steps):
-            for n in staged:
-                staged[n].copy_(pinned[n], non_blocking=True)
-            o, ST, g = step(staged)
+        copy.wait_stream(stream)
+
+        def upload(slot, after_step):
+            with torch.cuda.stream(copy):
+                if after_step:
+                    copy.wait_event(consumed[slot])
+                for n, t in staged[slot].items():
+                    t.copy_(pinned[n], non_blocking=True)
+                loaded[slot].record(copy)
+        upload(0, False)
+        for si in range(args.e2e_steps):
+            slot = si % 2
+            if si + 1 < args.e2e_steps:
+                upload(1 - slot, si >= 1)
+            stream.wait_event(loaded[slot])
+            o, ST, g = step(staged[slot])
+            consumed[slot].record(stream)
             out_h.copy_(o, non_blocking=True)
             dS0_h.copy_(g["dS0"], non_blocking=True)
         x1.record(stream)
@@ -523,7 +543,10 @@ def main(argv=None):
         barrier()
         xms = max_over_ranks(x0.elapsed_time(x1), ws_n, dev)
         e2e = dict(value=job_throughput(ws_n, B * T, args.e2e_steps, xms), unit="tokens/s",
-                   h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
+                   h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=xms / args.e2e_steps,
+                   h2d_gbs=h2d * args.e2e_steps / (xms / 1e3) / 1e9,
+                   pipelining="next step's H2D on a copy stream overlaps this step's compute; D2H after it")
+        del staged
 
     value = job_throughput(ws_n, B * T, args.steps, ms_total)
 

@@ -232,24 +232,40 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
 }
 
 // ---------------------------------------------------------------------------
+// The chain kernels and the output kernel keep their tiles in rows whose pitch
+// is a multiple of 4 floats and form every dot product with 16-byte shared
+// memory loads (four channels per load), so shared-memory bandwidth no longer
+// bounds them.
+__device__ __forceinline__ float dot4(float4 a, float4 b, float s) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, s))));
+}
+
+// sum over k < n (n a multiple of 4) of a[k] b[k], both 16-byte aligned
+__device__ __forceinline__ float dotv(const float* a, const float* b, int n, float s) {
+#pragma unroll 4
+  for (int k = 0; k < n; k += 4)
+    s = dot4(*reinterpret_cast<const float4*>(a + k), *reinterpret_cast<const float4*>(b + k), s);
+  return s;
+}
+
 // The chain: one CTA per (kRows value rows, head); chunks in order.
 template <int DK, int DV>
-__global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restrict__ S0, float* __restrict__ ST, int H,
-                                                  int NC, GdnWs p) {
-  using G = GP<DK, DV>;
-  constexpr int RS = kRows, PR = RS + 1, NT = kChainThreads;
-  extern __shared__ float gsm[];
-  float* Ws = gsm;                  // [C][PK]
-  float* Kes = Ws + C * G::PK;      // [C][PK]
-  float* Ss = Kes + C * G::PK;      // [RS][PK] state rows
-  float* Us = Ss + RS * G::PK;      // [C][PR]
-  float* gcs = Us + C * PR;         // [DK]
+__global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restrict__ S0, float* __restrict__ ST,
+                                                            int H, int NC, GdnWs p) {
+  constexpr int RS = kRows, NT = kChainThreads, P4 = DK + 4, NJ = DK / 4;
+  static_assert(RS * NJ <= NT && (C * RS) % NT == 0, "thread mapping");
+  extern __shared__ __align__(16) float gsm[];
+  float* Ws = gsm;                  // [C][P4]
+  float* Kes = Ws + C * P4;         // [C][P4]
+  float* Ss = Kes + C * P4;         // [RS][P4] state rows
+  float* Us = Ss + RS * P4;         // [C][RS]
+  float* gcs = Us + C * RS;         // [DK]
   const int tid = threadIdx.x;
   const int r0 = blockIdx.x * RS, h = blockIdx.y, bb = blockIdx.z;
   const size_t unit = (size_t)bb * H + h;
   for (int e = tid; e < RS * DK; e += NT) {
     const int r = e / DK, j = e % DK;
-    Ss[r * G::PK + j] = S0 ? S0[(unit * DV + r0 + r) * DK + j] : 0.f;
+    Ss[r * P4 + j] = S0 ? S0[(unit * DV + r0 + r) * DK + j] : 0.f;
   }
   // chunk n+1's W and K^e are loaded into registers while chunk n computes
   constexpr int UPT = C * RS / NT;  // U' values per thread
@@ -269,40 +285,50 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restr
   fetch(0);
   for (int n = 0; n < NC; ++n) {
     const size_t ch = unit * NC + n;
-    frag_store<C * DK, DK, G::PK>(Ws, fw);
-    frag_store<C * DK, DK, G::PK>(Kes, fk);
+    frag_store<C * DK, DK, P4>(Ws, fw);
+    frag_store<C * DK, DK, P4>(Kes, fk);
 #pragma unroll
-    for (int i = 0; i < UPT; ++i) {
-      const int e = tid + NT * i;
-      Us[(e / RS) * PR + e % RS] = up[i];
-    }
+    for (int i = 0; i < UPT; ++i) Us[tid + NT * i] = up[i];
     if (tid < DK) gcs[tid] = gc;
     __syncthreads();
     if (n + 1 < NC) fetch(n + 1);
     for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
-      p.S0[ch * DV * DK + (size_t)(r0 + r) * DK + j] = Ss[r * G::PK + j];
+      p.S0[ch * DV * DK + (size_t)(r0 + r) * DK + j] = Ss[r * P4 + j];
     }
+    // U[t][r] = U'[t][r] - W[t] . S[r]
     for (int e = tid; e < C * RS; e += NT) {
       const int t = e / RS, r = e % RS;
-      float s = Us[t * PR + r];
-      for (int j = 0; j < DK; ++j) s = fmaf(-Ws[t * G::PK + j], Ss[r * G::PK + j], s);
-      Us[t * PR + r] = s;
-      p.U[ch * C * DV + t * DV + r0 + r] = s;
+      const float u = Us[e] - dotv(Ws + t * P4, Ss + r * P4, DK, 0.f);
+      Us[e] = u;
+      p.U[ch * C * DV + t * DV + r0 + r] = u;
     }
     __syncthreads();
-    for (int e = tid; e < RS * DK; e += NT) {
-      const int r = e / DK, j = e % DK;
-      float s = Ss[r * G::PK + j] * gcs[j];
-      for (int t = 0; t < C; ++t) s = fmaf(Us[t * PR + r], Kes[t * G::PK + j], s);
-      Ss[r * G::PK + j] = s;
+    // S[r][j..j+3] = S gamma_C + sum_t U[t][r] K^e[t][j..j+3]
+    if (tid < RS * NJ) {
+      const int r = tid / NJ, j = 4 * (tid % NJ);
+      float4 acc = *reinterpret_cast<const float4*>(Ss + r * P4 + j);
+      acc.x *= gcs[j];
+      acc.y *= gcs[j + 1];
+      acc.z *= gcs[j + 2];
+      acc.w *= gcs[j + 3];
+#pragma unroll 8
+      for (int t = 0; t < C; ++t) {
+        const float u = Us[t * RS + r];
+        const float4 kv = *reinterpret_cast<const float4*>(Kes + t * P4 + j);
+        acc.x = fmaf(u, kv.x, acc.x);
+        acc.y = fmaf(u, kv.y, acc.y);
+        acc.z = fmaf(u, kv.z, acc.z);
+        acc.w = fmaf(u, kv.w, acc.w);
+      }
+      *reinterpret_cast<float4*>(Ss + r * P4 + j) = acc;
     }
     __syncthreads();
   }
   if (ST)
     for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
-      ST[(unit * DV + r0 + r) * DK + j] = Ss[r * G::PK + j];
+      ST[(unit * DV + r0 + r) * DK + j] = Ss[r * P4 + j];
     }
 }
 
@@ -310,12 +336,12 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restr
 // O = Q+ S0^T + P U per chunk, all chunks in parallel.
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, Tin* __restrict__ out) {
-  using G = GP<DK, DV>;
-  extern __shared__ float gsm[];
-  float* Qps = gsm;                 // [C][PK]
-  float* S0s = Qps + C * G::PK;     // [DV][PK]
-  float* Ps = S0s + DV * G::PK;     // [C][PC]
-  float* Uss = Ps + C * G::PC;      // [C][PV]
+  constexpr int P4 = DK + 4, PC4 = C + 4;
+  extern __shared__ __align__(16) float gsm[];
+  float* Qps = gsm;                 // [C][P4]
+  float* S0s = Qps + C * P4;        // [DV][P4]
+  float* Ps = S0s + DV * P4;        // [C][PC4]
+  float* Ut = Ps + C * PC4;         // [DV][PC4]  U transposed
   const int tid = threadIdx.x;
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
@@ -323,26 +349,22 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
   {
     Frag<DV * DK> fs;
     frag_load(fs, p.S0 + ch * DV * DK);
-    frag_store<DV * DK, DK, G::PK>(S0s, fs);
+    frag_store<DV * DK, DK, P4>(S0s, fs);
   }
   {
     Frag<C * DK> fq;
     Frag<C * C> fp;
-    Frag<C * DV> fu;
     frag_load(fq, p.Qp + ch * C * DK);
     frag_load(fp, p.P + ch * C * C);
-    frag_load(fu, p.U + ch * C * DV);
-    frag_store<C * DK, DK, G::PK>(Qps, fq);
-    frag_store<C * C, C, G::PC>(Ps, fp);
-    frag_store<C * DV, DV, G::PV>(Uss, fu);
+    frag_store<C * DK, DK, P4>(Qps, fq);
+    frag_store<C * C, C, PC4>(Ps, fp);
   }
+  for (int e = tid; e < C * DV; e += 256) Ut[(e % DV) * PC4 + e / DV] = p.U[ch * C * DV + e];
   __syncthreads();
   for (int e = tid; e < C * DV; e += 256) {
     const int t = e / DV, r = e % DV;
     if (t >= nv) continue;
-    float s = 0.f;
-    for (int j = 0; j < DK; ++j) s = fmaf(Qps[t * G::PK + j], S0s[r * G::PK + j], s);
-    for (int i = 0; i <= t; ++i) s = fmaf(Ps[t * G::PC + i], Uss[i * G::PV + r], s);
+    const float s = dotv(Ps + t * PC4, Ut + r * PC4, C, dotv(Qps + t * P4, S0s + r * P4, DK, 0.f));
     out[row_bthd(bb, T, t0 + t, H, h, DV) + r] = from_f<Tin>(s);
   }
 }
@@ -350,25 +372,27 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
 // ---------------------------------------------------------------------------
 // Reverse chain: one CTA per (kRows value rows, head); chunks last to first.
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restrict__ dO, const float* __restrict__ dST,
-                                                   float* __restrict__ dS0, int H, int T, int NC, GdnWs p) {
-  using G = GP<DK, DV>;
-  constexpr int RS = kRows, PR = RS + 1, NT = kChainThreads;
-  extern __shared__ float gsm[];
-  float* Ps = gsm;                  // [C][PC]
-  float* Kes = Ps + C * G::PC;      // [C][PK]
-  float* Qps = Kes + C * G::PK;     // [C][PK]
-  float* Ws = Qps + C * G::PK;      // [C][PK]
-  float* dOs = Ws + C * G::PK;      // [C][PR]
-  float* dUs = dOs + C * PR;        // [C][PR]
-  float* dSs = dUs + C * PR;        // [RS][PK]
-  float* gcs = dSs + RS * G::PK;    // [DK]
+__global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restrict__ dO,
+                                                             const float* __restrict__ dST, float* __restrict__ dS0,
+                                                             int H, int T, int NC, GdnWs p) {
+  constexpr int RS = kRows, NT = kChainThreads, P4 = DK + 4, PC4 = C + 4, NJ = DK / 4;
+  static_assert(RS * NJ <= NT, "thread mapping");
+  extern __shared__ __align__(16) float gsm[];
+  float* Pt = gsm;                  // [C][PC4]  P transposed
+  float* Kes = Pt + C * PC4;        // [C][P4]
+  float* Qps = Kes + C * P4;        // [C][P4]
+  float* Ws = Qps + C * P4;         // [C][P4]
+  float* dOt = Ws + C * P4;         // [RS][PC4] dO transposed
+  float* dOs = dOt + RS * PC4;      // [C][RS]
+  float* dUs = dOs + C * RS;        // [C][RS]
+  float* dSs = dUs + C * RS;        // [RS][P4]
+  float* gcs = dSs + RS * P4;       // [DK]
   const int tid = threadIdx.x;
   const int r0 = blockIdx.x * RS, h = blockIdx.y, bb = blockIdx.z;
   const size_t unit = (size_t)bb * H + h;
   for (int e = tid; e < RS * DK; e += NT) {
     const int r = e / DK, j = e % DK;
-    dSs[r * G::PK + j] = dST ? dST[(unit * DV + r0 + r) * DK + j] : 0.f;
+    dSs[r * P4 + j] = dST ? dST[(unit * DV + r0 + r) * DK + j] : 0.f;
   }
   for (int n = NC - 1; n >= 0; --n) {
     const size_t ch = unit * NC + n;
@@ -380,43 +404,64 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restri
       frag_load(fk, p.Ke + ch * C * DK);
       frag_load(fq, p.Qp + ch * C * DK);
       frag_load(fw, p.W + ch * C * DK);
-      frag_store<C * C, C, G::PC>(Ps, fp);
-      frag_store<C * DK, DK, G::PK>(Kes, fk);
-      frag_store<C * DK, DK, G::PK>(Qps, fq);
-      frag_store<C * DK, DK, G::PK>(Ws, fw);
+#pragma unroll
+      for (int i = 0; i < Frag<C * C, NT>::V; ++i) {
+        const int e = 4 * (tid + NT * i), t = e / C, c = e % C;
+        Pt[c * PC4 + t] = fp.x[i].x;
+        Pt[(c + 1) * PC4 + t] = fp.x[i].y;
+        Pt[(c + 2) * PC4 + t] = fp.x[i].z;
+        Pt[(c + 3) * PC4 + t] = fp.x[i].w;
+      }
+      frag_store<C * DK, DK, P4>(Kes, fk);
+      frag_store<C * DK, DK, P4>(Qps, fq);
+      frag_store<C * DK, DK, P4>(Ws, fw);
     }
     for (int e = tid; e < C * RS; e += NT) {
       const int t = e / RS, r = e % RS;
-      dOs[t * PR + r] = t < nv ? to_f(dO[row_bthd(bb, T, t0 + t, H, h, DV) + r0 + r]) : 0.f;
+      const float g = t < nv ? to_f(dO[row_bthd(bb, T, t0 + t, H, h, DV) + r0 + r]) : 0.f;
+      dOs[e] = g;
+      dOt[r * PC4 + t] = g;
     }
     if (tid < DK) gcs[tid] = p.gC[ch * DK + tid];
     __syncthreads();
     for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
-      p.dS[ch * DV * DK + (size_t)(r0 + r) * DK + j] = dSs[r * G::PK + j];
+      p.dS[ch * DV * DK + (size_t)(r0 + r) * DK + j] = dSs[r * P4 + j];
     }
+    // dU[t][r] = sum_t' P[t'][t] dO[t'][r] + K^e[t] . dS[r]
     for (int e = tid; e < C * RS; e += NT) {
       const int t = e / RS, r = e % RS;
-      float s = 0.f;
-      for (int tp = t; tp < C; ++tp) s = fmaf(Ps[tp * G::PC + t], dOs[tp * PR + r], s);
-      for (int j = 0; j < DK; ++j) s = fmaf(Kes[t * G::PK + j], dSs[r * G::PK + j], s);
-      dUs[t * PR + r] = s;
+      const float s = dotv(Pt + t * PC4, dOt + r * PC4, C, dotv(Kes + t * P4, dSs + r * P4, DK, 0.f));
+      dUs[e] = s;
       p.dU[ch * C * DV + t * DV + r0 + r] = s;
     }
     __syncthreads();
-    for (int e = tid; e < RS * DK; e += NT) {
-      const int r = e / DK, j = e % DK;
-      float s = dSs[r * G::PK + j] * gcs[j];
-      for (int t = 0; t < C; ++t)
-        s = fmaf(dOs[t * PR + r], Qps[t * G::PK + j], fmaf(-dUs[t * PR + r], Ws[t * G::PK + j], s));
-      dSs[r * G::PK + j] = s;
+    // dS[r][j..j+3] = dS gamma_C + sum_t dO[t][r] Q+[t] - dU[t][r] W[t]
+    if (tid < RS * NJ) {
+      const int r = tid / NJ, j = 4 * (tid % NJ);
+      float4 acc = *reinterpret_cast<const float4*>(dSs + r * P4 + j);
+      acc.x *= gcs[j];
+      acc.y *= gcs[j + 1];
+      acc.z *= gcs[j + 2];
+      acc.w *= gcs[j + 3];
+#pragma unroll 8
+      for (int t = 0; t < C; ++t) {
+        const float go = dOs[t * RS + r], du = dUs[t * RS + r];
+        const float4 qv = *reinterpret_cast<const float4*>(Qps + t * P4 + j);
+        const float4 wv = *reinterpret_cast<const float4*>(Ws + t * P4 + j);
+        acc.x = fmaf(go, qv.x, fmaf(-du, wv.x, acc.x));
+        acc.y = fmaf(go, qv.y, fmaf(-du, wv.y, acc.y));
+        acc.z = fmaf(go, qv.z, fmaf(-du, wv.z, acc.z));
+        acc.w = fmaf(go, qv.w, fmaf(-du, wv.w, acc.w));
+      }
+      *reinterpret_cast<float4*>(dSs + r * P4 + j) = acc;
     }
     __syncthreads();
   }
   if (dS0)
     for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
-      dS0[(unit * DV + r0 + r) * DK + j] = dSs[r * G::PK + j];
+      dS0[(unit * DV + r0 + r) * DK + j] = dSs[r * P4 + j];
     }
 }
 
@@ -803,10 +848,11 @@ template <int DK, int DV>
 struct GSmem {
   using G = GP<DK, DV>;
   static constexpr size_t prep = (size_t)(3 * C * G::PK + C * G::PZ + 2 * C * G::PC) * 4;
-  static constexpr size_t chain = (size_t)(2 * C * G::PK + kRows * G::PK + C * (kRows + 1) + DK) * 4;
-  static constexpr size_t out = (size_t)(C * G::PK + DV * G::PK + C * G::PC + C * G::PV) * 4;
+  static constexpr int P4 = DK + 4, PC4 = C + 4;
+  static constexpr size_t chain = (size_t)(2 * C * P4 + kRows * P4 + C * kRows + DK) * 4;
+  static constexpr size_t out = (size_t)(C * P4 + DV * P4 + C * PC4 + DV * PC4) * 4;
   static constexpr size_t bchain =
-      (size_t)(C * G::PC + 3 * C * G::PK + 2 * C * (kRows + 1) + kRows * G::PK + DK) * 4;
+      (size_t)(C * PC4 + 3 * C * P4 + kRows * PC4 + 2 * C * kRows + kRows * P4 + DK) * 4;
   static constexpr size_t bpa = (size_t)(3 * C * G::PZ + C * G::PK + 3 * C * G::PC) * 4;
   static constexpr size_t bpe = (size_t)(5 * C * G::PK + 2 * C * G::PC + 256) * 4;
   static constexpr size_t bpb = (size_t)(4 * C * (DK + 4) + 4 * C * (C + 4) + 8 * DK) * 4;
