@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
 
+#pragma unroll 8
   for (int e = tid; e < C * DK; e += 256) {
     const int t = e / DK, j = e % DK;
     const bool ok = t < nv;
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
   }
   if (tid < DK) p.gC[ch * DK + tid] = expf(Llast[tid]);
   __syncthreads();
+#pragma unroll 8
   for (int e = tid; e < C * DV; e += 256) {
     const int t = e / DV, r = e % DV;
     const bool ok = t < nv;
@@ -296,12 +298,28 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restr
       const int r = e / DK, j = e % DK;
       p.S0[ch * DV * DK + (size_t)(r0 + r) * DK + j] = Ss[r * P4 + j];
     }
-    // U[t][r] = U'[t][r] - W[t] . S[r]
-    for (int e = tid; e < C * RS; e += NT) {
-      const int t = e / RS, r = e % RS;
-      const float u = Us[e] - dotv(Ws + t * P4, Ss + r * P4, DK, 0.f);
-      Us[e] = u;
-      p.U[ch * C * DV + t * DV + r0 + r] = u;
+    // U[t][r] = U'[t][r] - W[t] . S[r]; the thread's outputs interleaved,
+    // each dot product split over two accumulators
+    {
+      float acc[UPT][2] = {};
+#pragma unroll 4
+      for (int k = 0; k < DK; k += 8) {
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) {
+          const int e = tid + NT * i, t = e / RS, r = e % RS;
+          acc[i][0] = dot4(*reinterpret_cast<const float4*>(Ws + t * P4 + k),
+                           *reinterpret_cast<const float4*>(Ss + r * P4 + k), acc[i][0]);
+          acc[i][1] = dot4(*reinterpret_cast<const float4*>(Ws + t * P4 + k + 4),
+                           *reinterpret_cast<const float4*>(Ss + r * P4 + k + 4), acc[i][1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < UPT; ++i) {
+        const int e = tid + NT * i, t = e / RS, r = e % RS;
+        const float u = Us[e] - (acc[i][0] + acc[i][1]);
+        Us[e] = u;
+        p.U[ch * C * DV + t * DV + r0 + r] = u;
+      }
     }
     __syncthreads();
     // S[r][j..j+3] = S gamma_C + sum_t U[t][r] K^e[t][j..j+3]
@@ -359,6 +377,7 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
     frag_store<C * DK, DK, P4>(Qps, fq);
     frag_store<C * C, C, PC4>(Ps, fp);
   }
+#pragma unroll 8
   for (int e = tid; e < C * DV; e += 256) Ut[(e % DV) * PC4 + e / DV] = p.U[ch * C * DV + e];
   __syncthreads();
   for (int e = tid; e < C * DV; e += 256) {
@@ -428,12 +447,40 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restri
       const int r = e / DK, j = e % DK;
       p.dS[ch * DV * DK + (size_t)(r0 + r) * DK + j] = dSs[r * P4 + j];
     }
-    // dU[t][r] = sum_t' P[t'][t] dO[t'][r] + K^e[t] . dS[r]
-    for (int e = tid; e < C * RS; e += NT) {
-      const int t = e / RS, r = e % RS;
-      const float s = dotv(Pt + t * PC4, dOt + r * PC4, C, dotv(Kes + t * P4, dSs + r * P4, DK, 0.f));
-      dUs[e] = s;
-      p.dU[ch * C * DV + t * DV + r0 + r] = s;
+    // dU[t][r] = sum_t' P[t'][t] dO[t'][r] + K^e[t] . dS[r]; the thread's
+    // outputs interleaved, each sum split over two accumulators
+    {
+      constexpr int UPT = C * RS / NT;
+      float acc[UPT][2] = {};
+#pragma unroll 4
+      for (int k = 0; k < C; k += 8) {
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) {
+          const int e = tid + NT * i, t = e / RS, r = e % RS;
+          acc[i][0] = dot4(*reinterpret_cast<const float4*>(Pt + t * PC4 + k),
+                           *reinterpret_cast<const float4*>(dOt + r * PC4 + k), acc[i][0]);
+          acc[i][1] = dot4(*reinterpret_cast<const float4*>(Pt + t * PC4 + k + 4),
+                           *reinterpret_cast<const float4*>(dOt + r * PC4 + k + 4), acc[i][1]);
+        }
+      }
+#pragma unroll 4
+      for (int k = 0; k < DK; k += 8) {
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) {
+          const int e = tid + NT * i, t = e / RS, r = e % RS;
+          acc[i][0] = dot4(*reinterpret_cast<const float4*>(Kes + t * P4 + k),
+                           *reinterpret_cast<const float4*>(dSs + r * P4 + k), acc[i][0]);
+          acc[i][1] = dot4(*reinterpret_cast<const float4*>(Kes + t * P4 + k + 4),
+                           *reinterpret_cast<const float4*>(dSs + r * P4 + k + 4), acc[i][1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < UPT; ++i) {
+        const int e = tid + NT * i, t = e / RS, r = e % RS;
+        const float v = acc[i][0] + acc[i][1];
+        dUs[e] = v;
+        p.dU[ch * C * DV + t * DV + r0 + r] = v;
+      }
     }
     __syncthreads();
     // dS[r][j..j+3] = dS gamma_C + sum_t dO[t][r] Q+[t] - dU[t][r] W[t]
@@ -484,12 +531,14 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
+#pragma unroll 8
   for (int e = tid; e < C * DV; e += 256) {
     const int t = e / DV, r = e % DV;
     R1[t * G::PZ + r] = t < nv ? to_f(dO[row_bthd(bb, T, t0 + t, H, h, DV) + r]) : 0.f;
     R2[t * G::PZ + r] = p.U[ch * C * DV + e];
     R3[t * G::PZ + r] = p.dU[ch * C * DV + e];
   }
+#pragma unroll 8
   for (int e = tid; e < C * C; e += 256) As[(e / C) * G::PC + e % C] = p.A[ch * C * C + e];
   __syncthreads();
   // dQ+ = dO S0, dK^e = U dS (to the workspace) and dW = -dU S0: each thread an
@@ -501,8 +550,13 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
       float aq[8][4] = {}, ak[8][4] = {}, aw[8][4] = {};
       const float4* s0 = reinterpret_cast<const float4*>(p.S0 + ch * DV * DK) + jg;
       const float4* ds = reinterpret_cast<const float4*>(p.dS + ch * DV * DK) + jg;
+      float4 na = __ldg(s0), nd = __ldg(ds);  // row r+1 is in flight while row r is used
       for (int r = 0; r < DV; ++r) {
-        const float4 a = __ldg(s0 + r * NJG), d = __ldg(ds + r * NJG);
+        const float4 a = na, d = nd;
+        if (r + 1 < DV) {
+          na = __ldg(s0 + (r + 1) * NJG);
+          nd = __ldg(ds + (r + 1) * NJG);
+        }
         const float av[4] = {a.x, a.y, a.z, a.w}, dv4[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -569,7 +623,9 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
       }
   }
   __syncthreads();
+#pragma unroll 8
   for (int e = tid; e < C * DV; e += 256) R3[(e / DV) * G::PZ + e % DV] = p.Up[ch * C * DV + e];
+#pragma unroll 8
   for (int e = tid; e < C * DK; e += 256) R4[(e / DK) * G::PK + e % DK] = p.W[ch * C * DK + e];
   __syncthreads();
   // dT = -tril(dZ U'^T + dE W^T, -1)
@@ -721,10 +777,12 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
+#pragma unroll 8
   for (int e = tid; e < C * DK; e += 256) {
     const int t = e / DK, j = e % DK;
     Ls[t * P4 + j] = t < nv ? loga[row_bthd(bb, T, t0 + t, H, h, DK) + j] : 0.f;
   }
+#pragma unroll 8
   for (int e = tid; e < C * C; e += 256) {
     const int t = e / C, i = e % C;
     const float a = p.dT[ch * C * C + e], c = p.dP[ch * C * C + e];
@@ -744,6 +802,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
     }
   }
   if (__syncthreads_or(!(mx < kGdnSafeLog))) return;  // the exact kernel takes this chunk
+#pragma unroll 8
   for (int e = tid; e < C * DK; e += 256) {
     const int t = e / DK, j = e % DK;
     const bool ok = t < nv;
