@@ -494,9 +494,39 @@ def main(argv=None):
         kd.lib().kron_delta_profile_enable(0)
         gk = {ln.split()[0]: float(ln.split()[2]) for ln in gbuf.value.decode().splitlines()}
         kd.device_status()
-        gdn2 = dict(value=job_throughput(ws_n, B * T, 1, gms), unit="tokens/s", ms_per_step=gms,
-                    step="gdn2_fwd + gdn2_bwd (bf16 q/k/v/dO, fp32 gates, CUDA cores)", per_kernel_ms=gk)
         del gi, gdO, gfws, gbws
+        # decode: 100 consecutive in-place steps, B=256, H=16, d=128 (the decode workload's shape)
+        Bd, Hd, nd = 256, 16, 100
+
+        def unit3(*sh):
+            x = torch.randn(sh, generator=g_, device=dev)
+            return (x / x.norm(dim=-1, keepdim=True)).to(bf)
+        dq_, dk_, dvv = unit3(nd, Bd, Hd, dk), unit3(nd, Bd, Hd, dk), unit3(nd, Bd, Hd, dv)
+        db_ = torch.sigmoid(torch.randn((nd, Bd, Hd, dk), generator=g_, device=dev))
+        dw_ = torch.sigmoid(torch.randn((nd, Bd, Hd, dv), generator=g_, device=dev))
+        dla = -torch.nn.functional.softplus(torch.randn((nd, Bd, Hd, dk), generator=g_, device=dev) - 4.0)
+        Sd = torch.randn((Bd, Hd, dv, dk), generator=g_, device=dev) * (1.0 / 128.0) ** 0.5
+        od = torch.empty((Bd, Hd, dv), dtype=bf, device=dev)
+        for t in range(3):
+            kd.gdn2_decode(dq_[t], dk_[t], dvv[t], db_[t], dw_[t], dla[t], Sd, out=od)
+        torch.cuda.synchronize()
+        barrier()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for t in range(nd):
+            kd.gdn2_decode(dq_[t], dk_[t], dvv[t], db_[t], dw_[t], dla[t], Sd, out=od)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(d0.elapsed_time(d1), ws_n, dev)
+        per_head = 2 * dv * dk * 4 + 2 * dk * 2 + dv * 2 + 2 * dk * 4 + dv * 4 + dv * 2
+        gdec = dict(value=ws_n * nd * Bd * Hd * per_head / (dms / 1e3) / 1e9, unit="GB/s", steps=nd,
+                    us_per_step=1e3 * dms / nd, B=Bd, H=Hd, bytes_per_head=per_head,
+                    hbm_frac=(nd * Bd * Hd * per_head / (dms / 1e3) / 1e9) / peaks["hbm_gbs"])
+        del dq_, dk_, dvv, db_, dw_, dla, Sd
+        gdn2 = dict(value=job_throughput(ws_n, B * T, 1, gms), unit="tokens/s", ms_per_step=gms,
+                    step="gdn2_fwd + gdn2_bwd (bf16 q/k/v/dO, fp32 gates, CUDA cores)", per_kernel_ms=gk,
+                    decode=gdec)
     clocks = sampler.stop()
 
     # ---- end to end through the public API with pinned host buffers -----

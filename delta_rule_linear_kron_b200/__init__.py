@@ -16,7 +16,7 @@ import ctypes
 import os
 
 __all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
-           "gdn2_fwd", "gdn2_bwd",
+           "gdn2_fwd", "gdn2_bwd", "gdn2_decode",
            "workspace_size", "device_status", "library_path",
            "KronDeltaError", "KronDeltaFunction", "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
 
@@ -83,6 +83,8 @@ def lib():
         L.kron_delta_gdn2_fwd.argtypes = [vp] * 9 + [i] * 6 + [vp, sz, vp]
         L.kron_delta_gdn2_bwd.restype = i
         L.kron_delta_gdn2_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp, sz, vp]
+        L.kron_delta_gdn2_decode.restype = i
+        L.kron_delta_gdn2_decode.argtypes = [vp] * 8 + [i] * 5 + [vp]
         L.kron_delta_profile_enable.restype = None
         L.kron_delta_profile_enable.argtypes = [i]
         L.kron_delta_profile_report.restype = i
@@ -371,6 +373,26 @@ def gdn2_bwd(q, k, v, b, w, loga, S0, dO, dST=None, *, fwd_workspace, workspace=
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _stream(stream)))
     return g
+
+
+def gdn2_decode(q, k, v, b, w, loga, S, *, out=None, stream=None):
+    """One Gated DeltaNet-2 decode step.  q,k [B,H,dk], v [B,H,dv] (bf16 or fp32);
+    b, loga [B,H,dk] and w [B,H,dv] fp32; S [B,H,dv,dk] fp32 (updated in place).
+    Returns out [B,H,dv]."""
+    import torch
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, H, dv))
+    _need(b, "b", f32, (B, H, dk)); _need(w, "w", f32, (B, H, dv)); _need(loga, "loga", f32, (B, H, dk))
+    _need(S, "S", f32, (B, H, dv, dk))
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, (B, H, dv))
+    _check(lib().kron_delta_gdn2_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(w), _ptr(loga), _ptr(S),
+                                        _ptr(out), B, H, dk, dv, dt, _stream(stream)))
+    return out
 
 
 def device_status(stream=None):

@@ -599,6 +599,27 @@ int kron_delta_gdn2_bwd(const void* q, const void* k, const void* v, const float
   return launched(kd::launch_gdn2_bwd(a, static_cast<cudaStream_t>(stream)), "gdn2 backward launch");
 }
 
+int kron_delta_gdn2_decode(const void* q, const void* k, const void* v, const float* b, const float* w,
+                           const float* loga, float* S, void* out, int B, int H, int dk, int dv, int dtype,
+                           void* stream) {
+  if (B <= 0 || H <= 0) return fail(KD_ERR_INVALID_ARG, "B, H must be >= 1 (got %d, %d)", B, H);
+  if ((size_t)B * H > 0x7fffffffu) return fail(KD_ERR_INVALID_ARG, "B*H too large");
+  if (!dim_supported(dk) || !dim_supported(dv))
+    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(b, "b", true));
+  KD_TRY(check_ptr(w, "w", true));
+  KD_TRY(check_ptr(loga, "loga", true));
+  KD_TRY(check_ptr(S, "S", true));
+  KD_TRY(check_ptr(out, "out", true));
+  KD_TRY(check_stream(stream));
+  kd::GdnDecodeArgs a{q, k, v, b, w, loga, S, out, B, H, dk, dv, dtype};
+  return launched(kd::launch_gdn2_decode(a, static_cast<cudaStream_t>(stream)), "gdn2 decode launch");
+}
+
 void kron_delta_profile_enable(int on) {
   ProfState& p = prof();
   std::lock_guard<std::mutex> g(p.mu);

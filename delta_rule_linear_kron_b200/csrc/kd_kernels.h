@@ -189,6 +189,14 @@ struct GdnArgs {
   char* ws;
   GdnLayout L;
 };
+struct GdnDecodeArgs {
+  const void *q, *k, *v;
+  const float *b, *w, *loga;
+  float* S;
+  void* out;
+  int B, H, dk, dv, dtype;
+};
+cudaError_t launch_gdn2_decode(const GdnDecodeArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_fwd(const GdnArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_bwd(const GdnArgs& a, cudaStream_t st);
 

@@ -343,6 +343,21 @@ KD_API int kron_delta_gdn2_bwd(const void *q, const void *k, const void *v, cons
                                void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * One recurrent decode step of the Gated DeltaNet-2 rule: one new token per
+ * (b, h), the state updated in place (same rule and convention as
+ * kron_delta_gdn2_fwd).
+ *   q, k : [B,H,dk] (dtype); v : [B,H,dv] (dtype).
+ *   b, loga : [B,H,dk] fp32; w : [B,H,dv] fp32.
+ *   S : [B,H,dv,dk] fp32, read and overwritten with the new state.
+ *   out : o = S q after the update, [B,H,dv] (dtype).
+ * No workspace.  Errors: KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_CUDA.
+ * Asynchronous on `stream`.
+ */
+KD_API int kron_delta_gdn2_decode(const void *q, const void *k, const void *v, const float *b,
+                                  const float *w, const float *loga, float *S, void *out, int B,
+                                  int H, int dk, int dv, int dtype, void *stream);
+
+/*
  * Synchronises `stream` and reports device-side failures of earlier calls:
  * KD_OK, KD_ERR_TIMEOUT (a bounded inter-CTA wait gave up; the outputs of that
  * call are invalid) or KD_ERR_CUDA.  Clears the device error word.

@@ -185,3 +185,22 @@ def test_phase_argument_errors(L):
     rc = L.kron_delta_fwd_phase(p, p, p, p, p, p, None, p, None, 1, 1, 64, 48, 32, 1, p, 1 << 20, 0,
                                 kd.KD_PHASE_LOCAL, None)
     assert rc == kd.KD_ERR_UNSUPPORTED
+
+
+def test_gdn2_argument_errors(L):
+    p = ctypes.c_void_p(256)
+    assert L.kron_delta_gdn2_decode(p, p, p, p, p, p, p, p, 1, 1, 128, 96, 1, None) == kd.KD_ERR_UNSUPPORTED
+    assert L.kron_delta_gdn2_decode(p, p, p, p, None, p, p, p, 1, 1, 64, 64, 1, None) == kd.KD_ERR_INVALID_ARG
+    assert b"w must not be NULL" in L.kron_delta_last_error()
+    assert L.kron_delta_gdn2_fwd(p, p, p, p, p, p, None, p, None, 1, 1, 64, 32, 32, 1, p, 0, None) == \
+        kd.KD_ERR_WORKSPACE
+    assert L.kron_delta_gdn2_fwd(p, p, p, None, p, p, None, p, None, 1, 1, 64, 32, 32, 1, p, 1 << 30, None) == \
+        kd.KD_ERR_INVALID_ARG
+    need_f = kd.workspace_size(kd.KD_WS_GDN2_FWD, 1, 2, 100, 64, 32)
+    need_b = kd.workspace_size(kd.KD_WS_GDN2_BWD, 1, 2, 100, 64, 32)
+    chunks = 2 * 2
+    assert need_f >= chunks * (2 * 64 * 64 + 3 * 64 * 64 + 2 * 64 * 32 + 32 * 64) * 4
+    assert need_b >= chunks * (64 * 32 + 32 * 64 + 3 * 64 * 64 + 2 * 64 * 64) * 4
+    rc = L.kron_delta_gdn2_bwd(p, p, p, p, p, p, None, p, None, p, p, p, p, p, p, None, 1, 2, 100, 64, 32, 1,
+                               p, need_f, p, need_b - 256, None)
+    assert rc == kd.KD_ERR_WORKSPACE

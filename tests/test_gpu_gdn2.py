@@ -123,3 +123,35 @@ def test_gdn2_deterministic():
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
     for n in g1:
         assert torch.equal(g1[n], g2[n]), n
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gdn2_decode_step(dk, dv, dtype):
+    """One decode step against the oracle's one-token forward from the same state."""
+    inp = kin.make_gdn2_inputs(4, 3, 1, dk, dv, dtype, seed=dk + 2 * dv)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    q, k, v = (torch.from_numpy(inp[n][:, 0]).to("cuda", dtype=tdt) for n in ("q", "k", "v"))
+    b, w, loga = (torch.from_numpy(inp[n][:, 0]).float().cuda() for n in ("b", "w", "loga"))
+    S = torch.from_numpy(inp["S0"]).float().cuda()
+    o = kd.gdn2_decode(q, k, v, b, w, loga, S)
+    torch.cuda.synchronize()
+    O_ref, S_ref = G.fwd(**{n: inp[n] for n in NAMES}, S0=inp["S0"])
+    tf = TOL[dtype][0]
+    assert rel(host(o), O_ref[:, 0]) <= tf
+    assert rel(host(S), S_ref) <= 1e-6
+
+
+def test_gdn2_decode_steps_match_chunked_forward():
+    """100 consecutive decode steps equal the chunked forward over the same 100 tokens."""
+    inp = kin.make_gdn2_inputs(2, 4, 100, 128, 128, "bf16", seed=33)
+    d = dev(inp, "bf16")
+    out, ST, _ = kd.gdn2_fwd(*(d[n] for n in NAMES), d["S0"])
+    S = d["S0"].clone()
+    outs = []
+    for t in range(100):
+        outs.append(kd.gdn2_decode(*(d[n][:, t].contiguous() for n in NAMES), S))
+    torch.cuda.synchronize()
+    dec = torch.stack(outs, dim=1)
+    assert rel(host(dec), host(out)) <= 5e-3
+    assert rel(host(S), host(ST)) <= 1e-4
