@@ -110,13 +110,13 @@ def kernel_work(name, d=128, C=CHUNK):
 # kernel lives in and the first 16 hex digits of its sha256 at capture time;
 # a kernel whose source has changed since reports no traffic.
 NCU_TRAFFIC = {
-    "fwd_prep_tc": (449185024, "kd_fwd_tc.cu", "3423dbfb894ff939"),
-    "fwd_cross_tc": (619071744, "kd_fwd_tc.cu", "3423dbfb894ff939"),
-    "fwd_chain_tc": (833273088, "kd_fwd_tc.cu", "3423dbfb894ff939"),
-    "fwd_out_tc": (662141440, "kd_fwd_tc.cu", "3423dbfb894ff939"),
-    "bwd_pre_tc": (514533888, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
-    "bwd_post_tc": (1126970880, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
-    "bwd_chain_tc": (586813952, "kd_bwd_tc.cu", "e5fe06fa04c57d84"),
+    "fwd_prep_tc": (450502144, "kd_fwd_tc.cu", "0781816bced3ea5c"),
+    "fwd_cross_tc": (619552512, "kd_fwd_tc.cu", "0781816bced3ea5c"),
+    "fwd_chain_tc": (835102720, "kd_fwd_tc.cu", "0781816bced3ea5c"),
+    "fwd_out_tc": (662231296, "kd_fwd_tc.cu", "0781816bced3ea5c"),
+    "bwd_pre_tc": (513970176, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
+    "bwd_post_tc": (1127943168, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
+    "bwd_chain_tc": (585809920, "kd_bwd_tc.cu", "2a91356380c07551"),
 }
 
 
