@@ -28,7 +28,7 @@
 //   dZ = A^T dU, dE = A^T dW, dT = -tril(dZ U'^T + dE W^T, -1),
 //   and through the gates and exact weights to dq, dk, db, dv, dw, dloga.
 //
-// Kernels: gdn2_prep (A, P, W, U', Q+, K^e, e^Lambda per chunk), gdn2_chain,
+// Kernels: gdn2_prep (A by a blocked inverse, P, W, U', Q+, K^e, e^Lambda per chunk), gdn2_chain,
 // gdn2_out; gdn2_bchain, gdn2_bpost_a (dP, dQ+, dK^e, dZ -> dv, dw, dE, dT),
 // gdn2_bpost_b (dq, dk, db, dloga; chunks inside the safe decay range, by
 // factorised products) and gdn2_bpost_exact (the other chunks, per-element
@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
   float* Qs = Es + C * G::PK;        // [C][PZ]  q, then Z, then U'
   float* Ts = Qs + C * G::PZ;        // [C][PC]  T
   float* As = Ts + C * G::PC;        // [C][PC]  A
+  float* Tb = As + C * G::PC;        // [3][16][17] block temporaries of the inverse
   const int tid = threadIdx.x;
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
@@ -211,25 +212,68 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
     const size_t g = row_bthd(bb, T, t0 + t, H, h, DV) + r;
     Qs[t * G::PZ + r] = ok ? wg[g] * to_f(v[g]) : 0.f;
   }
-  for (int e = tid; e < C * C; e += 256) As[(e / C) * G::PC + e % C] = (e / C == e % C) ? 1.f : 0.f;
   __syncthreads();
-  // forward substitution (I + T) X = R, in place, for X = W (R = E+), U' (R = Z), A (R = I)
-  constexpr int NCOL = DK + DV + C;
-  for (int t = 1; t < C; ++t) {
-    for (int c = tid; c < NCOL; c += 256) {
-      float* X;
-      int pitch, col;
-      if (c < DK) { X = Es; pitch = G::PK; col = c; }
-      else if (c < DK + DV) { X = Qs; pitch = G::PZ; col = c - DK; }
-      else { X = As; pitch = G::PC; col = c - DK - DV; }
-      float s = X[t * pitch + col];
-      for (int i = 0; i < t; ++i) s = fmaf(-Ts[t * G::PC + i], X[i * pitch + col], s);
-      X[t * pitch + col] = s;
+  // A = (I + T)^{-1} blocked by 16: the four diagonal blocks by substitution,
+  // then A_ab = -A_aa sum_{c=b}^{a-1} T_ac A_cb below the diagonal
+  {
+    if (tid < C) {
+      const int blk = tid >> 4, m = tid & 15, o = 16 * blk;
+      float col[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        float sacc = t == m ? 1.f : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2)
+          if (s2 >= m && s2 < t) sacc = fmaf(-Ts[(o + t) * G::PC + o + s2], col[s2], sacc);
+        col[t] = t < m ? 0.f : sacc;
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) As[(o + t) * G::PC + o + m] = col[t];
+    }
+    for (int e = tid; e < C * C; e += 256) {
+      const int t = e / C, i = e % C;
+      if ((i >> 4) > (t >> 4)) As[t * G::PC + i] = 0.f;
     }
     __syncthreads();
+    for (int a = 1; a < 4; ++a) {
+      for (int e = tid; e < a * 256; e += 256) {
+        const int bb2 = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        float sacc = 0.f;
+        for (int kk = 16 * bb2; kk < 16 * a; ++kk)
+          sacc = fmaf(Ts[(16 * a + rr) * G::PC + kk], As[kk * G::PC + 16 * bb2 + cc], sacc);
+        Tb[bb2 * 272 + rr * 17 + cc] = sacc;
+      }
+      __syncthreads();
+      for (int e = tid; e < a * 256; e += 256) {
+        const int bb2 = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        float sacc = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          sacc = fmaf(As[(16 * a + rr) * G::PC + 16 * a + kk], Tb[bb2 * 272 + kk * 17 + cc], sacc);
+        As[(16 * a + rr) * G::PC + 16 * bb2 + cc] = -sacc;
+      }
+      __syncthreads();
+    }
   }
-  for (int e = tid; e < C * DK; e += 256) p.W[ch * C * DK + e] = Es[(e / DK) * G::PK + e % DK];
-  for (int e = tid; e < C * DV; e += 256) p.Up[ch * C * DV + e] = Qs[(e / DV) * G::PZ + e % DV];
+  // W = A E+ and U' = A Z (A lower triangular), 4 x 4 tiles straight to the workspace
+  for (int tile = tid; tile < 16 * (DK / 4); tile += 256) {
+    const int t4 = (tile / (DK / 4)) * 4, j4 = (tile % (DK / 4)) * 4;
+    float acc[4][4] = {};
+    mm4x4(acc, As + t4 * G::PC, G::PC, 1, Es + j4, G::PK, 1, 0, t4 + 4);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<float4*>(p.W + ch * C * DK + (t4 + u) * DK + j4) =
+          make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+  }
+  for (int tile = tid; tile < 16 * (DV / 4); tile += 256) {
+    const int t4 = (tile / (DV / 4)) * 4, r4 = (tile % (DV / 4)) * 4;
+    float acc[4][4] = {};
+    mm4x4(acc, As + t4 * G::PC, G::PC, 1, Qs + r4, G::PZ, 1, 0, t4 + 4);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<float4*>(p.Up + ch * C * DV + (t4 + u) * DV + r4) =
+          make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+  }
   for (int e = tid; e < C * C; e += 256) p.A[ch * C * C + e] = As[(e / C) * G::PC + e % C];
 }
 
@@ -906,7 +950,7 @@ namespace {
 template <int DK, int DV>
 struct GSmem {
   using G = GP<DK, DV>;
-  static constexpr size_t prep = (size_t)(3 * C * G::PK + C * G::PZ + 2 * C * G::PC) * 4;
+  static constexpr size_t prep = (size_t)(3 * C * G::PK + C * G::PZ + 2 * C * G::PC + 3 * 16 * 17) * 4;
   static constexpr int P4 = DK + 4, PC4 = C + 4;
   static constexpr size_t chain = (size_t)(2 * C * P4 + kRows * P4 + C * kRows + DK) * 4;
   static constexpr size_t out = (size_t)(C * P4 + DV * P4 + C * PC4 + DV * PC4) * 4;
