@@ -457,36 +457,48 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restri
     const int r = e / DK, j = e % DK;
     dSs[r * P4 + j] = dST ? dST[(unit * DV + r0 + r) * DK + j] : 0.f;
   }
-  for (int n = NC - 1; n >= 0; --n) {
+  // chunk n-1's tiles and dO slice are loaded into registers while chunk n computes
+  constexpr int OPT = C * RS / NT;  // dO values per thread
+  Frag<C * C, NT> fp;
+  Frag<C * DK, NT> fk, fq, fw;
+  float go[OPT], gc = 0.f;
+  auto fetch = [&](int n) {
     const size_t ch = unit * NC + n;
     const int t0 = n * C, nv = min(C, T - t0);
-    {
-      Frag<C * C, NT> fp;
-      Frag<C * DK, NT> fk, fq, fw;
-      frag_load(fp, p.P + ch * C * C);
-      frag_load(fk, p.Ke + ch * C * DK);
-      frag_load(fq, p.Qp + ch * C * DK);
-      frag_load(fw, p.W + ch * C * DK);
+    frag_load(fp, p.P + ch * C * C);
+    frag_load(fk, p.Ke + ch * C * DK);
+    frag_load(fq, p.Qp + ch * C * DK);
+    frag_load(fw, p.W + ch * C * DK);
 #pragma unroll
-      for (int i = 0; i < Frag<C * C, NT>::V; ++i) {
-        const int e = 4 * (tid + NT * i), t = e / C, c = e % C;
-        Pt[c * PC4 + t] = fp.x[i].x;
-        Pt[(c + 1) * PC4 + t] = fp.x[i].y;
-        Pt[(c + 2) * PC4 + t] = fp.x[i].z;
-        Pt[(c + 3) * PC4 + t] = fp.x[i].w;
-      }
-      frag_store<C * DK, DK, P4>(Kes, fk);
-      frag_store<C * DK, DK, P4>(Qps, fq);
-      frag_store<C * DK, DK, P4>(Ws, fw);
+    for (int i = 0; i < OPT; ++i) {
+      const int e = tid + NT * i, t = e / RS, r = e % RS;
+      go[i] = t < nv ? to_f(dO[row_bthd(bb, T, t0 + t, H, h, DV) + r0 + r]) : 0.f;
     }
-    for (int e = tid; e < C * RS; e += NT) {
-      const int t = e / RS, r = e % RS;
-      const float g = t < nv ? to_f(dO[row_bthd(bb, T, t0 + t, H, h, DV) + r0 + r]) : 0.f;
-      dOs[e] = g;
-      dOt[r * PC4 + t] = g;
+    if (tid < DK) gc = p.gC[ch * DK + tid];
+  };
+  fetch(NC - 1);
+  for (int n = NC - 1; n >= 0; --n) {
+    const size_t ch = unit * NC + n;
+#pragma unroll
+    for (int i = 0; i < Frag<C * C, NT>::V; ++i) {
+      const int e = 4 * (tid + NT * i), t = e / C, c = e % C;
+      Pt[c * PC4 + t] = fp.x[i].x;
+      Pt[(c + 1) * PC4 + t] = fp.x[i].y;
+      Pt[(c + 2) * PC4 + t] = fp.x[i].z;
+      Pt[(c + 3) * PC4 + t] = fp.x[i].w;
     }
-    if (tid < DK) gcs[tid] = p.gC[ch * DK + tid];
+    frag_store<C * DK, DK, P4>(Kes, fk);
+    frag_store<C * DK, DK, P4>(Qps, fq);
+    frag_store<C * DK, DK, P4>(Ws, fw);
+#pragma unroll
+    for (int i = 0; i < OPT; ++i) {
+      const int e = tid + NT * i, t = e / RS, r = e % RS;
+      dOs[e] = go[i];
+      dOt[r * PC4 + t] = go[i];
+    }
+    if (tid < DK) gcs[tid] = gc;
     __syncthreads();
+    if (n > 0) fetch(n - 1);
     for (int e = tid; e < RS * DK; e += NT) {
       const int r = e / DK, j = e % DK;
       p.dS[ch * DV * DK + (size_t)(r0 + r) * DK + j] = dSs[r * P4 + j];
@@ -585,43 +597,72 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
 #pragma unroll 8
   for (int e = tid; e < C * C; e += 256) As[(e / C) * G::PC + e % C] = p.A[ch * C * C + e];
   __syncthreads();
-  // dQ+ = dO S0, dK^e = U dS (to the workspace) and dW = -dU S0: each thread an
-  // 8-position x 4-channel tile, the state rows streamed as float4
+  // dQ+ = dO S0 and dW = -dU S0 in one pass over the rows of S0, dK^e = U dS in
+  // a second over dS (to the workspace): each thread an 8-position x 4-channel
+  // tile, the state rows streamed as float4 four rows ahead
   {
-    constexpr int NJG = DK / 4;
+    constexpr int NJG = DK / 4, AHEAD = 4;
+    static_assert(DV % AHEAD == 0, "row groups");
     if (tid < NJG * 8) {
       const int jg = tid % NJG, t8 = (tid / NJG) * 8;
-      float aq[8][4] = {}, ak[8][4] = {}, aw[8][4] = {};
-      const float4* s0 = reinterpret_cast<const float4*>(p.S0 + ch * DV * DK) + jg;
-      const float4* ds = reinterpret_cast<const float4*>(p.dS + ch * DV * DK) + jg;
-      float4 na = __ldg(s0), nd = __ldg(ds);  // row r+1 is in flight while row r is used
-      for (int r = 0; r < DV; ++r) {
-        const float4 a = na, d = nd;
-        if (r + 1 < DV) {
-          na = __ldg(s0 + (r + 1) * NJG);
-          nd = __ldg(ds + (r + 1) * NJG);
-        }
-        const float av[4] = {a.x, a.y, a.z, a.w}, dv4[4] = {d.x, d.y, d.z, d.w};
+      {
+        float aq[8][4] = {}, aw[8][4] = {};
+        const float4* s0 = reinterpret_cast<const float4*>(p.S0 + ch * DV * DK) + jg;
+        float4 ring[AHEAD];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float o = R1[(t8 + u) * G::PZ + r], uu = R2[(t8 + u) * G::PZ + r], du = R3[(t8 + u) * G::PZ + r];
+        for (int i = 0; i < AHEAD; ++i) ring[i] = __ldg(s0 + i * NJG);
+        for (int r0 = 0; r0 < DV; r0 += AHEAD) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            aq[u][c] = fmaf(o, av[c], aq[u][c]);
-            ak[u][c] = fmaf(uu, dv4[c], ak[u][c]);
-            aw[u][c] = fmaf(du, av[c], aw[u][c]);
+          for (int i = 0; i < AHEAD; ++i) {
+            const int r = r0 + i;
+            const float4 a = ring[i];
+            if (r + AHEAD < DV) ring[i] = __ldg(s0 + (r + AHEAD) * NJG);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float o = R1[(t8 + u) * G::PZ + r], du = R3[(t8 + u) * G::PZ + r];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                aq[u][c] = fmaf(o, av[c], aq[u][c]);
+                aw[u][c] = fmaf(du, av[c], aw[u][c]);
+              }
+            }
           }
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = t8 + u;
+          *reinterpret_cast<float4*>(p.dQp + ch * C * DK + t * DK + 4 * jg) =
+              make_float4(aq[u][0], aq[u][1], aq[u][2], aq[u][3]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) R4[t * G::PK + 4 * jg + c] = -aw[u][c];
+        }
       }
+      {
+        float ak[8][4] = {};
+        const float4* ds = reinterpret_cast<const float4*>(p.dS + ch * DV * DK) + jg;
+        float4 ring[AHEAD];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = t8 + u;
-        *reinterpret_cast<float4*>(p.dQp + ch * C * DK + t * DK + 4 * jg) =
-            make_float4(aq[u][0], aq[u][1], aq[u][2], aq[u][3]);
-        *reinterpret_cast<float4*>(p.dKe + ch * C * DK + t * DK + 4 * jg) =
-            make_float4(ak[u][0], ak[u][1], ak[u][2], ak[u][3]);
+        for (int i = 0; i < AHEAD; ++i) ring[i] = __ldg(ds + i * NJG);
+        for (int r0 = 0; r0 < DV; r0 += AHEAD) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) R4[t * G::PK + 4 * jg + c] = -aw[u][c];
+          for (int i = 0; i < AHEAD; ++i) {
+            const int r = r0 + i;
+            const float4 d = ring[i];
+            if (r + AHEAD < DV) ring[i] = __ldg(ds + (r + AHEAD) * NJG);
+            const float dv4[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float uu = R2[(t8 + u) * G::PZ + r];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) ak[u][c] = fmaf(uu, dv4[c], ak[u][c]);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(p.dKe + ch * C * DK + (t8 + u) * DK + 4 * jg) =
+              make_float4(ak[u][0], ak[u][1], ak[u][2], ak[u][3]);
       }
     }
   }
