@@ -18,7 +18,8 @@ import os
 __all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
            "gdn2_fwd", "gdn2_bwd", "gdn2_decode",
            "workspace_size", "device_status", "library_path",
-           "KronDeltaError", "KronDeltaFunction", "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
+           "KronDeltaError", "KronDeltaFunction", "PrologueFunction", "EpilogueFunction", "Gdn2Function",
+           "KD_WS_FWD", "KD_WS_FWD_SAVE", "KD_WS_BWD"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libkron_delta.so")
@@ -423,9 +424,84 @@ def _make_function():
     return KronDeltaFunction
 
 
+def _make_prologue_function():
+    import torch
+
+    class PrologueFunction(torch.autograd.Function):
+        """autograd wrapper of prologue_fwd / prologue_bwd.  apply(q_raw, k_raw,
+        v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale) -> (q, k, v, beta, c, logf)."""
+
+        @staticmethod
+        def forward(ctx, q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale=1.0):
+            o = prologue_fwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale)
+            ctx.save_for_backward(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log)
+            ctx.beta_scale = beta_scale
+            return o["q"], o["k"], o["v"], o["beta"], o["c"], o["logf"]
+
+        @staticmethod
+        def backward(ctx, dq, dk, dv, dbeta, dc, dlogf):
+            saved = ctx.saved_tensors
+            z = [torch.zeros_like(t) if g is None else g.contiguous()
+                 for g, t in zip((dq, dk, dv, dbeta, dc, dlogf), (saved[0], saved[1], saved[2], saved[3],
+                                                                 saved[4], saved[5].float()))]
+            g = prologue_bwd(*saved, *z, ctx.beta_scale)
+            return g["dq_raw"], g["dk_raw"], g["dv_raw"], g["dbeta_pre"], g["dc_pre"], g["df_pre"], g["da_log"], None
+
+    return PrologueFunction
+
+
+def _make_epilogue_function():
+    import torch
+
+    class EpilogueFunction(torch.autograd.Function):
+        """autograd wrapper of epilogue_fwd / epilogue_bwd.  apply(o, g, w) -> y."""
+
+        @staticmethod
+        def forward(ctx, o, g, w):
+            ctx.save_for_backward(o, g, w)
+            return epilogue_fwd(o, g, w)
+
+        @staticmethod
+        def backward(ctx, dy):
+            o, g, w = ctx.saved_tensors
+            r = epilogue_bwd(o, g, w, dy.contiguous())
+            return r["dO"], r["dg"], r["dw"]
+
+    return EpilogueFunction
+
+
+def _make_gdn2_function():
+    import torch
+
+    class Gdn2Function(torch.autograd.Function):
+        """autograd wrapper of gdn2_fwd / gdn2_bwd.  apply(q, k, v, b, w, loga, S0)
+        -> (out, ST)."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, b, w, loga, S0=None):
+            out, ST, ws = gdn2_fwd(q, k, v, b, w, loga, S0)
+            ctx.save_for_backward(q, k, v, b, w, loga, S0, ws)
+            return out, ST
+
+        @staticmethod
+        def backward(ctx, dO, dST):
+            q, k, v, b, w, loga, S0, ws = ctx.saved_tensors
+            dO = (torch.zeros((*q.shape[:-1], v.shape[-1]), dtype=q.dtype, device=q.device) if dO is None
+                  else dO.contiguous())
+            g = gdn2_bwd(q, k, v, b, w, loga, S0, dO, None if dST is None else dST.contiguous(), fwd_workspace=ws,
+                         want_dS0=S0 is not None)
+            return g["dq"], g["dk"], g["dv"], g["db"], g["dw"], g["dloga"], g["dS0"]
+
+    return Gdn2Function
+
+
+_LAZY = {"KronDeltaFunction": _make_function, "PrologueFunction": _make_prologue_function,
+         "EpilogueFunction": _make_epilogue_function, "Gdn2Function": _make_gdn2_function}
+
+
 def __getattr__(name):
-    if name == "KronDeltaFunction":
-        fn = _make_function()
+    if name in _LAZY:
+        fn = _LAZY[name]()
         globals()[name] = fn
         return fn
     raise AttributeError(name)

@@ -155,3 +155,15 @@ def test_gdn2_decode_steps_match_chunked_forward():
     dec = torch.stack(outs, dim=1)
     assert rel(host(dec), host(out)) <= 5e-3
     assert rel(host(S), host(ST)) <= 1e-4
+
+
+def test_gdn2_autograd_matches_direct_calls():
+    inp = kin.make_gdn2_inputs(1, 2, 130, 64, 64, "f32", seed=44)
+    d = dev(inp, "f32")
+    leaves = [d[n].clone().requires_grad_(True) for n in (*NAMES, "S0")]
+    out, ST = kd.Gdn2Function.apply(*leaves)
+    (out * d["dO"]).sum().backward()
+    _, _, ws = kd.gdn2_fwd(*(d[n] for n in NAMES), d["S0"])
+    g = kd.gdn2_bwd(*(d[n] for n in NAMES), d["S0"], d["dO"], fwd_workspace=ws)
+    for leaf, gn in zip(leaves, ("dq", "dk", "dv", "db", "dw", "dloga", "dS0")):
+        assert torch.equal(leaf.grad, g[gn]), gn

@@ -141,3 +141,23 @@ def test_prologue_feeds_the_mixer(oracle):
     O_ref, ST_ref = oracle.fwd(q, k, v, ro["beta"], ro["c"], ro["logf"])
     for x, ref in ((host(out), O_ref), (host(ST), ST_ref)):
         assert np.linalg.norm(x - ref) <= 5e-3 * np.linalg.norm(ref)
+
+
+def test_prologue_and_epilogue_autograd_match_direct_calls():
+    inp = kin.make_prologue_inputs(1, 3, 90, 64, 64, "f32", seed=21)
+    d = dev(inp, "f32")
+    names = ("q_raw", "k_raw", "v_raw", "beta_pre", "c_pre", "f_pre", "a_log")
+    leaves = [d[n].clone().requires_grad_(True) for n in names]
+    outs = kd.PrologueFunction.apply(*leaves, 2.0)
+    ups = [d[n] for n in ("dq", "dk", "dv", "dbeta", "dc", "dlogf")]
+    sum((o * u).sum() for o, u in zip(outs, ups)).backward()
+    g = kd.prologue_bwd(*(d[n] for n in names), *ups, 2.0)
+    for leaf, gn in zip(leaves, ("dq_raw", "dk_raw", "dv_raw", "dbeta_pre", "dc_pre", "df_pre", "da_log")):
+        assert torch.equal(leaf.grad, g[gn]), gn
+    e = kin.make_epilogue_inputs(1, 3, 90, 64, "f32", seed=22)
+    et = {n: torch.from_numpy(x).float().cuda() for n, x in e.items()}
+    el = [et[n].clone().requires_grad_(True) for n in ("o", "g", "w")]
+    (kd.EpilogueFunction.apply(*el) * et["dy"]).sum().backward()
+    r = kd.epilogue_bwd(et["o"], et["g"], et["w"], et["dy"])
+    for leaf, gn in zip(el, ("dO", "dg", "dw")):
+        assert torch.equal(leaf.grad, r[gn]), gn
