@@ -424,11 +424,40 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
 #pragma unroll 8
   for (int e = tid; e < C * DV; e += 256) Ut[(e % DV) * PC4 + e / DV] = p.U[ch * C * DV + e];
   __syncthreads();
-  for (int e = tid; e < C * DV; e += 256) {
-    const int t = e / DV, r = e % DV;
-    if (t >= nv) continue;
-    const float s = dotv(Ps + t * PC4, Ut + r * PC4, C, dotv(Qps + t * P4, S0s + r * P4, DK, 0.f));
-    out[row_bthd(bb, T, t0 + t, H, h, DV) + r] = from_f<Tin>(s);
+  // two outputs per step, each sum split over two accumulators (four
+  // independent chains in flight per thread)
+  constexpr int PER = C * DV / 256;
+  static_assert(PER % 2 == 0, "pairs of outputs");
+  for (int i0 = 0; i0 < PER; i0 += 2) {
+    int t[2], r[2];
+    float a[2][2] = {};
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int e = tid + 256 * (i0 + x);
+      t[x] = e / DV;
+      r[x] = e % DV;
+    }
+#pragma unroll 4
+    for (int k = 0; k < DK; k += 8)
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        a[x][0] = dot4(*reinterpret_cast<const float4*>(Qps + t[x] * P4 + k),
+                       *reinterpret_cast<const float4*>(S0s + r[x] * P4 + k), a[x][0]);
+        a[x][1] = dot4(*reinterpret_cast<const float4*>(Qps + t[x] * P4 + k + 4),
+                       *reinterpret_cast<const float4*>(S0s + r[x] * P4 + k + 4), a[x][1]);
+      }
+#pragma unroll 4
+    for (int k = 0; k < C; k += 8)
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        a[x][0] = dot4(*reinterpret_cast<const float4*>(Ps + t[x] * PC4 + k),
+                       *reinterpret_cast<const float4*>(Ut + r[x] * PC4 + k), a[x][0]);
+        a[x][1] = dot4(*reinterpret_cast<const float4*>(Ps + t[x] * PC4 + k + 4),
+                       *reinterpret_cast<const float4*>(Ut + r[x] * PC4 + k + 4), a[x][1]);
+      }
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+      if (t[x] < nv) out[row_bthd(bb, T, t0 + t[x], H, h, DV) + r[x]] = from_f<Tin>(a[x][0] + a[x][1]);
   }
 }
 
