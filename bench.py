@@ -150,6 +150,25 @@ def fp32_alu_peak_tflops(sm_mhz):
 
 
 # ---------------------------------------------------------------------------
+# Gated DeltaNet-2 kernels (CUDA cores, fp32 FMA): algorithmic flops per
+# token-head at d_k = d_v = d, C = 64, counting each dense product of the chunk
+# form once (full C x C tiles, as for the Kronecker kernels; exponentials and
+# the O(C^3) inverse not counted).
+# ---------------------------------------------------------------------------
+def gdn2_kernel_flops(name, d=128, C=CHUNK):
+    dd, cd = 2 * d * d, 2 * C * d
+    table = {
+        "gdn2_prep": 2 * cd + 2 * cd,           # T, P; W = A E+, U' = A Z
+        "gdn2_chain": 2 * dd,                   # U = U' - W S0^T; S <- S Gamma + U^T K^e
+        "gdn2_out": dd + cd,                    # Q+ S0^T + P U
+        "gdn2_bchain": cd + 3 * dd,             # P^T dO, K^e dS^T; dO^T Q+, dU^T W
+        "gdn2_bpost_a": 3 * dd + 5 * cd,        # dQ+, dK^e, dW; dP, dZ, dE; dT (two products)
+        "gdn2_bpost_b": 4 * cd,                 # dT K-, dP K-, dT^T E+, dP^T Q+
+    }
+    return table.get(name)
+
+
+# ---------------------------------------------------------------------------
 class ClockSampler:
     """nvidia-smi clock/throttle samples every 200 ms while running."""
 
@@ -524,8 +543,21 @@ def main(argv=None):
                     us_per_step=1e3 * dms / nd, B=Bd, H=Hd, bytes_per_head=per_head,
                     hbm_frac=(nd * Bd * Hd * per_head / (dms / 1e3) / 1e9) / peaks["hbm_gbs"])
         del dq_, dk_, dvv, db_, dw_, dla, Sd
+        alu_peak = fp32_alu_peak_tflops(1965.0)
+        gkr = {}
+        for name, kms in gk.items():
+            f = gdn2_kernel_flops(name)
+            if f is None or kms <= 0:
+                continue
+            ach = f * B * H * T / (kms / 1e3) / 1e12
+            gkr[name] = dict(bound="alu", achieved=ach, peak=alu_peak, unit="TFLOP/s", frac=ach / alu_peak,
+                             algorithmic_flops_per_launch=f * B * H * T, ms=kms)
+        top = max(gkr, key=lambda n: gkr[n]["ms"]) if gkr else None
         gdn2 = dict(value=job_throughput(ws_n, B * T, 1, gms), unit="tokens/s", ms_per_step=gms,
                     step="gdn2_fwd + gdn2_bwd (bf16 q/k/v/dO, fp32 gates, CUDA cores)", per_kernel_ms=gk,
+                    kernel_rooflines=gkr,
+                    roofline=None if top is None else dict(kernel=top, **gkr[top],
+                                                           peak_note="148 SMs x 128 FP32 lanes x 2 x 1965 MHz"),
                     decode=gdec)
     clocks = sampler.stop()
 
