@@ -342,48 +342,61 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restr
       const int r = e / DK, j = e % DK;
       p.S0[ch * DV * DK + (size_t)(r0 + r) * DK + j] = Ss[r * P4 + j];
     }
-    // U[t][r] = U'[t][r] - W[t] . S[r]; the thread's outputs interleaved,
-    // each dot product split over two accumulators
-    {
-      float acc[UPT][2] = {};
-#pragma unroll 4
-      for (int k = 0; k < DK; k += 8) {
+    // U[t][r] = U'[t][r] - W[t] . S[r]: 4 positions x 4 rows per thread, so each
+    // 16-byte shared load feeds four dot products
+    if (tid < (C / 4) * (RS / 4)) {
+      const int t4 = (tid / (RS / 4)) * 4, r4 = (tid % (RS / 4)) * 4;
+      float acc[4][4] = {};
+#pragma unroll 2
+      for (int k = 0; k < DK; k += 4) {
+        float4 a[4], b[4];
 #pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-          const int e = tid + NT * i, t = e / RS, r = e % RS;
-          acc[i][0] = dot4(*reinterpret_cast<const float4*>(Ws + t * P4 + k),
-                           *reinterpret_cast<const float4*>(Ss + r * P4 + k), acc[i][0]);
-          acc[i][1] = dot4(*reinterpret_cast<const float4*>(Ws + t * P4 + k + 4),
-                           *reinterpret_cast<const float4*>(Ss + r * P4 + k + 4), acc[i][1]);
+        for (int u = 0; u < 4; ++u) {
+          a[u] = *reinterpret_cast<const float4*>(Ws + (t4 + u) * P4 + k);
+          b[u] = *reinterpret_cast<const float4*>(Ss + (r4 + u) * P4 + k);
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = dot4(a[u], b[v], acc[u][v]);
       }
 #pragma unroll
-      for (int i = 0; i < UPT; ++i) {
-        const int e = tid + NT * i, t = e / RS, r = e % RS;
-        const float u = Us[e] - (acc[i][0] + acc[i][1]);
-        Us[e] = u;
-        p.U[ch * C * DV + t * DV + r0 + r] = u;
-      }
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int t = t4 + u, r = r4 + v;
+          const float uu = Us[t * RS + r] - acc[u][v];
+          Us[t * RS + r] = uu;
+          p.U[ch * C * DV + t * DV + r0 + r] = uu;
+        }
     }
     __syncthreads();
-    // S[r][j..j+3] = S gamma_C + sum_t U[t][r] K^e[t][j..j+3]
-    if (tid < RS * NJ) {
-      const int r = tid / NJ, j = 4 * (tid % NJ);
-      float4 acc = *reinterpret_cast<const float4*>(Ss + r * P4 + j);
-      acc.x *= gcs[j];
-      acc.y *= gcs[j + 1];
-      acc.z *= gcs[j + 2];
-      acc.w *= gcs[j + 3];
-#pragma unroll 8
-      for (int t = 0; t < C; ++t) {
-        const float u = Us[t * RS + r];
-        const float4 kv = *reinterpret_cast<const float4*>(Kes + t * P4 + j);
-        acc.x = fmaf(u, kv.x, acc.x);
-        acc.y = fmaf(u, kv.y, acc.y);
-        acc.z = fmaf(u, kv.z, acc.z);
-        acc.w = fmaf(u, kv.w, acc.w);
+    // S[r][j..j+3] = S gamma_C + sum_t U[t][r] K^e[t][j..j+3]: 4 rows x 4 channels
+    // per thread
+    if (tid < (RS / 4) * NJ) {
+      const int r4 = (tid / NJ) * 4, j = 4 * (tid % NJ);
+      float acc[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 sv = *reinterpret_cast<const float4*>(Ss + (r4 + u) * P4 + j);
+        acc[u][0] = sv.x * gcs[j];
+        acc[u][1] = sv.y * gcs[j + 1];
+        acc[u][2] = sv.z * gcs[j + 2];
+        acc[u][3] = sv.w * gcs[j + 3];
       }
-      *reinterpret_cast<float4*>(Ss + r * P4 + j) = acc;
+#pragma unroll 4
+      for (int t = 0; t < C; ++t) {
+        const float4 uv = *reinterpret_cast<const float4*>(Us + t * RS + r4);
+        const float4 kv = *reinterpret_cast<const float4*>(Kes + t * P4 + j);
+        const float ua[4] = {uv.x, uv.y, uv.z, uv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[u][c] = fmaf(ua[u], ka[c], acc[u][c]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(Ss + (r4 + u) * P4 + j) = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
     __syncthreads();
   }
@@ -532,61 +545,76 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_bchain(const Tin* __restri
       const int r = e / DK, j = e % DK;
       p.dS[ch * DV * DK + (size_t)(r0 + r) * DK + j] = dSs[r * P4 + j];
     }
-    // dU[t][r] = sum_t' P[t'][t] dO[t'][r] + K^e[t] . dS[r]; the thread's
-    // outputs interleaved, each sum split over two accumulators
-    {
-      constexpr int UPT = C * RS / NT;
-      float acc[UPT][2] = {};
-#pragma unroll 4
-      for (int k = 0; k < C; k += 8) {
+    // dU[t][r] = sum_t' P[t'][t] dO[t'][r] + K^e[t] . dS[r]: 4 positions x 4 rows
+    // per thread
+    if (tid < (C / 4) * (RS / 4)) {
+      const int t4 = (tid / (RS / 4)) * 4, r4 = (tid % (RS / 4)) * 4;
+      float acc[4][4] = {};
+#pragma unroll 2
+      for (int k = 0; k < C; k += 4) {
+        float4 a[4], b[4];
 #pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-          const int e = tid + NT * i, t = e / RS, r = e % RS;
-          acc[i][0] = dot4(*reinterpret_cast<const float4*>(Pt + t * PC4 + k),
-                           *reinterpret_cast<const float4*>(dOt + r * PC4 + k), acc[i][0]);
-          acc[i][1] = dot4(*reinterpret_cast<const float4*>(Pt + t * PC4 + k + 4),
-                           *reinterpret_cast<const float4*>(dOt + r * PC4 + k + 4), acc[i][1]);
+        for (int u = 0; u < 4; ++u) {
+          a[u] = *reinterpret_cast<const float4*>(Pt + (t4 + u) * PC4 + k);
+          b[u] = *reinterpret_cast<const float4*>(dOt + (r4 + u) * PC4 + k);
         }
-      }
-#pragma unroll 4
-      for (int k = 0; k < DK; k += 8) {
 #pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-          const int e = tid + NT * i, t = e / RS, r = e % RS;
-          acc[i][0] = dot4(*reinterpret_cast<const float4*>(Kes + t * P4 + k),
-                           *reinterpret_cast<const float4*>(dSs + r * P4 + k), acc[i][0]);
-          acc[i][1] = dot4(*reinterpret_cast<const float4*>(Kes + t * P4 + k + 4),
-                           *reinterpret_cast<const float4*>(dSs + r * P4 + k + 4), acc[i][1]);
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = dot4(a[u], b[v], acc[u][v]);
+      }
+#pragma unroll 2
+      for (int k = 0; k < DK; k += 4) {
+        float4 a[4], b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          a[u] = *reinterpret_cast<const float4*>(Kes + (t4 + u) * P4 + k);
+          b[u] = *reinterpret_cast<const float4*>(dSs + (r4 + u) * P4 + k);
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = dot4(a[u], b[v], acc[u][v]);
       }
 #pragma unroll
-      for (int i = 0; i < UPT; ++i) {
-        const int e = tid + NT * i, t = e / RS, r = e % RS;
-        const float v = acc[i][0] + acc[i][1];
-        dUs[e] = v;
-        p.dU[ch * C * DV + t * DV + r0 + r] = v;
-      }
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int t = t4 + u, r = r4 + v;
+          dUs[t * RS + r] = acc[u][v];
+          p.dU[ch * C * DV + t * DV + r0 + r] = acc[u][v];
+        }
     }
     __syncthreads();
-    // dS[r][j..j+3] = dS gamma_C + sum_t dO[t][r] Q+[t] - dU[t][r] W[t]
-    if (tid < RS * NJ) {
-      const int r = tid / NJ, j = 4 * (tid % NJ);
-      float4 acc = *reinterpret_cast<const float4*>(dSs + r * P4 + j);
-      acc.x *= gcs[j];
-      acc.y *= gcs[j + 1];
-      acc.z *= gcs[j + 2];
-      acc.w *= gcs[j + 3];
-#pragma unroll 8
+    // dS[r][j..j+3] = dS gamma_C + sum_t dO[t][r] Q+[t] - dU[t][r] W[t]: 4 rows x
+    // 4 channels per thread
+    if (tid < (RS / 4) * NJ) {
+      const int r4 = (tid / NJ) * 4, j = 4 * (tid % NJ);
+      float acc[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 sv = *reinterpret_cast<const float4*>(dSs + (r4 + u) * P4 + j);
+        acc[u][0] = sv.x * gcs[j];
+        acc[u][1] = sv.y * gcs[j + 1];
+        acc[u][2] = sv.z * gcs[j + 2];
+        acc[u][3] = sv.w * gcs[j + 3];
+      }
+#pragma unroll 4
       for (int t = 0; t < C; ++t) {
-        const float go = dOs[t * RS + r], du = dUs[t * RS + r];
+        const float4 gv = *reinterpret_cast<const float4*>(dOs + t * RS + r4);
+        const float4 dv4 = *reinterpret_cast<const float4*>(dUs + t * RS + r4);
         const float4 qv = *reinterpret_cast<const float4*>(Qps + t * P4 + j);
         const float4 wv = *reinterpret_cast<const float4*>(Ws + t * P4 + j);
-        acc.x = fmaf(go, qv.x, fmaf(-du, wv.x, acc.x));
-        acc.y = fmaf(go, qv.y, fmaf(-du, wv.y, acc.y));
-        acc.z = fmaf(go, qv.z, fmaf(-du, wv.z, acc.z));
-        acc.w = fmaf(go, qv.w, fmaf(-du, wv.w, acc.w));
+        const float ga[4] = {gv.x, gv.y, gv.z, gv.w}, da[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+        const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[u][c] = fmaf(ga[u], qa[c], fmaf(-da[u], wa[c], acc[u][c]));
       }
-      *reinterpret_cast<float4*>(dSs + r * P4 + j) = acc;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(dSs + (r4 + u) * P4 + j) = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
     __syncthreads();
   }
@@ -767,7 +795,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_a(const Tin* __restrict__ v, c
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256) gdn2_bpost_exact(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                     const float* __restrict__ bg, const float* __restrict__ loga,
-                                                    const Tin* __restrict__ dO, int H, int T, int NC, GdnWs p,
+                                                    int H, int T, int NC, GdnWs p,
                                                     Tin* __restrict__ dq, Tin* __restrict__ dk,
                                                     float* __restrict__ db, float* __restrict__ dloga) {
   using G = GP<DK, DV>;
@@ -1095,7 +1123,7 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   KD_TRYC(cudaGetLastError());
   prof_begin(st, "gdn2_bpost_exact");
   gdn2_bpost_exact<DK, DV, Tin><<<gc, 256, S::bpe, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
-                                                         a.b, a.loga, dO, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
+                                                         a.b, a.loga, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
                                                          static_cast<Tin*>(a.dk), a.db, a.dloga);
   prof_end(st);
   return cudaGetLastError();
