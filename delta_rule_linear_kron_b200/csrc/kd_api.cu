@@ -257,7 +257,7 @@ void prof_end(cudaStream_t st) {
 
 extern "C" {
 
-int kron_delta_version(void) { return 100; }
+int kron_delta_version(void) { return 200; }
 
 const char* kron_delta_last_error(void) { return g_err.c_str(); }
 
