@@ -256,10 +256,20 @@ def oracle_baseline(T_sample, seed=1004):
     oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], inp["dO"],
                nthreads=cores)
     el = time.perf_counter() - t
+    # the same work on one thread, on a quarter of the sample
+    T1 = max(64, T_sample // 4)
+    one = {n: inp[n][:, :T1] for n in ("q", "k", "v", "beta", "c", "logf", "dO")}
+    one["S0"] = inp["S0"]
+    t = time.perf_counter()
+    oracle.fwd(one["q"], one["k"], one["v"], one["beta"], one["c"], one["logf"], one["S0"], nthreads=1)
+    oracle.bwd(one["q"], one["k"], one["v"], one["beta"], one["c"], one["logf"], one["S0"], one["dO"], nthreads=1)
+    el1 = time.perf_counter() - t
     return dict(value=WL["B"] * T_sample / el, unit="tokens/s", cores=min(cores, WL["H"]), kind="oracle",
                 sample=f"first {T_sample} tokens x {WL['H']} heads of the workload, fwd+bwd, fp64, "
                        f"threaded over heads ({min(cores, WL['H'])} threads used of {cores} cores)",
-                seconds=el)
+                seconds=el,
+                single_thread=dict(value=WL["B"] * T1 / el1, unit="tokens/s", cores=1, seconds=el1,
+                                   sample=f"first {T1} tokens x {WL['H']} heads, one thread"))
 
 
 def run_reference(args):
