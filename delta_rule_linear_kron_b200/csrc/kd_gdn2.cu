@@ -408,24 +408,22 @@ __global__ void __launch_bounds__(kChainThreads) gdn2_chain(const float* __restr
 }
 
 // ---------------------------------------------------------------------------
-// O = Q+ S0^T + P U per chunk, all chunks in parallel.
+// O = Q+ S0^T + P U per chunk, all chunks in parallel.  Each thread owns one
+// value row r and C / (256 / DV) positions; S0 passes through shared memory in
+// 32-channel slabs, which keeps the CTA at about 100 KB so two fit on an SM.
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, Tin* __restrict__ out) {
-  constexpr int P4 = DK + 4, PC4 = C + 4;
+__global__ void __launch_bounds__(256, 2) gdn2_out(int H, int T, int NC, GdnWs p, Tin* __restrict__ out) {
+  constexpr int P4 = DK + 4, PC4 = C + 4, SL = 32, PS = SL + 4;
+  constexpr int NTG = 256 / DV, TPT = C / NTG;  // position groups, positions per thread
   extern __shared__ __align__(16) float gsm[];
   float* Qps = gsm;                 // [C][P4]
-  float* S0s = Qps + C * P4;        // [DV][P4]
-  float* Ps = S0s + DV * P4;        // [C][PC4]
+  float* Ps = Qps + C * P4;         // [C][PC4]
   float* Ut = Ps + C * PC4;         // [DV][PC4]  U transposed
+  float* S0s = Ut + DV * PC4;       // [DV][PS]   one 32-channel slab of S0
   const int tid = threadIdx.x;
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
-  {
-    Frag<DV * DK> fs;
-    frag_load(fs, p.S0 + ch * DV * DK);
-    frag_store<DV * DK, DK, P4>(S0s, fs);
-  }
   {
     Frag<C * DK> fq;
     Frag<C * C> fp;
@@ -436,42 +434,37 @@ __global__ void __launch_bounds__(256) gdn2_out(int H, int T, int NC, GdnWs p, T
   }
 #pragma unroll 8
   for (int e = tid; e < C * DV; e += 256) Ut[(e % DV) * PC4 + e / DV] = p.U[ch * C * DV + e];
-  __syncthreads();
-  // two outputs per step, each sum split over two accumulators (four
-  // independent chains in flight per thread)
-  constexpr int PER = C * DV / 256;
-  static_assert(PER % 2 == 0, "pairs of outputs");
-  for (int i0 = 0; i0 < PER; i0 += 2) {
-    int t[2], r[2];
-    float a[2][2] = {};
+  const int r = tid % DV, tg = (tid / DV) * TPT;
+  float acc[TPT];
 #pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const int e = tid + 256 * (i0 + x);
-      t[x] = e / DV;
-      r[x] = e % DV;
+  for (int i = 0; i < TPT; ++i) acc[i] = 0.f;
+  const float* s0 = p.S0 + ch * DV * DK;
+  for (int j0 = 0; j0 < DK; j0 += SL) {
+    __syncthreads();  // the previous slab has been read (and, the first time, the tiles above are in)
+#pragma unroll
+    for (int e = tid; e < DV * SL / 4; e += 256) {
+      const int rr = e / (SL / 4), c4 = 4 * (e % (SL / 4));
+      *reinterpret_cast<float4*>(S0s + rr * PS + c4) = __ldg(reinterpret_cast<const float4*>(s0 + rr * DK + j0 + c4));
     }
-#pragma unroll 4
-    for (int k = 0; k < DK; k += 8)
+    __syncthreads();
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        a[x][0] = dot4(*reinterpret_cast<const float4*>(Qps + t[x] * P4 + k),
-                       *reinterpret_cast<const float4*>(S0s + r[x] * P4 + k), a[x][0]);
-        a[x][1] = dot4(*reinterpret_cast<const float4*>(Qps + t[x] * P4 + k + 4),
-                       *reinterpret_cast<const float4*>(S0s + r[x] * P4 + k + 4), a[x][1]);
-      }
-#pragma unroll 4
-    for (int k = 0; k < C; k += 8)
+    for (int j = 0; j < SL; j += 4) {
+      const float4 sv = *reinterpret_cast<const float4*>(S0s + r * PS + j);
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        a[x][0] = dot4(*reinterpret_cast<const float4*>(Ps + t[x] * PC4 + k),
-                       *reinterpret_cast<const float4*>(Ut + r[x] * PC4 + k), a[x][0]);
-        a[x][1] = dot4(*reinterpret_cast<const float4*>(Ps + t[x] * PC4 + k + 4),
-                       *reinterpret_cast<const float4*>(Ut + r[x] * PC4 + k + 4), a[x][1]);
-      }
-#pragma unroll
-    for (int x = 0; x < 2; ++x)
-      if (t[x] < nv) out[row_bthd(bb, T, t0 + t[x], H, h, DV) + r[x]] = from_f<Tin>(a[x][0] + a[x][1]);
+      for (int i = 0; i < TPT; ++i)
+        acc[i] = dot4(*reinterpret_cast<const float4*>(Qps + (tg + i) * P4 + j0 + j), sv, acc[i]);
+    }
   }
+#pragma unroll 4
+  for (int k = 0; k < C; k += 4) {
+    const float4 uv = *reinterpret_cast<const float4*>(Ut + r * PC4 + k);
+#pragma unroll
+    for (int i = 0; i < TPT; ++i)
+      acc[i] = dot4(*reinterpret_cast<const float4*>(Ps + (tg + i) * PC4 + k), uv, acc[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < TPT; ++i)
+    if (tg + i < nv) out[row_bthd(bb, T, t0 + tg + i, H, h, DV) + r] = from_f<Tin>(acc[i]);
 }
 
 // ---------------------------------------------------------------------------
@@ -1051,7 +1044,7 @@ struct GSmem {
   static constexpr size_t prep = (size_t)(3 * C * G::PK + C * G::PZ + 2 * C * G::PC + 3 * 16 * 17) * 4;
   static constexpr int P4 = DK + 4, PC4 = C + 4;
   static constexpr size_t chain = (size_t)(2 * C * P4 + kRows * P4 + C * kRows + DK) * 4;
-  static constexpr size_t out = (size_t)(C * P4 + DV * P4 + C * PC4 + DV * PC4) * 4;
+  static constexpr size_t out = (size_t)(C * P4 + C * PC4 + DV * PC4 + DV * 36) * 4;
   static constexpr size_t bchain =
       (size_t)(C * PC4 + 3 * C * P4 + kRows * PC4 + 2 * C * kRows + kRows * P4 + DK) * 4;
   static constexpr size_t bpa = (size_t)(3 * C * G::PZ + C * G::PK + 3 * C * G::PC) * 4;
