@@ -45,6 +45,7 @@ constexpr int C = kChunk;
 // chains of 16 heads at d_v = 128 fit in one wave on 148 SMs.
 constexpr int kRows = 16;
 constexpr int kChainThreads = 512;  // threads of a chain CTA
+constexpr int kPostThreads = 512;   // threads of the factorised backward kernel
 // In-chunk |L| below which the backward factors e^{L_t - L_i} = gamma_t / gamma_i
 // (e^{+-60} and their products stay well inside fp32's normal range).
 constexpr float kGdnSafeLog = 60.f;
@@ -890,14 +891,14 @@ __global__ void __launch_bounds__(256) gdn2_bpost_exact(const Tin* __restrict__ 
 //   X1 = dT K-,  X2 = dP K-,  Y = dT^T E+ + dP^T Q+                 ([C][DK])
 //   de = gamma (dE + X1),  dq = gamma (dQ+ + X2),  dk = dK^e e^{Lambda-L} + Y / gamma
 //   dL = dE E+ + dQ+ Q+ - dK^e K^e + E+ X1 + Q+ X2 - K- Y
-// Each thread owns an 8-position x 4-channel tile of all three products.
+// Each thread owns a 4-position x 4-channel tile of all three products.
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(kPostThreads) gdn2_bpost_b(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                     const float* __restrict__ bg, const float* __restrict__ loga,
                                                     int H, int T, int NC, GdnWs p, Tin* __restrict__ dq,
                                                     Tin* __restrict__ dk, float* __restrict__ db,
                                                     float* __restrict__ dloga) {
-  constexpr int P4 = DK + 4, PT = C + 4, NJG = DK / 4;
+  constexpr int P4 = DK + 4, PT = C + 4, NJG = DK / 4, NT = kPostThreads, NTG = C / 4;
   extern __shared__ __align__(16) float gsm[];
   float* Ls = gsm;                  // [C][P4]  L
   float* Km = Ls + C * P4;          // [C][P4]  K-
@@ -907,18 +908,18 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
   float* dPr = dTr + C * PT;        // [C][PT]  dP, rows t
   float* dTc = dPr + C * PT;        // [C][PT]  dT^T, then dL
   float* dPc = dTc + C * PT;        // [C][PT]  dP^T
-  float* red = dPc + C * PT;        // [8][DK]
+  float* red = dPc + C * PT;        // [NTG][DK]
   const int tid = threadIdx.x;
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
 #pragma unroll 8
-  for (int e = tid; e < C * DK; e += 256) {
+  for (int e = tid; e < C * DK; e += NT) {
     const int t = e / DK, j = e % DK;
     Ls[t * P4 + j] = t < nv ? loga[row_bthd(bb, T, t0 + t, H, h, DK) + j] : 0.f;
   }
 #pragma unroll 8
-  for (int e = tid; e < C * C; e += 256) {
+  for (int e = tid; e < C * C; e += NT) {
     const int t = e / C, i = e % C;
     const float a = p.dT[ch * C * C + e], c = p.dP[ch * C * C + e];
     dTr[t * PT + i] = a;
@@ -938,7 +939,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
   }
   if (__syncthreads_or(!(mx < kGdnSafeLog))) return;  // the exact kernel takes this chunk
 #pragma unroll 8
-  for (int e = tid; e < C * DK; e += 256) {
+  for (int e = tid; e < C * DK; e += NT) {
     const int t = e / DK, j = e % DK;
     const bool ok = t < nv;
     const size_t g = row_bthd(bb, T, t0 + t, H, h, DK) + j;
@@ -949,39 +950,37 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
     Qp[t * P4 + j] = p.Qp[ch * C * DK + e];
   }
   __syncthreads();
-  const bool act = tid < NJG * 8;
-  const int jg = tid % NJG, t8 = (tid / NJG) * 8;
-  float x1[8][4] = {}, x2[8][4] = {}, y[8][4] = {};
+  const bool act = tid < NJG * NTG;
+  const int jg = tid % NJG, t4 = (tid / NJG) * 4;
+  float x1[4][4] = {}, x2[4][4] = {}, y[4][4] = {};
   if (act) {
+#pragma unroll 4
     for (int i = 0; i < C; ++i) {
       const float4 km = *reinterpret_cast<const float4*>(Km + i * P4 + 4 * jg);
-      const float4 ta = *reinterpret_cast<const float4*>(dTc + i * PT + t8);
-      const float4 tb = *reinterpret_cast<const float4*>(dTc + i * PT + t8 + 4);
-      const float4 pa = *reinterpret_cast<const float4*>(dPc + i * PT + t8);
-      const float4 pb = *reinterpret_cast<const float4*>(dPc + i * PT + t8 + 4);
+      const float4 ta = *reinterpret_cast<const float4*>(dTc + i * PT + t4);
+      const float4 pa = *reinterpret_cast<const float4*>(dPc + i * PT + t4);
       const float kv[4] = {km.x, km.y, km.z, km.w};
-      const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-      const float pv[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+      const float tv[4] = {ta.x, ta.y, ta.z, ta.w};
+      const float pv[4] = {pa.x, pa.y, pa.z, pa.w};
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           x1[u][c] = fmaf(tv[u], kv[c], x1[u][c]);
           x2[u][c] = fmaf(pv[u], kv[c], x2[u][c]);
         }
     }
+#pragma unroll 4
     for (int tp = 0; tp < C; ++tp) {
       const float4 ea = *reinterpret_cast<const float4*>(Ep + tp * P4 + 4 * jg);
       const float4 qa = *reinterpret_cast<const float4*>(Qp + tp * P4 + 4 * jg);
-      const float4 ta = *reinterpret_cast<const float4*>(dTr + tp * PT + t8);
-      const float4 tb = *reinterpret_cast<const float4*>(dTr + tp * PT + t8 + 4);
-      const float4 pa = *reinterpret_cast<const float4*>(dPr + tp * PT + t8);
-      const float4 pb = *reinterpret_cast<const float4*>(dPr + tp * PT + t8 + 4);
+      const float4 ta = *reinterpret_cast<const float4*>(dTr + tp * PT + t4);
+      const float4 pa = *reinterpret_cast<const float4*>(dPr + tp * PT + t4);
       const float ev[4] = {ea.x, ea.y, ea.z, ea.w}, qv[4] = {qa.x, qa.y, qa.z, qa.w};
-      const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-      const float pv[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+      const float tv[4] = {ta.x, ta.y, ta.z, ta.w};
+      const float pv[4] = {pa.x, pa.y, pa.z, pa.w};
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int c = 0; c < 4; ++c) y[u][c] = fmaf(tv[u], ev[c], fmaf(pv[u], qv[c], y[u][c]));
     }
@@ -991,8 +990,8 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
   float lam[4] = {};
   if (act) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int t = t8 + u;
+    for (int u = 0; u < 4; ++u) {
+      const int t = t4 + u;
       const bool ok = t < nv;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -1022,7 +1021,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_b(const Tin* __restrict__ q, c
   if (tid < DK) {
     float lm = 0.f;
 #pragma unroll
-    for (int s8 = 0; s8 < 8; ++s8) lm += red[s8 * DK + tid];
+    for (int s8 = 0; s8 < NTG; ++s8) lm += red[s8 * DK + tid];
     float st = 0.f;
     for (int r = 0; r < DV; ++r)
       st = fmaf(p.dS[ch * DV * DK + (size_t)r * DK + tid], p.S0[ch * DV * DK + (size_t)r * DK + tid], st);
@@ -1049,7 +1048,7 @@ struct GSmem {
       (size_t)(C * PC4 + 3 * C * P4 + kRows * PC4 + 2 * C * kRows + kRows * P4 + DK) * 4;
   static constexpr size_t bpa = (size_t)(3 * C * G::PZ + C * G::PK + 3 * C * G::PC) * 4;
   static constexpr size_t bpe = (size_t)(5 * C * G::PK + 2 * C * G::PC + 256) * 4;
-  static constexpr size_t bpb = (size_t)(4 * C * (DK + 4) + 4 * C * (C + 4) + 8 * DK) * 4;
+  static constexpr size_t bpb = (size_t)(4 * C * (DK + 4) + 4 * C * (C + 4) + (C / 4) * DK) * 4;
 };
 
 template <typename F>
@@ -1109,7 +1108,7 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   prof_end(st);
   KD_TRYC(cudaGetLastError());
   prof_begin(st, "gdn2_bpost_b");
-  gdn2_bpost_b<DK, DV, Tin><<<gc, 256, S::bpb, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
+  gdn2_bpost_b<DK, DV, Tin><<<gc, kPostThreads, S::bpb, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
                                                      a.b, a.loga, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
                                                      static_cast<Tin*>(a.dk), a.db, a.dloga);
   prof_end(st);
