@@ -142,17 +142,16 @@ __global__ void __launch_bounds__(256) gdn2_prep(const Tin* __restrict__ q, cons
     Ls[t * G::PK + j] = ok ? loga[g] : 0.f;
   }
   __syncthreads();
+  float mx = 0.f;  // largest in-chunk |L| of this thread's channel
   if (tid < DK) {
     float acc = 0.f;
     for (int t = 0; t < C; ++t) {
       acc += Ls[t * G::PK + tid];
       Ls[t * G::PK + tid] = acc;
+      mx = fmaxf(mx, fabsf(acc));
     }
   }
-  __syncthreads();
   const float* Llast = Ls + (C - 1) * G::PK;  // padded rows carry loga = 0: L at row C-1 is Lambda
-  float mx = 0.f;
-  if (tid < DK) mx = fabsf(Llast[tid]);     // |L| is largest at the chunk end (L is monotone)
   if (__syncthreads_or(!(mx < kGdnSafeLog))) {
     // T and P with per-element decay weights e^{L_t - L_i} <= 1
     for (int e = tid; e < C * C; e += 256) {
