@@ -86,6 +86,8 @@ def lib():
         L.kron_delta_gdn2_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp, sz, vp]
         L.kron_delta_gdn2_decode.restype = i
         L.kron_delta_gdn2_decode.argtypes = [vp] * 8 + [i] * 5 + [vp]
+        L.kron_delta_selftest_timeout.restype = i
+        L.kron_delta_selftest_timeout.argtypes = [vp]
         L.kron_delta_profile_enable.restype = None
         L.kron_delta_profile_enable.argtypes = [i]
         L.kron_delta_profile_report.restype = i

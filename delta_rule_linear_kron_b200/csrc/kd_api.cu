@@ -620,6 +620,13 @@ int kron_delta_gdn2_decode(const void* q, const void* k, const void* v, const fl
   return launched(kd::launch_gdn2_decode(a, static_cast<cudaStream_t>(stream)), "gdn2 decode launch");
 }
 
+int kron_delta_selftest_timeout(void* stream) {
+  KD_TRY(check_stream(stream));
+  DeviceInfo di;
+  KD_TRY(device_info(&di));
+  return launched(kd::launch_selftest_timeout(di.err, static_cast<cudaStream_t>(stream)), "self-test launch");
+}
+
 void kron_delta_profile_enable(int on) {
   ProfState& p = prof();
   std::lock_guard<std::mutex> g(p.mu);

@@ -200,6 +200,9 @@ cudaError_t launch_gdn2_decode(const GdnDecodeArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_fwd(const GdnArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_bwd(const GdnArgs& a, cudaStream_t st);
 
+// Failure-reporting self-test (kd_selftest.cu): a bounded wait that runs out.
+cudaError_t launch_selftest_timeout(int* err, cudaStream_t st);
+
 template <typename T>
 inline T* ws_ptr(char* base, size_t off) { return reinterpret_cast<T*>(base + off); }
 template <typename T>

@@ -88,13 +88,13 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
                : "memory");
 }
-// Waits for phase `parity` to complete.  Gives up after kMaxPolls polls (or at
+// Waits for phase `parity` to complete.  Gives up after kPolls polls (or at
 // once if *abort is set), records `code` in *err and raises *abort.
-template <bool kClusterScope>
+template <bool kClusterScope, long kPolls = kMaxPolls>
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, int* err, int code,
                                           volatile int* abort) {
   const uint32_t a = smem_u32(b);
-  for (long i = 0; i < kMaxPolls; ++i) {
+  for (long i = 0; i < kPolls; ++i) {
     uint32_t done;
     if (kClusterScope)
       asm volatile(

@@ -365,6 +365,17 @@ KD_API int kron_delta_gdn2_decode(const void *q, const void *k, const void *v, c
 KD_API int kron_delta_device_status(void *stream);
 
 /*
+ * Self-test of the failure reporting: enqueues one small kernel whose bounded
+ * device-side wait runs out on purpose (a barrier nothing arrives at).  It
+ * faults, traps and hangs nothing; it records a timeout in the device error
+ * word and returns, so the next kron_delta_device_status(stream) reports
+ * KD_ERR_TIMEOUT (and clears it).  Other work in flight on the device at that
+ * moment would see its status reported as failed too: call it on an idle
+ * device.  Returns KD_OK or KD_ERR_CUDA.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_selftest_timeout(void *stream);
+
+/*
  * Per-kernel device timing (tracing aid for tests and benchmarks; off by
  * default).  While enabled, every kernel the library launches is bracketed by
  * two CUDA events recorded on its stream; the events are pooled and reused.
