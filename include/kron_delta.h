@@ -21,6 +21,20 @@
  *   Gated DeltaNet-2 article (aitrends.kr), section "기술 상세": chunk size
  *     C = 64 and forward substitution for the chunk's triangular inverse.
  *
+ * Entry points:
+ *   Kronecker delta rule  kron_delta_fwd, kron_delta_bwd, kron_delta_decode,
+ *                         kron_delta_fwd_phase / _bwd_phase (split at the
+ *                         carried state, for context parallelism),
+ *                         kron_delta_fwd_noalloc
+ *   around the mixer      kron_delta_prologue_fwd / _bwd (L2-norm, gates,
+ *                         log-decay), kron_delta_epilogue_fwd / _bwd
+ *                         (per-head RMSNorm and output gate)
+ *   Gated DeltaNet-2      kron_delta_gdn2_fwd / _bwd / _decode
+ *   support               kron_delta_workspace_size, kron_delta_device_status,
+ *                         kron_delta_selftest_timeout, kron_delta_last_error,
+ *                         kron_delta_version, kron_delta_profile_enable /
+ *                         _report
+ *
  * Conventions shared by every entry point
  *   - All pointers are DEVICE pointers on the current CUDA device unless
  *     stated otherwise.  The caller owns every buffer; the library allocates
