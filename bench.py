@@ -55,18 +55,59 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# Algorithmic work per kernel, per token-head (d_k = d_v = d = 128, C = 64,
-# bf16 activations).  flops: the dense contractions the kernel performs (2
-# per multiply-add).  They add up to 180,224 forward and 409,600 backward
-# flops per token-head, above the method's 163,840 / 360,448 because the
-# output kernel recomputes the masked Gram Q+ K-^T and the post-chain kernel
-# forms the chunk-end term from separate accumulators; the step-level tensor
-# fraction uses the method's 524,288.  bytes: the kernel's own inputs and
-# outputs in HBM.  kind: the unit that executes the contractions.  The exact
-# CUDA-core kernels that recompute flagged chunks (extreme decays) only touch
-# those chunks and have no per-token figure.
+# Algorithmic work, per token-head (d_k = d_v = d = 128, C = 64, bf16
+# activations, fp32 gates).  The method's rows and their dense contractions
+# (2 flops per multiply-add; C x C tiles counted whole, the O(C^3) solve and
+# elementwise work not counted):
+#   a2 Hadamard Gram       2 C x C x d   32,768     a3 query-key decay P   C x C x d   16,384
+#   a5 chain erase read    d x d x C     32,768     a7 chain state update  d x d x C   32,768
+#   a8 output              d x d x C + C x C x d                                       49,152
+#   a9 reverse chain       3 d x d x C                                                 98,304
+#   a10 backward intra     4 d x d x C + 8 C x C x d                                  262,144
+# forward 163,840, backward 360,448, step 524,288.  Bytes: only what the
+# operation must move (no intermediates): forward reads q, k, v (768 B),
+# beta, c (8 B), logf (512 B) and writes O (256 B) = 1,544 B; the backward
+# reads the same plus dO and writes dq, dk, dv, dbeta, dc, dlogf = 2,832 B;
+# step 4,376 B.  Per-head states (S0, S_T, dS0: 64 KB each) are added exactly.
 # ---------------------------------------------------------------------------
-def kernel_work(name, d=128, C=CHUNK):
+STEP_FLOPS = 524288
+STEP_BYTES = 4376
+FWD_FLOPS = 163840
+FWD_BYTES = 1544
+
+
+def method_work(name, d=128, C=CHUNK):
+    """The method rows a kernel of the step executes, their flops per
+    token-head, and the bytes of the method's own inputs it must read and
+    outputs it must write (its share of the step's 4,376 B; workspace
+    intermediates are not counted).  Kernels that only prepare lookahead
+    operands carry no method flops."""
+    act, lf, gate = d * 2, d * 4, 4
+    dd, cd = 2 * d * d, 2 * C * d
+    table = {
+        # a1-a4: decay prefix, Grams, P, the chunk inverse (reads q, k, v, beta, c, logf)
+        "fwd_prep_tc": ("a1-a4", 2 * cd + cd, 3 * act + 2 * gate + lf),
+        # chain operands and the lookahead's cross-chunk matrix (reads k, v, logf)
+        "fwd_cross_tc": ("lookahead operands", 0, 2 * act + lf),
+        # a5-a7 (reads beta; S0 in, S_T out per head)
+        "fwd_chain_tc": ("a5-a7", 2 * dd, gate),
+        # a8 (reads q, k, v, logf; writes O)
+        "fwd_out_tc": ("a8", dd + cd, 3 * act + lf + act),
+        # a10, the part known before the chain (reads k, v, dO, logf)
+        "bwd_pre_tc": ("a10 (pre-chain)", 0, 3 * act + lf),
+        # a9 (reads beta; dS_T in, dS0 out per head)
+        "bwd_chain_tc": ("a9", 3 * dd, gate),
+        # a10 (reads q, k, v, dO, logf, beta, c; writes dq, dk, dv, dbeta, dc, dlogf)
+        "bwd_post_tc": ("a10", 4 * dd + 8 * cd, 4 * act + lf + 2 * gate + 3 * act + 2 * gate + lf),
+    }
+    w = table.get(name)
+    return None if w is None else dict(rows=w[0], flops=w[1], bytes=w[2])
+
+
+# The bytes each kernel of the step actually moves by design, per token-head:
+# its method inputs and outputs plus the workspace intermediates it writes and
+# reads (for the traffic comparison with ncu's DRAM counters).
+def kernel_io_bytes(name, d=128, C=CHUNK):
     act = d * 2                      # one bf16 activation row
     lf = d * 4                       # one fp32 logf row
     tile_f32 = d * d * 4 // C        # one fp32 d x d tile per chunk, per token
@@ -74,35 +115,27 @@ def kernel_work(name, d=128, C=CHUNK):
     cc = C * 4                       # one fp32 C x C matrix per chunk, per token
     ccb = C * 2                      # one bf16 C x C tile per chunk, per token
     table = {
-        # Grams [K+; Q+] K-^T (tf32) and V V^T (bf16); writes A, y and P
-        "fwd_prep_tc": ("tf32", 6 * C * d, 3 * act + lf + 8 + cc + 4 + cc),
-        # K~, K^e, gamma_C, V^T and the cross-chunk matrix H for every chunk (reads chunks n and n-1)
-        # (chunk n-1's k, v, logf were read by the neighbouring CTA and come from L2)
-        "fwd_cross_tc": ("tf32", 4 * C * d, 2 * act + lf + 2 * lf + 8 + cc + act),
-        # X' = S K~^T (tf32) and dS = V^T diag(u) K^e (bf16 hi+lo) over an R=4 cluster: reads K~, K^e,
-        # gamma_C, V^T, A, H, y, beta (the cluster's repeated reads of A, H, V^T are served by L2);
-        # writes u, b0 and the chunk-start states (fp32 and bf16 tiles)
-        "fwd_chain_tc": ("tf32", 4 * d * d, 2 * lf + 8 + act + 2 * cc + 8 + tile_f32 + tile_bf16 + 8),
-        # S0 Q+^T, [Q+; K-] K-^T (tf32), V^T (u o P^T) (bf16); writes O
-        "fwd_out_tc": ("tf32", 2 * d * d + 4 * C * d, 3 * act + lf + 4 + tile_f32 + act),
-        # K+ K-^T (tf32), [V; dO] V^T and [V; dO] dO^T (bf16); writes du_intra, M u and three bf16 tiles
-        "bwd_pre_tc": ("bf16", 6 * C * d, 3 * act + lf + cc + 4 + 2 * ccb + ccb + ccb + 8),
-        # dS K^e^T (tf32), dO^T Q+ and V^T (db0 o K+) (bf16); writes the dS tile and g
-        "bwd_chain_tc": ("bf16", 6 * d * d, 4 * act + lf + 4 + cc + 4 + tile_bf16 + 4),
-        # the five state / intra-chunk accumulators; writes dq, dk, dv, dlogf, dbeta, dc
-        "bwd_post_tc": ("bf16", 16 * d * d, 4 * act + lf + 2 * tile_bf16 + 2 * ccb + ccb + ccb + 20
-                        + 3 * act + lf + 8),
-        # input prologue (not part of the step; timed on its own): reads q~, k~, v~, f~, beta~, c~;
-        # writes q, k, v, logf (fp32), beta, c.  About 20 flops per channel.
-        "prologue_fwd": ("alu", 20 * 4 * d, 4 * act + 8 + 3 * act + lf + 8),
-        # reads q~, k~, v~, f~, dq, dk, dv, dlogf and four gate scalars; writes dq~, dk~, dv~, df~ and two
-        "prologue_bwd": ("alu", 30 * 4 * d, 4 * act + 3 * act + lf + 16 + 4 * act + 8),
-        # output epilogue (timed on its own): reads o, g; writes y.  Backward: reads o, g, dy; writes dO, dg
-        "epilogue_fwd": ("alu", 20 * d, 2 * act + act),
-        "epilogue_bwd": ("alu", 40 * d, 3 * act + 2 * act),
+        "fwd_prep_tc": 3 * act + lf + 8 + cc + 4 + cc,
+        "fwd_cross_tc": 2 * act + lf + 2 * lf + 8 + cc + act,
+        "fwd_chain_tc": 2 * lf + 8 + act + 2 * cc + 8 + tile_f32 + tile_bf16 + 8,
+        "fwd_out_tc": 3 * act + lf + 4 + tile_f32 + act,
+        "bwd_pre_tc": 3 * act + lf + cc + 4 + 2 * ccb + ccb + ccb + 8,
+        "bwd_chain_tc": 4 * act + lf + 4 + cc + 4 + tile_bf16 + 4,
+        "bwd_post_tc": 4 * act + lf + 2 * tile_bf16 + 2 * ccb + ccb + ccb + 20 + 3 * act + lf + 8,
     }
-    w = table.get(name)
-    return None if w is None else dict(kind=w[0], flops=w[1], bytes=w[2])
+    return table.get(name)
+
+
+# The standalone prologue / epilogue passes (timed on their own): bytes per
+# token-head of their own inputs and outputs; they are row-wise and HBM-bound.
+def pass_bytes(name, d=128):
+    act, lf = d * 2, d * 4
+    return {
+        "prologue_fwd": 4 * act + 8 + 3 * act + lf + 8,
+        "prologue_bwd": 4 * act + 3 * act + lf + 16 + 4 * act + 8,
+        "epilogue_fwd": 2 * act + act,
+        "epilogue_bwd": 3 * act + 2 * act,
+    }.get(name)
 
 
 # DRAM bytes (read + write) per launch from one ncu capture of this workload
@@ -132,17 +165,6 @@ def ncu_traffic(name):
     except OSError:
         return None
     return t[0] if digest == t[2] else None
-
-
-def compute_peak_tflops(kind, peaks):
-    """Peak for a kernel timed inside a long step: sustained bf16 (measured);
-    tf32 = that x the nominal tf32/bf16 ratio (1.1 / 2.25 PF dense); alu =
-    148 SMs x 128 FP32 lanes x 2 flops x the max SM clock."""
-    if kind == "bf16":
-        return peaks["bf16_tflops_sustained"]
-    if kind == "tf32":
-        return peaks["bf16_tflops_sustained"] * 1.1 / 2.25
-    return fp32_alu_peak_tflops(peaks["sm_max_mhz"])
 
 
 def fp32_alu_peak_tflops(sm_mhz):
@@ -315,6 +337,7 @@ def main(argv=None):
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-fwd", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-gdn2", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -400,6 +423,49 @@ def main(argv=None):
         per_kernel[name] = dict(launches=int(n), ms=float(ms))
     launches = sum(v["launches"] for v in per_kernel.values())
 
+    # ---- forward only: the long-context workload (B1 H16 T16384, nonzero S0)
+    # and the B4 H16 T2048 workload (S0 = 0), each timed on its own ----------
+    fwd_lines = {}
+    if not args.no_fwd:
+        for wl_i, key in ((3, "fwd_long"), (2, "fwd_B4")):
+            wl = kin.WORKLOADS[wl_i]
+            fi = kin.make_inputs(wl_i, seed=rank_seed(wl.seed, rank), with_dO=False)
+            fd = {n: torch.from_numpy(fi[n]).to(dev, bf if n in ("q", "k", "v") else f32)
+                  for n in ("q", "k", "v", "beta", "c", "logf")}
+            fd["S0"] = None if fi["S0"] is None else torch.from_numpy(fi["S0"]).to(dev, f32)
+            del fi
+            fo = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=bf, device=dev)
+            fST = torch.empty((wl.B, wl.H, wl.dv, wl.dk), dtype=f32, device=dev)
+            fw = torch.empty(kd.workspace_size(kd.KD_WS_FWD, wl.B, wl.H, wl.T, wl.dk, wl.dv), dtype=torch.uint8,
+                             device=dev)
+
+            def fcall():
+                kd.fwd(fd["q"], fd["k"], fd["v"], fd["beta"], fd["c"], fd["logf"], fd["S0"], out=fo,
+                       state_out=fST, save=False, workspace=fw)
+            for _ in range(max(3, args.warmup)):
+                fcall()
+            torch.cuda.synchronize()
+            barrier()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for _ in range(args.steps):
+                fcall()
+            f1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            fms = max_over_ranks(f0.elapsed_time(f1), ws_n, dev) / args.steps
+            fu = wl.B * wl.H * wl.T
+            fbytes = FWD_BYTES * fu + (2 if fd["S0"] is not None else 1) * wl.B * wl.H * wl.dk * wl.dv * 4
+            fl = dict(workload=wl.name, ms=fms, tokens_per_s=job_throughput(ws_n, wl.B * wl.T, 1, fms),
+                      hbm_frac=fbytes / (fms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                      tc_frac=FWD_FLOPS * fu / (fms / 1e3) / 1e12 / peaks["bf16_tflops"])
+            fl["roofline_ms"] = 1e3 * max(fbytes / (peaks["hbm_gbs"] * 1e9),
+                                          FWD_FLOPS * fu / (peaks["bf16_tflops"] * 1e12))
+            fl["frac"] = fl["roofline_ms"] / fms
+            fwd_lines[key] = fl
+            del fd, fo, fST, fw
+        kd.device_status()
+
     # ---- decode: 1000 consecutive in-place steps --------------------------
     decode = None
     if not args.no_decode:
@@ -470,9 +536,9 @@ def main(argv=None):
             torch.cuda.synchronize()
             barrier()
             ms = max_over_ranks(p0.elapsed_time(p1), ws_n, dev) / args.steps
-            w = kernel_work(name)
-            gbs = w["bytes"] * B * H * T / (ms / 1e3) / 1e9
-            times[name] = dict(ms=ms, algorithmic_bytes_per_launch=w["bytes"] * B * H * T, achieved_gbs=gbs,
+            pb = pass_bytes(name)
+            gbs = pb * B * H * T / (ms / 1e3) / 1e9
+            times[name] = dict(ms=ms, algorithmic_bytes_per_launch=pb * B * H * T, achieved_gbs=gbs,
                                hbm_frac=gbs / peaks["hbm_gbs"])
         kd.device_status()
         prologue = dict(times, note="timed alone, not part of the step; each bwd time includes its small "
@@ -622,42 +688,59 @@ def main(argv=None):
 
     value = job_throughput(ws_n, B * T, args.steps, ms_total)
 
-    # ---- roofline of the dominant kernel ---------------------------------
-    roofline = None
-    kernels = {}
+    # ---- rooflines against the method's algorithmic work -----------------
+    # Per kernel: the method rows it executes (flops against the measured
+    # burst bf16 GEMM peak: the timed region is tens of ms) and the method
+    # bytes it must move (against the measured HBM copy bandwidth); the
+    # binding bound is the larger of the two times.  For the step: 524,288
+    # flops and 4,376 B per token-head against ms_per_step.
     units = B * H * T  # token-heads per launch of every per-step kernel
+    tc_peak, hbm_peak = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    kernels = {}
     for name, v in per_kernel.items():
-        w = kernel_work(name)
+        w = method_work(name)
         if w is None or v["launches"] == 0:
             continue
         avg_s = v["ms"] / v["launches"] / 1e3
-        pk = compute_peak_tflops(w["kind"], peaks)
-        t_c = w["flops"] * units / (pk * 1e12)
-        t_m = w["bytes"] * units / (peaks["hbm_gbs"] * 1e9)
+        t_c = w["flops"] * units / (tc_peak * 1e12)
+        t_m = w["bytes"] * units / (hbm_peak * 1e9)
+        io = kernel_io_bytes(name) * units
+        tr = ncu_traffic(name)
+        k = dict(rows=w["rows"], avg_launch_ms=avg_s * 1e3, algorithmic_flops_per_launch=w["flops"] * units,
+                 algorithmic_bytes_per_launch=w["bytes"] * units, design_io_bytes_per_launch=io, traffic=tr,
+                 traffic_ratio=None if tr is None else tr / (w["bytes"] * units))
         if t_c >= t_m:
             ach = w["flops"] * units / avg_s / 1e12
-            kernels[name] = dict(bound="alu" if w["kind"] == "alu" else "tensor", kind=w["kind"], achieved=ach,
-                                 peak=pk, unit="TFLOP/s", frac=ach / pk)
+            k.update(bound="tensor", achieved=ach, peak=tc_peak, unit="TFLOP/s", frac=ach / tc_peak)
         else:
             ach = w["bytes"] * units / avg_s / 1e9
-            kernels[name] = dict(bound="hbm", kind=w["kind"], achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
-                                 frac=ach / peaks["hbm_gbs"])
-        kernels[name].update(avg_launch_ms=avg_s * 1e3, algorithmic_flops_per_launch=w["flops"] * units,
-                             algorithmic_bytes_per_launch=w["bytes"] * units, traffic=ncu_traffic(name))
+            k.update(bound="hbm", achieved=ach, peak=hbm_peak, unit="GB/s", frac=ach / hbm_peak)
+        kernels[name] = k
+    roofline = None
     if kernels:
         top = max(kernels, key=lambda n: per_kernel[n]["ms"])
         k = kernels[top]
-        roofline = dict(kernel=top, bound=k["bound"], achieved=k["achieved"], peak=k["peak"], unit=k["unit"],
-                        frac=k["frac"], traffic=k["traffic"], avg_launch_ms=k["avg_launch_ms"],
+        roofline = dict(kernel=top, rows=k["rows"], bound=k["bound"], achieved=k["achieved"], peak=k["peak"],
+                        unit=k["unit"], frac=k["frac"], traffic=k["traffic"], avg_launch_ms=k["avg_launch_ms"],
                         algorithmic_flops_per_launch=k["algorithmic_flops_per_launch"],
                         algorithmic_bytes_per_launch=k["algorithmic_bytes_per_launch"],
                         peak_note=("measured HBM copy bandwidth" if k["bound"] == "hbm" else
-                                   "measured sustained bf16 GEMM" + (" x 1.1/2.25 (tf32)" if k["kind"] == "tf32" else "")
-                                   if k["bound"] == "tensor" else "148 SMs x 128 FP32 lanes x 2 x max SM clock")
-                        + " (" + peaks["source"] + ")",
+                                   "measured burst bf16 GEMM") + " (" + peaks["source"] + ")",
                         sm_mhz_median=clocks["sm_mhz"])
-    step_flops = 524288 * B * H * T
-    tc_frac = step_flops / (ms_total / args.steps / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
+    step_s = ms_total / args.steps / 1e3
+    st_bytes = STEP_BYTES * units + 3 * B * H * dk * dv * 4
+    st_flops = STEP_FLOPS * units
+    traffic_all = [kernels[n]["traffic"] for n in kernels]
+    roofline_step = dict(
+        flops_per_token_head=STEP_FLOPS, bytes_per_token_head=STEP_BYTES, ms=step_s * 1e3,
+        achieved_gbs=st_bytes / step_s / 1e9, hbm_frac=st_bytes / step_s / 1e9 / hbm_peak,
+        achieved_tflops=st_flops / step_s / 1e12, tc_frac=st_flops / step_s / 1e12 / tc_peak,
+        roofline_ms=1e3 * max(st_bytes / (hbm_peak * 1e9), st_flops / (tc_peak * 1e12)),
+        bound="hbm" if st_bytes / hbm_peak / 1e9 >= st_flops / tc_peak / 1e12 else "tensor",
+        traffic_bytes=(sum(traffic_all) if traffic_all and None not in traffic_all else None))
+    roofline_step["frac"] = roofline_step["roofline_ms"] / (step_s * 1e3)
+    roofline_step["traffic_ratio"] = (None if roofline_step["traffic_bytes"] is None
+                                      else roofline_step["traffic_bytes"] / st_bytes)
 
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
@@ -670,13 +753,22 @@ def main(argv=None):
                 "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "T": T, "dk": dk, "dv": dv, "chunk": CHUNK,
                            "global_batch": B * ws_n, "seq_len": T, "parallelism": f"dp{ws_n}",
                            "step": "fwd(save) + bwd", "l2": "inputs larger than L2 (no flush)"},
-                "tc_frac_of_bf16_peak": tc_frac,
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "prologue_epilogue": prologue, "gdn2": gdn2,
-                "gpu_launches": launches, "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
-                "kernel_rooflines": kernels,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches,
                 "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                            "reasons": clocks["reasons"], "samples": clocks["samples"]},
-                "peaks": peaks}
+                "peaks": peaks,
+                "per_kernel_ms": {k: v["ms"] / max(1, args.steps) for k, v in per_kernel.items()},
+                "kernel_rooflines": kernels,
+                "prologue_epilogue": prologue,
+                "gdn2": gdn2,
+                # compact summaries last (a truncated tail of the line keeps them)
+                "roofline_step": roofline_step,
+                "fwd_long": fwd_lines.get("fwd_long"), "fwd_B4": fwd_lines.get("fwd_B4"),
+                "gdn2_step": None if gdn2 is None else dict(ms=gdn2["ms_per_step"], tokens_per_s=gdn2["value"],
+                                                            decode_gbs=gdn2["decode"]["value"],
+                                                            decode_hbm_frac=gdn2["decode"]["hbm_frac"]),
+                "decode": decode}
         print(json.dumps(line), flush=True)
     if ws_n > 1:
         dist.destroy_process_group()

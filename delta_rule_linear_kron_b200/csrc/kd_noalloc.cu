@@ -24,8 +24,12 @@
 //     them.
 //   * The first call on each device looks up the array's device address with
 //     cudaGetSymbolAddress (with that device current) and caches it; make that
-//     first call before any stream capture begins.
+//     first call before any stream capture begins.  The cache is keyed on the
+//     current context's unique ID: if the device's primary context was reset
+//     (cudaDeviceReset) and recreated, the module is reloaded at a new
+//     address, and the next call looks the address up again.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <cstdio>
@@ -43,20 +47,48 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context ID the address belongs to
 
-// The device address of the scratch array on the current device (looked up
-// once per device; the array's name is only a host-side stand-in).
+// Unique ID of the calling thread's current context (0 if it cannot be
+// read), through the driver entry points, so no link-time libcuda.
+unsigned long long current_context_id() {
+  static std::once_flag once;
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// The device address of the scratch array on the current device (the
+// array's name is only a host-side stand-in).  Looked up once per device and
+// context; looked up again when the context has changed.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> g(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // also makes the primary context current
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

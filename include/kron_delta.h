@@ -151,6 +151,12 @@ KD_API int kron_delta_fwd(const void *q, const void *k, const void *v,
  *   workspace, ws_bytes : scratch of at least
  *         kron_delta_workspace_size(KD_WS_BWD, ...).
  * S0 is the same initial state given to the forward (NULL = zero).
+ * There is no recompute mode: the backward always reads the forward's saved
+ * chunk quantities (fwd_ws) and fails with KD_ERR_WORKSPACE without them.
+ * Recomputing them would rerun the forward's sequential chunk chain, which is
+ * a latency-bound critical path as long as the backward's own chain, while
+ * reading them back costs one pass over the saved bytes.  A caller that does
+ * not keep the forward's workspace reruns kron_delta_fwd with save = 1 first.
  * Errors as for kron_delta_fwd.  Asynchronous on `stream`.
  */
 KD_API int kron_delta_bwd(const void *q, const void *k, const void *v,

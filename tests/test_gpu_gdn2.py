@@ -73,6 +73,15 @@ def check(inp, dtype, dST=None, heads=None):
     errs["dS0"] = rel(host(g["dS0"])[:, sl], gr["dS0"])
     bad = {n: e for n, e in errs.items() if e > (tf if n in ("O", "ST") else tg)}
     assert not bad, errs
+    if heads is not None:
+        # each checked head on its own, at the same tolerances
+        for j, hh in enumerate(heads):
+            one = {"O": rel(host(out)[:, :, hh], O_ref[:, :, j]), "ST": rel(host(ST)[:, hh], ST_ref[:, j]),
+                   "dS0": rel(host(g["dS0"])[:, hh], gr["dS0"][:, j])}
+            for n in ("dq", "dk", "dv", "db", "dw", "dloga"):
+                one[n] = rel(host(g[n])[:, :, hh], gr[n][:, :, j])
+            bad = {n: e for n, e in one.items() if e > (tf if n in ("O", "ST") else tg)}
+            assert not bad, (hh, one)
     return errs
 
 

@@ -31,6 +31,29 @@ def rel(x, ref):
     return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
 
 
+def rel_units(x, ref, axes):
+    """Largest relative L2 error over the units left after reducing `axes`
+    (for example one value per (b, h) of a [B, T, H, d] tensor)."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    num = np.sqrt(np.sum((x - ref) ** 2, axis=axes))
+    den = np.maximum(np.sqrt(np.sum(ref ** 2, axis=axes)), 1e-300)
+    return float(np.max(num / den))
+
+
+# per-(b,h) reduction axes of each tensor: [B,T,H,d], [B,T,H] and [B,H,dv,dk]
+UNIT_AXES = {"O": (1, 3), "ST": (2, 3), "dq": (1, 3), "dk": (1, 3), "dv": (1, 3), "dbeta": (1,), "dc": (1,),
+             "dlogf": (1, 3), "dS0": (2, 3)}
+
+
+def rel_chunks(x, ref, C=64):
+    """Largest relative L2 error over (b, chunk, h) blocks of a [B, T, H, d]
+    tensor whose T is a multiple of C."""
+    B, T, H, d = np.shape(ref)
+    sh = (B, T // C, C, H, d)
+    return rel_units(np.reshape(x, sh), np.reshape(ref, sh), (2, 4))
+
+
 def dev(inp, dtype):
     tdt = torch.float32 if dtype == "f32" else torch.bfloat16
     out = {}
@@ -54,11 +77,18 @@ def run_fwd(inp, dtype, save=False):
     return d, out, ST, ws
 
 
-def check_fwd(inp, dtype, tol, oracle):
+def check_fwd(inp, dtype, tol, oracle, per_unit=False):
+    """Whole-tensor relative L2 errors of O and S_T; with per_unit, also the
+    largest error over single (b, h) heads and over single 64-token chunks of O,
+    at the same tolerance (so one wrong head or chunk cannot hide in the norm)."""
     d, out, ST, _ = run_fwd(inp, dtype)
     O_ref, ST_ref = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"])
-    eo, es = rel(host(out), O_ref), rel(host(ST), ST_ref)
+    o, s = host(out), host(ST)
+    eo, es = rel(o, O_ref), rel(s, ST_ref)
     assert eo <= tol and es <= tol, (eo, es)
+    if per_unit:
+        uo, us, co = rel_units(o, O_ref, UNIT_AXES["O"]), rel_units(s, ST_ref, UNIT_AXES["ST"]), rel_chunks(o, O_ref)
+        assert uo <= tol and us <= tol and co <= tol, dict(O_head=uo, ST_head=us, O_chunk=co)
     return eo, es
 
 
@@ -90,8 +120,12 @@ def test_decode_full_batch_first_steps(oracle):
         args += [torch.from_numpy(d[n][t]).float().cuda() for n in ("beta", "c", "logf")]
         o = kd.decode(*args, S)
         Sref, oref = oracle.decode(d["q"][t], d["k"][t], d["v"][t], d["beta"][t], d["c"][t], d["logf"][t], Sref)
-        assert rel(host(o), oref) <= TOL_BF16
-        assert rel(host(S), Sref) <= TOL_BF16
+        oh, Sh = host(o), host(S)
+        assert rel(oh, oref) <= TOL_BF16
+        assert rel(Sh, Sref) <= TOL_BF16
+        # every single head ([B, H, d] outputs, [B, H, dv, dk] states)
+        assert rel_units(oh, oref, (2,)) <= TOL_BF16
+        assert rel_units(Sh, Sref, (2, 3)) <= TOL_BF16
 
 
 def test_decode_1000_steps_sampled_heads(oracle):
@@ -114,6 +148,8 @@ def test_decode_1000_steps_sampled_heads(oracle):
         Sref, oref = oracle.decode(q[t][None], k[t][None], v[t][None], beta[t][None], c[t][None], logf[t][None], Sref)
     assert rel(host(S)[bi, hi], Sref[0]) <= TOL_BF16
     assert rel(host(o)[bi, hi], oref[0]) <= TOL_BF16
+    assert rel_units(host(S)[bi, hi], Sref[0], (1, 2)) <= TOL_BF16
+    assert rel_units(host(o)[bi, hi], oref[0], (1,)) <= TOL_BF16
 
 
 # ----------------------------------------------------------------------------- forward
@@ -137,11 +173,11 @@ def test_fwd_rectangular_state(oracle):
 
 
 def test_fwd_workload_B4_T2048(oracle):
-    check_fwd(kin.make_inputs(2, with_dO=False), "bf16", TOL_BF16, oracle)
+    check_fwd(kin.make_inputs(2, with_dO=False), "bf16", TOL_BF16, oracle, per_unit=True)
 
 
 def test_fwd_workload_T16384_nonzero_state(oracle):
-    check_fwd(kin.make_inputs(3, with_dO=False), "bf16", TOL_BF16, oracle)
+    check_fwd(kin.make_inputs(3, with_dO=False), "bf16", TOL_BF16, oracle, per_unit=True)
 
 
 @pytest.mark.parametrize("beta_val", [0.0, 1.0])
@@ -194,7 +230,10 @@ def test_fwd_deterministic():
 GRADS = ("dq", "dk", "dv", "dbeta", "dc", "dlogf", "dS0")
 
 
-def check_bwd(inp, dtype, tol_fwd, tol_grad, oracle, dST=None):
+def check_bwd(inp, dtype, tol_fwd, tol_grad, oracle, dST=None, per_unit=False):
+    """Forward and every gradient against the oracle (whole-tensor relative L2);
+    with per_unit, also per (b, h) head for every tensor and per 64-token chunk
+    for O, dq, dk and dv, at the same tolerances."""
     d, out, ST, ws = run_fwd(inp, dtype, save=True)
     dSTd = None if dST is None else torch.from_numpy(dST).float().cuda()
     g = kd.bwd(d["q"], d["k"], d["v"], d["beta"], d["c"], d["logf"], d["S0"], d["dO"], dSTd, fwd_workspace=ws)
@@ -203,8 +242,18 @@ def check_bwd(inp, dtype, tol_fwd, tol_grad, oracle, dST=None):
     O_ref, ST_ref = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"])
     assert rel(host(out), O_ref) <= tol_fwd and rel(host(ST), ST_ref) <= tol_fwd
     gr = oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], inp["dO"], dST)
-    errs = {n: rel(host(g[n]), gr[n]) for n in GRADS}
+    gh = {n: host(g[n]) for n in GRADS}
+    errs = {n: rel(gh[n], gr[n]) for n in GRADS}
     assert all(e <= tol_grad for e in errs.values()), errs
+    if per_unit:
+        o = host(out)
+        fw = dict(O_head=rel_units(o, O_ref, UNIT_AXES["O"]), ST_head=rel_units(host(ST), ST_ref, UNIT_AXES["ST"]),
+                  O_chunk=rel_chunks(o, O_ref))
+        assert all(e <= tol_fwd for e in fw.values()), fw
+        heads = {n: rel_units(gh[n], gr[n], UNIT_AXES[n]) for n in GRADS}
+        assert all(e <= tol_grad for e in heads.values()), heads
+        chunks = {n: rel_chunks(gh[n], gr[n]) for n in ("dq", "dk", "dv")}
+        assert all(e <= tol_grad for e in chunks.values()), chunks
     return errs
 
 
@@ -255,7 +304,7 @@ def test_bwd_bf16_decay_bands(oracle):
 
 def test_fwdbwd_workload_T16384_state_tracking(oracle):
     """Forward+backward workload: B=1, H=16, T=16384, d=128, beta in (0,2)."""
-    check_bwd(kin.make_inputs(4), "bf16", TOL_BF16, TOL_GRAD_BF16, oracle)
+    check_bwd(kin.make_inputs(4), "bf16", TOL_BF16, TOL_GRAD_BF16, oracle, per_unit=True)
 
 
 def test_autograd_function_matches_bwd():
