@@ -97,6 +97,8 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
     L->PU = take(chunks * C * C * 2);
     L->EK = take(chunks * C * C * 2);
     L->Mu = take(chunks * C * 4);
+    L->Kp = take((size_t)B * T * H * dk * 4);
+    L->QpT = take(chunks * (size_t)dk * C * 2);
   }
   L->bwd_bytes = off;
   return KD_OK;

@@ -97,18 +97,21 @@ struct PreCfg {
   static constexpr uint32_t PS = 147456;     // P fp32 [64][64]
   static constexpr uint32_t US = 163840;     // u [64]
   static constexpr uint32_t XCH = US + 256;  // prefix exchange [128]
-  static constexpr uint32_t BYTES = XCH + 512 + 1024;
-  static constexpr uint32_t LOAD_BYTES = 32768 + 16384 + 32768 + 16384 + 256;
+  static constexpr uint32_t QR = 165888;     // q bf16 [64][128] (TMA)
+  static constexpr uint32_t QT = 182272;     // Q+^T bf16 [j][t], 128 rows x 128 B, 128-byte swizzle (staging)
+  static constexpr uint32_t BYTES = QT + 16384 + 1024;
+  static constexpr uint32_t LOAD_BYTES = 32768 + 16384 + 32768 + 16384 + 256 + 16384;
   // output staging in the KPM area once the MMAs are done
   static constexpr uint32_t OT1 = 0, OPU = 16384, OEK = 24576;
 };
 
 __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf, int H, int NC,
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf,
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp, int H, int NC,
     const float* __restrict__ wP, const float* __restrict__ wu, float* __restrict__ wdu, float* __restrict__ wMu,
     __nv_bfloat16* __restrict__ wT1, __nv_bfloat16* __restrict__ wPU, __nv_bfloat16* __restrict__ wEK,
-    int* __restrict__ err) {
+    __nv_bfloat16* __restrict__ wQpT, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
     tc::tma_load_4d(sm + PreCfg::VD + 24576, &tm_do, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PreCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
     tc::bulk_g2s(sm + PreCfg::PS, wP + ch * C * C, 16384u, &ld_bar);
     tc::bulk_g2s(sm + PreCfg::US, wu + ch * C, 256u, &ld_bar);
   }
@@ -142,21 +146,26 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
 
-  // K+ and K- (fp32, read as tf32); thread (j, half) covers 32 positions.
-  // Chunks with extreme decays may overflow here: their E_K and M u are never
-  // used (the post-chain kernel hands such chunks to the exact path).
+  // K+ and K- (fp32, read as tf32), and Q+ (bf16, transposed for the reverse
+  // chain's dO^T Q+ MMA); thread (j, half) covers 32 positions.  K+ and Q+
+  // carry decays e^L <= 1 and are always finite; chunks with extreme decays
+  // may overflow K- here: their E_K and M u are never used (the post-chain
+  // kernel hands such chunks to the exact path).
   {
     const int j = tid & 127, half = tid >> 7;
     float Lr[32];
     split_prefix(reinterpret_cast<const float*>(sm + PreCfg::LG), j, half,
                  reinterpret_cast<float*>(sm + PreCfg::XCH), Lr);
     const unsigned char* kr = sm + PreCfg::KR;
+    const unsigned char* qr = sm + PreCfg::QR;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int t = 32 * half + i;
       const float kk = bf(kr + (t * D + j) * 2);
-      *reinterpret_cast<float*>(sm + PreCfg::KPM + tc::sw128_off(t, j, 128, 4)) = kk * expf(Lr[i]);
+      const float gm = expf(Lr[i]);
+      *reinterpret_cast<float*>(sm + PreCfg::KPM + tc::sw128_off(t, j, 128, 4)) = kk * gm;
       *reinterpret_cast<float*>(sm + PreCfg::KPM + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(-Lr[i]);
+      put_bf(sm + PreCfg::QT + tc::sw128_off(j, t, 128, 2), bf(qr + (t * D + j) * 2) * gm);
     }
   }
   tc::fence_proxy_async();
@@ -164,6 +173,11 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
   __syncthreads();
   tc::tc_after_sync();
   if (tid == 0) {
+    // K+ (rows 0-63 of each 32-channel block) and the Q+^T tile out for the reverse chain
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) tc::tma_store_4d(&tm_kp, sm + PreCfg::KPM + kb * 16384, 32 * kb, h, t0, b);
+    tc::bulk_s2g(wQpT + ch * (D * C), sm + PreCfg::QT, 16384u);
+    tc::bulk_commit();
     const uint32_t IDT = tc::idesc(128, 64, 2), IDB = tc::idesc(128, 64, 1);
     // cols 0-63: [K+; K-] K-^T (rows 0-63: G_K)
 #pragma unroll
@@ -186,6 +200,8 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
   }
   tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
+  if (tid == 0) tc::bulk_wait_read();  // the K+ stores have read the area the staging below reuses
+  __syncthreads();
 
   const float* us = reinterpret_cast<const float*>(sm + PreCfg::US);
   const float* Ps = reinterpret_cast<const float*>(sm + PreCfg::PS);
@@ -545,19 +561,21 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
 
 cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st) {
   const Layout& L = a.L;
-  CUtensorMap tm_v, tm_do, tm_k, tm_logf;
+  CUtensorMap tm_v, tm_do, tm_k, tm_logf, tm_q, tm_kp;
   if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_do, a.dO, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
-      !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false))
+      !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_kp, ws_ptr<float>(a.ws, L.Kp), 4, L.B, L.T, L.H, D, 32, true))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(bwd_pre_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PreCfg::BYTES);
   if (e != cudaSuccess) return e;
   prof_begin(st, "bwd_pre_tc");
   bwd_pre_tc<<<(unsigned)L.chunks, 256, PreCfg::BYTES, st>>>(
-      tm_v, tm_do, tm_k, tm_logf, L.H, L.NC, ws_ptr<float>(a.fws, L.P), ws_ptr<float>(a.fws, L.u),
+      tm_v, tm_do, tm_k, tm_logf, tm_q, tm_kp, L.H, L.NC, ws_ptr<float>(a.fws, L.P), ws_ptr<float>(a.fws, L.u),
       ws_ptr<float>(a.ws, L.du), ws_ptr<float>(a.ws, L.Mu), ws_ptr<__nv_bfloat16>(a.ws, L.T1),
-      ws_ptr<__nv_bfloat16>(a.ws, L.PU), ws_ptr<__nv_bfloat16>(a.ws, L.EK), err);
+      ws_ptr<__nv_bfloat16>(a.ws, L.PU), ws_ptr<__nv_bfloat16>(a.ws, L.EK), ws_ptr<__nv_bfloat16>(a.ws, L.QpT), err);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -39,455 +39,6 @@ namespace {
 constexpr int C = kChunk;
 constexpr int D = 128;
 
-template <int R>
-struct ChainCfg {
-  static constexpr int NJ = D / R;                    // key channels per CTA
-  static constexpr int KBJ = (R == 8) ? 2 : 0;        // K steps of the K~ block that precede this CTA's channels (odd R=8 ranks)
-  // tensor memory columns: X' (64), state slice, update
-  static constexpr int D1_COL = 0, S_COL = 64, D2_COL = 64 + NJ;
-  static constexpr uint32_t TMEM_COLS = (64 + 2 * NJ) <= 128 ? 128u : 256u;
-  static constexpr uint32_t up1k(uint32_t x) { return (x + 1023u) / 1024u * 1024u; }
-  // chunk slot (ring of three), all written by TMA / bulk copies
-  static constexpr uint32_t SL_V = 0;                          // V^T bf16 [r][t], K-major, 128-byte swizzle (16 KB)
-  static constexpr uint32_t SL_B1 = 16384;                     // K~, the 32-channel block holding this CTA's channels:
-                                                               //   tf32 [t][32], 128-byte swizzle (8 KB)
-  static constexpr uint32_t SL_KE = SL_B1 + 8192;              // K^e slice fp32 [64][NJ]
-  static constexpr uint32_t SL_GC = SL_KE + 64 * NJ * 4;       // gamma_C slice [NJ]
-  static constexpr uint32_t SL_Y = SL_GC + 128;                // y [64]
-  static constexpr uint32_t SL_SZ = up1k(SL_Y + 256);
-  static constexpr uint32_t LOAD_BYTES = 16384 + 8192 + 64 * NJ * 4 + NJ * 4 + 256;
-  // per-chunk matrices of the u recursion (ring of two): A, H
-  static constexpr uint32_t AUX = 3 * SL_SZ;
-  static constexpr uint32_t AUX_SZ = 32768;
-  static constexpr uint32_t B2 = AUX + 2 * AUX_SZ;             // diag(u) K^e slice, bf16 hi / lo, NJ rows x 128 B each
-  static constexpr uint32_t SM = B2 + 2 * NJ * 128;            // small arrays (floats)
-  static constexpr uint32_t SM_BS = SM;                        // beta [3][64]
-  static constexpr uint32_t SM_W = SM_BS + 3 * 64 * 4;         // beta o b0 [64]
-  static constexpr uint32_t SM_U = SM_W + 64 * 4;              // u [64] (previous chunk's until replaced)
-  static constexpr uint32_t SM_UP = SM_U + 64 * 4;             // partial sums [2][64]
-  static constexpr uint32_t SM_MINE = SM_UP + 2 * 64 * 4;      // own c partial [64]
-  static constexpr uint32_t SM_XRED = SM_MINE + 64 * 4;        // per-warp partials [4][64]
-  static constexpr uint32_t SM_RECV = SM_XRED + 4 * 64 * 4;    // [2][R][64]
-  static constexpr uint32_t SM_END = SM_RECV + 2 * R * 64 * 4;
-  static constexpr uint32_t BYTES = SM_END + 1024;             // + alignment slack
-};
-
-// Writes 16 state values (row r, columns j..j+15) of one chunk into the bf16
-// tile the backward's MMAs read: [r][j] (rows r, K = j), 128-byte-swizzled
-// K-major, 32 KB.  The backward also reads it transposed, as an MN-major operand.
-__device__ __forceinline__ void save_bf16_tile(__nv_bfloat16* rj, size_t ch, int r, int j, const float (&x)[16]) {
-  unsigned char* a = reinterpret_cast<unsigned char*>(rj + ch * D * D);
-#pragma unroll
-  for (int h8 = 0; h8 < 2; ++h8) {
-    __align__(16) __nv_bfloat16 v8[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v8[i] = __float2bfloat16_rn(x[8 * h8 + i]);
-    *reinterpret_cast<uint4*>(a + tc::sw128_off(r, j + 8 * h8, 128, 2)) = *reinterpret_cast<const uint4*>(v8);
-  }
-}
-
-// named barriers: 1 = the 4 chain warps, 2 = the 4 producer warps;
-// 3 = chain -> issuer "update operand ready", 4 = chain -> issuer "state updated"
-// (the chain warps arrive, the issuer warp waits: 160 threads)
-__device__ __forceinline__ void bar_chain() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ void bar_prod() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
-__device__ __forceinline__ void bar_arrive_issuer(int id) { asm volatile("bar.arrive %0, 160;" ::"r"(id) : "memory"); }
-__device__ __forceinline__ void bar_wait_chain(int id) { asm volatile("bar.sync %0, 160;" ::"r"(id) : "memory"); }
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(b)) : "memory");
-}
-
-// The chain with a one-chunk lookahead.  With c_{n+1} = rowdot(V_{n+1}, S_n K~_{n+1}^T),
-// K~_{n+1} = K+_{n+1} diag(gamma_C of chunk n), and the cross-chunk matrix
-// H_{n+1} = (V_{n+1} V_n^T) o (K+_{n+1} K^e_n^T) (fwd_cross_tc):
-//   b0_{n+1} = rowdot(V_{n+1}, S_{n+1} K+_{n+1}^T) = c_{n+1} + H_{n+1} u_n,
-// so c_{n+1} (an MMA on the state, a column dot and the cluster all-reduce)
-// is formed while u_n and the update of chunk n proceed; only two 64 x 64
-// matrix-vector products separate u_n from u_{n+1}.
-//
-// Warp roles (288 threads):
-//   warps 0-3  chain: u, the update operand, the column dots, the cluster
-//              all-reduce, the state update; thread r owns tensor-memory lane r.
-//   warps 4-7  producer: TMA / bulk loads of each chunk's operands (built by
-//              fwd_cross_tc) into a ring of three slots, A and H into a ring
-//              of two, and the save of each chunk-start state slice.
-//   warp 8     issuer: one thread issues every tcgen05 MMA.
-// Hand-offs: mbarriers raw_full (a slot's loads landed), slot_free (chain done
-// with a slot), aux_full / aux_free (A, H), s_ready (state of chunk n in
-// tensor memory), s_saved (producer has read it), mma1 / mma2 (MMA done);
-// named barriers 3 and 4 (chain -> issuer).
-template <int R>
-__global__ void __launch_bounds__(288, 1) fwd_chain_tc(
-    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
-    const __grid_constant__ CUtensorMap tm_ke, const float* __restrict__ beta, const float* __restrict__ S0,
-    float* __restrict__ ST, int H, int T, int NC, const float* __restrict__ wy, const float* __restrict__ wA,
-    const float* __restrict__ wHx, const float* __restrict__ wGC, const __nv_bfloat16* __restrict__ wVt,
-    float* __restrict__ wS0blob,
-    float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, int* __restrict__ err) {
-  using Cf = ChainCfg<R>;
-  constexpr int NJ = Cf::NJ;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ uint64_t raw_full[3], slot_free[3], aux_full[2], aux_free[2], s_ready, s_saved, x_bar[2], mma1_bar,
-      mma2_bar;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = tc::cluster_rank();
-  const int unit = blockIdx.x / R;  // (b, h)
-  const int b = unit / H, h = unit % H;
-  const int j0 = static_cast<int>(rank) * NJ;
-  const int jb = j0 & ~31;  // first channel of the 32-channel K~ block
-
-  float* bs = reinterpret_cast<float*>(sm + Cf::SM_BS);
-  float* ws = reinterpret_cast<float*>(sm + Cf::SM_W);
-  float* us = reinterpret_cast<float*>(sm + Cf::SM_U);
-  float* up = reinterpret_cast<float*>(sm + Cf::SM_UP);
-  float* mine = reinterpret_cast<float*>(sm + Cf::SM_MINE);
-  float* xred = reinterpret_cast<float*>(sm + Cf::SM_XRED);
-  float* recv = reinterpret_cast<float*>(sm + Cf::SM_RECV);
-  auto slot = [&](int m) { return sm + (m % 3) * Cf::SL_SZ; };
-
-  if (tid == 0) {
-    for (int i = 0; i < 3; ++i) {
-      tc::mbar_init(&raw_full[i], 1);
-      tc::mbar_init(&slot_free[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&aux_full[i], 1);
-      tc::mbar_init(&aux_free[i], 1);
-      tc::mbar_init(&x_bar[i], 1);
-    }
-    tc::mbar_init(&s_ready, 1);
-    tc::mbar_init(&s_saved, 1);
-    tc::mbar_init(&mma1_bar, 1);
-    tc::mbar_init(&mma2_bar, 1);
-    tc::mbar_init_fence();
-    abort_flag = 0;
-  }
-  if (warp == 0) tc::tmem_alloc(&tmem_slot, Cf::TMEM_COLS);
-  tc::tc_before_sync();
-  __syncthreads();
-  tc::cluster_sync();  // peers' barriers are initialised before any remote arrive
-  tc::tc_after_sync();
-  const uint32_t tmem = tmem_slot;
-  const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);  // lanes 32*(warp%4) ..
-
-  if (warp == 8) {
-    // ============================== issuer warp ==============================
-    const uint32_t ID1 = tc::idesc(128, 64, 2);
-    const uint32_t ID2 = tc::idesc(128, NJ, 1);  // bf16, both K-major
-    // X' = S K~_m^T  (M = 128 rows r, N = 64 positions, K = NJ; A = the state in tensor memory)
-    auto issue_x = [&](int m) {
-      tc::mbar_wait<false>(&raw_full[m % 3], (uint32_t)((m / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
-      tc::tc_after_sync();
-      if (lane == 0) {
-        const unsigned char* st = slot(m);
-#pragma unroll
-        for (int ks = 0; ks < NJ / 8; ++ks) {
-          const uint64_t bd = tc::desc_sw128(tc::smem_u32(st + Cf::SL_B1 + (Cf::KBJ * (rank & 1) + ks) * 32));
-          tc::mma_tf32_ts(tmem + Cf::D1_COL, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&mma1_bar);
-      }
-      __syncwarp();
-    };
-    bar_wait_chain(4);  // S_0 in tensor memory
-    tc::tc_after_sync();
-    issue_x(0);
-    for (int n = 0; n < NC; ++n) {
-      if (n + 1 < NC) {
-        if (n >= 1) {
-          bar_wait_chain(4);  // S_n in tensor memory (update of chunk n-1 done)
-          tc::tc_after_sync();
-        }
-        issue_x(n + 1);
-      }
-      bar_wait_chain(3);  // update operand of chunk n built
-      tc::tc_after_sync();
-      if (lane == 0) {
-        const unsigned char* st = slot(n);
-        // dS = V_n^T (B2hi + B2lo)^T  (M = 128 rows r, N = NJ, K = 64 positions)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = tc::desc_sw128(tc::smem_u32(st + Cf::SL_V + ks * 32));
-          tc::mma_bf16_ss(tmem + Cf::D2_COL, ad, tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + ks * 32)), ID2,
-                          ks > 0 ? 1u : 0u);
-          tc::mma_bf16_ss(tmem + Cf::D2_COL, ad, tc::desc_sw128(tc::smem_u32(sm + Cf::B2 + NJ * 128 + ks * 32)),
-                          ID2, 1u);
-        }
-        tc::mma_commit(&mma2_bar);
-      }
-      __syncwarp();
-    }
-  } else if (warp >= 4) {
-    // =========================== producer warps ===========================
-    const int p = tid - 128;
-    // the operands of chunk m into its slot (chunk m - 3 must be done)
-    auto prepare = [&](int m) {
-      unsigned char* st = slot(m);
-      const int si = m % 3;
-      if (m >= 3)
-        tc::mbar_wait<false>(&slot_free[si], (uint32_t)((m / 3 - 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
-      if (p == 0) {
-        uint64_t* bar = &raw_full[si];
-        const size_t ch = (size_t)unit * NC + m;
-        tc::fence_proxy_async();
-        tc::mbar_expect_tx(bar, Cf::LOAD_BYTES);
-        tc::bulk_g2s(st + Cf::SL_V, wVt + ch * (D * C), 16384u, bar);
-        tc::tma_load_4d(st + Cf::SL_B1, &tm_kt, jb, h, m * C, b, bar);
-        tc::tma_load_4d(st + Cf::SL_KE, &tm_ke, j0, h, m * C, b, bar);
-        tc::bulk_g2s(st + Cf::SL_GC, wGC + ch * D + j0, NJ * 4u, bar);
-        tc::bulk_g2s(st + Cf::SL_Y, wy + ch * C, 256u, bar);
-      }
-      if (p < C) bs[si * 64 + p] = (m * C + p < T) ? beta[((size_t)b * T + m * C + p) * H + h] : 0.f;
-    };
-    // A and H of chunk m (chunk m - 2 must have consumed its buffer)
-    auto aux = [&](int m) {
-      if (p != 0) return;
-      const int ai = m & 1;
-      if (m >= 2)
-        tc::mbar_wait<false>(&aux_free[ai], (uint32_t)(((m - 2) >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
-      unsigned char* ax = sm + Cf::AUX + ai * Cf::AUX_SZ;
-      const size_t ch = (size_t)unit * NC + m;
-      tc::fence_proxy_async();
-      tc::mbar_expect_tx(&aux_full[ai], m >= 1 ? 32768u : 16384u);
-      tc::bulk_g2s(ax, wA + ch * C * C, 16384u, &aux_full[ai]);
-      if (m >= 1) tc::bulk_g2s(ax + 16384, wHx + ch * C * C, 16384u, &aux_full[ai]);
-    };
-    prepare(0);
-    aux(0);
-    if (NC > 1) prepare(1);
-    for (int m = 0; m < NC; ++m) {
-      if (m + 2 < NC) prepare(m + 2);
-      if (m + 1 < NC) aux(m + 1);
-      // save the chunk-start state slice of chunk m once the chain has it in tensor memory
-      tc::mbar_wait<false>(&s_ready, (uint32_t)(m & 1), err, tc::kErrTimeoutMma, &abort_flag);
-      tc::tc_after_sync();
-      {
-        float* blob = wS0blob + ((size_t)unit * NC + m) * D * D;
-        const int r = p;
-#pragma unroll
-        for (int jj = 0; jj < NJ; jj += 16) {
-          float x[16];
-          tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int jg = j0 + jj + 4 * q4;
-            *reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(blob) + tc::sw128_off(r, jg, 128, 4)) =
-                make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
-          }
-          if (wS0b) save_bf16_tile(wS0b, (size_t)unit * NC + m, r, j0 + jj, x);
-        }
-      }
-      tc::tc_before_sync();
-      bar_prod();
-      if (p == 0) mbar_arrive(&s_saved);
-    }
-  } else {
-    // ============================= chain warps ============================
-    const int r = tid;  // tensor-memory lane = state row
-    {
-#pragma unroll
-      for (int jj = 0; jj < NJ; jj += 16) {
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = S0 ? S0[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] : 0.f;
-        tc::tmem_st16(my_lanes + Cf::S_COL + jj, x);
-      }
-      tc::tmem_st_wait();
-      tc::tc_before_sync();
-      bar_chain();
-      if (tid == 0) mbar_arrive(&s_ready);
-      bar_arrive_issuer(4);
-    }
-    int mma1_par = 0, mma2_par = 0;
-    // c_m partial: sum_r V_m[t,r] X'[r,t] over this CTA's rows, then all-reduce over the cluster
-    auto column_dot_send = [&](int m) {
-      tc::mbar_wait<false>(&mma1_bar, (uint32_t)mma1_par, err, tc::kErrTimeoutMma, &abort_flag);
-      mma1_par ^= 1;
-      tc::tc_after_sync();
-      {
-        float x[64];
-#pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          float y16[16];
-          tc::tmem_ld16(my_lanes + Cf::D1_COL + 16 * c16, y16);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) x[16 * c16 + i] = y16[i];
-        }
-        tc::tmem_ld_wait();
-        const unsigned char* vt = slot(m) + Cf::SL_V;  // row r of V^T: V[t, r] for t = 0..63
-        float lo[32], hi[32];
-#pragma unroll
-        for (int g8 = 0; g8 < 8; ++g8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(vt + tc::sw128_off(r, 8 * g8, 128, 2));
-          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int t = 8 * g8 + i;
-            if (t < 32) lo[t] = x[t] * __bfloat162float(e[i]);
-            else hi[t - 32] = x[t] * __bfloat162float(e[i]);
-          }
-        }
-        warp_transpose_reduce<32>(lo, lane);
-        warp_transpose_reduce<32>(hi, lane);
-        xred[warp * 64 + lane] = lo[0];
-        xred[warp * 64 + 32 + lane] = hi[0];
-      }
-      tc::tc_before_sync();
-      bar_chain();
-      if (tid < C) mine[tid] = xred[tid] + xred[64 + tid] + xred[128 + tid] + xred[192 + tid];
-      bar_chain();
-      const int xb = m & 1;
-      float* rv = recv + xb * R * 64;
-      if (tid == 0) tc::mbar_expect_tx(&x_bar[xb], R * 64u * 4u);
-      if (tid < 16 * R) {
-        const int peer = tid / 16, q4 = tid % 16;
-        const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
-        const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
-        const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[xb]), (uint32_t)peer);
-        tc::st_async_v4(raddr, val, rbar);
-      }
-    };
-    column_dot_send(0);
-    for (int n = 0; n < NC; ++n) {
-      const unsigned char* st = slot(n);
-      const size_t ch = (size_t)unit * NC + n;
-      // ---- b0_n = c_n + H_n u_{n-1};  u_n = y_n - A_n (beta o b0_n)
-      tc::mbar_wait<true>(&x_bar[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
-      tc::mbar_wait<false>(&aux_full[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
-      const float* Am = reinterpret_cast<const float*>(sm + Cf::AUX + (n & 1) * Cf::AUX_SZ);
-      const float* Hm = Am + C * C;
-      // two threads per position t (lanes 2t', 2t'+1 of a warp), halves of i, rotated reads
-      const int t = tid >> 1, half = tid & 1;
-      const int rot = t + 16 * half;
-      float s = 0.f;
-      {
-        const float* rv = recv + (n & 1) * R * 64;
-#pragma unroll
-        for (int c2 = 0; c2 < R; ++c2) s += rv[c2 * 64 + t];
-      }
-      if (n > 0) {
-        const float* Hrow = Hm + t * 64 + 32 * half;
-        const float* uh = us + 32 * half;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const int i0 = (i + rot) & 31, i1 = (i + 1 + rot) & 31, i2 = (i + 2 + rot) & 31, i3 = (i + 3 + rot) & 31;
-          a0 = fmaf(Hrow[i0], uh[i0], a0);
-          a1 = fmaf(Hrow[i1], uh[i1], a1);
-          a2 = fmaf(Hrow[i2], uh[i2], a2);
-          a3 = fmaf(Hrow[i3], uh[i3], a3);
-        }
-        float hu = (a0 + a1) + (a2 + a3);
-        hu += __shfl_xor_sync(0xffffffffu, hu, 1);
-        s += hu;
-      }
-      // s = b0_n[t] in both threads of the pair
-      if (half == 0) {
-        ws[t] = bs[(n % 3) * 64 + t] * s;
-        if (rank == 0 && wb0) wb0[ch * C + t] = s;
-      }
-      bar_chain();
-      float uval;
-      {
-        const float* Arow = Am + t * 64 + 32 * half;
-        const float* wh = ws + 32 * half;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const int i0 = (i + rot) & 31, i1 = (i + 1 + rot) & 31, i2 = (i + 2 + rot) & 31, i3 = (i + 3 + rot) & 31;
-          a0 = fmaf(Arow[i0], wh[i0], a0);
-          a1 = fmaf(Arow[i1], wh[i1], a1);
-          a2 = fmaf(Arow[i2], wh[i2], a2);
-          a3 = fmaf(Arow[i3], wh[i3], a3);
-        }
-        float aw = (a0 + a1) + (a2 + a3);
-        aw += __shfl_xor_sync(0xffffffffu, aw, 1);
-        uval = reinterpret_cast<const float*>(st + Cf::SL_Y)[t] - aw;
-      }
-      bar_chain();  // every thread has read u_{n-1} (us) and w
-      if (half == 0) {
-        us[t] = uval;
-        if (rank == 0 && wu) wu[ch * C + t] = uval;
-      }
-      bar_chain();
-      if (tid == 0) mbar_arrive(&aux_free[n & 1]);
-      // ---- B2 = diag(u_n) K^e_n slice as bf16 hi + lo (N = NJ rows j, K = 64 positions):
-      //      thread (channel jl, 64/TQ consecutive positions) writes 16-byte pieces of row jl
-      {
-        constexpr int TQ = 128 / NJ, TPT = C / TQ;  // position groups, positions per thread
-        const int jl = tid % NJ, tq = tid / NJ;
-        const float* KE = reinterpret_cast<const float*>(st + Cf::SL_KE);
-#pragma unroll
-        for (int g8 = 0; g8 < TPT; g8 += 8) {
-          __align__(16) __nv_bfloat16 hi8[8], lo8[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int tt = tq * TPT + g8 + i;
-            const float x = us[tt] * KE[tt * NJ + jl];
-            hi8[i] = __float2bfloat16_rn(x);
-            lo8[i] = __float2bfloat16_rn(x - __bfloat162float(hi8[i]));
-          }
-          const uint32_t off = tc::sw128_off(jl, tq * TPT + g8, NJ, 2);
-          *reinterpret_cast<uint4*>(sm + Cf::B2 + off) = *reinterpret_cast<const uint4*>(hi8);
-          *reinterpret_cast<uint4*>(sm + Cf::B2 + NJ * 128 + off) = *reinterpret_cast<const uint4*>(lo8);
-        }
-      }
-      tc::fence_proxy_async();
-      tc::tc_before_sync();
-      bar_arrive_issuer(3);
-      // ---- c_{n+1} from X' (its all-reduce overlaps the update)
-      if (n + 1 < NC) column_dot_send(n + 1);
-      tc::mbar_wait<false>(&mma2_bar, (uint32_t)mma2_par, err, tc::kErrTimeoutMma, &abort_flag);
-      mma2_par ^= 1;
-      // the producer must have saved this chunk's start state before it changes
-      tc::mbar_wait<false>(&s_saved, (uint32_t)(n & 1), err, tc::kErrTimeoutMma, &abort_flag);
-      tc::tc_after_sync();
-      // ---- S <- S diag(gamma_C) + dS
-      {
-        const float* gC = reinterpret_cast<const float*>(st + Cf::SL_GC);
-#pragma unroll
-        for (int jj = 0; jj < NJ; jj += 16) {
-          float s[16], d2[16];
-          tc::tmem_ld16(my_lanes + Cf::S_COL + jj, s);
-          tc::tmem_ld16(my_lanes + Cf::D2_COL + jj, d2);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], d2[i]);
-          tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
-        }
-        tc::tmem_st_wait();
-      }
-      tc::tc_before_sync();
-      bar_chain();
-      if (tid == 0) {
-        mbar_arrive(&slot_free[n % 3]);
-        mbar_arrive(&s_ready);
-      }
-      if (n + 2 < NC) bar_arrive_issuer(4);
-    }
-    if (ST) {
-      tc::tc_after_sync();
-#pragma unroll
-      for (int jj = 0; jj < NJ; jj += 16) {
-        float x[16];
-        tc::tmem_ld16(my_lanes + Cf::S_COL + jj, x);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) ST[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] = x[i];
-      }
-    }
-  }
-  tc::tc_before_sync();
-  __syncthreads();
-  tc::cluster_sync();  // no peer may still write into this CTA's shared memory
-  if (warp == 0) tc::tmem_dealloc(tmem, Cf::TMEM_COLS);
-}
-
 // ---------------------------------------------------------------------------
 // output kernel, one CTA per chunk:
 //   O^T[r,t] = sum_j S0[r,j] Q+[t,j] + sum_i V[i,r] u_i P[t,i],  P = tril(Q+ K-^T)
@@ -1133,73 +684,7 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
 }
 
-template <int R>
-cudaError_t launch_chain(const FwdArgs& a, const float* wy, const float* wA, float* blob, float* wu,
-                         float* wb0, int* err, cudaStream_t st) {
-  const Layout& L = a.L;
-  constexpr int NJ = ChainCfg<R>::NJ;
-  CUtensorMap tm_v, tm_kt, tm_ke;
-  if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
-      !make_tmap_bthd(&tm_kt, ws_ptr<float>(a.ws, L.Kt), 4, L.B, L.T, L.H, D, 32, true) ||
-      !make_tmap_bthd(&tm_ke, ws_ptr<float>(a.ws, L.Ke), 4, L.B, L.T, L.H, D, NJ, false))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_chain_tc<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)ChainCfg<R>::BYTES);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(L.B * L.H * R);
-  cfg.blockDim = dim3(288);
-  cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = R;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  prof_begin(st, "fwd_chain_tc");
-  __nv_bfloat16* s0b = a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0b) : nullptr;
-  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_v, tm_kt, tm_ke, a.beta, a.S0, a.ST, L.H, L.T, L.NC, wy, wA,
-                         (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt), blob, wu, wb0, s0b, err);
-  prof_end(st);
-  return e;
-}
-
 }  // namespace
-
-template <int R>
-static int max_active_clusters() {
-  if (cudaFuncSetAttribute(fwd_chain_tc<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)ChainCfg<R>::BYTES) != cudaSuccess)
-    return 0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(R * 1024);
-  cfg.blockDim = dim3(288);
-  cfg.dynamicSmemBytes = ChainCfg<R>::BYTES;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = R;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, fwd_chain_tc<R>, &cfg) != cudaSuccess) return 0;
-  return n;
-}
-
-// Largest cluster (8 or 4 CTAs per head) for which every head's cluster is
-// resident at once; 4 when none is.
-int choose_cluster(int units, int sms) {
-  (void)sms;
-  static int cap8 = -1, cap4 = -1;  // per process; the library targets one GPU model
-  if (cap8 < 0) cap8 = max_active_clusters<8>();
-  if (cap4 < 0) cap4 = max_active_clusters<4>();
-  if (units <= cap8) return 8;
-  return 4;
-}
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) {
   const Layout& L = a.L;
@@ -1235,16 +720,10 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (!(a.phases & kPhaseCarry)) return cudaSuccess;
-  const float* wy = ws_ptr<float>(a.ws, L.y);
-  const float* wA = ws_ptr<float>(a.ws, L.A);
   float* blob = ws_ptr<float>(a.ws, L.S0);
   float* wu = ws_ptr<float>(a.ws, L.u);
-  float* wb0 = ws_ptr<float>(a.ws, L.b0);
   int* flags = ws_ptr<int>(a.ws, L.flags);
-  const int R = choose_cluster(L.B * L.H, sms);
-  if (R == 8) e = launch_chain<8>(a, wy, wA, blob, wu, wb0, err, st);
-  else e = launch_chain<4>(a, wy, wA, blob, wu, wb0, err, st);
-  if (e != cudaSuccess) return e;
+  if ((e = launch_fwd_chain_tc(a, choose_cluster(L.B * L.H, sms), err, st)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(fwd_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)OutCfg::BYTES)) != cudaSuccess)
     return e;

@@ -45,6 +45,10 @@ struct Layout {
   // 128-byte-swizzled tiles): [dP; E_V] (128 x 64), P diag(u) and E_K
   // (64 x 64 each); M u [ch][64]
   size_t T1 = 0, PU = 0, EK = 0, Mu = 0;
+  // tensor-core path, written by the pre-chain kernel for the reverse chain:
+  // K+ [B][T][H][dk] fp32, and Q+^T per chunk as a bf16 128-byte-swizzled
+  // K-major tile [j][t] (128 rows x 64)
+  size_t Kp = 0, QpT = 0;
   size_t bwd_bytes = 0;
 };
 
@@ -100,6 +104,10 @@ cudaError_t launch_fwd_prep(const FwdArgs& a, bool with_P, cudaStream_t st);
 // err: the library's device error word; sms: multiprocessors of the device.
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st);
 int choose_cluster(int units, int sms);
+// the forward's sequential chunk chain on tensor cores, R CTAs per head (kd_fchain_tc.cu)
+cudaError_t launch_fwd_chain_tc(const FwdArgs& a, int R, int* err, cudaStream_t st);
+// the backward's reverse chunk chain on tensor cores (kd_bchain_tc.cu)
+cudaError_t launch_bwd_chain_tc(const BwdArgs& a, int R, int* err, cudaStream_t st);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t st);
 // CUDA-core backward kernels by stage; `only` (nullable) restricts the
 // per-chunk stages (cc, state, intra) to chunks whose flag is set.
