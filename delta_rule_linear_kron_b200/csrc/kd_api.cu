@@ -67,16 +67,15 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
     L->Ke = take((size_t)B * T * H * dk * 4);
     L->GC = take(chunks * (size_t)dk * 4);
     L->Vt = take(chunks * (size_t)dv * C * 2);
+    L->xflags = take(chunks * 4);
   }
   L->fwd_bytes = off;
-  L->S0 = take(chunks * (size_t)dv * dk * 4);
+  L->S0 = take(chunks * (size_t)dv * dk * 4);  // tensor-core path: written only for chunks with xflags set
   L->u = take(chunks * C * 4);
   L->b0 = take(chunks * C * 4);
   L->flags = take(chunks * 4);
-  if (L->tc) {
-    L->fwd_bytes = off;  // the output kernel reads the chunk-start states
-    L->S0b = take(chunks * (size_t)dv * dk * 2);
-  }
+  if (L->tc) L->S0b = take(chunks * (size_t)dv * dk * 2);
+  if (L->tc) L->fwd_bytes = off;  // the chain writes u, b0 and the chunk-start states on every call
   L->fwd_save_bytes = off;
 
   off = 0;

@@ -43,6 +43,9 @@ namespace {
 
 constexpr int C = kChunk;
 constexpr int D = 128;
+// Steps ahead of the shared-memory rings whose operands the producer pulls
+// into L2, so that the ring's own copies are L2 hits.
+constexpr int kL2Ahead = 3;
 
 template <int R>
 struct BcCfg {
@@ -459,6 +462,13 @@ __global__ void __launch_bounds__(320, 1) bwd_chain_tc(
         tc::tma_load_4d(es + Cf::E_DO + 8192, &tm_do, 64, h, n * C, b, &e_full[si]);
         tc::tma_load_4d(es + Cf::E_KE, &tm_ke, jb, h, n * C, b, &e_full[si]);
         tc::bulk_g2s(es + Cf::E_QP, wQpT + ch * (D * C) + (size_t)j0 * C, NJ * 128u, &e_full[si]);
+        if (k + kL2Ahead < NC) {
+          const int np = chunk_of(k + kL2Ahead);
+          tc::tma_prefetch_l2_4d(&tm_do, 0, h, np * C, b);
+          tc::tma_prefetch_l2_4d(&tm_do, 64, h, np * C, b);
+          tc::tma_prefetch_l2_4d(&tm_ke, jb, h, np * C, b);
+          tc::prefetch_l2(wQpT + (ch - kL2Ahead) * (D * C) + (size_t)j0 * C, NJ * 128u);
+        }
       }
       __syncwarp();
     };
@@ -474,6 +484,10 @@ __global__ void __launch_bounds__(320, 1) bwd_chain_tc(
         tc::bulk_g2s(ls + Cf::L_V, wVt + ch * (D * C), 16384u, &l_full[si]);
         tc::tma_load_4d(ls + Cf::L_KP, &tm_kp, j0, h, n * C, b, &l_full[si]);
         tc::bulk_g2s(ls + Cf::L_GC, wGC + ch * D + j0, NJ * 4u, &l_full[si]);
+        if (k + kL2Ahead < NC) {
+          tc::prefetch_l2(wVt + (ch - kL2Ahead) * (D * C), 16384u);
+          tc::tma_prefetch_l2_4d(&tm_kp, j0, h, chunk_of(k + kL2Ahead) * C, b);
+        }
       }
       __syncwarp();
     };
@@ -489,6 +503,10 @@ __global__ void __launch_bounds__(320, 1) bwd_chain_tc(
         tc::bulk_g2s(ax + Cf::AX_A, wA + ch * C * C, 16384u, &aux_full[ai]);
         if (k >= 1) tc::bulk_g2s(ax + Cf::AX_H, wHx + (ch + 1) * C * C, 16384u, &aux_full[ai]);  // H_{n+1}
         tc::bulk_g2s(ax + Cf::AX_DU, wdu + ch * C, 256u, &aux_full[ai]);
+        if (k + kL2Ahead < NC) {
+          tc::prefetch_l2(wA + (ch - kL2Ahead) * C * C, 16384u);
+          tc::prefetch_l2(wHx + (ch - kL2Ahead + 1) * C * C, 16384u);
+        }
       }
       float* bs = reinterpret_cast<float*>(ax + Cf::AX_B);
 #pragma unroll

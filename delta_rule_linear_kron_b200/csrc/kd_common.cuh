@@ -17,6 +17,16 @@ namespace kd {
 // per-element path.
 constexpr float kSafeLogRange = 80.0f;
 
+// |L| bound of the backward's factorised post-chain products: e^{-40} keeps
+// dS' = dS e^Lambda well inside bf16's normal range for any |dS| above 1e-20.
+// Chunks at or beyond it take the exact per-element backward path.
+constexpr float kPostSafe = 40.0f;
+
+// Chunks whose in-chunk |L| reaches this bound (below both bounds above, so
+// that float rounding of L cannot leave a chunk on an exact path without it)
+// also keep their chunk-start state in fp32 for the exact paths.
+constexpr float kExactStateRange = 36.0f;
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -26,8 +26,10 @@
 //              all-reduced c), the update operand diag(u) K^e in bf16 hi + lo.
 //   warps 4-7  state warps (thread r = tensor-memory lane r = state row r):
 //              the state update S <- S diag(gamma) + dS, the save of each
-//              chunk-start state, the column dot of the lookahead MMA and the
-//              send of its partial sums to every CTA of the cluster.
+//              chunk-start state (a bf16 tile for the output kernel and the
+//              backward; an fp32 copy as well for chunks bound for the exact
+//              paths), the column dot of the lookahead MMA and the send of
+//              its partial sums to every CTA of the cluster.
 //   warp 8     issuer: one thread issues every tcgen05 MMA.
 //   warp 9     producer: bulk / TMA loads of each chunk's operands (a ring of
 //              three slots) and of the u recursion's matrices (a ring of two).
@@ -44,6 +46,9 @@ namespace {
 
 constexpr int C = kChunk;
 constexpr int D = 128;
+// Chunks ahead of the shared-memory rings whose operands the producer pulls
+// into L2, so that the ring's own copies are L2 hits.
+constexpr int kL2Ahead = 3;
 
 template <int R>
 struct FcCfg {
@@ -119,8 +124,9 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
     const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_ke,
     const float* __restrict__ beta, const float* __restrict__ S0, float* __restrict__ ST, int H, int T, int NC,
     const float* __restrict__ wy, const float* __restrict__ wA, const float* __restrict__ wHx,
-    const float* __restrict__ wGC, const __nv_bfloat16* __restrict__ wVt, float* __restrict__ wS0blob,
-    float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b, int* __restrict__ err) {
+    const float* __restrict__ wGC, const __nv_bfloat16* __restrict__ wVt, const int* __restrict__ wxflags,
+    float* __restrict__ wS0blob, float* __restrict__ wu, float* __restrict__ wb0, __nv_bfloat16* __restrict__ wS0b,
+    int* __restrict__ err) {
   using Cf = FcCfg<R>;
   constexpr int NJ = Cf::NJ;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -284,14 +290,15 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
     // the initial state into tensor memory; it is also chunk 0's start state
     {
       const size_t ch0 = (size_t)unit * NC;
+      const bool f32copy = wxflags[ch0] != 0;
 #pragma unroll
       for (int jj = 0; jj < NJ; jj += 16) {
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = S0 ? S0[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] : 0.f;
         tc::tmem_st16(my_lanes + Cf::S_COL + jj, x);
-        save_f32_tile(wS0blob, ch0, r, j0 + jj, x);
-        if (wS0b) save_bf16_tile(wS0b, ch0, r, j0 + jj, x);
+        save_bf16_tile(wS0b, ch0, r, j0 + jj, x);
+        if (f32copy) save_f32_tile(wS0blob, ch0, r, j0 + jj, x);
       }
       tc::tmem_st_wait();
       tc::tc_before_sync();
@@ -354,6 +361,7 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
       {
         const float* gC = reinterpret_cast<const float*>(st + Cf::SL_GC);
         const size_t chn = (size_t)unit * NC + n + 1;
+        const bool f32copy = n + 1 < NC && wxflags[chn] != 0;
 #pragma unroll
         for (int jj = 0; jj < NJ; jj += 16) {
           float s[16], d2[16];
@@ -364,8 +372,8 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
           for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], d2[i]);
           tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
           if (n + 1 < NC) {
-            save_f32_tile(wS0blob, chn, r, j0 + jj, s);
-            if (wS0b) save_bf16_tile(wS0b, chn, r, j0 + jj, s);
+            save_bf16_tile(wS0b, chn, r, j0 + jj, s);
+            if (f32copy) save_f32_tile(wS0blob, chn, r, j0 + jj, s);
           } else if (ST) {
 #pragma unroll
             for (int i4 = 0; i4 < 4; ++i4)
@@ -451,6 +459,12 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
         tc::tma_load_4d(st + Cf::SL_KT, &tm_kt, jb, h, m * C, b, bar);
         tc::tma_load_4d(st + Cf::SL_KE, &tm_ke, j0, h, m * C, b, bar);
         tc::bulk_g2s(st + Cf::SL_GC, wGC + ch * D + j0, NJ * 4u, bar);
+        const int mp = m + kL2Ahead;
+        if (mp < NC) {
+          tc::prefetch_l2(wVt + (ch + kL2Ahead) * (D * C), 16384u);
+          tc::tma_prefetch_l2_4d(&tm_kt, jb, h, mp * C, b);
+          tc::tma_prefetch_l2_4d(&tm_ke, j0, h, mp * C, b);
+        }
       }
       __syncwarp();
     };
@@ -466,6 +480,10 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
         tc::bulk_g2s(ax + Cf::AX_A, wA + ch * C * C, 16384u, &aux_full[ai]);
         if (m >= 1) tc::bulk_g2s(ax + Cf::AX_H, wHx + ch * C * C, 16384u, &aux_full[ai]);
         tc::bulk_g2s(ax + Cf::AX_Y, wy + ch * C, 256u, &aux_full[ai]);
+        if (m + kL2Ahead < NC) {
+          tc::prefetch_l2(wA + (ch + kL2Ahead) * C * C, 16384u);
+          tc::prefetch_l2(wHx + (ch + kL2Ahead) * C * C, 16384u);
+        }
       }
       float* bs = reinterpret_cast<float*>(ax + Cf::AX_B);
 #pragma unroll
@@ -524,9 +542,9 @@ cudaError_t launch_chain_r(const FwdArgs& a, int* err, cudaStream_t st) {
   e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_kt, tm_ke, a.beta, a.S0, a.ST, L.H, L.T, L.NC,
                          (const float*)ws_ptr<float>(a.ws, L.y), (const float*)ws_ptr<float>(a.ws, L.A),
                          (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC),
-                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt), ws_ptr<float>(a.ws, L.S0),
-                         ws_ptr<float>(a.ws, L.u), ws_ptr<float>(a.ws, L.b0),
-                         a.save ? ws_ptr<__nv_bfloat16>(a.ws, L.S0b) : nullptr, err);
+                         (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt),
+                         (const int*)ws_ptr<int>(a.ws, L.xflags), ws_ptr<float>(a.ws, L.S0),
+                         ws_ptr<float>(a.ws, L.u), ws_ptr<float>(a.ws, L.b0), ws_ptr<__nv_bfloat16>(a.ws, L.S0b), err);
   prof_end(st);
   return e;
 }

@@ -8,26 +8,17 @@
 //   S  <- S diag(gamma_C) + V^T diag(u) K^e,
 //   O  = Q+ S0^T + P diag(u) V.
 //
-// Kernels:
-//  1. prep (kd_fwd_simt.cu, fwd_prep_simt): A = (I + diag(beta) M)^{-1}, y.
-//  2. fwd_chain_tc: the sequential chain.  One thread-block cluster of R CTAs
-//     per (b,h); CTA c owns the key-channel slice J_c (dk/R columns) of the
-//     state, kept in tensor memory as the A operand of the MMAs:
-//       X_c = S[:,J_c] K+[:,J_c]^T            (tcgen05, A from TMEM)
-//       b0_c[t] = sum_r V[t,r] X_c[r,t]       (column sum over TMEM lanes)
-//       b0 = sum_c b0_c                       (distributed shared memory:
-//                                              st.async + mbarrier tx count)
-//       u = y - A (beta o b0)                 (every CTA, identical order)
-//       dS_c = V^T (diag(u) K^e[:,J_c])       (tcgen05)
-//       S[:,J_c] <- S[:,J_c] diag(gamma_C) + dS_c
-//     The next chunk's rows are fetched with bulk async copies while the
-//     current chunk runs.  Each chunk-start state slice is written to global
-//     memory in the 128-byte-swizzled K-major tile layout the output kernel's
-//     MMA reads directly.
-//  3. fwd_out_tc: one CTA per chunk, all chunks in parallel:
-//       O^T = S0 Q+^T + V^T (diag(u) P^T)  with P = tril(Q+ K-^T) (tcgen05).
-//     Chunks whose log-decay range makes k/gamma leave the fp32 range are
-//     flagged and recomputed exactly by fwd_out_fixup.
+// Kernels of this file (the sequential chain is in kd_fchain_tc.cu):
+//  1. fwd_prep_tc, one CTA per chunk: the decay prefix, the Grams, the chunk
+//     inverse A = (I + diag(beta) M)^{-1}, y = A c, and P when saving.
+//  2. fwd_cross_tc, one CTA per chunk: the chain's per-chunk operands (K~,
+//     K^e, gamma_C, V^T) and the cross-chunk matrix H of its lookahead.
+//  3. fwd_out_tc, one CTA per chunk, after the chain:
+//       O^T = S0 Q+^T + V^T (diag(u) P^T)  with P = tril(Q+ K-^T) (tcgen05),
+//     S0 being the chain's bf16 chunk-start state tile.  Chunks whose
+//     log-decay range makes k/gamma leave the fp32 range are flagged and
+//     recomputed exactly by fwd_out_fixup from the fp32 copy the chain keeps
+//     for such chunks.
 #include "kd_common.cuh"
 #include "kd_kernels.h"
 #include "kd_tc.cuh"
@@ -46,7 +37,9 @@ constexpr int D = 128;
 // the intra-chunk product V^T (diag(u) P^T) in bf16 (V is bf16 already).
 // ---------------------------------------------------------------------------
 struct OutCfg {
-  static constexpr uint32_t S0 = 0;           // S0 blob, tf32 SW128 [4 kb][128][128 B]
+  static constexpr uint32_t S0B = 0;          // chunk-start state bf16 [r][j], 2 K blocks x 128 rows (32 KB)
+  static constexpr uint32_t QH = 32768;       // Q+ bf16 high part [t][j], 2 K blocks x 64 rows (16 KB)
+  static constexpr uint32_t QL = 49152;       // Q+ bf16 low part (Q+ - high), same layout
   static constexpr uint32_t QK = 65536;       // tf32 [Q+; K-]: per 32-channel K block rows 0-63 Q+, 64-127 K-
   static constexpr uint32_t VB = 131072;      // V bf16 [i][r], 2 K blocks x 64 rows (TMA, 128-byte swizzle)
   static constexpr uint32_t B3 = 147456;      // diag(u) P^T as bf16 [t][i], 64 rows x 64
@@ -56,14 +49,14 @@ struct OutCfg {
   static constexpr uint32_t U = 221184;       // u [64]
   static constexpr uint32_t XCH = U + 256;    // prefix exchange [128]
   static constexpr uint32_t BYTES = XCH + 512 + 1024;
-  static constexpr uint32_t LOAD_BYTES = 65536 + 16384 + 2 * 16384 + 32768 + 256;
+  static constexpr uint32_t LOAD_BYTES = 32768 + 16384 + 2 * 16384 + 32768 + 256;
   static constexpr uint32_t OO = QK;          // output staging O bf16 [t][r] (after the MMAs)
 };
 
 __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_logf,
-    const __grid_constant__ CUtensorMap tm_out, int H, int NC, const float* __restrict__ wS0blob,
+    const __grid_constant__ CUtensorMap tm_out, int H, int NC, const __nv_bfloat16* __restrict__ wS0b,
     const float* __restrict__ wu, int* __restrict__ unsafe_flags, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -83,8 +76,8 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     abort_flag = 0;
     tc::mbar_expect_tx(&ld_bar, OutCfg::LOAD_BYTES);
 #pragma unroll
-    for (int part = 0; part < 4; ++part)
-      tc::bulk_g2s(sm + OutCfg::S0 + part * 16384, wS0blob + ch * D * D + part * 4096, 16384u, &ld_bar);
+    for (int part = 0; part < 2; ++part)
+      tc::bulk_g2s(sm + OutCfg::S0B + part * 16384, wS0b + ch * D * D + part * 8192, 16384u, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::VB, &tm_v, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::VB + 8192, &tm_v, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
@@ -122,8 +115,13 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
       mx = fmaxf(mx, fabsf(L));
       const float qq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OutCfg::QR + (t * D + j) * 2));
       const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OutCfg::KR + (t * D + j) * 2));
-      *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = qq * expf(L);
+      const float qp = qq * expf(L);
+      *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(t, j, 128, 4)) = qp;
       *reinterpret_cast<float*>(sm + OutCfg::QK + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(-L);
+      const __nv_bfloat16 qh = __float2bfloat16_rn(qp);
+      *reinterpret_cast<__nv_bfloat16*>(sm + OutCfg::QH + tc::sw128_off(t, j, 64, 2)) = qh;
+      *reinterpret_cast<__nv_bfloat16*>(sm + OutCfg::QL + tc::sw128_off(t, j, 64, 2)) =
+          __float2bfloat16_rn(qp - __bfloat162float(qh));
     }
   }
   const bool is_unsafe = __syncthreads_or(!(mx < kSafeLogRange)) != 0;
@@ -131,17 +129,23 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
-  // MMA: D_P[t,i] (cols 0..63, lanes 0..63) = [Q+; K-] K-^T ; D_O[r,t] (cols 64..127) = S0 Q+^T
+  // MMA: D_P[t,i] (cols 0..63, lanes 0..63) = [Q+; K-] K-^T (tf32);
+  //      D_O[r,t] (cols 64..127) = S0 (Q+hi + Q+lo)^T (bf16: the state tile is bf16)
   if (tid == 0) {
-    const uint32_t IDT = tc::idesc(128, 64, 2);
+    const uint32_t IDT = tc::idesc(128, 64, 2), IDB = tc::idesc(128, 64, 1);
 #pragma unroll
     for (int ks = 0; ks < 16; ++ks) {
       const uint32_t o = (ks / 4) * 16384 + (ks % 4) * 32;
       const uint64_t qa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::QK + o));
       const uint64_t kmb = tc::desc_sw128(tc::smem_u32(sm + OutCfg::QK + o + 8192));
-      const uint64_t sa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::S0 + o));
       tc::mma_tf32_ss(tmem + 0, qa, kmb, IDT, ks > 0 ? 1u : 0u);
-      tc::mma_tf32_ss(tmem + 64, sa, qa, IDT, ks > 0 ? 1u : 0u);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint64_t sa = tc::desc_sw128(tc::smem_u32(sm + OutCfg::S0B + (ks / 4) * 16384 + (ks % 4) * 32));
+      const uint32_t qo = (ks / 4) * 8192 + (ks % 4) * 32;
+      tc::mma_bf16_ss(tmem + 64, sa, tc::desc_sw128(tc::smem_u32(sm + OutCfg::QH + qo)), IDB, ks > 0 ? 1u : 0u);
+      tc::mma_bf16_ss(tmem + 64, sa, tc::desc_sw128(tc::smem_u32(sm + OutCfg::QL + qo)), IDB, 1u);
     }
     tc::mma_commit(&mma_bar);
   }
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf,
     const float* __restrict__ beta, const float* __restrict__ c, int H, int T, int NC, float* __restrict__ wy,
-    float* __restrict__ wA, float* __restrict__ wP, int* __restrict__ err) {
+    float* __restrict__ wA, float* __restrict__ wP, int* __restrict__ wxflags, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -371,6 +375,8 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     }
   }
   const bool is_unsafe = __syncthreads_or(!(mx < kSafeLogRange)) != 0;
+  const bool exact_state = __syncthreads_or(!(mx < kExactStateRange)) != 0;
+  if (tid == 0) wxflags[ch] = exact_state ? 1 : 0;
   tc::fence_proxy_async();
   tc::tc_before_sync();
   __syncthreads();
@@ -702,7 +708,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     prof_begin(st, "fwd_prep_tc");
     fwd_prep_tc<<<(unsigned)L.chunks, 256, PrepCfg::BYTES, st>>>(
         tm_v, tm_q, tm_k, tm_logf, a.beta, a.c, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
-        a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, err);
+        a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, ws_ptr<int>(a.ws, L.xflags), err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     CUtensorMap tm_kt, tm_ke;
@@ -736,8 +742,9 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
         !make_tmap_bthd(&tm_out, a.out, 2, L.B, L.T, L.H, D, 64, true))
       return cudaErrorInvalidValue;
     prof_begin(st, "fwd_out_tc");
-    fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, blob,
-                                                               wu, flags, err);
+    fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(
+        tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.S0b), wu,
+        flags, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -28,11 +28,15 @@ struct Layout {
   // tensor-core path, operands of the chain: cross-chunk matrix Hx [ch][64][64],
   // K~ and K^e [B][T][H][dk] (fp32), gamma_C [ch][dk], V^T [ch][dv][64] (bf16 tile)
   size_t y = 0, A = 0, P = 0, Hx = 0, Kt = 0, Ke = 0, GC = 0, Vt = 0;
+  // tensor-core path: one int per chunk, set by the preparation kernel when
+  // the chunk's in-chunk |L| reaches kExactStateRange (the chain then also
+  // keeps its chunk-start state in fp32 for the exact paths)
+  size_t xflags = 0;
   size_t fwd_bytes = 0;
   // saved for the backward: S0 [ch][dv][dk], u [ch][64], b0 [ch][64]
   size_t S0 = 0, u = 0, b0 = 0, flags = 0;  // flags: one int per chunk (tensor-core path)
-  // tensor-core path, saved for the backward: chunk-start states as bf16
-  // 128-byte-swizzled K-major tiles [r][j] (rows r, K = j)
+  // tensor-core path: chunk-start states as bf16 128-byte-swizzled K-major
+  // tiles [r][j] (rows r, K = j), read by the output kernel and the backward
   size_t S0b = 0;
   size_t fwd_save_bytes = 0;
   // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],

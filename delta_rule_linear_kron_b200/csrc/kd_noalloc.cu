@@ -14,7 +14,7 @@
 //     (32 MiB).  Every GPU that loads the library holds it until the process
 //     exits.  A problem whose forward scratch (kron_delta_workspace_size with
 //     KD_WS_FWD) exceeds it is rejected with KD_ERR_WORKSPACE before anything
-//     is enqueued: beyond 169 chunk-heads (B * H * ceil(T/64)) on the
+//     is enqueued: beyond 145 chunk-heads (B * H * ceil(T/64)) on the
 //     tensor-core path (bf16, dk = dv = 128, whose chain also keeps per-token
 //     operands there), beyond 1016 on the others.
 //   * All calls share the one array and it keeps the last call's contents.

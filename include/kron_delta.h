@@ -227,7 +227,7 @@ KD_API int kron_delta_decode(const void *q, const void *k, const void *v,
  * library until exit).
  *   - Problems whose forward scratch (kron_delta_workspace_size, KD_WS_FWD)
  *     exceeds that return KD_ERR_WORKSPACE (use kron_delta_fwd then): beyond
- *     169 chunk-heads B * H * ceil(T/64) for bf16 with dk = dv = 128, beyond
+ *     145 chunk-heads B * H * ceil(T/64) for bf16 with dk = dv = 128, beyond
  *     1016 for the other shapes.
  *   - All calls share the array; concurrent calls that overlap on the GPU
  *     race on it, so the caller must serialise them (e.g. one stream).
