@@ -8,28 +8,35 @@
 // (both built in parallel by fwd_cross_tc), the erase read of chunk n splits
 // into a part that needs only the state one chunk earlier and a correction
 // linear in the previous chunk's write coefficients:
-//   c_n  = rowdot(V_n, S_{n-1} K~_n^T)            (one-chunk lookahead)
+//   c_n  = rowdot(V_n S_{n-1}, K~_n)             (one-chunk lookahead)
 //   b0_n = c_n + H_n u_{n-1}
 //   u_n  = y_n - A_n (beta_n o b0_n)
 //   S_{n+1} = S_n diag(gamma_C,n) + V_n^T diag(u_n) K^e_n.
-// So two loops run through the chain:
+// Two loops run through the chain:
 //   short: u_{n-1} -> u_n, two 64 x 64 matrix-vector products (CUDA cores);
-//   long:  u_n -> update MMA -> S_{n+1} -> lookahead MMA and column dot ->
-//          cluster all-reduce -> c_{n+2} -> u_{n+2}, spanning two chunks.
-// Each loop runs on its own warps, so the two overlap: the chain's step time
-// is about half the long loop, not the sum of every stage.
+//   long:  u_n -> update MMA -> S_{n+1} -> lookahead MMA U = V_{n+2} S_{n+1}
+//          and the row dot with K~ -> cluster all-reduce -> c_{n+2} -> u_{n+2},
+//          spanning two chunks.
+// Each loop runs on its own warps, so the two overlap.  The lookahead MMA
+// contracts over the state's rows (value channels), so each lane of its
+// accumulator holds one position's partial sum over this CTA's key channels:
+// the column dot is a per-lane dot product, with no reduction across lanes.
 //
 // One thread-block cluster of R CTAs per (b, h); CTA c owns the key-channel
-// slice J_c (128 / R channels) of the state, kept in tensor memory.
+// slice J_c (128 / R channels) of the state: row r of the slice lives in the
+// registers of state thread r, in fp32.  Its bf16 high and low parts are also
+// kept in shared memory as the lookahead MMA's B operand (MN-major: row r
+// holds the slice's channels).
 // Warp roles (320 threads):
 //   warps 0-3  u warps: b0, u (every CTA computes the same u from the
 //              all-reduced c), the update operand diag(u) K^e in bf16 hi + lo.
-//   warps 4-7  state warps (thread r = tensor-memory lane r = state row r):
-//              the state update S <- S diag(gamma) + dS, the save of each
-//              chunk-start state (a bf16 tile for the output kernel and the
-//              backward; an fp32 copy as well for chunks bound for the exact
-//              paths), the column dot of the lookahead MMA and the send of
-//              its partial sums to every CTA of the cluster.
+//   warps 4-7  state warps (thread r = state row r = tensor-memory lane r):
+//              the state update S <- S diag(gamma) + dS, its bf16 operand
+//              copy, the save of each chunk-start state (a bf16 tile for the
+//              output kernel and the backward; an fp32 copy as well for chunks
+//              bound for the exact paths); warps 4-5 (lanes = positions) the
+//              row dot of the lookahead and the send of its partial sums to
+//              every CTA of the cluster.
 //   warp 8     issuer: one thread issues every tcgen05 MMA.
 //   warp 9     producer: bulk / TMA loads of each chunk's operands (a ring of
 //              three slots) and of the u recursion's matrices (a ring of two).
@@ -52,16 +59,16 @@ constexpr int kL2Ahead = 3;
 
 template <int R>
 struct FcCfg {
-  static constexpr int NJ = D / R;              // key channels per CTA
-  static constexpr int KBJ = (R == 8) ? 2 : 0;  // K steps of the K~ block before this CTA's channels (odd R=8 ranks)
-  // tensor memory: X' [2] (64 columns each), the state slice, the update accumulators [2]
-  static constexpr int X_COL = 0, S_COL = 128, D2_COL = 128 + NJ;
-  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr int NJ = D / R;  // key channels per CTA
+  // tensor memory: the lookahead accumulators U [2] and the update accumulators [2], NJ columns each
+  static constexpr int U_COL = 0, D2_COL = 2 * NJ;
+  static constexpr uint32_t TMEM_COLS = (4 * NJ) <= 64 ? 64u : 128u;
   static constexpr uint32_t up1k(uint32_t x) { return (x + 1023u) / 1024u * 1024u; }
   // chunk operand ring (3 slots), written by bulk copies / TMA
   static constexpr int NSLOT = 3;
-  static constexpr uint32_t SL_V = 0;                     // V^T bf16 [r][t], K-major, 128-byte swizzle (16 KB)
-  static constexpr uint32_t SL_KT = 16384;                // K~, the 32-channel block holding this CTA's channels
+  static constexpr uint32_t SL_V = 0;                     // V^T bf16 [r][t], 128-byte swizzle (16 KB)
+  static constexpr uint32_t SL_KT = 16384;                // K~, the 32-channel block holding this CTA's
+                                                          //   channels, fp32 [64][32], 128-byte swizzle (8 KB)
   static constexpr uint32_t SL_KE = SL_KT + 8192;         // K^e slice fp32 [64][NJ]
   static constexpr uint32_t SL_GC = SL_KE + 64 * NJ * 4;  // gamma_C slice [NJ]
   static constexpr uint32_t SL_SZ = up1k(SL_GC + NJ * 4);
@@ -73,20 +80,20 @@ struct FcCfg {
   // update operand diag(u) K^e slice [2 buffers][hi, lo][NJ rows x 128 B]
   static constexpr uint32_t B2 = AUX + 2 * AUX_SZ;
   static constexpr uint32_t B2_SZ = 2 * NJ * 128;
-  static constexpr uint32_t SM = B2 + 2 * B2_SZ;
+  // the state slice's bf16 high / low parts, MN-major B operand [r][j] (128 rows x 128 B each)
+  static constexpr uint32_t SC = B2 + 2 * B2_SZ;
+  static constexpr uint32_t SM = SC + 2 * 16384;
   static constexpr uint32_t SM_RECV = SM;                        // c partials [4][R][64]
-  static constexpr uint32_t SM_XRED = SM_RECV + 4 * R * 64 * 4;  // per-warp column sums [4][64]
-  static constexpr uint32_t SM_MINE = SM_XRED + 4 * 64 * 4;      // own c partial [64]
-  static constexpr uint32_t SM_US = SM_MINE + 64 * 4;            // u [2][64]
+  static constexpr uint32_t SM_US = SM_RECV + 4 * R * 64 * 4;    // u [2][64]
   static constexpr uint32_t SM_WS = SM_US + 2 * 64 * 4;          // beta o b0 [64]
   static constexpr uint32_t SM_END = SM_WS + 64 * 4;
   static constexpr uint32_t BYTES = SM_END + 1024;  // + alignment slack
 };
 
 // Writes 16 state values (row r, columns j..j+15) of one chunk into the bf16
-// tile the backward's MMAs read: [r][j] (rows r, K = j), 128-byte-swizzled
-// K-major, 32 KB.
-__device__ __forceinline__ void save_bf16_tile(__nv_bfloat16* rj, size_t ch, int r, int j, const float (&x)[16]) {
+// tile the output kernel and the backward read: [r][j] (rows r, K = j),
+// 128-byte-swizzled K-major, 32 KB per chunk.
+__device__ __forceinline__ void save_bf16_tile(__nv_bfloat16* rj, size_t ch, int r, int j, const float* x) {
   unsigned char* a = reinterpret_cast<unsigned char*>(rj + ch * D * D);
 #pragma unroll
   for (int h8 = 0; h8 < 2; ++h8) {
@@ -96,9 +103,9 @@ __device__ __forceinline__ void save_bf16_tile(__nv_bfloat16* rj, size_t ch, int
     *reinterpret_cast<uint4*>(a + tc::sw128_off(r, j + 8 * h8, 128, 2)) = *reinterpret_cast<const uint4*>(v8);
   }
 }
-// The same 16 values into the fp32 tile the output kernel's tf32 MMA reads
-// (128-byte-swizzled K-major, [r][j], 64 KB per chunk).
-__device__ __forceinline__ void save_f32_tile(float* blob, size_t ch, int r, int j, const float (&x)[16]) {
+// The same 16 values into the fp32 copy the exact paths read (128-byte-swizzled
+// K-major, [r][j], 64 KB per chunk).
+__device__ __forceinline__ void save_f32_tile(float* blob, size_t ch, int r, int j, const float* x) {
   unsigned char* a = reinterpret_cast<unsigned char*>(blob + ch * D * D);
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4)
@@ -144,8 +151,6 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
   const int jb = j0 & ~31;  // first channel of the 32-channel K~ block
 
   float* recv = reinterpret_cast<float*>(sm + Cf::SM_RECV);
-  float* xred = reinterpret_cast<float*>(sm + Cf::SM_XRED);
-  float* mine = reinterpret_cast<float*>(sm + Cf::SM_MINE);
   float* us = reinterpret_cast<float*>(sm + Cf::SM_US);
   float* ws = reinterpret_cast<float*>(sm + Cf::SM_WS);
   auto slot = [&](int m) { return sm + (m % 3) * Cf::SL_SZ; };
@@ -185,11 +190,21 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
     // two threads per position t, each half of the 64 columns; float4 reads
     // rotated by thread so the 8 threads of a quarter-warp hit distinct banks
     const int t = tid >> 1, half = tid & 1;
+    // Waits that are normally complete long before they are reached are taken
+    // one chunk early, off the u -> u step: chunk n's matrices and operand
+    // slot, and the update operand buffer (read by the update MMA of chunk n-2).
+    auto early_waits = [&](int n) {
+      tc::mbar_wait<false>(&aux_full[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      tc::mbar_wait<false>(&slot_full[n % 3], (uint32_t)((n / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      if (n >= 2)
+        tc::mbar_wait<false>(&mma2_bar[n & 1], (uint32_t)(((n - 2) >> 1) & 1), err, tc::kErrTimeoutMma,
+                             &abort_flag);
+    };
+    early_waits(0);
     for (int n = 0; n < NC; ++n) {
       const size_t ch = (size_t)unit * NC + n;
       const int xs = n & 3;
       tc::mbar_wait<true>(&x_bar[xs], (uint32_t)((n >> 2) & 1), err, tc::kErrTimeoutCluster, &abort_flag);
-      tc::mbar_wait<false>(&aux_full[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
       const unsigned char* ax = auxp(n);
       float s = 0.f;
       {
@@ -216,10 +231,7 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
         s += hu;
       }
       // s = b0_n[t] in both threads of the pair
-      if (half == 0) {
-        ws[t] = reinterpret_cast<const float*>(ax + Cf::AX_B)[t] * s;
-        if (rank == 0 && wb0) wb0[ch * C + t] = s;
-      }
+      if (half == 0) ws[t] = reinterpret_cast<const float*>(ax + Cf::AX_B)[t] * s;
       bar_u();  // every thread has read recv[xs]: arm it for chunk n + 4
       if (tid == 0 && n + 4 < NC) tc::mbar_expect_tx(&x_bar[xs], R * 64u * 4u);
       float uval;
@@ -242,20 +254,10 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
         uval = reinterpret_cast<const float*>(ax + Cf::AX_Y)[t] - aw;
       }
       float* un = us + (n & 1) * 64;
-      if (half == 0) {
-        un[t] = uval;
-        if (rank == 0 && wu) wu[ch * C + t] = uval;
-      }
+      if (half == 0) un[t] = uval;
       bar_u();
       if (tid == 0) mbar_arrive(&aux_free[n & 1]);
-      // ---- B2 = diag(u_n) K^e_n slice as bf16 hi + lo (N = NJ rows j, K = 64 positions),
-      //      into buffer n & 1 once the update MMA of chunk n - 2 has read it
-      if (n >= 2)
-        tc::mbar_wait<false>(&mma2_bar[n & 1], (uint32_t)(((n - 2) >> 1) & 1), err, tc::kErrTimeoutMma,
-                             &abort_flag);
-      // chunk n's operand slot has landed (already known through the lookahead's
-      // chain of hand-offs; this wait makes the copy's writes visible here)
-      tc::mbar_wait<false>(&slot_full[n % 3], (uint32_t)((n / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      // ---- B2 = diag(u_n) K^e_n slice as bf16 hi + lo (N = NJ rows j, K = 64 positions)
       {
         constexpr int TQ = 128 / NJ, TPT = C / TQ;  // position groups, positions per thread
         const int jl = tid % NJ, tq = tid / NJ;
@@ -278,6 +280,12 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
       }
       tc::fence_proxy_async();
       mbar_arrive(&b2_full[n & 1]);
+      // the chain's outputs for the backward, off the step: u_n and b0_n
+      if (rank == 0 && half == 0) {
+        if (wu) wu[ch * C + t] = uval;
+        if (wb0) wb0[ch * C + t] = s;
+      }
+      if (n + 1 < NC) early_waits(n + 1);
     }
     // drain: every peer sends all NC partial sums; wait for the last round of
     // each buffer so no peer still writes here once this CTA exits
@@ -285,141 +293,166 @@ __global__ void __launch_bounds__(320, 1) fwd_chain_tc(
       for (int m = NC - 1; m >= 0 && m >= NC - 4; --m) mbar_drain(&x_bar[m & 3], (uint32_t)((m >> 2) & 1));
   } else if (warp < 8) {
     // ============================== state warps ==============================
-    const int r = tid - 128;  // tensor-memory lane = state row
+    const int r = tid - 128;  // state row = tensor-memory lane (lookahead rows: positions)
     const uint32_t my_lanes = tc::tmem_lane_addr(tmem, warp, 0);
-    // the initial state into tensor memory; it is also chunk 0's start state
+    float sreg[NJ];           // row r of the state slice
+    float kt[NJ];             // warps 4-5: row t = r of the next chunk's K~ slice
+    // the state slice's bf16 parts into the lookahead MMA's operand, row r
+    auto write_operand = [&]() {
+      unsigned char* sc = sm + Cf::SC;
+#pragma unroll
+      for (int j8 = 0; j8 < NJ; j8 += 8) {
+        __align__(16) __nv_bfloat16 hi8[8], lo8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          hi8[i] = __float2bfloat16_rn(sreg[j8 + i]);
+          lo8[i] = __float2bfloat16_rn(sreg[j8 + i] - __bfloat162float(hi8[i]));
+        }
+        const uint32_t off = tc::sw128_off(r, j8, 128, 2);
+        *reinterpret_cast<uint4*>(sc + off) = *reinterpret_cast<const uint4*>(hi8);
+        *reinterpret_cast<uint4*>(sc + 16384 + off) = *reinterpret_cast<const uint4*>(lo8);
+      }
+    };
+    // warps 4-5: chunk m's K~ row into registers (overlapping the wait for its
+    // MMA); the swizzled block spreads a quarter-warp's 16-byte reads over all banks
+    auto load_kt = [&](int m) {
+      tc::mbar_wait<false>(&slot_full[m % 3], (uint32_t)((m / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
+      const unsigned char* kb = slot(m) + Cf::SL_KT;
+#pragma unroll
+      for (int q = 0; q < NJ / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(kb + tc::sw128_off(r, j0 - jb + 4 * q, 64, 4));
+        kt[4 * q] = v.x;
+        kt[4 * q + 1] = v.y;
+        kt[4 * q + 2] = v.z;
+        kt[4 * q + 3] = v.w;
+      }
+    };
+    // warps 4-5: c_m partial for position t = r: sum over this CTA's channels of
+    // U[t, j] K~[t, j], sent to every CTA of the cluster
+    auto row_dot_send = [&](int m) {
+      load_kt(m);
+      tc::mbar_wait<false>(&mma1_bar[m & 1], (uint32_t)((m >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      float c0 = 0.f, c1 = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < NJ; jj += 16) {
+        float u16[16];
+        tc::tmem_ld16(my_lanes + Cf::U_COL + (m & 1) * NJ + jj, u16);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          c0 = fmaf(u16[i], kt[jj + i], c0);
+          c1 = fmaf(u16[i + 1], kt[jj + i + 1], c1);
+        }
+      }
+      const float c = c0 + c1;
+      float* rv = recv + (m & 3) * R * 64;
+      const uint32_t la = tc::smem_u32(rv + rank * 64 + r), lb = tc::smem_u32(&x_bar[m & 3]);
+#pragma unroll
+      for (int peer = 0; peer < R; ++peer)
+        tc::st_async_f32(tc::mapa(la, (uint32_t)peer), c, tc::mapa(lb, (uint32_t)peer));
+    };
+    const bool dots = warp < 6;  // lanes 0-63 of the lookahead accumulator are the positions
+    // the initial state: registers and the operand copy (chunk 0's start state)
     {
+#pragma unroll
+      for (int j = 0; j < NJ; j += 4) {
+        const float4 v = S0 ? *reinterpret_cast<const float4*>(S0 + (size_t)unit * D * D + (size_t)r * D + j0 + j)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        sreg[j] = v.x;
+        sreg[j + 1] = v.y;
+        sreg[j + 2] = v.z;
+        sreg[j + 3] = v.w;
+      }
+      write_operand();
+      tc::fence_proxy_async();
+      bar_s();
+      if (r == 0) mbar_arrive(&s_ready);
       const size_t ch0 = (size_t)unit * NC;
       const bool f32copy = wxflags[ch0] != 0;
 #pragma unroll
       for (int jj = 0; jj < NJ; jj += 16) {
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = S0 ? S0[(size_t)unit * D * D + (size_t)r * D + j0 + jj + i] : 0.f;
-        tc::tmem_st16(my_lanes + Cf::S_COL + jj, x);
-        save_bf16_tile(wS0b, ch0, r, j0 + jj, x);
-        if (f32copy) save_f32_tile(wS0blob, ch0, r, j0 + jj, x);
+        save_bf16_tile(wS0b, ch0, r, j0 + jj, sreg + jj);
+        if (f32copy) save_f32_tile(wS0blob, ch0, r, j0 + jj, sreg + jj);
       }
-      tc::tmem_st_wait();
-      tc::tc_before_sync();
-      bar_s();
-      if (r == 0) mbar_arrive(&s_ready);
     }
-    // c_m partial: sum_r V_m[t,r] X'_m[r,t] over this CTA's rows, then sent to every CTA
-    auto column_dot_send = [&](int m) {
-      tc::mbar_wait<false>(&slot_full[m % 3], (uint32_t)((m / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
-      tc::mbar_wait<false>(&mma1_bar[m & 1], (uint32_t)((m >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
-      tc::tc_after_sync();
-      {
-        float x[64];
-#pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          float y16[16];
-          tc::tmem_ld16(my_lanes + Cf::X_COL + (m & 1) * 64 + 16 * c16, y16);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) x[16 * c16 + i] = y16[i];
-        }
-        tc::tmem_ld_wait();
-        const unsigned char* vt = slot(m) + Cf::SL_V;  // row r of V^T: V[t, r] for t = 0..63
-        float lo[32], hi[32];
-#pragma unroll
-        for (int g8 = 0; g8 < 8; ++g8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(vt + tc::sw128_off(r, 8 * g8, 128, 2));
-          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int tt = 8 * g8 + i;
-            if (tt < 32) lo[tt] = x[tt] * __bfloat162float(e[i]);
-            else hi[tt - 32] = x[tt] * __bfloat162float(e[i]);
-          }
-        }
-        warp_transpose_reduce<32>(lo, lane);
-        warp_transpose_reduce<32>(hi, lane);
-        xred[(warp & 3) * 64 + lane] = lo[0];
-        xred[(warp & 3) * 64 + 32 + lane] = hi[0];
-      }
-      tc::tc_before_sync();
-      bar_s();
-      if (r < C) mine[r] = (xred[r] + xred[64 + r]) + (xred[128 + r] + xred[192 + r]);
-      bar_s();
-      if (r < 16 * R) {
-        const int peer = r / 16, q4 = r % 16;
-        const float4 val = *reinterpret_cast<const float4*>(mine + 4 * q4);
-        float* rv = recv + (m & 3) * R * 64;
-        const uint32_t raddr = tc::mapa(tc::smem_u32(rv + rank * 64 + 4 * q4), (uint32_t)peer);
-        const uint32_t rbar = tc::mapa(tc::smem_u32(&x_bar[m & 3]), (uint32_t)peer);
-        tc::st_async_v4(raddr, val, rbar);
-      }
-    };
-    column_dot_send(0);
-    if (NC > 1) column_dot_send(1);
+    if (dots) {
+      row_dot_send(0);
+      if (NC > 1) row_dot_send(1);
+    }
     for (int n = 0; n < NC; ++n) {
-      const unsigned char* st = slot(n);
+      const float* gC = reinterpret_cast<const float*>(slot(n) + Cf::SL_GC);
       tc::mbar_wait<false>(&mma2_bar[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
-      // ---- S_{n+1} = S_n diag(gamma_C) + dS_n; saved as chunk n+1's start state (or S_T)
-      {
-        const float* gC = reinterpret_cast<const float*>(st + Cf::SL_GC);
-        const size_t chn = (size_t)unit * NC + n + 1;
-        const bool f32copy = n + 1 < NC && wxflags[chn] != 0;
+      // ---- S_{n+1} = S_n diag(gamma_C) + dS_n
 #pragma unroll
-        for (int jj = 0; jj < NJ; jj += 16) {
-          float s[16], d2[16];
-          tc::tmem_ld16(my_lanes + Cf::S_COL + jj, s);
-          tc::tmem_ld16(my_lanes + Cf::D2_COL + (n & 1) * NJ + jj, d2);
-          tc::tmem_ld_wait();
+      for (int jj = 0; jj < NJ; jj += 16) {
+        float d2[16];
+        tc::tmem_ld16(my_lanes + Cf::D2_COL + (n & 1) * NJ + jj, d2);
+        tc::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) s[i] = fmaf(s[i], gC[jj + i], d2[i]);
-          tc::tmem_st16(my_lanes + Cf::S_COL + jj, s);
-          if (n + 1 < NC) {
-            save_bf16_tile(wS0b, chn, r, j0 + jj, s);
-            if (f32copy) save_f32_tile(wS0blob, chn, r, j0 + jj, s);
-          } else if (ST) {
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4)
-              *reinterpret_cast<float4*>(ST + (size_t)unit * D * D + (size_t)r * D + j0 + jj + 4 * i4) =
-                  make_float4(s[4 * i4], s[4 * i4 + 1], s[4 * i4 + 2], s[4 * i4 + 3]);
-          }
-        }
-        tc::tmem_st_wait();
+        for (int i = 0; i < 16; ++i) sreg[jj + i] = fmaf(sreg[jj + i], gC[jj + i], d2[i]);
       }
+      if (n + 2 < NC) write_operand();  // read by the lookahead MMA of chunk n + 2
+      tc::fence_proxy_async();
       tc::tc_before_sync();
       bar_s();
       if (r == 0) {
         mbar_arrive(&slot_free[n % 3]);
         mbar_arrive(&s_ready);
       }
-      // ---- c_{n+2} from X'_{n+2} = S_{n+1} K~_{n+2}^T
-      if (n + 2 < NC) column_dot_send(n + 2);
+      // ---- c_{n+2}
+      if (dots && n + 2 < NC) row_dot_send(n + 2);
+      // ---- saved as chunk n+1's start state (or S_T), off the step
+      if (n + 1 < NC) {
+        const size_t chn = (size_t)unit * NC + n + 1;
+        const bool f32copy = wxflags[chn] != 0;
+#pragma unroll
+        for (int jj = 0; jj < NJ; jj += 16) {
+          save_bf16_tile(wS0b, chn, r, j0 + jj, sreg + jj);
+          if (f32copy) save_f32_tile(wS0blob, chn, r, j0 + jj, sreg + jj);
+        }
+      } else if (ST) {
+#pragma unroll
+        for (int j = 0; j < NJ; j += 4)
+          *reinterpret_cast<float4*>(ST + (size_t)unit * D * D + (size_t)r * D + j0 + j) =
+              make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
+      }
     }
   } else if (warp == 8) {
     // ================================ issuer ================================
-    const uint32_t ID1 = tc::idesc(128, 64, 2);  // tf32: M = 128 rows r, N = 64 positions
-    const uint32_t ID2 = tc::idesc(128, NJ, 1);  // bf16: M = 128 rows r, N = NJ channels
-    // X'_m = S_{m-1} K~_m^T (K = NJ channels; A = the state in tensor memory)
-    auto issue_x = [&](int m) {
+    // lookahead U_m = V_m S_{m-1}^T: A = V^T read MN-major (M = 128 positions,
+    // rows 64-127 are unused), B = the state operand read MN-major (N = NJ
+    // channels), K = 128 value channels, hi and lo parts
+    const uint32_t IDU = tc::idesc(128, NJ, 1) | tc::kMajorA | tc::kMajorB;
+    const uint32_t ID2 = tc::idesc(128, NJ, 1);  // bf16: M = 128 rows r, N = NJ channels, both K-major
+    auto issue_u = [&](int m) {
       tc::mbar_wait<false>(&slot_full[m % 3], (uint32_t)((m / 3) & 1), err, tc::kErrTimeoutLoad, &abort_flag);
       tc::tc_after_sync();
       if (lane == 0) {
-        const unsigned char* st = slot(m);
+        const unsigned char* vt = slot(m) + Cf::SL_V;
 #pragma unroll
-        for (int ks = 0; ks < NJ / 8; ++ks) {
-          const uint64_t bd = tc::desc_sw128(tc::smem_u32(st + Cf::SL_KT + (Cf::KBJ * (rank & 1) + ks) * 32));
-          tc::mma_tf32_ts(tmem + Cf::X_COL + (m & 1) * 64, tmem + Cf::S_COL + ks * 8, bd, ID1, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks) {
+          // second 64-position block of A: the next 16 KB of the slot (in bounds, results unused)
+          const uint64_t ad = tc::desc_sw128_mn(tc::smem_u32(vt + ks * 2048), 16384u);
+          tc::mma_bf16_ss(tmem + Cf::U_COL + (m & 1) * NJ, ad,
+                          tc::desc_sw128_mn(tc::smem_u32(sm + Cf::SC + ks * 2048), 16384u), IDU, ks > 0 ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + Cf::U_COL + (m & 1) * NJ, ad,
+                          tc::desc_sw128_mn(tc::smem_u32(sm + Cf::SC + 16384 + ks * 2048), 16384u), IDU, 1u);
         }
         tc::mma_commit(&mma1_bar[m & 1]);
       }
       __syncwarp();
     };
-    tc::mbar_wait<false>(&s_ready, 0u, err, tc::kErrTimeoutMma, &abort_flag);  // S_0 in tensor memory
+    tc::mbar_wait<false>(&s_ready, 0u, err, tc::kErrTimeoutMma, &abort_flag);  // S_0's operand
     tc::tc_after_sync();
-    issue_x(0);
-    if (NC > 1) issue_x(1);
+    issue_u(0);
+    if (NC > 1) issue_u(1);
     for (int n = 0; n < NC; ++n) {
       if (n >= 1 && n + 1 < NC) {
         tc::mbar_wait<false>(&s_ready, (uint32_t)(n & 1), err, tc::kErrTimeoutMma, &abort_flag);  // S_n
         tc::tc_after_sync();
-        issue_x(n + 1);
+        issue_u(n + 1);
       }
       tc::mbar_wait<false>(&b2_full[n & 1], (uint32_t)((n >> 1) & 1), err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();

@@ -60,11 +60,13 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t lbo) 
 }
 
 // Instruction descriptor: dense, fp32 accumulator, A and B K-major.
-// fmt: 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32).
+// fmt: 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32).  OR in kMajorA / kMajorB
+// for an MN-major A / B operand.
 __host__ __device__ constexpr uint32_t idesc(int M, int N, int fmt) {
   return (1u << 4) | (static_cast<uint32_t>(fmt) << 7) | (static_cast<uint32_t>(fmt) << 10) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
+constexpr uint32_t kMajorA = 1u << 15, kMajorB = 1u << 16;
 
 // ---- fences ---------------------------------------------------------------
 __device__ __forceinline__ void fence_proxy_async() {
@@ -262,6 +264,12 @@ __device__ __forceinline__ void st_async_v4(uint32_t raddr, float4 v, uint32_t r
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(raddr),
       "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar)
       : "memory");
+}
+// 4-byte form of the same
+__device__ __forceinline__ void st_async_f32(uint32_t raddr, float v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(raddr),
+               "r"(__float_as_uint(v)), "r"(rbar)
+               : "memory");
 }
 
 }  // namespace tc
