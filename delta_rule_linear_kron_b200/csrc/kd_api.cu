@@ -81,13 +81,16 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   off = 0;
   L->dSC = L->tc ? 0 : take(chunks * (size_t)dv * dk * 4);  // the tensor-core path keeps bf16 tiles
   L->g = take(chunks * C * 4);
-  L->dP = take(chunks * C * C * 4);
-  L->dGK = take(chunks * C * C * 4);
-  L->dGVs = take(chunks * C * C * 4);
-  L->accq = take(chunks * C * dk * 4);
-  L->acck = take(chunks * C * dk * 4);
-  L->accL = take(chunks * C * dk * 4);
-  L->accv = take(chunks * C * dv * 4);
+  // exact-path scratch: every chunk on the CUDA-core path; on the tensor-core
+  // path only the flagged chunks use it, one kExactSlots slot per CTA
+  const size_t slots = L->tc ? (chunks < (size_t)kd::kExactSlots ? chunks : (size_t)kd::kExactSlots) : chunks;
+  L->dP = take(slots * C * C * 4);
+  L->dGK = take(slots * C * C * 4);
+  L->dGVs = take(slots * C * C * 4);
+  L->accq = take(slots * C * dk * 4);
+  L->acck = take(slots * C * dk * 4);
+  L->accL = take(slots * C * dk * 4);
+  L->accv = take(slots * C * dv * 4);
   L->du = take(chunks * C * 4);
   if (L->tc) {
     L->dSCb = take(chunks * (size_t)dv * dk * 2);

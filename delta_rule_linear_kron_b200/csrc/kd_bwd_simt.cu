@@ -167,13 +167,17 @@ constexpr size_t bcc_smem_floats() {
   return 3 * (size_t)C * (DK + 1) + 2 * (size_t)C * (DV + 1) + (size_t)C * (C + 1) + 4 * C;
 }
 
+// Stage bodies take the chunk (n, h, b) and the scratch slot their dP, dG_K,
+// dG_V' and accumulator tiles use: the chunk index on the CUDA-core path,
+// a per-CTA slot in the tensor-core path's exact kernel.
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) bwd_cc_simt(
+__device__ __forceinline__ void bwd_cc_body(
+    int n, int h, int b, size_t slot,
     const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ beta,
     const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T, int NC,
     const float* __restrict__ wu, const float* __restrict__ wb0, const float* __restrict__ wg,
     float* __restrict__ dbeta, float* __restrict__ dc, float* __restrict__ wdP,
-    float* __restrict__ wdGK, float* __restrict__ wdGVs, const int* __restrict__ only) {
+    float* __restrict__ wdGK, float* __restrict__ wdGVs) {
   constexpr int SK = DK + 1, SV = DV + 1, SC = C + 1;
   extern __shared__ float smem[];
   float* Kp = smem;            // [C][SK]
@@ -187,10 +191,9 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
   float* bs = gs + C;
   float* b0s = bs + C;
   __shared__ int unsafe;
-  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)b * H + h) * NC + n;
-  if (only && only[ch] == 0) return;  // only the chunks flagged by the tensor-core kernel
 
   for (int e = tid; e < C * DK; e += blockDim.x) {
     const int t = e / DK, j = e % DK;
@@ -255,8 +258,8 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
       const float mm = i < t ? gk * gv : 0.f;
       brow = fmaf(mm, us[i], brow);
       const float dM = i < t ? -bs[t] * gs[t] * us[i] : 0.f;
-      wdP[ch * C * C + t * C + i] = i <= t ? us[i] * dov : 0.f;
-      wdGK[ch * C * C + t * C + i] = dM * gv;
+      wdP[slot * C * C + t * C + i] = i <= t ? us[i] * dov : 0.f;
+      wdGK[slot * C * C + t * C + i] = dM * gv;
       dGV[t * SC + i] = dM * gk;
     }
     brow = warp_sum(brow);
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
   __syncthreads();
   for (int e = tid; e < C * C; e += blockDim.x) {
     const int t = e / C, i = e % C;
-    wdGVs[ch * C * C + e] = dGV[t * SC + i] + dGV[i * SC + t];
+    wdGVs[slot * C * C + e] = dGV[t * SC + i] + dGV[i * SC + t];
   }
 }
 
@@ -302,13 +305,14 @@ constexpr size_t bstate_smem_floats() {
 }
 
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) bwd_state_simt(
+__device__ __forceinline__ void bwd_state_body(
+    int n, int h, int b, size_t slot,
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     const float* __restrict__ beta, const float* __restrict__ logf, const Tin* __restrict__ dO,
     int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wg,
     const float* __restrict__ wS0, const float* __restrict__ wdSC, float* __restrict__ waccq,
     float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv, int s0_swizzled,
-    const __nv_bfloat16* __restrict__ wdSb, const int* __restrict__ only) {
+    const __nv_bfloat16* __restrict__ wdSb) {
   constexpr int SK = DK + 1, SV = DV + 1;
   constexpr int TPJ = 256 / DK;   // thread groups over j
   constexpr int TPG = C / TPJ;    // rows per group
@@ -326,10 +330,9 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
   float* gC = csum + DK;          // [DK]
   float* lastL = gC + DK;         // [DK]
   float* ekL = lastL + DK;        // per-group partials [256/DK][DK]
-  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)b * H + h) * NC + n;
-  if (only && only[ch] == 0) return;  // only the chunks flagged by the tensor-core kernel
 
   for (int e = tid; e < C * DK; e += blockDim.x) {
     const int t = e / DK, j = e % DK;
@@ -409,7 +412,7 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
           kps = fmaf(Kp[t * SK + jj], S0s[rr * SK + jj], kps);
           keds = fmaf(Ke[t * SK + jj], dSs[rr * SK + jj], keds);
         }
-        waccv[ch * C * DV + (size_t)t * DV + r0 + rr] = db0s[t] * kps + us[t] * keds;
+        waccv[slot * C * DV + (size_t)t * DV + r0 + rr] = db0s[t] * kps + us[t] * keds;
       }
     }
     __syncthreads();
@@ -423,7 +426,7 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
     const float gam = expf(l), eC = expf(Ls[(C - 1) * SK + j] - l);
     const float qv = t < nv ? to_f(q[(((size_t)b * T + t0 + t) * H + h) * DK + j]) : 0.f;
     const float dKp = db0s[t] * aVS[i], dKe = us[t] * aVD[i];
-    const size_t o = ch * C * DK + (size_t)t * DK + j;
+    const size_t o = slot * C * DK + (size_t)t * DK + j;
     waccq[o] = aQ[i] * gam;
     wacck[o] = dKp * gam + dKe * eC;
     const float keT = Ke[t * SK + j];
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
   if (tid < DK) {
     float e = 0.f;
     for (int g2 = 0; g2 < TPJ; ++g2) e += ekL[g2 * DK + tid];  // fixed order: deterministic
-    waccL[ch * C * DK + (size_t)(C - 1) * DK + tid] = lastL[tid] + e + gC[tid] * csum[tid];
+    waccL[slot * C * DK + (size_t)(C - 1) * DK + tid] = lastL[tid] + e + gC[tid] * csum[tid];
   }
 }
 
@@ -452,23 +455,23 @@ constexpr size_t bintra_smem_floats() {
 }
 
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(256) bwd_intra_simt(
+__device__ __forceinline__ void bwd_intra_body(
+    int n, int h, int b, size_t slot,
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T, int NC,
     const float* __restrict__ wP, const float* __restrict__ wu, const float* __restrict__ wdP,
     const float* __restrict__ wdGK, const float* __restrict__ wdGVs,
     const float* __restrict__ waccq, const float* __restrict__ wacck,
     const float* __restrict__ waccL, const float* __restrict__ waccv, Tin* __restrict__ dq,
-    Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf, const int* __restrict__ only) {
+    Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf) {
   constexpr int SK = DK + 1, SV = DV + 1, SC = C + 1;
   extern __shared__ float smem[];
   float* us = smem;            // [C]
   float* base = smem + C;
   __shared__ int unsafe;
-  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)b * H + h) * NC + n;
-  if (only && only[ch] == 0) return;  // only the chunks flagged by the tensor-core kernel
 
   // ---- phase A: dv = accv + u o (P^T dO) + (dG_V + dG_V^T) V
   {
@@ -478,7 +481,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
     float* Ds = Vs + C * SV;
     for (int e = tid; e < C * C; e += blockDim.x) {
       Ps[(e / C) * SC + e % C] = wP[ch * C * C + e];
-      Gs[(e / C) * SC + e % C] = wdGVs[ch * C * C + e];
+      Gs[(e / C) * SC + e % C] = wdGVs[slot * C * C + e];
     }
     for (int e = tid; e < C * DV; e += blockDim.x) {
       const int t = e / DV, rr = e % DV;
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
       for (int t = 0; t < C; ++t) s = fmaf(Gs[i * SC + t], Vs[t * SV + rr], s);
       if (i < nv) {
         const size_t o = (((size_t)b * T + t0 + i) * H + h) * DV + rr;
-        dv[o] = from_f<Tin>(waccv[ch * C * DV + (size_t)i * DV + rr] + us[i] * a + s);
+        dv[o] = from_f<Tin>(waccv[slot * C * DV + (size_t)i * DV + rr] + us[i] * a + s);
       }
     }
     __syncthreads();
@@ -519,8 +522,8 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
     Ls[t * SK + j] = ok ? logf[g] : 0.f;
   }
   for (int e = tid; e < C * C; e += blockDim.x) {
-    dPs[(e / C) * SC + e % C] = wdP[ch * C * C + e];
-    dGs[(e / C) * SC + e % C] = wdGK[ch * C * C + e];
+    dPs[(e / C) * SC + e % C] = wdP[slot * C * C + e];
+    dGs[(e / C) * SC + e % C] = wdGK[slot * C * C + e];
   }
   __syncthreads();
   if (tid < DK) {
@@ -589,7 +592,7 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
         }
       }
     }
-    const size_t o = ch * C * DK + (size_t)t * DK + j;
+    const size_t o = slot * C * DK + (size_t)t * DK + j;
     const float dqv = waccq[o] + dqP;
     const float dkv = wacck[o] + dkP + dkG1 + dkG2;
     dLv[i] = waccL[o] + qraw[i] * dqP - kraw[i] * dkP + kraw[i] * dkG1 - kraw[i] * dkG2;
@@ -612,6 +615,75 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
   }
 }
 
+// The CUDA-core path: one CTA per chunk for each stage, scratch indexed by chunk.
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256) bwd_cc_simt(
+    const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ beta,
+    const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T, int NC,
+    const float* __restrict__ wu, const float* __restrict__ wb0, const float* __restrict__ wg,
+    float* __restrict__ dbeta, float* __restrict__ dc, float* __restrict__ wdP,
+    float* __restrict__ wdGK, float* __restrict__ wdGVs) {
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  bwd_cc_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, k, v, beta, logf, dO, H, T, NC, wu, wb0, wg,
+                           dbeta, dc, wdP, wdGK, wdGVs);
+}
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256) bwd_state_simt(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    const float* __restrict__ beta, const float* __restrict__ logf, const Tin* __restrict__ dO,
+    int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wg,
+    const float* __restrict__ wS0, const float* __restrict__ wdSC, float* __restrict__ waccq,
+    float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv) {
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  bwd_state_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, q, k, v, beta, logf, dO, H, T, NC, wu, wg,
+                              wS0, wdSC, waccq, wacck, waccL, waccv, 0, nullptr);
+}
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256) bwd_intra_simt(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T, int NC,
+    const float* __restrict__ wP, const float* __restrict__ wu, const float* __restrict__ wdP,
+    const float* __restrict__ wdGK, const float* __restrict__ wdGVs,
+    const float* __restrict__ waccq, const float* __restrict__ wacck,
+    const float* __restrict__ waccL, const float* __restrict__ waccv, Tin* __restrict__ dq,
+    Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf) {
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  bwd_intra_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, q, k, v, logf, dO, H, T, NC, wP, wu, wdP,
+                              wdGK, wdGVs, waccq, wacck, waccL, waccv, dq, dk, dv, dlogf);
+}
+
+// The tensor-core path's exact recomputation of the chunks the per-chunk
+// kernels flagged (in-chunk |L| beyond their factorised range): the three
+// stages in one CTA, chunk after chunk, each CTA with its own scratch slot.
+// Unflagged chunks are skipped, so the kernel is nearly free when none is
+// flagged, and the scratch is sized by the number of CTAs, not of chunks.
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256) bwd_exact_simt(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    const float* __restrict__ beta, const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T,
+    int NC, size_t chunks, const float* __restrict__ wP, const float* __restrict__ wu,
+    const float* __restrict__ wb0, const float* __restrict__ wg, const float* __restrict__ wS0,
+    const __nv_bfloat16* __restrict__ wdSb, float* __restrict__ dbeta, float* __restrict__ dc,
+    float* __restrict__ wdP, float* __restrict__ wdGK, float* __restrict__ wdGVs, float* __restrict__ waccq,
+    float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv, Tin* __restrict__ dq,
+    Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf, const int* __restrict__ only) {
+  const size_t slot = blockIdx.x;
+  for (size_t ch = blockIdx.x; ch < chunks; ch += gridDim.x) {
+    if (only[ch] == 0) continue;  // uniform across the CTA
+    const int n = static_cast<int>(ch % NC), u = static_cast<int>(ch / NC);
+    const int h = u % H, b = u / H;
+    bwd_cc_body<DK, DV, Tin>(n, h, b, slot, k, v, beta, logf, dO, H, T, NC, wu, wb0, wg, dbeta, dc, wdP, wdGK,
+                             wdGVs);
+    __syncthreads();
+    bwd_state_body<DK, DV, Tin>(n, h, b, slot, q, k, v, beta, logf, dO, H, T, NC, wu, wg, wS0, nullptr, waccq,
+                                wacck, waccL, waccv, 1, wdSb);
+    __syncthreads();
+    bwd_intra_body<DK, DV, Tin>(n, h, b, slot, q, k, v, logf, dO, H, T, NC, wP, wu, wdP, wdGK, wdGVs, waccq,
+                                wacck, waccL, waccv, dq, dk, dv, dlogf);
+    __syncthreads();
+  }
+}
+
 template <int DK, int DV, typename Tin>
 static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaStream_t st) {
   const Layout& L = a.L;
@@ -626,6 +698,8 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
   KD_ATTR((bwd_cc_simt<DK, DV, Tin>), s2)
   KD_ATTR((bwd_state_simt<DK, DV, Tin>), s3)
   KD_ATTR((bwd_intra_simt<DK, DV, Tin>), s4)
+  const size_t s5 = s2 > s3 ? (s2 > s4 ? s2 : s4) : (s3 > s4 ? s3 : s4);
+  KD_ATTR((bwd_exact_simt<DK, DV, Tin>), s5)
 #undef KD_ATTR
   const Tin* q = static_cast<const Tin*>(a.q);
   const Tin* k = static_cast<const Tin*>(a.k);
@@ -653,27 +727,37 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (only) {
+    // tensor-core path: the flagged chunks only, all stages in one kernel
+    if (stages != (kStageCC | kStageState | kStageIntra)) return cudaErrorInvalidValue;
+    prof_begin(st, "bwd_exact_simt");
+    bwd_exact_simt<DK, DV, Tin><<<(unsigned)(L.chunks < (size_t)kExactSlots ? L.chunks : kExactSlots), 256, s5,
+                                  st>>>(
+        q, k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, L.chunks, wP, wu, wb0, wg, wS0,
+        ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), a.dbeta, a.dc, wdP, wdGK, wdGVs, waccq, wacck, waccL, waccv,
+        static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf, only);
+    prof_end(st);
+    return cudaGetLastError();
+  }
   if (stages & kStageCC) {
     prof_begin(st, "bwd_cc_simt");
     bwd_cc_simt<DK, DV, Tin><<<gridc, 256, s2, st>>>(k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, wu,
-                                                     wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs, only);
+                                                     wb0, wg, a.dbeta, a.dc, wdP, wdGK, wdGVs);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (stages & kStageState) {
-  prof_begin(st, "bwd_state_simt");
-  bwd_state_simt<DK, DV, Tin><<<gridc, 256, s3, st>>>(q, k, v, a.beta, a.logf, dO, L.H, L.T,
-                                                      L.NC, wu, wg, wS0, wdSC, waccq, wacck,
-                                                      waccL, waccv, L.tc ? 1 : 0,
-                                                      L.tc ? ws_ptr<__nv_bfloat16>(a.ws, L.dSCb) : nullptr, only);
-  prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    prof_begin(st, "bwd_state_simt");
+    bwd_state_simt<DK, DV, Tin><<<gridc, 256, s3, st>>>(q, k, v, a.beta, a.logf, dO, L.H, L.T, L.NC, wu, wg,
+                                                        wS0, wdSC, waccq, wacck, waccL, waccv);
+    prof_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (!(stages & kStageIntra)) return cudaSuccess;
   prof_begin(st, "bwd_intra_simt");
   bwd_intra_simt<DK, DV, Tin><<<gridc, 256, s4, st>>>(
       q, k, v, a.logf, dO, L.H, L.T, L.NC, wP, wu, wdP, wdGK, wdGVs, waccq, wacck, waccL, waccv,
-      static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf, only);
+      static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf);
   prof_end(st);
   return cudaGetLastError();
 }

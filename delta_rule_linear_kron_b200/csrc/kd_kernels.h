@@ -13,6 +13,11 @@ namespace kd {
 // inverse is built by forward substitution).
 constexpr int kChunk = 64;
 
+// Scratch slots of the tensor-core backward's exact recomputation (the CTAs
+// of bwd_exact_simt): its per-chunk scratch is sized by this, not by the
+// number of chunks.
+constexpr int kExactSlots = 128;
+
 // Workspace layout of one problem (B, H, T, dk, dv), decided by the chunk
 // scheduler.  Offsets are in bytes from the workspace base, 256-byte aligned.
 // "chunk" index ch = ((b * H) + h) * NC + n.
@@ -39,8 +44,9 @@ struct Layout {
   // tiles [r][j] (rows r, K = j), read by the output kernel and the backward
   size_t S0b = 0;
   size_t fwd_save_bytes = 0;
-  // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [ch][64][64],
-  // accq/acck/accL [ch][64][dk], accv [ch][64][dv]
+  // backward scratch: dSC [ch][dv][dk], g [ch][64], dP/dGK/dGVs [slot][64][64],
+  // accq/acck/accL [slot][64][dk], accv [slot][64][dv] (slot = chunk on the
+  // CUDA-core path; on the tensor-core path one of kExactSlots slots)
   size_t dSC = 0, g = 0, dP = 0, dGK = 0, dGVs = 0, accq = 0, acck = 0, accL = 0, accv = 0;
   size_t du = 0;  // per-chunk intra-chunk part of du (tensor-core path) [ch][64]
   size_t dSCb = 0;    // tensor-core path: dS per chunk as a bf16 tile (as S0b)
