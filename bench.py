@@ -338,6 +338,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-fwd", action="store_true")
+    ap.add_argument("--no-gated", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-gdn2", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -465,6 +466,46 @@ def main(argv=None):
             fwd_lines[key] = fl
             del fd, fo, fST, fw
         kd.device_status()
+
+    # ---- the same step with gated inputs: the forget gate as its bf16
+    # pre-activation f_pre and a per-head exponent a_log, logf = e^a_log log
+    # sigma(f_pre) formed inside the chunk kernels and df_pre, da_log in their
+    # epilogues (fwd_gated(save) + bwd_gated), timed on its own ----------------
+    gated = None
+    if not args.no_gated:
+        g_ = torch.Generator(device=dev)
+        g_.manual_seed(rank_seed(3004, rank))
+        f_pre = (torch.randn((B, T, H, dk), generator=g_, device=dev) + 3.0).to(bf)
+        a_log = torch.rand((H,), generator=g_, device=dev) * 2 - 1
+        gfw = torch.empty(kd.workspace_size(kd.KD_WS_FWD_GATED, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+        gbw = torch.empty(kd.workspace_size(kd.KD_WS_BWD_GATED, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+
+        def gated_step():
+            kd.fwd_gated(d["q"], d["k"], d["v"], d["beta"], d["c"], f_pre, a_log, d["S0"], out=out, save=True,
+                         workspace=gfw)
+            kd.bwd_gated(d["q"], d["k"], d["v"], d["beta"], d["c"], f_pre, a_log, d["S0"], d["dO"],
+                         fwd_workspace=gfw, workspace=gbw)
+        for _ in range(max(3, args.warmup)):
+            gated_step()
+        torch.cuda.synchronize()
+        barrier()
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for _ in range(args.steps):
+            gated_step()
+        q1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        qms = max_over_ranks(q0.elapsed_time(q1), ws_n, dev) / args.steps
+        kd.device_status()
+        # inputs a step uploads: the plain step's with bf16 f_pre and a_log in place of fp32 logf
+        h2d_plain = sum(t.numel() * t.element_size() for t in host.values())
+        h2d_gated = (h2d_plain - host["logf"].numel() * host["logf"].element_size()
+                     + f_pre.numel() * f_pre.element_size() + a_log.numel() * a_log.element_size())
+        gated = dict(ms=qms, tokens_per_s=job_throughput(ws_n, B * T, 1, qms),
+                     input_bytes_per_step=h2d_gated, plain_input_bytes_per_step=h2d_plain,
+                     step="fwd_gated(save) + bwd_gated (bf16 f_pre, fp32 a_log [H]; outputs df_pre, da_log)")
+        del f_pre, a_log, gfw, gbw
 
     # ---- decode: 1000 consecutive in-place steps --------------------------
     decode = None
@@ -765,6 +806,7 @@ def main(argv=None):
                 # compact summaries last (a truncated tail of the line keeps them)
                 "roofline_step": roofline_step,
                 "fwd_long": fwd_lines.get("fwd_long"), "fwd_B4": fwd_lines.get("fwd_B4"),
+                "gated_step": gated,
                 "gdn2_step": None if gdn2 is None else dict(ms=gdn2["ms_per_step"], tokens_per_s=gdn2["value"],
                                                             decode_gbs=gdn2["decode"]["value"],
                                                             decode_hbm_frac=gdn2["decode"]["hbm_frac"]),

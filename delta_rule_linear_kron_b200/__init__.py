@@ -15,7 +15,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["fwd", "bwd", "decode", "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
+__all__ = ["fwd", "bwd", "decode", "fwd_gated", "bwd_gated",
+           "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
            "gdn2_fwd", "gdn2_bwd", "gdn2_decode",
            "workspace_size", "device_status", "library_path",
            "KronDeltaError", "KronDeltaFunction", "PrologueFunction", "EpilogueFunction", "Gdn2Function",
@@ -29,6 +30,7 @@ KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE, KD_ERR_CUDA, KD
 KD_F32, KD_BF16 = 0, 1
 KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD, KD_WS_EPILOGUE_BWD = 0, 1, 2, 3, 4
 KD_WS_GDN2_FWD, KD_WS_GDN2_BWD = 5, 6
+KD_WS_FWD_GATED, KD_WS_BWD_GATED, KD_WS_BWD_RECOMPUTE = 7, 8, 9
 KD_PHASE_LOCAL, KD_PHASE_CARRY, KD_PHASE_ALL = 1, 2, 3
 _CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
           4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
@@ -71,6 +73,12 @@ def lib():
         L.kron_delta_bwd_phase.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp, sz, i, vp]
         L.kron_delta_fwd_noalloc.restype = i
         L.kron_delta_fwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [vp]
+        L.kron_delta_bwd_recompute.restype = i
+        L.kron_delta_bwd_recompute.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
+        L.kron_delta_fwd_gated.restype = i
+        L.kron_delta_fwd_gated.argtypes = [vp] * 10 + [i] * 6 + [vp, sz, i, vp]
+        L.kron_delta_bwd_gated.restype = i
+        L.kron_delta_bwd_gated.argtypes = [vp] * 18 + [i] * 6 + [vp, sz, vp, sz, vp]
         L.kron_delta_prologue_fwd.restype = i
         L.kron_delta_prologue_fwd.argtypes = [vp] * 7 + [ctypes.c_float] + [vp] * 6 + [i] * 6 + [vp]
         L.kron_delta_prologue_bwd.restype = i
@@ -181,6 +189,9 @@ def bwd(q, k, v, beta, c, logf, S0, dO, dST=None, *, fwd_workspace, workspace=No
         want_dS0=True, phase=KD_PHASE_ALL, grads=None, stream=None):
     """Backward for loss <dO, out> + <dST, ST>, reading what fwd(save=True)
     left in fwd_workspace.  Returns dict dq, dk, dv, dbeta, dc, dlogf, dS0.
+    fwd_workspace=None recomputes the forward's chunk quantities instead
+    (kron_delta_bwd_recompute; the workspace is then sized by
+    KD_WS_BWD_RECOMPUTE and phase must be KD_PHASE_ALL).
     phase: KD_PHASE_LOCAL enqueues only the dST-independent work, KD_PHASE_CARRY
     the rest (allocate the workspace with workspace_size(KD_WS_BWD, ...) and pass
     it, and the LOCAL call's returned grads, to both calls)."""
@@ -202,6 +213,17 @@ def bwd(q, k, v, beta, c, logf, S0, dO, dST=None, *, fwd_workspace, workspace=No
         for n, ref in (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta), ("dc", c), ("dlogf", logf)):
             _need(g[n], n, ref.dtype, ref.shape)
         _need(g.get("dS0"), "dS0", f32, (B, H, dv, dk))
+    if fwd_workspace is None:
+        if phase != KD_PHASE_ALL:
+            raise ValueError("recompute (fwd_workspace=None) needs phase=KD_PHASE_ALL")
+        if workspace is None:
+            workspace = _alloc_ws(workspace_size(KD_WS_BWD_RECOMPUTE, B, H, T, dk, dv, dt), q.device)
+        _check(lib().kron_delta_bwd_recompute(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(logf),
+                                              _ptr(S0), _ptr(dO), _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]),
+                                              _ptr(g["dv"]), _ptr(g["dbeta"]), _ptr(g["dc"]), _ptr(g["dlogf"]),
+                                              _ptr(g.get("dS0")), B, H, T, dk, dv, dt, _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(stream)))
+        return g
     need = workspace_size(KD_WS_BWD, B, H, T, dk, dv, dt)
     if workspace is None:
         workspace = _alloc_ws(need, q.device)
@@ -211,6 +233,67 @@ def bwd(q, k, v, beta, c, logf, S0, dO, dST=None, *, fwd_workspace, workspace=No
                                       B, H, T, dk, dv, dt, _ptr(fwd_workspace),
                                       fwd_workspace.numel() * fwd_workspace.element_size(),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(), int(phase),
+                                      _stream(stream)))
+    return g
+
+
+def fwd_gated(q, k, v, beta, c, f_pre, a_log, S0=None, *, out=None, want_state=True, save=False,
+              workspace=None, stream=None):
+    """Forward with the forget gate given as its pre-activation: identical to
+    fwd on logf = exp(a_log) * log sigmoid(f_pre), with logf formed inside the
+    kernels.  f_pre [B,T,H,dk] in q's dtype; a_log [H] fp32.  Returns (out, ST,
+    workspace); pass the workspace (save=True) to bwd_gated."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(beta, "beta", f32, (B, T, H)); _need(c, "c", f32, (B, T, H))
+    _need(f_pre, "f_pre", q.dtype, (B, T, H, dk)); _need(a_log, "a_log", f32, (H,))
+    _need(S0, "S0", f32, (B, H, dv, dk))
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype, (B, T, H, dv))
+    ST = torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_state else None
+    need = workspace_size(KD_WS_FWD_GATED, B, H, T, dk, dv, dt)
+    if workspace is None:
+        workspace = _alloc_ws(need, q.device)
+    _check(lib().kron_delta_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(f_pre), _ptr(a_log),
+                                      _ptr(S0), _ptr(out), _ptr(ST), B, H, T, dk, dv, dt, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), int(bool(save)),
+                                      _stream(stream)))
+    return out, ST, workspace
+
+
+def bwd_gated(q, k, v, beta, c, f_pre, a_log, S0, dO, dST=None, *, fwd_workspace, workspace=None,
+              want_dS0=True, stream=None):
+    """Backward of fwd_gated.  Returns dict dq, dk, dv, dbeta, dc, df_pre
+    (fp32), da_log ([H] fp32, summed over the batch in a fixed order), dS0."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = torch.float32
+    _need(q, "q"); _need(k, "k", q.dtype, q.shape); _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(beta, "beta", f32, (B, T, H)); _need(c, "c", f32, (B, T, H))
+    _need(f_pre, "f_pre", q.dtype, (B, T, H, dk)); _need(a_log, "a_log", f32, (H,))
+    _need(S0, "S0", f32, (B, H, dv, dk))
+    _need(dO, "dO", q.dtype, (B, T, H, dv)); _need(dST, "dST", f32, (B, H, dv, dk))
+    dt = _dtype_code(q)
+    g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+             dbeta=torch.empty_like(beta), dc=torch.empty_like(c),
+             df_pre=torch.empty((B, T, H, dk), dtype=f32, device=q.device),
+             da_log=torch.empty((H,), dtype=f32, device=q.device),
+             dS0=torch.empty((B, H, dv, dk), dtype=f32, device=q.device) if want_dS0 else None)
+    need = workspace_size(KD_WS_BWD_GATED, B, H, T, dk, dv, dt)
+    if workspace is None:
+        workspace = _alloc_ws(need, q.device)
+    _check(lib().kron_delta_bwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(c), _ptr(f_pre), _ptr(a_log),
+                                      _ptr(S0), _ptr(dO), _ptr(dST), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                      _ptr(g["dbeta"]), _ptr(g["dc"]), _ptr(g["df_pre"]), _ptr(g["da_log"]),
+                                      _ptr(g.get("dS0")), B, H, T, dk, dv, dt, _ptr(fwd_workspace),
+                                      fwd_workspace.numel() * fwd_workspace.element_size(),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream(stream)))
     return g
 

@@ -77,6 +77,8 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   if (L->tc) L->S0b = take(chunks * (size_t)dv * dk * 2);
   if (L->tc) L->fwd_bytes = off;  // the chain writes u, b0 and the chunk-start states on every call
   L->fwd_save_bytes = off;
+  if (!L->tc) L->glogf = take((size_t)B * T * H * dk * 4);  // gated inputs, CUDA-core path: logf
+  L->fwd_gated_bytes = off;
 
   off = 0;
   L->dSC = L->tc ? 0 : take(chunks * (size_t)dv * dk * 4);  // the tensor-core path keeps bf16 tiles
@@ -102,7 +104,10 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
     L->Kp = take((size_t)B * T * H * dk * 4);
     L->QpT = take(chunks * (size_t)dk * C * 2);
   }
+  L->dapart = take(chunks * 4);
   L->bwd_bytes = off;
+  if (!L->tc) L->gdlogf = take((size_t)B * T * H * dk * 4);  // gated inputs, CUDA-core path: dlogf
+  L->bwd_gated_bytes = off;
   return KD_OK;
 }
 
@@ -225,6 +230,16 @@ ProfState& prof() {
   return *p;
 }
 
+// The backward with recompute: its workspace holds a save-forward workspace,
+// then (CUDA-core path only, whose forward always writes the output) a scratch
+// output, then the backward's own scratch.
+size_t recompute_out_bytes(const kd::Layout& L, int B, int H, int T, int dv, int dtype) {
+  return L.tc ? 0 : align256((size_t)B * T * H * dv * (dtype == KD_BF16 ? 2 : 4));
+}
+size_t recompute_bytes(const kd::Layout& L, int B, int H, int T, int dv, int dtype) {
+  return align256(L.fwd_save_bytes) + recompute_out_bytes(L, B, H, T, dv, dtype) + L.bwd_bytes;
+}
+
 }  // namespace
 
 namespace kd {
@@ -272,6 +287,9 @@ size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv, 
     case KD_WS_FWD: ok(); return L.fwd_bytes;
     case KD_WS_FWD_SAVE: ok(); return L.fwd_save_bytes;
     case KD_WS_BWD: ok(); return L.bwd_bytes;
+    case KD_WS_BWD_RECOMPUTE: ok(); return recompute_bytes(L, B, H, T, dv, dtype);
+    case KD_WS_FWD_GATED: ok(); return L.fwd_gated_bytes;
+    case KD_WS_BWD_GATED: ok(); return L.bwd_gated_bytes;
     case KD_WS_PROLOGUE_BWD:
       ok();
       return align256((size_t)kd::prologue_blocks((long long)B * T) * H * sizeof(float));
@@ -386,6 +404,148 @@ int kron_delta_bwd_phase(const void* q, const void* k, const void* v, const floa
                     "backward launch");
   }
   return launched(kd::launch_bwd_simt(a, static_cast<cudaStream_t>(stream)), "backward launch");
+}
+
+int kron_delta_bwd_recompute(const void* q, const void* k, const void* v, const float* beta,
+                             const float* c, const float* logf, const float* S0, const void* dO,
+                             const float* dST, void* dq, void* dk, void* dv, float* dbeta, float* dc,
+                             float* dlogf, float* dS0, int B, int H, int T, int dk_, int dv_, int dtype,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk_, dv_, dtype, &L));
+  KD_TRY(check_ptr(q, "q", true));
+  KD_TRY(check_ptr(k, "k", true));
+  KD_TRY(check_ptr(v, "v", true));
+  KD_TRY(check_ptr(beta, "beta", true));
+  KD_TRY(check_ptr(c, "c", true));
+  KD_TRY(check_ptr(logf, "logf", true));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(dO, "dO", true));
+  KD_TRY(check_ptr(dST, "dST", false));
+  KD_TRY(check_ptr(dq, "dq", true));
+  KD_TRY(check_ptr(dk, "dk", true));
+  KD_TRY(check_ptr(dv, "dv", true));
+  KD_TRY(check_ptr(dbeta, "dbeta", true));
+  KD_TRY(check_ptr(dc, "dc", true));
+  KD_TRY(check_ptr(dlogf, "dlogf", true));
+  KD_TRY(check_ptr(dS0, "dS0", false));
+  const size_t need = recompute_bytes(L, B, H, T, dv_, dtype);
+  if (!workspace || ws_bytes < need)
+    return fail(KD_ERR_WORKSPACE, "backward-with-recompute workspace of %zu bytes needed (got %zu)", need,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  char* ws = static_cast<char*>(workspace);
+  const size_t fwd_part = align256(L.fwd_save_bytes), out_part = recompute_out_bytes(L, B, H, T, dv_, dtype);
+  // the forward with save = 1 into the first part; its output is not kept
+  if (L.tc) {
+    kd::FwdArgs a{q, k, v, beta, c, logf, S0, nullptr, nullptr, 1, ws, L, KD_PHASE_ALL};
+    a.keep_out = false;
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    KD_TRY(launched(kd::launch_fwd_tc(a, di.err, di.sms, static_cast<cudaStream_t>(stream)), "forward launch"));
+  } else {
+    KD_TRY(kron_delta_fwd(q, k, v, beta, c, logf, S0, ws + fwd_part, nullptr, B, H, T, dk_, dv_, dtype, ws,
+                          fwd_part, 1, stream));
+  }
+  return kron_delta_bwd(q, k, v, beta, c, logf, S0, dO, dST, dq, dk, dv, dbeta, dc, dlogf, dS0, B, H, T, dk_, dv_,
+                        dtype, ws, fwd_part, ws + fwd_part + out_part, ws_bytes - fwd_part - out_part, stream);
+}
+
+int kron_delta_fwd_gated(const void* q, const void* k, const void* v, const float* beta,
+                         const float* c, const void* f_pre, const float* a_log, const float* S0, void* out,
+                         float* ST, int B, int H, int T, int dk, int dv, int dtype, void* workspace,
+                         size_t ws_bytes, int save, void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk, dv, dtype, &L));
+  KD_TRY(check_ptr(f_pre, "f_pre", true));
+  KD_TRY(check_ptr(a_log, "a_log", true));
+  if (!workspace || ws_bytes < L.fwd_gated_bytes)
+    return fail(KD_ERR_WORKSPACE, "gated forward workspace of %zu bytes needed (got %zu)", L.fwd_gated_bytes,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (save != 0 && save != 1) return fail(KD_ERR_INVALID_ARG, "save must be 0 or 1");
+  KD_TRY(check_stream(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (L.tc) {
+    KD_TRY(check_ptr(q, "q", true));
+    KD_TRY(check_ptr(k, "k", true));
+    KD_TRY(check_ptr(v, "v", true));
+    KD_TRY(check_ptr(beta, "beta", true));
+    KD_TRY(check_ptr(c, "c", true));
+    KD_TRY(check_ptr(S0, "S0", false));
+    KD_TRY(check_ptr(out, "out", true));
+    KD_TRY(check_ptr(ST, "ST", false));
+    kd::FwdArgs a{q, k, v, beta, c, static_cast<const float*>(f_pre), S0, out, ST, save,
+                  static_cast<char*>(workspace), L, KD_PHASE_ALL};
+    a.a_log = a_log;
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    return launched(kd::launch_fwd_tc(a, di.err, di.sms, st), "gated forward launch");
+  }
+  // CUDA-core path: logf into the workspace, then the plain forward on it
+  float* glogf = kd::ws_ptr<float>(static_cast<char*>(workspace), L.glogf);
+  const cudaError_t e = kd::launch_gate_logf(f_pre, dtype, a_log, glogf, B, T, H, dk, st);
+  if (e != cudaSuccess) return launched(e, "gated forward launch");
+  return kron_delta_fwd(q, k, v, beta, c, glogf, S0, out, ST, B, H, T, dk, dv, dtype, workspace, ws_bytes, save,
+                        stream);
+}
+
+int kron_delta_bwd_gated(const void* q, const void* k, const void* v, const float* beta,
+                         const float* c, const void* f_pre, const float* a_log, const float* S0,
+                         const void* dO, const float* dST, void* dq, void* dk, void* dv, float* dbeta,
+                         float* dc, float* df_pre, float* da_log, float* dS0, int B, int H, int T,
+                         int dk_, int dv_, int dtype, const void* fwd_ws, size_t fwd_ws_bytes,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk_, dv_, dtype, &L));
+  KD_TRY(check_ptr(f_pre, "f_pre", true));
+  KD_TRY(check_ptr(a_log, "a_log", true));
+  KD_TRY(check_ptr(df_pre, "df_pre", true));
+  KD_TRY(check_ptr(da_log, "da_log", true));
+  if (!fwd_ws || fwd_ws_bytes < L.fwd_gated_bytes)
+    return fail(KD_ERR_WORKSPACE, "the gated forward's workspace (save=1) of %zu bytes needed (got %zu)",
+                L.fwd_gated_bytes, fwd_ws ? fwd_ws_bytes : 0);
+  if (!workspace || ws_bytes < L.bwd_gated_bytes)
+    return fail(KD_ERR_WORKSPACE, "gated backward workspace of %zu bytes needed (got %zu)", L.bwd_gated_bytes,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256) || !aligned(fwd_ws, 256))
+    return fail(KD_ERR_WORKSPACE, "workspaces must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* dapart = kd::ws_ptr<float>(ws, L.dapart);
+  if (L.tc) {
+    KD_TRY(check_ptr(q, "q", true));
+    KD_TRY(check_ptr(k, "k", true));
+    KD_TRY(check_ptr(v, "v", true));
+    KD_TRY(check_ptr(beta, "beta", true));
+    KD_TRY(check_ptr(c, "c", true));
+    KD_TRY(check_ptr(dO, "dO", true));
+    KD_TRY(check_ptr(dST, "dST", false));
+    KD_TRY(check_ptr(dq, "dq", true));
+    KD_TRY(check_ptr(dk, "dk", true));
+    KD_TRY(check_ptr(dv, "dv", true));
+    KD_TRY(check_ptr(dbeta, "dbeta", true));
+    KD_TRY(check_ptr(dc, "dc", true));
+    KD_TRY(check_ptr(dS0, "dS0", false));
+    kd::BwdArgs a{q, k, v, beta, c, static_cast<const float*>(f_pre), S0, dO, dST, dq, dk, dv, dbeta, dc, df_pre,
+                  dS0, static_cast<const char*>(fwd_ws), ws, L, KD_PHASE_ALL};
+    a.a_log = a_log;
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    cudaError_t e = kd::launch_bwd_tc(a, di.err, di.sms, st);
+    if (e == cudaSuccess) e = kd::launch_reduce_dalog(dapart, B, H, L.NC, da_log, st);
+    return launched(e, "gated backward launch");
+  }
+  // CUDA-core path: the plain backward on the forward's logf, then df~ and da_log from dlogf
+  const float* glogf = kd::ws_ptr<float>(static_cast<const char*>(fwd_ws), L.glogf);
+  float* gdlogf = kd::ws_ptr<float>(ws, L.gdlogf);
+  KD_TRY(kron_delta_bwd(q, k, v, beta, c, glogf, S0, dO, dST, dq, dk, dv, dbeta, dc, gdlogf, dS0, B, H, T, dk_,
+                        dv_, dtype, fwd_ws, fwd_ws_bytes, workspace, ws_bytes, stream));
+  cudaError_t e = kd::launch_gate_dlogf(gdlogf, glogf, a_log, df_pre, dapart, B, T, H, dk_, L.NC, st);
+  if (e == cudaSuccess) e = kd::launch_reduce_dalog(dapart, B, H, L.NC, da_log, st);
+  return launched(e, "gated backward launch");
 }
 
 int kron_delta_decode(const void* q, const void* k, const void* v, const float* beta,

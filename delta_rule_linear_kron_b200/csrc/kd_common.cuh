@@ -36,6 +36,65 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
   return __float2bfloat16_rn(x);
 }
 
+// ---- gated inputs: the forget gate formed from its pre-activation ----------
+// KronLSTM digest, "어떻게 쓰나": f = sigma(f~)^a with a = e^{a_log} per head, so
+// the log-decay is logf = a log sigma(f~), and log sigma(x) = -softplus(-x) =
+// min(x, 0) - log(1 + e^{-|x|}).  These run once per element of every tile a
+// chunk kernel loads, so they use the hardware exp2/log2 approximations with
+// short Taylor series where those would cancel.
+
+// log(1 + e) for e in [0, 1]: the series e - e^2/2 + e^3/3 - e^4/4 while
+// e < 1/32 (truncation below e^5/5, relative 2e-7), else log of 1 + e, which
+// is at least 0.03 there (relative error about 5e-6).
+__device__ __forceinline__ float log1p_unit(float e) {
+  return e < 0.03125f ? e * (1.f - e * (0.5f - e * (0.33333334f - 0.25f * e))) : __logf(1.f + e);
+}
+__device__ __forceinline__ float log_sigmoid(float x) { return fminf(x, 0.f) - log1p_unit(__expf(-fabsf(x))); }
+// e^s - 1 for s <= 0: the series s + s^2/2 + s^3/6 + s^4/24 while s > -1/16
+// (relative truncation below s^4/120 = 1.3e-7), else e^s - 1, at most -0.06 there.
+__device__ __forceinline__ float expm1_nonpos(float s) {
+  return s > -0.0625f ? s * (1.f + s * (0.5f + s * (0.16666667f + s * 0.041666668f))) : __expf(s) - 1.f;
+}
+// d logf / d f~ = a sigma(-f~); with ls = log sigma(f~) = logf / a, sigma(-f~) =
+// 1 - e^{ls} = -(e^{ls} - 1), accurate when sigma(f~) is close to 1.
+__device__ __forceinline__ float dlogf_dfpre(float logf, float a, float inv_a) {
+  return -a * expm1_nonpos(fminf(logf * inv_a, 0.f));
+}
+
+// A chunk's bf16 forget pre-activation tile [64][128] (16 KB, landed at `src`,
+// which may be the upper half of `dst`) becomes its fp32 log-decay tile at
+// `dst` (32 KB): logf = a log sigma(f~), and 0 on positions t >= nv beyond the
+// sequence (the zero-padded tail).  Thread tid takes the 4-element groups
+// tid, tid + 256, ..., tid + 1792, so a warp's 8-byte loads and 16-byte stores
+// are contiguous (no shared-memory bank conflicts).  All 256 threads of the
+// CTA take part; the call ends with a CTA barrier.
+__device__ __forceinline__ void gate_logf_tile(float* dst, const unsigned char* src, float a, int nv) {
+  const int tid = threadIdx.x;
+  uint2 raw[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) raw[r] = reinterpret_cast<const uint2*>(src)[r * 256 + tid];
+  __syncthreads();  // every thread has read its source before any destination is written
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int grp = r * 256 + tid;  // elements 4 grp .. 4 grp + 3, all in row grp / 32
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw[r]);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (grp / 32 < nv)
+      o = make_float4(a * log_sigmoid(__bfloat162float(e[0])), a * log_sigmoid(__bfloat162float(e[1])),
+                      a * log_sigmoid(__bfloat162float(e[2])), a * log_sigmoid(__bfloat162float(e[3])));
+    reinterpret_cast<float4*>(dst)[grp] = o;
+  }
+  __syncthreads();
+}
+
+// One log-decay value from global memory: logf itself, or formed from the
+// forget pre-activation (gated inputs, fpre != nullptr).
+template <typename Tf>
+__device__ __forceinline__ float load_logf(const float* __restrict__ logf, const Tf* __restrict__ fpre, float a,
+                                           size_t g) {
+  return fpre ? a * log_sigmoid(to_f(fpre[g])) : logf[g];
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

@@ -59,7 +59,14 @@ struct Layout {
   // K+ [B][T][H][dk] fp32, and Q+^T per chunk as a bf16 128-byte-swizzled
   // K-major tile [j][t] (128 rows x 64)
   size_t Kp = 0, QpT = 0;
+  size_t dapart = 0;  // gated inputs: each chunk's part of da_log [ch]
   size_t bwd_bytes = 0;
+  // Gated inputs (forget pre-activations in place of logf).  The CUDA-core
+  // path converts them to logf in the forward's workspace (glogf, [B][T][H][dk]
+  // fp32, after the saved region) and takes dlogf in the backward's (gdlogf);
+  // the tensor-core kernels read the pre-activations directly.
+  size_t glogf = 0, gdlogf = 0;
+  size_t fwd_gated_bytes = 0, bwd_gated_bytes = 0;
 };
 
 // Phases of a forward or backward call.  kPhaseLocal: the work that does not
@@ -86,6 +93,12 @@ struct FwdArgs {
   char* ws;  // workspace base
   Layout L;
   int phases = kPhaseAll;
+  // gated inputs (tensor-core path): logf then points at the bf16 forget
+  // pre-activations and a_log at the per-head exponents; nullptr otherwise
+  const float* a_log = nullptr;
+  // false: stop after the chunk chain (the backward's recompute of the saved
+  // quantities needs no output; tensor-core path)
+  bool keep_out = true;
 };
 
 struct BwdArgs {
@@ -99,6 +112,10 @@ struct BwdArgs {
   char* ws;         // backward workspace
   Layout L;
   int phases = kPhaseAll;
+  // gated inputs (tensor-core path): logf points at the bf16 forget
+  // pre-activations, dlogf receives df~ (fp32) and a_log holds the per-head
+  // exponents; nullptr otherwise
+  const float* a_log = nullptr;
 };
 
 // Sets the calling thread's kron_delta_last_error() string.
@@ -217,6 +234,16 @@ struct GdnDecodeArgs {
 cudaError_t launch_gdn2_decode(const GdnDecodeArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_fwd(const GdnArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_bwd(const GdnArgs& a, cudaStream_t st);
+
+// Gated inputs (kd_gate.cu): logf = e^{a_log} log sigma(f~) into a buffer
+// (the CUDA-core path); df~ = dlogf a sigma(-f~) and each chunk's part of
+// da_log from dlogf and logf (the CUDA-core path); da_log per head from the
+// per-chunk parts, summed in a fixed order.
+cudaError_t launch_gate_logf(const void* fpre, int dtype, const float* a_log, float* logf, int B, int T, int H,
+                             int dk, cudaStream_t st);
+cudaError_t launch_gate_dlogf(const float* dlogf, const float* logf, const float* a_log, float* dfpre,
+                              float* dapart, int B, int T, int H, int dk, int NC, cudaStream_t st);
+cudaError_t launch_reduce_dalog(const float* dapart, int B, int H, int NC, float* da_log, cudaStream_t st);
 
 // Failure-reporting self-test (kd_selftest.cu): a bounded wait that runs out.
 cudaError_t launch_selftest_timeout(int* err, cudaStream_t st);

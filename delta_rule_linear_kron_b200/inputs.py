@@ -41,7 +41,8 @@ from dataclasses import dataclass, replace
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs", "make_prologue_inputs",
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_gated_inputs", "make_decode_inputs",
+           "make_prologue_inputs",
            "make_epilogue_inputs", "make_gdn2_inputs",
            "round_to_dtype", "decode_token_inputs_torch"]
 
@@ -130,6 +131,21 @@ def make_inputs(wl: Workload | int, *, B=None, H=None, T=None, dk=None, dv=None,
     if with_dO:
         out["dO"] = round_to_dtype(rng.standard_normal((B, T, H, dv)), wl.dtype)
     return out
+
+
+def make_gated_inputs(wl: Workload | int, *, seed_gate=3000, **kw):
+    """A workload's inputs with the forget gate given as its pre-activation:
+    make_inputs(wl, **kw) without logf, plus f_pre [B,T,H,dk] ~ N(3,1) in the
+    storage dtype and a_log [H] ~ U(-1,1) (fp32), drawn in that order from
+    default_rng(seed_gate) (the prologue inputs' forget-gate distributions)."""
+    inp = make_inputs(wl, **kw)
+    dtype = (WORKLOADS[wl] if isinstance(wl, int) else wl).dtype
+    B, T, H, dk = inp["q"].shape
+    rng = np.random.default_rng(seed_gate)
+    inp["f_pre"] = round_to_dtype(rng.normal(3.0, 1.0, size=(B, T, H, dk)), dtype)
+    inp["a_log"] = round_to_dtype(rng.uniform(-1.0, 1.0, size=(H,)), "f32")
+    del inp["logf"]
+    return inp
 
 
 def make_prologue_inputs(B, H, T, dk, dv, dtype="bf16", seed=2000, with_grads=True):

@@ -1,11 +1,13 @@
 """Runs the forward+backward step of the Kronecker delta rule mixer at a
 chosen shape, for profilers (ncu) that need a small, repeatable case.
 
-    python -m delta_rule_linear_kron_b200.profile_step [--B 1] [--H 16] [--T 2048] [--steps 4]
+    python -m delta_rule_linear_kron_b200.profile_step [--B 1] [--H 16] [--T 2048] [--steps 4] [--gated]
 
 Inputs follow the forward+backward workload's recipe (bf16 q, k, v, dO; fp32
 gates; beta in (0, 2); nonzero S0) at the given shape.  Each step is one
-forward (saving for the backward) and one backward, as in bench.py.
+forward (saving for the backward) and one backward, as in bench.py.  With
+--gated the step goes through the gated entry points instead, with the forget
+gate as a bf16 pre-activation ~ N(3, 1) and a_log ~ U(-1, 1).
 """
 from __future__ import annotations
 
@@ -19,6 +21,7 @@ def main(argv=None):
     ap.add_argument("--H", type=int, default=16)
     ap.add_argument("--T", type=int, default=2048)
     ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--gated", action="store_true")
     a = ap.parse_args(argv)
 
     import torch
@@ -29,16 +32,26 @@ def main(argv=None):
     inp = kin.make_inputs(4, B=a.B, H=a.H, T=a.T)
     d = {n: torch.from_numpy(inp[n]).to("cuda", torch.bfloat16 if n in ("q", "k", "v", "dO") else torch.float32)
          for n in ("q", "k", "v", "dO", "beta", "c", "logf", "S0")}
-    fws = torch.empty(kd.workspace_size(kd.KD_WS_FWD_SAVE, a.B, a.H, a.T, 128, 128), dtype=torch.uint8,
-                      device="cuda")
-    bws = torch.empty(kd.workspace_size(kd.KD_WS_BWD, a.B, a.H, a.T, 128, 128), dtype=torch.uint8, device="cuda")
+    kf, kb = (kd.KD_WS_FWD_GATED, kd.KD_WS_BWD_GATED) if a.gated else (kd.KD_WS_FWD_SAVE, kd.KD_WS_BWD)
+    fws = torch.empty(kd.workspace_size(kf, a.B, a.H, a.T, 128, 128), dtype=torch.uint8, device="cuda")
+    bws = torch.empty(kd.workspace_size(kb, a.B, a.H, a.T, 128, 128), dtype=torch.uint8, device="cuda")
+    if a.gated:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(3004)
+        f_pre = (torch.randn(d["logf"].shape, generator=g, device="cuda") + 3.0).to(torch.bfloat16)
+        a_log = torch.rand((a.H,), generator=g, device="cuda") * 2 - 1
     for _ in range(a.steps):
-        kd.fwd(d["q"], d["k"], d["v"], d["beta"], d["c"], d["logf"], d["S0"], save=True, workspace=fws)
-        kd.bwd(d["q"], d["k"], d["v"], d["beta"], d["c"], d["logf"], d["S0"], d["dO"], fwd_workspace=fws,
-               workspace=bws)
+        if a.gated:
+            kd.fwd_gated(d["q"], d["k"], d["v"], d["beta"], d["c"], f_pre, a_log, d["S0"], save=True, workspace=fws)
+            kd.bwd_gated(d["q"], d["k"], d["v"], d["beta"], d["c"], f_pre, a_log, d["S0"], d["dO"],
+                         fwd_workspace=fws, workspace=bws)
+        else:
+            kd.fwd(d["q"], d["k"], d["v"], d["beta"], d["c"], d["logf"], d["S0"], save=True, workspace=fws)
+            kd.bwd(d["q"], d["k"], d["v"], d["beta"], d["c"], d["logf"], d["S0"], d["dO"], fwd_workspace=fws,
+                   workspace=bws)
     torch.cuda.synchronize()
     kd.device_status()
-    print(f"profile_step: {a.steps} fwd+bwd steps at B={a.B} H={a.H} T={a.T} done")
+    print(f"profile_step: {a.steps} {'gated ' if a.gated else ''}fwd+bwd steps at B={a.B} H={a.H} T={a.T} done")
     return 0
 
 

@@ -23,9 +23,12 @@
  *
  * Entry points:
  *   Kronecker delta rule  kron_delta_fwd, kron_delta_bwd, kron_delta_decode,
+ *                         kron_delta_bwd_recompute (no saved forward),
  *                         kron_delta_fwd_phase / _bwd_phase (split at the
  *                         carried state, for context parallelism),
- *                         kron_delta_fwd_noalloc
+ *                         kron_delta_fwd_noalloc,
+ *                         kron_delta_fwd_gated / _bwd_gated (forget gate
+ *                         from its pre-activation, formed inside the kernels)
  *   around the mixer      kron_delta_prologue_fwd / _bwd (L2-norm, gates,
  *                         log-decay), kron_delta_epilogue_fwd / _bwd
  *                         (per-head RMSNorm and output gate)
@@ -98,6 +101,9 @@ extern "C" {
                                  must be valid but do not change the size) */
 #define KD_WS_GDN2_FWD 5      /* kron_delta_gdn2_fwd (kept for kron_delta_gdn2_bwd) */
 #define KD_WS_GDN2_BWD 6      /* backward scratch of kron_delta_gdn2_bwd */
+#define KD_WS_FWD_GATED 7     /* kron_delta_fwd_gated (kept for kron_delta_bwd_gated) */
+#define KD_WS_BWD_GATED 8     /* backward scratch of kron_delta_bwd_gated */
+#define KD_WS_BWD_RECOMPUTE 9 /* kron_delta_bwd_recompute (forward scratch included) */
 
 /* phases of kron_delta_fwd_phase / kron_delta_bwd_phase */
 #define KD_PHASE_LOCAL 1   /* the work that does not depend on the carried state */
@@ -151,12 +157,9 @@ KD_API int kron_delta_fwd(const void *q, const void *k, const void *v,
  *   workspace, ws_bytes : scratch of at least
  *         kron_delta_workspace_size(KD_WS_BWD, ...).
  * S0 is the same initial state given to the forward (NULL = zero).
- * There is no recompute mode: the backward always reads the forward's saved
- * chunk quantities (fwd_ws) and fails with KD_ERR_WORKSPACE without them.
- * Recomputing them would rerun the forward's sequential chunk chain, which is
- * a latency-bound critical path as long as the backward's own chain, while
- * reading them back costs one pass over the saved bytes.  A caller that does
- * not keep the forward's workspace reruns kron_delta_fwd with save = 1 first.
+ * kron_delta_bwd reads the forward's saved chunk quantities (fwd_ws) and
+ * fails with KD_ERR_WORKSPACE without them; kron_delta_bwd_recompute (below)
+ * is the backward for a caller that did not keep them.
  * Errors as for kron_delta_fwd.  Asynchronous on `stream`.
  */
 KD_API int kron_delta_bwd(const void *q, const void *k, const void *v,
@@ -166,6 +169,61 @@ KD_API int kron_delta_bwd(const void *q, const void *k, const void *v,
                    float *dlogf, float *dS0, int B, int H, int T, int dk_,
                    int dv_, int dtype, const void *fwd_ws, size_t fwd_ws_bytes,
                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Backward of kron_delta_fwd that recomputes the forward's chunk quantities
+ * instead of reading a saved forward workspace: it enqueues the forward's
+ * chunk-local work and its chunk chain with save = 1 into the first part of
+ * `workspace` (without writing an output), then kron_delta_bwd on it.  The
+ * gradients are bitwise those of kron_delta_fwd(save = 1) + kron_delta_bwd on
+ * the same inputs.  The cost is the forward's chain again, a sequential pass
+ * over the chunks as long as the backward's own, and the workspace is the two
+ * added together.
+ *   workspace, ws_bytes : at least kron_delta_workspace_size(KD_WS_BWD_RECOMPUTE, ...).
+ * The other arguments, layouts and errors are those of kron_delta_bwd.
+ * Asynchronous on `stream`.
+ */
+KD_API int kron_delta_bwd_recompute(const void *q, const void *k, const void *v,
+                             const float *beta, const float *c, const float *logf,
+                             const float *S0, const void *dO, const float *dST,
+                             void *dq, void *dk, void *dv, float *dbeta, float *dc,
+                             float *dlogf, float *dS0, int B, int H, int T, int dk_,
+                             int dv_, int dtype, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/*
+ * Forward and backward with the forget gate taken as its pre-activation
+ * (KronLSTM digest, "어떻게 쓰나": the forget gate is f = sigma(f~)^a with
+ * a = e^{a_log} per head, so logf = a log sigma(f~)).  Identical to
+ * kron_delta_fwd / kron_delta_bwd on logf = e^{a_log} log sigma(f_pre), but
+ * on the tensor-core path (bf16, dk = dv = 128) every kernel reads the bf16
+ * pre-activations and forms logf while loading them, so the fp32 logf tensor
+ * (a third of the forward's input bytes) is never written or read.
+ *   f_pre : forget pre-activations [B,T,H,dk] (dtype).
+ *   a_log : per-head exponent [H] fp32.
+ *   workspace (forward) : at least kron_delta_workspace_size(KD_WS_FWD_GATED, ...);
+ *         pass it with save = 1 to kron_delta_bwd_gated as fwd_ws.
+ *   df_pre : gradient of f_pre [B,T,H,dk] fp32 (dlogf a sigma(-f_pre)).
+ *   da_log : gradient of a_log [H] fp32, the sum over the batch, the tokens
+ *         and the key channels of dlogf logf, reduced in a fixed order
+ *         (bitwise reproducible).
+ *   workspace (backward) : at least kron_delta_workspace_size(KD_WS_BWD_GATED, ...).
+ * The other arguments, layouts and errors are those of kron_delta_fwd and
+ * kron_delta_bwd.  Asynchronous on `stream`.
+ */
+KD_API int kron_delta_fwd_gated(const void *q, const void *k, const void *v,
+                         const float *beta, const float *c, const void *f_pre,
+                         const float *a_log, const float *S0, void *out, float *ST,
+                         int B, int H, int T, int dk, int dv, int dtype,
+                         void *workspace, size_t ws_bytes, int save, void *stream);
+KD_API int kron_delta_bwd_gated(const void *q, const void *k, const void *v,
+                         const float *beta, const float *c, const void *f_pre,
+                         const float *a_log, const float *S0, const void *dO,
+                         const float *dST, void *dq, void *dk, void *dv, float *dbeta,
+                         float *dc, float *df_pre, float *da_log, float *dS0, int B,
+                         int H, int T, int dk_, int dv_, int dtype, const void *fwd_ws,
+                         size_t fwd_ws_bytes, void *workspace, size_t ws_bytes,
+                         void *stream);
 
 /*
  * The forward and backward split at the carried state, for a caller that

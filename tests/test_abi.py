@@ -58,7 +58,27 @@ def test_workspace_sizes(L):
     assert kd.workspace_size(kd.KD_WS_FWD, 1, 1, 65, 32, 32) > kd.workspace_size(kd.KD_WS_FWD, 1, 1, 64, 32, 32)
     assert L.kron_delta_workspace_size(0, 1, 1, 64, 48, 32, 1) == 0
     assert b"32, 64 or 128" in L.kron_delta_last_error()
-    assert L.kron_delta_workspace_size(9, 1, 1, 64, 32, 32, 1) == 0
+    assert L.kron_delta_workspace_size(10, 1, 1, 64, 32, 32, 1) == 0
+    # the backward with recompute holds a save-forward workspace and the backward's
+    # own (the CUDA-core path, whose forward always writes an output, one more buffer)
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert kd.workspace_size(kd.KD_WS_BWD_RECOMPUTE, B, H, T, d, d) == a256(fs) + bw
+    f32s = kd.workspace_size(kd.KD_WS_FWD_SAVE, B, H, T, d, d, kd.KD_F32)
+    f32b = kd.workspace_size(kd.KD_WS_BWD, B, H, T, d, d, kd.KD_F32)
+    assert kd.workspace_size(kd.KD_WS_BWD_RECOMPUTE, B, H, T, d, d, kd.KD_F32) == \
+        a256(f32s) + a256(B * T * H * d * 4) + f32b
+
+
+def test_bwd_recompute_rejects_a_short_workspace(L):
+    p = ctypes.c_void_p(256)
+    need = kd.workspace_size(kd.KD_WS_BWD_RECOMPUTE, 1, 1, 64, 32, 32)
+    rc = L.kron_delta_bwd_recompute(p, p, p, p, p, p, None, p, None, p, p, p, p, p, p, None, 1, 1, 64, 32, 32, 1,
+                                    p, need - 256, None)
+    assert rc == kd.KD_ERR_WORKSPACE
+    assert b"recompute" in L.kron_delta_last_error()
+    rc = L.kron_delta_bwd_recompute(p, p, p, p, p, None, None, p, None, p, p, p, p, p, p, None, 1, 1, 64, 32, 32, 1,
+                                    p, need, None)
+    assert rc == kd.KD_ERR_INVALID_ARG and b"logf" in L.kron_delta_last_error()
 
 
 def _fwd_call(L, **over):
