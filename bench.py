@@ -38,7 +38,6 @@ WL = dict(B=1, H=16, T=16384, dk=128, dv=128)
 CHUNK = 64
 METRIC = "Kron-delta fwd+bwd tokens/s (H16,d128,T16K) & % bf16 TC peak; decode GB/s"
 WORKLOAD_NAME = "fwdbwd-B1-H16-T16384-d128-beta2"
-CPU_SAMPLE_T = 4096     # tokens of the workload the oracle baseline runs (all 16 heads)
 REF_STEP_T = 512        # tokens per step of the reference (oracle) arm
 
 
@@ -106,22 +105,32 @@ def method_work(name, d=128, C=CHUNK):
 
 # The bytes each kernel of the step actually moves by design, per token-head:
 # its method inputs and outputs plus the workspace intermediates it writes and
-# reads (for the traffic comparison with ncu's DRAM counters).
+# reads (for the traffic comparison with ncu's DRAM counters).  The
+# cross-chunk kernel's tiles of the previous chunk, read just before by that
+# chunk's own CTA and found in L2, are not counted.
 def kernel_io_bytes(name, d=128, C=CHUNK):
     act = d * 2                      # one bf16 activation row
-    lf = d * 4                       # one fp32 logf row
-    tile_f32 = d * d * 4 // C        # one fp32 d x d tile per chunk, per token
-    tile_bf16 = d * d * 2 // C
+    lf = d * 4                       # one fp32 row (logf, K~, K^e, K+)
+    tile_bf16 = d * d * 2 // C       # one bf16 d x d tile per chunk, per token
     cc = C * 4                       # one fp32 C x C matrix per chunk, per token
     ccb = C * 2                      # one bf16 C x C tile per chunk, per token
+    vt = d * C * 2 // C              # one bf16 d x C tile per chunk (V^T, Q+^T), per token
     table = {
-        "fwd_prep_tc": 3 * act + lf + 8 + cc + 4 + cc,
-        "fwd_cross_tc": 2 * act + lf + 2 * lf + 8 + cc + act,
-        "fwd_chain_tc": 2 * lf + 8 + act + 2 * cc + 8 + tile_f32 + tile_bf16 + 8,
-        "fwd_out_tc": 3 * act + lf + 4 + tile_f32 + act,
-        "bwd_pre_tc": 3 * act + lf + cc + 4 + 2 * ccb + ccb + ccb + 8,
-        "bwd_chain_tc": 4 * act + lf + 4 + cc + 4 + tile_bf16 + 4,
-        "bwd_post_tc": 4 * act + lf + 2 * tile_bf16 + 2 * ccb + ccb + ccb + 20 + 3 * act + lf + 8,
+        # q, k, v, logf, beta, c in; y, A, P out
+        "fwd_prep_tc": 3 * act + lf + 8 + 4 + 2 * cc,
+        # v, k, logf in; K~, K^e, gamma_C, H, V^T out
+        "fwd_cross_tc": 2 * act + lf + 2 * lf + 8 + cc + vt,
+        # K~, K^e, V^T, A, H, y, beta, gamma_C in; u, b0, the bf16 chunk-start state out
+        "fwd_chain_tc": 2 * lf + vt + 2 * cc + 4 + 4 + 8 + 8 + tile_bf16,
+        # q, k, v, logf, u, chunk-start state in; O out
+        "fwd_out_tc": 3 * act + lf + 4 + tile_bf16 + act,
+        # v, dO, k, q, logf, P, u in; du, M u, [dP; E_V], P diag(u), E_K, K+, Q+^T out
+        "bwd_pre_tc": 4 * act + lf + cc + 4 + 8 + 2 * ccb + ccb + ccb + lf + vt,
+        # dO, K^e, K+, beta, A, H, gamma_C, V^T, Q+^T, du in; dS tile, g out
+        "bwd_chain_tc": act + 2 * lf + 4 + 2 * cc + 8 + 2 * vt + 4 + tile_bf16 + 4,
+        # logf, q, k, E_K, S0, dS, dO, v, [dP; E_V], P diag(u), u, b0, g, M u, beta in;
+        # dq, dk, dv, dlogf, dbeta, dc out
+        "bwd_post_tc": lf + 2 * act + ccb + 2 * tile_bf16 + 2 * act + 2 * ccb + ccb + 16 + 4 + 3 * act + lf + 8,
     }
     return table.get(name)
 
@@ -266,32 +275,50 @@ def rank_seed(base, rank):
     return base + rank
 
 
-def oracle_baseline(T_sample, seed=1004):
-    """The fp64 oracle, as it stands, on the first T_sample tokens of the
-    workload (all heads), fwd + bwd, all host cores."""
-    from delta_rule_linear_kron_b200 import inputs as kin
+def _oracle_time(inp, nthreads, bwd=True):
     from oracle import oracle
-    inp = kin.make_inputs(4, T=T_sample, seed=seed)
-    cores = len(os.sched_getaffinity(0))
     t = time.perf_counter()
-    oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], nthreads=cores)
-    oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], inp["dO"],
-               nthreads=cores)
-    el = time.perf_counter() - t
-    # the same work on one thread, on a quarter of the sample
-    T1 = max(64, T_sample // 4)
+    oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], nthreads=nthreads)
+    if bwd:
+        oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["c"], inp["logf"], inp["S0"], inp["dO"],
+                   nthreads=nthreads)
+    return time.perf_counter() - t
+
+
+def oracle_baseline(T1=1024, full=False, seed=1004):
+    """The fp64 oracle, as it stands, on the host cores: the whole forward +
+    backward workload threaded over its heads, and its first T1 tokens of
+    every head on one thread.  full=True adds the whole workload on one thread
+    and the long-context forward workload (B1 H16 T16384, forward only) both
+    ways, a few minutes of CPU time."""
+    from delta_rule_linear_kron_b200 import inputs as kin
+    cores = len(os.sched_getaffinity(0))
+    used = min(cores, WL["H"])
+    inp = kin.make_inputs(4, seed=seed)
+    el = _oracle_time(inp, cores)
     one = {n: inp[n][:, :T1] for n in ("q", "k", "v", "beta", "c", "logf", "dO")}
     one["S0"] = inp["S0"]
-    t = time.perf_counter()
-    oracle.fwd(one["q"], one["k"], one["v"], one["beta"], one["c"], one["logf"], one["S0"], nthreads=1)
-    oracle.bwd(one["q"], one["k"], one["v"], one["beta"], one["c"], one["logf"], one["S0"], one["dO"], nthreads=1)
-    el1 = time.perf_counter() - t
-    return dict(value=WL["B"] * T_sample / el, unit="tokens/s", cores=min(cores, WL["H"]), kind="oracle",
-                sample=f"first {T_sample} tokens x {WL['H']} heads of the workload, fwd+bwd, fp64, "
-                       f"threaded over heads ({min(cores, WL['H'])} threads used of {cores} cores)",
-                seconds=el,
-                single_thread=dict(value=WL["B"] * T1 / el1, unit="tokens/s", cores=1, seconds=el1,
-                                   sample=f"first {T1} tokens x {WL['H']} heads, one thread"))
+    el1 = _oracle_time(one, 1)
+    out = dict(value=WL["B"] * WL["T"] / el, unit="tokens/s", cores=used, kind="oracle",
+               sample=f"the whole workload ({WL['B']}x{WL['T']} tokens x {WL['H']} heads), fwd+bwd, fp64, "
+                      f"threaded over heads ({used} threads used of {cores} cores)",
+               seconds=el,
+               single_thread=dict(value=WL["B"] * T1 / el1, unit="tokens/s", cores=1, seconds=el1,
+                                  sample=f"first {T1} tokens x {WL['H']} heads, one thread"))
+    if full:
+        e1 = _oracle_time(inp, 1)
+        out["single_thread_full"] = dict(value=WL["B"] * WL["T"] / e1, unit="tokens/s", cores=1, seconds=e1,
+                                         sample="the whole workload, fwd+bwd, one thread")
+        del inp, one
+        wl3 = kin.WORKLOADS[3]
+        f3 = kin.make_inputs(3, with_dO=False)
+        ef = _oracle_time(f3, cores, bwd=False)
+        ef1 = _oracle_time(f3, 1, bwd=False)
+        out["fwd_long"] = dict(workload=wl3.name, threaded=dict(value=wl3.B * wl3.T / ef, unit="tokens/s",
+                                                                 cores=min(cores, wl3.H), seconds=ef),
+                               single_thread=dict(value=wl3.B * wl3.T / ef1, unit="tokens/s", cores=1,
+                                                  seconds=ef1))
+    return out
 
 
 def run_reference(args):
@@ -339,10 +366,14 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-fwd", action="store_true")
     ap.add_argument("--no-gated", action="store_true")
+    ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-gdn2", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-full", action="store_true",
+                    help="also time the oracle on one thread over the whole workload, and on the long-context "
+                         "forward workload (a few minutes)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
@@ -506,6 +537,56 @@ def main(argv=None):
                      input_bytes_per_step=h2d_gated, plain_input_bytes_per_step=h2d_plain,
                      step="fwd_gated(save) + bwd_gated (bf16 f_pre, fp32 a_log [H]; outputs df_pre, da_log)")
         del f_pre, a_log, gfw, gbw
+
+    # ---- the same step from raw projections and gate pre-activations: the
+    # input prologue fused into the chunk kernels (fwd_fused(save) +
+    # bwd_fused), against the unfused layer (prologue pass, fwd, bwd, prologue
+    # backward pass), each timed on its own ---------------------------------
+    fused = None
+    if not args.no_fused:
+        g_ = torch.Generator(device=dev)
+        g_.manual_seed(rank_seed(5004, rank))
+        rn = lambda *sh, m=0.0: torch.randn(sh, generator=g_, device=dev) + m  # noqa: E731
+        raw = dict(q_raw=rn(B, T, H, dk).to(bf), k_raw=rn(B, T, H, dk).to(bf), v_raw=rn(B, T, H, dv).to(bf),
+                   beta_pre=rn(B, T, H), c_pre=rn(B, T, H), f_pre=rn(B, T, H, dk, m=3.0).to(bf),
+                   a_log=torch.rand((H,), generator=g_, device=dev) * 2 - 1)
+        rorder = ("q_raw", "k_raw", "v_raw", "beta_pre", "c_pre", "f_pre", "a_log")
+        ffw = torch.empty(kd.workspace_size(kd.KD_WS_FWD_FUSED, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+        fbw = torch.empty(kd.workspace_size(kd.KD_WS_BWD_FUSED, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+        pws = torch.empty(kd.workspace_size(kd.KD_WS_PROLOGUE_BWD, B, H, T, dk, dv), dtype=torch.uint8,
+                          device=dev)
+
+        def fused_step():
+            kd.fwd_fused(*(raw[n] for n in rorder), 2.0, d["S0"], out=out, save=True, workspace=ffw)
+            kd.bwd_fused(*(raw[n] for n in rorder), 2.0, d["S0"], d["dO"], fwd_workspace=ffw, workspace=fbw)
+
+        def unfused_step():
+            pp = kd.prologue_fwd(*(raw[n] for n in rorder), 2.0)
+            pa = [pp[n] for n in ("q", "k", "v", "beta", "c", "logf")]
+            kd.fwd(*pa, d["S0"], out=out, save=True, workspace=fws)
+            gg = kd.bwd(*pa, d["S0"], d["dO"], fwd_workspace=fws, workspace=bws)
+            kd.prologue_bwd(*(raw[n] for n in rorder), gg["dq"], gg["dk"], gg["dv"], gg["dbeta"], gg["dc"],
+                            gg["dlogf"], 2.0, workspace=pws)
+        fl = {}
+        for key, fn in (("fused", fused_step), ("unfused", unfused_step)):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            barrier()
+            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            q0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            q1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            fl[key] = max_over_ranks(q0.elapsed_time(q1), ws_n, dev) / args.steps
+        kd.device_status()
+        fused = dict(ms=fl["fused"], tokens_per_s=job_throughput(ws_n, B * T, 1, fl["fused"]),
+                     unfused_ms=fl["unfused"], unfused_tokens_per_s=job_throughput(ws_n, B * T, 1, fl["unfused"]),
+                     step="fwd_fused(save) + bwd_fused from raw bf16 q, k, v, f_pre and fp32 beta_pre, c_pre, "
+                          "a_log; unfused: prologue_fwd + fwd(save) + bwd + prologue_bwd")
+        del raw, ffw, fbw, pws
 
     # ---- decode: 1000 consecutive in-place steps --------------------------
     decode = None
@@ -785,7 +866,7 @@ def main(argv=None):
 
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
-        cpu = oracle_baseline(CPU_SAMPLE_T)
+        cpu = oracle_baseline(full=args.cpu_full)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
@@ -807,6 +888,7 @@ def main(argv=None):
                 "roofline_step": roofline_step,
                 "fwd_long": fwd_lines.get("fwd_long"), "fwd_B4": fwd_lines.get("fwd_B4"),
                 "gated_step": gated,
+                "fused_step": fused,
                 "gdn2_step": None if gdn2 is None else dict(ms=gdn2["ms_per_step"], tokens_per_s=gdn2["value"],
                                                             decode_gbs=gdn2["decode"]["value"],
                                                             decode_hbm_frac=gdn2["decode"]["hbm_frac"]),

@@ -15,7 +15,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["fwd", "bwd", "decode", "fwd_gated", "bwd_gated",
+__all__ = ["fwd", "bwd", "decode", "fwd_gated", "bwd_gated", "fwd_fused", "bwd_fused",
            "prologue_fwd", "prologue_bwd", "epilogue_fwd", "epilogue_bwd",
            "gdn2_fwd", "gdn2_bwd", "gdn2_decode",
            "workspace_size", "device_status", "library_path",
@@ -31,6 +31,7 @@ KD_F32, KD_BF16 = 0, 1
 KD_WS_FWD, KD_WS_FWD_SAVE, KD_WS_BWD, KD_WS_PROLOGUE_BWD, KD_WS_EPILOGUE_BWD = 0, 1, 2, 3, 4
 KD_WS_GDN2_FWD, KD_WS_GDN2_BWD = 5, 6
 KD_WS_FWD_GATED, KD_WS_BWD_GATED, KD_WS_BWD_RECOMPUTE = 7, 8, 9
+KD_WS_FWD_FUSED, KD_WS_BWD_FUSED = 10, 11
 KD_PHASE_LOCAL, KD_PHASE_CARRY, KD_PHASE_ALL = 1, 2, 3
 _CODES = {1: "KD_ERR_INVALID_ARG", 2: "KD_ERR_UNSUPPORTED", 3: "KD_ERR_WORKSPACE",
           4: "KD_ERR_CUDA", 5: "KD_ERR_TIMEOUT"}
@@ -75,6 +76,10 @@ def lib():
         L.kron_delta_fwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [vp]
         L.kron_delta_bwd_recompute.restype = i
         L.kron_delta_bwd_recompute.argtypes = [vp] * 16 + [i] * 6 + [vp, sz, vp]
+        L.kron_delta_fwd_fused.restype = i
+        L.kron_delta_fwd_fused.argtypes = [vp] * 7 + [ctypes.c_float] + [vp] * 3 + [i] * 6 + [vp, sz, i, vp]
+        L.kron_delta_bwd_fused.restype = i
+        L.kron_delta_bwd_fused.argtypes = [vp] * 7 + [ctypes.c_float] + [vp] * 11 + [i] * 6 + [vp, sz, vp, sz, vp]
         L.kron_delta_fwd_gated.restype = i
         L.kron_delta_fwd_gated.argtypes = [vp] * 10 + [i] * 6 + [vp, sz, i, vp]
         L.kron_delta_bwd_gated.restype = i
@@ -295,6 +300,69 @@ def bwd_gated(q, k, v, beta, c, f_pre, a_log, S0, dO, dST=None, *, fwd_workspace
                                       fwd_workspace.numel() * fwd_workspace.element_size(),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream(stream)))
+    return g
+
+
+def fwd_fused(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, S0=None, *, out=None,
+              want_state=True, save=False, workspace=None, stream=None):
+    """Forward from the raw projections and gate pre-activations (the input
+    prologue fused into the chunk kernels): equal, up to rounding, to
+    prologue_fwd followed by fwd.  q_raw, k_raw, f_pre [B,T,H,dk] and v_raw
+    [B,T,H,dv] in one dtype; beta_pre, c_pre [B,T,H] and a_log [H] fp32.
+    Returns (out, ST, workspace); pass the workspace (save=True) to bwd_fused."""
+    import torch
+    B, T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    f32 = torch.float32
+    _need(q_raw, "q_raw"); _need(k_raw, "k_raw", q_raw.dtype, q_raw.shape)
+    _need(v_raw, "v_raw", q_raw.dtype, (B, T, H, dv)); _need(f_pre, "f_pre", q_raw.dtype, (B, T, H, dk))
+    _need(beta_pre, "beta_pre", f32, (B, T, H)); _need(c_pre, "c_pre", f32, (B, T, H))
+    _need(a_log, "a_log", f32, (H,)); _need(S0, "S0", f32, (B, H, dv, dk))
+    dt = _dtype_code(q_raw)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q_raw.dtype, device=q_raw.device)
+    _need(out, "out", q_raw.dtype, (B, T, H, dv))
+    ST = torch.empty((B, H, dv, dk), dtype=f32, device=q_raw.device) if want_state else None
+    if workspace is None:
+        workspace = _alloc_ws(workspace_size(KD_WS_FWD_FUSED, B, H, T, dk, dv, dt), q_raw.device)
+    _check(lib().kron_delta_fwd_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(beta_pre), _ptr(c_pre),
+                                      _ptr(f_pre), _ptr(a_log), float(beta_scale), _ptr(S0), _ptr(out), _ptr(ST),
+                                      B, H, T, dk, dv, dt, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), int(bool(save)),
+                                      _stream(stream)))
+    return out, ST, workspace
+
+
+def bwd_fused(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, S0, dO, dST=None, *,
+              fwd_workspace, workspace=None, want_dS0=True, stream=None):
+    """Backward of fwd_fused.  Returns dict dq_raw, dk_raw, dv_raw (input
+    dtype), dbeta_pre, dc_pre, df_pre (fp32), da_log ([H] fp32, fixed-order
+    sum), dS0."""
+    import torch
+    B, T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    f32 = torch.float32
+    _need(q_raw, "q_raw"); _need(k_raw, "k_raw", q_raw.dtype, q_raw.shape)
+    _need(v_raw, "v_raw", q_raw.dtype, (B, T, H, dv)); _need(f_pre, "f_pre", q_raw.dtype, (B, T, H, dk))
+    _need(beta_pre, "beta_pre", f32, (B, T, H)); _need(c_pre, "c_pre", f32, (B, T, H))
+    _need(a_log, "a_log", f32, (H,)); _need(S0, "S0", f32, (B, H, dv, dk))
+    _need(dO, "dO", q_raw.dtype, (B, T, H, dv)); _need(dST, "dST", f32, (B, H, dv, dk))
+    dt = _dtype_code(q_raw)
+    dev = q_raw.device
+    g = dict(dq_raw=torch.empty_like(q_raw), dk_raw=torch.empty_like(k_raw), dv_raw=torch.empty_like(v_raw),
+             dbeta_pre=torch.empty_like(beta_pre), dc_pre=torch.empty_like(c_pre),
+             df_pre=torch.empty((B, T, H, dk), dtype=f32, device=dev),
+             da_log=torch.empty((H,), dtype=f32, device=dev),
+             dS0=torch.empty((B, H, dv, dk), dtype=f32, device=dev) if want_dS0 else None)
+    if workspace is None:
+        workspace = _alloc_ws(workspace_size(KD_WS_BWD_FUSED, B, H, T, dk, dv, dt), dev)
+    _check(lib().kron_delta_bwd_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(beta_pre), _ptr(c_pre),
+                                      _ptr(f_pre), _ptr(a_log), float(beta_scale), _ptr(S0), _ptr(dO), _ptr(dST),
+                                      _ptr(g["dq_raw"]), _ptr(g["dk_raw"]), _ptr(g["dv_raw"]),
+                                      _ptr(g["dbeta_pre"]), _ptr(g["dc_pre"]), _ptr(g["df_pre"]), _ptr(g["da_log"]),
+                                      _ptr(g.get("dS0")), B, H, T, dk, dv, dt, _ptr(fwd_workspace),
+                                      fwd_workspace.numel() * fwd_workspace.element_size(), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)))
     return g
 
 

@@ -79,6 +79,16 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->fwd_save_bytes = off;
   if (!L->tc) L->glogf = take((size_t)B * T * H * dk * 4);  // gated inputs, CUDA-core path: logf
   L->fwd_gated_bytes = off;
+  // fused prologue: the gated beta and c of every token; q, k, v normalised
+  // (tensor-core path: rows of chunks with xflags set, for the exact paths;
+  // CUDA-core path: all, written by the prologue pass)
+  const size_t act = dtype == KD_BF16 ? 2 : 4;
+  L->fbeta = take((size_t)B * T * H * 4);
+  L->fc = take((size_t)B * T * H * 4);
+  L->fq = take((size_t)B * T * H * dk * act);
+  L->fk = take((size_t)B * T * H * dk * act);
+  L->fv = take((size_t)B * T * H * dv * act);
+  L->fwd_fused_bytes = off;
 
   off = 0;
   L->dSC = L->tc ? 0 : take(chunks * (size_t)dv * dk * 4);  // the tensor-core path keeps bf16 tiles
@@ -108,6 +118,18 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   L->bwd_bytes = off;
   if (!L->tc) L->gdlogf = take((size_t)B * T * H * dk * 4);  // gated inputs, CUDA-core path: dlogf
   L->bwd_gated_bytes = off;
+  // fused prologue, CUDA-core path: the recurrence's gradients, then the
+  // prologue backward's own scratch (the tensor-core path finishes in place)
+  if (!L->tc) {
+    L->gdq = take((size_t)B * T * H * dk * act);
+    L->gdk = take((size_t)B * T * H * dk * act);
+    L->gdv = take((size_t)B * T * H * dv * act);
+    L->gdbeta = take((size_t)B * T * H * 4);
+    L->gdc = take((size_t)B * T * H * 4);
+    L->gdf = take((size_t)B * T * H * dk * act);  // the prologue backward's df~ (the fp32 one is formed apart)
+    L->gpro = take((size_t)kd::prologue_blocks((long long)B * T) * H * sizeof(float));
+  }
+  L->bwd_fused_bytes = off;
   return KD_OK;
 }
 
@@ -288,6 +310,8 @@ size_t kron_delta_workspace_size(int kind, int B, int H, int T, int dk, int dv, 
     case KD_WS_FWD_SAVE: ok(); return L.fwd_save_bytes;
     case KD_WS_BWD: ok(); return L.bwd_bytes;
     case KD_WS_BWD_RECOMPUTE: ok(); return recompute_bytes(L, B, H, T, dv, dtype);
+    case KD_WS_FWD_FUSED: ok(); return L.fwd_fused_bytes;
+    case KD_WS_BWD_FUSED: ok(); return L.bwd_fused_bytes;
     case KD_WS_FWD_GATED: ok(); return L.fwd_gated_bytes;
     case KD_WS_BWD_GATED: ok(); return L.bwd_gated_bytes;
     case KD_WS_PROLOGUE_BWD:
@@ -548,6 +572,131 @@ int kron_delta_bwd_gated(const void* q, const void* k, const void* v, const floa
   return launched(e, "gated backward launch");
 }
 
+namespace {
+int check_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
+                   const float* c_pre, const void* f_pre, const float* a_log, float beta_scale, int B,
+                   int H, int T, int dk, int dv, int dtype) {
+  if (B <= 0 || H <= 0 || T <= 0) return fail(KD_ERR_INVALID_ARG, "B, H, T must be >= 1 (got %d, %d, %d)", B, H, T);
+  if (H > 65535) return fail(KD_ERR_INVALID_ARG, "H must be <= 65535 (got %d)", H);
+  if (!dim_supported(dk) || !dim_supported(dv))
+    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
+  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
+  if (!(beta_scale > 0.f && beta_scale <= 2.f))
+    return fail(KD_ERR_INVALID_ARG, "beta_scale must be in (0, 2] (got %g)", (double)beta_scale);
+  KD_TRY(check_ptr(q_raw, "q_raw", true));
+  KD_TRY(check_ptr(k_raw, "k_raw", true));
+  KD_TRY(check_ptr(v_raw, "v_raw", true));
+  KD_TRY(check_ptr(beta_pre, "beta_pre", true));
+  KD_TRY(check_ptr(c_pre, "c_pre", true));
+  KD_TRY(check_ptr(f_pre, "f_pre", true));
+  return check_ptr(a_log, "a_log", true);
+}
+}  // namespace
+
+int kron_delta_fwd_fused(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
+                         const float* c_pre, const void* f_pre, const float* a_log, float beta_scale,
+                         const float* S0, void* out, float* ST, int B, int H, int T, int dk, int dv, int dtype,
+                         void* workspace, size_t ws_bytes, int save, void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk, dv, dtype, &L));
+  KD_TRY(check_prologue(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, B, H, T, dk, dv, dtype));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(out, "out", true));
+  KD_TRY(check_ptr(ST, "ST", false));
+  if (!workspace || ws_bytes < L.fwd_fused_bytes)
+    return fail(KD_ERR_WORKSPACE, "fused forward workspace of %zu bytes needed (got %zu)", L.fwd_fused_bytes,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256)) return fail(KD_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (save != 0 && save != 1) return fail(KD_ERR_INVALID_ARG, "save must be 0 or 1");
+  KD_TRY(check_stream(stream));
+  char* ws = static_cast<char*>(workspace);
+  if (L.tc) {
+    kd::FwdArgs a{q_raw, k_raw, v_raw, beta_pre, c_pre, static_cast<const float*>(f_pre), S0, out, ST, save, ws, L,
+                  KD_PHASE_ALL};
+    a.a_log = a_log;
+    a.pro.bscale = beta_scale;
+    a.pro.norm = 1;
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    return launched(kd::launch_fwd_tc(a, di.err, di.sms, static_cast<cudaStream_t>(stream)), "fused forward launch");
+  }
+  // CUDA-core path: the prologue pass into the workspace, then the forward on its outputs
+  float* logf = kd::ws_ptr<float>(ws, L.glogf);
+  KD_TRY(kron_delta_prologue_fwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, ws + L.fq,
+                                 ws + L.fk, ws + L.fv, kd::ws_ptr<float>(ws, L.fbeta), kd::ws_ptr<float>(ws, L.fc),
+                                 logf, B, H, T, dk, dv, dtype, stream));
+  return kron_delta_fwd(ws + L.fq, ws + L.fk, ws + L.fv, kd::ws_ptr<float>(ws, L.fbeta), kd::ws_ptr<float>(ws, L.fc),
+                        logf, S0, out, ST, B, H, T, dk, dv, dtype, workspace, L.fwd_save_bytes, save, stream);
+}
+
+int kron_delta_bwd_fused(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
+                         const float* c_pre, const void* f_pre, const float* a_log, float beta_scale,
+                         const float* S0, const void* dO, const float* dST, void* dq_raw, void* dk_raw,
+                         void* dv_raw, float* dbeta_pre, float* dc_pre, float* df_pre, float* da_log, float* dS0,
+                         int B, int H, int T, int dk, int dv, int dtype, const void* fwd_ws, size_t fwd_ws_bytes,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  kd::Layout L;
+  KD_TRY(plan(B, H, T, dk, dv, dtype, &L));
+  KD_TRY(check_prologue(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, B, H, T, dk, dv, dtype));
+  KD_TRY(check_ptr(S0, "S0", false));
+  KD_TRY(check_ptr(dO, "dO", true));
+  KD_TRY(check_ptr(dST, "dST", false));
+  KD_TRY(check_ptr(dq_raw, "dq_raw", true));
+  KD_TRY(check_ptr(dk_raw, "dk_raw", true));
+  KD_TRY(check_ptr(dv_raw, "dv_raw", true));
+  KD_TRY(check_ptr(dbeta_pre, "dbeta_pre", true));
+  KD_TRY(check_ptr(dc_pre, "dc_pre", true));
+  KD_TRY(check_ptr(df_pre, "df_pre", true));
+  KD_TRY(check_ptr(da_log, "da_log", true));
+  KD_TRY(check_ptr(dS0, "dS0", false));
+  if (!fwd_ws || fwd_ws_bytes < L.fwd_fused_bytes)
+    return fail(KD_ERR_WORKSPACE, "the fused forward's workspace (save=1) of %zu bytes needed (got %zu)",
+                L.fwd_fused_bytes, fwd_ws ? fwd_ws_bytes : 0);
+  if (!workspace || ws_bytes < L.bwd_fused_bytes)
+    return fail(KD_ERR_WORKSPACE, "fused backward workspace of %zu bytes needed (got %zu)", L.bwd_fused_bytes,
+                workspace ? ws_bytes : 0);
+  if (!aligned(workspace, 256) || !aligned(fwd_ws, 256))
+    return fail(KD_ERR_WORKSPACE, "workspaces must be 256-byte aligned");
+  KD_TRY(check_stream(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const char* fws = static_cast<const char*>(fwd_ws);
+  float* dapart = kd::ws_ptr<float>(ws, L.dapart);
+  if (L.tc) {
+    // the chunk kernels write the gradients of the normalised q, k, v and of
+    // the gated beta, c into the outputs, and df~ with its da_log parts; the
+    // tail pass then carries the first five through the prologue in place
+    kd::BwdArgs a{q_raw, k_raw, v_raw, beta_pre, c_pre, static_cast<const float*>(f_pre), S0, dO, dST, dq_raw,
+                  dk_raw, dv_raw, dbeta_pre, dc_pre, df_pre, dS0, fws, ws, L, KD_PHASE_ALL};
+    a.a_log = a_log;
+    a.pro.bscale = beta_scale;
+    a.pro.norm = 1;
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    cudaError_t e = kd::launch_bwd_tc(a, di.err, di.sms, st);
+    if (e == cudaSuccess) e = kd::launch_reduce_dalog(dapart, B, H, L.NC, da_log, st);
+    if (e == cudaSuccess)
+      e = kd::launch_prologue_tail_bwd(q_raw, k_raw, v_raw, beta_pre, c_pre, beta_scale, dq_raw, dk_raw, dv_raw,
+                                       dbeta_pre, dc_pre, (size_t)B * T * H, st);
+    return launched(e, "fused backward launch");
+  }
+  // CUDA-core path: the backward on the prologue's outputs, then the prologue's
+  // backward; df~ (fp32) and da_log are formed from dlogf as on the gated path
+  const float* logf = kd::ws_ptr<float>(fws, L.glogf);
+  float* gdlogf = kd::ws_ptr<float>(ws, L.gdlogf);
+  KD_TRY(kron_delta_bwd(fws + L.fq, fws + L.fk, fws + L.fv, kd::ws_ptr<float>(fws, L.fbeta),
+                        kd::ws_ptr<float>(fws, L.fc), logf, S0, dO, dST, ws + L.gdq, ws + L.gdk, ws + L.gdv,
+                        kd::ws_ptr<float>(ws, L.gdbeta), kd::ws_ptr<float>(ws, L.gdc), gdlogf, dS0, B, H, T, dk, dv,
+                        dtype, fwd_ws, L.fwd_save_bytes, workspace, L.bwd_bytes, stream));
+  KD_TRY(kron_delta_prologue_bwd(q_raw, k_raw, v_raw, beta_pre, c_pre, f_pre, a_log, beta_scale, ws + L.gdq,
+                                 ws + L.gdk, ws + L.gdv, kd::ws_ptr<float>(ws, L.gdbeta), kd::ws_ptr<float>(ws, L.gdc),
+                                 gdlogf, dq_raw, dk_raw, dv_raw, dbeta_pre, dc_pre, ws + L.gdf, da_log, B, H, T, dk,
+                                 dv, dtype, ws + L.gpro, ws_bytes - L.gpro, stream));
+  cudaError_t e = kd::launch_gate_dlogf(gdlogf, logf, a_log, df_pre, dapart, B, T, H, dk, L.NC, st);
+  if (e == cudaSuccess) e = kd::launch_reduce_dalog(dapart, B, H, L.NC, da_log, st);
+  return launched(e, "fused backward launch");
+}
+
 int kron_delta_decode(const void* q, const void* k, const void* v, const float* beta,
                       const float* c, const float* logf, float* S, void* out, int B, int H,
                       int dk, int dv, int dtype, void* stream) {
@@ -569,26 +718,6 @@ int kron_delta_decode(const void* q, const void* k, const void* v, const float* 
   return launched(kd::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
 }
 
-namespace {
-int check_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
-                   const float* c_pre, const void* f_pre, const float* a_log, float beta_scale, int B,
-                   int H, int T, int dk, int dv, int dtype) {
-  if (B <= 0 || H <= 0 || T <= 0) return fail(KD_ERR_INVALID_ARG, "B, H, T must be >= 1 (got %d, %d, %d)", B, H, T);
-  if (H > 65535) return fail(KD_ERR_INVALID_ARG, "H must be <= 65535 (got %d)", H);
-  if (!dim_supported(dk) || !dim_supported(dv))
-    return fail(KD_ERR_UNSUPPORTED, "dk and dv must be 32, 64 or 128 (got %d, %d)", dk, dv);
-  if (dtype != KD_F32 && dtype != KD_BF16) return fail(KD_ERR_UNSUPPORTED, "dtype must be KD_F32 or KD_BF16 (got %d)", dtype);
-  if (!(beta_scale > 0.f && beta_scale <= 2.f))
-    return fail(KD_ERR_INVALID_ARG, "beta_scale must be in (0, 2] (got %g)", (double)beta_scale);
-  KD_TRY(check_ptr(q_raw, "q_raw", true));
-  KD_TRY(check_ptr(k_raw, "k_raw", true));
-  KD_TRY(check_ptr(v_raw, "v_raw", true));
-  KD_TRY(check_ptr(beta_pre, "beta_pre", true));
-  KD_TRY(check_ptr(c_pre, "c_pre", true));
-  KD_TRY(check_ptr(f_pre, "f_pre", true));
-  return check_ptr(a_log, "a_log", true);
-}
-}  // namespace
 
 int kron_delta_prologue_fwd(const void* q_raw, const void* k_raw, const void* v_raw,
                             const float* beta_pre, const float* c_pre, const void* f_pre,

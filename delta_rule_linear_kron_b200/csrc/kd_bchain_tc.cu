@@ -566,7 +566,9 @@ cudaError_t launch_bchain_r(const BwdArgs& a, int* err, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(st, "bwd_chain_tc");
-  e = cudaLaunchKernelEx(&cfg, bwd_chain_tc<R>, tm_do, tm_ke, tm_kp, a.beta, a.dST, a.dS0, L.H, L.T, L.NC,
+  // fused prologue: beta as gated by the forward's preparation kernel
+  const float* beta = a.pro.bscale > 0.f ? ws_ptr<const float>(a.fws, L.fbeta) : a.beta;
+  e = cudaLaunchKernelEx(&cfg, bwd_chain_tc<R>, tm_do, tm_ke, tm_kp, beta, a.dST, a.dS0, L.H, L.T, L.NC,
                          ws_ptr<const float>(a.fws, L.A), ws_ptr<const float>(a.fws, L.Hx),
                          ws_ptr<const float>(a.fws, L.GC), ws_ptr<const __nv_bfloat16>(a.fws, L.Vt),
                          (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.QpT),

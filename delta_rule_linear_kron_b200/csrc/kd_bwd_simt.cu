@@ -753,10 +753,15 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
   if (only) {
     // tensor-core path: the flagged chunks only, all stages in one kernel
     if (stages != (kStageCC | kStageState | kStageIntra)) return cudaErrorInvalidValue;
+    // fused prologue: the flagged chunks' normalised q, k, v rows and the
+    // gated beta, from the forward's preparation kernel
+    const bool nrm = a.pro.norm != 0;
+    const float* beta = a.pro.bscale > 0.f ? ws_ptr<float>(a.fws, L.fbeta) : a.beta;
     prof_begin(st, "bwd_exact_simt");
     bwd_exact_simt<DK, DV, Tin><<<(unsigned)(L.chunks < (size_t)kExactSlots ? L.chunks : kExactSlots), 256, s5,
                                   st>>>(
-        q, k, v, a.beta, a.a_log ? nullptr : a.logf,
+        nrm ? ws_ptr<Tin>(a.fws, L.fq) : q, nrm ? ws_ptr<Tin>(a.fws, L.fk) : k,
+        nrm ? ws_ptr<Tin>(a.fws, L.fv) : v, beta, a.a_log ? nullptr : a.logf,
         a.a_log ? reinterpret_cast<const __nv_bfloat16*>(a.logf) : nullptr, a.a_log, dO, L.H, L.T, L.NC, L.chunks,
         wP, wu, wb0, wg, wS0, ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), a.dbeta, a.dc, wdP, wdGK, wdGVs, waccq, wacck,
         waccL, waccv, static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf,

@@ -87,6 +87,57 @@ __device__ __forceinline__ void gate_logf_tile(float* dst, const unsigned char* 
   __syncthreads();
 }
 
+// ---- the rest of the fused input prologue (struct Pro in kd_kernels.h) ----
+// The L2 normalisation's epsilon: x / sqrt(|x|^2 + kNormEps).
+constexpr float kNormEps = 1e-6f;
+
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float gate_beta(float x, Pro p) { return p.bscale > 0.f ? p.bscale * sigmoid_f(x) : x; }
+__device__ __forceinline__ float gate_c(float x, Pro p) { return p.bscale > 0.f ? sigmoid_f(x) : x; }
+// d sigma(x) / dx = sigma(x) sigma(-x), each factor formed directly (no 1 - sigma cancellation)
+__device__ __forceinline__ float dsigmoid_f(float x) { return sigmoid_f(x) * sigmoid_f(-x); }
+
+// Normalises the rows of a [64][128] bf16 tile in shared memory in place.  Row
+// t is two 128-byte halves, at seg0 + t * pitch and seg1 + t * pitch, each
+// holding 64 channels in any order of its 16-byte chunks (a 128-byte swizzle
+// permutes chunks only within a row, so the row's norm and scaling do not
+// depend on it).  Four threads take a row, two chunks of each half apiece;
+// each rewrites only what it read, so there is no barrier inside; the caller
+// places one before any other thread reads the tile.  Zero rows (the padded
+// tail) stay zero.  All 256 threads of the CTA call it.
+__device__ __forceinline__ void l2norm_tile(unsigned char* seg0, unsigned char* seg1, int pitch) {
+  const int t = threadIdx.x >> 2, q = threadIdx.x & 3;
+  uint4* p[4] = {reinterpret_cast<uint4*>(seg0 + t * pitch + q * 16),
+                 reinterpret_cast<uint4*>(seg0 + t * pitch + (q + 4) * 16),
+                 reinterpret_cast<uint4*>(seg1 + t * pitch + q * 16),
+                 reinterpret_cast<uint4*>(seg1 + t * pitch + (q + 4) * 16)};
+  uint4 x[4];
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    x[c] = *p[c];
+    const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&x[c]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(e[i]);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  const float r = rsqrtf(ss + kNormEps);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&x[c]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(e[i]);
+      e[i] = __floats2bfloat162_rn(f.x * r, f.y * r);
+    }
+    *p[c] = x[c];
+  }
+}
+
 // One log-decay value from global memory: logf itself, or formed from the
 // forget pre-activation (gated inputs, fpre != nullptr).
 template <typename Tf>

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_logf,
     const __grid_constant__ CUtensorMap tm_out, int H, int T, int NC, const __nv_bfloat16* __restrict__ wS0b,
-    const float* __restrict__ wu, int* __restrict__ unsafe_flags, const float* __restrict__ a_log,
+    const float* __restrict__ wu, int* __restrict__ unsafe_flags, const float* __restrict__ a_log, Pro pro,
     int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -92,6 +92,12 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  if (pro.norm) {  // fused prologue: q, k, v arrive raw and are normalised in place
+    l2norm_tile(sm + OutCfg::QR, sm + OutCfg::QR + 128, 256);
+    l2norm_tile(sm + OutCfg::KR, sm + OutCfg::KR + 128, 256);
+    l2norm_tile(sm + OutCfg::VB, sm + OutCfg::VB + 8192, 128);
+    __syncthreads();
+  }
   if (a_log)  // gated inputs: the bf16 forget pre-activations become logf in place
     gate_logf_tile(reinterpret_cast<float*>(sm + OutCfg::LG), sm + OutCfg::LG + 16384, expf(a_log[h]),
                    min(C, T - t0));
@@ -309,7 +315,8 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf,
     const float* __restrict__ beta, const float* __restrict__ c, int H, int T, int NC, float* __restrict__ wy,
     float* __restrict__ wA, float* __restrict__ wP, int* __restrict__ wxflags, const float* __restrict__ a_log,
-    int* __restrict__ err) {
+    Pro pro, float* __restrict__ fbeta, float* __restrict__ fc, __nv_bfloat16* __restrict__ fq,
+    __nv_bfloat16* __restrict__ fk, __nv_bfloat16* __restrict__ fv, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -344,14 +351,24 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
   if (tid < C) {
     const bool ok = tid < nv;
     const size_t g = ((size_t)b * T + t0 + tid) * H + h;
-    bs[tid] = ok ? beta[g] : 0.f;
-    cs[tid] = ok ? c[g] : 0.f;
+    bs[tid] = ok ? gate_beta(beta[g], pro) : 0.f;
+    cs[tid] = ok ? gate_c(c[g], pro) : 0.f;
+    if (pro.bscale > 0.f && ok) {  // fused prologue: the gated values, for the chain and the backward
+      fbeta[g] = bs[tid];
+      fc[g] = cs[tid];
+    }
   }
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  if (pro.norm) {  // fused prologue: q, k, v arrive raw and are normalised in place
+    l2norm_tile(sm + PrepCfg::QR, sm + PrepCfg::QR + 128, 256);
+    l2norm_tile(sm + PrepCfg::KR, sm + PrepCfg::KR + 128, 256);
+    l2norm_tile(sm + PrepCfg::VT, sm + PrepCfg::VT + 8192, 128);
+    __syncthreads();
+  }
   if (a_log)  // gated inputs: the bf16 forget pre-activations become logf in place
     gate_logf_tile(Ls, sm + PrepCfg::LS + 16384, expf(a_log[h]), nv);
   // decay prefix (thread (j, half) covers 32 positions; L is written back for
@@ -386,6 +403,18 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
   const bool is_unsafe = __syncthreads_or(!(mx < kSafeLogRange)) != 0;
   const bool exact_state = __syncthreads_or(!(mx < kExactStateRange)) != 0;
   if (tid == 0) wxflags[ch] = exact_state ? 1 : 0;
+  if (pro.norm && exact_state) {
+    // fused prologue: the exact paths (CUDA cores, global loads) read this
+    // chunk's normalised q, k, v rows from the workspace
+    for (int e = tid; e < nv * (D / 8); e += 256) {
+      const int t = e / (D / 8), c8 = e % (D / 8);
+      const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + 8 * c8;
+      *reinterpret_cast<uint4*>(fq + g) = *reinterpret_cast<const uint4*>(sm + PrepCfg::QR + (t * D + 8 * c8) * 2);
+      *reinterpret_cast<uint4*>(fk + g) = *reinterpret_cast<const uint4*>(sm + PrepCfg::KR + (t * D + 8 * c8) * 2);
+      *reinterpret_cast<uint4*>(fv + g) = *reinterpret_cast<const uint4*>(
+          sm + PrepCfg::VT + (c8 / 8) * 8192 + tc::sw128_off(t, 8 * (c8 % 8), 64, 2));
+    }
+  }
   tc::fence_proxy_async();
   tc::tc_before_sync();
   __syncthreads();
@@ -550,7 +579,7 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_logf, const __grid_constant__ CUtensorMap tm_kt,
     const __grid_constant__ CUtensorMap tm_ke, int H, int T, int NC, float* __restrict__ wGC,
-    float* __restrict__ wHx, __nv_bfloat16* __restrict__ wVt, const float* __restrict__ a_log,
+    float* __restrict__ wHx, __nv_bfloat16* __restrict__ wVt, const float* __restrict__ a_log, Pro pro,
     int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -588,6 +617,15 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  if (pro.norm) {  // fused prologue: v and k of both chunks arrive raw and are normalised in place
+    l2norm_tile(sm + CrossCfg::VV, sm + CrossCfg::VV + 16384, 128);
+    l2norm_tile(sm + CrossCfg::KR, sm + CrossCfg::KR + 128, 256);
+    if (has_prev) {
+      l2norm_tile(sm + CrossCfg::VV + 8192, sm + CrossCfg::VV + 24576, 128);
+      l2norm_tile(sm + CrossCfg::KR + 16384, sm + CrossCfg::KR + 16384 + 128, 256);
+    }
+    __syncthreads();
+  }
   if (a_log) {  // gated inputs: the bf16 forget pre-activations become logf in place
     const float ga = expf(a_log[h]);
     gate_logf_tile(reinterpret_cast<float*>(sm + CrossCfg::LG), sm + CrossCfg::LG + 16384, ga, min(C, T - t0));
@@ -725,7 +763,9 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     prof_begin(st, "fwd_prep_tc");
     fwd_prep_tc<<<(unsigned)L.chunks, 256, PrepCfg::BYTES, st>>>(
         tm_v, tm_q, tm_k, tm_logf, a.beta, a.c, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
-        a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, ws_ptr<int>(a.ws, L.xflags), a.a_log, err);
+        a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, ws_ptr<int>(a.ws, L.xflags), a.a_log, a.pro,
+        ws_ptr<float>(a.ws, L.fbeta), ws_ptr<float>(a.ws, L.fc), ws_ptr<__nv_bfloat16>(a.ws, L.fq),
+        ws_ptr<__nv_bfloat16>(a.ws, L.fk), ws_ptr<__nv_bfloat16>(a.ws, L.fv), err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     CUtensorMap tm_kt, tm_ke;
@@ -738,7 +778,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     prof_begin(st, "fwd_cross_tc");
     fwd_cross_tc<<<(unsigned)L.chunks, 256, CrossCfg::BYTES, st>>>(
         tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx),
-        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), a.a_log, err);
+        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), a.a_log, a.pro, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -762,7 +802,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     prof_begin(st, "fwd_out_tc");
     fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(
         tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.T, L.NC, (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.S0b),
-        wu, flags, a.a_log, err);
+        wu, flags, a.a_log, a.pro, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -771,9 +811,12 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
       cudaSuccess)
     return e;
   prof_begin(st, "fwd_out_fixup");
+  // fused prologue: the flagged chunks' normalised q, k, v rows, from the preparation kernel
+  const bool nrm = a.pro.norm != 0;
   fwd_out_fixup<<<(unsigned)L.chunks, 128, kFixSmem, st>>>(
-      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-      static_cast<const __nv_bfloat16*>(a.v), a.a_log ? nullptr : a.logf,
+      nrm ? ws_ptr<__nv_bfloat16>(a.ws, L.fq) : static_cast<const __nv_bfloat16*>(a.q),
+      nrm ? ws_ptr<__nv_bfloat16>(a.ws, L.fk) : static_cast<const __nv_bfloat16*>(a.k),
+      nrm ? ws_ptr<__nv_bfloat16>(a.ws, L.fv) : static_cast<const __nv_bfloat16*>(a.v), a.a_log ? nullptr : a.logf,
       a.a_log ? reinterpret_cast<const __nv_bfloat16*>(a.logf) : nullptr, a.a_log, L.H, L.T, L.NC, blob, wu, flags,
       static_cast<__nv_bfloat16*>(a.out));
   prof_end(st);

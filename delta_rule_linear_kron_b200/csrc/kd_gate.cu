@@ -1,4 +1,6 @@
-// kd_gate.cu -- gated inputs: the forget gate formed from its pre-activation.
+// kd_gate.cu -- gated inputs and the fused prologue: the forget gate formed
+// from its pre-activation, and the backward through the normalisation and the
+// erase/write gate sigmoids.
 //
 // KronLSTM digest, "어떻게 쓰나": the forget gate is f = sigma(f~)^a with
 // a = e^{a_log} per head, so logf = a log sigma(f~).  Its backward:
@@ -63,7 +65,63 @@ __global__ void __launch_bounds__(32) reduce_dalog_kernel(const float* __restric
   if (lane == 0) da_log[h] = s;
 }
 
+// The fused prologue's backward through the normalisation and the gate
+// sigmoids (tensor-core path: bf16, d = 128), in place on the gradients the
+// chunk kernels wrote for the normalised q, k, v and the gated beta, c.  With
+// y = x r, r = (|x|^2 + eps)^(-1/2), the gradient of x is r (dy - y (y . dy));
+// beta = s sigma(x) gives dx = dbeta s sigma(x) sigma(-x), and c likewise with
+// s = 1.  One warp per token and head, each lane four channels.
+__global__ void __launch_bounds__(256) prologue_tail_bwd(const __nv_bfloat16* __restrict__ q_raw,
+                                                         const __nv_bfloat16* __restrict__ k_raw,
+                                                         const __nv_bfloat16* __restrict__ v_raw,
+                                                         const float* __restrict__ beta_pre,
+                                                         const float* __restrict__ c_pre, float bscale,
+                                                         __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
+                                                         __nv_bfloat16* __restrict__ dv, float* __restrict__ dbeta,
+                                                         float* __restrict__ dc, size_t rows) {
+  const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const __nv_bfloat16* xs[3] = {q_raw, k_raw, v_raw};
+  __nv_bfloat16* ds[3] = {dq, dk, dv};
+#pragma unroll
+  for (int m = 0; m < 3; ++m) {
+    const size_t o = row * 128 + 4 * lane;
+    const uint2 xr = *reinterpret_cast<const uint2*>(xs[m] + o);
+    const uint2 dr = *reinterpret_cast<const uint2*>(ds[m] + o);
+    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xr);
+    const __nv_bfloat162* dp = reinterpret_cast<const __nv_bfloat162*>(&dr);
+    const float2 x0 = __bfloat1622float2(xp[0]), x1 = __bfloat1622float2(xp[1]);
+    const float2 d0 = __bfloat1622float2(dp[0]), d1 = __bfloat1622float2(dp[1]);
+    const float ss = warp_sum(fmaf(x0.x, x0.x, fmaf(x0.y, x0.y, fmaf(x1.x, x1.x, x1.y * x1.y))));
+    const float r = rsqrtf(ss + kNormEps);
+    const float dot = warp_sum(fmaf(x0.x, d0.x, fmaf(x0.y, d0.y, fmaf(x1.x, d1.x, x1.y * d1.y)))) * r;  // y . dy
+    uint2 out;
+    __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&out);
+    const float rd = r * dot * r;  // r (y . dy) r: y = x r
+    op[0] = __floats2bfloat162_rn(fmaf(-x0.x, rd, r * d0.x), fmaf(-x0.y, rd, r * d0.y));
+    op[1] = __floats2bfloat162_rn(fmaf(-x1.x, rd, r * d1.x), fmaf(-x1.y, rd, r * d1.y));
+    *reinterpret_cast<uint2*>(ds[m] + o) = out;
+  }
+  if (lane == 0) {
+    dbeta[row] *= bscale * dsigmoid_f(beta_pre[row]);
+    dc[row] *= dsigmoid_f(c_pre[row]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_prologue_tail_bwd(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
+                                     const float* c_pre, float bscale, void* dq, void* dk, void* dv, float* dbeta,
+                                     float* dc, size_t rows, cudaStream_t st) {
+  prof_begin(st, "prologue_tail_bwd");
+  prologue_tail_bwd<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(k_raw),
+      static_cast<const __nv_bfloat16*>(v_raw), beta_pre, c_pre, bscale, static_cast<__nv_bfloat16*>(dq),
+      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dbeta, dc, rows);
+  prof_end(st);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gate_logf(const void* fpre, int dtype, const float* a_log, float* logf, int B, int T, int H,
                              int dk, cudaStream_t st) {

@@ -18,6 +18,16 @@ constexpr int kChunk = 64;
 // number of chunks.
 constexpr int kExactSlots = 128;
 
+// The fused input prologue inside the chunk kernels (KronLSTM digest, "어떻게
+// 쓰나"): the erase and write gates arrive as pre-activations (beta = s
+// sigma(x), c = sigma(x)), and q, k, v as raw projections, L2-normalised per
+// token and head, x / sqrt(|x|^2 + 1e-6), where a kernel loads them.  Both
+// zero: the inputs are the recurrence's own.
+struct Pro {
+  float bscale = 0.f;  // > 0: beta and c are pre-activations, beta = bscale sigma(.), c = sigma(.)
+  int norm = 0;        // 1: q, k, v are raw
+};
+
 // Workspace layout of one problem (B, H, T, dk, dv), decided by the chunk
 // scheduler.  Offsets are in bytes from the workspace base, 256-byte aligned.
 // "chunk" index ch = ((b * H) + h) * NC + n.
@@ -67,6 +77,15 @@ struct Layout {
   // the tensor-core kernels read the pre-activations directly.
   size_t glogf = 0, gdlogf = 0;
   size_t fwd_gated_bytes = 0, bwd_gated_bytes = 0;
+  // Fused prologue (raw q, k, v and gate pre-activations).  Forward: the
+  // gated beta and c [B][T][H] (fp32) of every token, and normalised q, k, v
+  // [B][T][H][d] (activation dtype): on the tensor-core path only the rows of
+  // chunks with xflags set (the exact paths read them), on the CUDA-core path
+  // all of them.  Backward, CUDA-core path: the recurrence's gradients and the
+  // prologue backward's scratch.
+  size_t fbeta = 0, fc = 0, fq = 0, fk = 0, fv = 0;
+  size_t gdq = 0, gdk = 0, gdv = 0, gdbeta = 0, gdc = 0, gdf = 0, gpro = 0;
+  size_t fwd_fused_bytes = 0, bwd_fused_bytes = 0;
 };
 
 // Phases of a forward or backward call.  kPhaseLocal: the work that does not
@@ -96,6 +115,7 @@ struct FwdArgs {
   // gated inputs (tensor-core path): logf then points at the bf16 forget
   // pre-activations and a_log at the per-head exponents; nullptr otherwise
   const float* a_log = nullptr;
+  Pro pro;  // fused prologue (tensor-core path)
   // false: stop after the chunk chain (the backward's recompute of the saved
   // quantities needs no output; tensor-core path)
   bool keep_out = true;
@@ -116,6 +136,7 @@ struct BwdArgs {
   // pre-activations, dlogf receives df~ (fp32) and a_log holds the per-head
   // exponents; nullptr otherwise
   const float* a_log = nullptr;
+  Pro pro;  // fused prologue (tensor-core path): dbeta and dc then receive the pre-activations' gradients
 };
 
 // Sets the calling thread's kron_delta_last_error() string.
@@ -243,6 +264,9 @@ cudaError_t launch_gate_logf(const void* fpre, int dtype, const float* a_log, fl
                              int dk, cudaStream_t st);
 cudaError_t launch_gate_dlogf(const float* dlogf, const float* logf, const float* a_log, float* dfpre,
                               float* dapart, int B, int T, int H, int dk, int NC, cudaStream_t st);
+cudaError_t launch_prologue_tail_bwd(const void* q_raw, const void* k_raw, const void* v_raw, const float* beta_pre,
+                                     const float* c_pre, float bscale, void* dq, void* dk, void* dv, float* dbeta,
+                                     float* dc, size_t rows, cudaStream_t st);
 cudaError_t launch_reduce_dalog(const float* dapart, int B, int H, int NC, float* da_log, cudaStream_t st);
 
 // Failure-reporting self-test (kd_selftest.cu): a bounded wait that runs out.

@@ -36,12 +36,6 @@
 
 namespace kd {
 
-namespace {
-
-constexpr float kNormEps = 1e-6f;
-
-}  // namespace
-
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(256) prologue_fwd_kernel(
     const Tin* __restrict__ qr, const Tin* __restrict__ kr, const Tin* __restrict__ vr,

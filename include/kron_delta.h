@@ -28,7 +28,9 @@
  *                         carried state, for context parallelism),
  *                         kron_delta_fwd_noalloc,
  *                         kron_delta_fwd_gated / _bwd_gated (forget gate
- *                         from its pre-activation, formed inside the kernels)
+ *                         from its pre-activation, formed inside the kernels),
+ *                         kron_delta_fwd_fused / _bwd_fused (the whole input
+ *                         prologue inside the kernels)
  *   around the mixer      kron_delta_prologue_fwd / _bwd (L2-norm, gates,
  *                         log-decay), kron_delta_epilogue_fwd / _bwd
  *                         (per-head RMSNorm and output gate)
@@ -104,6 +106,8 @@ extern "C" {
 #define KD_WS_FWD_GATED 7     /* kron_delta_fwd_gated (kept for kron_delta_bwd_gated) */
 #define KD_WS_BWD_GATED 8     /* backward scratch of kron_delta_bwd_gated */
 #define KD_WS_BWD_RECOMPUTE 9 /* kron_delta_bwd_recompute (forward scratch included) */
+#define KD_WS_FWD_FUSED 10    /* kron_delta_fwd_fused (kept for kron_delta_bwd_fused) */
+#define KD_WS_BWD_FUSED 11    /* backward scratch of kron_delta_bwd_fused */
 
 /* phases of kron_delta_fwd_phase / kron_delta_bwd_phase */
 #define KD_PHASE_LOCAL 1   /* the work that does not depend on the carried state */
@@ -224,6 +228,50 @@ KD_API int kron_delta_bwd_gated(const void *q, const void *k, const void *v,
                          int H, int T, int dk_, int dv_, int dtype, const void *fwd_ws,
                          size_t fwd_ws_bytes, void *workspace, size_t ws_bytes,
                          void *stream);
+
+/*
+ * Forward and backward with the whole input prologue fused into the chunk
+ * kernels (KronLSTM digest, section "어떻게 쓰나"): the inputs are the raw
+ * projections and gate pre-activations of kron_delta_prologue_fwd, and the
+ * result equals kron_delta_prologue_fwd followed by kron_delta_fwd (and, for
+ * the backward, kron_delta_bwd followed by kron_delta_prologue_bwd) up to
+ * rounding.  On the tensor-core path (bf16, dk = dv = 128) no normalised or
+ * gated copy of the inputs is written: each chunk kernel normalises the q, k,
+ * v rows it loads (x / sqrt(|x|^2 + 1e-6), rounded to bf16 as the prologue
+ * would store them), the preparation kernel applies the gate sigmoids and
+ * keeps the gated beta, c (8 bytes per token and head) for the chain, and
+ * logf is formed from f_pre as in kron_delta_fwd_gated.  The backward's chunk
+ * kernels form df_pre and da_log in their epilogue; one row-wise pass then
+ * carries the gradients of the normalised q, k, v and of the gated beta, c
+ * through the normalisation and the sigmoids, in place in the outputs.  Other
+ * shapes run kron_delta_prologue_fwd / _bwd around the plain calls, inside the
+ * workspace.
+ *   q_raw, k_raw, f_pre [B,T,H,dk], v_raw [B,T,H,dv] (dtype); beta_pre, c_pre
+ *   [B,T,H] fp32; a_log [H] fp32; beta_scale in (0, 2], as for
+ *   kron_delta_prologue_fwd.
+ *   workspace (forward) : at least kron_delta_workspace_size(KD_WS_FWD_FUSED, ...);
+ *         pass it with save = 1 to kron_delta_bwd_fused as fwd_ws.
+ *   dq_raw, dk_raw [B,T,H,dk], dv_raw [B,T,H,dv] (dtype); dbeta_pre, dc_pre
+ *   [B,T,H] fp32; df_pre [B,T,H,dk] fp32; da_log [H] fp32 (fixed-order sum,
+ *   bitwise reproducible).
+ *   workspace (backward) : at least kron_delta_workspace_size(KD_WS_BWD_FUSED, ...).
+ * S0, out, ST, dO, dST, dS0 and the errors are those of kron_delta_fwd and
+ * kron_delta_bwd (beta_scale outside (0, 2] gives KD_ERR_INVALID_ARG).
+ * Asynchronous on `stream`.
+ */
+KD_API int kron_delta_fwd_fused(const void *q_raw, const void *k_raw, const void *v_raw,
+                                const float *beta_pre, const float *c_pre, const void *f_pre,
+                                const float *a_log, float beta_scale, const float *S0, void *out,
+                                float *ST, int B, int H, int T, int dk, int dv, int dtype,
+                                void *workspace, size_t ws_bytes, int save, void *stream);
+KD_API int kron_delta_bwd_fused(const void *q_raw, const void *k_raw, const void *v_raw,
+                                const float *beta_pre, const float *c_pre, const void *f_pre,
+                                const float *a_log, float beta_scale, const float *S0,
+                                const void *dO, const float *dST, void *dq_raw, void *dk_raw,
+                                void *dv_raw, float *dbeta_pre, float *dc_pre, float *df_pre,
+                                float *da_log, float *dS0, int B, int H, int T, int dk, int dv,
+                                int dtype, const void *fwd_ws, size_t fwd_ws_bytes,
+                                void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * The forward and backward split at the carried state, for a caller that

@@ -58,7 +58,7 @@ def test_workspace_sizes(L):
     assert kd.workspace_size(kd.KD_WS_FWD, 1, 1, 65, 32, 32) > kd.workspace_size(kd.KD_WS_FWD, 1, 1, 64, 32, 32)
     assert L.kron_delta_workspace_size(0, 1, 1, 64, 48, 32, 1) == 0
     assert b"32, 64 or 128" in L.kron_delta_last_error()
-    assert L.kron_delta_workspace_size(10, 1, 1, 64, 32, 32, 1) == 0
+    assert L.kron_delta_workspace_size(12, 1, 1, 64, 32, 32, 1) == 0
     # the backward with recompute holds a save-forward workspace and the backward's
     # own (the CUDA-core path, whose forward always writes an output, one more buffer)
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
