@@ -77,7 +77,7 @@ int plan(int B, int H, int T, int dk, int dv, int dtype, kd::Layout* L) {
   if (L->tc) L->S0b = take(chunks * (size_t)dv * dk * 2);
   if (L->tc) L->fwd_bytes = off;  // the chain writes u, b0 and the chunk-start states on every call
   L->fwd_save_bytes = off;
-  if (!L->tc) L->glogf = take((size_t)B * T * H * dk * 4);  // gated inputs, CUDA-core path: logf
+  L->glogf = take((size_t)B * T * H * dk * 4);  // gated inputs: logf, formed once
   L->fwd_gated_bytes = off;
   // fused prologue: the gated beta and c of every token; q, k, v normalised
   // (tensor-core path: rows of chunks with xflags set, for the exact paths;

@@ -566,9 +566,7 @@ cudaError_t launch_bchain_r(const BwdArgs& a, int* err, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(st, "bwd_chain_tc");
-  // fused prologue: beta as gated by the forward's preparation kernel
-  const float* beta = a.pro.bscale > 0.f ? ws_ptr<const float>(a.fws, L.fbeta) : a.beta;
-  e = cudaLaunchKernelEx(&cfg, bwd_chain_tc<R>, tm_do, tm_ke, tm_kp, beta, a.dST, a.dS0, L.H, L.T, L.NC,
+  e = cudaLaunchKernelEx(&cfg, bwd_chain_tc<R>, tm_do, tm_ke, tm_kp, a.beta, a.dST, a.dS0, L.H, L.T, L.NC,
                          ws_ptr<const float>(a.fws, L.A), ws_ptr<const float>(a.fws, L.Hx),
                          ws_ptr<const float>(a.fws, L.GC), ws_ptr<const __nv_bfloat16>(a.fws, L.Vt),
                          (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.QpT),
@@ -587,7 +585,29 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, int R, int* err, cudaStream_t 
 // The tensor-core backward: per-chunk adjoints (bwd_pre_tc), the reverse
 // chain, the per-chunk gradients (bwd_post_tc), then the exact CUDA-core
 // stages for chunks flagged outside the factorised decay range.
-cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st) {
+// Gated or fused inputs: the forward's preparation kernel kept the prologue's
+// outputs (logf; for fused inputs the normalised q, k, v and the gated beta,
+// c) in the forward's workspace, and the backward reads them there.  a_log
+// stays set: the post-chain kernels write df~ and da_log parts in place of dlogf.
+BwdArgs plain_view(const BwdArgs& a) {
+  BwdArgs p = a;
+  const Layout& L = a.L;
+  if (a.a_log) p.logf = ws_ptr<const float>(a.fws, L.glogf);
+  if (a.pro.norm) {
+    p.q = ws_ptr<const __nv_bfloat16>(a.fws, L.fq);
+    p.k = ws_ptr<const __nv_bfloat16>(a.fws, L.fk);
+    p.v = ws_ptr<const __nv_bfloat16>(a.fws, L.fv);
+  }
+  if (a.pro.bscale > 0.f) {
+    p.beta = ws_ptr<const float>(a.fws, L.fbeta);
+    p.c = ws_ptr<const float>(a.fws, L.fc);
+  }
+  p.pro = Pro{};
+  return p;
+}
+
+cudaError_t launch_bwd_tc(const BwdArgs& in, int* err, int sms, cudaStream_t st) {
+  const BwdArgs a = plain_view(in);
   const Layout& L = a.L;
   cudaError_t e;
   if (a.phases & kPhaseLocal) {

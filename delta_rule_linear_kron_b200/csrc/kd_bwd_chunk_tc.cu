@@ -108,10 +108,10 @@ struct PreCfg {
 __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf,
-    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp, int H, int T, int NC,
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp, int H, int NC,
     const float* __restrict__ wP, const float* __restrict__ wu, float* __restrict__ wdu, float* __restrict__ wMu,
     __nv_bfloat16* __restrict__ wT1, __nv_bfloat16* __restrict__ wPU, __nv_bfloat16* __restrict__ wEK,
-    __nv_bfloat16* __restrict__ wQpT, const float* __restrict__ a_log, Pro pro, int* __restrict__ err) {
+    __nv_bfloat16* __restrict__ wQpT, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -128,13 +128,13 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    tc::mbar_expect_tx(&ld_bar, PreCfg::LOAD_BYTES - (a_log ? 16384u : 0u));
+    tc::mbar_expect_tx(&ld_bar, PreCfg::LOAD_BYTES);
     tc::tma_load_4d(sm + PreCfg::VD, &tm_v, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::VD + 16384, &tm_v, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::VD + 8192, &tm_do, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::VD + 24576, &tm_do, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
-    tc::tma_load_4d(sm + PreCfg::LG + (a_log ? 16384 : 0), &tm_logf, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + PreCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + PreCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
     tc::bulk_g2s(sm + PreCfg::PS, wP + ch * C * C, 16384u, &ld_bar);
     tc::bulk_g2s(sm + PreCfg::US, wu + ch * C, 256u, &ld_bar);
@@ -145,15 +145,6 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
-  if (pro.norm) {  // fused prologue: v, k, q arrive raw and are normalised in place
-    l2norm_tile(sm + PreCfg::VD, sm + PreCfg::VD + 16384, 128);
-    l2norm_tile(sm + PreCfg::KR, sm + PreCfg::KR + 128, 256);
-    l2norm_tile(sm + PreCfg::QR, sm + PreCfg::QR + 128, 256);
-    __syncthreads();
-  }
-  if (a_log)  // gated inputs: the bf16 forget pre-activations become logf in place
-    gate_logf_tile(reinterpret_cast<float*>(sm + PreCfg::LG), sm + PreCfg::LG + 16384, expf(a_log[h]),
-                   min(C, T - t0));
 
   // K+ and K- (fp32, read as tf32), and Q+ (bf16, transposed for the reverse
   // chain's dO^T Q+ MMA); thread (j, half) covers 32 positions.  K+ and Q+
@@ -324,8 +315,7 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
     const float* __restrict__ wMu, const __nv_bfloat16* __restrict__ wS0b, const __nv_bfloat16* __restrict__ wdSb,
     const __nv_bfloat16* __restrict__ wT1, const __nv_bfloat16* __restrict__ wPU,
     const __nv_bfloat16* __restrict__ wEK, float* __restrict__ dbeta, float* __restrict__ dc,
-    int* __restrict__ flags, const float* __restrict__ a_log, float* __restrict__ dapart, Pro pro,
-    int* __restrict__ err) {
+    int* __restrict__ flags, const float* __restrict__ a_log, float* __restrict__ dapart, int* __restrict__ err) {
   using Cf = PostCfg;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -352,8 +342,8 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    tc::mbar_expect_tx(&bar_a, Cf::LOAD_A - (a_log ? 16384u : 0u));
-    tc::tma_load_4d(sm + Cf::LG + (a_log ? 16384 : 0), &tm_logf, 0, h, t0, b, &bar_a);
+    tc::mbar_expect_tx(&bar_a, Cf::LOAD_A);
+    tc::tma_load_4d(sm + Cf::LG, &tm_logf, 0, h, t0, b, &bar_a);
     tc::tma_load_4d(sm + Cf::A4, &tm_q, 0, h, t0, b, &bar_a);
     tc::tma_load_4d(sm + Cf::A4 + 16384, &tm_q, 64, h, t0, b, &bar_a);
     tc::tma_load_4d(sm + Cf::A4 + 8192, &tm_k, 0, h, t0, b, &bar_a);
@@ -388,14 +378,9 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&bar_a, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  // gated inputs: logf (formed by the forward's preparation kernel) with the
+  // exponent a = e^{a_log}, for the epilogue's df~ and da_log
   const float ga = a_log ? expf(a_log[h]) : 0.f, inv_ga = a_log ? expf(-a_log[h]) : 0.f;
-  if (pro.norm) {  // fused prologue: q and k arrive raw and are normalised in place
-    l2norm_tile(sm + Cf::A4, sm + Cf::A4 + 16384, 128);
-    l2norm_tile(sm + Cf::A4 + 8192, sm + Cf::A4 + 24576, 128);
-    __syncthreads();
-  }
-  if (a_log)  // gated inputs: the bf16 forget pre-activations become logf in place
-    gate_logf_tile(reinterpret_cast<float*>(sm + Cf::LG), sm + Cf::LG + 16384, ga, nv);
 
   // decay prefix: thread (j, half) holds L for positions 32*half .. +31
   const int j = tid & 127, half = tid >> 7;
@@ -437,11 +422,6 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
     }
   }
   tc::mbar_wait<false>(&bar_b, 0, err, tc::kErrTimeoutLoad, &abort_flag);
-  if (pro.norm && !unsafe) {  // fused prologue: v arrives raw and is normalised in place
-    l2norm_tile(sm + Cf::DOV + 8192, sm + Cf::DOV + 24576, 128);
-    tc::fence_proxy_async();  // the MMAs read it
-    __syncthreads();
-  }
   if (!unsafe) {
     // dS' = dS diag(e^Lambda) in place, with the half sums of dS' o S0 over r
     const float eL = expf(lam[j]);
@@ -610,7 +590,7 @@ cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st) {
   if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_do, a.dO, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
-      !make_tmap_bthd(&tm_logf, a.logf, a.a_log ? 2 : 4, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
       !make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
       !make_tmap_bthd(&tm_kp, ws_ptr<float>(a.ws, L.Kp), 4, L.B, L.T, L.H, D, 32, true))
     return cudaErrorInvalidValue;
@@ -618,10 +598,10 @@ cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   prof_begin(st, "bwd_pre_tc");
   bwd_pre_tc<<<(unsigned)L.chunks, 256, PreCfg::BYTES, st>>>(
-      tm_v, tm_do, tm_k, tm_logf, tm_q, tm_kp, L.H, L.T, L.NC, ws_ptr<float>(a.fws, L.P),
+      tm_v, tm_do, tm_k, tm_logf, tm_q, tm_kp, L.H, L.NC, ws_ptr<float>(a.fws, L.P),
       ws_ptr<float>(a.fws, L.u), ws_ptr<float>(a.ws, L.du), ws_ptr<float>(a.ws, L.Mu),
       ws_ptr<__nv_bfloat16>(a.ws, L.T1), ws_ptr<__nv_bfloat16>(a.ws, L.PU), ws_ptr<__nv_bfloat16>(a.ws, L.EK),
-      ws_ptr<__nv_bfloat16>(a.ws, L.QpT), a.a_log, a.pro, err);
+      ws_ptr<__nv_bfloat16>(a.ws, L.QpT), err);
   prof_end(st);
   return cudaGetLastError();
 }
@@ -633,7 +613,7 @@ cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st) {
       !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_do, a.dO, 2, L.B, L.T, L.H, D, 64, true) ||
-      !make_tmap_bthd(&tm_logf, a.logf, a.a_log ? 2 : 4, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
       !make_tmap_bthd(&tm_dq, a.dq, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_dk, a.dk, 2, L.B, L.T, L.H, D, 64, true) ||
       !make_tmap_bthd(&tm_dv, a.dv, 2, L.B, L.T, L.H, D, 64, true) ||
@@ -644,12 +624,11 @@ cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   prof_begin(st, "bwd_post_tc");
   bwd_post_tc<<<(unsigned)L.chunks, 256, PostCfg::BYTES, st>>>(
-      tm_q, tm_k, tm_v, tm_do, tm_logf, tm_dq, tm_dk, tm_dv, tm_dlogf,
-      a.pro.bscale > 0.f ? ws_ptr<const float>(a.fws, L.fbeta) : a.beta, L.H, L.T, L.NC,
+      tm_q, tm_k, tm_v, tm_do, tm_logf, tm_dq, tm_dk, tm_dv, tm_dlogf, a.beta, L.H, L.T, L.NC,
       ws_ptr<float>(a.fws, L.u), ws_ptr<float>(a.fws, L.b0), ws_ptr<float>(a.ws, L.g), ws_ptr<float>(a.ws, L.Mu),
       ws_ptr<__nv_bfloat16>(a.fws, L.S0b), ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), ws_ptr<__nv_bfloat16>(a.ws, L.T1),
       ws_ptr<__nv_bfloat16>(a.ws, L.PU), ws_ptr<__nv_bfloat16>(a.ws, L.EK), a.dbeta, a.dc,
-      ws_ptr<int>(a.ws, L.bflags), a.a_log, ws_ptr<float>(a.ws, L.dapart), a.pro, err);
+      ws_ptr<int>(a.ws, L.bflags), a.a_log, ws_ptr<float>(a.ws, L.dapart), err);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -174,7 +174,7 @@ template <int DK, int DV, typename Tin>
 __device__ __forceinline__ void bwd_cc_body(
     int n, int h, int b, size_t slot,
     const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ beta,
-    const float* __restrict__ logf, const __nv_bfloat16* __restrict__ fpre, float ga, const Tin* __restrict__ dO,
+    const float* __restrict__ logf, const Tin* __restrict__ dO,
     int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wb0, const float* __restrict__ wg,
     float* __restrict__ dbeta, float* __restrict__ dc, float* __restrict__ wdP,
     float* __restrict__ wdGK, float* __restrict__ wdGVs) {
@@ -200,7 +200,7 @@ __device__ __forceinline__ void bwd_cc_body(
     const bool ok = t < nv;
     const size_t g = (((size_t)b * T + t0 + t) * H + h) * DK + j;
     Km[t * SK + j] = ok ? to_f(k[g]) : 0.f;
-    Ls[t * SK + j] = ok ? load_logf(logf, fpre, ga, g) : 0.f;
+    Ls[t * SK + j] = ok ? logf[g] : 0.f;
   }
   for (int e = tid; e < C * DV; e += blockDim.x) {
     const int t = e / DV, rr = e % DV;
@@ -308,8 +308,7 @@ template <int DK, int DV, typename Tin>
 __device__ __forceinline__ void bwd_state_body(
     int n, int h, int b, size_t slot,
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-    const float* __restrict__ beta, const float* __restrict__ logf, const __nv_bfloat16* __restrict__ fpre, float ga,
-    const Tin* __restrict__ dO, int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wg,
+    const float* __restrict__ beta, const float* __restrict__ logf, const Tin* __restrict__ dO, int H, int T, int NC, const float* __restrict__ wu, const float* __restrict__ wg,
     const float* __restrict__ wS0, const float* __restrict__ wdSC, float* __restrict__ waccq,
     float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv, int s0_swizzled,
     const __nv_bfloat16* __restrict__ wdSb) {
@@ -339,7 +338,7 @@ __device__ __forceinline__ void bwd_state_body(
     const bool ok = t < nv;
     const size_t g = (((size_t)b * T + t0 + t) * H + h) * DK + j;
     Kp[t * SK + j] = ok ? to_f(k[g]) : 0.f;
-    Ls[t * SK + j] = ok ? load_logf(logf, fpre, ga, g) : 0.f;
+    Ls[t * SK + j] = ok ? logf[g] : 0.f;
   }
   for (int e = tid; e < C * DV; e += blockDim.x) {
     const int t = e / DV, rr = e % DV;
@@ -458,7 +457,7 @@ template <int DK, int DV, typename Tin>
 __device__ __forceinline__ void bwd_intra_body(
     int n, int h, int b, size_t slot,
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-    const float* __restrict__ logf, const __nv_bfloat16* __restrict__ fpre, float ga, const Tin* __restrict__ dO,
+    const float* __restrict__ logf, float ga, const Tin* __restrict__ dO,
     int H, int T, int NC,
     const float* __restrict__ wP, const float* __restrict__ wu, const float* __restrict__ wdP,
     const float* __restrict__ wdGK, const float* __restrict__ wdGVs,
@@ -520,7 +519,7 @@ __device__ __forceinline__ void bwd_intra_body(
     const size_t g = (((size_t)b * T + t0 + t) * H + h) * DK + j;
     Km[t * SK + j] = ok ? to_f(k[g]) : 0.f;
     Qp[t * SK + j] = ok ? to_f(q[g]) : 0.f;
-    Ls[t * SK + j] = ok ? load_logf(logf, fpre, ga, g) : 0.f;
+    Ls[t * SK + j] = ok ? logf[g] : 0.f;
   }
   for (int e = tid; e < C * C; e += blockDim.x) {
     dPs[(e / C) * SC + e % C] = wdP[slot * C * C + e];
@@ -613,9 +612,9 @@ __device__ __forceinline__ void bwd_intra_body(
       acc += Ls[t * SK + tid];
       if (t < nv) {
         const size_t g = (((size_t)b * T + t0 + t) * H + h) * DK + tid;
-        if (fpre) {
+        if (ga > 0.f) {
           // gated inputs: df~ = dlogf a sigma(-f~); this chunk's part of da_log = sum dlogf logf
-          const float lf = load_logf(logf, fpre, ga, g);
+          const float lf = logf[g];
           dap = fmaf(acc, lf, dap);
           dlogf[g] = acc * dlogf_dfpre(lf, ga, 1.f / ga);
         } else {
@@ -623,9 +622,9 @@ __device__ __forceinline__ void bwd_intra_body(
         }
       }
     }
-    if (fpre) Ls[tid] = dap;  // the tile's row 0 is free again
+    if (ga > 0.f) Ls[tid] = dap;  // the tile's row 0 is free again
   }
-  if (fpre) {
+  if (ga > 0.f) {
     __syncthreads();
     if (tid == 0) {
       float s2 = 0.f;
@@ -644,8 +643,8 @@ __global__ void __launch_bounds__(256) bwd_cc_simt(
     float* __restrict__ dbeta, float* __restrict__ dc, float* __restrict__ wdP,
     float* __restrict__ wdGK, float* __restrict__ wdGVs) {
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  bwd_cc_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, k, v, beta, logf, nullptr, 0.f, dO, H, T, NC,
-                           wu, wb0, wg, dbeta, dc, wdP, wdGK, wdGVs);
+  bwd_cc_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, k, v, beta, logf, dO, H, T, NC, wu, wb0, wg,
+                           dbeta, dc, wdP, wdGK, wdGVs);
 }
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256) bwd_state_simt(
@@ -655,8 +654,8 @@ __global__ void __launch_bounds__(256) bwd_state_simt(
     const float* __restrict__ wS0, const float* __restrict__ wdSC, float* __restrict__ waccq,
     float* __restrict__ wacck, float* __restrict__ waccL, float* __restrict__ waccv) {
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  bwd_state_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, q, k, v, beta, logf, nullptr, 0.f, dO, H, T,
-                              NC, wu, wg, wS0, wdSC, waccq, wacck, waccL, waccv, 0, nullptr);
+  bwd_state_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, q, k, v, beta, logf, dO, H, T, NC, wu, wg,
+                              wS0, wdSC, waccq, wacck, waccL, waccv, 0, nullptr);
 }
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256) bwd_intra_simt(
@@ -668,8 +667,8 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
     const float* __restrict__ waccL, const float* __restrict__ waccv, Tin* __restrict__ dq,
     Tin* __restrict__ dk, Tin* __restrict__ dv, float* __restrict__ dlogf) {
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  bwd_intra_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, q, k, v, logf, nullptr, 0.f, dO, H, T, NC, wP,
-                              wu, wdP, wdGK, wdGVs, waccq, wacck, waccL, waccv, dq, dk, dv, dlogf, nullptr);
+  bwd_intra_body<DK, DV, Tin>(n, h, b, ((size_t)b * H + h) * NC + n, q, k, v, logf, 0.f, dO, H, T, NC, wP, wu,
+                              wdP, wdGK, wdGVs, waccq, wacck, waccL, waccv, dq, dk, dv, dlogf, nullptr);
 }
 
 // The tensor-core path's exact recomputation of the chunks the per-chunk
@@ -680,8 +679,8 @@ __global__ void __launch_bounds__(256) bwd_intra_simt(
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256) bwd_exact_simt(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-    const float* __restrict__ beta, const float* __restrict__ logf, const __nv_bfloat16* __restrict__ fpre,
-    const float* __restrict__ a_log, const Tin* __restrict__ dO, int H, int T,
+    const float* __restrict__ beta, const float* __restrict__ logf, const float* __restrict__ a_log,
+    const Tin* __restrict__ dO, int H, int T,
     int NC, size_t chunks, const float* __restrict__ wP, const float* __restrict__ wu,
     const float* __restrict__ wb0, const float* __restrict__ wg, const float* __restrict__ wS0,
     const __nv_bfloat16* __restrict__ wdSb, float* __restrict__ dbeta, float* __restrict__ dc,
@@ -694,14 +693,14 @@ __global__ void __launch_bounds__(256) bwd_exact_simt(
     if (only[ch] == 0) continue;  // uniform across the CTA
     const int n = static_cast<int>(ch % NC), u = static_cast<int>(ch / NC);
     const int h = u % H, b = u / H;
-    const float ga = fpre ? expf(a_log[h]) : 0.f;
-    bwd_cc_body<DK, DV, Tin>(n, h, b, slot, k, v, beta, logf, fpre, ga, dO, H, T, NC, wu, wb0, wg, dbeta, dc, wdP,
-                             wdGK, wdGVs);
+    const float ga = a_log ? expf(a_log[h]) : 0.f;  // gated inputs: df~ and da_log parts in place of dlogf
+    bwd_cc_body<DK, DV, Tin>(n, h, b, slot, k, v, beta, logf, dO, H, T, NC, wu, wb0, wg, dbeta, dc, wdP, wdGK,
+                             wdGVs);
     __syncthreads();
-    bwd_state_body<DK, DV, Tin>(n, h, b, slot, q, k, v, beta, logf, fpre, ga, dO, H, T, NC, wu, wg, wS0, nullptr,
+    bwd_state_body<DK, DV, Tin>(n, h, b, slot, q, k, v, beta, logf, dO, H, T, NC, wu, wg, wS0, nullptr,
                                 waccq, wacck, waccL, waccv, 1, wdSb);
     __syncthreads();
-    bwd_intra_body<DK, DV, Tin>(n, h, b, slot, q, k, v, logf, fpre, ga, dO, H, T, NC, wP, wu, wdP, wdGK, wdGVs,
+    bwd_intra_body<DK, DV, Tin>(n, h, b, slot, q, k, v, logf, ga, dO, H, T, NC, wP, wu, wdP, wdGK, wdGVs,
                                 waccq, wacck, waccL, waccv, dq, dk, dv, dlogf, dapart);
     __syncthreads();
   }
@@ -753,16 +752,10 @@ static cudaError_t run_bwd(const BwdArgs& a, int stages, const int* only, cudaSt
   if (only) {
     // tensor-core path: the flagged chunks only, all stages in one kernel
     if (stages != (kStageCC | kStageState | kStageIntra)) return cudaErrorInvalidValue;
-    // fused prologue: the flagged chunks' normalised q, k, v rows and the
-    // gated beta, from the forward's preparation kernel
-    const bool nrm = a.pro.norm != 0;
-    const float* beta = a.pro.bscale > 0.f ? ws_ptr<float>(a.fws, L.fbeta) : a.beta;
     prof_begin(st, "bwd_exact_simt");
     bwd_exact_simt<DK, DV, Tin><<<(unsigned)(L.chunks < (size_t)kExactSlots ? L.chunks : kExactSlots), 256, s5,
                                   st>>>(
-        nrm ? ws_ptr<Tin>(a.fws, L.fq) : q, nrm ? ws_ptr<Tin>(a.fws, L.fk) : k,
-        nrm ? ws_ptr<Tin>(a.fws, L.fv) : v, beta, a.a_log ? nullptr : a.logf,
-        a.a_log ? reinterpret_cast<const __nv_bfloat16*>(a.logf) : nullptr, a.a_log, dO, L.H, L.T, L.NC, L.chunks,
+        q, k, v, a.beta, a.logf, a.a_log, dO, L.H, L.T, L.NC, L.chunks,
         wP, wu, wb0, wg, wS0, ws_ptr<__nv_bfloat16>(a.ws, L.dSCb), a.dbeta, a.dc, wdP, wdGK, wdGVs, waccq, wacck,
         waccL, waccv, static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), a.dlogf,
         ws_ptr<float>(a.ws, L.dapart), only);

@@ -138,13 +138,6 @@ __device__ __forceinline__ void l2norm_tile(unsigned char* seg0, unsigned char* 
   }
 }
 
-// One log-decay value from global memory: logf itself, or formed from the
-// forget pre-activation (gated inputs, fpre != nullptr).
-template <typename Tf>
-__device__ __forceinline__ float load_logf(const float* __restrict__ logf, const Tf* __restrict__ fpre, float a,
-                                           size_t g) {
-  return fpre ? a * log_sigmoid(to_f(fpre[g])) : logf[g];
-}
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll

@@ -572,9 +572,7 @@ cudaError_t launch_chain_r(const FwdArgs& a, int* err, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(st, "fwd_chain_tc");
-  // fused prologue: beta as gated by the preparation kernel
-  const float* beta = a.pro.bscale > 0.f ? (const float*)ws_ptr<float>(a.ws, L.fbeta) : a.beta;
-  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_kt, tm_ke, beta, a.S0, a.ST, L.H, L.T, L.NC,
+  e = cudaLaunchKernelEx(&cfg, fwd_chain_tc<R>, tm_kt, tm_ke, a.beta, a.S0, a.ST, L.H, L.T, L.NC,
                          (const float*)ws_ptr<float>(a.ws, L.y), (const float*)ws_ptr<float>(a.ws, L.A),
                          (const float*)ws_ptr<float>(a.ws, L.Hx), (const float*)ws_ptr<float>(a.ws, L.GC),
                          (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.Vt),

@@ -56,9 +56,8 @@ struct OutCfg {
 __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_logf,
-    const __grid_constant__ CUtensorMap tm_out, int H, int T, int NC, const __nv_bfloat16* __restrict__ wS0b,
-    const float* __restrict__ wu, int* __restrict__ unsafe_flags, const float* __restrict__ a_log, Pro pro,
-    int* __restrict__ err) {
+    const __grid_constant__ CUtensorMap tm_out, int H, int NC, const __nv_bfloat16* __restrict__ wS0b,
+    const float* __restrict__ wu, int* __restrict__ unsafe_flags, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -75,7 +74,7 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    tc::mbar_expect_tx(&ld_bar, OutCfg::LOAD_BYTES - (a_log ? 16384u : 0u));
+    tc::mbar_expect_tx(&ld_bar, OutCfg::LOAD_BYTES);
 #pragma unroll
     for (int part = 0; part < 2; ++part)
       tc::bulk_g2s(sm + OutCfg::S0B + part * 16384, wS0b + ch * D * D + part * 8192, 16384u, &ld_bar);
@@ -83,7 +82,7 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     tc::tma_load_4d(sm + OutCfg::VB + 8192, &tm_v, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
-    tc::tma_load_4d(sm + OutCfg::LG + (a_log ? 16384 : 0), &tm_logf, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + OutCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
     tc::bulk_g2s(sm + OutCfg::U, wu + ch * C, 256u, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
@@ -92,15 +91,6 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
-  if (pro.norm) {  // fused prologue: q, k, v arrive raw and are normalised in place
-    l2norm_tile(sm + OutCfg::QR, sm + OutCfg::QR + 128, 256);
-    l2norm_tile(sm + OutCfg::KR, sm + OutCfg::KR + 128, 256);
-    l2norm_tile(sm + OutCfg::VB, sm + OutCfg::VB + 8192, 128);
-    __syncthreads();
-  }
-  if (a_log)  // gated inputs: the bf16 forget pre-activations become logf in place
-    gate_logf_tile(reinterpret_cast<float*>(sm + OutCfg::LG), sm + OutCfg::LG + 16384, expf(a_log[h]),
-                   min(C, T - t0));
 
   // Q+ = q o gamma, K- = k / gamma (tf32); thread (j, half) covers 32 positions
   const int j = tid & 127, half = tid >> 7;
@@ -235,8 +225,7 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
 // factorised form's fp32 range (flagged by fwd_out_tc): per-element decays.
 __global__ void __launch_bounds__(128) fwd_out_fixup(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const float* __restrict__ logf, const __nv_bfloat16* __restrict__ fpre,
-    const float* __restrict__ a_log, int H, int T, int NC,
+    const __nv_bfloat16* __restrict__ v, const float* __restrict__ logf, int H, int T, int NC,
     const float* __restrict__ wS0blob, const float* __restrict__ wu, const int* __restrict__ unsafe_flags,
     __nv_bfloat16* __restrict__ out) {
   const size_t ch = blockIdx.x;
@@ -250,12 +239,11 @@ __global__ void __launch_bounds__(128) fwd_out_fixup(
   const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
   const int b = unit / H, h = unit % H;
   const int t0 = n * C, nv = min(C, T - t0);
-  const float ga = a_log ? expf(a_log[h]) : 0.f;
   for (int e = tid; e < C * D; e += 128) {
     const int t = e / D, j = e % D;
     const bool ok = t < nv;
     const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + j;
-    Ls[t][j] = ok ? load_logf(logf, fpre, ga, g) : 0.f;
+    Ls[t][j] = ok ? logf[g] : 0.f;
     qs[t][j] = ok ? __bfloat162float(q[g]) : 0.f;
     ks[t][j] = ok ? __bfloat162float(k[g]) : 0.f;
   }
@@ -315,8 +303,9 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_logf,
     const float* __restrict__ beta, const float* __restrict__ c, int H, int T, int NC, float* __restrict__ wy,
     float* __restrict__ wA, float* __restrict__ wP, int* __restrict__ wxflags, const float* __restrict__ a_log,
-    Pro pro, float* __restrict__ fbeta, float* __restrict__ fc, __nv_bfloat16* __restrict__ fq,
-    __nv_bfloat16* __restrict__ fk, __nv_bfloat16* __restrict__ fv, int* __restrict__ err) {
+    Pro pro, float* __restrict__ glogf, float* __restrict__ fbeta, float* __restrict__ fc,
+    __nv_bfloat16* __restrict__ fq, __nv_bfloat16* __restrict__ fk, __nv_bfloat16* __restrict__ fv,
+    int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -369,8 +358,16 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     l2norm_tile(sm + PrepCfg::VT, sm + PrepCfg::VT + 8192, 128);
     __syncthreads();
   }
-  if (a_log)  // gated inputs: the bf16 forget pre-activations become logf in place
+  if (a_log) {
+    // gated inputs: the bf16 forget pre-activations become logf in place, and
+    // logf goes to the workspace, where every later kernel reads it
     gate_logf_tile(Ls, sm + PrepCfg::LS + 16384, expf(a_log[h]), nv);
+    for (int e = tid; e < nv * (D / 4); e += 256) {
+      const int t = e / (D / 4), c4 = e % (D / 4);
+      *reinterpret_cast<float4*>(glogf + (((size_t)b * T + t0 + t) * H + h) * D + 4 * c4) =
+          *reinterpret_cast<const float4*>(Ls + t * D + 4 * c4);
+    }
+  }
   // decay prefix (thread (j, half) covers 32 positions; L is written back for
   // the exact path) and the tf32 operands K+, Q+, K-
   float mx = 0.f;
@@ -403,9 +400,9 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
   const bool is_unsafe = __syncthreads_or(!(mx < kSafeLogRange)) != 0;
   const bool exact_state = __syncthreads_or(!(mx < kExactStateRange)) != 0;
   if (tid == 0) wxflags[ch] = exact_state ? 1 : 0;
-  if (pro.norm && exact_state) {
-    // fused prologue: the exact paths (CUDA cores, global loads) read this
-    // chunk's normalised q, k, v rows from the workspace
+  if (pro.norm) {
+    // fused prologue: the normalised q, k, v rows go to the workspace, where
+    // every later kernel reads them
     for (int e = tid; e < nv * (D / 8); e += 256) {
       const int t = e / (D / 8), c8 = e % (D / 8);
       const size_t g = (((size_t)b * T + t0 + t) * H + h) * D + 8 * c8;
@@ -578,9 +575,8 @@ struct CrossCfg {
 __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_logf, const __grid_constant__ CUtensorMap tm_kt,
-    const __grid_constant__ CUtensorMap tm_ke, int H, int T, int NC, float* __restrict__ wGC,
-    float* __restrict__ wHx, __nv_bfloat16* __restrict__ wVt, const float* __restrict__ a_log, Pro pro,
-    int* __restrict__ err) {
+    const __grid_constant__ CUtensorMap tm_ke, int H, int NC, float* __restrict__ wGC, float* __restrict__ wHx,
+    __nv_bfloat16* __restrict__ wVt, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -598,17 +594,16 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    const uint32_t lg_less = a_log ? 16384u : 0u;  // gated inputs: a bf16 tile in place of fp32 logf
-    tc::mbar_expect_tx(&ld_bar, CrossCfg::LOAD_CUR - lg_less + (has_prev ? CrossCfg::LOAD_PREV - lg_less : 0u));
+    tc::mbar_expect_tx(&ld_bar, CrossCfg::LOAD_CUR + (has_prev ? CrossCfg::LOAD_PREV : 0u));
     tc::tma_load_4d(sm + CrossCfg::VV, &tm_v, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + CrossCfg::VV + 16384, &tm_v, 64, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + CrossCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
-    tc::tma_load_4d(sm + CrossCfg::LG + lg_less, &tm_logf, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + CrossCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
     if (has_prev) {
       tc::tma_load_4d(sm + CrossCfg::VV + 8192, &tm_v, 0, h, tp, b, &ld_bar);
       tc::tma_load_4d(sm + CrossCfg::VV + 24576, &tm_v, 64, h, tp, b, &ld_bar);
       tc::tma_load_4d(sm + CrossCfg::KR + 16384, &tm_k, 0, h, tp, b, &ld_bar);
-      tc::tma_load_4d(sm + CrossCfg::LG + 32768 + lg_less, &tm_logf, 0, h, tp, b, &ld_bar);
+      tc::tma_load_4d(sm + CrossCfg::LG + 32768, &tm_logf, 0, h, tp, b, &ld_bar);
     }
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
@@ -617,21 +612,6 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
-  if (pro.norm) {  // fused prologue: v and k of both chunks arrive raw and are normalised in place
-    l2norm_tile(sm + CrossCfg::VV, sm + CrossCfg::VV + 16384, 128);
-    l2norm_tile(sm + CrossCfg::KR, sm + CrossCfg::KR + 128, 256);
-    if (has_prev) {
-      l2norm_tile(sm + CrossCfg::VV + 8192, sm + CrossCfg::VV + 24576, 128);
-      l2norm_tile(sm + CrossCfg::KR + 16384, sm + CrossCfg::KR + 16384 + 128, 256);
-    }
-    __syncthreads();
-  }
-  if (a_log) {  // gated inputs: the bf16 forget pre-activations become logf in place
-    const float ga = expf(a_log[h]);
-    gate_logf_tile(reinterpret_cast<float*>(sm + CrossCfg::LG), sm + CrossCfg::LG + 16384, ga, min(C, T - t0));
-    if (has_prev)
-      gate_logf_tile(reinterpret_cast<float*>(sm + CrossCfg::LG + 32768), sm + CrossCfg::LG + 49152, ga, C);
-  }
   // half 0: chunk n (channel j); half 1: chunk n-1 (channel j)
   const int j = tid & 127, half = tid >> 7;
   float* lg = reinterpret_cast<float*>(sm + CrossCfg::LG + half * 32768);
@@ -747,27 +727,56 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
 
 }  // namespace
 
-cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) {
+// Gated or fused inputs: fwd_prep_tc forms the prologue's outputs once (logf;
+// for fused inputs also the normalised q, k, v and the gated beta, c) and
+// keeps them in the workspace; every later kernel, here and in the backward,
+// reads them there as plain inputs.
+FwdArgs plain_view(const FwdArgs& a) {
+  FwdArgs p = a;
   const Layout& L = a.L;
+  if (a.a_log) p.logf = ws_ptr<float>(a.ws, L.glogf);
+  if (a.pro.norm) {
+    p.q = ws_ptr<__nv_bfloat16>(a.ws, L.fq);
+    p.k = ws_ptr<__nv_bfloat16>(a.ws, L.fk);
+    p.v = ws_ptr<__nv_bfloat16>(a.ws, L.fv);
+  }
+  if (a.pro.bscale > 0.f) {
+    p.beta = ws_ptr<float>(a.ws, L.fbeta);
+    p.c = ws_ptr<float>(a.ws, L.fc);
+  }
+  p.a_log = nullptr;
+  p.pro = Pro{};
+  return p;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs& in, int* err, int sms, cudaStream_t st) {
+  const Layout& L = in.L;
+  const FwdArgs a = plain_view(in);
   cudaError_t e;
   if (a.phases & kPhaseLocal) {
-    CUtensorMap tm_v, tm_q, tm_k, tm_logf;  // gated inputs: tm_logf covers the bf16 pre-activations
-    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
-        !make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
-        !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
-        !make_tmap_bthd(&tm_logf, a.logf, a.a_log ? 2 : 4, L.B, L.T, L.H, D, 128, false))
+    CUtensorMap tm_v, tm_q, tm_k, tm_logf;  // the caller's inputs (gated: tm_logf covers bf16 pre-activations)
+    if (!make_tmap_bthd(&tm_v, in.v, 2, L.B, L.T, L.H, D, 64, true) ||
+        !make_tmap_bthd(&tm_q, in.q, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_k, in.k, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_logf, in.logf, in.a_log ? 2 : 4, L.B, L.T, L.H, D, 128, false))
       return cudaErrorInvalidValue;
     if ((e = cudaFuncSetAttribute(fwd_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)PrepCfg::BYTES)) != cudaSuccess)
       return e;
     prof_begin(st, "fwd_prep_tc");
     fwd_prep_tc<<<(unsigned)L.chunks, 256, PrepCfg::BYTES, st>>>(
-        tm_v, tm_q, tm_k, tm_logf, a.beta, a.c, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y), ws_ptr<float>(a.ws, L.A),
-        a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, ws_ptr<int>(a.ws, L.xflags), a.a_log, a.pro,
-        ws_ptr<float>(a.ws, L.fbeta), ws_ptr<float>(a.ws, L.fc), ws_ptr<__nv_bfloat16>(a.ws, L.fq),
-        ws_ptr<__nv_bfloat16>(a.ws, L.fk), ws_ptr<__nv_bfloat16>(a.ws, L.fv), err);
+        tm_v, tm_q, tm_k, tm_logf, in.beta, in.c, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.y),
+        ws_ptr<float>(a.ws, L.A), a.save ? ws_ptr<float>(a.ws, L.P) : nullptr, ws_ptr<int>(a.ws, L.xflags), in.a_log,
+        in.pro, ws_ptr<float>(a.ws, L.glogf), ws_ptr<float>(a.ws, L.fbeta), ws_ptr<float>(a.ws, L.fc),
+        ws_ptr<__nv_bfloat16>(a.ws, L.fq), ws_ptr<__nv_bfloat16>(a.ws, L.fk), ws_ptr<__nv_bfloat16>(a.ws, L.fv),
+        err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // from here on, the prologue's outputs
+    if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
+        !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false))
+      return cudaErrorInvalidValue;
     CUtensorMap tm_kt, tm_ke;
     if (!make_tmap_bthd(&tm_kt, ws_ptr<float>(a.ws, L.Kt), 4, L.B, L.T, L.H, D, 128, false) ||
         !make_tmap_bthd(&tm_ke, ws_ptr<float>(a.ws, L.Ke), 4, L.B, L.T, L.H, D, 128, false))
@@ -777,8 +786,8 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
       return e;
     prof_begin(st, "fwd_cross_tc");
     fwd_cross_tc<<<(unsigned)L.chunks, 256, CrossCfg::BYTES, st>>>(
-        tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.T, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx),
-        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), a.a_log, a.pro, err);
+        tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx),
+        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -796,28 +805,25 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* err, int sms, cudaStream_t st) 
     if (!make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
         !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
         !make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
-        !make_tmap_bthd(&tm_logf, a.logf, a.a_log ? 2 : 4, L.B, L.T, L.H, D, 128, false) ||
+        !make_tmap_bthd(&tm_logf, a.logf, 4, L.B, L.T, L.H, D, 128, false) ||
         !make_tmap_bthd(&tm_out, a.out, 2, L.B, L.T, L.H, D, 64, true))
       return cudaErrorInvalidValue;
     prof_begin(st, "fwd_out_tc");
     fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(
-        tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.T, L.NC, (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.S0b),
-        wu, flags, a.a_log, a.pro, err);
+        tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.S0b), wu,
+        flags, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  // unsafe chunks only: exact per-element recomputation of O
   constexpr int kFixSmem = (3 * C * (D + 1) + C) * 4;
   if ((e = cudaFuncSetAttribute(fwd_out_fixup, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem)) !=
       cudaSuccess)
     return e;
   prof_begin(st, "fwd_out_fixup");
-  // fused prologue: the flagged chunks' normalised q, k, v rows, from the preparation kernel
-  const bool nrm = a.pro.norm != 0;
   fwd_out_fixup<<<(unsigned)L.chunks, 128, kFixSmem, st>>>(
-      nrm ? ws_ptr<__nv_bfloat16>(a.ws, L.fq) : static_cast<const __nv_bfloat16*>(a.q),
-      nrm ? ws_ptr<__nv_bfloat16>(a.ws, L.fk) : static_cast<const __nv_bfloat16*>(a.k),
-      nrm ? ws_ptr<__nv_bfloat16>(a.ws, L.fv) : static_cast<const __nv_bfloat16*>(a.v), a.a_log ? nullptr : a.logf,
-      a.a_log ? reinterpret_cast<const __nv_bfloat16*>(a.logf) : nullptr, a.a_log, L.H, L.T, L.NC, blob, wu, flags,
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), a.logf, L.H, L.T, L.NC, blob, wu, flags,
       static_cast<__nv_bfloat16*>(a.out));
   prof_end(st);
   return cudaGetLastError();

@@ -71,18 +71,19 @@ struct Layout {
   size_t Kp = 0, QpT = 0;
   size_t dapart = 0;  // gated inputs: each chunk's part of da_log [ch]
   size_t bwd_bytes = 0;
-  // Gated inputs (forget pre-activations in place of logf).  The CUDA-core
-  // path converts them to logf in the forward's workspace (glogf, [B][T][H][dk]
-  // fp32, after the saved region) and takes dlogf in the backward's (gdlogf);
-  // the tensor-core kernels read the pre-activations directly.
+  // Gated inputs (forget pre-activations in place of logf): logf is formed
+  // once into the forward's workspace (glogf, [B][T][H][dk] fp32, after the
+  // saved region; on the tensor-core path by the preparation kernel), and
+  // every later kernel reads it there.  The CUDA-core path takes dlogf in the
+  // backward's workspace (gdlogf) before forming df~.
   size_t glogf = 0, gdlogf = 0;
   size_t fwd_gated_bytes = 0, bwd_gated_bytes = 0;
   // Fused prologue (raw q, k, v and gate pre-activations).  Forward: the
-  // gated beta and c [B][T][H] (fp32) of every token, and normalised q, k, v
-  // [B][T][H][d] (activation dtype): on the tensor-core path only the rows of
-  // chunks with xflags set (the exact paths read them), on the CUDA-core path
-  // all of them.  Backward, CUDA-core path: the recurrence's gradients and the
-  // prologue backward's scratch.
+  // gated beta and c [B][T][H] (fp32) and the normalised q, k, v [B][T][H][d]
+  // (activation dtype) of every token, written by the preparation kernel on
+  // the tensor-core path and by the prologue pass on the CUDA-core path, and
+  // read by every later kernel.  Backward, CUDA-core path: the recurrence's
+  // gradients and the prologue backward's scratch.
   size_t fbeta = 0, fc = 0, fq = 0, fk = 0, fv = 0;
   size_t gdq = 0, gdk = 0, gdv = 0, gdbeta = 0, gdc = 0, gdf = 0, gpro = 0;
   size_t fwd_fused_bytes = 0, bwd_fused_bytes = 0;
