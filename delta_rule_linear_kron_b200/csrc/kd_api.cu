@@ -847,6 +847,11 @@ int kron_delta_gdn2_fwd(const void* q, const void* k, const void* v, const float
   a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.loga = loga; a.S0 = S0; a.out = out; a.ST = ST;
   a.ws = static_cast<char*>(workspace);
   a.L = L;
+  if (kd::gdn2_tc_supported(L)) {  // the tensor-core kernels report bounded-wait timeouts here
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    a.err = di.err;
+  }
   return launched(kd::launch_gdn2_fwd(a, static_cast<cudaStream_t>(stream)), "gdn2 forward launch");
 }
 

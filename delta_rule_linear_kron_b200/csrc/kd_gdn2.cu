@@ -1067,18 +1067,28 @@ cudaError_t gdn2_fwd_t(const GdnArgs& a, cudaStream_t st) {
   const GdnLayout& L = a.L;
   const GdnWs p = gdn_ws(a.ws, L);
   const dim3 gc(L.NC, L.H, L.B), gr(DV / kRows, L.H, L.B);
-  KD_TRYC(set_smem(gdn2_prep<DK, DV, Tin>, S::prep));
   KD_TRYC(set_smem(gdn2_chain<DK, DV>, S::chain));
-  KD_TRYC(set_smem(gdn2_out<DK, DV, Tin>, S::out));
-  prof_begin(st, "gdn2_prep");
-  gdn2_prep<DK, DV, Tin><<<gc, 256, S::prep, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
-                                                   static_cast<const Tin*>(a.v), a.b, a.w, a.loga, L.H, L.T, L.NC, p);
-  prof_end(st);
-  KD_TRYC(cudaGetLastError());
-  prof_begin(st, "gdn2_chain");
-  gdn2_chain<DK, DV><<<gr, kChainThreads, S::chain, st>>>(a.S0, a.ST, L.H, L.NC, p);
-  prof_end(st);
-  KD_TRYC(cudaGetLastError());
+  if (!gdn2_tc_supported(L)) KD_TRYC(set_smem(gdn2_out<DK, DV, Tin>, S::out));
+  if (gdn2_tc_supported(L)) {
+    KD_TRYC(launch_gdn2_prep_tc(a, a.err, st));
+  } else {
+    KD_TRYC(set_smem(gdn2_prep<DK, DV, Tin>, S::prep));
+    prof_begin(st, "gdn2_prep");
+    gdn2_prep<DK, DV, Tin><<<gc, 256, S::prep, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
+                                                     static_cast<const Tin*>(a.v), a.b, a.w, a.loga, L.H, L.T, L.NC,
+                                                     p);
+    prof_end(st);
+    KD_TRYC(cudaGetLastError());
+  }
+  if (gdn2_tc_supported(L)) {
+    KD_TRYC(launch_gdn2_chain_tc(a, a.err, st));
+  } else {
+    prof_begin(st, "gdn2_chain");
+    gdn2_chain<DK, DV><<<gr, kChainThreads, S::chain, st>>>(a.S0, a.ST, L.H, L.NC, p);
+    prof_end(st);
+    KD_TRYC(cudaGetLastError());
+  }
+  if (gdn2_tc_supported(L)) return launch_gdn2_out_tc(a, a.err, st);
   prof_begin(st, "gdn2_out");
   gdn2_out<DK, DV, Tin><<<gc, 256, S::out, st>>>(L.H, L.T, L.NC, p, static_cast<Tin*>(a.out));
   prof_end(st);

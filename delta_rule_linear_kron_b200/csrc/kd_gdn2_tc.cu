@@ -1,0 +1,752 @@
+// kd_gdn2_tc.cu -- Gated DeltaNet-2's per-chunk preparation on tensor cores
+// (bf16 q, k, v and d_k = d_v = 128).
+//
+// Gated DeltaNet-2 article (aitrends.kr), sections "방법론" and "기술 상세": the
+// chunkwise WY form with the channel decay absorbed into the erase side.  In
+// the library's state convention (S in R^{dv x dk}, decay from the right), per
+// chunk of C = 64 positions with in-chunk cumulative log-decay L (per key
+// channel), gamma = e^L and Lambda = L at the chunk end:
+//   E+ = b o k o gamma,  K- = k / gamma,  Q+ = q o gamma,  Z = w o v
+//   T = tril(E+ K-^T, -1),  P = tril(Q+ K-^T),  A = (I + T)^{-1}
+//   W = A E+,  U' = A Z,  K^e = k o e^{Lambda - L},  gamma_C = e^Lambda
+// One CTA per chunk, all chunks in parallel:
+//   1. [E+; Q+] K-^T on tcgen05 (M = 128: rows 0-63 give T, rows 64-127 P),
+//      with bf16 high and low parts of both operands as in step 3.
+//   2. A by a blocked inverse on CUDA cores (16 x 16 diagonal blocks by
+//      substitution, then block rows), in fp32.
+//   3. W^T = E+^T A^T and U'^T = Z^T A^T on tcgen05 (bf16 high and low parts of
+//      both operands: hi hi + hi lo + lo hi, so the products keep about 16
+//      significant bits of each factor), M = 128 channels, N = 64 positions.
+// Chunks whose in-chunk |L| reaches 60 (where k / gamma could overflow) take T
+// and P with per-element weights e^{L_t - L_i} <= 1 on CUDA cores instead of
+// step 1.  The outputs are those of the CUDA-core kernel (kd_gdn2.cu), in the
+// same layouts, so the chain, output and backward kernels read them unchanged.
+#include "kd_common.cuh"
+#include "kd_kernels.h"
+#include "kd_tc.cuh"
+#include "kd_tmap.h"
+
+namespace kd {
+namespace {
+
+constexpr int C = kChunk;
+constexpr int D = 128;
+// in-chunk |L| below which the weights factor (e^{+-60} stays well inside fp32)
+constexpr float kGdnTcSafeLog = 60.f;
+// chunks ahead of the chain's slots whose operands its producer pulls into L2
+constexpr int kChainAhead = 3;
+
+struct GPrepCfg {
+  static constexpr uint32_t AKQ = 0;        // [E+; Q+] bf16 hi, lo (2 K blocks x 128 rows each, 32 KB); then
+                                            // the bf16 operands E+^T hi, lo and Z^T hi, lo (16 KB each)
+  static constexpr uint32_t BKM = 65536;    // K- bf16 hi, lo (2 K blocks x 64 rows each, 16 KB); then A hi, lo
+  static constexpr uint32_t QR = 98304;     // q bf16 [64][128] (TMA)
+  static constexpr uint32_t KR = 114688;    // k bf16 [64][128] (TMA)
+  static constexpr uint32_t VR = 131072;    // v bf16 [64][128] (TMA)
+  static constexpr uint32_t LS = 147456;    // loga fp32 [64][128] (TMA), then L in place
+  static constexpr uint32_t TS = 180224;    // T fp32 [64][65]
+  static constexpr uint32_t XS = TS + 64 * 65 * 4;        // A fp32 [64][65]
+  static constexpr uint32_t TB = XS + 64 * 65 * 4;        // block temporaries [3][16][17]
+  static constexpr uint32_t SMALL = TB + 3 * 16 * 17 * 4;  // prefix exchange [128], Lambda [128]
+  static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
+  static constexpr uint32_t LOAD_BYTES = 3 * 16384 + 32768;
+  // the bf16 operands of step 3
+  static constexpr uint32_t EH = 0, EL = 16384, ZH = 32768, ZL = 49152, AH = 65536, AL = 73728;
+};
+
+__device__ __forceinline__ void put_hl(unsigned char* hi, unsigned char* lo, uint32_t off, float x) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  *reinterpret_cast<__nv_bfloat16*>(hi + off) = h;
+  *reinterpret_cast<__nv_bfloat16*>(lo + off) = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
+__global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_loga,
+    const float* __restrict__ bg, const float* __restrict__ wg, int H, int T, int NC, GdnWs p,
+    int* __restrict__ err) {
+  using Cf = GPrepCfg;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar, mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = blockIdx.x;
+  float* Ls = reinterpret_cast<float*>(sm + Cf::LS);
+  float* Ts = reinterpret_cast<float*>(sm + Cf::TS);
+  float* Xs = reinterpret_cast<float*>(sm + Cf::XS);
+  float* Tb = reinterpret_cast<float*>(sm + Cf::TB);
+  float* xch = reinterpret_cast<float*>(sm + Cf::SMALL);
+  float* lam = xch + 128;
+  const auto row = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * D; };
+
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+    tc::mbar_expect_tx(&ld_bar, Cf::LOAD_BYTES);
+    tc::tma_load_4d(sm + Cf::QR, &tm_q, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + Cf::KR, &tm_k, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + Cf::VR, &tm_v, 0, h, t0, b, &ld_bar);
+    tc::tma_load_4d(sm + Cf::LS, &tm_loga, 0, h, t0, b, &ld_bar);
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+
+  // decay prefix of key channel j, split over two threads (half 0: positions
+  // 0-31, half 1: 32-63), then the operands of step 1 and the per-token outputs
+  const int j = tid & 127, half = tid >> 7;
+  float mx = 0.f;
+  {
+    float Lr[32];
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      acc += Ls[(32 * half + i) * D + j];
+      Lr[i] = acc;
+    }
+    if (half == 0) xch[j] = acc;
+    __syncthreads();
+    const float off = half ? xch[j] : 0.f;
+    if (half) lam[j] = acc + off;  // padded positions carry loga = 0: L at 63 is Lambda
+    __syncthreads();
+    const float lj = lam[j];
+    if (half == 0) p.gC[ch * D + j] = expf(lj);
+    float bv[32];  // the erase gates of this thread's positions, all loads in flight together
+#pragma unroll
+    for (int i = 0; i < 32; ++i) bv[i] = 32 * half + i < nv ? bg[row(32 * half + i) + j] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = 32 * half + i;
+      const float L = Lr[i] + off;
+      mx = fmaxf(mx, fabsf(L));
+      Ls[t * D + j] = L;
+      const float qq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::QR + (t * D + j) * 2));
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::KR + (t * D + j) * 2));
+      const float bb = bv[i];
+      const float gm = expf(L), ig = expf(-L);
+      const float qp = qq * gm;
+      put_hl(sm + Cf::AKQ, sm + Cf::AKQ + 32768, tc::sw128_off(t, j, 128, 2), bb * kk * gm);
+      put_hl(sm + Cf::AKQ, sm + Cf::AKQ + 32768, tc::sw128_off(64 + t, j, 128, 2), qp);
+      put_hl(sm + Cf::BKM, sm + Cf::BKM + 16384, tc::sw128_off(t, j, 64, 2), kk * ig);
+      p.Qp[(ch * C + t) * D + j] = qp;
+      p.Ke[(ch * C + t) * D + j] = kk * expf(lj - L);
+    }
+  }
+  const bool is_unsafe = __syncthreads_or(!(mx < kGdnTcSafeLog)) != 0;
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0 && !is_unsafe) {
+    const uint32_t IDB = tc::idesc(128, 64, 1);
+    const uint32_t ops[3][2] = {{0u, 0u}, {0u, 16384u}, {32768u, 0u}};  // hi hi, hi lo, lo hi
+#pragma unroll
+    for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kb = ks / 4, w = (ks % 4) * 32;
+        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + Cf::AKQ + ops[pr][0] + kb * 16384 + w)),
+                        tc::desc_sw128(tc::smem_u32(sm + Cf::BKM + ops[pr][1] + kb * 8192 + w)), IDB,
+                        (pr | ks) ? 1u : 0u);
+      }
+    tc::mma_commit(&mma_bar);
+  }
+  if (!is_unsafe) {
+    tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+    tc::tc_after_sync();
+    // lanes 0-63: T row t (strictly lower); lanes 64-127: P row t (lower with the diagonal)
+    if (warp < 4) {
+      const int r = warp * 32 + lane;
+      const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, 0);
+      const int t = r & 63;
+      float* prow = p.P + (ch * C + t) * C;
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float v[16];
+        tc::tmem_ld16(lanes + 16 * c16, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+          const int i = 16 * c16 + ii;
+          if (r < 64)
+            Ts[t * 65 + i] = i < t ? v[ii] : 0.f;
+          else
+            prow[i] = i <= t ? v[ii] : 0.f;
+        }
+      }
+    }
+  } else {
+    // exact decay weights e^{L_t - L_i} <= 1 per element (rare: extreme decays)
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + Cf::QR);
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(sm + Cf::KR);
+    for (int e = tid; e < C * C; e += 256) {
+      const int t = e / C, i = e % C;
+      float st = 0.f, sp = 0.f;
+      if (i <= t && t < nv) {
+        for (int jj = 0; jj < D; ++jj) {
+          const float kw = __bfloat162float(ks[i * D + jj]) * expf(Ls[t * D + jj] - Ls[i * D + jj]);
+          st = fmaf(bg[row(t) + jj] * __bfloat162float(ks[t * D + jj]), kw, st);
+          sp = fmaf(__bfloat162float(qs[t * D + jj]), kw, sp);
+        }
+      }
+      Ts[t * 65 + i] = i < t ? st : 0.f;
+      p.P[(ch * C + t) * C + i] = i <= t ? sp : 0.f;
+    }
+  }
+  __syncthreads();
+
+  // ---- A = (I + T)^{-1}, blocked by 16
+  if (tid < 64) {
+    const int blk = tid >> 4, m = tid & 15, o = 16 * blk;
+    float col[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float s = t == m ? 1.f : 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2)
+        if (s2 >= m && s2 < t) s = fmaf(-Ts[(o + t) * 65 + o + s2], col[s2], s);
+      col[t] = t < m ? 0.f : s;
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) Xs[(o + t) * 65 + o + m] = col[t];
+  }
+  for (int e = tid; e < C * C; e += 256) {
+    const int t = e / C, i = e % C;
+    if ((i >> 4) > (t >> 4)) Xs[t * 65 + i] = 0.f;
+  }
+  __syncthreads();
+  for (int a = 1; a < 4; ++a) {
+    for (int e = tid; e < a * 256; e += 256) {
+      const int bb = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      float s = 0.f;
+      for (int kk = 16 * bb; kk < 16 * a; ++kk) s = fmaf(Ts[(16 * a + rr) * 65 + kk], Xs[kk * 65 + 16 * bb + cc], s);
+      Tb[bb * 272 + rr * 17 + cc] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < a * 256; e += 256) {
+      const int bb = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      float s = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) s = fmaf(Xs[(16 * a + rr) * 65 + 16 * a + kk], Tb[bb * 272 + kk * 17 + cc], s);
+      Xs[(16 * a + rr) * 65 + 16 * bb + cc] = -s;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < C * C; e += 256) p.A[ch * C * C + e] = Xs[(e / C) * 65 + (e % C)];
+
+  // ---- the bf16 operands of step 3, over the operands of step 1 (the
+  // MMA that read them has completed): E+ is read back before any is
+  // overwritten
+  float wv[32];  // the write gates of this thread's positions, loads in flight together
+#pragma unroll
+  for (int i = 0; i < 32; ++i) wv[i] = 32 * half + i < nv ? wg[row(32 * half + i) + j] : 0.f;
+  float ev[32];  // E+ (its factors are at most |b k|, so every chunk has it)
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t o = tc::sw128_off(32 * half + i, j, 128, 2);
+    ev[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::AKQ + o)) +
+            __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::AKQ + 32768 + o));
+  }
+  __syncthreads();
+  {
+    unsigned char* eh = sm + Cf::EH;
+    unsigned char* el = sm + Cf::EL;
+    unsigned char* zh = sm + Cf::ZH;
+    unsigned char* zl = sm + Cf::ZL;
+#pragma unroll
+    for (int i0 = 0; i0 < 32; ++i0) {
+      const int i = 32 * half + i0;
+      put_hl(eh, el, tc::sw128_off(j, i, 128, 2), ev[i0]);
+      const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::VR + (i * D + j) * 2));
+      put_hl(zh, zl, tc::sw128_off(j, i, 128, 2), wv[i0] * vv);  // Z^T row r = j
+    }
+    for (int e = tid; e < C * C; e += 256) {
+      const int t = e / C, i = e % C;
+      put_hl(sm + Cf::AH, sm + Cf::AL, tc::sw128_off(t, i, 64, 2), Xs[t * 65 + i]);
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    // TMEM columns 0-63: W^T = E+^T A^T; columns 64-127: U'^T = Z^T A^T
+    const uint32_t IDB = tc::idesc(128, 64, 1);
+    const uint32_t ops[3][2] = {{Cf::EH, Cf::AH}, {Cf::EH, Cf::AL}, {Cf::EL, Cf::AH}};
+    const uint32_t zops[3][2] = {{Cf::ZH, Cf::AH}, {Cf::ZH, Cf::AL}, {Cf::ZL, Cf::AH}};
+#pragma unroll
+    for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + ops[pr][0] + ks * 32)),
+                        tc::desc_sw128(tc::smem_u32(sm + ops[pr][1] + ks * 32)), IDB, (pr | ks) ? 1u : 0u);
+        tc::mma_bf16_ss(tmem + 64, tc::desc_sw128(tc::smem_u32(sm + zops[pr][0] + ks * 32)),
+                        tc::desc_sw128(tc::smem_u32(sm + zops[pr][1] + ks * 32)), IDB, (pr | ks) ? 1u : 0u);
+      }
+    tc::mma_commit(&mma_bar);
+  }
+  tc::mbar_wait<false>(&mma_bar, is_unsafe ? 0 : 1, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  {
+    // warps 0-3: lane j of W^T -> W[t][j]; warps 4-7: lane r of U'^T -> U'[t][r]
+    const int lr = (warp & 3) * 32 + lane;
+    const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, warp < 4 ? 0 : 64);
+    float* dst = (warp < 4 ? p.W : p.Up) + ch * C * D + lr;
+#pragma unroll
+    for (int c16 = 0; c16 < 4; ++c16) {
+      float v[16];
+      tc::tmem_ld16(lanes + 16 * c16, v);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) dst[(16 * c16 + ii) * D] = v[ii];
+    }
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------------------
+// The chunk outputs O = Q+ S0^T + P U, one CTA per chunk, all chunks in
+// parallel, computed transposed on tcgen05 (M = 128 value channels, N = 64
+// positions): O^T = S0 Q+^T + U^T P^T, every operand as bf16 high and low
+// parts (hi hi + hi lo + lo hi).  The operands arrive in fp32 from the
+// preparation kernel (Q+, P) and the chain (S0, U) and are split while they
+// are staged into shared memory.
+// ---------------------------------------------------------------------------
+struct GOutCfg {
+  static constexpr uint32_t SH = 0, SL = 32768;          // S0 [r][j], 2 K blocks x 128 rows
+  static constexpr uint32_t QH = 65536, QL = 81920;      // Q+ [t][j], 2 K blocks x 64 rows
+  static constexpr uint32_t UH = 98304, UL = 114688;     // U^T [r][i], 128 rows
+  static constexpr uint32_t PH = 131072, PL = 139264;    // P [t][i], 64 rows
+  static constexpr uint32_t BYTES = 147456 + 1024;
+};
+
+// four consecutive K elements (a 16-byte-aligned quarter of a swizzle chunk) as hi and lo parts
+__device__ __forceinline__ void put_hl4(unsigned char* hi, unsigned char* lo, uint32_t off, float4 x) {
+  const __nv_bfloat162 h0 = __floats2bfloat162_rn(x.x, x.y), h1 = __floats2bfloat162_rn(x.z, x.w);
+  const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+  uint2 hv, lv;
+  hv.x = *reinterpret_cast<const uint32_t*>(&h0);
+  hv.y = *reinterpret_cast<const uint32_t*>(&h1);
+  const __nv_bfloat162 l0 = __floats2bfloat162_rn(x.x - f0.x, x.y - f0.y), l1 = __floats2bfloat162_rn(x.z - f1.x, x.w - f1.y);
+  lv.x = *reinterpret_cast<const uint32_t*>(&l0);
+  lv.y = *reinterpret_cast<const uint32_t*>(&l1);
+  *reinterpret_cast<uint2*>(hi + off) = hv;
+  *reinterpret_cast<uint2*>(lo + off) = lv;
+}
+
+__global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnWs p, __nv_bfloat16* __restrict__ out,
+                                                      int* __restrict__ err) {
+  using Cf = GOutCfg;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = blockIdx.x;
+  if (tid == 0) {
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 64);
+  // stage the operands: four consecutive elements per thread and step, read as
+  // float4, every load of a group issued before its data is used
+  {
+    const float4* s0 = reinterpret_cast<const float4*>(p.S0 + ch * D * D);
+    const float4* qp = reinterpret_cast<const float4*>(p.Qp + ch * C * D);
+    const float4* pp = reinterpret_cast<const float4*>(p.P + ch * C * C);
+    const float4* uu = reinterpret_cast<const float4*>(p.U + ch * C * D);
+    float4 x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = s0[tid + 256 * i];
+    float4 y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = qp[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {  // S0 [r][j]
+      const int e = tid + 256 * i, r = e / (D / 4), j = 4 * (e % (D / 4));
+      put_hl4(sm + Cf::SH, sm + Cf::SL, tc::sw128_off(r, j, 128, 2), x[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = uu[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[8 + i] = pp[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // Q+ [t][j]
+      const int e = tid + 256 * i, t = e / (D / 4), j = 4 * (e % (D / 4));
+      put_hl4(sm + Cf::QH, sm + Cf::QL, tc::sw128_off(t, j, 64, 2), y[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // P [t][i]
+      const int e = tid + 256 * i, t = e / (C / 4), ii = 4 * (e % (C / 4));
+      put_hl4(sm + Cf::PH, sm + Cf::PL, tc::sw128_off(t, ii, 64, 2), x[8 + i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // U [i][r] -> U^T [r][i]
+      const int e = tid + 256 * i, ii = e / (D / 4), r = 4 * (e % (D / 4));
+      const float xs[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const __nv_bfloat16 hh = __float2bfloat16_rn(xs[c]);
+        const uint32_t off = tc::sw128_off(r + c, ii, 128, 2);
+        *reinterpret_cast<__nv_bfloat16*>(sm + Cf::UH + off) = hh;
+        *reinterpret_cast<__nv_bfloat16*>(sm + Cf::UL + off) = __float2bfloat16_rn(xs[c] - __bfloat162float(hh));
+      }
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 0) {
+    const uint32_t IDB = tc::idesc(128, 64, 1);
+    const uint32_t sq[3][2] = {{Cf::SH, Cf::QH}, {Cf::SH, Cf::QL}, {Cf::SL, Cf::QH}};
+    const uint32_t up[3][2] = {{Cf::UH, Cf::PH}, {Cf::UH, Cf::PL}, {Cf::UL, Cf::PH}};
+#pragma unroll
+    for (int pr = 0; pr < 3; ++pr) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)  // S0 Q+^T: K = 128 channels, two swizzle blocks
+        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + sq[pr][0] + (ks / 4) * 16384 + (ks % 4) * 32)),
+                        tc::desc_sw128(tc::smem_u32(sm + sq[pr][1] + (ks / 4) * 8192 + (ks % 4) * 32)), IDB,
+                        (pr | ks) ? 1u : 0u);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)  // U^T P^T: K = 64 positions
+        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + up[pr][0] + ks * 32)),
+                        tc::desc_sw128(tc::smem_u32(sm + up[pr][1] + ks * 32)), IDB, 1u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  {
+    // lane r of O^T; warps 0-3 take positions 0-31, warps 4-7 positions 32-63
+    const int r = (warp & 3) * 32 + lane, tb = (warp >> 2) * 32;
+    const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, tb);
+#pragma unroll
+    for (int c16 = 0; c16 < 2; ++c16) {
+      float v[16];
+      tc::tmem_ld16(lanes + 16 * c16, v);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) {
+        const int t = tb + 16 * c16 + ii;
+        if (t < nv) out[(((size_t)b * T + t0 + t) * H + h) * D + r] = __float2bfloat16_rn(v[ii]);
+      }
+    }
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 64);
+}
+
+// ---------------------------------------------------------------------------
+// The forward chain on tcgen05, one CTA per (b, h), chunks in order:
+//   U_n     = U'_n - W_n S_n^T                 (MMA 1: X^T = S W^T, M = 128 rows of S, N = 64)
+//   S_{n+1} = S_n diag(gamma_C,n) + U_n^T K^e_n  (MMA 2: U^T K^e, M = 128, N = 128)
+// Every value row of the state evolves on its own (the erase reads S e, one
+// value per row), so one CTA holds the whole state, row r in TMEM lane r, and
+// no exchange between CTAs is needed.  Both products take bf16 high and low
+// parts of both operands (hi hi + hi lo + lo hi); the state itself stays fp32
+// in registers.
+// Warp roles (416 threads):
+//   warps 0-7   state warps: thread (r, c) holds row r, key channels 64c..64c+63
+//               of S, and positions 32c..32c+31 of U; U = U' - X, the operand
+//               U^T, the state update, its operand copy and its saves.
+//   warps 8-11  producer: chunk n+1's W and K^e^T (bf16 hi, lo) and gamma_C
+//               staged into one of two slots while chunk n runs.
+//   warp 12     issuer: one thread issues every MMA.
+// Every wait is bounded; on expiry the kernel records a timeout in the
+// library's error word and each role runs its loop out without waiting.
+// ---------------------------------------------------------------------------
+struct GChainCfg {
+  static constexpr uint32_t SH = 0, SL = 32768;        // S [r][j] hi, lo: 2 K blocks x 128 rows
+  static constexpr uint32_t UH = 65536, UL = 81920;    // U^T [r][t] hi, lo: 128 rows
+  static constexpr uint32_t SLOT = 98304;              // 2 slots of 64 KB:
+  static constexpr uint32_t SLOT_SZ = 65536;
+  static constexpr uint32_t WH = 0, WL = 16384;        //   W [t][j] hi, lo: 2 K blocks x 64 rows
+  static constexpr uint32_t KH = 32768, KL = 49152;    //   K^e^T [j][t] hi, lo: 128 rows
+  static constexpr uint32_t BYTES = SLOT + 2 * SLOT_SZ + 1024;
+  static constexpr int THREADS = 416;
+  static constexpr uint32_t X_COL = 0, D_COL = 64;     // TMEM: X^T (64 columns), S update (128 columns)
+};
+
+__device__ __forceinline__ void g_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(b)) : "memory");
+}
+
+// eight consecutive K elements (one 16-byte swizzle chunk) of an operand row as hi and lo parts
+__device__ __forceinline__ void put_hl8(unsigned char* hi, unsigned char* lo, uint32_t off, const float* x) {
+  uint4 hv, lv;
+  uint32_t* hp = reinterpret_cast<uint32_t*>(&hv);
+  uint32_t* lp = reinterpret_cast<uint32_t*>(&lv);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+    const float2 f = __bfloat1622float2(hh);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * q] - f.x, x[2 * q + 1] - f.y);
+    hp[q] = *reinterpret_cast<const uint32_t*>(&hh);
+    lp[q] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  *reinterpret_cast<uint4*>(hi + off) = hv;
+  *reinterpret_cast<uint4*>(lo + off) = lv;
+}
+
+__global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const float* __restrict__ S0,
+                                                                      float* __restrict__ ST, int H, int NC,
+                                                                      GdnWs p, int* __restrict__ err) {
+  using Cf = GChainCfg;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  // full / empty: a slot's tiles staged / read by the MMAs; g_free: its gamma_C read by the state warps
+  __shared__ uint64_t full[2], empty[2], g_free[2], s_ready, x_done, u_ready, d_done;
+  __shared__ float gs[2][D];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t unit = blockIdx.x;  // b * H + h
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&full[i], 128);
+      tc::mbar_init(&empty[i], 1);
+      tc::mbar_init(&g_free[i], 256);
+    }
+    tc::mbar_init(&s_ready, 256);
+    tc::mbar_init(&x_done, 1);
+    tc::mbar_init(&u_ready, 256);
+    tc::mbar_init(&d_done, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 256);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp < 8) {
+    // ---- state warps
+    const int r = (warp & 3) * 32 + lane, c = warp >> 2;
+    float S[64];
+    {
+      const float* src = S0 ? S0 + (unit * D + r) * D + 64 * c : nullptr;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 v = src ? reinterpret_cast<const float4*>(src)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        S[4 * q] = v.x;
+        S[4 * q + 1] = v.y;
+        S[4 * q + 2] = v.z;
+        S[4 * q + 3] = v.w;
+      }
+    }
+    for (int n = 0; n < NC; ++n) {
+      const size_t ch = unit * NC + n;
+      // this chunk's start state: its save, and its operand copy for MMA 1
+      float4* sv = reinterpret_cast<float4*>(p.S0 + (ch * D + r) * D + 64 * c);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) sv[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        put_hl8(sm + Cf::SH, sm + Cf::SL, tc::sw128_off(r, 64 * c + 8 * q, 128, 2), S + 8 * q);
+      tc::fence_proxy_async();
+      g_arrive(&s_ready);
+      // U' for this thread's positions, loaded while MMA 1 runs
+      float up[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) up[i] = p.Up[(ch * C + 32 * c + i) * D + r];
+      tc::mbar_wait<false>(&x_done, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      {
+        const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, Cf::X_COL + 32 * c);
+        float u[32];
+#pragma unroll
+        for (int h16 = 0; h16 < 2; ++h16) {
+          float x[16];
+          tc::tmem_ld16(lanes + 16 * h16, x);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) u[16 * h16 + i] = up[16 * h16 + i] - x[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p.U[(ch * C + 32 * c + i) * D + r] = u[i];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          put_hl8(sm + Cf::UH, sm + Cf::UL, tc::sw128_off(r, 32 * c + 8 * q, 128, 2), u + 8 * q);
+      }
+      tc::fence_proxy_async();
+      tc::tc_before_sync();
+      g_arrive(&u_ready);
+      tc::mbar_wait<false>(&d_done, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      {
+        const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, Cf::D_COL + 64 * c);
+        const float* g = gs[n & 1] + 64 * c;
+#pragma unroll
+        for (int h16 = 0; h16 < 4; ++h16) {
+          float dd[16];
+          tc::tmem_ld16(lanes + 16 * h16, dd);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) S[16 * h16 + i] = fmaf(S[16 * h16 + i], g[16 * h16 + i], dd[i]);
+        }
+      }
+      g_arrive(&g_free[n & 1]);
+      tc::tc_before_sync();
+    }
+    if (ST) {
+      float4* dst = reinterpret_cast<float4*>(ST + (unit * D + r) * D + 64 * c);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+    }
+  } else if (warp < 12) {
+    // ---- producer: chunk n's W and K^e^T into slot n % 2
+    const int pt = tid - 256;  // 0..127
+    for (int n = 0; n < NC; ++n) {
+      const int slot = n & 1;
+      if (n >= 2) {
+        tc::mbar_wait<false>(&empty[slot], ((n >> 1) - 1) & 1, err, tc::kErrTimeoutMma, &abort_flag);
+        tc::mbar_wait<false>(&g_free[slot], ((n >> 1) - 1) & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      }
+      unsigned char* sl = sm + Cf::SLOT + slot * Cf::SLOT_SZ;
+      const size_t ch = unit * NC + n;
+      if (pt < 3 && n + kChainAhead < NC) {
+        // pull chunk n + kChainAhead's operands into L2, so that this role's
+        // loads and the state warps' loads of U' find them there
+        const size_t ca = ch + kChainAhead;
+        const float* src = pt == 0 ? p.W : pt == 1 ? p.Ke : p.Up;
+        tc::prefetch_l2(src + ca * C * D, C * D * 4);
+      }
+      // W [t][j]: eight channels per group, consecutive threads along a row;
+      // every load of a tile is issued before any of its data is used
+      const float4* w = reinterpret_cast<const float4*>(p.W + ch * C * D);
+      {
+        float4 a[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = pt + 128 * i;  // group e: row e / 16, channels 8 (e % 16) ..
+          a[2 * i] = w[2 * e];
+          a[2 * i + 1] = w[2 * e + 1];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = pt + 128 * i, t = e / (D / 8), j = 8 * (e % (D / 8));
+          const float x[8] = {a[2 * i].x, a[2 * i].y, a[2 * i].z, a[2 * i].w,
+                              a[2 * i + 1].x, a[2 * i + 1].y, a[2 * i + 1].z, a[2 * i + 1].w};
+          put_hl8(sl + Cf::WH, sl + Cf::WL, tc::sw128_off(t, j, 64, 2), x);
+        }
+      }
+      // K^e^T [j][t]: thread pt takes channel j = pt, all 64 positions
+      {
+        const float* ke = p.Ke + ch * C * D + pt;
+        float x[C];
+#pragma unroll
+        for (int t = 0; t < C; ++t) x[t] = ke[t * D];
+#pragma unroll
+        for (int t8 = 0; t8 < C; t8 += 8) put_hl8(sl + Cf::KH, sl + Cf::KL, tc::sw128_off(pt, t8, 128, 2), x + t8);
+      }
+      gs[slot][pt] = p.gC[ch * D + pt];
+      tc::fence_proxy_async();
+      g_arrive(&full[slot]);
+    }
+  } else if (warp == 12 && lane == 0) {
+    // ---- issuer
+    const uint32_t ID1 = tc::idesc(128, 64, 1), ID2 = tc::idesc(128, 128, 1);
+    for (int n = 0; n < NC; ++n) {
+      const int slot = n & 1;
+      const uint32_t sl = Cf::SLOT + slot * Cf::SLOT_SZ;
+      tc::mbar_wait<false>(&full[slot], (n >> 1) & 1, err, tc::kErrTimeoutLoad, &abort_flag);
+      tc::mbar_wait<false>(&s_ready, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      const uint32_t a1[3] = {Cf::SH, Cf::SH, Cf::SL}, b1[3] = {sl + Cf::WH, sl + Cf::WL, sl + Cf::WH};
+#pragma unroll
+      for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_bf16_ss(tmem + Cf::X_COL,
+                          tc::desc_sw128(tc::smem_u32(sm + a1[pr] + (ks / 4) * 16384 + (ks % 4) * 32)),
+                          tc::desc_sw128(tc::smem_u32(sm + b1[pr] + (ks / 4) * 8192 + (ks % 4) * 32)), ID1,
+                          (pr | ks) ? 1u : 0u);
+      tc::mma_commit(&x_done);
+      tc::mbar_wait<false>(&u_ready, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      tc::tc_after_sync();
+      const uint32_t a2[3] = {Cf::UH, Cf::UH, Cf::UL}, b2[3] = {sl + Cf::KH, sl + Cf::KL, sl + Cf::KH};
+#pragma unroll
+      for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          tc::mma_bf16_ss(tmem + Cf::D_COL, tc::desc_sw128(tc::smem_u32(sm + a2[pr] + ks * 32)),
+                          tc::desc_sw128(tc::smem_u32(sm + b2[pr] + ks * 32)), ID2, (pr | ks) ? 1u : 0u);
+      tc::mma_commit(&d_done);
+      tc::mma_commit(&empty[slot]);
+    }
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+}
+
+}  // namespace
+
+bool gdn2_tc_supported(const GdnLayout& L) { return L.dtype == 1 && L.dk == D && L.dv == D; }
+
+cudaError_t launch_gdn2_chain_tc(const GdnArgs& a, int* err, cudaStream_t st) {
+  const GdnLayout& L = a.L;
+  const GdnWs p = gdn_ws(a.ws, L);
+  cudaError_t e = cudaFuncSetAttribute(gdn2_chain_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)GChainCfg::BYTES);
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "gdn2_chain_tc");
+  gdn2_chain_tc<<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(a.S0, a.ST, L.H, L.NC, p, err);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gdn2_out_tc(const GdnArgs& a, int* err, cudaStream_t st) {
+  const GdnLayout& L = a.L;
+  const GdnWs p = gdn_ws(a.ws, L);
+  cudaError_t e = cudaFuncSetAttribute(gdn2_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)GOutCfg::BYTES);
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "gdn2_out_tc");
+  gdn2_out_tc<<<(unsigned)L.chunks, 256, GOutCfg::BYTES, st>>>(L.H, L.T, L.NC, p,
+                                                               static_cast<__nv_bfloat16*>(a.out), err);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gdn2_prep_tc(const GdnArgs& a, int* err, cudaStream_t st) {
+  const GdnLayout& L = a.L;
+  const GdnWs p = gdn_ws(a.ws, L);
+  CUtensorMap tm_q, tm_k, tm_v, tm_loga;
+  if (!make_tmap_bthd(&tm_q, a.q, 2, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_k, a.k, 2, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 128, false) ||
+      !make_tmap_bthd(&tm_loga, a.loga, 4, L.B, L.T, L.H, D, 128, false))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(gdn2_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)GPrepCfg::BYTES);
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "gdn2_prep_tc");
+  gdn2_prep_tc<<<(unsigned)L.chunks, 256, GPrepCfg::BYTES, st>>>(tm_q, tm_k, tm_v, tm_loga, a.b, a.w, L.H, L.T,
+                                                                 L.NC, p, err);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+}  // namespace kd

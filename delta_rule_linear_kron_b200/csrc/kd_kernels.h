@@ -245,6 +245,7 @@ struct GdnArgs {
   const char* fws;
   char* ws;
   GdnLayout L;
+  int* err = nullptr;  // the library's device error word (tensor-core kernels' bounded waits)
 };
 struct GdnDecodeArgs {
   const void *q, *k, *v;
@@ -255,6 +256,11 @@ struct GdnDecodeArgs {
 };
 cudaError_t launch_gdn2_decode(const GdnDecodeArgs& a, cudaStream_t st);
 cudaError_t launch_gdn2_fwd(const GdnArgs& a, cudaStream_t st);
+// bf16 with d_k = d_v = 128: the per-chunk preparation runs on tensor cores
+bool gdn2_tc_supported(const GdnLayout& L);
+cudaError_t launch_gdn2_prep_tc(const GdnArgs& a, int* err, cudaStream_t st);
+cudaError_t launch_gdn2_out_tc(const GdnArgs& a, int* err, cudaStream_t st);
+cudaError_t launch_gdn2_chain_tc(const GdnArgs& a, int* err, cudaStream_t st);
 cudaError_t launch_gdn2_bwd(const GdnArgs& a, cudaStream_t st);
 
 // Gated inputs (kd_gate.cu): logf = e^{a_log} log sigma(f~) into a buffer

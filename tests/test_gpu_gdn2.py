@@ -118,6 +118,17 @@ def test_gdn2_extreme_decay():
     check(inp, "f32")
 
 
+def test_gdn2_extreme_decay_tensor_cores():
+    """The same extreme decays on the tensor-core preparation (bf16, d = 128):
+    chunks whose in-chunk |L| reaches its factorised range take per-element
+    weights, the others the tf32 products; both in one problem."""
+    inp = kin.make_gdn2_inputs(1, 2, 260, 128, 128, "bf16", seed=18)
+    inp["loga"][:, 70:78, 0, :8] = -30.0
+    inp["loga"][:, :, 1, :] *= 40.0
+    inp["loga"] = kin.round_to_dtype(inp["loga"], "f32")
+    check(inp, "bf16")
+
+
 def test_gdn2_workload_B1_H16_T16384_sampled_heads():
     """The mixer's full-size shape (B=1, H=16, T=16384, d=128, bf16), run whole
     on the GPU; heads 0 and 11 checked against the oracle."""
