@@ -154,7 +154,14 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
   L->Ke = take(chunks * C * dk);
   L->Qp = take(chunks * C * dk);
   L->gC = take(chunks * dk);
-  L->S0 = take(chunks * (size_t)dv * dk);
+  L->tc = dtype == KD_BF16 && dk == 128 && dv == 128;
+  if (L->tc) {
+    L->S0img = take(chunks * (size_t)dv * dk);  // bf16 hi + lo: the bytes of one fp32 tile
+    L->Wimg = take(chunks * C * dk);
+    L->KeTimg = take(chunks * C * dk);
+  } else {
+    L->S0 = take(chunks * (size_t)dv * dk);
+  }
   L->U = take(chunks * C * dv);
   L->fwd_bytes = off;
   off = 0;
@@ -165,6 +172,14 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
   L->dP = take(chunks * C * C);
   L->dQp = take(chunks * C * dk);
   L->dKe = take(chunks * C * dk);
+  if (L->tc) {
+    L->S0b = take(chunks * (size_t)dv * dk);
+    L->Keimg = take(chunks * C * dk);
+    L->WTimg = take(chunks * C * dk);
+    L->dUi = take(chunks * C * dv);
+    L->L2t = take(chunks * (size_t)dk * dv);
+    L->dSimg = take(chunks * (size_t)dv * dk);
+  }
   L->bwd_bytes = off;
   return KD_OK;
 }
@@ -894,6 +909,11 @@ int kron_delta_gdn2_bwd(const void* q, const void* k, const void* v, const float
   a.fws = static_cast<const char*>(fwd_ws);
   a.ws = static_cast<char*>(workspace);
   a.L = L;
+  if (kd::gdn2_tc_supported(L)) {  // the tensor-core kernels report bounded-wait timeouts here
+    DeviceInfo di;
+    KD_TRY(device_info(&di));
+    a.err = di.err;
+  }
   return launched(kd::launch_gdn2_bwd(a, static_cast<cudaStream_t>(stream)), "gdn2 backward launch");
 }
 

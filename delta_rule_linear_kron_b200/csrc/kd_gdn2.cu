@@ -1101,16 +1101,22 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   const GdnLayout& L = a.L;
   GdnWs p = gdn_ws(const_cast<char*>(a.fws), L);
   gdn_bwd_ws(a.ws, L, &p);
+  // tensor-core forward: its chunk-start states were kept as bf16 hi, lo images
+  if (L.tc) KD_TRYC(launch_gdn2_s0_unpack(p.S0img, p.S0, L.chunks, st));
   const dim3 gc(L.NC, L.H, L.B), gr(DV / kRows, L.H, L.B);
-  KD_TRYC(set_smem(gdn2_bchain<DK, DV, Tin>, S::bchain));
+  if (!L.tc) KD_TRYC(set_smem(gdn2_bchain<DK, DV, Tin>, S::bchain));
   KD_TRYC(set_smem(gdn2_bpost_a<DK, DV, Tin>, S::bpa));
   KD_TRYC(set_smem(gdn2_bpost_b<DK, DV, Tin>, S::bpb));
   KD_TRYC(set_smem(gdn2_bpost_exact<DK, DV, Tin>, S::bpe));
   const Tin* dO = static_cast<const Tin*>(a.dO);
-  prof_begin(st, "gdn2_bchain");
-  gdn2_bchain<DK, DV, Tin><<<gr, kChainThreads, S::bchain, st>>>(dO, a.dST, a.dS0, L.H, L.T, L.NC, p);
-  prof_end(st);
-  KD_TRYC(cudaGetLastError());
+  if (L.tc) {
+    KD_TRYC(launch_gdn2_bchain_tc(a, p, a.err, st));
+  } else {
+    prof_begin(st, "gdn2_bchain");
+    gdn2_bchain<DK, DV, Tin><<<gr, kChainThreads, S::bchain, st>>>(dO, a.dST, a.dS0, L.H, L.T, L.NC, p);
+    prof_end(st);
+    KD_TRYC(cudaGetLastError());
+  }
   prof_begin(st, "gdn2_bpost_a");
   gdn2_bpost_a<DK, DV, Tin><<<gc, 256, S::bpa, st>>>(static_cast<const Tin*>(a.v), a.w, dO, L.H, L.T, L.NC, p,
                                                      static_cast<Tin*>(a.dv), a.dw);

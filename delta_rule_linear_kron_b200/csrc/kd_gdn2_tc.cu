@@ -52,6 +52,8 @@ struct GPrepCfg {
   static constexpr uint32_t LOAD_BYTES = 3 * 16384 + 32768;
   // the bf16 operands of step 3
   static constexpr uint32_t EH = 0, EL = 16384, ZH = 32768, ZL = 49152, AH = 65536, AL = 73728;
+  // the forward chain's operand images, staged once step 3 is done (32 KB each)
+  static constexpr uint32_t IW = 0, IK = 32768;
 };
 
 __device__ __forceinline__ void put_hl(unsigned char* hi, unsigned char* lo, uint32_t off, float x) {
@@ -298,7 +300,10 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
   tc::mbar_wait<false>(&mma_bar, is_unsafe ? 0 : 1, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
   {
-    // warps 0-3: lane j of W^T -> W[t][j]; warps 4-7: lane r of U'^T -> U'[t][r]
+    // warps 0-3: lane j of W^T -> W[t][j] and the forward chain's image of W
+    // ([t][j], bf16 hi, lo); warps 4-7: lane r of U'^T -> U'[t][r], then the
+    // chain's image of K^e^T ([j][t], bf16 hi, lo) for channel j = r.  The
+    // operand tiles of steps 1 and 3 are free (their MMAs have completed).
     const int lr = (warp & 3) * 32 + lane;
     const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, warp < 4 ? 0 : 64);
     float* dst = (warp < 4 ? p.W : p.Up) + ch * C * D + lr;
@@ -308,10 +313,30 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
       tc::tmem_ld16(lanes + 16 * c16, v);
       tc::tmem_ld_wait();
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) dst[(16 * c16 + ii) * D] = v[ii];
+      for (int ii = 0; ii < 16; ++ii) {
+        const int t = 16 * c16 + ii;
+        dst[t * D] = v[ii];
+        if (warp < 4) put_hl(sm + Cf::IW, sm + Cf::IW + 16384, tc::sw128_off(t, lr, 64, 2), v[ii]);
+      }
+    }
+    if (warp >= 4) {
+      const float lj = lam[lr];
+#pragma unroll 8
+      for (int t = 0; t < C; ++t) {
+        const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::KR + (t * D + lr) * 2));
+        put_hl(sm + Cf::IK, sm + Cf::IK + 16384, tc::sw128_off(lr, t, 128, 2), kk * expf(lj - Ls[t * D + lr]));
+      }
     }
   }
+  tc::fence_proxy_async();
   tc::tc_before_sync();
+  __syncthreads();
+  if (tid == 0) {
+    tc::bulk_s2g(p.Wimg + ch * (2 * C * D), sm + Cf::IW, 4u * C * D);
+    tc::bulk_s2g(p.KeTimg + ch * (2 * C * D), sm + Cf::IK, 4u * C * D);
+    tc::bulk_commit();
+    tc::bulk_wait_read();
+  }
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
 }
@@ -320,9 +345,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
 // The chunk outputs O = Q+ S0^T + P U, one CTA per chunk, all chunks in
 // parallel, computed transposed on tcgen05 (M = 128 value channels, N = 64
 // positions): O^T = S0 Q+^T + U^T P^T, every operand as bf16 high and low
-// parts (hi hi + hi lo + lo hi).  The operands arrive in fp32 from the
-// preparation kernel (Q+, P) and the chain (S0, U) and are split while they
-// are staged into shared memory.
+// parts (hi hi + hi lo + lo hi).  S0 arrives as the chain's saved image (one
+// bulk copy); Q+, P (preparation kernel) and U (chain) arrive in fp32 and are
+// split while they are staged into shared memory.
 // ---------------------------------------------------------------------------
 struct GOutCfg {
   static constexpr uint32_t SH = 0, SL = 32768;          // S0 [r][j], 2 K blocks x 128 rows
@@ -351,7 +376,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
   using Cf = GOutCfg;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ uint64_t mma_bar;
+  __shared__ uint64_t ld_bar, mma_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -360,29 +385,25 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = blockIdx.x;
   if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
+    // S0 arrives as the chain's saved image: its hi and lo tiles as they are
+    tc::mbar_expect_tx(&ld_bar, 4u * D * D);
+    tc::bulk_g2s(sm + Cf::SH, p.S0img + ch * (2 * D * D), 2u * D * D, &ld_bar);
+    tc::bulk_g2s(sm + Cf::SL, p.S0img + ch * (2 * D * D) + D * D, 2u * D * D, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 64);
   // stage the operands: four consecutive elements per thread and step, read as
   // float4, every load of a group issued before its data is used
   {
-    const float4* s0 = reinterpret_cast<const float4*>(p.S0 + ch * D * D);
     const float4* qp = reinterpret_cast<const float4*>(p.Qp + ch * C * D);
     const float4* pp = reinterpret_cast<const float4*>(p.P + ch * C * C);
     const float4* uu = reinterpret_cast<const float4*>(p.U + ch * C * D);
-    float4 x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = s0[tid + 256 * i];
-    float4 y[8];
+    float4 x[12], y[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = qp[tid + 256 * i];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {  // S0 [r][j]
-      const int e = tid + 256 * i, r = e / (D / 4), j = 4 * (e % (D / 4));
-      put_hl4(sm + Cf::SH, sm + Cf::SL, tc::sw128_off(r, j, 128, 2), x[i]);
-    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[i] = uu[tid + 256 * i];
 #pragma unroll
@@ -415,6 +436,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
   __syncthreads();
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
   if (tid == 0) {
     const uint32_t IDB = tc::idesc(128, 64, 1);
     const uint32_t sq[3][2] = {{Cf::SH, Cf::QH}, {Cf::SH, Cf::QL}, {Cf::SL, Cf::QH}};
@@ -465,13 +487,15 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
 // no exchange between CTAs is needed.  Both products take bf16 high and low
 // parts of both operands (hi hi + hi lo + lo hi); the state itself stays fp32
 // in registers.
-// Warp roles (416 threads):
+// Warp roles (320 threads):
 //   warps 0-7   state warps: thread (r, c) holds row r, key channels 64c..64c+63
 //               of S, and positions 32c..32c+31 of U; U = U' - X, the operand
-//               U^T, the state update, its operand copy and its saves.
-//   warps 8-11  producer: chunk n+1's W and K^e^T (bf16 hi, lo) and gamma_C
-//               staged into one of two slots while chunk n runs.
-//   warp 12     issuer: one thread issues every MMA.
+//               U^T, the state update and its operand copy (bf16 hi, lo), which
+//               the issuer also copies out as the chunk's saved start state.
+//   warp 8      producer: one thread copies chunk n+1's operand images (bf16
+//               hi, lo, written by the preparation kernel) and gamma_C into one
+//               of two slots while chunk n runs, and pulls later chunks into L2.
+//   warp 9      issuer: one thread issues every MMA.
 // Every wait is bounded; on expiry the kernel records a timeout in the
 // library's error word and each role runs its loop out without waiting.
 // ---------------------------------------------------------------------------
@@ -483,7 +507,7 @@ struct GChainCfg {
   static constexpr uint32_t WH = 0, WL = 16384;        //   W [t][j] hi, lo: 2 K blocks x 64 rows
   static constexpr uint32_t KH = 32768, KL = 49152;    //   K^e^T [j][t] hi, lo: 128 rows
   static constexpr uint32_t BYTES = SLOT + 2 * SLOT_SZ + 1024;
-  static constexpr int THREADS = 416;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t X_COL = 0, D_COL = 64;     // TMEM: X^T (64 columns), S update (128 columns)
 };
 
@@ -508,22 +532,34 @@ __device__ __forceinline__ void put_hl8(unsigned char* hi, unsigned char* lo, ui
   *reinterpret_cast<uint4*>(lo + off) = lv;
 }
 
-__global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const float* __restrict__ S0,
-                                                                      float* __restrict__ ST, int H, int NC,
-                                                                      GdnWs p, int* __restrict__ err) {
+// What the two directions of the chain read and write.
+struct GChainIO {
+  const float* init;   // S0 (forward) or dS_T (backward) [B][H][dv][dk]; nullptr: zero
+  float* fin;          // S_T or dS0; nullptr: not written
+  const __nv_bfloat16* b1;  // MMA 1's B operand image [ch] ([t][j] hi, lo): W (forward) or K^e (backward)
+  const __nv_bfloat16* b2;  // MMA 2's B operand image [ch] ([j][t] hi, lo): K^e^T (forward) or W^T (backward)
+  const float* gC;     // gamma_C [ch][j]
+  const float* ul;     // [ch][t][r]: U' (forward) or P^T dO (backward)
+  const float* l2t;    // backward: (dO^T Q+)^T [ch][j][r], added to the state update
+  float* uout;         // U (forward) or dU (backward) [ch][t][r]
+  __nv_bfloat16* img;  // the saved state images [ch] (bf16 hi, lo)
+};
+
+template <bool BWD>
+__global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO io, int NC, int* __restrict__ err) {
   using Cf = GChainCfg;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   // full / empty: a slot's tiles staged / read by the MMAs; g_free: its gamma_C read by the state warps
   __shared__ uint64_t full[2], empty[2], g_free[2], s_ready, x_done, u_ready, d_done;
-  __shared__ float gs[2][D];
+  __shared__ __align__(16) float gs[2][D];  // gamma_C per slot (a bulk-copy destination)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t unit = blockIdx.x;  // b * H + h
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&full[i], 128);
+      tc::mbar_init(&full[i], 1);
       tc::mbar_init(&empty[i], 1);
       tc::mbar_init(&g_free[i], 256);
     }
@@ -545,7 +581,7 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const flo
     const int r = (warp & 3) * 32 + lane, c = warp >> 2;
     float S[64];
     {
-      const float* src = S0 ? S0 + (unit * D + r) * D + 64 * c : nullptr;
+      const float* src = io.init ? io.init + (unit * D + r) * D + 64 * c : nullptr;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
         const float4 v = src ? reinterpret_cast<const float4*>(src)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -555,22 +591,23 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const flo
         S[4 * q + 3] = v.w;
       }
     }
-    for (int n = 0; n < NC; ++n) {
+    for (int k = 0; k < NC; ++k) {
+      const int n = BWD ? NC - 1 - k : k;  // the backward runs from the last chunk to the first
       const size_t ch = unit * NC + n;
-      // this chunk's start state: its save, and its operand copy for MMA 1
-      float4* sv = reinterpret_cast<float4*>(p.S0 + (ch * D + r) * D + 64 * c);
-#pragma unroll
-      for (int q = 0; q < 16; ++q) sv[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+      // this chunk's start state as MMA 1's operand; the issuer also copies
+      // this image out as the chunk's saved start state (one bulk copy: the
+      // rows of a thread-per-row state would scatter over 128 rows)
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         put_hl8(sm + Cf::SH, sm + Cf::SL, tc::sw128_off(r, 64 * c + 8 * q, 128, 2), S + 8 * q);
       tc::fence_proxy_async();
       g_arrive(&s_ready);
-      // U' for this thread's positions, loaded while MMA 1 runs
+      // U' (forward) or P^T dO (backward) at this thread's positions, loaded
+      // while MMA 1 runs
       float up[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) up[i] = p.Up[(ch * C + 32 * c + i) * D + r];
-      tc::mbar_wait<false>(&x_done, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      for (int i = 0; i < 32; ++i) up[i] = io.ul[(ch * C + 32 * c + i) * D + r];
+      tc::mbar_wait<false>(&x_done, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
       {
         const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, Cf::X_COL + 32 * c);
@@ -581,10 +618,14 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const flo
           tc::tmem_ld16(lanes + 16 * h16, x);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) u[16 * h16 + i] = up[16 * h16 + i] - x[i];
+          for (int i = 0; i < 16; ++i) u[16 * h16 + i] = BWD ? up[16 * h16 + i] + x[i] : up[16 * h16 + i] - x[i];
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) p.U[(ch * C + 32 * c + i) * D + r] = u[i];
+        for (int i = 0; i < 32; ++i) io.uout[(ch * C + 32 * c + i) * D + r] = u[i];
+        if (BWD) {  // MMA 2 subtracts dU^T W: its operand is -dU^T
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = -u[i];
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           put_hl8(sm + Cf::UH, sm + Cf::UL, tc::sw128_off(r, 32 * c + 8 * q, 128, 2), u + 8 * q);
@@ -592,106 +633,99 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const flo
       tc::fence_proxy_async();
       tc::tc_before_sync();
       g_arrive(&u_ready);
-      tc::mbar_wait<false>(&d_done, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      // the backward's dO^T Q+ term of this thread's state row, loaded while MMA 2 runs
+      float l2[BWD ? 64 : 1];
+      if (BWD) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) l2[i] = io.l2t[(ch * D + 64 * c + i) * D + r];
+      }
+      tc::mbar_wait<false>(&d_done, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
       {
         const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, Cf::D_COL + 64 * c);
-        const float* g = gs[n & 1] + 64 * c;
+        const float* g = gs[k & 1] + 64 * c;
 #pragma unroll
         for (int h16 = 0; h16 < 4; ++h16) {
           float dd[16];
           tc::tmem_ld16(lanes + 16 * h16, dd);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) S[16 * h16 + i] = fmaf(S[16 * h16 + i], g[16 * h16 + i], dd[i]);
+          for (int i = 0; i < 16; ++i)
+            S[16 * h16 + i] = fmaf(S[16 * h16 + i], g[16 * h16 + i], BWD ? dd[i] + l2[16 * h16 + i] : dd[i]);
         }
       }
-      g_arrive(&g_free[n & 1]);
+      g_arrive(&g_free[k & 1]);
       tc::tc_before_sync();
     }
-    if (ST) {
-      float4* dst = reinterpret_cast<float4*>(ST + (unit * D + r) * D + 64 * c);
+    if (io.fin) {
+      float4* dst = reinterpret_cast<float4*>(io.fin + (unit * D + r) * D + 64 * c);
 #pragma unroll
       for (int q = 0; q < 16; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
     }
-  } else if (warp < 12) {
-    // ---- producer: chunk n's W and K^e^T into slot n % 2
-    const int pt = tid - 256;  // 0..127
-    for (int n = 0; n < NC; ++n) {
-      const int slot = n & 1;
-      if (n >= 2) {
-        tc::mbar_wait<false>(&empty[slot], ((n >> 1) - 1) & 1, err, tc::kErrTimeoutMma, &abort_flag);
-        tc::mbar_wait<false>(&g_free[slot], ((n >> 1) - 1) & 1, err, tc::kErrTimeoutMma, &abort_flag);
+  } else if (warp == 8 && lane == 0) {
+    // ---- producer: chunk k's operand images and gamma_C into slot k % 2
+    for (int k = 0; k < NC; ++k) {
+      const int slot = k & 1, n = BWD ? NC - 1 - k : k;
+      if (k >= 2) {
+        tc::mbar_wait<false>(&empty[slot], ((k >> 1) - 1) & 1, err, tc::kErrTimeoutMma, &abort_flag);
+        tc::mbar_wait<false>(&g_free[slot], ((k >> 1) - 1) & 1, err, tc::kErrTimeoutMma, &abort_flag);
       }
       unsigned char* sl = sm + Cf::SLOT + slot * Cf::SLOT_SZ;
       const size_t ch = unit * NC + n;
-      if (pt < 3 && n + kChainAhead < NC) {
-        // pull chunk n + kChainAhead's operands into L2, so that this role's
-        // loads and the state warps' loads of U' find them there
-        const size_t ca = ch + kChainAhead;
-        const float* src = pt == 0 ? p.W : pt == 1 ? p.Ke : p.Up;
-        tc::prefetch_l2(src + ca * C * D, C * D * 4);
+      tc::mbar_expect_tx(&full[slot], 4u * (2 * C * D) + 4u * D);
+      tc::bulk_g2s(sl + Cf::WH, io.b1 + ch * (2 * C * D), 4u * C * D, &full[slot]);
+      tc::bulk_g2s(sl + Cf::KH, io.b2 + ch * (2 * C * D), 4u * C * D, &full[slot]);
+      tc::bulk_g2s(gs[slot], io.gC + ch * D, 4u * D, &full[slot]);
+      if (k + kChainAhead < NC) {
+        // pull the operands kChainAhead chunks ahead into L2, so that the
+        // copies above and the state warps' loads find them there
+        const size_t ca = unit * NC + (BWD ? n - kChainAhead : n + kChainAhead);
+        tc::prefetch_l2(io.b1 + ca * (2 * C * D), 4u * C * D);
+        tc::prefetch_l2(io.b2 + ca * (2 * C * D), 4u * C * D);
+        tc::prefetch_l2(io.ul + ca * C * D, 4u * C * D);
+        if (BWD) tc::prefetch_l2(io.l2t + ca * D * D, 4u * D * D);
       }
-      // W [t][j]: eight channels per group, consecutive threads along a row;
-      // every load of a tile is issued before any of its data is used
-      const float4* w = reinterpret_cast<const float4*>(p.W + ch * C * D);
-      {
-        float4 a[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int e = pt + 128 * i;  // group e: row e / 16, channels 8 (e % 16) ..
-          a[2 * i] = w[2 * e];
-          a[2 * i + 1] = w[2 * e + 1];
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int e = pt + 128 * i, t = e / (D / 8), j = 8 * (e % (D / 8));
-          const float x[8] = {a[2 * i].x, a[2 * i].y, a[2 * i].z, a[2 * i].w,
-                              a[2 * i + 1].x, a[2 * i + 1].y, a[2 * i + 1].z, a[2 * i + 1].w};
-          put_hl8(sl + Cf::WH, sl + Cf::WL, tc::sw128_off(t, j, 64, 2), x);
-        }
-      }
-      // K^e^T [j][t]: thread pt takes channel j = pt, all 64 positions
-      {
-        const float* ke = p.Ke + ch * C * D + pt;
-        float x[C];
-#pragma unroll
-        for (int t = 0; t < C; ++t) x[t] = ke[t * D];
-#pragma unroll
-        for (int t8 = 0; t8 < C; t8 += 8) put_hl8(sl + Cf::KH, sl + Cf::KL, tc::sw128_off(pt, t8, 128, 2), x + t8);
-      }
-      gs[slot][pt] = p.gC[ch * D + pt];
-      tc::fence_proxy_async();
-      g_arrive(&full[slot]);
     }
-  } else if (warp == 12 && lane == 0) {
+  } else if (warp == 9 && lane == 0) {
     // ---- issuer
     const uint32_t ID1 = tc::idesc(128, 64, 1), ID2 = tc::idesc(128, 128, 1);
-    for (int n = 0; n < NC; ++n) {
-      const int slot = n & 1;
-      const uint32_t sl = Cf::SLOT + slot * Cf::SLOT_SZ;
-      tc::mbar_wait<false>(&full[slot], (n >> 1) & 1, err, tc::kErrTimeoutLoad, &abort_flag);
-      tc::mbar_wait<false>(&s_ready, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+    // descriptors of the operand bases; a byte offset o moves a descriptor by
+    // o >> 4 in its start-address field (shared addresses stay below 2^18)
+    const uint64_t dSH = tc::desc_sw128(tc::smem_u32(sm + Cf::SH)), dSL = tc::desc_sw128(tc::smem_u32(sm + Cf::SL));
+    const uint64_t dUH = tc::desc_sw128(tc::smem_u32(sm + Cf::UH)), dUL = tc::desc_sw128(tc::smem_u32(sm + Cf::UL));
+    const uint64_t dSlot = tc::desc_sw128(tc::smem_u32(sm + Cf::SLOT));
+    for (int k = 0; k < NC; ++k) {
+      const int slot = k & 1, n = BWD ? NC - 1 - k : k;
+      const uint64_t ds = dSlot + ((slot * Cf::SLOT_SZ) >> 4);
+      tc::mbar_wait<false>(&full[slot], (k >> 1) & 1, err, tc::kErrTimeoutLoad, &abort_flag);
+      tc::mbar_wait<false>(&s_ready, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
-      const uint32_t a1[3] = {Cf::SH, Cf::SH, Cf::SL}, b1[3] = {sl + Cf::WH, sl + Cf::WL, sl + Cf::WH};
+      {
+        __nv_bfloat16* img = io.img + (unit * NC + n) * (2 * D * D);
+        tc::bulk_s2g(img, sm + Cf::SH, 2u * D * D);
+        tc::bulk_s2g(img + D * D, sm + Cf::SL, 2u * D * D);
+        tc::bulk_commit();
+      }
+      const uint64_t a1[3] = {dSH, dSH, dSL};
+      const uint64_t b1[3] = {ds + (Cf::WH >> 4), ds + (Cf::WL >> 4), ds + (Cf::WH >> 4)};
 #pragma unroll
       for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          tc::mma_bf16_ss(tmem + Cf::X_COL,
-                          tc::desc_sw128(tc::smem_u32(sm + a1[pr] + (ks / 4) * 16384 + (ks % 4) * 32)),
-                          tc::desc_sw128(tc::smem_u32(sm + b1[pr] + (ks / 4) * 8192 + (ks % 4) * 32)), ID1,
-                          (pr | ks) ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + Cf::X_COL, a1[pr] + (((ks / 4) * 16384 + (ks % 4) * 32) >> 4),
+                          b1[pr] + (((ks / 4) * 8192 + (ks % 4) * 32) >> 4), ID1, (pr | ks) ? 1u : 0u);
       tc::mma_commit(&x_done);
-      tc::mbar_wait<false>(&u_ready, n & 1, err, tc::kErrTimeoutMma, &abort_flag);
+      tc::mbar_wait<false>(&u_ready, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
-      const uint32_t a2[3] = {Cf::UH, Cf::UH, Cf::UL}, b2[3] = {sl + Cf::KH, sl + Cf::KL, sl + Cf::KH};
+      const uint64_t a2[3] = {dUH, dUH, dUL};
+      const uint64_t b2[3] = {ds + (Cf::KH >> 4), ds + (Cf::KL >> 4), ds + (Cf::KH >> 4)};
 #pragma unroll
       for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          tc::mma_bf16_ss(tmem + Cf::D_COL, tc::desc_sw128(tc::smem_u32(sm + a2[pr] + ks * 32)),
-                          tc::desc_sw128(tc::smem_u32(sm + b2[pr] + ks * 32)), ID2, (pr | ks) ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + Cf::D_COL, a2[pr] + ((ks * 32) >> 4), b2[pr] + ((ks * 32) >> 4), ID2,
+                          (pr | ks) ? 1u : 0u);
+      tc::bulk_wait_read();  // the state image is read out before the state warps write the next one
       tc::mma_commit(&d_done);
       tc::mma_commit(&empty[slot]);
     }
@@ -701,18 +735,228 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(const flo
   if (warp == 0) tc::tmem_dealloc(tmem, 256);
 }
 
+// ---------------------------------------------------------------------------
+// The backward's chunk-local terms and the reverse chain's operand images, one
+// CTA per chunk, all chunks in parallel.  Reverse mode of the chain
+// (derivation in kd_gdn2.cu's header):
+//   dU = P^T dO + K^e dS^T,   dS <- dS Gamma + dO^T Q+ - dU^T W
+// P^T dO and dO^T Q+ need no state, so they are formed here, transposed on
+// tcgen05 with M = 128 value rows r (dO is exact in bf16; P and Q+ as hi + lo):
+//   columns 0-63:   (P^T dO)^T [r][t]  -> dUi [t][r]
+//   columns 64-191: dO^T Q+   [r][j]  -> L2t [j][r]
+// and K^e [t][j], W^T [j][t] become the reverse chain's bf16 hi, lo images.
+// ---------------------------------------------------------------------------
+struct GBpreCfg {
+  static constexpr uint32_t OT = 0;                      // dO^T [r][i] bf16, 128 rows (16 KB)
+  static constexpr uint32_t PH = 16384, PL = 24576;      // P^T [t][i] hi, lo, 64 rows (8 KB each)
+  static constexpr uint32_t QH = 32768, QL = 49152;      // Q+^T [j][t] hi, lo, 128 rows (16 KB each)
+  static constexpr uint32_t IK = 65536, IW = 98304;      // images: K^e [t][j], W^T [j][t] (hi, lo: 32 KB each)
+  static constexpr uint32_t BYTES = 131072 + 1024;
+};
+
+__global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __restrict__ dO, int H, int T, int NC,
+                                                       GdnWs p, int* __restrict__ err) {
+  using Cf = GBpreCfg;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
+  const size_t ch = blockIdx.x;
+  if (tid == 0) {
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 256);
+  {
+    // loads first (every load of a group in flight together), then the
+    // transposes and hi, lo splits into the operand tiles
+    const float4* pp = reinterpret_cast<const float4*>(p.P + ch * C * C);
+    const float4* qp = reinterpret_cast<const float4*>(p.Qp + ch * C * D);
+    float4 q4[8], p4[4];
+    uint4 o8[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q4[i] = qp[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p4[i] = pp[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // dO rows: eight channels per step
+      const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
+      o8[i] = t < nv ? *reinterpret_cast<const uint4*>(dO + (((size_t)b * T + t0 + t) * H + h) * D + r)
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // dO [t][r] -> dO^T [r][t]
+      const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
+      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&o8[i]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) *reinterpret_cast<__nv_bfloat16*>(sm + Cf::OT + tc::sw128_off(r + c, t, 128, 2)) = v[c];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // P [i][t] -> P^T [t][i]
+      const int e = tid + 256 * i, ii = e / (C / 4), t = 4 * (e % (C / 4));
+      const float xs[4] = {p4[i].x, p4[i].y, p4[i].z, p4[i].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) put_hl(sm + Cf::PH, sm + Cf::PL, tc::sw128_off(t + c, ii, 64, 2), xs[c]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // Q+ [t][j] -> Q+^T [j][t]
+      const int e = tid + 256 * i, t = e / (D / 4), j = 4 * (e % (D / 4));
+      const float xs[4] = {q4[i].x, q4[i].y, q4[i].z, q4[i].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) put_hl(sm + Cf::QH, sm + Cf::QL, tc::sw128_off(j + c, t, 128, 2), xs[c]);
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 0) {
+    const uint32_t ID1 = tc::idesc(128, 64, 1), ID2 = tc::idesc(128, 128, 1);
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t a = tc::desc_sw128(tc::smem_u32(sm + Cf::OT + ks * 32));
+        tc::mma_bf16_ss(tmem, a, tc::desc_sw128(tc::smem_u32(sm + (pr ? Cf::PL : Cf::PH) + ks * 32)), ID1,
+                        (pr | ks) ? 1u : 0u);
+        tc::mma_bf16_ss(tmem + 64, a, tc::desc_sw128(tc::smem_u32(sm + (pr ? Cf::QL : Cf::QH) + ks * 32)), ID2,
+                        (pr | ks) ? 1u : 0u);
+      }
+    tc::mma_commit(&mma_bar);
+  }
+  {
+    // meanwhile, the reverse chain's operand images: K^e [t][j] and W^T [j][t]
+    const float4* kp = reinterpret_cast<const float4*>(p.Ke + ch * C * D);
+    const float4* wp = reinterpret_cast<const float4*>(p.W + ch * C * D);
+    float4 k4[8], w4[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      k4[i] = kp[tid + 256 * i];
+      w4[i] = wp[tid + 256 * i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = tid + 256 * i, t = e / (D / 4), j = 4 * (e % (D / 4));
+      put_hl4(sm + Cf::IK, sm + Cf::IK + 16384, tc::sw128_off(t, j, 64, 2), k4[i]);
+      const float xs[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) put_hl(sm + Cf::IW, sm + Cf::IW + 16384, tc::sw128_off(j + c, t, 128, 2), xs[c]);
+    }
+  }
+  tc::fence_proxy_async();
+  __syncthreads();
+  if (tid == 0) {
+    tc::bulk_s2g(p.Keimg + ch * (2 * C * D), sm + Cf::IK, 4u * C * D);
+    tc::bulk_s2g(p.WTimg + ch * (2 * C * D), sm + Cf::IW, 4u * C * D);
+    tc::bulk_commit();
+  }
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  {
+    // lane r: warps 0-3 take columns 0-95 (the 64 of P^T dO, then j 0-31),
+    // warps 4-7 columns 96-191 (j 32-127)
+    const int r = (warp & 3) * 32 + lane, c0 = (warp >> 2) * 96;
+    const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, c0);
+#pragma unroll
+    for (int c16 = 0; c16 < 6; ++c16) {
+      float v[16];
+      tc::tmem_ld16(lanes + 16 * c16, v);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) {
+        const int col = c0 + 16 * c16 + ii;
+        if (col < 64)
+          p.dUi[(ch * C + col) * D + r] = v[ii];
+        else
+          p.L2t[(ch * D + col - 64) * D + r] = v[ii];
+      }
+    }
+  }
+  if (tid == 0) tc::bulk_wait_read();
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+}
+
+// The chain's saved state images -> fp32 [ch][r][j] = hi + lo, the layout the
+// backward's CUDA-core kernels read; one CTA per chunk, eight channels (one
+// 16-byte swizzle chunk of each part) per step.
+__global__ void __launch_bounds__(256) gdn2_s0_unpack(const __nv_bfloat16* __restrict__ img, float* __restrict__ S0) {
+  const size_t ch = blockIdx.x;
+  const unsigned char* hi = reinterpret_cast<const unsigned char*>(img + ch * 2 * D * D);
+  const unsigned char* lo = hi + 2 * D * D;
+  float* dst = S0 + ch * D * D;
+#pragma unroll 2
+  for (int e = threadIdx.x; e < D * D / 8; e += 256) {
+    const int r = e / (D / 8), j = 8 * (e % (D / 8));
+    const uint32_t off = tc::sw128_off(r, j, 128, 2);
+    const uint4 hv = *reinterpret_cast<const uint4*>(hi + off), lv = *reinterpret_cast<const uint4*>(lo + off);
+    const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&hv);
+    const __nv_bfloat162* lp = reinterpret_cast<const __nv_bfloat162*>(&lv);
+    float o[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 a = __bfloat1622float2(hp[q]), b2 = __bfloat1622float2(lp[q]);
+      o[2 * q] = a.x + b2.x;
+      o[2 * q + 1] = a.y + b2.y;
+    }
+    reinterpret_cast<float4*>(dst + r * D + j)[0] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4*>(dst + r * D + j)[1] = make_float4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 }  // namespace
 
 bool gdn2_tc_supported(const GdnLayout& L) { return L.dtype == 1 && L.dk == D && L.dv == D; }
 
+cudaError_t launch_gdn2_bchain_tc(const GdnArgs& a, const GdnWs& p, int* err, cudaStream_t st) {
+  const GdnLayout& L = a.L;
+  cudaError_t e = cudaFuncSetAttribute(gdn2_bpre_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)GBpreCfg::BYTES);
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "gdn2_bpre_tc");
+  gdn2_bpre_tc<<<(unsigned)L.chunks, 256, GBpreCfg::BYTES, st>>>(static_cast<const __nv_bfloat16*>(a.dO), L.H,
+                                                                 L.T, L.NC, p, err);
+  prof_end(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(gdn2_chain_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GChainCfg::BYTES)) != cudaSuccess)
+    return e;
+  const GChainIO io{a.dST, a.dS0, p.Keimg, p.WTimg, p.gC, p.dUi, p.L2t, p.dU, p.dSimg};
+  prof_begin(st, "gdn2_bchain_tc");
+  gdn2_chain_tc<true><<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(io, L.NC, err);
+  prof_end(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the per-chunk gradient kernels read dS in fp32 [ch][r][j]
+  prof_begin(st, "gdn2_ds_unpack");
+  gdn2_s0_unpack<<<(unsigned)L.chunks, 256, 0, st>>>(p.dSimg, p.dS);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gdn2_s0_unpack(const __nv_bfloat16* img, float* S0, size_t chunks, cudaStream_t st) {
+  prof_begin(st, "gdn2_s0_unpack");
+  gdn2_s0_unpack<<<(unsigned)chunks, 256, 0, st>>>(img, S0);
+  prof_end(st);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gdn2_chain_tc(const GdnArgs& a, int* err, cudaStream_t st) {
   const GdnLayout& L = a.L;
   const GdnWs p = gdn_ws(a.ws, L);
-  cudaError_t e = cudaFuncSetAttribute(gdn2_chain_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(gdn2_chain_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)GChainCfg::BYTES);
   if (e != cudaSuccess) return e;
+  const GChainIO io{a.S0, a.ST, p.Wimg, p.KeTimg, p.gC, p.Up, nullptr, p.U, p.S0img};
   prof_begin(st, "gdn2_chain_tc");
-  gdn2_chain_tc<<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(a.S0, a.ST, L.H, L.NC, p, err);
+  gdn2_chain_tc<false><<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(io, L.NC, err);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -2,6 +2,7 @@
 // and the CUDA kernels.  Not part of the public header.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -218,20 +219,51 @@ struct GdnLayout {
   size_t chunks = 0;
   size_t A = 0, P = 0, W = 0, Up = 0, Ke = 0, Qp = 0, gC = 0, S0 = 0, U = 0, fwd_bytes = 0;
   size_t dU = 0, dS = 0, dE = 0, dT = 0, dP = 0, dQp = 0, dKe = 0, bwd_bytes = 0;
+  // tensor-core path (bf16, dk = dv = 128): the chunk-start states are kept as
+  // bf16 high and low parts in the 128-byte-swizzled K-major image the chain
+  // and the output kernel hold in shared memory ([ch] 32 KB hi + 32 KB lo, in
+  // the forward's workspace, where S0 is not allocated); the backward unpacks
+  // them once into fp32 [ch][r][j] in its own workspace (S0 there)
+  bool tc = false;
+  size_t S0img = 0, S0b = 0;
+  // tensor-core path: the chains' B operands as bf16 hi, lo images (32 KB per
+  // chunk each): W [t][j] and K^e^T [j][t] for the forward chain (written by
+  // the preparation kernel), K^e [t][j] and W^T [j][t] for the backward chain
+  // (written by its pre-chain kernel, in the backward's workspace)
+  size_t Wimg = 0, KeTimg = 0, Keimg = 0, WTimg = 0;
+  // tensor-core backward: the reverse chain's chunk-local terms P^T dO [ch][t][r]
+  // and (dO^T Q+)^T [ch][j][r] (fp32), and its saved dS images (as S0img)
+  size_t dUi = 0, L2t = 0, dSimg = 0;
 };
 struct GdnWs {
   float *A, *P, *W, *Up, *Ke, *Qp, *gC, *S0, *U;
   float *dU, *dS, *dE, *dT, *dP, *dQp, *dKe;
+  __nv_bfloat16* S0img;  // tensor-core path: the chunk-start state images
+  __nv_bfloat16 *Wimg, *KeTimg, *Keimg, *WTimg;  // tensor-core path: the chains' operand images
+  float *dUi, *L2t;                              // tensor-core backward: the chain's chunk-local terms
+  __nv_bfloat16* dSimg;                          // tensor-core backward: the saved dS images
 };
 inline GdnWs gdn_ws(char* base, const GdnLayout& L) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
-  return GdnWs{f(L.A), f(L.P), f(L.W), f(L.Up), f(L.Ke), f(L.Qp), f(L.gC), f(L.S0), f(L.U),
-               nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  return GdnWs{f(L.A), f(L.P), f(L.W), f(L.Up), f(L.Ke), f(L.Qp), f(L.gC), L.tc ? nullptr : f(L.S0), f(L.U),
+               nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+               L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.S0img) : nullptr,
+               L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.Wimg) : nullptr,
+               L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.KeTimg) : nullptr, nullptr, nullptr,
+               nullptr, nullptr, nullptr};
 }
 inline void gdn_bwd_ws(char* base, const GdnLayout& L, GdnWs* p) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
   p->dU = f(L.dU); p->dS = f(L.dS); p->dE = f(L.dE); p->dT = f(L.dT); p->dP = f(L.dP);
   p->dQp = f(L.dQp); p->dKe = f(L.dKe);
+  if (L.tc) {
+    p->S0 = f(L.S0b);
+    p->Keimg = reinterpret_cast<__nv_bfloat16*>(base + L.Keimg);
+    p->WTimg = reinterpret_cast<__nv_bfloat16*>(base + L.WTimg);
+    p->dUi = f(L.dUi);
+    p->L2t = f(L.L2t);
+    p->dSimg = reinterpret_cast<__nv_bfloat16*>(base + L.dSimg);
+  }
 }
 struct GdnArgs {
   const void *q, *k, *v;
@@ -261,6 +293,9 @@ bool gdn2_tc_supported(const GdnLayout& L);
 cudaError_t launch_gdn2_prep_tc(const GdnArgs& a, int* err, cudaStream_t st);
 cudaError_t launch_gdn2_out_tc(const GdnArgs& a, int* err, cudaStream_t st);
 cudaError_t launch_gdn2_chain_tc(const GdnArgs& a, int* err, cudaStream_t st);
+// the backward's pre-chain terms and operand images, and its reverse chain
+cudaError_t launch_gdn2_bchain_tc(const GdnArgs& a, const GdnWs& p, int* err, cudaStream_t st);
+cudaError_t launch_gdn2_s0_unpack(const __nv_bfloat16* img, float* S0, size_t chunks, cudaStream_t st);
 cudaError_t launch_gdn2_bwd(const GdnArgs& a, cudaStream_t st);
 
 // Gated inputs (kd_gate.cu): logf = e^{a_log} log sigma(f~) into a buffer
