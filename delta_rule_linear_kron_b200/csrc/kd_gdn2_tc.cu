@@ -620,19 +620,19 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
 #pragma unroll
           for (int i = 0; i < 16; ++i) u[16 * h16 + i] = BWD ? up[16 * h16 + i] + x[i] : up[16 * h16 + i] - x[i];
         }
+        float ua[32];  // MMA 2's operand: U^T, or -dU^T (the backward subtracts dU^T W)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) io.uout[(ch * C + 32 * c + i) * D + r] = u[i];
-        if (BWD) {  // MMA 2 subtracts dU^T W: its operand is -dU^T
-#pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = -u[i];
-        }
+        for (int i = 0; i < 32; ++i) ua[i] = BWD ? -u[i] : u[i];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          put_hl8(sm + Cf::UH, sm + Cf::UL, tc::sw128_off(r, 32 * c + 8 * q, 128, 2), u + 8 * q);
+          put_hl8(sm + Cf::UH, sm + Cf::UL, tc::sw128_off(r, 32 * c + 8 * q, 128, 2), ua + 8 * q);
+        tc::fence_proxy_async();
+        tc::tc_before_sync();
+        g_arrive(&u_ready);
+        // U (dU) to the workspace while MMA 2 runs
+#pragma unroll
+        for (int i = 0; i < 32; ++i) io.uout[(ch * C + 32 * c + i) * D + r] = u[i];
       }
-      tc::fence_proxy_async();
-      tc::tc_before_sync();
-      g_arrive(&u_ready);
       // the backward's dO^T Q+ term of this thread's state row, loaded while MMA 2 runs
       float l2[BWD ? 64 : 1];
       if (BWD) {
@@ -700,12 +700,6 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
       tc::mbar_wait<false>(&full[slot], (k >> 1) & 1, err, tc::kErrTimeoutLoad, &abort_flag);
       tc::mbar_wait<false>(&s_ready, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
-      {
-        __nv_bfloat16* img = io.img + (unit * NC + n) * (2 * D * D);
-        tc::bulk_s2g(img, sm + Cf::SH, 2u * D * D);
-        tc::bulk_s2g(img + D * D, sm + Cf::SL, 2u * D * D);
-        tc::bulk_commit();
-      }
       const uint64_t a1[3] = {dSH, dSH, dSL};
       const uint64_t b1[3] = {ds + (Cf::WH >> 4), ds + (Cf::WL >> 4), ds + (Cf::WH >> 4)};
 #pragma unroll
@@ -715,6 +709,13 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
           tc::mma_bf16_ss(tmem + Cf::X_COL, a1[pr] + (((ks / 4) * 16384 + (ks % 4) * 32) >> 4),
                           b1[pr] + (((ks / 4) * 8192 + (ks % 4) * 32) >> 4), ID1, (pr | ks) ? 1u : 0u);
       tc::mma_commit(&x_done);
+      {
+        // the chunk's start state image out, while MMA 1 runs
+        __nv_bfloat16* img = io.img + (unit * NC + n) * (2 * D * D);
+        tc::bulk_s2g(img, sm + Cf::SH, 2u * D * D);
+        tc::bulk_s2g(img + D * D, sm + Cf::SL, 2u * D * D);
+        tc::bulk_commit();
+      }
       tc::mbar_wait<false>(&u_ready, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
       const uint64_t a2[3] = {dUH, dUH, dUL};
