@@ -611,7 +611,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& in, int* err, int sms, cudaStream_t st)
   const Layout& L = a.L;
   cudaError_t e;
   if (a.phases & kPhaseLocal) {
-    if ((e = launch_bwd_pre_tc(a, err, st)) != cudaSuccess) return e;
+    if ((e = launch_bwd_pre_tc(a, err, sms, st)) != cudaSuccess) return e;
   }
   if (!(a.phases & kPhaseCarry)) return cudaSuccess;
   if ((e = launch_bwd_chain_tc(a, choose_cluster(L.B * L.H, sms), err, st)) != cudaSuccess) return e;

@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp, int H, int NC,
     const float* __restrict__ wP, const float* __restrict__ wu, float* __restrict__ wdu, float* __restrict__ wMu,
     __nv_bfloat16* __restrict__ wT1, __nv_bfloat16* __restrict__ wPU, __nv_bfloat16* __restrict__ wEK,
-    __nv_bfloat16* __restrict__ wQpT, int* __restrict__ err) {
+    __nv_bfloat16* __restrict__ wQpT, int ahead, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -138,6 +138,18 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
     tc::tma_load_4d(sm + PreCfg::QR, &tm_q, 0, h, t0, b, &ld_bar);
     tc::bulk_g2s(sm + PreCfg::PS, wP + ch * C * C, 16384u, &ld_bar);
     tc::bulk_g2s(sm + PreCfg::US, wu + ch * C, 256u, &ld_bar);
+    const size_t nx = ch + (size_t)ahead;
+    if (nx < gridDim.x) {  // the chunk this SM most likely runs next: its tiles into L2
+      const int nn = static_cast<int>(nx % NC), un = static_cast<int>(nx / NC), tn = nn * C;
+      tc::tma_prefetch_l2_4d(&tm_v, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_v, 64, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_do, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_do, 64, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_k, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_logf, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_q, 0, un % H, tn, un / H);
+      tc::prefetch_l2(wP + nx * C * C, 16384u);
+    }
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 256);
   tc::tc_before_sync();
@@ -584,7 +596,7 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
 
 }  // namespace
 
-cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st) {
+cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st) {
   const Layout& L = a.L;
   CUtensorMap tm_v, tm_do, tm_k, tm_logf, tm_q, tm_kp;
   if (!make_tmap_bthd(&tm_v, a.v, 2, L.B, L.T, L.H, D, 64, true) ||
@@ -601,7 +613,7 @@ cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st) {
       tm_v, tm_do, tm_k, tm_logf, tm_q, tm_kp, L.H, L.NC, ws_ptr<float>(a.fws, L.P),
       ws_ptr<float>(a.fws, L.u), ws_ptr<float>(a.ws, L.du), ws_ptr<float>(a.ws, L.Mu),
       ws_ptr<__nv_bfloat16>(a.ws, L.T1), ws_ptr<__nv_bfloat16>(a.ws, L.PU), ws_ptr<__nv_bfloat16>(a.ws, L.EK),
-      ws_ptr<__nv_bfloat16>(a.ws, L.QpT), err);
+      ws_ptr<__nv_bfloat16>(a.ws, L.QpT), sms, err);
   prof_end(st);
   return cudaGetLastError();
 }

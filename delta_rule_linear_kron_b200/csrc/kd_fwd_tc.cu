@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_logf,
     const __grid_constant__ CUtensorMap tm_out, int H, int NC, const __nv_bfloat16* __restrict__ wS0b,
-    const float* __restrict__ wu, int* __restrict__ unsafe_flags, int* __restrict__ err) {
+    const float* __restrict__ wu, int* __restrict__ unsafe_flags, int ahead, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -84,6 +84,16 @@ __global__ void __launch_bounds__(256, 1) fwd_out_tc(
     tc::tma_load_4d(sm + OutCfg::KR, &tm_k, 0, h, t0, b, &ld_bar);
     tc::tma_load_4d(sm + OutCfg::LG, &tm_logf, 0, h, t0, b, &ld_bar);
     tc::bulk_g2s(sm + OutCfg::U, wu + ch * C, 256u, &ld_bar);
+    const size_t nx = ch + (size_t)ahead;
+    if (nx < gridDim.x) {  // the chunk this SM most likely runs next: its tiles into L2
+      const int nn = static_cast<int>(nx % NC), un = static_cast<int>(nx / NC), tn = nn * C;
+      tc::prefetch_l2(wS0b + nx * D * D, 32768u);
+      tc::tma_prefetch_l2_4d(&tm_v, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_v, 64, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_q, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_k, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_logf, 0, un % H, tn, un / H);
+    }
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
   tc::tc_before_sync();
@@ -576,7 +586,7 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_logf, const __grid_constant__ CUtensorMap tm_kt,
     const __grid_constant__ CUtensorMap tm_ke, int H, int NC, float* __restrict__ wGC, float* __restrict__ wHx,
-    __nv_bfloat16* __restrict__ wVt, int* __restrict__ err) {
+    __nv_bfloat16* __restrict__ wVt, int ahead, int* __restrict__ err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, mma_bar;
@@ -604,6 +614,14 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
       tc::tma_load_4d(sm + CrossCfg::VV + 24576, &tm_v, 64, h, tp, b, &ld_bar);
       tc::tma_load_4d(sm + CrossCfg::KR + 16384, &tm_k, 0, h, tp, b, &ld_bar);
       tc::tma_load_4d(sm + CrossCfg::LG + 32768, &tm_logf, 0, h, tp, b, &ld_bar);
+    }
+    const size_t nx = ch + (size_t)ahead;
+    if (nx < gridDim.x) {  // the chunk this SM most likely runs next: its tiles into L2
+      const int nn = static_cast<int>(nx % NC), un = static_cast<int>(nx / NC), tn = nn * C;
+      tc::tma_prefetch_l2_4d(&tm_v, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_v, 64, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_k, 0, un % H, tn, un / H);
+      tc::tma_prefetch_l2_4d(&tm_logf, 0, un % H, tn, un / H);
     }
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
@@ -787,7 +805,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& in, int* err, int sms, cudaStream_t st)
     prof_begin(st, "fwd_cross_tc");
     fwd_cross_tc<<<(unsigned)L.chunks, 256, CrossCfg::BYTES, st>>>(
         tm_v, tm_k, tm_logf, tm_kt, tm_ke, L.H, L.NC, ws_ptr<float>(a.ws, L.GC), ws_ptr<float>(a.ws, L.Hx),
-        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), err);
+        ws_ptr<__nv_bfloat16>(a.ws, L.Vt), sms, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -811,7 +829,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& in, int* err, int sms, cudaStream_t st)
     prof_begin(st, "fwd_out_tc");
     fwd_out_tc<<<(unsigned)L.chunks, 256, OutCfg::BYTES, st>>>(
         tm_q, tm_k, tm_v, tm_logf, tm_out, L.H, L.NC, (const __nv_bfloat16*)ws_ptr<__nv_bfloat16>(a.ws, L.S0b), wu,
-        flags, err);
+        flags, sms, err);
     prof_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -165,7 +165,7 @@ constexpr int kStageChain = 1, kStageCC = 2, kStageState = 4, kStageIntra = 8, k
 cudaError_t launch_bwd_simt_stages(const BwdArgs& a, int stages, const int* only, cudaStream_t st);
 cudaError_t launch_bwd_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
 // per-chunk tensor-core kernels before / after the reverse chain (kd_bwd_chunk_tc.cu)
-cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, cudaStream_t st);
+cudaError_t launch_bwd_pre_tc(const BwdArgs& a, int* err, int sms, cudaStream_t st);
 cudaError_t launch_bwd_post_tc(const BwdArgs& a, int* err, cudaStream_t st);
 
 // Input prologue (kd_prologue.cu).  N = B*T tokens; rows are [N][H][d].
