@@ -152,13 +152,13 @@ def pass_bytes(name, d=128):
 # kernel lives in and the first 16 hex digits of its sha256 at capture time;
 # a kernel whose source has changed since reports no traffic.
 NCU_TRAFFIC = {
-    "fwd_prep_tc": (450502144, "kd_fwd_tc.cu", "0781816bced3ea5c"),
-    "fwd_cross_tc": (619552512, "kd_fwd_tc.cu", "0781816bced3ea5c"),
-    "fwd_chain_tc": (835102720, "kd_fwd_tc.cu", "0781816bced3ea5c"),
-    "fwd_out_tc": (662231296, "kd_fwd_tc.cu", "0781816bced3ea5c"),
-    "bwd_pre_tc": (513970176, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
-    "bwd_post_tc": (1127943168, "kd_bwd_chunk_tc.cu", "991160f0c6cbc9a1"),
-    "bwd_chain_tc": (585809920, "kd_bwd_tc.cu", "2a91356380c07551"),
+    "fwd_prep_tc": (447366741, "kd_fwd_tc.cu", "c85ecadcbf3d814a"),
+    "fwd_cross_tc": (618602410, "kd_fwd_tc.cu", "c85ecadcbf3d814a"),
+    "fwd_chain_tc": (591054848, "kd_fchain_tc.cu", "cac9ee1a46a36d26"),
+    "fwd_out_tc": (525747114, "kd_fwd_tc.cu", "c85ecadcbf3d814a"),
+    "bwd_pre_tc": (768303189, "kd_bwd_chunk_tc.cu", "5f9a1fca015fc250"),
+    "bwd_chain_tc": (726999552, "kd_bchain_tc.cu", "b514c715eaf3ed73"),
+    "bwd_post_tc": (1127135573, "kd_bwd_chunk_tc.cu", "5f9a1fca015fc250"),
 }
 
 
