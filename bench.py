@@ -181,10 +181,11 @@ def fp32_alu_peak_tflops(sm_mhz):
 
 
 # ---------------------------------------------------------------------------
-# Gated DeltaNet-2 kernels (CUDA cores, fp32 FMA): algorithmic flops per
-# token-head at d_k = d_v = d, C = 64, counting each dense product of the chunk
-# form once (full C x C tiles, as for the Kronecker kernels; exponentials and
-# the O(C^3) inverse not counted).
+# Gated DeltaNet-2 kernels: algorithmic flops per token-head at d_k = d_v = d,
+# C = 64, counting each dense product of the chunk form once (full C x C tiles,
+# as for the Kronecker kernels; exponentials and the O(C^3) inverse not
+# counted).  The "_tc" kernels (bf16, d = 128) run their products on tcgen05
+# and are held against the bf16 tensor peak; the others run on fp32 CUDA cores.
 # ---------------------------------------------------------------------------
 def gdn2_kernel_flops(name, d=128, C=CHUNK):
     dd, cd = 2 * d * d, 2 * C * d
@@ -195,6 +196,12 @@ def gdn2_kernel_flops(name, d=128, C=CHUNK):
         "gdn2_bchain": cd + 3 * dd,             # P^T dO, K^e dS^T; dO^T Q+, dU^T W
         "gdn2_bpost_a": 3 * dd + 5 * cd,        # dQ+, dK^e, dW; dP, dZ, dE; dT (two products)
         "gdn2_bpost_b": 4 * cd,                 # dT K-, dP K-, dT^T E+, dP^T Q+
+        "gdn2_prep_tc": 2 * cd + 2 * cd,
+        "gdn2_chain_tc": 2 * dd,
+        "gdn2_out_tc": dd + cd,
+        "gdn2_bpre_tc": cd + dd,                # P^T dO; dO^T Q+
+        "gdn2_bchain_tc": 2 * dd,               # K^e dS^T; dU^T W
+        "gdn2_bpost_tc": 3 * dd + 9 * cd,       # the products of bpost_a and bpost_b
     }
     return table.get(name)
 
@@ -748,14 +755,18 @@ def main(argv=None):
             if f is None or kms <= 0:
                 continue
             ach = f * B * H * T / (kms / 1e3) / 1e12
-            gkr[name] = dict(bound="alu", achieved=ach, peak=alu_peak, unit="TFLOP/s", frac=ach / alu_peak,
-                             algorithmic_flops_per_launch=f * B * H * T, ms=kms)
+            tcn = name.endswith("_tc")
+            pk = peaks["bf16_tflops"] if tcn else alu_peak
+            gkr[name] = dict(bound="tensor" if tcn else "alu", achieved=ach, peak=pk, unit="TFLOP/s",
+                             frac=ach / pk, algorithmic_flops_per_launch=f * B * H * T, ms=kms)
         top = max(gkr, key=lambda n: gkr[n]["ms"]) if gkr else None
         gdn2 = dict(value=job_throughput(ws_n, B * T, 1, gms), unit="tokens/s", ms_per_step=gms,
-                    step="gdn2_fwd + gdn2_bwd (bf16 q/k/v/dO, fp32 gates, CUDA cores)", per_kernel_ms=gk,
-                    kernel_rooflines=gkr,
-                    roofline=None if top is None else dict(kernel=top, **gkr[top],
-                                                           peak_note="148 SMs x 128 FP32 lanes x 2 x 1965 MHz"),
+                    step="gdn2_fwd + gdn2_bwd (bf16 q/k/v/dO, fp32 gates; chunk products on tcgen05)",
+                    per_kernel_ms=gk, kernel_rooflines=gkr,
+                    roofline=None if top is None else dict(
+                        kernel=top, **gkr[top],
+                        peak_note=("measured bf16 dense (burst)" if gkr[top]["bound"] == "tensor"
+                                   else "148 SMs x 128 FP32 lanes x 2 x 1965 MHz")),
                     decode=gdec)
     clocks = sampler.stop()
 

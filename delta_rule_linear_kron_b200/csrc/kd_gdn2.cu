@@ -46,9 +46,6 @@ constexpr int C = kChunk;
 constexpr int kRows = 16;
 constexpr int kChainThreads = 512;  // threads of a chain CTA
 constexpr int kPostThreads = 512;   // threads of the factorised backward kernel
-// In-chunk |L| below which the backward factors e^{L_t - L_i} = gamma_t / gamma_i
-// (e^{+-60} and their products stay well inside fp32's normal range).
-constexpr float kGdnSafeLog = 60.f;
 
 template <int DK, int DV>
 struct GP {
@@ -1101,8 +1098,6 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   const GdnLayout& L = a.L;
   GdnWs p = gdn_ws(const_cast<char*>(a.fws), L);
   gdn_bwd_ws(a.ws, L, &p);
-  // tensor-core forward: its chunk-start states were kept as bf16 hi, lo images
-  if (L.tc) KD_TRYC(launch_gdn2_s0_unpack(p.S0img, p.S0, L.chunks, st));
   const dim3 gc(L.NC, L.H, L.B), gr(DV / kRows, L.H, L.B);
   if (!L.tc) KD_TRYC(set_smem(gdn2_bchain<DK, DV, Tin>, S::bchain));
   KD_TRYC(set_smem(gdn2_bpost_a<DK, DV, Tin>, S::bpa));
@@ -1117,17 +1112,24 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
     prof_end(st);
     KD_TRYC(cudaGetLastError());
   }
-  prof_begin(st, "gdn2_bpost_a");
-  gdn2_bpost_a<DK, DV, Tin><<<gc, 256, S::bpa, st>>>(static_cast<const Tin*>(a.v), a.w, dO, L.H, L.T, L.NC, p,
-                                                     static_cast<Tin*>(a.dv), a.dw);
-  prof_end(st);
-  KD_TRYC(cudaGetLastError());
-  prof_begin(st, "gdn2_bpost_b");
-  gdn2_bpost_b<DK, DV, Tin><<<gc, kPostThreads, S::bpb, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
-                                                     a.b, a.loga, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
-                                                     static_cast<Tin*>(a.dk), a.db, a.dloga);
-  prof_end(st);
-  KD_TRYC(cudaGetLastError());
+  if (L.tc) {
+    // tensor cores: every gradient of the factorised chunks, and the exact
+    // kernel's inputs for the others (read from the chains' state images)
+    KD_TRYC(launch_gdn2_bpost_tc(a, p, a.err, st));
+  } else {
+    prof_begin(st, "gdn2_bpost_a");
+    gdn2_bpost_a<DK, DV, Tin><<<gc, 256, S::bpa, st>>>(static_cast<const Tin*>(a.v), a.w, dO, L.H, L.T, L.NC, p,
+                                                       static_cast<Tin*>(a.dv), a.dw);
+    prof_end(st);
+    KD_TRYC(cudaGetLastError());
+    prof_begin(st, "gdn2_bpost_b");
+    gdn2_bpost_b<DK, DV, Tin><<<gc, kPostThreads, S::bpb, st>>>(static_cast<const Tin*>(a.q),
+                                                                static_cast<const Tin*>(a.k), a.b, a.loga, L.H, L.T,
+                                                                L.NC, p, static_cast<Tin*>(a.dq),
+                                                                static_cast<Tin*>(a.dk), a.db, a.dloga);
+    prof_end(st);
+    KD_TRYC(cudaGetLastError());
+  }
   prof_begin(st, "gdn2_bpost_exact");
   gdn2_bpost_exact<DK, DV, Tin><<<gc, 256, S::bpe, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
                                                          a.b, a.loga, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),

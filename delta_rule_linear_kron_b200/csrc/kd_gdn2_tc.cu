@@ -886,31 +886,519 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __re
   if (warp == 0) tc::tmem_dealloc(tmem, 256);
 }
 
-// The chain's saved state images -> fp32 [ch][r][j] = hi + lo, the layout the
-// backward's CUDA-core kernels read; one CTA per chunk, eight channels (one
-// 16-byte swizzle chunk of each part) per step.
-__global__ void __launch_bounds__(256) gdn2_s0_unpack(const __nv_bfloat16* __restrict__ img, float* __restrict__ S0) {
+// ---------------------------------------------------------------------------
+// The backward's per-chunk gradients on tcgen05, one CTA per chunk, all chunks
+// in parallel (reverse mode of the chunk form, derivation in kd_gdn2.cu's
+// header).  With S0 and dS the chunk's start state and the gradient of its end
+// state (the chains' saved images), U, dU from the chains and A, U', W from
+// the forward's preparation:
+//   1. dQ+ = dO S0,  dW = -dU S0,  dK^e = U dS,  dP = tril(dO U^T)
+//   2. dZ = A^T dU (-> dv = dZ o w, dw = dZ o v),  dE = A^T dW
+//   3. dT = -tril(dZ U'^T + dE W^T, -1)
+// and, for chunks whose in-chunk |L| stays below kGdnSafeLog (the decay
+// weights factor as gamma_t / gamma_i), the pair sums of dq, dk, db and dloga
+// as three more products with K- = k / gamma, E+ = b o k o gamma, Q+ = q o gamma:
+//   4. X1 = dT K-,  X2 = dP K-,  Y = dT^T E+ + dP^T Q+
+//      de = gamma (dE + X1),  dq = gamma (dQ+ + X2),  dk~ = dK^e e^{Lambda-L} + Y / gamma
+//      dk = de o b + dk~,  db = de o k,  dL = b k de + q dq - k dk~
+//      dloga_t = sum_{t' >= t} dL_t' + sum_t dK^e o K^e + e^Lambda sum_r dS[r] o S0[r]
+// Every product runs transposed, with M = 128 key or value channels in TMEM
+// lanes; the two 64 x 64 results (dP^T, dT^T) take their 64-row operand
+// stacked as [hi; lo] parts over the 128 lanes, and the two halves are summed.
+// Operands are bf16 high and low parts (hi hi + hi lo + lo hi; dO is exact in
+// bf16).  A thread owns key (or value) channel j = lane of its warp's TMEM
+// quarter and positions 32 * (warp / 4) .. + 31, so the dloga suffix sums run
+// down its own registers.  Chunks beyond the factorised range leave dQ+, dK^e,
+// dE, dT, dP and S0, dS (fp32) in the workspace for the exact kernel.
+// ---------------------------------------------------------------------------
+struct GBpostCfg {
+  // step 1
+  static constexpr uint32_t SI = 0;                      // S0 image [r][j] hi, lo (32 KB each)
+  static constexpr uint32_t DI = 65536;                  // dS image, the same
+  static constexpr uint32_t BO = 131072;                 // [dO; dU hi] [t][r], 128 rows (32 KB)
+  static constexpr uint32_t DUL = 163840;                // dU lo [t][r], 64 rows (16 KB)
+  static constexpr uint32_t US = 180224;                 // [U hi; U lo] [t][r], 128 rows (32 KB)
+  // from step 2 on, over U: the decay prefix L fp32 [t][j] (32 KB)
+  static constexpr uint32_t LS = 180224;
+  // step 2, over the state images
+  static constexpr uint32_t AH = 0, AL = 8192;           // A [i][t], 64 rows (8 KB each)
+  static constexpr uint32_t DWH = 16384, DWL = 32768;    // dW [i][j], 64 rows (16 KB each)
+  static constexpr uint32_t UPS = 49152;                 // [U' hi; U' lo] [i][r], 128 rows
+  static constexpr uint32_t WS = 81920;                  // [W hi; W lo] [i][j], 128 rows
+  // step 3, over dO and dU
+  static constexpr uint32_t ZH = 114688, ZL = 131072;    // dZ [t][r], 64 rows
+  static constexpr uint32_t EH = 147456, EL = 163840;    // dE [t][j], 64 rows
+  // step 4, over everything before it but L
+  static constexpr uint32_t KMH = 0, KML = 16384;        // K- [i][j], 64 rows
+  static constexpr uint32_t EPH = 32768, EPL = 49152;    // E+ [t][j]
+  static constexpr uint32_t QPH = 65536, QPL = 81920;    // Q+ [t][j]
+  static constexpr uint32_t TPH = 98304, TPL = 114688;   // [dT; dP] [t][i], 128 rows (16 KB each)
+  static constexpr uint32_t SCT = 131072;                // fp32 [64][65]: the lo halves of dT^T, dP^T
+  static constexpr uint32_t SCP = SCT + 64 * 65 * 4;
+  static constexpr uint32_t DLS = 131072;                // fp32 [64][128]: dL, over the halves once read
+  static constexpr uint32_t BYTES = 212992 + 1024;
+  // TMEM columns: dQ+^T, dW^T (then Y^T), dK^e^T, dP^T, dZ^T, dE^T, dT^T (then X1^T, X2^T)
+  static constexpr uint32_t C_DQ = 0, C_DW = 64, C_Y = 64, C_DK = 128, C_DP = 192, C_DZ = 256, C_DE = 320,
+                            C_DT = 384, C_X = 384;
+};
+
+__device__ __forceinline__ float ld_bf(const unsigned char* p) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+
+__global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const float* __restrict__ bg, const float* __restrict__ wg, const float* __restrict__ loga,
+    const __nv_bfloat16* __restrict__ dO, int H, int T, int NC, GdnWs p, __nv_bfloat16* __restrict__ dq,
+    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, float* __restrict__ db,
+    float* __restrict__ dw, float* __restrict__ dloga, int* __restrict__ err) {
+  using Cf = GBpostCfg;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t ld_bar, w_bar, mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  // per key channel: the first half's prefix, Lambda, and each half's share of
+  // sum dS o S0, of sum dK^e o K^e and of sum dL
+  __shared__ float xpre[D], xlam[D], xst[2][D], xkk[2][D], xdl[D];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
+  const int b = unit / H, h = unit % H;
+  const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = blockIdx.x;
-  const unsigned char* hi = reinterpret_cast<const unsigned char*>(img + ch * 2 * D * D);
-  const unsigned char* lo = hi + 2 * D * D;
-  float* dst = S0 + ch * D * D;
-#pragma unroll 2
-  for (int e = threadIdx.x; e < D * D / 8; e += 256) {
-    const int r = e / (D / 8), j = 8 * (e % (D / 8));
-    const uint32_t off = tc::sw128_off(r, j, 128, 2);
-    const uint4 hv = *reinterpret_cast<const uint4*>(hi + off), lv = *reinterpret_cast<const uint4*>(lo + off);
-    const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&hv);
-    const __nv_bfloat162* lp = reinterpret_cast<const __nv_bfloat162*>(&lv);
-    float o[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 a = __bfloat1622float2(hp[q]), b2 = __bfloat1622float2(lp[q]);
-      o[2 * q] = a.x + b2.x;
-      o[2 * q + 1] = a.y + b2.y;
-    }
-    reinterpret_cast<float4*>(dst + r * D + j)[0] = make_float4(o[0], o[1], o[2], o[3]);
-    reinterpret_cast<float4*>(dst + r * D + j)[1] = make_float4(o[4], o[5], o[6], o[7]);
+  const int j = (warp & 3) * 32 + lane, half = warp >> 2, tb = 32 * half;  // this thread's channel, positions
+  const auto row = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * D; };
+
+  if (tid == 0) {
+    tc::mbar_init(&ld_bar, 1);
+    tc::mbar_init(&w_bar, 1);
+    tc::mbar_init(&mma_bar, 1);
+    tc::mbar_init_fence();
+    abort_flag = 0;
+    tc::mbar_expect_tx(&ld_bar, 8u * D * D);
+    const __nv_bfloat16* s0 = p.S0img + ch * (2 * D * D);
+    const __nv_bfloat16* ds = p.dSimg + ch * (2 * D * D);
+    tc::bulk_g2s(sm + Cf::SI, s0, 2u * D * D, &ld_bar);
+    tc::bulk_g2s(sm + Cf::SI + 2 * D * D, s0 + D * D, 2u * D * D, &ld_bar);
+    tc::bulk_g2s(sm + Cf::DI, ds, 2u * D * D, &ld_bar);
+    tc::bulk_g2s(sm + Cf::DI + 2 * D * D, ds + D * D, 2u * D * D, &ld_bar);
   }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
+
+  // the decay prefix of channel j over this thread's positions, in the same
+  // sequential order as the exact kernel's (so both take the same chunks)
+  float L[32];
+  {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) L[i] = tb + i < nv ? loga[row(tb + i) + j] : 0.f;
+    if (half == 0) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) L[i] = acc = acc + L[i];
+      xpre[j] = acc;
+    }
+  }
+  // step 1's operands: dO exact, dU and U as hi, lo
+  float4 a4[4], u4[8];  // A and U', held for step 2
+  {
+    const float4* dup = reinterpret_cast<const float4*>(p.dU + ch * C * D);
+    const float4* up = reinterpret_cast<const float4*>(p.U + ch * C * D);
+    float4 x[8], y[8];
+    uint4 o8[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = dup[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = up[tid + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
+      o8[i] = t < nv ? *reinterpret_cast<const uint4*>(dO + row(t) + r) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = tid + 256 * i, t = e / (D / 4), r = 4 * (e % (D / 4));
+      const uint32_t o = tc::sw128_off(t, r, 128, 2);
+      put_hl4(sm + Cf::BO + 8192 + o, sm + Cf::DUL + tc::sw128_off(t, r, 64, 2), 0u, x[i]);  // dU hi, lo
+      put_hl4(sm + Cf::US, sm + Cf::US + 8192, o, y[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
+      *reinterpret_cast<uint4*>(sm + Cf::BO + tc::sw128_off(t, r, 128, 2)) = o8[i];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a4[i] = reinterpret_cast<const float4*>(p.A + ch * C * C)[tid + 256 * i];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) u4[i] = reinterpret_cast<const float4*>(p.Up + ch * C * D)[tid + 256 * i];
+  __syncthreads();  // xpre
+  float mx = 0.f;
+  if (half == 1) {
+    float acc = xpre[j];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) L[i] = acc = acc + L[i];
+    xlam[j] = acc;  // padded positions carry loga = 0: L at 63 is Lambda
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(L[i]));
+  const bool exact = __syncthreads_or(!(mx < kGdnSafeLog)) != 0;
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tmem = tmem_slot;
+  tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  const auto sd = [&](uint32_t o) { return tc::smem_u32(sm + o); };
+  if (tid == 0) {
+    tc::tc_after_sync();
+    const uint32_t ID128 = tc::idesc(128, 128, 1) | tc::kMajorA, ID64 = tc::idesc(128, 64, 1) | tc::kMajorA;
+    const uint32_t ID64K = tc::idesc(128, 64, 1);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t kb = (ks / 4) * 16384 + (ks % 4) * 32, kb64 = (ks / 4) * 8192 + (ks % 4) * 32;
+      const uint32_t mn = ks * 2048;
+      // [dQ+^T | (dU S0)^T] = S0^T [dO; dU]^T: hi hi, lo hi, and hi lo on the dU half
+      tc::mma_bf16_ss(tmem + Cf::C_DQ, tc::desc_sw128_mn(sd(Cf::SI + mn), 16384u), tc::desc_sw128(sd(Cf::BO + kb)),
+                      ID128, ks > 0 ? 1u : 0u);
+      tc::mma_bf16_ss(tmem + Cf::C_DQ, tc::desc_sw128_mn(sd(Cf::SI + 32768 + mn), 16384u),
+                      tc::desc_sw128(sd(Cf::BO + kb)), ID128, 1u);
+      tc::mma_bf16_ss(tmem + Cf::C_DW, tc::desc_sw128_mn(sd(Cf::SI + mn), 16384u), tc::desc_sw128(sd(Cf::DUL + kb64)),
+                      ID64, 1u);
+      // dK^e^T = dS^T U^T
+      tc::mma_bf16_ss(tmem + Cf::C_DK, tc::desc_sw128_mn(sd(Cf::DI + mn), 16384u), tc::desc_sw128(sd(Cf::US + kb)),
+                      ID64, ks > 0 ? 1u : 0u);
+      tc::mma_bf16_ss(tmem + Cf::C_DK, tc::desc_sw128_mn(sd(Cf::DI + mn), 16384u),
+                      tc::desc_sw128(sd(Cf::US + 8192 + kb)), ID64, 1u);
+      tc::mma_bf16_ss(tmem + Cf::C_DK, tc::desc_sw128_mn(sd(Cf::DI + 32768 + mn), 16384u),
+                      tc::desc_sw128(sd(Cf::US + kb)), ID64, 1u);
+      // [U hi; U lo] dO^T: lanes 0-63 and 64-127 are the two parts of dP^T
+      tc::mma_bf16_ss(tmem + Cf::C_DP, tc::desc_sw128(sd(Cf::US + kb)), tc::desc_sw128(sd(Cf::BO + kb)), ID64K,
+                      ks > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  {
+    // sum_r dS[r][j] S0[r][j] over this thread's half of the rows, while the MMAs run
+    float st = 0.f;
+#pragma unroll 8
+    for (int r = 64 * half; r < 64 * half + 64; ++r) {
+      const uint32_t o = tc::sw128_off(r, j, 128, 2);
+      st = fmaf(ld_bf(sm + Cf::DI + o) + ld_bf(sm + Cf::DI + 32768 + o),
+                ld_bf(sm + Cf::SI + o) + ld_bf(sm + Cf::SI + 32768 + o), st);
+    }
+    xst[half][j] = st;
+    if (exact) {
+      // the exact kernel reads S0 and dS in fp32 [r][j]
+      float* s0 = p.S0 + ch * D * D;
+      float* ds = p.dS + ch * D * D;
+      for (int e = tid; e < D * D; e += 256) {
+        const int r = e / D, jj = e % D;
+        const uint32_t o = tc::sw128_off(r, jj, 128, 2);
+        s0[e] = ld_bf(sm + Cf::SI + o) + ld_bf(sm + Cf::SI + 32768 + o);
+        ds[e] = ld_bf(sm + Cf::DI + o) + ld_bf(sm + Cf::DI + 32768 + o);
+      }
+    }
+  }
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  __syncthreads();  // the state images and U are read: step 2's operands and L go over them
+  if (tid == 0) {
+    // W's image as [hi; lo] per K block
+    const unsigned char* wi = reinterpret_cast<const unsigned char*>(p.Wimg + ch * (2 * C * D));
+    tc::mbar_expect_tx(&w_bar, 4u * C * D);
+    tc::bulk_g2s(sm + Cf::WS, wi, 8192u, &w_bar);
+    tc::bulk_g2s(sm + Cf::WS + 8192, wi + 16384, 8192u, &w_bar);
+    tc::bulk_g2s(sm + Cf::WS + 16384, wi + 8192, 8192u, &w_bar);
+    tc::bulk_g2s(sm + Cf::WS + 24576, wi + 24576, 8192u, &w_bar);
+  }
+  float* Ls = reinterpret_cast<float*>(sm + Cf::LS);  // [64][128]: L at (t, j)
+#pragma unroll
+  for (int i = 0; i < 32; ++i) Ls[(tb + i) * D + j] = L[i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // A [i][t]
+    const int e = tid + 256 * i, r = e / (C / 4), c = 4 * (e % (C / 4));
+    put_hl4(sm + Cf::AH, sm + Cf::AL, tc::sw128_off(r, c, 64, 2), a4[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {  // [U' hi; U' lo]
+    const int e = tid + 256 * i, t = e / (D / 4), r = 4 * (e % (D / 4));
+    put_hl4(sm + Cf::UPS, sm + Cf::UPS + 8192, tc::sw128_off(t, r, 128, 2), u4[i]);
+  }
+  // dW = -(dU S0) from TMEM into dW [i][j] (MN-major operand of dE^T)
+#pragma unroll 1
+  for (int c8 = 0; c8 < 4; ++c8) {
+    const int c0 = tb + 8 * c8;
+    float x[8];
+    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DW + c0), x);
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) put_hl(sm + Cf::DWH, sm + Cf::DWL, tc::sw128_off(c0 + i, j, 64, 2), -x[i]);
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    // dZ^T = dU^T A, dE^T = dW^T A (A as the MN-major B operand)
+    const uint32_t ID = tc::idesc(128, 64, 1) | tc::kMajorA | tc::kMajorB;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint32_t mn = ks * 2048;
+      const uint64_t ah = tc::desc_sw128_mn(sd(Cf::AH + mn), 8192u), al = tc::desc_sw128_mn(sd(Cf::AL + mn), 8192u);
+      const uint64_t uh = tc::desc_sw128_mn(sd(Cf::BO + 8192 + mn), 16384u);
+      const uint64_t ul = tc::desc_sw128_mn(sd(Cf::DUL + mn), 8192u);
+      const uint64_t wh = tc::desc_sw128_mn(sd(Cf::DWH + mn), 8192u), wl = tc::desc_sw128_mn(sd(Cf::DWL + mn), 8192u);
+      tc::mma_bf16_ss(tmem + Cf::C_DZ, uh, ah, ID, ks > 0 ? 1u : 0u);
+      tc::mma_bf16_ss(tmem + Cf::C_DZ, uh, al, ID, 1u);
+      tc::mma_bf16_ss(tmem + Cf::C_DZ, ul, ah, ID, 1u);
+      tc::mma_bf16_ss(tmem + Cf::C_DE, wh, ah, ID, ks > 0 ? 1u : 0u);
+      tc::mma_bf16_ss(tmem + Cf::C_DE, wh, al, ID, 1u);
+      tc::mma_bf16_ss(tmem + Cf::C_DE, wl, ah, ID, 1u);
+    }
+    tc::mma_commit(&mma_bar);
+  }
+  // the write gates and values at this thread's (t, channel r = j) for dv and
+  // dw, eight positions per step, the next step's loads in flight meanwhile
+  const auto ld_wv = [&](int c0, float (&w8)[8], float (&v8)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool ok = c0 + i < nv;
+      w8[i] = ok ? wg[row(c0 + i) + j] : 0.f;
+      v8[i] = ok ? __bfloat162float(v[row(c0 + i) + j]) : 0.f;
+    }
+  };
+  float wn[8], vn[8];
+  ld_wv(tb, wn, vn);
+  tc::mbar_wait<false>(&mma_bar, 1, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  // dZ^T (lane r) -> dZ [t][r] operand, dv and dw; dE^T (lane j) -> dE [t][j] operand
+#pragma unroll 1
+  for (int c8 = 0; c8 < 4; ++c8) {
+    const int c0 = tb + 8 * c8;
+    float w8[8], v8[8], z[8], e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w8[i] = wn[i];
+      v8[i] = vn[i];
+    }
+    if (c8 < 3) ld_wv(c0 + 8, wn, vn);
+    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DZ + c0), z);
+    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), e);
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int t = c0 + i;
+      const uint32_t o = tc::sw128_off(t, j, 64, 2);
+      put_hl(sm + Cf::ZH, sm + Cf::ZL, o, z[i]);
+      put_hl(sm + Cf::EH, sm + Cf::EL, o, e[i]);
+      if (t < nv) {
+        dv[row(t) + j] = __float2bfloat16_rn(z[i] * w8[i]);
+        dw[row(t) + j] = z[i] * v8[i];
+      }
+    }
+  }
+  tc::fence_proxy_async();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    // [U' hi; U' lo] dZ^T + [W hi; W lo] dE^T, with dZ, dE hi and then lo
+    tc::mbar_wait<false>(&w_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+    const uint32_t ID = tc::idesc(128, 64, 1);
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kb = (ks / 4) * 16384 + (ks % 4) * 32, kb64 = (ks / 4) * 8192 + (ks % 4) * 32;
+        tc::mma_bf16_ss(tmem + Cf::C_DT, tc::desc_sw128(sd(Cf::UPS + kb)),
+                        tc::desc_sw128(sd((pr ? Cf::ZL : Cf::ZH) + kb64)), ID, (pr | ks) ? 1u : 0u);
+        tc::mma_bf16_ss(tmem + Cf::C_DT, tc::desc_sw128(sd(Cf::WS + kb)),
+                        tc::desc_sw128(sd((pr ? Cf::EL : Cf::EH) + kb64)), ID, 1u);
+      }
+    tc::mma_commit(&mma_bar);
+  }
+  // k, b, q at this thread's (t, j), eight positions per step
+  const auto ld_kbq = [&](int c0, float (&k8)[8], float (&b8)[8], float (&q8)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool ok = c0 + i < nv;
+      k8[i] = ok ? __bfloat162float(k[row(c0 + i) + j]) : 0.f;
+      b8[i] = ok ? bg[row(c0 + i) + j] : 0.f;
+      q8[i] = ok ? __bfloat162float(q[row(c0 + i) + j]) : 0.f;
+    }
+  };
+  float kn[8], bn[8], qn[8];
+  if (!exact) ld_kbq(tb, kn, bn, qn);
+  tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
+  tc::tc_after_sync();
+  __syncthreads();  // every operand of steps 2 and 3 is read
+  // dT^T and dP^T: lanes 64-127 (the lo parts) park their halves in shared
+  // memory, lanes 0-63 add them and write the [dT; dP] operand
+  float* sct = reinterpret_cast<float*>(sm + Cf::SCT);
+  float* scp = reinterpret_cast<float*>(sm + Cf::SCP);
+  if ((warp & 3) >= 2) {
+    const int i = j - 64;
+#pragma unroll 1
+    for (int c8 = 0; c8 < 4; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float x[8], y[8];
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + c0), x);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + c0), y);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) {
+        sct[i * 65 + c0 + ii] = x[ii];
+        scp[i * 65 + c0 + ii] = y[ii];
+      }
+    }
+  }
+  if (!exact) {
+    // step 4's operands K-, E+, Q+ [t][j] at this thread's positions
+#pragma unroll 1
+    for (int c8 = 0; c8 < 4; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float k8[8], b8[8], q8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        k8[i] = kn[i];
+        b8[i] = bn[i];
+        q8[i] = qn[i];
+      }
+      if (c8 < 3) ld_kbq(c0 + 8, kn, bn, qn);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t o = tc::sw128_off(c0 + i, j, 64, 2);
+        const float Lt = Ls[(c0 + i) * D + j], gm = __expf(Lt), ig = __expf(-Lt);
+        put_hl(sm + Cf::KMH, sm + Cf::KML, o, k8[i] * ig);
+        put_hl(sm + Cf::EPH, sm + Cf::EPL, o, b8[i] * k8[i] * gm);
+        put_hl(sm + Cf::QPH, sm + Cf::QPL, o, q8[i] * gm);
+      }
+    }
+  }
+  __syncthreads();
+  if ((warp & 3) < 2) {
+    const int i = j;
+#pragma unroll 1
+    for (int c8 = 0; c8 < 4; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float x[8], y[8];
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + c0), x);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + c0), y);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) {
+        const int t = c0 + ii;
+        const float dtv = i < t ? -(x[ii] + sct[i * 65 + t]) : 0.f;
+        const float dpv = i <= t ? y[ii] + scp[i * 65 + t] : 0.f;
+        if (exact) {
+          p.dT[(ch * C + t) * C + i] = dtv;
+          p.dP[(ch * C + t) * C + i] = dpv;
+        } else {
+          put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(t, i, 128, 2), dtv);
+          put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(64 + t, i, 128, 2), dpv);
+        }
+      }
+    }
+  }
+  if (exact) {
+    // dQ+, dK^e and dE [t][j] for the exact kernel
+#pragma unroll 1
+    for (int c8 = 0; c8 < 4; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float x[8], y[8], z[8];
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DQ + c0), x);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DK + c0), y);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), z);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) {
+        const size_t o = (ch * C + c0 + ii) * D + j;
+        p.dQp[o] = x[ii];
+        p.dKe[o] = y[ii];
+        p.dE[o] = z[ii];
+      }
+    }
+  } else {
+    tc::fence_proxy_async();
+    tc::tc_before_sync();
+    __syncthreads();
+    tc::tc_after_sync();
+    if (tid == 0) {
+      // [X1^T | X2^T] = K-^T [dT; dP]^T and Y^T = E+^T dT + Q+^T dP
+      const uint32_t IDX = tc::idesc(128, 128, 1) | tc::kMajorA;
+      const uint32_t IDY = tc::idesc(128, 64, 1) | tc::kMajorA | tc::kMajorB;
+      const uint32_t ops[3][2] = {{0u, 0u}, {0u, 16384u}, {16384u, 0u}};  // (A, B) part offsets: hi hi, hi lo, lo hi
+#pragma unroll
+      for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t mn = ks * 2048, a = ops[pr][0], bo = ops[pr][1];
+          tc::mma_bf16_ss(tmem + Cf::C_X, tc::desc_sw128_mn(sd(Cf::KMH + a + mn), 8192u),
+                          tc::desc_sw128(sd(Cf::TPH + bo + ks * 32)), IDX, (pr | ks) ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + Cf::C_Y, tc::desc_sw128_mn(sd(Cf::EPH + a + mn), 8192u),
+                          tc::desc_sw128_mn(sd(Cf::TPH + bo + mn), 8192u), IDY, (pr | ks) ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + Cf::C_Y, tc::desc_sw128_mn(sd(Cf::QPH + a + mn), 8192u),
+                          tc::desc_sw128_mn(sd(Cf::TPH + 8192 + bo + mn), 8192u), IDY, 1u);
+        }
+      tc::mma_commit(&mma_bar);
+    }
+    ld_kbq(tb, kn, bn, qn);
+    tc::mbar_wait<false>(&mma_bar, 1, err, tc::kErrTimeoutMma, &abort_flag);
+    tc::tc_after_sync();
+    const float lam = xlam[j];
+    float* dLs = reinterpret_cast<float*>(sm + Cf::DLS);  // [64][128]: dL at (t, j)
+    float kpart = 0.f, tot = 0.f;
+#pragma unroll 1
+    for (int c8 = 0; c8 < 4; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float k8[8], b8[8], q8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        k8[i] = kn[i];
+        b8[i] = bn[i];
+        q8[i] = qn[i];
+      }
+      if (c8 < 3) ld_kbq(c0 + 8, kn, bn, qn);
+      float xq[8], xk[8], xe[8], x1[8], x2[8], yy[8];
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DQ + c0), xq);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DK + c0), xk);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), xe);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_X + c0), x1);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_X + 64 + c0), x2);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_Y + c0), yy);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = c0 + i;
+        const float Lt = Ls[t * D + j], gm = __expf(Lt), ke = __expf(lam - Lt), ig = __expf(-Lt);
+        const float dee = gm * (xe[i] + x1[i]);
+        const float dqq = gm * (xq[i] + x2[i]);
+        const float dkk = fmaf(xk[i], ke, yy[i] * ig);
+        kpart = fmaf(xk[i], k8[i] * ke, kpart);
+        const float dl = b8[i] * k8[i] * dee + q8[i] * dqq - k8[i] * dkk;
+        dLs[t * D + j] = dl;
+        tot += dl;
+        if (t < nv) {
+          const size_t g = row(t) + j;
+          dq[g] = __float2bfloat16_rn(dqq);
+          dk[g] = __float2bfloat16_rn(fmaf(dee, b8[i], dkk));
+          db[g] = dee * k8[i];
+        }
+      }
+    }
+    xkk[half][j] = kpart;
+    if (half) xdl[j] = tot;
+    __syncthreads();
+    float acc = xkk[0][j] + xkk[1][j] + (xst[0][j] + xst[1][j]) * __expf(lam) + (half ? 0.f : xdl[j]);
+#pragma unroll 8
+    for (int i = 31; i >= 0; --i) {
+      acc += dLs[(tb + i) * D + j];
+      if (tb + i < nv) dloga[row(tb + i) + j] = acc;
+    }
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
@@ -934,17 +1422,20 @@ cudaError_t launch_gdn2_bchain_tc(const GdnArgs& a, const GdnWs& p, int* err, cu
   prof_begin(st, "gdn2_bchain_tc");
   gdn2_chain_tc<true><<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(io, L.NC, err);
   prof_end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // the per-chunk gradient kernels read dS in fp32 [ch][r][j]
-  prof_begin(st, "gdn2_ds_unpack");
-  gdn2_s0_unpack<<<(unsigned)L.chunks, 256, 0, st>>>(p.dSimg, p.dS);
-  prof_end(st);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gdn2_s0_unpack(const __nv_bfloat16* img, float* S0, size_t chunks, cudaStream_t st) {
-  prof_begin(st, "gdn2_s0_unpack");
-  gdn2_s0_unpack<<<(unsigned)chunks, 256, 0, st>>>(img, S0);
+cudaError_t launch_gdn2_bpost_tc(const GdnArgs& a, const GdnWs& p, int* err, cudaStream_t st) {
+  const GdnLayout& L = a.L;
+  cudaError_t e = cudaFuncSetAttribute(gdn2_bpost_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)GBpostCfg::BYTES);
+  if (e != cudaSuccess) return e;
+  prof_begin(st, "gdn2_bpost_tc");
+  gdn2_bpost_tc<<<(unsigned)L.chunks, 256, GBpostCfg::BYTES, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), a.b, a.w, a.loga, static_cast<const __nv_bfloat16*>(a.dO), L.H, L.T,
+      L.NC, p, static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv),
+      a.db, a.dw, a.dloga, err);
   prof_end(st);
   return cudaGetLastError();
 }

@@ -13,6 +13,11 @@ namespace kd {
 // "기술 상세": the chunk size is fixed at 64 and the chunk's triangular
 // inverse is built by forward substitution).
 constexpr int kChunk = 64;
+// Gated DeltaNet-2 backward: in-chunk |L| below which the per-chunk gradient
+// kernels factor e^{L_t - L_i} = gamma_t / gamma_i (e^{+-60} and their products
+// stay well inside fp32's normal range); the chunks beyond it take the exact
+// kernel.  Both sides decide from the same sequential prefix sum.
+constexpr float kGdnSafeLog = 60.f;
 
 // Scratch slots of the tensor-core backward's exact recomputation (the CTAs
 // of bwd_exact_simt): its per-chunk scratch is sized by this, not by the
@@ -295,7 +300,9 @@ cudaError_t launch_gdn2_out_tc(const GdnArgs& a, int* err, cudaStream_t st);
 cudaError_t launch_gdn2_chain_tc(const GdnArgs& a, int* err, cudaStream_t st);
 // the backward's pre-chain terms and operand images, and its reverse chain
 cudaError_t launch_gdn2_bchain_tc(const GdnArgs& a, const GdnWs& p, int* err, cudaStream_t st);
-cudaError_t launch_gdn2_s0_unpack(const __nv_bfloat16* img, float* S0, size_t chunks, cudaStream_t st);
+// the backward's per-chunk gradients (every chunk's dv, dw; the factorised
+// chunks' dq, dk, db, dloga; the exact kernel's inputs for the others)
+cudaError_t launch_gdn2_bpost_tc(const GdnArgs& a, const GdnWs& p, int* err, cudaStream_t st);
 cudaError_t launch_gdn2_bwd(const GdnArgs& a, cudaStream_t st);
 
 // Gated inputs (kd_gate.cu): logf = e^{a_log} log sigma(f~) into a buffer
