@@ -946,27 +946,31 @@ __device__ __forceinline__ float ld_bf(const unsigned char* p) {
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
 }
 
-__global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
+constexpr int kBpostThreads = 512;
+
+__global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ bg, const float* __restrict__ wg, const float* __restrict__ loga,
     const __nv_bfloat16* __restrict__ dO, int H, int T, int NC, GdnWs p, __nv_bfloat16* __restrict__ dq,
     __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, float* __restrict__ db,
     float* __restrict__ dw, float* __restrict__ dloga, int* __restrict__ err) {
   using Cf = GBpostCfg;
+  constexpr int NT = kBpostThreads, NG = NT / 128;  // NG groups of 16 positions
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ uint64_t ld_bar, w_bar, mma_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  // per key channel: the first half's prefix, Lambda, and each half's share of
-  // sum dS o S0, of sum dK^e o K^e and of sum dL
-  __shared__ float xpre[D], xlam[D], xst[2][D], xkk[2][D], xdl[D];
+  // per key channel: the running prefix, Lambda, sum dS o S0 (per warp, then
+  // total), and each position group's sum of dK^e o K^e and of dL
+  __shared__ float xpre[D], xlam[D], xst[D], xred[NT / 32][D], xkk[NG][D], xdl[NG][D];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % NC, unit = blockIdx.x / NC;
   const int b = unit / H, h = unit % H;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = blockIdx.x;
-  const int j = (warp & 3) * 32 + lane, half = warp >> 2, tb = 32 * half;  // this thread's channel, positions
+  // this thread: channel j (the lane of its warp's TMEM quarter), positions tb .. tb + 15
+  const int j = (warp & 3) * 32 + lane, grp = warp >> 2, tb = 16 * grp;
   const auto row = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * D; };
 
   if (tid == 0) {
@@ -985,62 +989,58 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
 
-  // the decay prefix of channel j over this thread's positions, in the same
-  // sequential order as the exact kernel's (so both take the same chunks)
-  float L[32];
-  {
+  float L[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) L[i] = tb + i < nv ? loga[row(tb + i) + j] : 0.f;
-    if (half == 0) {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) L[i] = acc = acc + L[i];
-      xpre[j] = acc;
-    }
-  }
-  // step 1's operands: dO exact, dU and U as hi, lo
-  float4 a4[4], u4[8];  // A and U', held for step 2
+  for (int i = 0; i < 16; ++i) L[i] = tb + i < nv ? loga[row(tb + i) + j] : 0.f;
+  // step 1's operands: dO exact, dU and U as hi, lo; A and U' held for step 2
+  float4 a4[2], u4[4];
   {
     const float4* dup = reinterpret_cast<const float4*>(p.dU + ch * C * D);
     const float4* up = reinterpret_cast<const float4*>(p.U + ch * C * D);
-    float4 x[8], y[8];
-    uint4 o8[4];
+    float4 x[4], y[4];
+    uint4 o8[2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = dup[tid + 256 * i];
+    for (int i = 0; i < 4; ++i) x[i] = dup[tid + NT * i];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = up[tid + 256 * i];
+    for (int i = 0; i < 4; ++i) y[i] = up[tid + NT * i];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
+    for (int i = 0; i < 2; ++i) {
+      const int e = tid + NT * i, t = e / (D / 8), r = 8 * (e % (D / 8));
       o8[i] = t < nv ? *reinterpret_cast<const uint4*>(dO + row(t) + r) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = tid + 256 * i, t = e / (D / 4), r = 4 * (e % (D / 4));
+    for (int i = 0; i < 4; ++i) {
+      const int e = tid + NT * i, t = e / (D / 4), r = 4 * (e % (D / 4));
       const uint32_t o = tc::sw128_off(t, r, 128, 2);
       put_hl4(sm + Cf::BO + 8192 + o, sm + Cf::DUL + tc::sw128_off(t, r, 64, 2), 0u, x[i]);  // dU hi, lo
       put_hl4(sm + Cf::US, sm + Cf::US + 8192, o, y[i]);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
+    for (int i = 0; i < 2; ++i) {
+      const int e = tid + NT * i, t = e / (D / 8), r = 8 * (e % (D / 8));
       *reinterpret_cast<uint4*>(sm + Cf::BO + tc::sw128_off(t, r, 128, 2)) = o8[i];
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) a4[i] = reinterpret_cast<const float4*>(p.A + ch * C * C)[tid + 256 * i];
+  for (int i = 0; i < 2; ++i) a4[i] = reinterpret_cast<const float4*>(p.A + ch * C * C)[tid + NT * i];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) u4[i] = reinterpret_cast<const float4*>(p.Up + ch * C * D)[tid + 256 * i];
-  __syncthreads();  // xpre
-  float mx = 0.f;
-  if (half == 1) {
-    float acc = xpre[j];
+  for (int i = 0; i < 4; ++i) u4[i] = reinterpret_cast<const float4*>(p.Up + ch * C * D)[tid + NT * i];
+  // the decay prefix of channel j, group after group, in the same sequential
+  // order as the exact kernel's (so both take the same chunks)
+#pragma unroll 1
+  for (int g = 0; g < NG; ++g) {
+    if (grp == g) {
+      float acc = g ? xpre[j] : 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) L[i] = acc = acc + L[i];
-    xlam[j] = acc;  // padded positions carry loga = 0: L at 63 is Lambda
+      for (int i = 0; i < 16; ++i) L[i] = acc = acc + L[i];
+      xpre[j] = acc;
+      if (g == NG - 1) xlam[j] = acc;  // padded positions carry loga = 0: L at 63 is Lambda
+    }
+    __syncthreads();
   }
+  float mx = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(L[i]));
+  for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(L[i]));
   const bool exact = __syncthreads_or(!(mx < kGdnSafeLog)) != 0;
   tc::fence_proxy_async();
   tc::tc_before_sync();
@@ -1078,20 +1078,41 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
     tc::mma_commit(&mma_bar);
   }
   {
-    // sum_r dS[r][j] S0[r][j] over this thread's half of the rows, while the MMAs run
-    float st = 0.f;
-#pragma unroll 8
-    for (int r = 64 * half; r < 64 * half + 64; ++r) {
-      const uint32_t o = tc::sw128_off(r, j, 128, 2);
-      st = fmaf(ld_bf(sm + Cf::DI + o) + ld_bf(sm + Cf::DI + 32768 + o),
-                ld_bf(sm + Cf::SI + o) + ld_bf(sm + Cf::SI + 32768 + o), st);
+    // sum_r dS[r][j] S0[r][j] while the MMAs run: a thread takes eight
+    // channels (one 16-byte swizzle chunk of each part) of four rows; the two
+    // row groups of a warp are added by a shuffle, the warps in order
+    const int jg = lane & 15, rg = 2 * warp + (lane >> 4);
+    float acc8[8] = {};
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const uint32_t o = tc::sw128_off(4 * rg + rr, 8 * jg, 128, 2);
+      const uint4 sh = *reinterpret_cast<const uint4*>(sm + Cf::SI + o);
+      const uint4 sl = *reinterpret_cast<const uint4*>(sm + Cf::SI + 32768 + o);
+      const uint4 dh = *reinterpret_cast<const uint4*>(sm + Cf::DI + o);
+      const uint4 dl = *reinterpret_cast<const uint4*>(sm + Cf::DI + 32768 + o);
+      const __nv_bfloat162* a0 = reinterpret_cast<const __nv_bfloat162*>(&sh);
+      const __nv_bfloat162* a1 = reinterpret_cast<const __nv_bfloat162*>(&sl);
+      const __nv_bfloat162* b0 = reinterpret_cast<const __nv_bfloat162*>(&dh);
+      const __nv_bfloat162* b1 = reinterpret_cast<const __nv_bfloat162*>(&dl);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float2 s2 = __bfloat1622float2(a0[c]), s2l = __bfloat1622float2(a1[c]);
+        const float2 d2 = __bfloat1622float2(b0[c]), d2l = __bfloat1622float2(b1[c]);
+        acc8[2 * c] = fmaf(d2.x + d2l.x, s2.x + s2l.x, acc8[2 * c]);
+        acc8[2 * c + 1] = fmaf(d2.y + d2l.y, s2.y + s2l.y, acc8[2 * c + 1]);
+      }
     }
-    xst[half][j] = st;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc8[c] += __shfl_xor_sync(0xffffffffu, acc8[c], 16);
+    if (lane < 16) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) xred[warp][8 * jg + c] = acc8[c];
+    }
     if (exact) {
       // the exact kernel reads S0 and dS in fp32 [r][j]
       float* s0 = p.S0 + ch * D * D;
       float* ds = p.dS + ch * D * D;
-      for (int e = tid; e < D * D; e += 256) {
+      for (int e = tid; e < D * D; e += NT) {
         const int r = e / D, jj = e % D;
         const uint32_t o = tc::sw128_off(r, jj, 128, 2);
         s0[e] = ld_bf(sm + Cf::SI + o) + ld_bf(sm + Cf::SI + 32768 + o);
@@ -1111,22 +1132,28 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
     tc::bulk_g2s(sm + Cf::WS + 16384, wi + 8192, 8192u, &w_bar);
     tc::bulk_g2s(sm + Cf::WS + 24576, wi + 24576, 8192u, &w_bar);
   }
+  if (tid < D) {
+    float st = 0.f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) st += xred[w][tid];
+    xst[tid] = st;
+  }
   float* Ls = reinterpret_cast<float*>(sm + Cf::LS);  // [64][128]: L at (t, j)
 #pragma unroll
-  for (int i = 0; i < 32; ++i) Ls[(tb + i) * D + j] = L[i];
+  for (int i = 0; i < 16; ++i) Ls[(tb + i) * D + j] = L[i];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {  // A [i][t]
-    const int e = tid + 256 * i, r = e / (C / 4), c = 4 * (e % (C / 4));
+  for (int i = 0; i < 2; ++i) {  // A [i][t]
+    const int e = tid + NT * i, r = e / (C / 4), c = 4 * (e % (C / 4));
     put_hl4(sm + Cf::AH, sm + Cf::AL, tc::sw128_off(r, c, 64, 2), a4[i]);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {  // [U' hi; U' lo]
-    const int e = tid + 256 * i, t = e / (D / 4), r = 4 * (e % (D / 4));
+  for (int i = 0; i < 4; ++i) {  // [U' hi; U' lo]
+    const int e = tid + NT * i, t = e / (D / 4), r = 4 * (e % (D / 4));
     put_hl4(sm + Cf::UPS, sm + Cf::UPS + 8192, tc::sw128_off(t, r, 128, 2), u4[i]);
   }
   // dW = -(dU S0) from TMEM into dW [i][j] (MN-major operand of dE^T)
 #pragma unroll 1
-  for (int c8 = 0; c8 < 4; ++c8) {
+  for (int c8 = 0; c8 < 2; ++c8) {
     const int c0 = tb + 8 * c8;
     float x[8];
     tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DW + c0), x);
@@ -1157,43 +1184,31 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
     }
     tc::mma_commit(&mma_bar);
   }
-  // the write gates and values at this thread's (t, channel r = j) for dv and
-  // dw, eight positions per step, the next step's loads in flight meanwhile
-  const auto ld_wv = [&](int c0, float (&w8)[8], float (&v8)[8]) {
+  // the write gates and values at this thread's (t, channel r = j) for dv and dw
+  float w16[16], v16[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool ok = c0 + i < nv;
-      w8[i] = ok ? wg[row(c0 + i) + j] : 0.f;
-      v8[i] = ok ? __bfloat162float(v[row(c0 + i) + j]) : 0.f;
-    }
-  };
-  float wn[8], vn[8];
-  ld_wv(tb, wn, vn);
+  for (int i = 0; i < 16; ++i) {
+    const bool ok = tb + i < nv;
+    w16[i] = ok ? wg[row(tb + i) + j] : 0.f;
+    v16[i] = ok ? __bfloat162float(v[row(tb + i) + j]) : 0.f;
+  }
   tc::mbar_wait<false>(&mma_bar, 1, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
   // dZ^T (lane r) -> dZ [t][r] operand, dv and dw; dE^T (lane j) -> dE [t][j] operand
-#pragma unroll 1
-  for (int c8 = 0; c8 < 4; ++c8) {
-    const int c0 = tb + 8 * c8;
-    float w8[8], v8[8], z[8], e[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      w8[i] = wn[i];
-      v8[i] = vn[i];
-    }
-    if (c8 < 3) ld_wv(c0 + 8, wn, vn);
-    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DZ + c0), z);
-    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), e);
+  {
+    float z[16], e[16];
+    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DZ + tb), z);
+    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + tb), e);
     tc::tmem_ld_wait();
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int t = c0 + i;
+    for (int i = 0; i < 16; ++i) {
+      const int t = tb + i;
       const uint32_t o = tc::sw128_off(t, j, 64, 2);
       put_hl(sm + Cf::ZH, sm + Cf::ZL, o, z[i]);
       put_hl(sm + Cf::EH, sm + Cf::EL, o, e[i]);
       if (t < nv) {
-        dv[row(t) + j] = __float2bfloat16_rn(z[i] * w8[i]);
-        dw[row(t) + j] = z[i] * v8[i];
+        dv[row(t) + j] = __float2bfloat16_rn(z[i] * w16[i]);
+        dw[row(t) + j] = z[i] * v16[i];
       }
     }
   }
@@ -1238,24 +1253,20 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
   float* scp = reinterpret_cast<float*>(sm + Cf::SCP);
   if ((warp & 3) >= 2) {
     const int i = j - 64;
-#pragma unroll 1
-    for (int c8 = 0; c8 < 4; ++c8) {
-      const int c0 = tb + 8 * c8;
-      float x[8], y[8];
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + c0), x);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + c0), y);
-      tc::tmem_ld_wait();
+    float x[16], y[16];
+    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + tb), x);
+    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + tb), y);
+    tc::tmem_ld_wait();
 #pragma unroll
-      for (int ii = 0; ii < 8; ++ii) {
-        sct[i * 65 + c0 + ii] = x[ii];
-        scp[i * 65 + c0 + ii] = y[ii];
-      }
+    for (int ii = 0; ii < 16; ++ii) {
+      sct[i * 65 + tb + ii] = x[ii];
+      scp[i * 65 + tb + ii] = y[ii];
     }
   }
   if (!exact) {
     // step 4's operands K-, E+, Q+ [t][j] at this thread's positions
 #pragma unroll 1
-    for (int c8 = 0; c8 < 4; ++c8) {
+    for (int c8 = 0; c8 < 2; ++c8) {
       const int c0 = tb + 8 * c8;
       float k8[8], b8[8], q8[8];
 #pragma unroll
@@ -1264,7 +1275,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
         b8[i] = bn[i];
         q8[i] = qn[i];
       }
-      if (c8 < 3) ld_kbq(c0 + 8, kn, bn, qn);
+      if (c8 == 0) ld_kbq(c0 + 8, kn, bn, qn);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t o = tc::sw128_off(c0 + i, j, 64, 2);
@@ -1278,32 +1289,28 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
   __syncthreads();
   if ((warp & 3) < 2) {
     const int i = j;
-#pragma unroll 1
-    for (int c8 = 0; c8 < 4; ++c8) {
-      const int c0 = tb + 8 * c8;
-      float x[8], y[8];
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + c0), x);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + c0), y);
-      tc::tmem_ld_wait();
+    float x[16], y[16];
+    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + tb), x);
+    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + tb), y);
+    tc::tmem_ld_wait();
 #pragma unroll
-      for (int ii = 0; ii < 8; ++ii) {
-        const int t = c0 + ii;
-        const float dtv = i < t ? -(x[ii] + sct[i * 65 + t]) : 0.f;
-        const float dpv = i <= t ? y[ii] + scp[i * 65 + t] : 0.f;
-        if (exact) {
-          p.dT[(ch * C + t) * C + i] = dtv;
-          p.dP[(ch * C + t) * C + i] = dpv;
-        } else {
-          put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(t, i, 128, 2), dtv);
-          put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(64 + t, i, 128, 2), dpv);
-        }
+    for (int ii = 0; ii < 16; ++ii) {
+      const int t = tb + ii;
+      const float dtv = i < t ? -(x[ii] + sct[i * 65 + t]) : 0.f;
+      const float dpv = i <= t ? y[ii] + scp[i * 65 + t] : 0.f;
+      if (exact) {
+        p.dT[(ch * C + t) * C + i] = dtv;
+        p.dP[(ch * C + t) * C + i] = dpv;
+      } else {
+        put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(t, i, 128, 2), dtv);
+        put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(64 + t, i, 128, 2), dpv);
       }
     }
   }
   if (exact) {
     // dQ+, dK^e and dE [t][j] for the exact kernel
 #pragma unroll 1
-    for (int c8 = 0; c8 < 4; ++c8) {
+    for (int c8 = 0; c8 < 2; ++c8) {
       const int c0 = tb + 8 * c8;
       float x[8], y[8], z[8];
       tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DQ + c0), x);
@@ -1349,7 +1356,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
     float* dLs = reinterpret_cast<float*>(sm + Cf::DLS);  // [64][128]: dL at (t, j)
     float kpart = 0.f, tot = 0.f;
 #pragma unroll 1
-    for (int c8 = 0; c8 < 4; ++c8) {
+    for (int c8 = 0; c8 < 2; ++c8) {
       const int c0 = tb + 8 * c8;
       float k8[8], b8[8], q8[8];
 #pragma unroll
@@ -1358,21 +1365,30 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
         b8[i] = bn[i];
         q8[i] = qn[i];
       }
-      if (c8 < 3) ld_kbq(c0 + 8, kn, bn, qn);
-      float xq[8], xk[8], xe[8], x1[8], x2[8], yy[8];
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DQ + c0), xq);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DK + c0), xk);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), xe);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_X + c0), x1);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_X + 64 + c0), x2);
-      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_Y + c0), yy);
-      tc::tmem_ld_wait();
+      if (c8 == 0) ld_kbq(c0 + 8, kn, bn, qn);
+      float se[8], sq[8], xk[8], yy[8];
+      {
+        float a8[8], b8x[8];
+        tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), a8);
+        tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_X + c0), b8x);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) se[i] = a8[i] + b8x[i];  // dE + X1
+        tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DQ + c0), a8);
+        tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_X + 64 + c0), b8x);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sq[i] = a8[i] + b8x[i];  // dQ+ + X2
+        tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DK + c0), xk);
+        tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_Y + c0), yy);
+        tc::tmem_ld_wait();
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int t = c0 + i;
         const float Lt = Ls[t * D + j], gm = __expf(Lt), ke = __expf(lam - Lt), ig = __expf(-Lt);
-        const float dee = gm * (xe[i] + x1[i]);
-        const float dqq = gm * (xq[i] + x2[i]);
+        const float dee = gm * se[i];
+        const float dqq = gm * sq[i];
         const float dkk = fmaf(xk[i], ke, yy[i] * ig);
         kpart = fmaf(xk[i], k8[i] * ke, kpart);
         const float dl = b8[i] * k8[i] * dee + q8[i] * dqq - k8[i] * dkk;
@@ -1386,12 +1402,14 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpost_tc(
         }
       }
     }
-    xkk[half][j] = kpart;
-    if (half) xdl[j] = tot;
+    xkk[grp][j] = kpart;
+    xdl[grp][j] = tot;
     __syncthreads();
-    float acc = xkk[0][j] + xkk[1][j] + (xst[0][j] + xst[1][j]) * __expf(lam) + (half ? 0.f : xdl[j]);
-#pragma unroll 8
-    for (int i = 31; i >= 0; --i) {
+    float acc = xst[j] * __expf(lam);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) acc += xkk[g][j] + (g > grp ? xdl[g][j] : 0.f);
+#pragma unroll 4
+    for (int i = 15; i >= 0; --i) {
       acc += dLs[(tb + i) * D + j];
       if (tb + i < nv) dloga[row(tb + i) + j] = acc;
     }
@@ -1431,7 +1449,7 @@ cudaError_t launch_gdn2_bpost_tc(const GdnArgs& a, const GdnWs& p, int* err, cud
                                        (int)GBpostCfg::BYTES);
   if (e != cudaSuccess) return e;
   prof_begin(st, "gdn2_bpost_tc");
-  gdn2_bpost_tc<<<(unsigned)L.chunks, 256, GBpostCfg::BYTES, st>>>(
+  gdn2_bpost_tc<<<(unsigned)L.chunks, kBpostThreads, GBpostCfg::BYTES, st>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
       static_cast<const __nv_bfloat16*>(a.v), a.b, a.w, a.loga, static_cast<const __nv_bfloat16*>(a.dO), L.H, L.T,
       L.NC, p, static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv),
