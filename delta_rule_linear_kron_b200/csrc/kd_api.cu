@@ -147,19 +147,19 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
   const size_t C = kd::kChunk;
   size_t off = 0;
   auto take = [&](size_t floats) { size_t o = off; off = align256(off + floats * 4); return o; };
+  L->tc = dtype == KD_BF16 && dk == 128 && dv == 128;
   L->A = take(chunks * C * C);
   L->P = take(chunks * C * C);
-  L->W = take(chunks * C * dk);
   L->Up = take(chunks * C * dv);
-  L->Ke = take(chunks * C * dk);
   L->Qp = take(chunks * C * dk);
   L->gC = take(chunks * dk);
-  L->tc = dtype == KD_BF16 && dk == 128 && dv == 128;
   if (L->tc) {
     L->S0img = take(chunks * (size_t)dv * dk);  // bf16 hi + lo: the bytes of one fp32 tile
     L->Wimg = take(chunks * C * dk);
-    L->KeTimg = take(chunks * C * dk);
+    L->Kimg = take(chunks * C * dk);
   } else {
+    L->W = take(chunks * C * dk);
+    L->Ke = take(chunks * C * dk);
     L->S0 = take(chunks * (size_t)dv * dk);
   }
   L->U = take(chunks * C * dv);
@@ -174,8 +174,6 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
   L->dKe = take(chunks * C * dk);
   if (L->tc) {
     L->S0b = take(chunks * (size_t)dv * dk);
-    L->Keimg = take(chunks * C * dk);
-    L->WTimg = take(chunks * C * dk);
     L->dUi = take(chunks * C * dv);
     L->L2t = take(chunks * (size_t)dk * dv);
     L->dSimg = take(chunks * (size_t)dv * dk);

@@ -16,11 +16,13 @@
 //      substitution, then block rows), in fp32.
 //   3. W^T = E+^T A^T and U'^T = Z^T A^T on tcgen05 (bf16 high and low parts of
 //      both operands: hi hi + hi lo + lo hi, so the products keep about 16
-//      significant bits of each factor), M = 128 channels, N = 64 positions.
+//      significant bits of each factor), M = 128 channels, N = 64 positions;
+//      E+^T and Z^T are the MN-major views of E+ [i][j] and Z [i][r].
 // Chunks whose in-chunk |L| reaches 60 (where k / gamma could overflow) take T
 // and P with per-element weights e^{L_t - L_i} <= 1 on CUDA cores instead of
-// step 1.  The outputs are those of the CUDA-core kernel (kd_gdn2.cu), in the
-// same layouts, so the chain, output and backward kernels read them unchanged.
+// step 1.  Its outputs: A, P, Q+, U' and e^Lambda in fp32 (the CUDA-core
+// kernel's layouts), and W and K^e as bf16 hi, lo images [t][j] for the two
+// chains (the operand tiles as the chains' shared memory holds them).
 #include "kd_common.cuh"
 #include "kd_kernels.h"
 #include "kd_tc.cuh"
@@ -38,7 +40,7 @@ constexpr int kChainAhead = 3;
 
 struct GPrepCfg {
   static constexpr uint32_t AKQ = 0;        // [E+; Q+] bf16 hi, lo (2 K blocks x 128 rows each, 32 KB); then
-                                            // the bf16 operands E+^T hi, lo and Z^T hi, lo (16 KB each)
+                                            // [E+; Z] for step 3 (Z = w o v over Q+)
   static constexpr uint32_t BKM = 65536;    // K- bf16 hi, lo (2 K blocks x 64 rows each, 16 KB); then A hi, lo
   static constexpr uint32_t QR = 98304;     // q bf16 [64][128] (TMA)
   static constexpr uint32_t KR = 114688;    // k bf16 [64][128] (TMA)
@@ -50,9 +52,9 @@ struct GPrepCfg {
   static constexpr uint32_t SMALL = TB + 3 * 16 * 17 * 4;  // prefix exchange [128], Lambda [128]
   static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
   static constexpr uint32_t LOAD_BYTES = 3 * 16384 + 32768;
-  // the bf16 operands of step 3
-  static constexpr uint32_t EH = 0, EL = 16384, ZH = 32768, ZL = 49152, AH = 65536, AL = 73728;
-  // the forward chain's operand images, staged once step 3 is done (32 KB each)
+  // A (the B operand of step 3), hi and lo
+  static constexpr uint32_t AH = 65536, AL = 73728;
+  // the chains' operand images W [t][j] and K^e [t][j], staged once step 3 is done (32 KB each)
   static constexpr uint32_t IW = 0, IK = 32768;
 };
 
@@ -141,7 +143,6 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
       put_hl(sm + Cf::AKQ, sm + Cf::AKQ + 32768, tc::sw128_off(64 + t, j, 128, 2), qp);
       put_hl(sm + Cf::BKM, sm + Cf::BKM + 16384, tc::sw128_off(t, j, 64, 2), kk * ig);
       p.Qp[(ch * C + t) * D + j] = qp;
-      p.Ke[(ch * C + t) * D + j] = kk * expf(lj - L);
     }
   }
   const bool is_unsafe = __syncthreads_or(!(mx < kGdnTcSafeLog)) != 0;
@@ -246,67 +247,54 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
   }
   for (int e = tid; e < C * C; e += 256) p.A[ch * C * C + e] = Xs[(e / C) * 65 + (e % C)];
 
-  // ---- the bf16 operands of step 3, over the operands of step 1 (the
-  // MMA that read them has completed): E+ is read back before any is
-  // overwritten
+  // ---- the bf16 operands of step 3: E+ stays where step 1 read it (rows
+  // 0-63 of the [E+; Q+] tile, its MN-major view is E+^T); Z = w o v goes over
+  // Q+ in rows 64-127, and A into the K- tile (that MMA has completed)
   float wv[32];  // the write gates of this thread's positions, loads in flight together
 #pragma unroll
   for (int i = 0; i < 32; ++i) wv[i] = 32 * half + i < nv ? wg[row(32 * half + i) + j] : 0.f;
-  float ev[32];  // E+ (its factors are at most |b k|, so every chunk has it)
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t o = tc::sw128_off(32 * half + i, j, 128, 2);
-    ev[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::AKQ + o)) +
-            __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::AKQ + 32768 + o));
+  for (int i0 = 0; i0 < 32; ++i0) {
+    const int i = 32 * half + i0;
+    const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::VR + (i * D + j) * 2));
+    put_hl(sm + Cf::AKQ, sm + Cf::AKQ + 32768, tc::sw128_off(64 + i, j, 128, 2), wv[i0] * vv);  // Z [i][r = j]
   }
-  __syncthreads();
-  {
-    unsigned char* eh = sm + Cf::EH;
-    unsigned char* el = sm + Cf::EL;
-    unsigned char* zh = sm + Cf::ZH;
-    unsigned char* zl = sm + Cf::ZL;
-#pragma unroll
-    for (int i0 = 0; i0 < 32; ++i0) {
-      const int i = 32 * half + i0;
-      put_hl(eh, el, tc::sw128_off(j, i, 128, 2), ev[i0]);
-      const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::VR + (i * D + j) * 2));
-      put_hl(zh, zl, tc::sw128_off(j, i, 128, 2), wv[i0] * vv);  // Z^T row r = j
-    }
-    for (int e = tid; e < C * C; e += 256) {
-      const int t = e / C, i = e % C;
-      put_hl(sm + Cf::AH, sm + Cf::AL, tc::sw128_off(t, i, 64, 2), Xs[t * 65 + i]);
-    }
+  for (int e = tid; e < C * C; e += 256) {
+    const int t = e / C, i = e % C;
+    put_hl(sm + Cf::AH, sm + Cf::AL, tc::sw128_off(t, i, 64, 2), Xs[t * 65 + i]);
   }
   tc::fence_proxy_async();
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
   if (tid == 0) {
-    // TMEM columns 0-63: W^T = E+^T A^T; columns 64-127: U'^T = Z^T A^T
-    const uint32_t IDB = tc::idesc(128, 64, 1);
-    const uint32_t ops[3][2] = {{Cf::EH, Cf::AH}, {Cf::EH, Cf::AL}, {Cf::EL, Cf::AH}};
-    const uint32_t zops[3][2] = {{Cf::ZH, Cf::AH}, {Cf::ZH, Cf::AL}, {Cf::ZL, Cf::AH}};
+    // TMEM columns 0-63: W^T = E+^T A^T; columns 64-127: U'^T = Z^T A^T (E+^T and
+    // Z^T as the MN-major views of E+ [i][j] and Z [i][r])
+    const uint32_t IDB = tc::idesc(128, 64, 1) | tc::kMajorA;
+    const uint32_t ops[3][2] = {{0u, Cf::AH}, {0u, Cf::AL}, {32768u, Cf::AH}};  // hi hi, hi lo, lo hi
 #pragma unroll
     for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + ops[pr][0] + ks * 32)),
-                        tc::desc_sw128(tc::smem_u32(sm + ops[pr][1] + ks * 32)), IDB, (pr | ks) ? 1u : 0u);
-        tc::mma_bf16_ss(tmem + 64, tc::desc_sw128(tc::smem_u32(sm + zops[pr][0] + ks * 32)),
-                        tc::desc_sw128(tc::smem_u32(sm + zops[pr][1] + ks * 32)), IDB, (pr | ks) ? 1u : 0u);
+        const uint64_t bd = tc::desc_sw128(tc::smem_u32(sm + ops[pr][1] + ks * 32));
+        tc::mma_bf16_ss(tmem, tc::desc_sw128_mn(tc::smem_u32(sm + Cf::AKQ + ops[pr][0] + ks * 2048), 16384u), bd,
+                        IDB, (pr | ks) ? 1u : 0u);
+        tc::mma_bf16_ss(tmem + 64,
+                        tc::desc_sw128_mn(tc::smem_u32(sm + Cf::AKQ + ops[pr][0] + 8192 + ks * 2048), 16384u), bd,
+                        IDB, (pr | ks) ? 1u : 0u);
       }
     tc::mma_commit(&mma_bar);
   }
   tc::mbar_wait<false>(&mma_bar, is_unsafe ? 0 : 1, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
   {
-    // warps 0-3: lane j of W^T -> W[t][j] and the forward chain's image of W
-    // ([t][j], bf16 hi, lo); warps 4-7: lane r of U'^T -> U'[t][r], then the
-    // chain's image of K^e^T ([j][t], bf16 hi, lo) for channel j = r.  The
-    // operand tiles of steps 1 and 3 are free (their MMAs have completed).
+    // warps 0-3: lane j of W^T -> the chains' image of W ([t][j], bf16 hi, lo);
+    // warps 4-7: lane r of U'^T -> U'[t][r], then the chains' image of K^e
+    // ([t][j], bf16 hi, lo) for channel j = r.  The operand tiles of steps 1
+    // and 3 are free (their MMAs have completed).
     const int lr = (warp & 3) * 32 + lane;
     const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, warp < 4 ? 0 : 64);
-    float* dst = (warp < 4 ? p.W : p.Up) + ch * C * D + lr;
+    float* up = p.Up + ch * C * D + lr;
 #pragma unroll
     for (int c16 = 0; c16 < 4; ++c16) {
       float v[16];
@@ -315,8 +303,10 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
 #pragma unroll
       for (int ii = 0; ii < 16; ++ii) {
         const int t = 16 * c16 + ii;
-        dst[t * D] = v[ii];
-        if (warp < 4) put_hl(sm + Cf::IW, sm + Cf::IW + 16384, tc::sw128_off(t, lr, 64, 2), v[ii]);
+        if (warp < 4)
+          put_hl(sm + Cf::IW, sm + Cf::IW + 16384, tc::sw128_off(t, lr, 64, 2), v[ii]);
+        else
+          up[t * D] = v[ii];
       }
     }
     if (warp >= 4) {
@@ -324,7 +314,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
 #pragma unroll 8
       for (int t = 0; t < C; ++t) {
         const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::KR + (t * D + lr) * 2));
-        put_hl(sm + Cf::IK, sm + Cf::IK + 16384, tc::sw128_off(lr, t, 128, 2), kk * expf(lj - Ls[t * D + lr]));
+        put_hl(sm + Cf::IK, sm + Cf::IK + 16384, tc::sw128_off(t, lr, 64, 2), kk * expf(lj - Ls[t * D + lr]));
       }
     }
   }
@@ -333,7 +323,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
   __syncthreads();
   if (tid == 0) {
     tc::bulk_s2g(p.Wimg + ch * (2 * C * D), sm + Cf::IW, 4u * C * D);
-    tc::bulk_s2g(p.KeTimg + ch * (2 * C * D), sm + Cf::IK, 4u * C * D);
+    tc::bulk_s2g(p.Kimg + ch * (2 * C * D), sm + Cf::IK, 4u * C * D);
     tc::bulk_commit();
     tc::bulk_wait_read();
   }
@@ -504,8 +494,8 @@ struct GChainCfg {
   static constexpr uint32_t UH = 65536, UL = 81920;    // U^T [r][t] hi, lo: 128 rows
   static constexpr uint32_t SLOT = 98304;              // 2 slots of 64 KB:
   static constexpr uint32_t SLOT_SZ = 65536;
-  static constexpr uint32_t WH = 0, WL = 16384;        //   W [t][j] hi, lo: 2 K blocks x 64 rows
-  static constexpr uint32_t KH = 32768, KL = 49152;    //   K^e^T [j][t] hi, lo: 128 rows
+  static constexpr uint32_t WH = 0, WL = 16384;        //   MMA 1's B [t][j] hi, lo: 2 K blocks x 64 rows
+  static constexpr uint32_t KH = 32768, KL = 49152;    //   MMA 2's B [t][j] hi, lo, read MN-major
   static constexpr uint32_t BYTES = SLOT + 2 * SLOT_SZ + 1024;
   static constexpr int THREADS = 320;
   static constexpr uint32_t X_COL = 0, D_COL = 64;     // TMEM: X^T (64 columns), S update (128 columns)
@@ -537,7 +527,7 @@ struct GChainIO {
   const float* init;   // S0 (forward) or dS_T (backward) [B][H][dv][dk]; nullptr: zero
   float* fin;          // S_T or dS0; nullptr: not written
   const __nv_bfloat16* b1;  // MMA 1's B operand image [ch] ([t][j] hi, lo): W (forward) or K^e (backward)
-  const __nv_bfloat16* b2;  // MMA 2's B operand image [ch] ([j][t] hi, lo): K^e^T (forward) or W^T (backward)
+  const __nv_bfloat16* b2;  // MMA 2's B operand image [ch] ([t][j] hi, lo): K^e (forward) or W (backward)
   const float* gC;     // gamma_C [ch][j]
   const float* ul;     // [ch][t][r]: U' (forward) or P^T dO (backward)
   const float* l2t;    // backward: (dO^T Q+)^T [ch][j][r], added to the state update
@@ -688,12 +678,13 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
     }
   } else if (warp == 9 && lane == 0) {
     // ---- issuer
-    const uint32_t ID1 = tc::idesc(128, 64, 1), ID2 = tc::idesc(128, 128, 1);
+    const uint32_t ID1 = tc::idesc(128, 64, 1), ID2 = tc::idesc(128, 128, 1) | tc::kMajorB;
     // descriptors of the operand bases; a byte offset o moves a descriptor by
     // o >> 4 in its start-address field (shared addresses stay below 2^18)
     const uint64_t dSH = tc::desc_sw128(tc::smem_u32(sm + Cf::SH)), dSL = tc::desc_sw128(tc::smem_u32(sm + Cf::SL));
     const uint64_t dUH = tc::desc_sw128(tc::smem_u32(sm + Cf::UH)), dUL = tc::desc_sw128(tc::smem_u32(sm + Cf::UL));
     const uint64_t dSlot = tc::desc_sw128(tc::smem_u32(sm + Cf::SLOT));
+    const uint64_t dSlotMN = tc::desc_sw128_mn(tc::smem_u32(sm + Cf::SLOT), 8192u);
     for (int k = 0; k < NC; ++k) {
       const int slot = k & 1, n = BWD ? NC - 1 - k : k;
       const uint64_t ds = dSlot + ((slot * Cf::SLOT_SZ) >> 4);
@@ -718,13 +709,15 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
       }
       tc::mbar_wait<false>(&u_ready, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
       tc::tc_after_sync();
+      // B [t][j] MN-major: a K step of 16 positions is 16 rows (2048 bytes)
+      const uint64_t dm = dSlotMN + ((slot * Cf::SLOT_SZ) >> 4);
       const uint64_t a2[3] = {dUH, dUH, dUL};
-      const uint64_t b2[3] = {ds + (Cf::KH >> 4), ds + (Cf::KL >> 4), ds + (Cf::KH >> 4)};
+      const uint64_t b2[3] = {dm + (Cf::KH >> 4), dm + (Cf::KL >> 4), dm + (Cf::KH >> 4)};
 #pragma unroll
       for (int pr = 0; pr < 3; ++pr)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          tc::mma_bf16_ss(tmem + Cf::D_COL, a2[pr] + ((ks * 32) >> 4), b2[pr] + ((ks * 32) >> 4), ID2,
+          tc::mma_bf16_ss(tmem + Cf::D_COL, a2[pr] + ((ks * 32) >> 4), b2[pr] + ((ks * 2048) >> 4), ID2,
                           (pr | ks) ? 1u : 0u);
       tc::bulk_wait_read();  // the state image is read out before the state warps write the next one
       tc::mma_commit(&d_done);
@@ -737,22 +730,21 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
 }
 
 // ---------------------------------------------------------------------------
-// The backward's chunk-local terms and the reverse chain's operand images, one
-// CTA per chunk, all chunks in parallel.  Reverse mode of the chain
-// (derivation in kd_gdn2.cu's header):
+// The backward's chunk-local terms, one CTA per chunk, all chunks in parallel.
+// Reverse mode of the chain (derivation in kd_gdn2.cu's header):
 //   dU = P^T dO + K^e dS^T,   dS <- dS Gamma + dO^T Q+ - dU^T W
 // P^T dO and dO^T Q+ need no state, so they are formed here, transposed on
-// tcgen05 with M = 128 value rows r (dO is exact in bf16; P and Q+ as hi + lo):
+// tcgen05 with M = 128 value rows r (dO is exact in bf16; P and Q+ as hi + lo),
+// every operand read MN-major from its natural layout:
 //   columns 0-63:   (P^T dO)^T [r][t]  -> dUi [t][r]
 //   columns 64-191: dO^T Q+   [r][j]  -> L2t [j][r]
-// and K^e [t][j], W^T [j][t] become the reverse chain's bf16 hi, lo images.
+// (The reverse chain's operand images are the forward's: K^e and W [t][j].)
 // ---------------------------------------------------------------------------
 struct GBpreCfg {
-  static constexpr uint32_t OT = 0;                      // dO^T [r][i] bf16, 128 rows (16 KB)
-  static constexpr uint32_t PH = 16384, PL = 24576;      // P^T [t][i] hi, lo, 64 rows (8 KB each)
-  static constexpr uint32_t QH = 32768, QL = 49152;      // Q+^T [j][t] hi, lo, 128 rows (16 KB each)
-  static constexpr uint32_t IK = 65536, IW = 98304;      // images: K^e [t][j], W^T [j][t] (hi, lo: 32 KB each)
-  static constexpr uint32_t BYTES = 131072 + 1024;
+  static constexpr uint32_t DO = 0;                      // dO [t][r] bf16, 64 rows (16 KB)
+  static constexpr uint32_t PH = 16384, PL = 24576;      // P [i][t] hi, lo, 64 rows (8 KB each)
+  static constexpr uint32_t QH = 32768, QL = 49152;      // Q+ [t][j] hi, lo, 64 rows (16 KB each)
+  static constexpr uint32_t BYTES = 65536 + 1024;
 };
 
 __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __restrict__ dO, int H, int T, int NC,
@@ -775,8 +767,8 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __re
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 256);
   {
-    // loads first (every load of a group in flight together), then the
-    // transposes and hi, lo splits into the operand tiles
+    // loads first (every load of a group in flight together), then the hi, lo
+    // splits into the operand tiles, all in their natural layouts
     const float4* pp = reinterpret_cast<const float4*>(p.P + ch * C * C);
     const float4* qp = reinterpret_cast<const float4*>(p.Qp + ch * C * D);
     float4 q4[8], p4[4];
@@ -792,25 +784,19 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __re
                      : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {  // dO [t][r] -> dO^T [r][t]
+    for (int i = 0; i < 4; ++i) {
       const int e = tid + 256 * i, t = e / (D / 8), r = 8 * (e % (D / 8));
-      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&o8[i]);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) *reinterpret_cast<__nv_bfloat16*>(sm + Cf::OT + tc::sw128_off(r + c, t, 128, 2)) = v[c];
+      *reinterpret_cast<uint4*>(sm + Cf::DO + tc::sw128_off(t, r, 64, 2)) = o8[i];
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {  // P [i][t] -> P^T [t][i]
+    for (int i = 0; i < 4; ++i) {  // P [i][t]
       const int e = tid + 256 * i, ii = e / (C / 4), t = 4 * (e % (C / 4));
-      const float xs[4] = {p4[i].x, p4[i].y, p4[i].z, p4[i].w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) put_hl(sm + Cf::PH, sm + Cf::PL, tc::sw128_off(t + c, ii, 64, 2), xs[c]);
+      put_hl4(sm + Cf::PH, sm + Cf::PL, tc::sw128_off(ii, t, 64, 2), p4[i]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // Q+ [t][j] -> Q+^T [j][t]
+    for (int i = 0; i < 8; ++i) {  // Q+ [t][j]
       const int e = tid + 256 * i, t = e / (D / 4), j = 4 * (e % (D / 4));
-      const float xs[4] = {q4[i].x, q4[i].y, q4[i].z, q4[i].w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) put_hl(sm + Cf::QH, sm + Cf::QL, tc::sw128_off(j + c, t, 128, 2), xs[c]);
+      put_hl4(sm + Cf::QH, sm + Cf::QL, tc::sw128_off(t, j, 64, 2), q4[i]);
     }
   }
   tc::fence_proxy_async();
@@ -819,44 +805,21 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __re
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   if (tid == 0) {
-    const uint32_t ID1 = tc::idesc(128, 64, 1), ID2 = tc::idesc(128, 128, 1);
+    // A = dO^T (MN-major view of dO [t][r]); B = P^T, Q+^T (MN-major views of P, Q+)
+    const uint32_t ID1 = tc::idesc(128, 64, 1) | tc::kMajorA | tc::kMajorB;
+    const uint32_t ID2 = tc::idesc(128, 128, 1) | tc::kMajorA | tc::kMajorB;
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t a = tc::desc_sw128(tc::smem_u32(sm + Cf::OT + ks * 32));
-        tc::mma_bf16_ss(tmem, a, tc::desc_sw128(tc::smem_u32(sm + (pr ? Cf::PL : Cf::PH) + ks * 32)), ID1,
+        const uint32_t mn = ks * 2048;
+        const uint64_t a = tc::desc_sw128_mn(tc::smem_u32(sm + Cf::DO + mn), 8192u);
+        tc::mma_bf16_ss(tmem, a, tc::desc_sw128_mn(tc::smem_u32(sm + (pr ? Cf::PL : Cf::PH) + mn), 8192u), ID1,
                         (pr | ks) ? 1u : 0u);
-        tc::mma_bf16_ss(tmem + 64, a, tc::desc_sw128(tc::smem_u32(sm + (pr ? Cf::QL : Cf::QH) + ks * 32)), ID2,
+        tc::mma_bf16_ss(tmem + 64, a, tc::desc_sw128_mn(tc::smem_u32(sm + (pr ? Cf::QL : Cf::QH) + mn), 8192u), ID2,
                         (pr | ks) ? 1u : 0u);
       }
     tc::mma_commit(&mma_bar);
-  }
-  {
-    // meanwhile, the reverse chain's operand images: K^e [t][j] and W^T [j][t]
-    const float4* kp = reinterpret_cast<const float4*>(p.Ke + ch * C * D);
-    const float4* wp = reinterpret_cast<const float4*>(p.W + ch * C * D);
-    float4 k4[8], w4[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      k4[i] = kp[tid + 256 * i];
-      w4[i] = wp[tid + 256 * i];
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = tid + 256 * i, t = e / (D / 4), j = 4 * (e % (D / 4));
-      put_hl4(sm + Cf::IK, sm + Cf::IK + 16384, tc::sw128_off(t, j, 64, 2), k4[i]);
-      const float xs[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) put_hl(sm + Cf::IW, sm + Cf::IW + 16384, tc::sw128_off(j + c, t, 128, 2), xs[c]);
-    }
-  }
-  tc::fence_proxy_async();
-  __syncthreads();
-  if (tid == 0) {
-    tc::bulk_s2g(p.Keimg + ch * (2 * C * D), sm + Cf::IK, 4u * C * D);
-    tc::bulk_s2g(p.WTimg + ch * (2 * C * D), sm + Cf::IW, 4u * C * D);
-    tc::bulk_commit();
   }
   tc::mbar_wait<false>(&mma_bar, 0, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
@@ -880,7 +843,6 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __re
       }
     }
   }
-  if (tid == 0) tc::bulk_wait_read();
   tc::tc_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 256);
@@ -1436,7 +1398,7 @@ cudaError_t launch_gdn2_bchain_tc(const GdnArgs& a, const GdnWs& p, int* err, cu
   if ((e = cudaFuncSetAttribute(gdn2_chain_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)GChainCfg::BYTES)) != cudaSuccess)
     return e;
-  const GChainIO io{a.dST, a.dS0, p.Keimg, p.WTimg, p.gC, p.dUi, p.L2t, p.dU, p.dSimg};
+  const GChainIO io{a.dST, a.dS0, p.Kimg, p.Wimg, p.gC, p.dUi, p.L2t, p.dU, p.dSimg};
   prof_begin(st, "gdn2_bchain_tc");
   gdn2_chain_tc<true><<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(io, L.NC, err);
   prof_end(st);
@@ -1464,7 +1426,7 @@ cudaError_t launch_gdn2_chain_tc(const GdnArgs& a, int* err, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gdn2_chain_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)GChainCfg::BYTES);
   if (e != cudaSuccess) return e;
-  const GChainIO io{a.S0, a.ST, p.Wimg, p.KeTimg, p.gC, p.Up, nullptr, p.U, p.S0img};
+  const GChainIO io{a.S0, a.ST, p.Wimg, p.Kimg, p.gC, p.Up, nullptr, p.U, p.S0img};
   prof_begin(st, "gdn2_chain_tc");
   gdn2_chain_tc<false><<<(unsigned)(L.B * L.H), GChainCfg::THREADS, GChainCfg::BYTES, st>>>(io, L.NC, err);
   prof_end(st);

@@ -227,15 +227,15 @@ struct GdnLayout {
   // tensor-core path (bf16, dk = dv = 128): the chunk-start states are kept as
   // bf16 high and low parts in the 128-byte-swizzled K-major image the chain
   // and the output kernel hold in shared memory ([ch] 32 KB hi + 32 KB lo, in
-  // the forward's workspace, where S0 is not allocated); the backward unpacks
-  // them once into fp32 [ch][r][j] in its own workspace (S0 there)
+  // the forward's workspace, where S0 is not allocated), and so are the
+  // backward's dS; its gradient kernel reads both images and writes fp32 S0
+  // (S0b) and dS only for the chunks the exact kernel takes
   bool tc = false;
   size_t S0img = 0, S0b = 0;
   // tensor-core path: the chains' B operands as bf16 hi, lo images (32 KB per
-  // chunk each): W [t][j] and K^e^T [j][t] for the forward chain (written by
-  // the preparation kernel), K^e [t][j] and W^T [j][t] for the backward chain
-  // (written by its pre-chain kernel, in the backward's workspace)
-  size_t Wimg = 0, KeTimg = 0, Keimg = 0, WTimg = 0;
+  // chunk each), W [t][j] and K^e [t][j], written by the preparation kernel
+  // and read by both chains; W and K^e are not kept in fp32 there
+  size_t Wimg = 0, Kimg = 0;
   // tensor-core backward: the reverse chain's chunk-local terms P^T dO [ch][t][r]
   // and (dO^T Q+)^T [ch][j][r] (fp32), and its saved dS images (as S0img)
   size_t dUi = 0, L2t = 0, dSimg = 0;
@@ -244,17 +244,18 @@ struct GdnWs {
   float *A, *P, *W, *Up, *Ke, *Qp, *gC, *S0, *U;
   float *dU, *dS, *dE, *dT, *dP, *dQp, *dKe;
   __nv_bfloat16* S0img;  // tensor-core path: the chunk-start state images
-  __nv_bfloat16 *Wimg, *KeTimg, *Keimg, *WTimg;  // tensor-core path: the chains' operand images
+  __nv_bfloat16 *Wimg, *Kimg;                    // tensor-core path: the chains' operand images
   float *dUi, *L2t;                              // tensor-core backward: the chain's chunk-local terms
   __nv_bfloat16* dSimg;                          // tensor-core backward: the saved dS images
 };
 inline GdnWs gdn_ws(char* base, const GdnLayout& L) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
-  return GdnWs{f(L.A), f(L.P), f(L.W), f(L.Up), f(L.Ke), f(L.Qp), f(L.gC), L.tc ? nullptr : f(L.S0), f(L.U),
+  return GdnWs{f(L.A), f(L.P), L.tc ? nullptr : f(L.W), f(L.Up), L.tc ? nullptr : f(L.Ke), f(L.Qp), f(L.gC),
+               L.tc ? nullptr : f(L.S0), f(L.U),
                nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.S0img) : nullptr,
                L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.Wimg) : nullptr,
-               L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.KeTimg) : nullptr, nullptr, nullptr,
+               L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.Kimg) : nullptr,
                nullptr, nullptr, nullptr};
 }
 inline void gdn_bwd_ws(char* base, const GdnLayout& L, GdnWs* p) {
@@ -263,8 +264,6 @@ inline void gdn_bwd_ws(char* base, const GdnLayout& L, GdnWs* p) {
   p->dQp = f(L.dQp); p->dKe = f(L.dKe);
   if (L.tc) {
     p->S0 = f(L.S0b);
-    p->Keimg = reinterpret_cast<__nv_bfloat16*>(base + L.Keimg);
-    p->WTimg = reinterpret_cast<__nv_bfloat16*>(base + L.WTimg);
     p->dUi = f(L.dUi);
     p->L2t = f(L.L2t);
     p->dSimg = reinterpret_cast<__nv_bfloat16*>(base + L.dSimg);
