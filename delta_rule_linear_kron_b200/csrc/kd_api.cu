@@ -177,6 +177,7 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
     L->dUi = take(chunks * C * dv);
     L->L2t = take(chunks * (size_t)dk * dv);
     L->dSimg = take(chunks * (size_t)dv * dk);
+    L->xflag = take((chunks + 3) / 4);
   }
   L->bwd_bytes = off;
   return KD_OK;

@@ -787,7 +787,8 @@ __global__ void __launch_bounds__(256) gdn2_bpost_exact(const Tin* __restrict__ 
                                                     const float* __restrict__ bg, const float* __restrict__ loga,
                                                     int H, int T, int NC, GdnWs p,
                                                     Tin* __restrict__ dq, Tin* __restrict__ dk,
-                                                    float* __restrict__ db, float* __restrict__ dloga) {
+                                                    float* __restrict__ db, float* __restrict__ dloga,
+                                                    const unsigned char* __restrict__ xflag) {
   using G = GP<DK, DV>;
   constexpr int TPJ = 256 / DK;     // threads sharing one key channel
   extern __shared__ float gsm[];
@@ -803,6 +804,8 @@ __global__ void __launch_bounds__(256) gdn2_bpost_exact(const Tin* __restrict__ 
   const int n = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int t0 = n * C, nv = min(C, T - t0);
   const size_t ch = ((size_t)bb * H + h) * NC + n;
+  // the tensor-core gradient kernel flags the chunks it leaves to this one
+  if (xflag && !xflag[ch]) return;
   // the decay prefix first: chunks inside the safe range leave at once
   float mx = 0.f;
   if (tid < DK) {
@@ -813,7 +816,7 @@ __global__ void __launch_bounds__(256) gdn2_bpost_exact(const Tin* __restrict__ 
       mx = fmaxf(mx, fabsf(acc));
     }
   }
-  if (!__syncthreads_or(!(mx < kGdnSafeLog))) return;  // the factorised kernel took this chunk
+  if (!__syncthreads_or(!(mx < kGdnSafeLog)) && !xflag) return;  // the factorised kernel took this chunk
   for (int e = tid; e < C * DK; e += 256) {
     const int t = e / DK, j = e % DK;
     const bool ok = t < nv;
@@ -1133,7 +1136,7 @@ cudaError_t gdn2_bwd_t(const GdnArgs& a, cudaStream_t st) {
   prof_begin(st, "gdn2_bpost_exact");
   gdn2_bpost_exact<DK, DV, Tin><<<gc, 256, S::bpe, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
                                                          a.b, a.loga, L.H, L.T, L.NC, p, static_cast<Tin*>(a.dq),
-                                                         static_cast<Tin*>(a.dk), a.db, a.dloga);
+                                                         static_cast<Tin*>(a.dk), a.db, a.dloga, p.xflag);
   prof_end(st);
   return cudaGetLastError();
 }

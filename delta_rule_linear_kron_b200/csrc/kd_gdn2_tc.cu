@@ -1004,6 +1004,7 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
 #pragma unroll
   for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(L[i]));
   const bool exact = __syncthreads_or(!(mx < kGdnSafeLog)) != 0;
+  if (tid == 0) p.xflag[ch] = exact ? 1 : 0;
   tc::fence_proxy_async();
   tc::tc_before_sync();
   __syncthreads();

@@ -239,6 +239,8 @@ struct GdnLayout {
   // tensor-core backward: the reverse chain's chunk-local terms P^T dO [ch][t][r]
   // and (dO^T Q+)^T [ch][j][r] (fp32), and its saved dS images (as S0img)
   size_t dUi = 0, L2t = 0, dSimg = 0;
+  // tensor-core backward: one byte per chunk, set where the exact kernel takes the chunk
+  size_t xflag = 0;
 };
 struct GdnWs {
   float *A, *P, *W, *Up, *Ke, *Qp, *gC, *S0, *U;
@@ -247,6 +249,7 @@ struct GdnWs {
   __nv_bfloat16 *Wimg, *Kimg;                    // tensor-core path: the chains' operand images
   float *dUi, *L2t;                              // tensor-core backward: the chain's chunk-local terms
   __nv_bfloat16* dSimg;                          // tensor-core backward: the saved dS images
+  unsigned char* xflag;                          // tensor-core backward: the exact kernel's chunks
 };
 inline GdnWs gdn_ws(char* base, const GdnLayout& L) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
@@ -256,7 +259,7 @@ inline GdnWs gdn_ws(char* base, const GdnLayout& L) {
                L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.S0img) : nullptr,
                L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.Wimg) : nullptr,
                L.tc ? reinterpret_cast<__nv_bfloat16*>(base + L.Kimg) : nullptr,
-               nullptr, nullptr, nullptr};
+               nullptr, nullptr, nullptr, nullptr};
 }
 inline void gdn_bwd_ws(char* base, const GdnLayout& L, GdnWs* p) {
   auto f = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
@@ -267,6 +270,7 @@ inline void gdn_bwd_ws(char* base, const GdnLayout& L, GdnWs* p) {
     p->dUi = f(L.dUi);
     p->L2t = f(L.L2t);
     p->dSimg = reinterpret_cast<__nv_bfloat16*>(base + L.dSimg);
+    p->xflag = reinterpret_cast<unsigned char*>(base + L.xflag);
   }
 }
 struct GdnArgs {
