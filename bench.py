@@ -771,14 +771,13 @@ def main(argv=None):
     clocks = sampler.stop()
 
     # ---- end to end through the public API with pinned host buffers -----
-    e2e = None
-    if not args.no_e2e:
+    def end_to_end(host_in, step_fn):
         # Every step copies its inputs from pinned host memory and reads its
         # results back inside the timed region.  Step s+1's inputs travel on a
         # copy stream into the other of two device buffers while step s
         # computes; a buffer is refilled only after the step that read it ended.
-        pinned = {n: t.pin_memory() for n, t in host.items()}
-        staged = [{n: torch.empty_like(t, device=dev) for n, t in host.items()} for _ in range(2)]
+        pinned = {n: t.pin_memory() for n, t in host_in.items()}
+        staged = [{n: torch.empty_like(t, device=dev) for n, t in host_in.items()} for _ in range(2)]
         out_h = torch.empty((B, T, H, dv), dtype=bf).pin_memory()
         dS0_h = torch.empty((B, H, dv, dk), dtype=f32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in pinned.values())
@@ -805,19 +804,50 @@ def main(argv=None):
             if si + 1 < args.e2e_steps:
                 upload(1 - slot, si >= 1)
             stream.wait_event(loaded[slot])
-            o, ST, g = step(staged[slot])
+            o, dS0 = step_fn(staged[slot])
             consumed[slot].record(stream)
             out_h.copy_(o, non_blocking=True)
-            dS0_h.copy_(g["dS0"], non_blocking=True)
+            dS0_h.copy_(dS0, non_blocking=True)
         x1.record(stream)
         torch.cuda.synchronize()
         barrier()
         xms = max_over_ranks(x0.elapsed_time(x1), ws_n, dev)
-        e2e = dict(value=job_throughput(ws_n, B * T, args.e2e_steps, xms), unit="tokens/s",
-                   h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=xms / args.e2e_steps,
-                   h2d_gbs=h2d * args.e2e_steps / (xms / 1e3) / 1e9,
-                   pipelining="next step's H2D on a copy stream overlaps this step's compute; D2H after it")
         del staged
+        return dict(value=job_throughput(ws_n, B * T, args.e2e_steps, xms), unit="tokens/s",
+                    h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=xms / args.e2e_steps,
+                    h2d_gbs=h2d * args.e2e_steps / (xms / 1e3) / 1e9,
+                    pipelining="next step's H2D on a copy stream overlaps this step's compute; D2H after it")
+
+    e2e = e2e_gated = None
+    if not args.no_e2e:
+        def plain_e2e_step(src):
+            o, _, g = step(src)
+            return o, g["dS0"]
+        e2e = end_to_end(host, plain_e2e_step)
+        # the same step through the gated entry points: the forget gate
+        # uploaded as its bf16 pre-activation (and a_log per head) in place of
+        # the fp32 log-decay
+        gen = torch.Generator()
+        gen.manual_seed(rank_seed(5004, rank))
+        ghost = {n: t for n, t in host.items() if n != "logf"}
+        ghost["f_pre"] = (torch.randn((B, T, H, dk), generator=gen) + 3.0).to(bf)
+        ghost["a_log"] = torch.rand((H,), generator=gen) * 2 - 1
+        e_fw = torch.empty(kd.workspace_size(kd.KD_WS_FWD_GATED, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+        e_bw = torch.empty(kd.workspace_size(kd.KD_WS_BWD_GATED, B, H, T, dk, dv), dtype=torch.uint8, device=dev)
+
+        def gated_e2e_step(src):
+            o, _, _ = kd.fwd_gated(src["q"], src["k"], src["v"], src["beta"], src["c"], src["f_pre"], src["a_log"],
+                                   src["S0"], out=out, save=True, workspace=e_fw)
+            g = kd.bwd_gated(src["q"], src["k"], src["v"], src["beta"], src["c"], src["f_pre"], src["a_log"],
+                             src["S0"], src["dO"], fwd_workspace=e_fw, workspace=e_bw)
+            return o, g["dS0"]
+        for _ in range(2):
+            gated_e2e_step({n: t.to(dev) for n, t in ghost.items()})
+        torch.cuda.synchronize()
+        e2e_gated = end_to_end(ghost, gated_e2e_step)
+        e2e_gated["step"] = "fwd_gated(save) + bwd_gated: bf16 f_pre and a_log [H] uploaded in place of fp32 logf"
+        del e_fw, e_bw, ghost
+        kd.device_status()
 
     value = job_throughput(ws_n, B * T, args.steps, ms_total)
 
@@ -886,7 +916,7 @@ def main(argv=None):
                 "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "T": T, "dk": dk, "dv": dv, "chunk": CHUNK,
                            "global_batch": B * ws_n, "seq_len": T, "parallelism": f"dp{ws_n}",
                            "step": "fwd(save) + bwd", "l2": "inputs larger than L2 (no flush)"},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "e2e_gated": e2e_gated,
                 "gpu_launches": launches,
                 "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                            "reasons": clocks["reasons"], "samples": clocks["samples"]},
