@@ -129,6 +129,25 @@ def test_gdn2_extreme_decay_tensor_cores():
     check(inp, "bf16")
 
 
+def test_gdn2_tensor_cores_batched_ragged_with_final_state_gradient():
+    """The tensor-core path (bf16, d = 128) with two batch entries, a ragged last
+    chunk and a final-state gradient: every (b, h) checked on its own."""
+    inp = kin.make_gdn2_inputs(2, 3, 200, 128, 128, "bf16", seed=71)
+    dST = np.random.default_rng(72).standard_normal((2, 3, 128, 128)) / 128
+    out, ST, g = run(inp, "bf16", dST)
+    O_ref, ST_ref = G.fwd(**{n: inp[n] for n in NAMES}, S0=inp["S0"])
+    gr = G.bwd(**{n: inp[n] for n in NAMES}, S0=inp["S0"], dO=inp["dO"], dST=dST)
+    tf, tg = TOL["bf16"]
+    for bb in range(2):
+        for hh in range(3):
+            one = {"O": rel(host(out)[bb, :, hh], O_ref[bb, :, hh]), "ST": rel(host(ST)[bb, hh], ST_ref[bb, hh]),
+                   "dS0": rel(host(g["dS0"])[bb, hh], gr["dS0"][bb, hh])}
+            for n in ("dq", "dk", "dv", "db", "dw", "dloga"):
+                one[n] = rel(host(g[n])[bb, :, hh], gr[n][bb, :, hh])
+            bad = {n: e for n, e in one.items() if e > (tf if n in ("O", "ST") else tg)}
+            assert not bad, (bb, hh, one)
+
+
 def test_gdn2_workload_B1_H16_T16384_sampled_heads():
     """The mixer's full-size shape (B=1, H=16, T=16384, d=128, bf16), run whole
     on the GPU; heads 0 and 11 checked against the oracle."""
