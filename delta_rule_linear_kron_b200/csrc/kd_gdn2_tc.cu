@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
 struct GOutCfg {
   static constexpr uint32_t SH = 0, SL = 32768;          // S0 [r][j], 2 K blocks x 128 rows
   static constexpr uint32_t QH = 65536, QL = 81920;      // Q+ [t][j], 2 K blocks x 64 rows
-  static constexpr uint32_t UH = 98304, UL = 114688;     // U^T [r][i], 128 rows
+  static constexpr uint32_t UH = 98304, UL = 114688;     // U [i][r], 64 rows (read MN-major as U^T)
   static constexpr uint32_t PH = 131072, PL = 139264;    // P [t][i], 64 rows
   static constexpr uint32_t BYTES = 147456 + 1024;
 };
@@ -409,16 +409,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
       put_hl4(sm + Cf::PH, sm + Cf::PL, tc::sw128_off(t, ii, 64, 2), x[8 + i]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // U [i][r] -> U^T [r][i]
+    for (int i = 0; i < 8; ++i) {  // U [i][r]
       const int e = tid + 256 * i, ii = e / (D / 4), r = 4 * (e % (D / 4));
-      const float xs[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const __nv_bfloat16 hh = __float2bfloat16_rn(xs[c]);
-        const uint32_t off = tc::sw128_off(r + c, ii, 128, 2);
-        *reinterpret_cast<__nv_bfloat16*>(sm + Cf::UH + off) = hh;
-        *reinterpret_cast<__nv_bfloat16*>(sm + Cf::UL + off) = __float2bfloat16_rn(xs[c] - __bfloat162float(hh));
-      }
+      put_hl4(sm + Cf::UH, sm + Cf::UL, tc::sw128_off(ii, r, 64, 2), x[i]);
     }
   }
   tc::fence_proxy_async();
@@ -428,7 +421,7 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
   if (tid == 0) {
-    const uint32_t IDB = tc::idesc(128, 64, 1);
+    const uint32_t IDB = tc::idesc(128, 64, 1), IDU = tc::idesc(128, 64, 1) | tc::kMajorA;
     const uint32_t sq[3][2] = {{Cf::SH, Cf::QH}, {Cf::SH, Cf::QL}, {Cf::SL, Cf::QH}};
     const uint32_t up[3][2] = {{Cf::UH, Cf::PH}, {Cf::UH, Cf::PL}, {Cf::UL, Cf::PH}};
 #pragma unroll
@@ -439,9 +432,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
                         tc::desc_sw128(tc::smem_u32(sm + sq[pr][1] + (ks / 4) * 8192 + (ks % 4) * 32)), IDB,
                         (pr | ks) ? 1u : 0u);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)  // U^T P^T: K = 64 positions
-        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + up[pr][0] + ks * 32)),
-                        tc::desc_sw128(tc::smem_u32(sm + up[pr][1] + ks * 32)), IDB, 1u);
+      for (int ks = 0; ks < 4; ++ks)  // U^T P^T: K = 64 positions (U^T the MN-major view of U)
+        tc::mma_bf16_ss(tmem, tc::desc_sw128_mn(tc::smem_u32(sm + up[pr][0] + ks * 2048), 8192u),
+                        tc::desc_sw128(tc::smem_u32(sm + up[pr][1] + ks * 32)), IDU, 1u);
     }
     tc::mma_commit(&mma_bar);
   }
@@ -1016,7 +1009,7 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     tc::tc_after_sync();
     const uint32_t ID128 = tc::idesc(128, 128, 1) | tc::kMajorA, ID64 = tc::idesc(128, 64, 1) | tc::kMajorA;
     const uint32_t ID64K = tc::idesc(128, 64, 1);
-#pragma unroll
+#pragma unroll 1
     for (int ks = 0; ks < 8; ++ks) {
       const uint32_t kb = (ks / 4) * 16384 + (ks % 4) * 32, kb64 = (ks / 4) * 8192 + (ks % 4) * 32;
       const uint32_t mn = ks * 2048;
@@ -1131,7 +1124,7 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
   if (tid == 0) {
     // dZ^T = dU^T A, dE^T = dW^T A (A as the MN-major B operand)
     const uint32_t ID = tc::idesc(128, 64, 1) | tc::kMajorA | tc::kMajorB;
-#pragma unroll
+#pragma unroll 1
     for (int ks = 0; ks < 4; ++ks) {
       const uint32_t mn = ks * 2048;
       const uint64_t ah = tc::desc_sw128_mn(sd(Cf::AH + mn), 8192u), al = tc::desc_sw128_mn(sd(Cf::AL + mn), 8192u);
@@ -1147,31 +1140,43 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     }
     tc::mma_commit(&mma_bar);
   }
-  // the write gates and values at this thread's (t, channel r = j) for dv and dw
-  float w16[16], v16[16];
+  // the write gates and values at this thread's (t, channel r = j) for dv and
+  // dw, eight positions per step, the next step's loads in flight meanwhile
+  const auto ld_wv = [&](int c0, float (&w8)[8], float (&v8)[8]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const bool ok = tb + i < nv;
-    w16[i] = ok ? wg[row(tb + i) + j] : 0.f;
-    v16[i] = ok ? __bfloat162float(v[row(tb + i) + j]) : 0.f;
-  }
+    for (int i = 0; i < 8; ++i) {
+      const bool ok = c0 + i < nv;
+      w8[i] = ok ? wg[row(c0 + i) + j] : 0.f;
+      v8[i] = ok ? __bfloat162float(v[row(c0 + i) + j]) : 0.f;
+    }
+  };
+  float wn[8], vn[8];
+  ld_wv(tb, wn, vn);
   tc::mbar_wait<false>(&mma_bar, 1, err, tc::kErrTimeoutMma, &abort_flag);
   tc::tc_after_sync();
   // dZ^T (lane r) -> dZ [t][r] operand, dv and dw; dE^T (lane j) -> dE [t][j] operand
-  {
-    float z[16], e[16];
-    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DZ + tb), z);
-    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + tb), e);
+#pragma unroll 1
+  for (int c8 = 0; c8 < 2; ++c8) {
+    const int c0 = tb + 8 * c8;
+    float w8[8], v8[8], z[8], e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w8[i] = wn[i];
+      v8[i] = vn[i];
+    }
+    if (c8 == 0) ld_wv(c0 + 8, wn, vn);
+    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DZ + c0), z);
+    tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DE + c0), e);
     tc::tmem_ld_wait();
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int t = tb + i;
+    for (int i = 0; i < 8; ++i) {
+      const int t = c0 + i;
       const uint32_t o = tc::sw128_off(t, j, 64, 2);
       put_hl(sm + Cf::ZH, sm + Cf::ZL, o, z[i]);
       put_hl(sm + Cf::EH, sm + Cf::EL, o, e[i]);
       if (t < nv) {
-        dv[row(t) + j] = __float2bfloat16_rn(z[i] * w16[i]);
-        dw[row(t) + j] = z[i] * v16[i];
+        dv[row(t) + j] = __float2bfloat16_rn(z[i] * w8[i]);
+        dw[row(t) + j] = z[i] * v8[i];
       }
     }
   }
@@ -1183,9 +1188,9 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     // [U' hi; U' lo] dZ^T + [W hi; W lo] dE^T, with dZ, dE hi and then lo
     tc::mbar_wait<false>(&w_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
     const uint32_t ID = tc::idesc(128, 64, 1);
-#pragma unroll
+#pragma unroll 1
     for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kb = (ks / 4) * 16384 + (ks % 4) * 32, kb64 = (ks / 4) * 8192 + (ks % 4) * 32;
         tc::mma_bf16_ss(tmem + Cf::C_DT, tc::desc_sw128(sd(Cf::UPS + kb)),
@@ -1216,14 +1221,18 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
   float* scp = reinterpret_cast<float*>(sm + Cf::SCP);
   if ((warp & 3) >= 2) {
     const int i = j - 64;
-    float x[16], y[16];
-    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + tb), x);
-    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + tb), y);
-    tc::tmem_ld_wait();
+#pragma unroll 1
+    for (int c8 = 0; c8 < 2; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float x[8], y[8];
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + c0), x);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + c0), y);
+      tc::tmem_ld_wait();
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      sct[i * 65 + tb + ii] = x[ii];
-      scp[i * 65 + tb + ii] = y[ii];
+      for (int ii = 0; ii < 8; ++ii) {
+        sct[i * 65 + c0 + ii] = x[ii];
+        scp[i * 65 + c0 + ii] = y[ii];
+      }
     }
   }
   if (!exact) {
@@ -1252,21 +1261,25 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
   __syncthreads();
   if ((warp & 3) < 2) {
     const int i = j;
-    float x[16], y[16];
-    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + tb), x);
-    tc::tmem_ld16(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + tb), y);
-    tc::tmem_ld_wait();
+#pragma unroll 1
+    for (int c8 = 0; c8 < 2; ++c8) {
+      const int c0 = tb + 8 * c8;
+      float x[8], y[8];
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DT + c0), x);
+      tc::tmem_ld8(tc::tmem_lane_addr(tmem, warp, Cf::C_DP + c0), y);
+      tc::tmem_ld_wait();
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      const int t = tb + ii;
-      const float dtv = i < t ? -(x[ii] + sct[i * 65 + t]) : 0.f;
-      const float dpv = i <= t ? y[ii] + scp[i * 65 + t] : 0.f;
-      if (exact) {
-        p.dT[(ch * C + t) * C + i] = dtv;
-        p.dP[(ch * C + t) * C + i] = dpv;
-      } else {
-        put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(t, i, 128, 2), dtv);
-        put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(64 + t, i, 128, 2), dpv);
+      for (int ii = 0; ii < 8; ++ii) {
+        const int t = c0 + ii;
+        const float dtv = i < t ? -(x[ii] + sct[i * 65 + t]) : 0.f;
+        const float dpv = i <= t ? y[ii] + scp[i * 65 + t] : 0.f;
+        if (exact) {
+          p.dT[(ch * C + t) * C + i] = dtv;
+          p.dP[(ch * C + t) * C + i] = dpv;
+        } else {
+          put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(t, i, 128, 2), dtv);
+          put_hl(sm + Cf::TPH, sm + Cf::TPL, tc::sw128_off(64 + t, i, 128, 2), dpv);
+        }
       }
     }
   }
@@ -1297,12 +1310,12 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
       // [X1^T | X2^T] = K-^T [dT; dP]^T and Y^T = E+^T dT + Q+^T dP
       const uint32_t IDX = tc::idesc(128, 128, 1) | tc::kMajorA;
       const uint32_t IDY = tc::idesc(128, 64, 1) | tc::kMajorA | tc::kMajorB;
-      const uint32_t ops[3][2] = {{0u, 0u}, {0u, 16384u}, {16384u, 0u}};  // (A, B) part offsets: hi hi, hi lo, lo hi
-#pragma unroll
+#pragma unroll 1
       for (int pr = 0; pr < 3; ++pr)
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t mn = ks * 2048, a = ops[pr][0], bo = ops[pr][1];
+          // (A, B) part offsets: hi hi, hi lo, lo hi
+          const uint32_t mn = ks * 2048, a = pr == 2 ? 16384u : 0u, bo = pr == 1 ? 16384u : 0u;
           tc::mma_bf16_ss(tmem + Cf::C_X, tc::desc_sw128_mn(sd(Cf::KMH + a + mn), 8192u),
                           tc::desc_sw128(sd(Cf::TPH + bo + ks * 32)), IDX, (pr | ks) ? 1u : 0u);
           tc::mma_bf16_ss(tmem + Cf::C_Y, tc::desc_sw128_mn(sd(Cf::EPH + a + mn), 8192u),
