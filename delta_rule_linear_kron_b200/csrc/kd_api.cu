@@ -154,7 +154,7 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
   L->Qp = take(chunks * C * dk);
   L->gC = take(chunks * dk);
   if (L->tc) {
-    L->S0img = take(chunks * (size_t)dv * dk);  // bf16 hi + lo: the bytes of one fp32 tile
+    L->S0img = take(chunks * (size_t)dv * dk / 2);  // bf16
     L->Wimg = take(chunks * C * dk);
     L->Kimg = take(chunks * C * dk);
   } else {
@@ -176,7 +176,7 @@ int gdn_plan(int B, int H, int T, int dk, int dv, int dtype, kd::GdnLayout* L) {
     L->S0b = take(chunks * (size_t)dv * dk);
     L->dUi = take(chunks * C * dv);
     L->L2t = take(chunks * (size_t)dk * dv);
-    L->dSimg = take(chunks * (size_t)dv * dk);
+    L->dSimg = take(chunks * (size_t)dv * dk / 2);
     L->xflag = take((chunks + 3) / 4);
   }
   L->bwd_bytes = off;

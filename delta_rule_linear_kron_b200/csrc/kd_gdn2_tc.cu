@@ -334,13 +334,13 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
 // ---------------------------------------------------------------------------
 // The chunk outputs O = Q+ S0^T + P U, one CTA per chunk, all chunks in
 // parallel, computed transposed on tcgen05 (M = 128 value channels, N = 64
-// positions): O^T = S0 Q+^T + U^T P^T, every operand as bf16 high and low
-// parts (hi hi + hi lo + lo hi).  S0 arrives as the chain's saved image (one
-// bulk copy); Q+, P (preparation kernel) and U (chain) arrive in fp32 and are
-// split while they are staged into shared memory.
+// positions): O^T = S0 Q+^T + U^T P^T.  S0 arrives as the chain's saved bf16
+// image (one bulk copy) and meets Q+'s high and low parts; Q+, P (preparation
+// kernel) and U (chain) arrive in fp32 and are split into bf16 high and low
+// parts while they are staged (hi hi + hi lo + lo hi).
 // ---------------------------------------------------------------------------
 struct GOutCfg {
-  static constexpr uint32_t SH = 0, SL = 32768;          // S0 [r][j], 2 K blocks x 128 rows
+  static constexpr uint32_t SH = 0;                      // S0 [r][j] bf16, 2 K blocks x 128 rows (32 KB)
   static constexpr uint32_t QH = 65536, QL = 81920;      // Q+ [t][j], 2 K blocks x 64 rows
   static constexpr uint32_t UH = 98304, UL = 114688;     // U [i][r], 64 rows (read MN-major as U^T)
   static constexpr uint32_t PH = 131072, PL = 139264;    // P [t][i], 64 rows
@@ -379,10 +379,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    // S0 arrives as the chain's saved image: its hi and lo tiles as they are
-    tc::mbar_expect_tx(&ld_bar, 4u * D * D);
-    tc::bulk_g2s(sm + Cf::SH, p.S0img + ch * (2 * D * D), 2u * D * D, &ld_bar);
-    tc::bulk_g2s(sm + Cf::SL, p.S0img + ch * (2 * D * D) + D * D, 2u * D * D, &ld_bar);
+    // S0 arrives as the chain's saved bf16 image, as it is
+    tc::mbar_expect_tx(&ld_bar, 2u * D * D);
+    tc::bulk_g2s(sm + Cf::SH, p.S0img + ch * (D * D), 2u * D * D, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 64);
   // stage the operands: four consecutive elements per thread and step, read as
@@ -422,15 +421,17 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
   if (tid == 0) {
     const uint32_t IDB = tc::idesc(128, 64, 1), IDU = tc::idesc(128, 64, 1) | tc::kMajorA;
-    const uint32_t sq[3][2] = {{Cf::SH, Cf::QH}, {Cf::SH, Cf::QL}, {Cf::SL, Cf::QH}};
+    const uint32_t sq[2] = {Cf::QH, Cf::QL};  // S0 (bf16) Q+^T: Q+ hi, then lo
     const uint32_t up[3][2] = {{Cf::UH, Cf::PH}, {Cf::UH, Cf::PL}, {Cf::UL, Cf::PH}};
 #pragma unroll
     for (int pr = 0; pr < 3; ++pr) {
+      if (pr < 2) {
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)  // S0 Q+^T: K = 128 channels, two swizzle blocks
-        tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + sq[pr][0] + (ks / 4) * 16384 + (ks % 4) * 32)),
-                        tc::desc_sw128(tc::smem_u32(sm + sq[pr][1] + (ks / 4) * 8192 + (ks % 4) * 32)), IDB,
-                        (pr | ks) ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks)  // S0 Q+^T: K = 128 channels, two swizzle blocks
+          tc::mma_bf16_ss(tmem, tc::desc_sw128(tc::smem_u32(sm + Cf::SH + (ks / 4) * 16384 + (ks % 4) * 32)),
+                          tc::desc_sw128(tc::smem_u32(sm + sq[pr] + (ks / 4) * 8192 + (ks % 4) * 32)), IDB,
+                          (pr | ks) ? 1u : 0u);
+      }
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)  // U^T P^T: K = 64 positions (U^T the MN-major view of U)
         tc::mma_bf16_ss(tmem, tc::desc_sw128_mn(tc::smem_u32(sm + up[pr][0] + ks * 2048), 8192u),
@@ -473,8 +474,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_out_tc(int H, int T, int NC, GdnW
 // Warp roles (320 threads):
 //   warps 0-7   state warps: thread (r, c) holds row r, key channels 64c..64c+63
 //               of S, and positions 32c..32c+31 of U; U = U' - X, the operand
-//               U^T, the state update and its operand copy (bf16 hi, lo), which
-//               the issuer also copies out as the chunk's saved start state.
+//               U^T, the state update and its operand copy (bf16 hi, lo), whose
+//               hi part the issuer also copies out as the chunk's saved start
+//               state (bf16).
 //   warp 8      producer: one thread copies chunk n+1's operand images (bf16
 //               hi, lo, written by the preparation kernel) and gamma_C into one
 //               of two slots while chunk n runs, and pulls later chunks into L2.
@@ -525,7 +527,7 @@ struct GChainIO {
   const float* ul;     // [ch][t][r]: U' (forward) or P^T dO (backward)
   const float* l2t;    // backward: (dO^T Q+)^T [ch][j][r], added to the state update
   float* uout;         // U (forward) or dU (backward) [ch][t][r]
-  __nv_bfloat16* img;  // the saved state images [ch] (bf16 hi, lo)
+  __nv_bfloat16* img;  // the saved state images [ch] (bf16: the hi part of MMA 1's operand)
 };
 
 template <bool BWD>
@@ -578,7 +580,7 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
       const int n = BWD ? NC - 1 - k : k;  // the backward runs from the last chunk to the first
       const size_t ch = unit * NC + n;
       // this chunk's start state as MMA 1's operand; the issuer also copies
-      // this image out as the chunk's saved start state (one bulk copy: the
+      // its hi part out as the chunk's saved start state (one bulk copy: the
       // rows of a thread-per-row state would scatter over 128 rows)
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -695,9 +697,8 @@ __global__ void __launch_bounds__(GChainCfg::THREADS, 1) gdn2_chain_tc(GChainIO 
       tc::mma_commit(&x_done);
       {
         // the chunk's start state image out, while MMA 1 runs
-        __nv_bfloat16* img = io.img + (unit * NC + n) * (2 * D * D);
+        __nv_bfloat16* img = io.img + (unit * NC + n) * (D * D);
         tc::bulk_s2g(img, sm + Cf::SH, 2u * D * D);
-        tc::bulk_s2g(img + D * D, sm + Cf::SL, 2u * D * D);
         tc::bulk_commit();
       }
       tc::mbar_wait<false>(&u_ready, k & 1, err, tc::kErrTimeoutMma, &abort_flag);
@@ -860,15 +861,16 @@ __global__ void __launch_bounds__(256, 1) gdn2_bpre_tc(const __nv_bfloat16* __re
 // Every product runs transposed, with M = 128 key or value channels in TMEM
 // lanes; the two 64 x 64 results (dP^T, dT^T) take their 64-row operand
 // stacked as [hi; lo] parts over the 128 lanes, and the two halves are summed.
-// Operands are bf16 high and low parts (hi hi + hi lo + lo hi; dO is exact in
-// bf16).  A thread owns key (or value) channel j = lane of its warp's TMEM
-// quarter and positions 32 * (warp / 4) .. + 31, so the dloga suffix sums run
-// down its own registers.  Chunks beyond the factorised range leave dQ+, dK^e,
+// Operands are bf16 high and low parts (hi hi + hi lo + lo hi); dO is exact in
+// bf16, and the saved states S0 and dS arrive as the chains' bf16 images.  A
+// thread owns key (or value) channel j = lane of its warp's TMEM quarter and
+// positions 16 * (warp / 4) .. + 15, so the dloga suffix sums run down its own
+// registers (one exchange between the four position groups).  Chunks beyond the factorised range leave dQ+, dK^e,
 // dE, dT, dP and S0, dS (fp32) in the workspace for the exact kernel.
 // ---------------------------------------------------------------------------
 struct GBpostCfg {
   // step 1
-  static constexpr uint32_t SI = 0;                      // S0 image [r][j] hi, lo (32 KB each)
+  static constexpr uint32_t SI = 0;                      // S0 image [r][j] bf16 (32 KB)
   static constexpr uint32_t DI = 65536;                  // dS image, the same
   static constexpr uint32_t BO = 131072;                 // [dO; dU hi] [t][r], 128 rows (32 KB)
   static constexpr uint32_t DUL = 163840;                // dU lo [t][r], 64 rows (16 KB)
@@ -934,13 +936,9 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     tc::mbar_init(&mma_bar, 1);
     tc::mbar_init_fence();
     abort_flag = 0;
-    tc::mbar_expect_tx(&ld_bar, 8u * D * D);
-    const __nv_bfloat16* s0 = p.S0img + ch * (2 * D * D);
-    const __nv_bfloat16* ds = p.dSimg + ch * (2 * D * D);
-    tc::bulk_g2s(sm + Cf::SI, s0, 2u * D * D, &ld_bar);
-    tc::bulk_g2s(sm + Cf::SI + 2 * D * D, s0 + D * D, 2u * D * D, &ld_bar);
-    tc::bulk_g2s(sm + Cf::DI, ds, 2u * D * D, &ld_bar);
-    tc::bulk_g2s(sm + Cf::DI + 2 * D * D, ds + D * D, 2u * D * D, &ld_bar);
+    tc::mbar_expect_tx(&ld_bar, 4u * D * D);
+    tc::bulk_g2s(sm + Cf::SI, p.S0img + ch * (D * D), 2u * D * D, &ld_bar);
+    tc::bulk_g2s(sm + Cf::DI, p.dSimg + ch * (D * D), 2u * D * D, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
 
@@ -1013,20 +1011,16 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     for (int ks = 0; ks < 8; ++ks) {
       const uint32_t kb = (ks / 4) * 16384 + (ks % 4) * 32, kb64 = (ks / 4) * 8192 + (ks % 4) * 32;
       const uint32_t mn = ks * 2048;
-      // [dQ+^T | (dU S0)^T] = S0^T [dO; dU]^T: hi hi, lo hi, and hi lo on the dU half
+      // [dQ+^T | (dU S0)^T] = S0^T [dO; dU]^T (S0 in bf16), with dU's lo part on the dU half
       tc::mma_bf16_ss(tmem + Cf::C_DQ, tc::desc_sw128_mn(sd(Cf::SI + mn), 16384u), tc::desc_sw128(sd(Cf::BO + kb)),
                       ID128, ks > 0 ? 1u : 0u);
-      tc::mma_bf16_ss(tmem + Cf::C_DQ, tc::desc_sw128_mn(sd(Cf::SI + 32768 + mn), 16384u),
-                      tc::desc_sw128(sd(Cf::BO + kb)), ID128, 1u);
       tc::mma_bf16_ss(tmem + Cf::C_DW, tc::desc_sw128_mn(sd(Cf::SI + mn), 16384u), tc::desc_sw128(sd(Cf::DUL + kb64)),
                       ID64, 1u);
-      // dK^e^T = dS^T U^T
+      // dK^e^T = dS^T U^T (dS in bf16; U hi and lo)
       tc::mma_bf16_ss(tmem + Cf::C_DK, tc::desc_sw128_mn(sd(Cf::DI + mn), 16384u), tc::desc_sw128(sd(Cf::US + kb)),
                       ID64, ks > 0 ? 1u : 0u);
       tc::mma_bf16_ss(tmem + Cf::C_DK, tc::desc_sw128_mn(sd(Cf::DI + mn), 16384u),
                       tc::desc_sw128(sd(Cf::US + 8192 + kb)), ID64, 1u);
-      tc::mma_bf16_ss(tmem + Cf::C_DK, tc::desc_sw128_mn(sd(Cf::DI + 32768 + mn), 16384u),
-                      tc::desc_sw128(sd(Cf::US + kb)), ID64, 1u);
       // [U hi; U lo] dO^T: lanes 0-63 and 64-127 are the two parts of dP^T
       tc::mma_bf16_ss(tmem + Cf::C_DP, tc::desc_sw128(sd(Cf::US + kb)), tc::desc_sw128(sd(Cf::BO + kb)), ID64K,
                       ks > 0 ? 1u : 0u);
@@ -1043,19 +1037,14 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
     for (int rr = 0; rr < 4; ++rr) {
       const uint32_t o = tc::sw128_off(4 * rg + rr, 8 * jg, 128, 2);
       const uint4 sh = *reinterpret_cast<const uint4*>(sm + Cf::SI + o);
-      const uint4 sl = *reinterpret_cast<const uint4*>(sm + Cf::SI + 32768 + o);
       const uint4 dh = *reinterpret_cast<const uint4*>(sm + Cf::DI + o);
-      const uint4 dl = *reinterpret_cast<const uint4*>(sm + Cf::DI + 32768 + o);
       const __nv_bfloat162* a0 = reinterpret_cast<const __nv_bfloat162*>(&sh);
-      const __nv_bfloat162* a1 = reinterpret_cast<const __nv_bfloat162*>(&sl);
       const __nv_bfloat162* b0 = reinterpret_cast<const __nv_bfloat162*>(&dh);
-      const __nv_bfloat162* b1 = reinterpret_cast<const __nv_bfloat162*>(&dl);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float2 s2 = __bfloat1622float2(a0[c]), s2l = __bfloat1622float2(a1[c]);
-        const float2 d2 = __bfloat1622float2(b0[c]), d2l = __bfloat1622float2(b1[c]);
-        acc8[2 * c] = fmaf(d2.x + d2l.x, s2.x + s2l.x, acc8[2 * c]);
-        acc8[2 * c + 1] = fmaf(d2.y + d2l.y, s2.y + s2l.y, acc8[2 * c + 1]);
+        const float2 s2 = __bfloat1622float2(a0[c]), d2 = __bfloat1622float2(b0[c]);
+        acc8[2 * c] = fmaf(d2.x, s2.x, acc8[2 * c]);
+        acc8[2 * c + 1] = fmaf(d2.y, s2.y, acc8[2 * c + 1]);
       }
     }
 #pragma unroll
@@ -1071,8 +1060,8 @@ __global__ void __launch_bounds__(kBpostThreads, 1) gdn2_bpost_tc(
       for (int e = tid; e < D * D; e += NT) {
         const int r = e / D, jj = e % D;
         const uint32_t o = tc::sw128_off(r, jj, 128, 2);
-        s0[e] = ld_bf(sm + Cf::SI + o) + ld_bf(sm + Cf::SI + 32768 + o);
-        ds[e] = ld_bf(sm + Cf::DI + o) + ld_bf(sm + Cf::DI + 32768 + o);
+        s0[e] = ld_bf(sm + Cf::SI + o);
+        ds[e] = ld_bf(sm + Cf::DI + o);
       }
     }
   }

@@ -224,12 +224,12 @@ struct GdnLayout {
   size_t chunks = 0;
   size_t A = 0, P = 0, W = 0, Up = 0, Ke = 0, Qp = 0, gC = 0, S0 = 0, U = 0, fwd_bytes = 0;
   size_t dU = 0, dS = 0, dE = 0, dT = 0, dP = 0, dQp = 0, dKe = 0, bwd_bytes = 0;
-  // tensor-core path (bf16, dk = dv = 128): the chunk-start states are kept as
-  // bf16 high and low parts in the 128-byte-swizzled K-major image the chain
-  // and the output kernel hold in shared memory ([ch] 32 KB hi + 32 KB lo, in
-  // the forward's workspace, where S0 is not allocated), and so are the
-  // backward's dS; its gradient kernel reads both images and writes fp32 S0
-  // (S0b) and dS only for the chunks the exact kernel takes
+  // tensor-core path (bf16, dk = dv = 128): the chunk-start states are kept in
+  // bf16 (the high part of the chain's fp32 state) in the 128-byte-swizzled
+  // K-major image the chain and the output kernel hold in shared memory ([ch]
+  // 32 KB, in the forward's workspace, where S0 is not allocated), and so are
+  // the backward's dS; its gradient kernel reads both images and writes fp32
+  // S0 (S0b) and dS only for the chunks the exact kernel takes
   bool tc = false;
   size_t S0img = 0, S0b = 0;
   // tensor-core path: the chains' B operands as bf16 hi, lo images (32 KB per
