@@ -100,6 +100,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
     tc::tma_load_4d(sm + Cf::LS, &tm_loga, 0, h, t0, b, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
+  // the erase and write gates' rows into L2 while the tiles land: their loads
+  // (steps 1 and 3) then wait on L2, not on HBM
+  if (tid < 2 * C && (tid & 63) < nv) tc::prefetch_l2((tid < C ? bg : wg) + row(tid & 63), 4u * D);
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
@@ -289,9 +292,9 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
   tc::tc_after_sync();
   {
     // warps 0-3: lane j of W^T -> the chains' image of W ([t][j], bf16 hi, lo);
-    // warps 4-7: lane r of U'^T -> U'[t][r], then the chains' image of K^e
-    // ([t][j], bf16 hi, lo) for channel j = r.  The operand tiles of steps 1
-    // and 3 are free (their MMAs have completed).
+    // warps 4-7: lane r of U'^T -> U'[t][r]; then each group half of the
+    // chains' image of K^e ([t][j], bf16 hi, lo) for channel j = lane.  The
+    // operand tiles of steps 1 and 3 are free (their MMAs have completed).
     const int lr = (warp & 3) * 32 + lane;
     const uint32_t lanes = tc::tmem_lane_addr(tmem, warp, warp < 4 ? 0 : 64);
     float* up = p.Up + ch * C * D + lr;
@@ -309,10 +312,11 @@ __global__ void __launch_bounds__(256, 1) gdn2_prep_tc(
           up[t * D] = v[ii];
       }
     }
-    if (warp >= 4) {
+    {
       const float lj = lam[lr];
+      const int tk = warp < 4 ? 0 : 32;
 #pragma unroll 8
-      for (int t = 0; t < C; ++t) {
+      for (int t = tk; t < tk + 32; ++t) {
         const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Cf::KR + (t * D + lr) * 2));
         put_hl(sm + Cf::IK, sm + Cf::IK + 16384, tc::sw128_off(t, lr, 64, 2), kk * expf(lj - Ls[t * D + lr]));
       }
