@@ -372,24 +372,30 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
     tc::bulk_g2s(sm + Cf::B7, wPU + ch * (C * C), 8192u, &bar_b);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
+  // per position: g, beta, u and the chain's two dbeta terms, loaded now and
+  // used after the tiles land (their round trip overlaps the tile loads)
+  float gt = 0.f, bt = 0.f, ut = 0.f, b0t = 0.f, mut = 0.f;
+  const size_t gi = ((size_t)b * T + t0 + tid) * H + h;
   if (tid < C) {
-    const int t = tid;
-    const float gt = wg[ch * C + t];
-    const bool ok = t < nv;
-    const size_t gi = ((size_t)b * T + t0 + t) * H + h;
-    const float bt = ok ? beta[gi] : 0.f;
-    us[t] = wu[ch * C + t];
-    db0s[t] = -bt * gt;
-    if (ok) {
-      dc[gi] = gt;
-      dbeta[gi] = -gt * (wb0[ch * C + t] + wMu[ch * C + t]);
-    }
+    gt = wg[ch * C + tid];
+    bt = tid < nv ? beta[gi] : 0.f;
+    ut = wu[ch * C + tid];
+    b0t = wb0[ch * C + tid];
+    mut = wMu[ch * C + tid];
   }
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&bar_a, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  if (tid < C) {  // read after the prefix's barrier below
+    us[tid] = ut;
+    db0s[tid] = -bt * gt;
+    if (tid < nv) {
+      dc[gi] = gt;
+      dbeta[gi] = -gt * (b0t + mut);
+    }
+  }
   // gated inputs: logf (formed by the forward's preparation kernel) with the
   // exponent a = e^{a_log}, for the epilogue's df~ and da_log
   const float ga = a_log ? expf(a_log[h]) : 0.f, inv_ga = a_log ? expf(-a_log[h]) : 0.f;

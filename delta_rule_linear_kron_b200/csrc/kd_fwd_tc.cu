@@ -347,21 +347,24 @@ __global__ void __launch_bounds__(256, 1) fwd_prep_tc(
     tc::tma_load_4d(sm + PrepCfg::LS + (a_log ? 16384 : 0), &tm_logf, 0, h, t0, b, &ld_bar);
   }
   if (warp == 0) tc::tmem_alloc(&tmem_slot, 128);
-  if (tid < C) {
-    const bool ok = tid < nv;
-    const size_t g = ((size_t)b * T + t0 + tid) * H + h;
-    bs[tid] = ok ? gate_beta(beta[g], pro) : 0.f;
-    cs[tid] = ok ? gate_c(c[g], pro) : 0.f;
-    if (pro.bscale > 0.f && ok) {  // fused prologue: the gated values, for the chain and the backward
-      fbeta[g] = bs[tid];
-      fc[g] = cs[tid];
-    }
-  }
+  // beta and c of each position, loaded now and used after the tiles land
+  // (their round trip overlaps the tile loads)
+  const size_t gpos = ((size_t)b * T + t0 + tid) * H + h;
+  const float braw = tid < nv ? beta[gpos] : 0.f, craw = tid < nv ? c[gpos] : 0.f;
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
+  if (tid < C) {  // read after the prefix's barrier below
+    const bool ok = tid < nv;
+    bs[tid] = ok ? gate_beta(braw, pro) : 0.f;
+    cs[tid] = ok ? gate_c(craw, pro) : 0.f;
+    if (pro.bscale > 0.f && ok) {  // fused prologue: the gated values, for the chain and the backward
+      fbeta[gpos] = bs[tid];
+      fc[gpos] = cs[tid];
+    }
+  }
   if (pro.norm) {  // fused prologue: q, k, v arrive raw and are normalised in place
     l2norm_tile(sm + PrepCfg::QR, sm + PrepCfg::QR + 128, 256);
     l2norm_tile(sm + PrepCfg::KR, sm + PrepCfg::KR + 128, 256);
