@@ -343,10 +343,11 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
   float* db0s = us + 64;
   float* xch = db0s + 64;    // [128]
   float* lam = xch + 128;    // [128] Lambda_j
-  float* csp = lam + 128;    // [2][128] sum_r dS'[r,j] S0[r,j] by row half
+  float* csp = lam + 128;    // [2][128] sum_r dS'[r,j] S0[r,j] (in the first half; the second is zero)
   float* ekp = csp + 256;    // [2][128] sum_t k o u o e^{-L} o XB by position half
   float* tail = ekp + 256;   // [128] sum of dL over positions 32..63
   __shared__ float dred[8];  // gated inputs: per-warp parts of this chunk's da_log term
+  __shared__ float csred[8][D];  // per-warp parts of sum_r dS'[r,j] S0[r,j]
 
   if (tid == 0) {
     tc::mbar_init(&bar_a, 1);
@@ -441,22 +442,53 @@ __global__ void __launch_bounds__(256, 1) bwd_post_tc(
   }
   tc::mbar_wait<false>(&bar_b, 0, err, tc::kErrTimeoutLoad, &abort_flag);
   if (!unsafe) {
-    // dS' = dS diag(e^Lambda) in place, with the half sums of dS' o S0 over r
-    const float eL = expf(lam[j]);
-    float cs = 0.f;
-#pragma unroll 8
-    for (int rr = 0; rr < 64; ++rr) {
-      const uint32_t off = tc::sw128_off(64 * half + rr, j, 128, 2);
-      const float ds = bf(sm + Cf::DST + off) * eL;
-      put_bf(sm + Cf::DST + off, ds);
-      cs = fmaf(ds, bf(sm + Cf::S0T + off), cs);
+    // dS' = dS diag(e^Lambda) in place, with the sums of dS' o S0 over r: a
+    // thread takes eight channels (one 16-byte swizzle chunk) of eight rows;
+    // the two row groups of a warp meet by a shuffle, the warps below in order
+    const int g = tid & 15, rg = tid >> 4, lane = tid & 31;
+    float e8[8], acc8[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      e8[c] = expf(lam[8 * g + c]);
+      acc8[c] = 0.f;
     }
-    csp[half * 128 + j] = cs;
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const uint32_t off = tc::sw128_off(8 * rg + rr, 8 * g, 128, 2);
+      uint4 dv = *reinterpret_cast<const uint4*>(sm + Cf::DST + off);
+      const uint4 sv = *reinterpret_cast<const uint4*>(sm + Cf::S0T + off);
+      __nv_bfloat162* dp = reinterpret_cast<__nv_bfloat162*>(&dv);
+      const __nv_bfloat162* sp = reinterpret_cast<const __nv_bfloat162*>(&sv);
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float2 d2 = __bfloat1622float2(dp[c2]);
+        const float2 s2 = __bfloat1622float2(sp[c2]);
+        d2.x *= e8[2 * c2];
+        d2.y *= e8[2 * c2 + 1];
+        acc8[2 * c2] = fmaf(d2.x, s2.x, acc8[2 * c2]);
+        acc8[2 * c2 + 1] = fmaf(d2.y, s2.y, acc8[2 * c2 + 1]);
+        dp[c2] = __floats2bfloat162_rn(d2.x, d2.y);
+      }
+      *reinterpret_cast<uint4*>(sm + Cf::DST + off) = dv;
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc8[c] += __shfl_xor_sync(0xffffffffu, acc8[c], 16);
+    if (lane < 16) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) csred[warp][8 * g + c] = acc8[c];
+    }
     tc::fence_proxy_async();
   }
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
+  if (!unsafe && tid < D) {  // read by the epilogue, after its barriers
+    float cs = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) cs += csred[w][tid];
+    csp[tid] = cs;
+    csp[128 + tid] = 0.f;
+  }
 
   if (!unsafe) {
     if (tid == 0) {
