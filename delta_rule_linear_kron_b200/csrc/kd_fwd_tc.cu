@@ -579,8 +579,8 @@ struct CrossCfg {
   static constexpr uint32_t VV = 65536;    // bf16, 2 K blocks x 128 rows: rows 0-63 V_n, 64-127 V_{n-1} (TMA)
   static constexpr uint32_t KR = 98304;    // k_n, k_{n-1} bf16 [64][128] each (TMA)
   static constexpr uint32_t LG = 131072;   // logf_n, then K~_n staged in place; logf_{n-1}, then K^e_n (fp32 [64][128])
-  static constexpr uint32_t XCH = 196608;  // Lambda_{n-1} [128]
-  static constexpr uint32_t VT = 197632;   // V_n^T bf16 [r][t], 128 rows x 128 B, 128-byte swizzle (staging)
+  static constexpr uint32_t XCH = 196608;  // half sums of logf_n, logf_{n-1} [2][2][128]
+  static constexpr uint32_t VT = 198656;   // V_n^T bf16 [r][t], 128 rows x 128 B, 128-byte swizzle (staging)
   static constexpr uint32_t BYTES = VT + 16384 + 1024;
   static constexpr uint32_t LOAD_CUR = 16384 + 16384 + 32768, LOAD_PREV = LOAD_CUR;
 };
@@ -633,40 +633,49 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
   tc::tc_after_sync();
   const uint32_t tmem = tmem_slot;
   tc::mbar_wait<false>(&ld_bar, 0, err, tc::kErrTimeoutLoad, &abort_flag);
-  // half 0: chunk n (channel j); half 1: chunk n-1 (channel j)
-  const int j = tid & 127, half = tid >> 7;
-  float* lg = reinterpret_cast<float*>(sm + CrossCfg::LG + half * 32768);
-  const unsigned char* kr = sm + CrossCfg::KR + half * 16384;
-  float tot = 0.f;
-  if (half == 0 || has_prev) {
+  // thread (j, half): key channel j, positions 32*half .. +31 of both chunks
+  const int j = tid & 127, half = tid >> 7, tb = 32 * half;
+  float* lgn = reinterpret_cast<float*>(sm + CrossCfg::LG);          // logf_n, then K~_n
+  float* lgp = reinterpret_cast<float*>(sm + CrossCfg::LG + 32768);  // logf_{n-1}, then K^e_n
+  const unsigned char* krn = sm + CrossCfg::KR;
+  const unsigned char* krp = sm + CrossCfg::KR + 16384;
+  {
+    float sn = 0.f, sp = 0.f;
 #pragma unroll 8
-    for (int t = 0; t < C; ++t) tot += lg[t * D + j];
-  }
-  if (half) xch[j] = has_prev ? tot : 0.f;
-  __syncthreads();
-  float Lr[C];
-  if (half == 0) {
-    // K+_n (Gram operand, tf32) and K~_n (staged in place of logf_n)
-    const float lam_prev = xch[j];
-    float L = 0.f;
-#pragma unroll
-    for (int t = 0; t < C; ++t) {
-      L += lg[t * D + j];
-      Lr[t] = L;
-      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kr + (t * D + j) * 2));
-      const float kp = kk * expf(L);
-      *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(t, j, 128, 4)) = kp;
-      lg[t * D + j] = kk * expf(L + lam_prev);
+    for (int i = 0; i < 32; ++i) {
+      sn += lgn[(tb + i) * D + j];
+      if (has_prev) sp += lgp[(tb + i) * D + j];
     }
-    wGC[ch * D + j] = expf(tot);
-  } else if (has_prev) {
-    // K^e_{n-1} (Gram operand, tf32)
-    float L = 0.f;
+    xch[half * D + j] = sn;
+    xch[(2 + half) * D + j] = sp;
+  }
+  __syncthreads();
+  const float tot = xch[j] + xch[D + j];                                      // Lambda_n
+  const float lam_prev = has_prev ? xch[2 * D + j] + xch[3 * D + j] : 0.f;    // Lambda_{n-1}
+  if (half == 0) wGC[ch * D + j] = expf(tot);
+  if (has_prev) {
+    // K^e_{n-1} (Gram operand, tf32), at this thread's positions
+    float L = half ? xch[2 * D + j] : 0.f;
 #pragma unroll 8
-    for (int t = 0; t < C; ++t) {
-      L += lg[t * D + j];
-      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kr + (t * D + j) * 2));
-      *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(tot - L);
+    for (int i = 0; i < 32; ++i) {
+      const int t = tb + i;
+      L += lgp[t * D + j];
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(krp + (t * D + j) * 2));
+      *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(lam_prev - L);
+    }
+  }
+  {
+    // K+_n (Gram operand, tf32), K~_n in place of logf_n and K^e_n in place of
+    // logf_{n-1}: each thread overwrites only the entries it has just read
+    float L = half ? xch[j] : 0.f;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+      const int t = tb + i;
+      L += lgn[t * D + j];
+      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(krn + (t * D + j) * 2));
+      *reinterpret_cast<float*>(sm + CrossCfg::KK + tc::sw128_off(t, j, 128, 4)) = kk * expf(L);
+      lgn[t * D + j] = kk * expf(L + lam_prev);
+      lgp[t * D + j] = kk * expf(tot - L);
     }
   }
   // V_n^T as the K-major tile [r][t] the chain's column dot and update MMA read
@@ -680,15 +689,6 @@ __global__ void __launch_bounds__(256, 1) fwd_cross_tc(
         v8[i] = *reinterpret_cast<const __nv_bfloat16*>(sm + CrossCfg::VV + tc::sw128_off(tb + g8 + i, r, 128, 2));
       *reinterpret_cast<uint4*>(sm + CrossCfg::VT + tc::sw128_off(r, tb + g8, 128, 2)) =
           *reinterpret_cast<const uint4*>(v8);
-    }
-  }
-  __syncthreads();  // logf_{n-1} is dead: K^e_n goes there
-  if (half == 0) {
-    float* ke = reinterpret_cast<float*>(sm + CrossCfg::LG + 32768);
-#pragma unroll
-    for (int t = 0; t < C; ++t) {
-      const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kr + (t * D + j) * 2));
-      ke[t * D + j] = kk * expf(tot - Lr[t]);
     }
   }
   tc::fence_proxy_async();
