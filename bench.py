@@ -152,13 +152,13 @@ def pass_bytes(name, d=128):
 # kernel lives in and the first 16 hex digits of its sha256 at capture time;
 # a kernel whose source has changed since reports no traffic.
 NCU_TRAFFIC = {
-    "fwd_prep_tc": (448477867, "kd_fwd_tc.cu", "cde3897fd7273271"),
-    "fwd_cross_tc": (619198805, "kd_fwd_tc.cu", "cde3897fd7273271"),
-    "fwd_chain_tc": (590972672, "kd_fchain_tc.cu", "cac9ee1a46a36d26"),
-    "fwd_out_tc": (525964117, "kd_fwd_tc.cu", "cde3897fd7273271"),
-    "bwd_pre_tc": (768108459, "kd_bwd_chunk_tc.cu", "7c3d2764ee32d35f"),
-    "bwd_chain_tc": (727255637, "kd_bchain_tc.cu", "b514c715eaf3ed73"),
-    "bwd_post_tc": (1125903616, "kd_bwd_chunk_tc.cu", "7c3d2764ee32d35f"),
+    "fwd_prep_tc": (447285931, "kd_fwd_tc.cu", "0ec6969ffa6a3978"),
+    "fwd_cross_tc": (619036160, "kd_fwd_tc.cu", "0ec6969ffa6a3978"),
+    "fwd_chain_tc": (591101867, "kd_fchain_tc.cu", "cac9ee1a46a36d26"),
+    "fwd_out_tc": (525770240, "kd_fwd_tc.cu", "0ec6969ffa6a3978"),
+    "bwd_pre_tc": (768061696, "kd_bwd_chunk_tc.cu", "7c3d2764ee32d35f"),
+    "bwd_chain_tc": (727406592, "kd_bchain_tc.cu", "b514c715eaf3ed73"),
+    "bwd_post_tc": (1127274325, "kd_bwd_chunk_tc.cu", "7c3d2764ee32d35f"),
 }
 
 
