@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
                  reinterpret_cast<float*>(sm + PreCfg::XCH), Lr);
     const unsigned char* kr = sm + PreCfg::KR;
     const unsigned char* qr = sm + PreCfg::QR;
+    __align__(16) __nv_bfloat16 q8[8];  // eight consecutive positions of Q+^T row j: one 16-byte store
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int t = 32 * half + i;
@@ -177,7 +178,9 @@ __global__ void __launch_bounds__(256, 1) bwd_pre_tc(
       const float gm = expf(Lr[i]);
       *reinterpret_cast<float*>(sm + PreCfg::KPM + tc::sw128_off(t, j, 128, 4)) = kk * gm;
       *reinterpret_cast<float*>(sm + PreCfg::KPM + tc::sw128_off(64 + t, j, 128, 4)) = kk * expf(-Lr[i]);
-      put_bf(sm + PreCfg::QT + tc::sw128_off(j, t, 128, 2), bf(qr + (t * D + j) * 2) * gm);
+      q8[i & 7] = __float2bfloat16_rn(bf(qr + (t * D + j) * 2) * gm);
+      if ((i & 7) == 7)
+        *reinterpret_cast<uint4*>(sm + PreCfg::QT + tc::sw128_off(j, t - 7, 128, 2)) = *reinterpret_cast<const uint4*>(q8);
     }
   }
   tc::fence_proxy_async();
