@@ -444,8 +444,11 @@ KD_API int kron_delta_epilogue_bwd(const void *o, const void *g, const float *w,
  *   ST : [B,H,dv,dk] fp32 or NULL.
  *   workspace : at least kron_delta_workspace_size(KD_WS_GDN2_FWD, ...) bytes,
  *   256-byte aligned; it keeps what kron_delta_gdn2_bwd reads.
- * Computed on CUDA cores in fp32 (no tensor-core path yet).  Errors as for
- * kron_delta_fwd.  Asynchronous on `stream`.
+ * With dtype bf16 and dk = dv = 128 every chunk contraction runs on tensor
+ * cores, on fp32 operands split into bf16 high and low parts; the chain's
+ * state stays fp32, and the chunk-start states kept in the workspace for
+ * the backward are bf16.  Other shapes run on CUDA cores in fp32.  Errors as
+ * for kron_delta_fwd.  Asynchronous on `stream`.
  */
 KD_API int kron_delta_gdn2_fwd(const void *q, const void *k, const void *v, const float *b,
                                const float *w, const float *loga, const float *S0, void *out,
@@ -459,6 +462,9 @@ KD_API int kron_delta_gdn2_fwd(const void *q, const void *k, const void *v, cons
  *   dq, dk [B,T,H,dk] and dv [B,T,H,dv] (dtype); db, dloga [B,T,H,dk] and
  *   dw [B,T,H,dv] fp32; dS0 [B,H,dv,dk] fp32 or NULL.
  *   workspace : at least kron_delta_workspace_size(KD_WS_GDN2_BWD, ...).
+ * Same precision split as the forward (the per-chunk gradients read the
+ * saved bf16 states); chunks whose in-chunk decay leaves the factorised range
+ * (|cumulative loga| >= 60) take an exact CUDA-core kernel.  Deterministic.
  * Errors as for kron_delta_bwd.  Asynchronous on `stream`.
  */
 KD_API int kron_delta_gdn2_bwd(const void *q, const void *k, const void *v, const float *b,
