@@ -224,3 +224,22 @@ def test_gdn2_argument_errors(L):
     rc = L.kron_delta_gdn2_bwd(p, p, p, p, p, p, None, p, None, p, p, p, p, p, p, None, 1, 2, 100, 64, 32, 1,
                                p, need_f, p, need_b - 256, None)
     assert rc == kd.KD_ERR_WORKSPACE
+
+
+def test_gdn2_tensor_core_workspace_layout(L):
+    """The planner's tensor-core layout for Gated DeltaNet-2 (bf16, d = 128),
+    per chunk of C = 64: the forward keeps A, P [C][C], U', Q+, U [C][d] in
+    fp32, e^Lambda [d], the chunk-start state as one bf16 image [d][d] and the
+    chains' W, K^e images (bf16 hi, lo [C][d]), with no fp32 W, K^e or state;
+    the backward adds dU, dE, dQ+, dK^e, P^T dO [C][d], dT, dP [C][C], dS,
+    S0 and (dO^T Q+)^T [d][d] in fp32, the dS image in bf16 and one flag byte
+    per chunk.  Every region is a multiple of 256 bytes here, so the sizes are
+    exact sums."""
+    C, d, chunks = 64, 128, 16 * (16384 // 64)
+    fwd_floats = 2 * C * C + 3 * C * d + d + d * d // 2 + 2 * C * d
+    bwd_floats = 6 * C * d + 2 * C * C + 3 * d * d
+    assert kd.workspace_size(kd.KD_WS_GDN2_FWD, 1, 16, 16384, d, d, 1) == chunks * fwd_floats * 4
+    assert kd.workspace_size(kd.KD_WS_GDN2_BWD, 1, 16, 16384, d, d, 1) == chunks * bwd_floats * 4 + chunks
+    # the CUDA-core layout (fp32 inputs): fp32 W and K^e in place of the two
+    # images (the same bytes) and the state in fp32 (twice its bf16 image)
+    assert kd.workspace_size(kd.KD_WS_GDN2_FWD, 1, 16, 16384, d, d, 0) == chunks * (fwd_floats + d * d // 2) * 4
